@@ -1,0 +1,518 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the Mamba-3 SSM layer core (libm3) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch of the page-1-shaped layer
+(batch 4, seqlen 2048, 24 heads x 64, d_state 64, MIMO rank 2, bf16 x/B/C, fp32 state):
+m3_scan_fwd over the 4 x 2048 prompt tokens, then m3_decode_step for one more token
+per sequence from the final state.  value = tokens/s over all ranks (weak scaling:
+every rank runs its own batch; no data-path collective).  Inputs are seeded and
+synthetic; a ring of input sets larger than L2 rotates between steps.
+
+Extra keys: "prefill" / "decode" give each kernel measured on its own (decode on the
+1.5B-scale layer, batch 128, state 256 MiB > L2); "roofline" is the dominant kernel
+(the tensor-core prefill) against MEASURED_PEAKS.json; "cpu_baseline" times the fp64
+oracle (test infrastructure) on a bounded sample; "e2e" times the same step through
+the C ABI with pinned host buffers and the host<->device copies inside the timed region.
+
+--impl reference times the fp64 CPU oracle alone (the reference arm of this build).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Mamba-3 SSM tokens/s (prefill, decode) and % of tensor-core / HBM roofline"
+WORKLOAD = "p1_layer"
+DECODE_WORKLOAD = "decode_b128"
+L2_BYTES = 126 * 1024 * 1024
+
+# dram bytes (read + write) per launch of the prefill kernel from the ncu capture
+# summarised in profiles/scan_tc_p1_layer.md; None until that capture matches the
+# current kernel.
+PREFILL_DRAM_BYTES_PER_LAUNCH = None
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ------------------------------------------------------------------ algorithmic counts
+
+def prefill_bytes(d):
+    """Algorithmic HBM bytes of one m3_scan_fwd: every input read once, y written once,
+    state (h, carry) read and written once."""
+    b, L, H, P, N, R, G = (d[k] for k in ("b", "L", "H", "P", "N", "R", "G"))
+    e = 2 if d["dtype"] == "bf16" else 4
+    tok = b * L
+    io = tok * (H * P * e * 2 + 2 * G * R * N * e + G * (N // 2) * 4 + 3 * H * 4)
+    state = 2 * b * H * (N * P + R * N + P) * 4
+    return io + state
+
+
+def prefill_flops(d, chunk=32):
+    """Algorithmic FLOPs of the chunked scan at the model's chunk length (dense chunk
+    tiles): per token and head 2 Q R^2 (N + P) (intra-chunk C B^T and its product
+    with X) + 4 R N P (state readout and state update)."""
+    b, L, H, P, N, R = (d[k] for k in ("b", "L", "H", "P", "N", "R"))
+    intra = 2 * chunk * R * R * (N + P)
+    inter = 4 * R * N * P
+    return b * L * H * (intra + inter), b * L * H * intra
+
+
+def decode_bytes(d):
+    """Algorithmic HBM bytes of one m3_decode_step: state read + written, token I/O."""
+    b, H, P, N, R, G = (d[k] for k in ("b", "H", "P", "N", "R", "G"))
+    e = 2 if d["dtype"] == "bf16" else 4
+    state = 2 * b * H * (N * P + R * N + P) * 4
+    io = b * (2 * H * P * e + 2 * G * R * N * e + G * (N // 2) * 4 + 3 * H * 4)
+    return state + io
+
+
+def decode_flops(d):
+    b, H, P, N, R = (d[k] for k in ("b", "H", "P", "N", "R"))
+    # per state element: rank-R u_t and u_{t-1} (4R), rotation + decay + add (~8), readout (2R)
+    return b * H * N * P * (6 * R + 8)
+
+
+# ------------------------------------------------------------------ peaks, clocks
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return dict(hbm=float(j["hbm_gbs"]), bf16=float(j["bf16_tflops"]),
+                    bf16_sus=float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML (read-only) while running."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, index, period=0.005):
+        self.index, self.period = index, period
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        except Exception as e:  # sampling is best effort; the line says so
+            log(f"clock sampling unavailable: {e}")
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+        return False
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples), "source": "nvml"}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
+
+
+# ------------------------------------------------------------------ our arm
+
+def dist_setup(n_gpus):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, world):
+    import torch
+    if world == 1:
+        return float(x)
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], device="cuda", dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def make_ring(inp, n_sets, device):
+    """n_sets device copies of the layer inputs (distinct buffers, same values) plus
+    per-set y buffers and states, so consecutive steps touch > L2 bytes."""
+    import torch
+    from selective_state_space_53_b200 import m3
+    sets = []
+    for _ in range(n_sets):
+        dev = m3.to_device(inp, device)
+        dims = m3.dims_of(inp)
+        st, keep = m3.state_tensors(dims, device=device)
+        y = torch.empty_like(dev["x"])
+        sets.append(dict(dev=dev, state=st, keep=keep, y=y))
+    return sets
+
+
+def token_slice(dev, t):
+    seq = ("x", "dt", "A", "lam", "B", "C", "theta")
+    return {k: (v[:, t].contiguous() if (v is not None and k in seq) else v) for k, v in dev.items()}
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    from selective_state_space_53_b200 import m3
+    from selective_state_space_53_b200.inputs import CONFIGS, SEEDS, config_inputs
+
+    rank, world, local = dist_setup(args.gpus)
+    device = f"cuda:{local}"
+    peaks = measured_peaks()
+    cfg = dict(CONFIGS[WORKLOAD])
+    inp = config_inputs(WORKLOAD, seed=SEEDS[WORKLOAD] + rank)
+    dims = m3.dims_of(inp)
+    dims1 = m3.dims_of(inp, L=1)
+    per_set = prefill_bytes(cfg)
+    n_sets = max(2, -(-3 * L2_BYTES // per_set))
+    ring = make_ring(inp, n_sets, device)
+    # the decode token of each set: a fresh draw's first token
+    tok_inp = config_inputs(WORKLOAD, seed=SEEDS[WORKLOAD] + 100 + rank, L=1)
+    tok_dev = token_slice(m3.to_device(tok_inp, device), 0)
+    for s in ring:
+        s["state1"] = m3.State.wrap(dims1, *s["keep"])
+        s["y1"] = torch.empty_like(tok_dev["x"])
+    stream = torch.cuda.current_stream()
+
+    def step(i, ev=None):
+        s = ring[i % n_sets]
+        if ev is not None:
+            ev[0].record(stream)
+        m3.scan(dims, s["dev"], s["state"], y=s["y"])
+        if ev is not None:
+            ev[1].record(stream)
+        m3.decode(dims1, tok_dev, s["state1"], y=s["y1"])
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert m3.m3_check() == 0
+
+    # ---- timed region: K steps, events per prefill launch for the roofline
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        t0.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i, evs[i])
+        t1.record(stream)
+        barrier(world)
+    assert m3.m3_check() == 0
+    ms_local = t0.elapsed_time(t1)
+    ms = max_over_ranks(ms_local, world)
+    prefill_ms = [a.elapsed_time(b) for a, b in evs]
+    tokens_step = cfg["b"] * (cfg["L"] + 1)
+    value = world * tokens_step * args.steps / (ms / 1e3)
+    gpu_launches = 2 * args.steps
+
+    pf_ms = statistics.mean(prefill_ms)
+    pbytes = prefill_bytes(cfg)
+    pflops, pflops_intra = prefill_flops(cfg)
+    prefill = {
+        "workload": "p1_layer m3_scan_fwd b4 L2048 H24 P64 N64 R2",
+        "tokens_per_s": cfg["b"] * cfg["L"] / (pf_ms / 1e3),
+        "ms_per_launch": pf_ms,
+        "hbm_gbs": pbytes / (pf_ms / 1e-3) / 1e9 * 1e-6 * 1e6 if False else pbytes / (pf_ms * 1e-3) / 1e9,
+        "hbm_frac_of_measured": pbytes / (pf_ms * 1e-3) / 1e9 / peaks["hbm"],
+        "tflops": pflops / (pf_ms * 1e-3) / 1e12,
+        "tensor_frac_of_measured_burst": pflops / (pf_ms * 1e-3) / 1e12 / peaks["bf16"],
+        "intra_chunk_tflops": pflops_intra / (pf_ms * 1e-3) / 1e12,
+        "intra_chunk_frac_of_measured_burst": pflops_intra / (pf_ms * 1e-3) / 1e12 / peaks["bf16"],
+        "algorithmic_bytes": pbytes, "algorithmic_flops": pflops,
+    }
+    hbm_frac = prefill["hbm_frac_of_measured"]
+    ten_frac = prefill["tensor_frac_of_measured_burst"]
+    bound = "hbm" if hbm_frac >= ten_frac else "tensor"
+    roofline = {
+        "kernel": "scan_tc_kernel (m3_scan_fwd)",
+        "bound": bound,
+        "achieved": prefill["hbm_gbs"] if bound == "hbm" else prefill["tflops"],
+        "peak": peaks["hbm"] if bound == "hbm" else peaks["bf16"],
+        "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+        "frac": hbm_frac if bound == "hbm" else ten_frac,
+        "traffic": PREFILL_DRAM_BYTES_PER_LAUNCH,
+        "peak_source": f"{peaks['src']} (MEASURED_PEAKS.json burst)" if peaks["src"] == "measured" else "fallback",
+        "other_bound_frac": ten_frac if bound == "hbm" else hbm_frac,
+    }
+
+    decode = run_decode(args, device, peaks) if not args.no_decode else None
+    e2e = run_e2e(args, inp, tok_inp, device, world) if not args.no_e2e else None
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; shapes of the page-1 layer)",
+        "config": {"workload": "p1_layer: m3_scan_fwd over b4 x L2048 (H24 P64 N64 R2, chunk 32) + 1 m3_decode_step",
+                   "global_batch": cfg["b"] * world, "seq_len": cfg["L"], "parallelism": f"dp{world}",
+                   "l2": f"ring of {n_sets} input sets ({n_sets * per_set / 2**20:.0f} MiB) > L2"},
+        "roofline": roofline, "prefill": prefill, "decode": decode, "e2e": e2e,
+        "gpu_launches": gpu_launches, "clocks": clk.summary(),
+    }
+    if rank == 0 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(cfg, inp, tokens_step, seconds=args.cpu_seconds)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_decode(args, device, peaks):
+    """m3_decode_step on the 1.5B-scale layer, batch 128 (state 256 MiB > L2)."""
+    import torch
+    from selective_state_space_53_b200 import m3
+    from selective_state_space_53_b200.inputs import CONFIGS, SEEDS, make_inputs, make_state
+    cfg = dict(CONFIGS[DECODE_WORKLOAD])
+    steps = args.decode_steps
+    cfg_draw = dict(cfg, L=min(steps, 16))
+    inp = make_inputs(seed=SEEDS[DECODE_WORKLOAD], **cfg_draw)
+    dims1 = m3.dims_of(inp, L=1)
+    h, cB, cx = make_state(cfg["b"], cfg["H"], cfg["P"], cfg["N"], cfg["R"], seed=7, scale=0.1)
+    st, keep = m3.state_tensors(dims1, device=device, h=h, carry_B=cB, carry_x=cx)
+    dev = m3.to_device(inp, device)
+    toks = [token_slice(dev, t) for t in range(cfg_draw["L"])]
+    y = torch.empty_like(toks[0]["x"])
+    stream = torch.cuda.current_stream()
+    for i in range(3):
+        m3.decode(dims1, toks[i % len(toks)], st, y=y)
+    torch.cuda.synchronize()
+    # capture the steps in a CUDA graph: launch overhead out of the per-token time
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(steps):
+            m3.decode(dims1, toks[i % len(toks)], st, y=y)
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    g.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    assert m3.m3_check() == 0
+    ms = a.elapsed_time(b) / steps
+    by = decode_bytes(cfg)
+    fl = decode_flops(cfg)
+    del g
+    return {"workload": "decode_b128: m3_decode_step, b128 H32 P128 N128 R4, CUDA graph of %d steps" % steps,
+            "tokens_per_s": cfg["b"] / (ms * 1e-3), "us_per_step": ms * 1e3,
+            "hbm_gbs": by / (ms * 1e-3) / 1e9, "hbm_frac_of_measured": by / (ms * 1e-3) / 1e9 / peaks["hbm"],
+            "tflops": fl / (ms * 1e-3) / 1e12, "algorithmic_bytes": by}
+
+
+def run_e2e(args, inp, tok_inp, device, world):
+    """Same step through the C ABI from pinned host buffers: H2D of the step's inputs,
+    prefill + decode, D2H of y (prefill and decode outputs)."""
+    import torch
+    from selective_state_space_53_b200 import m3
+    host = {}
+    for k in ("x", "dt", "A", "lam", "B", "C", "theta", "bias_B", "bias_C", "W_x", "W_o", "D"):
+        a = getattr(inp, k)
+        if a is None:
+            host[k] = None
+            continue
+        t = torch.from_numpy(a)
+        if k in ("x", "B", "C"):
+            t = t.to(torch.bfloat16)
+        host[k] = t.pin_memory()
+    htok = {}
+    for k in ("x", "dt", "A", "lam", "B", "C", "theta"):
+        t = torch.from_numpy(getattr(tok_inp, k)[:, 0].copy())
+        if k in ("x", "B", "C"):
+            t = t.to(torch.bfloat16)
+        htok[k] = t.pin_memory()
+    dev = {k: (None if v is None else torch.empty_like(v, device=device)) for k, v in host.items()}
+    dtok = {k: torch.empty_like(v, device=device) for k, v in htok.items()}
+    for k in ("bias_B", "bias_C", "W_x", "W_o", "D"):
+        dtok[k] = dev[k]
+    dims = m3.dims_of(inp)
+    dims1 = m3.dims_of(inp, L=1)
+    st, keep = m3.state_tensors(dims, device=device)
+    st1 = m3.State.wrap(dims1, *keep)
+    y = torch.empty_like(dev["x"])
+    y1 = torch.empty_like(dtok["x"])
+    y_host = torch.empty_like(y, device="cpu").pin_memory()
+    y1_host = torch.empty_like(y1, device="cpu").pin_memory()
+    stream = torch.cuda.current_stream()
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None) + \
+        sum(v.numel() * v.element_size() for v in htok.values())
+    d2h = y.numel() * y.element_size() + y1.numel() * y1.element_size()
+
+    def step():
+        for k, v in host.items():
+            if v is not None:
+                dev[k].copy_(v, non_blocking=True)
+        for k, v in htok.items():
+            dtok[k].copy_(v, non_blocking=True)
+        m3.scan(dims, dev, st, y=y)
+        m3.decode(dims1, dtok, st1, y=y1)
+        y_host.copy_(y, non_blocking=True)
+        y1_host.copy_(y1, non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    n = max(1, min(args.steps, 10))
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    a.record(stream)
+    for _ in range(n):
+        step()
+    b.record(stream)
+    barrier(world)
+    ms = max_over_ranks(a.elapsed_time(b), world) / n
+    tokens = inp.dims["b"] * (inp.dims["L"] + 1)
+    return {"value": world * tokens / (ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": n}
+
+
+# ------------------------------------------------------------------ fp64 oracle (CPU)
+
+def _oracle_rate(cfg, inp, pairs, threads=0):
+    """Seconds for the oracle to run `pairs` (batch, head) sequences of the layer."""
+    from oracle import oracle as orc
+    t = time.perf_counter()
+    orc.scan_inputs(inp, sel=pairs, threads=threads)
+    return time.perf_counter() - t
+
+
+def cpu_baseline(cfg, inp, tokens_step, seconds=12.0):
+    """The fp64 oracle as it stands, OpenMP over (batch, head) on all host cores, on a
+    bounded sample: as many whole (batch, head) sequences of the layer as fit in about
+    `seconds`.  Scaled to layer tokens/s: a layer token needs all H heads."""
+    from oracle import oracle as orc
+    H, b = cfg["H"], cfg["b"]
+    allp = [(bi, hi) for bi in range(b) for hi in range(H)]
+    cores = orc.max_threads()
+    probe = allp[:cores]
+    t1 = _oracle_rate(cfg, inp, probe)
+    per_pair = t1 / len(probe)  # seconds per pair at full parallelism
+    n = int(max(len(probe), min(len(allp), seconds / max(per_pair, 1e-9))))
+    n = max(cores, (n // cores) * cores)
+    n = min(n, len(allp))
+    sample = allp[:n]
+    t = _oracle_rate(cfg, inp, sample)
+    layer_tokens = len(sample) * cfg["L"] / H
+    return {"value": layer_tokens / t, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(sample)} of {len(allp)} (batch, head) sequences x {cfg['L']} tokens of p1_layer "
+                      f"({t:.1f} s); tokens/s counts layer tokens (all {H} heads)",
+            "seconds": t}
+
+
+def run_reference(args):
+    """Reference arm: the fp64 oracle on the host cores, on the same workload and metric."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from oracle import oracle as orc
+    from selective_state_space_53_b200.inputs import CONFIGS, SEEDS, config_inputs
+    cfg = dict(CONFIGS[WORKLOAD])
+    inp = config_inputs(WORKLOAD)
+    H, b = cfg["H"], cfg["b"]
+    cores = orc.max_threads()
+    allp = [(bi, hi) for bi in range(b) for hi in range(H)]
+    # each step: one sample of `cores` whole (batch, head) sequences (about a second)
+    sample = allp[:min(len(allp), cores)]
+    for i in range(args.warmup):
+        _oracle_rate(cfg, inp, sample)
+    t = 0.0
+    for i in range(args.steps):
+        t += _oracle_rate(cfg, inp, sample)
+    layer_tokens_per_step = len(sample) * cfg["L"] / H
+    value = layer_tokens_per_step * args.steps / t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; shapes of the page-1 layer)",
+        "config": {"workload": "p1_layer: m3_scan_fwd over b4 x L2048 (H24 P64 N64 R2, chunk 32) + 1 m3_decode_step",
+                   "global_batch": b, "seq_len": cfg["L"], "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {len(sample)} of {len(allp)} (batch, head) sequences x {cfg['L']} "
+                                   f"tokens; tokens/s counts layer tokens (all {H} heads)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-steps", type=int, default=256)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle timing")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

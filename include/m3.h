@@ -1,0 +1,163 @@
+/*
+ * m3.h -- C ABI of the B200-native Mamba-3 SSM layer core (libm3.so).
+ *
+ * The layer core is the exponential-trapezoidal selective scan with complex
+ * (rotation / data-dependent RoPE) transitions and MIMO rank R, as described in
+ * the Mamba-3 paper note (docsaid.org, "Mamba-3: Improved Sequence Modeling using
+ * State Space Principles"):
+ *   - section "その1 表現力の高い離散化": h_t = alpha_t h_{t-1} + beta_t B_{t-1}x_{t-1}
+ *     + gamma_t B_t x_t with alpha = e^{dt A}, beta = (1-lam) dt e^{dt A}, gamma = lam dt;
+ *   - section "その2 複素数の状態": complex A, i.e. a decay times 2x2 rotations of
+ *     adjacent state pairs, equivalently a data-dependent RoPE of B and C;
+ *   - section "その3 MIMO": R input branches and R readouts, rank <= R update.
+ * Per (batch b, head h; group g = h / (H/G)) and token t:
+ *   Bb_{t,r} = B[b,t,g,r,:] + bias_B[h,r,:],  Cb_{t,r} = C[b,t,g,r,:] + bias_C[h,r,:]
+ *   X_{t,r} = W_x[h,r,:] * x[b,t,h,:],        u_t = sum_r Bb_{t,r} X_{t,r}^T   (N x P)
+ *   h_t = e^{dt_t A_t} Rot(dt_t theta_t) (h_{t-1} + (1-lam_t) dt_t u_{t-1}) + lam_t dt_t u_t
+ *   y[b,t,h,:] = sum_r W_o[h,r,:] * (Cb_{t,r}^T h_t) + D[h] x[b,t,h,:]
+ * Rot rotates rows (2k, 2k+1) of the state by angle dt_t theta[b,t,g,k] with the
+ * matrix [[cos, -sin], [sin, cos]].
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are caller-owned DEVICE memory, contiguous row-major in the
+ *     layouts below, 16-byte aligned.  The library never frees them.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL is
+ *     the legacy default stream).  m3_scan_fwd and m3_decode_step allocate nothing
+ *     and never synchronise the host.
+ *   - Every call returns an m3_status; nothing throws across the ABI.  Argument
+ *     errors are detected on the host before anything is launched.  A kernel
+ *     that gives up a bounded wait records M3_ERR_TIMEOUT in a device status
+ *     word, which m3_check() returns.
+ *
+ * Layouts (dtype: M3_BF16 or M3_F32 for x, B, C, y; fp32 for everything else):
+ *   x, y          (b, L, H, P)        dt, A, lam   (b, L, H)
+ *   B, C          (b, L, G, R, N)     theta        (b, L, G, N/2)
+ *   bias_B/bias_C (H, R, N)  may be NULL (zero)
+ *   W_x, W_o      (H, R, P)  may be NULL (all ones)
+ *   D             (H)        may be NULL (no skip term)
+ * State (m3_state): h (b, H, N, P) fp32, carry_B (b, H, R, N) fp32 (previous
+ * token's raw B, before bias), carry_x (b, H, P) fp32 (previous token's raw x).
+ * An all-zero state is a fresh sequence (no previous-token term at t = 0).
+ */
+#ifndef M3_H
+#define M3_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  M3_OK = 0,
+  M3_ERR_DIMS = -1,        /* bad sizes: N odd, G does not divide H, R/P/N out of range */
+  M3_ERR_DTYPE = -2,       /* dtype not M3_BF16 / M3_F32 */
+  M3_ERR_ALIGN = -3,       /* a tensor pointer is not 16-byte aligned */
+  M3_ERR_NULL = -4,        /* a required pointer is NULL */
+  M3_ERR_WORKSPACE = -5,   /* workspace missing or smaller than m3_scan_workspace_size */
+  M3_ERR_CUDA = -6,        /* a CUDA runtime call or kernel launch failed */
+  M3_ERR_TIMEOUT = -7,     /* a kernel gave up a bounded wait (device status word) */
+  M3_ERR_UNSUPPORTED = -8, /* valid dims that no kernel of this build handles */
+  M3_ERR_STATE = -9        /* state was made for other dims, or buffer size mismatch */
+} m3_status;
+
+enum { M3_F32 = 0, M3_BF16 = 1 };
+
+/* flags */
+enum {
+  M3_FLAG_SEQUENTIAL = 1u  /* run the token-sequential SIMT scan even where the chunked
+                              tensor-core scan applies (diagnostic / cross-check) */
+};
+
+typedef struct {
+  int64_t b;      /* batch */
+  int64_t L;      /* sequence length (ignored by m3_decode_step: one token) */
+  int32_t H;      /* heads */
+  int32_t P;      /* head dim (multiple of 8, <= 256) */
+  int32_t N;      /* state dim d_state (even, multiple of 8, <= 256) */
+  int32_t R;      /* MIMO rank (1..8) */
+  int32_t G;      /* B/C/theta groups (divides H) */
+  int32_t chunk;  /* chunk length of the model (0 = default 32).  The chunked scan is
+                     exact, so this does not change the result; the kernel packs
+                     128/R tokens per tensor-core tile whatever this value is. */
+  int32_t dtype;  /* M3_BF16 or M3_F32: storage type of x, B, C, y */
+  uint32_t flags; /* M3_FLAG_* */
+} m3_dims;
+
+typedef struct m3_state m3_state; /* opaque */
+
+/* ---- state ------------------------------------------------------------- */
+
+/* Bytes of device memory an m3_state for these dims holds (h + carry_B + carry_x). */
+m3_status m3_state_bytes(const m3_dims* dims, size_t* out_bytes);
+
+/* Allocate a zero-initialised state on the current device (cudaMallocAsync on
+ * `stream`).  The library owns the memory; release it with m3_state_free. */
+m3_status m3_state_alloc(const m3_dims* dims, void* stream, m3_state** out);
+
+/* Wrap caller-owned device buffers (h, carry_B, carry_x in the layouts above) as a
+ * state.  The library does not free them; m3_state_free releases only the handle. */
+m3_status m3_state_wrap(const m3_dims* dims, float* h, float* carry_B, float* carry_x,
+                        m3_state** out);
+
+/* Release the handle (and the memory, if m3_state_alloc made it). */
+m3_status m3_state_free(m3_state* state);
+
+/* Device pointers of the three state tensors (any out pointer may be NULL). */
+m3_status m3_state_tensors(const m3_state* state, float** h, float** carry_B, float** carry_x);
+
+/* Copy the whole state (h, then carry_B, then carry_x, fp32) to / from a host
+ * buffer of exactly m3_state_bytes bytes.  Synchronises `stream`. */
+m3_status m3_state_copy_to_host(const m3_state* state, void* dst, size_t nbytes, void* stream);
+m3_status m3_state_copy_from_host(m3_state* state, const void* src, size_t nbytes, void* stream);
+
+/* ---- prefill (chunked scan) ------------------------------------------- */
+
+/* Scratch bytes m3_scan_fwd needs for these dims (0 when it needs none). */
+m3_status m3_scan_workspace_size(const m3_dims* dims, size_t* out_bytes);
+
+/* Run the layer core over L tokens of every sequence of the batch.
+ * state: in = state before token 0 (fresh or carried), out = state after token
+ * L-1 (h_{L-1} and the carry of token L-1).  y: (b, L, H, P) in dims->dtype.
+ * workspace: device scratch of at least m3_scan_workspace_size bytes (may be NULL
+ * when that size is 0).  L = 0 leaves the state unchanged and writes nothing.
+ * Mamba-3 paper note, sections その1-その3 (recurrence above); the chunked form
+ * follows the IBM Mamba page's SSD description (matrix form within a chunk,
+ * state passed between chunks). */
+m3_status m3_scan_fwd(const m3_dims* dims, const void* x, const float* dt, const float* A,
+                      const float* lam, const void* B, const void* C, const float* theta,
+                      const float* bias_B, const float* bias_C, const float* W_x,
+                      const float* W_o, const float* D, m3_state* state, void* y,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---- decode (one token) ------------------------------------------------ */
+
+/* Advance every sequence by one token.  Token inputs have L = 1 in the layouts
+ * above: x_t (b, H, P), dt_t/A_t/lam_t (b, H), B_t/C_t (b, G, R, N),
+ * theta_t (b, G, N/2); y_t (b, H, P).  dims->L is ignored.  Reads and rewrites the
+ * state in place.  Same recurrence as m3_scan_fwd (section その3 of the paper note:
+ * decode reads and writes the whole fixed-size state every token). */
+m3_status m3_decode_step(const m3_dims* dims, const void* x_t, const float* dt_t,
+                         const float* A_t, const float* lam_t, const void* B_t,
+                         const void* C_t, const float* theta_t, const float* bias_B,
+                         const float* bias_C, const float* W_x, const float* W_o,
+                         const float* D, m3_state* state, void* y_t, void* stream);
+
+/* ---- status -------------------------------------------------------------- */
+
+/* Synchronise `stream`, then return (and clear) the device status word:
+ * M3_OK, M3_ERR_TIMEOUT, or M3_ERR_CUDA if the stream reports an error. */
+m3_status m3_check(void* stream);
+
+/* Static description of a status code. */
+const char* m3_status_str(m3_status status);
+
+/* Library version string. */
+const char* m3_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* M3_H */

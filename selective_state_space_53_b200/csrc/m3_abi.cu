@@ -1,0 +1,312 @@
+// m3_abi.cu -- the extern "C" entry points of libm3 (declared in include/m3.h):
+// argument validation, state handles, kernel dispatch, status codes.
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "m3_common.cuh"
+
+namespace m3 {
+__device__ int g_status = 0;
+bool seq_scan_supported(int P, int N, int R);
+}  // namespace m3
+
+namespace {
+// Device address of the status word, looked up once per device.
+int* status_word() {
+  static int* cache[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!cache[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, m3::g_status) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<int*>(ptr);
+  }
+  return cache[dev];
+}
+}  // namespace
+
+struct m3_state {
+  m3_dims dims;
+  float* h;
+  float* carry_B;
+  float* carry_x;
+  void* block;  // single allocation owned by the library (null when wrapped)
+};
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+m3_status check_dims(const m3_dims* d) {
+  if (!d) return M3_ERR_NULL;
+  if (d->b < 0 || d->L < 0 || d->H < 1 || d->G < 1 || d->R < 1 || d->R > 8) return M3_ERR_DIMS;
+  if (d->P < 8 || d->P > 256 || (d->P % 8) != 0) return M3_ERR_DIMS;
+  if (d->N < 8 || d->N > 256 || (d->N % 8) != 0) return M3_ERR_DIMS;
+  if ((d->H % d->G) != 0) return M3_ERR_DIMS;
+  if (d->chunk < 0) return M3_ERR_DIMS;
+  if (d->dtype != M3_F32 && d->dtype != M3_BF16) return M3_ERR_DTYPE;
+  if (d->b * (int64_t)d->H > (int64_t)0x7fffffff) return M3_ERR_DIMS;
+  if (!m3::seq_scan_supported(d->P, d->N, d->R)) return M3_ERR_UNSUPPORTED;
+  return M3_OK;
+}
+
+size_t state_bytes(const m3_dims* d) {
+  const size_t bh = (size_t)d->b * d->H;
+  return sizeof(float) * bh * ((size_t)d->N * d->P + (size_t)d->R * d->N + d->P);
+}
+
+bool same_state_dims(const m3_dims* a, const m3_dims* s) {
+  return a->b == s->b && a->H == s->H && a->P == s->P && a->N == s->N && a->R == s->R;
+}
+
+// Validate the tensor operands shared by scan and decode.
+m3_status check_operands(const m3_dims* d, const void* x, const float* dt, const float* A,
+                         const float* lam, const void* B, const void* C, const float* theta,
+                         const float* bias_B, const float* bias_C, const float* W_x,
+                         const float* W_o, const float* D, const m3_state* state, const void* y,
+                         bool tokens) {
+  if (!state) return M3_ERR_NULL;
+  if (!same_state_dims(d, &state->dims)) return M3_ERR_STATE;
+  if (tokens) {
+    const void* req[] = {x, dt, A, lam, B, C, theta, y};
+    for (const void* q : req)
+      if (!q) return M3_ERR_NULL;
+  }
+  const void* all[] = {x, dt, A, lam, B, C, theta, bias_B, bias_C, W_x, W_o, D, y,
+                       state->h, state->carry_B, state->carry_x};
+  for (const void* q : all)
+    if (q && !aligned16(q)) return M3_ERR_ALIGN;
+  return M3_OK;
+}
+
+m3::Params make_params(const m3_dims* d, int64_t L, const void* x, const float* dt,
+                       const float* A, const float* lam, const void* B, const void* C,
+                       const float* theta, const float* bias_B, const float* bias_C,
+                       const float* W_x, const float* W_o, const float* D, m3_state* s,
+                       void* y) {
+  m3::Params p;
+  p.b = d->b;
+  p.L = L;
+  p.H = d->H;
+  p.P = d->P;
+  p.N = d->N;
+  p.R = d->R;
+  p.G = d->G;
+  p.dtype = d->dtype;
+  p.x = x;
+  p.dt = dt;
+  p.A = A;
+  p.lam = lam;
+  p.B = B;
+  p.C = C;
+  p.theta = theta;
+  p.bias_B = bias_B;
+  p.bias_C = bias_C;
+  p.W_x = W_x;
+  p.W_o = W_o;
+  p.D = D;
+  p.h = s->h;
+  p.carry_B = s->carry_B;
+  p.carry_x = s->carry_x;
+  p.y = y;
+  p.status = nullptr;
+  return p;
+}
+
+}  // namespace
+
+extern "C" {
+
+m3_status m3_state_bytes(const m3_dims* dims, size_t* out_bytes) {
+  m3_status st = check_dims(dims);
+  if (st != M3_OK) return st;
+  if (!out_bytes) return M3_ERR_NULL;
+  *out_bytes = state_bytes(dims);
+  return M3_OK;
+}
+
+m3_status m3_state_alloc(const m3_dims* dims, void* stream, m3_state** out) {
+  m3_status st = check_dims(dims);
+  if (st != M3_OK) return st;
+  if (!out) return M3_ERR_NULL;
+  *out = nullptr;
+  const size_t bytes = state_bytes(dims);
+  void* block = nullptr;
+  if (bytes > 0) {
+    if (cudaMalloc(&block, bytes) != cudaSuccess) return M3_ERR_CUDA;
+    if (cudaMemsetAsync(block, 0, bytes, (cudaStream_t)stream) != cudaSuccess) {
+      cudaFree(block);
+      return M3_ERR_CUDA;
+    }
+  }
+  m3_state* s = new (std::nothrow) m3_state;
+  if (!s) {
+    cudaFree(block);
+    return M3_ERR_CUDA;
+  }
+  const size_t bh = (size_t)dims->b * dims->H;
+  s->dims = *dims;
+  s->block = block;
+  s->h = static_cast<float*>(block);
+  s->carry_B = s->h + bh * dims->N * dims->P;
+  s->carry_x = s->carry_B + bh * dims->R * dims->N;
+  *out = s;
+  return M3_OK;
+}
+
+m3_status m3_state_wrap(const m3_dims* dims, float* h, float* carry_B, float* carry_x,
+                        m3_state** out) {
+  m3_status st = check_dims(dims);
+  if (st != M3_OK) return st;
+  if (!out) return M3_ERR_NULL;
+  *out = nullptr;
+  if ((dims->b * dims->H > 0) && (!h || !carry_B || !carry_x)) return M3_ERR_NULL;
+  if ((h && !aligned16(h)) || (carry_B && !aligned16(carry_B)) || (carry_x && !aligned16(carry_x)))
+    return M3_ERR_ALIGN;
+  m3_state* s = new (std::nothrow) m3_state;
+  if (!s) return M3_ERR_CUDA;
+  s->dims = *dims;
+  s->block = nullptr;
+  s->h = h;
+  s->carry_B = carry_B;
+  s->carry_x = carry_x;
+  *out = s;
+  return M3_OK;
+}
+
+m3_status m3_state_free(m3_state* state) {
+  if (!state) return M3_ERR_NULL;
+  m3_status st = M3_OK;
+  if (state->block && cudaFree(state->block) != cudaSuccess) st = M3_ERR_CUDA;
+  delete state;
+  return st;
+}
+
+m3_status m3_state_tensors(const m3_state* state, float** h, float** carry_B, float** carry_x) {
+  if (!state) return M3_ERR_NULL;
+  if (h) *h = state->h;
+  if (carry_B) *carry_B = state->carry_B;
+  if (carry_x) *carry_x = state->carry_x;
+  return M3_OK;
+}
+
+m3_status m3_state_copy_to_host(const m3_state* state, void* dst, size_t nbytes, void* stream) {
+  if (!state || !dst) return M3_ERR_NULL;
+  const m3_dims* d = &state->dims;
+  const size_t bh = (size_t)d->b * d->H;
+  const size_t nh = sizeof(float) * bh * d->N * d->P, nb = sizeof(float) * bh * d->R * d->N,
+               nx = sizeof(float) * bh * d->P;
+  if (nbytes != nh + nb + nx) return M3_ERR_STATE;
+  cudaStream_t s = (cudaStream_t)stream;
+  char* out = static_cast<char*>(dst);
+  if (cudaMemcpyAsync(out, state->h, nh, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemcpyAsync(out + nh, state->carry_B, nb, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaMemcpyAsync(out + nh + nb, state->carry_x, nx, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return M3_ERR_CUDA;
+  return M3_OK;
+}
+
+m3_status m3_state_copy_from_host(m3_state* state, const void* src, size_t nbytes, void* stream) {
+  if (!state || !src) return M3_ERR_NULL;
+  const m3_dims* d = &state->dims;
+  const size_t bh = (size_t)d->b * d->H;
+  const size_t nh = sizeof(float) * bh * d->N * d->P, nb = sizeof(float) * bh * d->R * d->N,
+               nx = sizeof(float) * bh * d->P;
+  if (nbytes != nh + nb + nx) return M3_ERR_STATE;
+  cudaStream_t s = (cudaStream_t)stream;
+  const char* in = static_cast<const char*>(src);
+  if (cudaMemcpyAsync(state->h, in, nh, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(state->carry_B, in + nh, nb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(state->carry_x, in + nh + nb, nx, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return M3_ERR_CUDA;
+  return M3_OK;
+}
+
+m3_status m3_scan_workspace_size(const m3_dims* dims, size_t* out_bytes) {
+  m3_status st = check_dims(dims);
+  if (st != M3_OK) return st;
+  if (!out_bytes) return M3_ERR_NULL;
+  *out_bytes = 0;
+  return M3_OK;
+}
+
+m3_status m3_scan_fwd(const m3_dims* dims, const void* x, const float* dt, const float* A,
+                      const float* lam, const void* B, const void* C, const float* theta,
+                      const float* bias_B, const float* bias_C, const float* W_x,
+                      const float* W_o, const float* D, m3_state* state, void* y,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  m3_status st = check_dims(dims);
+  if (st != M3_OK) return st;
+  const bool tokens = dims->b * dims->L > 0;
+  st = check_operands(dims, x, dt, A, lam, B, C, theta, bias_B, bias_C, W_x, W_o, D, state, y,
+                      tokens);
+  if (st != M3_OK) return st;
+  (void)workspace;
+  (void)workspace_bytes;
+  if (!tokens) return M3_OK;
+  m3::Params p = make_params(dims, dims->L, x, dt, A, lam, B, C, theta, bias_B, bias_C, W_x, W_o,
+                             D, state, y);
+  p.status = status_word();
+  if (!p.status) return M3_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e;
+  if (!(dims->flags & M3_FLAG_SEQUENTIAL) && m3::tc_scan_supported(p))
+    e = m3::launch_scan_tc(p, s);
+  else
+    e = m3::launch_scan_sequential(p, s);
+  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
+m3_status m3_decode_step(const m3_dims* dims, const void* x_t, const float* dt_t,
+                         const float* A_t, const float* lam_t, const void* B_t,
+                         const void* C_t, const float* theta_t, const float* bias_B,
+                         const float* bias_C, const float* W_x, const float* W_o,
+                         const float* D, m3_state* state, void* y_t, void* stream) {
+  m3_status st = check_dims(dims);
+  if (st != M3_OK) return st;
+  const bool tokens = dims->b > 0;
+  st = check_operands(dims, x_t, dt_t, A_t, lam_t, B_t, C_t, theta_t, bias_B, bias_C, W_x, W_o, D,
+                      state, y_t, tokens);
+  if (st != M3_OK) return st;
+  if (!tokens) return M3_OK;
+  m3::Params p = make_params(dims, 1, x_t, dt_t, A_t, lam_t, B_t, C_t, theta_t, bias_B, bias_C,
+                             W_x, W_o, D, state, y_t);
+  p.status = status_word();
+  if (!p.status) return M3_ERR_CUDA;
+  return m3::launch_scan_sequential(p, (cudaStream_t)stream) == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
+m3_status m3_check(void* stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return M3_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, m3::g_status, sizeof(int)) != cudaSuccess) return M3_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(m3::g_status, &zero, sizeof(int)) != cudaSuccess) return M3_ERR_CUDA;
+  }
+  return (m3_status)v;
+}
+
+const char* m3_status_str(m3_status status) {
+  switch (status) {
+    case M3_OK: return "ok";
+    case M3_ERR_DIMS: return "bad dimensions";
+    case M3_ERR_DTYPE: return "unsupported dtype";
+    case M3_ERR_ALIGN: return "tensor pointer not 16-byte aligned";
+    case M3_ERR_NULL: return "required pointer is NULL";
+    case M3_ERR_WORKSPACE: return "workspace missing or too small";
+    case M3_ERR_CUDA: return "CUDA error";
+    case M3_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
+    case M3_ERR_UNSUPPORTED: return "dimensions not supported by this build";
+    case M3_ERR_STATE: return "state does not match the dimensions";
+  }
+  return "unknown status";
+}
+
+const char* m3_version(void) { return "m3 0.1 (sm_100a)"; }
+
+}  // extern "C"
