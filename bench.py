@@ -98,58 +98,65 @@ def measured_peaks():
         return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
 
 
+_SAMPLER = r"""
+import sys, time, pynvml
+pynvml.nvmlInit()
+h = pynvml.nvmlDeviceGetHandleByIndex(int(sys.argv[1]))
+print("max", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM), flush=True)
+while True:
+    try:
+        print(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+              pynvml.nvmlDeviceGetCurrentClocksEventReasons(h), flush=True)
+    except Exception:
+        pass
+    time.sleep(float(sys.argv[2]))
+"""
+
+
 class ClockSampler:
-    """Samples SM clock and throttle reasons with NVML (read-only) while running."""
+    """Samples SM clock and clock-event reasons with NVML (read-only queries) from a
+    separate process while the timed region runs."""
 
     REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
-               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, index, period=0.005):
+    def __init__(self, index, period=0.002):
         self.index, self.period = index, period
         self.samples, self.reasons, self.max_mhz = [], set(), None
-        self._stop = threading.Event()
-        self._t = None
-        self.ok = False
+        self.proc = None
 
     def __enter__(self):
+        import subprocess
         try:
-            import pynvml
-            pynvml.nvmlInit()
-            self._nv = pynvml
-            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
-            self.ok = True
-            self._t = threading.Thread(target=self._run, daemon=True)
-            self._t.start()
+            self.proc = subprocess.Popen([sys.executable, "-c", _SAMPLER, str(self.index), str(self.period)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            first = self.proc.stdout.readline().split()   # wait until sampling runs
+            if first and first[0] == "max":
+                self.max_mhz = int(first[1])
         except Exception as e:  # sampling is best effort; the line says so
             log(f"clock sampling unavailable: {e}")
+            self.proc = None
         return self
 
-    def _run(self):
-        nv = self._nv
-        while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-                for bit, name in self.REASONS.items():
-                    if mask & bit:
-                        self.reasons.add(name)
-            except Exception:
-                pass
-            time.sleep(self.period)
-
     def __exit__(self, *exc):
-        self._stop.set()
-        if self._t is not None:
-            self._t.join()
+        if self.proc is not None:
+            time.sleep(3 * self.period)
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            for line in out.splitlines():
+                f = line.split()
+                if len(f) == 2:
+                    self.samples.append(int(f[0]))
+                    mask = int(f[1])
+                    for bit, name in self.REASONS.items():
+                        if mask & bit:
+                            self.reasons.add(name)
         return False
 
     def summary(self):
-        if not self.ok or not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-                    "samples": len(self.samples), "source": "nvml"}
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples), "source": "nvml, separate process"}
 
 
 # ------------------------------------------------------------------ our arm
