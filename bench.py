@@ -237,13 +237,15 @@ def run_ours(args):
     for s in ring:
         s["state1"] = m3.State.wrap(dims1, *s["keep"])
         s["y1"] = torch.empty_like(tok_dev["x"])
+    ws_bytes = m3.m3_scan_workspace_size(dims)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)  # steps run in stream order
     stream = torch.cuda.current_stream()
 
     def step(i, ev=None):
         s = ring[i % n_sets]
         if ev is not None:
             ev[0].record(stream)
-        m3.scan(dims, s["dev"], s["state"], y=s["y"])
+        m3.scan(dims, s["dev"], s["state"], y=s["y"], workspace=ws)
         if ev is not None:
             ev[1].record(stream)
         m3.decode(dims1, tok_dev, s["state1"], y=s["y1"])
@@ -269,7 +271,7 @@ def run_ours(args):
     prefill_ms = [a.elapsed_time(b) for a, b in evs]
     tokens_step = cfg["b"] * (cfg["L"] + 1)
     value = world * tokens_step * args.steps / (ms / 1e3)
-    gpu_launches = 2 * args.steps
+    gpu_launches = (3 if ws_bytes > 0 else 2) * args.steps  # [state pass] + full pass + decode
 
     pf_ms = statistics.mean(prefill_ms)
     pbytes = prefill_bytes(cfg)
@@ -396,6 +398,7 @@ def run_e2e(args, inp, tok_inp, device, world):
     st1 = m3.State.wrap(dims1, *keep)
     y = torch.empty_like(dev["x"])
     y1 = torch.empty_like(dtok["x"])
+    ws = torch.empty(max(m3.m3_scan_workspace_size(dims), 16), dtype=torch.uint8, device=device)
     y_host = torch.empty_like(y, device="cpu").pin_memory()
     y1_host = torch.empty_like(y1, device="cpu").pin_memory()
     stream = torch.cuda.current_stream()
@@ -409,7 +412,7 @@ def run_e2e(args, inp, tok_inp, device, world):
                 dev[k].copy_(v, non_blocking=True)
         for k, v in htok.items():
             dtok[k].copy_(v, non_blocking=True)
-        m3.scan(dims, dev, st, y=y)
+        m3.scan(dims, dev, st, y=y, workspace=ws)
         m3.decode(dims1, dtok, st1, y=y1)
         y_host.copy_(y, non_blocking=True)
         y1_host.copy_(y1, non_blocking=True)

@@ -107,9 +107,9 @@ m3::Params make_params(const m3_dims* d, int64_t L, const void* x, const float* 
   p.W_x = W_x;
   p.W_o = W_o;
   p.D = D;
-  p.h = s->h;
-  p.carry_B = s->carry_B;
-  p.carry_x = s->carry_x;
+  p.h = s ? s->h : nullptr;
+  p.carry_B = s ? s->carry_B : nullptr;
+  p.carry_x = s ? s->carry_x : nullptr;
   p.y = y;
   p.status = nullptr;
   return p;
@@ -231,6 +231,10 @@ m3_status m3_scan_workspace_size(const m3_dims* dims, size_t* out_bytes) {
   if (st != M3_OK) return st;
   if (!out_bytes) return M3_ERR_NULL;
   *out_bytes = 0;
+  if (dims->b * dims->L == 0) return M3_OK;
+  m3::Params p = make_params(dims, dims->L, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                             nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+  if (!(dims->flags & M3_FLAG_SEQUENTIAL) && m3::tc_scan_supported(p)) *out_bytes = m3::tc_scan_workspace_bytes(p);
   return M3_OK;
 }
 
@@ -245,19 +249,19 @@ m3_status m3_scan_fwd(const m3_dims* dims, const void* x, const float* dt, const
   st = check_operands(dims, x, dt, A, lam, B, C, theta, bias_B, bias_C, W_x, W_o, D, state, y,
                       tokens);
   if (st != M3_OK) return st;
-  (void)workspace;
-  (void)workspace_bytes;
   if (!tokens) return M3_OK;
   m3::Params p = make_params(dims, dims->L, x, dt, A, lam, B, C, theta, bias_B, bias_C, W_x, W_o,
                              D, state, y);
+  const bool tc = !(dims->flags & M3_FLAG_SEQUENTIAL) && m3::tc_scan_supported(p);
+  if (tc) {
+    const size_t need = m3::tc_scan_workspace_bytes(p);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return M3_ERR_WORKSPACE;
+    if (need > 0 && !aligned16(workspace)) return M3_ERR_ALIGN;
+  }
   p.status = status_word();
   if (!p.status) return M3_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e;
-  if (!(dims->flags & M3_FLAG_SEQUENTIAL) && m3::tc_scan_supported(p))
-    e = m3::launch_scan_tc(p, s);
-  else
-    e = m3::launch_scan_sequential(p, s);
+  const cudaError_t e = tc ? m3::launch_scan_tc(p, workspace, workspace_bytes, s) : m3::launch_scan_sequential(p, s);
   return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
 }
 

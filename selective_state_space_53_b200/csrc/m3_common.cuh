@@ -57,6 +57,7 @@ __device__ __forceinline__ void store_out(void* base, int64_t i, float v) {
 // Launchers (defined in the kernel files); return cudaGetLastError() of the launch.
 cudaError_t launch_scan_sequential(const Params& p, cudaStream_t stream);
 bool tc_scan_supported(const Params& p);
-cudaError_t launch_scan_tc(const Params& p, cudaStream_t stream);
+size_t tc_scan_workspace_bytes(const Params& p);  // scratch the chunked scan needs (0: none)
+cudaError_t launch_scan_tc(const Params& p, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 }  // namespace m3

@@ -1,41 +1,48 @@
-// m3_scan_tc.cu -- chunked Mamba-3 prefill scan on the sm_100a tensor cores (tcgen05 + TMEM).
+// m3_scan_tc.cu -- chunked Mamba-3 prefill scan on the sm_100a tensor cores (TMA + tcgen05 + TMEM).
 //
-// One CTA walks one (batch, head) sequence in tiles of Q = 128 / R tokens, so that a
-// tile has exactly 128 rows i = t * R + r (token t, MIMO branch r) -- the M of one
-// tcgen05.mma.  The chunked form is exact (the IBM Mamba page, SSD section: a
-// selective scan can be cut into chunks whose results combine associatively), so
-// the tile length does not change the result; for R = 4 it is the model's chunk of 32.
+// A CTA walks one segment of one (batch, head) sequence in tiles of Q = 128 / R tokens, so
+// that a tile has exactly 128 rows i = t * R + r (token t, MIMO branch r) -- the M of one
+// tcgen05.mma.  The chunked form is exact (IBM Mamba page, SSD section: the scan splits into
+// chunks combined associatively), so the tile length does not change the result; for R = 4
+// it is the model's chunk of 32 tokens.
 //
 // Per tile, with Lc_t the tile-local cumulative sum of dt A (log decay) and Phi_t the
-// cumulative rotation angle from the sequence start (kept per pair in fp64, reduced
-// mod 2 pi, so that fp32 angles stay small):
+// cumulative rotation angle from the segment start (kept per pair in fp64, reduced mod 2 pi):
 //   Bt_i = Rot(-Phi_t)(B_{t,r} + bias_B),  Ct_i = Rot(-Phi_t)(C_{t,r} + bias_C)
-//     -- the rotation absorbed into B and C as a data-dependent RoPE (Mamba-3 paper
-//        note, docsaid.org, section その2, statement 2);
-//   S  = Ct Bt^T                                     (MMA1, 128 x 128, K = N)
+//     -- the rotation absorbed into B and C as a data-dependent RoPE (Mamba-3 paper note,
+//        docsaid.org, section その2, statement 2);
+//   S  = Ct Bt^T                                        (MMA1, 128 x 128, K = N)
 //   S'[i,j] = S[i,j] e^{Lc_t - Lc_s} (gamma_s + [s<t] beta'_{s+1}) for s <= t, else 0
-//     -- the trapezoid weights of section その1 (gamma = lam dt, beta' = (1-lam) dt):
+//     -- the trapezoid weights of section その1 (gamma = lam dt, beta' = (1 - lam) dt):
 //        the input of token s enters h_s with gamma_s and h_{s+1} with beta'_{s+1};
-//   Y  = (e^{Lc_t} Ct) h+  +  S' X                    (MMA3 + MMA2, K = N and K = 128)
-//     with X_i = W_x[r] * x_t (MIMO branches, section その3), h+ the rotated-frame
-//     state entering the tile (plus the trapezoid carry of its last token);
-//   h+ <- e^{Lc_e} h+ + Xs^T Bt,  Xs_i = e^{Lc_e - Lc_t} (gamma_t + beta'_{t+1}) X_i
-//                                                     (MMA4, state update, K = 128)
+//   Y  = S' X + diag(e^{Lc}) Ct h+                      (MMA2 + MMA3)
+//     with X_i = W_x[r] * x_t (MIMO branches, section その3) and h+ the rotated-frame state
+//     entering the tile (including the previous token's trapezoid term);
+//   h+ <- e^{Lc_e} h+ + Xs^T Bt,  Xs_i = e^{Lc_e - Lc_t} (gamma_t + beta'_{t+1}) X_i   (MMA4)
 //   y_t = sum_r W_o[r] * Y_{t,r} + D x_t.
-// Working in the rotated frame (Bt, Ct carry the rotation) leaves the state a
-// plain decay-and-add; it is rotated back once at the end of the sequence.
+// In the rotated frame the state update is a plain decay-and-add; the state is rotated back
+// once, at the end of the sequence.
 //
-// Data layout on chip: Bt, Ct, e^{Lc}Ct, X, Xs and the bf16 copy of h+ are bf16
-// tiles in shared memory in the 128-byte-swizzled canonical UMMA layouts; the
-// accumulators S, Y, H = Xs^T Bt and the fp32 state h+ live in tensor memory
-// (columns 0, 128, 256, 384).  S is masked in place and consumed from TMEM as the
-// A operand of MMA2 (bf16 packed two per column).
+// Sequence splitting.  With few (batch, head) sequences the grid is b * H * nseg CTAs: a
+// state-only pass (MODE_STATE: Bt, Xs, MMA4, state update) first runs segments 0..nseg-2 from
+// a zero state and writes each segment's end state, total log decay and total angle to the
+// workspace; the full pass (MODE_FULL) then starts segment k from the combination of those
+// summaries.  Both passes are the same chunk algebra; only the starting state differs.
 //
-// Warp roles per tile: all 8 warps stage the tiles; thread 0 issues the MMAs and
-// commits them to an mbarrier; warps 0-3 mask S while warps 4-7 update the state;
-// all 8 warps run the epilogue (two column halves of Y).  Every mbarrier wait is
-// bounded by %globaltimer; a timeout sets M3_ERR_TIMEOUT and the CTA releases its
-// TMEM and returns.
+// On chip: B and C tiles arrive by TMA (cp.async.bulk.tensor, 128-byte swizzle) directly in
+// the canonical K-major UMMA layout and are rotated in place; x and theta arrive by TMA into
+// staging buffers.  The next tile's loads are issued as soon as the buffers they overwrite
+// are consumed, so they land while the current tile computes.  Accumulators S, Y, H and the
+// fp32 state live in tensor memory; the masked S is written back into TMEM as bf16 pairs and
+// consumed as the A operand of MMA2.
+//
+// Warp roles: all 8 warps stage tiles; thread 0 issues TMA and MMAs and commits the MMAs to
+// an mbarrier; warps 0-3 mask S while warps 4-7 update the state; all warps run the epilogue.
+// Every mbarrier wait is bounded by %globaltimer; a timeout sets M3_ERR_TIMEOUT in the device
+// status word and the CTA frees its TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "m3_common.cuh"
 
 namespace m3 {
@@ -43,23 +50,20 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kRows = 128;
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t TM_S = 0, TM_Y = 128, TM_H = 256, TM_ST = 384;
 constexpr unsigned kFull = 0xffffffffu;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s bound on any mbarrier wait
+constexpr int MODE_FULL = 0, MODE_STATE = 1;
 
 // ------------------------------------------------------------------ PTX helpers
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-
 __device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
                "r"(ncols));
@@ -70,18 +74,16 @@ __device__ __forceinline__ void tmem_relinquish() {
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
 }
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t done;
@@ -101,7 +103,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
   return true;
 }
-
+// TMA tile loads (no multicast), completion counted in bytes on `bar`.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+      "%5}], [%6];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
 // D[tmem] (+)= A[smem] * B[smem]
 __device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
@@ -117,11 +138,9 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint3
       "r"(a), "l"(b), "r"(idesc), "r"(acc));
 }
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
 }
-
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -164,7 +183,6 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
-
 // Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, dense.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
@@ -188,53 +206,96 @@ __device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
 }
-
-// Byte offset of 16-byte chunk `ch` of row `row` in a 128B-swizzled tile whose rows are
-// 128 bytes per 64-element block and whose blocks are `block_bytes` apart.
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+// Byte offset of 16-byte chunk `ch` of row `row` in a 128B-swizzled tile with 128-byte rows
+// per 64-element block, blocks `block_bytes` apart (the TMA SWIZZLE_128B / UMMA SW128 layout).
 __device__ __forceinline__ uint32_t sw128(int row, int ch, uint32_t block_bytes) {
   return (uint32_t)(ch >> 3) * block_bytes + (uint32_t)row * 128u + ((uint32_t)((ch & 7) ^ (row & 7)) << 4);
+}
+// sin and cos of an angle of moderate size: Cody-Waite reduction to [-pi, pi] with a two-term
+// split of 2 pi (Cody & Waite, "Software Manual for the Elementary Functions", 1980), then the
+// hardware approximations, which are accurate on that interval.
+__device__ __forceinline__ void sincos_reduced(float x, float* s, float* c) {
+  const float n = rintf(x * 0.15915494309189535f);
+  float r = fmaf(-n, 6.28318548202514648f, x);
+  r = fmaf(-n, -1.7484555314695172e-7f, r);
+  *s = __sinf(r);
+  *c = __cosf(r);
 }
 
 // ------------------------------------------------------------------ configuration
 
-template <int R, int N, int P>
+struct SegInfo {
+  int nseg;        // segments per sequence
+  int seg_tiles;   // tiles per segment
+  float* ws_init;  // (b*H, N, P): rotated-frame state entering segment 0 (nseg > 1)
+  float* ws_h;     // (b*H, nseg-1, N, P): end state of segments 0..nseg-2 from a zero start
+  float* ws_l;     // (b*H, nseg-1): total log decay of those segments
+  double* ws_phi;  // (b*H, nseg-1, N/2): total angle of those segments, reduced mod 2 pi
+};
+
+template <int R, int N, int P, int MODE>
 struct Cfg {
-  static constexpr int Q = kRows / R;  // tokens per tile
-  static constexpr int K2 = N / 2;     // rotation pairs
+  static constexpr bool FULL = (MODE == MODE_FULL);
+  static constexpr int Q = kRows / R;   // tokens per tile
+  static constexpr int K2 = N / 2;      // rotation pairs
+  // P = 64: the inter-chunk readout goes to the free half of the S columns after masking.
+  static constexpr bool kInterInS = (P == 64);
   static constexpr int TILE_N = kRows * N * 2;
   static constexpr int TILE_P = kRows * P * 2;
   static constexpr int TILE_H = P * N * 2;
   static constexpr int OFF_BT = 0;
   static constexpr int OFF_CT = OFF_BT + TILE_N;
-  static constexpr int OFF_C2 = OFF_CT + TILE_N;
-  static constexpr int OFF_X = OFF_C2 + TILE_N;
-  static constexpr int OFF_XS = OFF_X + TILE_P;
+  static constexpr int OFF_C2 = OFF_CT + (FULL ? TILE_N : 0);
+  static constexpr int OFF_X = OFF_C2 + ((FULL && !kInterInS) ? TILE_N : 0);
+  static constexpr int OFF_XS = OFF_X + (FULL ? TILE_P : 0);
   static constexpr int OFF_H = OFF_XS + TILE_P;
-  static constexpr int OFF_CS = OFF_H + TILE_H;  // float2 [Q][K2]
-  static constexpr int OFF_BIASB = OFF_CS + Q * K2 * 8;
-  static constexpr int OFF_BIASC = OFF_BIASB + R * N * 4;
-  static constexpr int OFF_WX = OFF_BIASC + R * N * 4;
-  static constexpr int OFF_WO = OFF_WX + R * P * 4;
-  static constexpr int OFF_BASE = OFF_WO + R * P * 4;  // double [K2]
-  static constexpr int TOKF = Q + 4;                    // floats per per-token array
-  static constexpr int OFF_TOK = OFF_BASE + K2 * 8;     // 8 arrays of TOKF floats
-  static constexpr int OFF_MISC = OFF_TOK + 8 * TOKF * 4;
+  static constexpr int OFF_CS = OFF_H + (FULL ? TILE_H : 0);       // float2 [Q][K2]
+  static constexpr int OFF_TH = OFF_CS + Q * K2 * 4;                // theta staging: 2nd half of CS
+  static constexpr int OFF_XSTG = OFF_CS + Q * K2 * 8;              // x staging [Q][P] bf16
+  static constexpr int OFF_WX = OFF_XSTG + Q * P * 2;              // W_x [R][P]
+  static constexpr int OFF_BASE = OFF_WX + R * P * 4;               // double [K2]
+  static constexpr int SEGS = kThreads / K2;                        // angle prefix segments
+  static constexpr int SEGLEN = (Q + SEGS - 1) / SEGS;
+  static constexpr int OFF_SEGSUM = OFF_BASE + K2 * 8;              // float [SEGS][K2]
+  static constexpr int TOKF = Q + 4;
+  static constexpr int OFF_TOK = OFF_SEGSUM + SEGS * K2 * 4;        // per-token float arrays
+  static constexpr int NTOKARR = 10;
+  static constexpr int OFF_MREC = OFF_TOK + NTOKARR * TOKF * 4;     // float4 [Q] mask records
+  static constexpr int OFF_MISC = OFF_MREC + Q * 16;
   static constexpr int BYTES = OFF_MISC + 64;
   static constexpr int SMEM = BYTES + 1024;  // slack for 1024-byte alignment
-  static constexpr int SEGS = kThreads / K2;  // angle prefix: segments per pair
-  static constexpr int SEGLEN = (Q + SEGS - 1) / SEGS;
+  // tensor memory columns
+  static constexpr uint32_t TM_S = 0;
+  static constexpr uint32_t TM_YI = 64;            // kInterInS: Ct h+ in S columns 64..64+P
+  static constexpr uint32_t TM_Y = 128;
+  static constexpr uint32_t TM_H = 128 + P;
+  static constexpr uint32_t TM_ST = (P == 64) ? TM_H : TM_H + N;  // P = 64: lanes 16-31 of H's columns
+  static constexpr uint32_t TMEM_NEED = (P == 64) ? (TM_H + N) : (TM_ST + N);
+  static constexpr uint32_t TMEM_COLS = TMEM_NEED <= 256 ? 256 : 512;
   static constexpr uint32_t ID_S = idesc_bf16(128, 128, false, false);
   static constexpr uint32_t ID_Y3 = idesc_bf16(128, P, false, false);
   static constexpr uint32_t ID_H = idesc_bf16(P, N, true, true);
   static constexpr uint32_t ID_Y2 = idesc_bf16(128, P, false, true);
+  static constexpr int TX_B = kRows * N * 2;
+  static constexpr int TX_X = Q * P * 2;
+  static constexpr int TX_T = Q * K2 * 4;
 };
 
-// per-token array slots
-enum { T_LA = 0, T_GAM = 1, T_BP = 2, T_LC = 3, T_DEC = 4, T_CW = 5, T_DT = 6, T_SCAL = 7 };
+// per-token array slots (each TOKF floats)
+enum { A_DT0 = 0, A_A0, A_LM0, A_DT1, A_A1, A_LM1, A_GAM, A_CW, A_DEC, A_SCAL };
 
-template <int R, int N, int P>
-__global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(Params p) {
-  using C = Cfg<R, N, P>;
+template <int R, int N, int P, int MODE>
+__global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
+    scan_tc_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
+                   const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmT,
+                   const Params p, const SegInfo sg) {
+  using C = Cfg<R, N, P, MODE>;
+  constexpr bool FULL = C::FULL;
   constexpr int Q = C::Q;
   constexpr int K2 = C::K2;
   extern __shared__ uint8_t smem_raw[];
@@ -243,94 +304,192 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(Params p) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = p.H, G = p.G;
   const int64_t L = p.L;
-  const int bh = blockIdx.x;
+  // segment decomposition
+  const int nseg_grid = FULL ? sg.nseg : (sg.nseg - 1);
+  const int bh = blockIdx.x / nseg_grid;
+  const int seg = blockIdx.x % nseg_grid;
   const int bi = bh / H, hi = bh % H;
   const int g = hi / (H / G);
+  const int64_t ntiles_seq = (L + Q - 1) / Q;
+  const int64_t j0 = (int64_t)seg * sg.seg_tiles;
+  const int64_t j1 = (j0 + sg.seg_tiles < ntiles_seq) ? (j0 + sg.seg_tiles) : ntiles_seq;
+  const bool last_seg = (seg == sg.nseg - 1);
+  const int64_t tok_base = (int64_t)bi * L;  // first token of this sequence (flattened b*L index)
 
   const uint32_t sBT = smem_u32(sm + C::OFF_BT), sCT = smem_u32(sm + C::OFF_CT), sC2 = smem_u32(sm + C::OFF_C2);
   const uint32_t sX = smem_u32(sm + C::OFF_X), sXS = smem_u32(sm + C::OFF_XS), sH = smem_u32(sm + C::OFF_H);
+  const uint32_t sXSTG = smem_u32(sm + C::OFF_XSTG), sTH = smem_u32(sm + C::OFF_TH);
   float2* cs = reinterpret_cast<float2*>(sm + C::OFF_CS);
-  float* biasB = reinterpret_cast<float*>(sm + C::OFF_BIASB);
-  float* biasC = reinterpret_cast<float*>(sm + C::OFF_BIASC);
+  const float* th_stg = reinterpret_cast<const float*>(sm + C::OFF_TH);
   float* wx = reinterpret_cast<float*>(sm + C::OFF_WX);
-  float* wo = reinterpret_cast<float*>(sm + C::OFF_WO);
   double* base = reinterpret_cast<double*>(sm + C::OFF_BASE);
+  float* segsum = reinterpret_cast<float*>(sm + C::OFF_SEGSUM);
   float* tokf = reinterpret_cast<float*>(sm + C::OFF_TOK);
-  float* la = tokf + T_LA * C::TOKF;
-  float* gam = tokf + T_GAM * C::TOKF;
-  float* bpv = tokf + T_BP * C::TOKF;
-  float* Lc = tokf + T_LC * C::TOKF;
-  float* dec0 = tokf + T_DEC * C::TOKF;
-  float* cw = tokf + T_CW * C::TOKF;
-  float* dtv = tokf + T_DT * C::TOKF;
-  float* scal = tokf + T_SCAL * C::TOKF;  // [0] = e^{Lc_e}
-  uint64_t* mbar = reinterpret_cast<uint64_t*>(sm + C::OFF_MISC);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC + 8);
+  float4* mrec = reinterpret_cast<float4*>(sm + C::OFF_MREC);
+  float* gamA = tokf + A_GAM * C::TOKF;
+  float* cwA = tokf + A_CW * C::TOKF;
+  float* decA = tokf + A_DEC * C::TOKF;
+  float* scal = tokf + A_SCAL * C::TOKF;  // [0] e^{Lc_e}, [1] tile log decay, [2..3] next-token beta' by parity
+  uint64_t* mma_bar = reinterpret_cast<uint64_t*>(sm + C::OFF_MISC);
+  uint64_t* load_bar = reinterpret_cast<uint64_t*>(sm + C::OFF_MISC + 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC + 16);
 
   const __nv_bfloat16* xg = static_cast<const __nv_bfloat16*>(p.x);
   const __nv_bfloat16* Bg = static_cast<const __nv_bfloat16*>(p.B);
-  const __nv_bfloat16* Cg = static_cast<const __nv_bfloat16*>(p.C);
   __nv_bfloat16* yg = static_cast<__nv_bfloat16*>(p.y);
-  const float Dh = p.D ? p.D[hi] : 0.0f;
+  const float Dh = (FULL && p.D) ? p.D[hi] : 0.0f;
+
+  // ---- issue the TMA loads of tile j (thread 0); B/C boxes: 64 columns x R x 1 x Q tokens
+  auto issue_loads = [&](int64_t j) {
+    const int tok = (int)(tok_base + j * Q);
+    constexpr uint32_t tx = C::TX_B * (FULL ? 2 : 1) + (C::TX_X) + C::TX_T;
+    mbar_expect_tx(load_bar, tx);
+#pragma unroll
+    for (int blk = 0; blk < N / 64; ++blk) {
+      tma_load_4d(sBT + blk * (kRows * 128), &tmB, 64 * blk, 0, g, tok, load_bar);
+      if constexpr (FULL) tma_load_4d(sCT + blk * (kRows * 128), &tmC, 64 * blk, 0, g, tok, load_bar);
+    }
+    tma_load_3d(sXSTG, &tmX, 0, hi, tok, load_bar);
+    tma_load_3d(sTH, &tmT, 0, g, tok, load_bar);
+  };
+  // per-token coefficient loads (registers), tile j: threads t < Q; thread Q loads the
+  // first token after tile j (its beta' is the carry weight of the tile's last token)
+  float r_dt = 0.f, r_a = 0.f, r_lm = 0.f;
+  auto load_coefs = [&](int64_t j) {
+    const int64_t c0 = j * Q;
+    if (tid < Q) {
+      const int64_t t = c0 + tid;
+      r_dt = r_a = r_lm = 0.0f;
+      if (t < L) {
+        const int64_t ti = (tok_base + t) * H + hi;
+        r_dt = p.dt[ti];
+        r_a = p.A[ti];
+        r_lm = p.lam[ti];
+      }
+    } else if (tid == Q) {
+      const int64_t t = c0 + Q;
+      r_dt = r_lm = 0.0f;
+      if (t < L) {
+        const int64_t ti = (tok_base + t) * H + hi;
+        r_dt = p.dt[ti];
+        r_lm = p.lam[ti];
+      }
+    }
+  };
+  auto store_coefs = [&](int par) {
+    if (tid < Q) {
+      tokf[(A_DT0 + 3 * par) * C::TOKF + tid] = r_dt;
+      tokf[(A_A0 + 3 * par) * C::TOKF + tid] = r_a;
+      tokf[(A_LM0 + 3 * par) * C::TOKF + tid] = r_lm;
+    } else if (tid == Q) {
+      scal[2 + par] = (1.0f - r_lm) * r_dt;
+    }
+  };
 
   // ---- setup
   if (warp == 0) {
-    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (tid == 0) mbar_init(mbar, 1);
-  for (int i = tid; i < R * N; i += kThreads) {
-    biasB[i] = p.bias_B ? p.bias_B[(int64_t)hi * R * N + i] : 0.0f;
-    biasC[i] = p.bias_C ? p.bias_C[(int64_t)hi * R * N + i] : 0.0f;
+  if (tid == 0) {
+    mbar_init(mma_bar, 1);
+    mbar_init(load_bar, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tmB);
+    if constexpr (FULL) prefetch_tmap(&tmC);
+    prefetch_tmap(&tmX);
+    prefetch_tmap(&tmT);
   }
-  for (int i = tid; i < R * P; i += kThreads) {
-    wx[i] = p.W_x ? p.W_x[(int64_t)hi * R * P + i] : 1.0f;
-    wo[i] = p.W_o ? p.W_o[(int64_t)hi * R * P + i] : 1.0f;
-  }
+  for (int i = tid; i < R * P; i += kThreads) wx[i] = p.W_x ? p.W_x[(int64_t)hi * R * P + i] : 1.0f;
+  const float* biasBg = p.bias_B ? p.bias_B + (int64_t)hi * R * N : nullptr;
+  const float* biasCg = p.bias_C ? p.bias_C + (int64_t)hi * R * N : nullptr;
+  const float* wog = p.W_o ? p.W_o + (int64_t)hi * R * P : nullptr;
   for (int k = tid; k < K2; k += kThreads) base[k] = 0.0;
+  load_coefs(j0);
+  store_coefs(0);
+  if (j0 + 1 < j1) load_coefs(j0 + 1);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (tid == 0 && j0 < j1) issue_loads(j0);
 
-  // state warps: lanes of the P-row accumulators (M = 128: p = lane quarter * 32 + lane;
-  // M = 64: rows 16 per quarter in lanes 0-15)
+  // state warps: TMEM lane of accumulator row p (M = 128: lane = p; M = 64: rows in lanes
+  // 0-15 of each quarter, and the state is kept in lanes 16-31 of the same columns)
   const int q4 = warp & 3;
   const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
-  const int prow = (P == 128) ? (32 * q4 + lane) : (16 * q4 + lane);
-  const bool pvalid = (P == 128) || (lane < 16);
   const bool state_warp = warp >= 4;
+  const int prow = (P == 128) ? (32 * q4 + lane) : (16 * q4 + (lane & 15));
+  const bool st_owner = (P == 128) || (lane >= 16);  // holds the fp32 state of row prow
 
-  // ---- initial rotated-frame state h+ = h_{-1} + beta'_0 u_{-1} (angle 0 at the start)
+  // ---- incoming rotated-frame state h+ of this segment
+  //   nseg == 1 (full pass): h_{-1} + beta'_0 u_{-1} from the state / carry;
+  //   state pass, segment 0: same, written to ws_init; other state-pass segments: zero;
+  //   full pass, segment k > 0: ws_init folded through the summaries of segments 0..k-1.
   if (state_warp) {
-    const int64_t tok0 = (int64_t)bi * L;
-    const float bp0 = (1.0f - p.lam[tok0 * H + hi]) * p.dt[tok0 * H + hi];
+    const bool from_state = (sg.nseg == 1) || (!FULL && seg == 0);
     float xprev[R];
+    float bp0 = 0.0f;
+    if (from_state) {
+      bp0 = (1.0f - p.lam[tok_base * H + hi]) * p.dt[tok_base * H + hi];
 #pragma unroll
-    for (int r = 0; r < R; ++r)
-      xprev[r] = pvalid ? wx[r * P + prow] * p.carry_x[(int64_t)bh * P + prow] : 0.0f;
+      for (int r = 0; r < R; ++r) xprev[r] = wx[r * P + prow] * p.carry_x[(int64_t)bh * P + prow];
+    }
     const float* h0 = p.h + (int64_t)bh * N * P;
     const float* cB = p.carry_B + (int64_t)bh * R * N;
 #pragma unroll 1
     for (int c = 0; c < N / 32; ++c) {
-      uint32_t v[32];
+      float v[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int n = 32 * c + e;
-        float u = 0.0f;
+      for (int e = 0; e < 32; ++e) v[e] = 0.0f;
+      if (from_state) {
 #pragma unroll
-        for (int r = 0; r < R; ++r) u = fmaf(cB[r * N + n] + biasB[r * N + n], xprev[r], u);
-        const float hv = pvalid ? fmaf(bp0, u, h0[(int64_t)n * P + prow]) : 0.0f;
-        v[e] = __float_as_uint(hv);
+        for (int e = 0; e < 32; ++e) {
+          const int n = 32 * c + e;
+          float u = 0.0f;
+#pragma unroll
+          for (int r = 0; r < R; ++r) u = fmaf(cB[r * N + n] + (biasBg ? __ldg(biasBg + r * N + n) : 0.0f), xprev[r], u);
+          v[e] = fmaf(bp0, u, h0[(int64_t)n * P + prow]);
+        }
+        if (!FULL && sg.nseg > 1 && st_owner) {
+          float* wi = sg.ws_init + (int64_t)bh * N * P;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) wi[(int64_t)(32 * c + e) * P + prow] = v[e];
+        }
+      } else if (FULL) {
+        const float* wi = sg.ws_init + (int64_t)bh * N * P;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = wi[(int64_t)(32 * c + e) * P + prow];
+        for (int k = 0; k < seg; ++k) {
+          const int64_t sidx = (int64_t)bh * (sg.nseg - 1) + k;
+          const float dec = __expf(sg.ws_l[sidx]);
+          const float* wh = sg.ws_h + sidx * N * P;
+          const double* ph = sg.ws_phi + sidx * K2;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int n0 = 32 * c + 2 * e;
+            float sn, cn;
+            sincosf((float)ph[n0 / 2], &sn, &cn);
+            const float a0 = fmaf(dec, v[2 * e], wh[(int64_t)n0 * P + prow]);
+            const float a1 = fmaf(dec, v[2 * e + 1], wh[(int64_t)(n0 + 1) * P + prow]);
+            v[2 * e] = cn * a0 - sn * a1;
+            v[2 * e + 1] = sn * a0 + cn * a1;
+          }
+        }
       }
-      tmem_st32(tmem + lane_base + TM_ST + 32 * c, v);
-      if (pvalid) {
+      uint32_t u32[32];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float f[8];
+      for (int e = 0; e < 32; ++e) u32[e] = __float_as_uint(v[e]);
+      tmem_st32(tmem + lane_base + C::TM_ST + 32 * c, u32);
+      if constexpr (FULL) {
+        if (st_owner) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * q + e]);
-          sts128(sH + sw128(prow, 4 * c + q, P * 128), pack8(f));
+          for (int q = 0; q < 4; ++q) {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = v[8 * q + e];
+            sts128(sH + sw128(prow, 4 * c + q, P * 128), pack8(f));
+          }
         }
       }
     }
@@ -341,40 +500,28 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(Params p) {
   __syncthreads();
   tc_fence_after();
 
-  uint32_t phase = 0;
+  uint32_t mma_phase = 0, load_phase = 0;
   bool failed = false;
-  const int64_t ntiles = (L + Q - 1) / Q;
-  for (int64_t j = 0; j < ntiles; ++j) {
+  float seg_logdec = 0.0f;
+  for (int64_t j = j0; j < j1; ++j) {
     const int64_t c0 = j * Q;
     const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
+    const int par = (int)((j - j0) & 1);
+    const float* dtA = tokf + (A_DT0 + 3 * par) * C::TOKF;
+    const float* aA = tokf + (A_A0 + 3 * par) * C::TOKF;
+    const float* lmA = tokf + (A_LM0 + 3 * par) * C::TOKF;
 
-    // ---- A1: per-token coefficients (invalid tail tokens are identity steps)
-    if (tid < Q) {
-      const int t = tid;
-      if (t < nv) {
-        const int64_t ti = ((int64_t)bi * L + c0 + t) * H + hi;
-        const float d = p.dt[ti], lm = p.lam[ti];
-        la[t] = d * p.A[ti];
-        gam[t] = lm * d;
-        bpv[t] = (1.0f - lm) * d;
-        dtv[t] = d;
-      } else {
-        la[t] = 0.0f;
-        gam[t] = 0.0f;
-        bpv[t] = 0.0f;
-        dtv[t] = 0.0f;
+    // ---- wait for this tile's TMA loads
+    {
+      const bool ok = mbar_wait(load_bar, load_phase);
+      load_phase ^= 1;
+      if (__syncthreads_or(!ok)) {
+        failed = true;
+        break;
       }
-    } else if (tid == Q) {
-      float nb = 0.0f;
-      if (c0 + Q < L) {
-        const int64_t ti = ((int64_t)bi * L + c0 + Q) * H + hi;
-        nb = (1.0f - p.lam[ti]) * p.dt[ti];
-      }
-      bpv[Q] = nb;
     }
-    __syncthreads();
 
-    // ---- A2: cumulative log decay (warp 0) and angle partial sums (all threads)
+    // ---- A: coefficients (warp 0), angle prefixes (all threads)
     if (warp == 0) {
       constexpr int PER = (Q + 31) / 32;
       float loc[PER];
@@ -382,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(Params p) {
 #pragma unroll
       for (int e = 0; e < PER; ++e) {
         const int t = lane * PER + e;
-        run += (t < Q) ? la[t] : 0.0f;
+        run += (t < Q) ? dtA[t] * aA[t] : 0.0f;
         loc[e] = run;
       }
       float incl = run;
@@ -391,117 +538,143 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(Params p) {
         const float nbv = __shfl_up_sync(kFull, incl, off);
         if (lane >= off) incl += nbv;
       }
+      const float Le = __shfl_sync(kFull, incl, 31);
       const float excl = incl - run;
 #pragma unroll
       for (int e = 0; e < PER; ++e) {
         const int t = lane * PER + e;
-        if (t < Q) Lc[t] = excl + loc[e];
+        if (t < Q) {
+          const float Lct = excl + loc[e];
+          const float gm = lmA[t] * dtA[t];
+          const float bpn = (t + 1 < Q) ? (1.0f - lmA[t + 1]) * dtA[t + 1] : scal[2 + par];
+          // mask record: log2 cumulative decay, gamma, gamma + beta'_{t+1}
+          mrec[t] = make_float4(Lct * 1.4426950408889634f, gm, gm + bpn, 0.0f);
+          gamA[t] = gm;
+          cwA[t] = __expf(Le - Lct) * (gm + bpn);
+          decA[t] = __expf(Lct);
+        }
       }
-      __syncwarp();
-      const float Le = Lc[Q - 1];
-      for (int t = lane; t < Q; t += 32) {
-        dec0[t] = __expf(Lc[t]);
-        cw[t] = __expf(Le - Lc[t]) * (gam[t] + bpv[t + 1]);
+      if (lane == 0) {
+        scal[0] = __expf(Le);
+        scal[1] = Le;
       }
-      if (lane == 0) scal[0] = __expf(Le);
     }
     const int ak = tid % K2, aseg = tid / K2;
+    float aloc[C::SEGLEN];
+    double ang_total = 0.0;
     {
       float run = 0.0f;
-      const float* th = p.theta + (((int64_t)bi * L + c0) * G + g) * K2 + ak;
+#pragma unroll
+      for (int e = 0; e < C::SEGLEN; ++e) {
+        const int t = aseg * C::SEGLEN + e;
+        if (t < Q) run += (t < nv) ? dtA[t] * th_stg[t * K2 + ak] : 0.0f;
+        aloc[e] = run;
+      }
+      segsum[aseg * K2 + ak] = run;
+    }
+    __syncthreads();
+    {
+      double total = 0.0;
+      float aoff = 0.0f;
+      for (int s = 0; s < C::SEGS; ++s) {
+        const float v = segsum[s * K2 + ak];
+        if (s < aseg) aoff += v;
+        total += (double)v;
+      }
+      aoff += (float)base[ak];
+      // theta staging (2nd half of cs) is consumed: every thread read its values above
+#pragma unroll
       for (int e = 0; e < C::SEGLEN; ++e) {
         const int t = aseg * C::SEGLEN + e;
         if (t < Q) {
-          run += (t < nv) ? dtv[t] * th[(int64_t)t * G * K2] : 0.0f;
-          cs[t * K2 + ak].x = run;
+          float sn, cn;
+          sincos_reduced(aoff + aloc[e], &sn, &cn);
+          cs[t * K2 + ak] = make_float2(cn, sn);
         }
       }
+      ang_total = total;
     }
+    if (tid == 0) seg_logdec += scal[1];
     __syncthreads();
-    float aoff = (float)base[ak];
-    double total = 0.0;
-    for (int s = 0; s < C::SEGS; ++s) {
-      const int tend = ((s + 1) * C::SEGLEN < Q ? (s + 1) * C::SEGLEN : Q) - 1;
-      if (s * C::SEGLEN < Q) {
-        const float segsum = cs[tend * K2 + ak].x;
-        if (s < aseg) aoff += segsum;
-        total += (double)segsum;
-      }
-    }
-    __syncthreads();
-    for (int e = 0; e < C::SEGLEN; ++e) {
-      const int t = aseg * C::SEGLEN + e;
-      if (t < Q) {
-        float sn, cn;
-        sincosf(aoff + cs[t * K2 + ak].x, &sn, &cn);
-        cs[t * K2 + ak] = make_float2(cn, sn);
-      }
-    }
+    // every thread has read base[]: advance it by this tile's total angle
     if (aseg == 0) {
-      double nbse = base[ak] + total;
-      nbse -= 6.283185307179586 * rint(nbse * 0.15915494309189535);
-      base[ak] = nbse;
+      double nb = base[ak] + ang_total;
+      nb -= 6.283185307179586 * rint(nb * 0.15915494309189535);
+      base[ak] = nb;
     }
-    __syncthreads();
 
-    // ---- B: stage the bf16 operand tiles (rows i = t * R + r)
+    // ---- B: rotate B (and C) in place; build X, Xs (and e^{Lc} C~)
     {
       constexpr int CHN = N / 8;
-      for (int idx = tid; idx < kRows * CHN; idx += kThreads) {
-        const int i = idx / CHN, ch = idx % CHN;
-        const int t = i / R, r = i % R;
-        uint4 ob = make_uint4(0, 0, 0, 0), oc = ob, oc2 = ob;
-        if (t < nv) {
-          const int64_t row = ((((int64_t)bi * L + c0 + t) * G + g) * R + r) * N + ch * 8;
-          float fb[8], fc[8];
-          unpack8(__ldg(reinterpret_cast<const uint4*>(Bg + row)), fb);
-          unpack8(__ldg(reinterpret_cast<const uint4*>(Cg + row)), fc);
+      constexpr int ROWS_PER_IT = kThreads / CHN;
+      const int ch = tid % CHN;
+      const int r = (tid / CHN) % R;  // fixed: ROWS_PER_IT is a multiple of R
+      float bB[8], bC[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            fb[e] += biasB[r * N + ch * 8 + e];
-            fc[e] += biasC[r * N + ch * 8 + e];
-          }
+      for (int e = 0; e < 8; ++e) {
+        bB[e] = biasBg ? __ldg(biasBg + r * N + ch * 8 + e) : 0.0f;
+        bC[e] = biasCg ? __ldg(biasCg + r * N + ch * 8 + e) : 0.0f;
+      }
+#pragma unroll 2
+      for (int i = tid / CHN; i < kRows; i += ROWS_PER_IT) {
+        const int t = i / R;
+        const uint32_t off = sw128(i, ch, kRows * 128);
+        const float4 w01 = *reinterpret_cast<const float4*>(&cs[t * K2 + ch * 4]);
+        const float4 w23 = *reinterpret_cast<const float4*>(&cs[t * K2 + ch * 4 + 2]);
+        const float wc[4] = {w01.x, w01.z, w23.x, w23.z};
+        const float ws[4] = {w01.y, w01.w, w23.y, w23.w};
+        const bool valid = t < nv;
+        {
+          float f[8];
+          unpack8(lds128(sBT + off), f);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const float2 w = cs[t * K2 + ch * 4 + q];  // (cos Phi, sin Phi); apply Rot(-Phi)
-            const float b0 = fb[2 * q], b1 = fb[2 * q + 1], d0 = fc[2 * q], d1 = fc[2 * q + 1];
-            fb[2 * q] = w.x * b0 + w.y * b1;
-            fb[2 * q + 1] = w.x * b1 - w.y * b0;
-            fc[2 * q] = w.x * d0 + w.y * d1;
-            fc[2 * q + 1] = w.x * d1 - w.y * d0;
+            const float b0 = f[2 * q] + bB[2 * q], b1 = f[2 * q + 1] + bB[2 * q + 1];
+            f[2 * q] = valid ? (wc[q] * b0 + ws[q] * b1) : 0.0f;  // Rot(-Phi)
+            f[2 * q + 1] = valid ? (wc[q] * b1 - ws[q] * b0) : 0.0f;
           }
-          ob = pack8(fb);
-          oc = pack8(fc);
-          const float dd = dec0[t];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) fc[e] *= dd;
-          oc2 = pack8(fc);
+          sts128(sBT + off, pack8(f));
         }
-        const uint32_t off = sw128(i, ch, kRows * 128);
-        sts128(sBT + off, ob);
-        sts128(sCT + off, oc);
-        sts128(sC2 + off, oc2);
+        if constexpr (FULL) {
+          float f[8];
+          unpack8(lds128(sCT + off), f);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float d0 = f[2 * q] + bC[2 * q], d1 = f[2 * q + 1] + bC[2 * q + 1];
+            f[2 * q] = valid ? (wc[q] * d0 + ws[q] * d1) : 0.0f;
+            f[2 * q + 1] = valid ? (wc[q] * d1 - ws[q] * d0) : 0.0f;
+          }
+          sts128(sCT + off, pack8(f));
+          if constexpr (!C::kInterInS) {
+            const float dd = decA[t];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] *= dd;
+            sts128(sC2 + off, pack8(f));
+          }
+        }
       }
       constexpr int CHP = P / 8;
-      for (int idx = tid; idx < kRows * CHP; idx += kThreads) {
-        const int i = idx / CHP, ch = idx % CHP;
-        const int t = i / R, r = i % R;
-        uint4 ox = make_uint4(0, 0, 0, 0), oxs = ox;
-        if (t < nv) {
-          const int64_t row = (((int64_t)bi * L + c0 + t) * H + hi) * P + ch * 8;
-          float fx[8];
-          unpack8(__ldg(reinterpret_cast<const uint4*>(xg + row)), fx);
+      for (int idx = tid; idx < Q * CHP; idx += kThreads) {
+        const int t = idx / CHP, chp = idx % CHP;
+        float fx[8];
+        unpack8(lds128(sXSTG + (uint32_t)(t * P + chp * 8) * 2), fx);
+        const bool valid = t < nv;
+        const float cwt = cwA[t];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) fx[e] *= wx[r * P + ch * 8 + e];
-          ox = pack8(fx);
-          const float cwt = cw[t];
+        for (int rr = 0; rr < R; ++rr) {
+          const int i = t * R + rr;
+          const float4 w0 = *reinterpret_cast<const float4*>(&wx[rr * P + chp * 8]);
+          const float4 w1 = *reinterpret_cast<const float4*>(&wx[rr * P + chp * 8 + 4]);
+          const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+          float xr[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) fx[e] *= cwt;
-          oxs = pack8(fx);
+          for (int e = 0; e < 8; ++e) xr[e] = valid ? fx[e] * wv[e] : 0.0f;
+          const uint32_t off = sw128(i, chp, kRows * 128);
+          if constexpr (FULL) sts128(sX + off, pack8(xr));
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xr[e] *= cwt;
+          sts128(sXS + off, pack8(xr));
         }
-        const uint32_t off = sw128(i, ch, kRows * 128);
-        sts128(sX + off, ox);
-        sts128(sXS + off, oxs);
       }
     }
     fence_async_smem();
@@ -509,224 +682,465 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(Params p) {
     __syncthreads();
     tc_fence_after();
 
-    // ---- C: MMA1 (S), MMA3 (Y = e^{Lc} Ct h+), MMA4 (H = Xs^T Bt)
+    // ---- C: MMAs that need only this tile's staged operands
     if (tid == 0) {
+      // x and theta staging are consumed: prefetch the next tile's ...
+      // (B and C follow once the MMAs that read them have completed)
+      if constexpr (FULL) {
 #pragma unroll
-      for (int k = 0; k < N / 16; ++k) {
-        const uint32_t koff = (uint32_t)(k >> 2) * (kRows * 128) + (uint32_t)(k & 3) * 32;
-        mma_ss(tmem + TM_S, sdesc(sCT + koff, 16, 1024), sdesc(sBT + koff, 16, 1024), C::ID_S, k > 0);
-      }
+        for (int k = 0; k < N / 16; ++k) {
+          const uint32_t koff = (uint32_t)(k >> 2) * (kRows * 128) + (uint32_t)(k & 3) * 32;
+          mma_ss(tmem + C::TM_S, sdesc(sCT + koff, 16, 1024), sdesc(sBT + koff, 16, 1024), C::ID_S, k > 0);
+        }
+        if constexpr (!C::kInterInS) {
 #pragma unroll
-      for (int k = 0; k < N / 16; ++k) {
-        const uint32_t aoff2 = (uint32_t)(k >> 2) * (kRows * 128) + (uint32_t)(k & 3) * 32;
-        const uint32_t boff = (uint32_t)(k >> 2) * (P * 128) + (uint32_t)(k & 3) * 32;
-        mma_ss(tmem + TM_Y, sdesc(sC2 + aoff2, 16, 1024), sdesc(sH + boff, 16, 1024), C::ID_Y3, k > 0);
+          for (int k = 0; k < N / 16; ++k) {
+            const uint32_t aoff2 = (uint32_t)(k >> 2) * (kRows * 128) + (uint32_t)(k & 3) * 32;
+            const uint32_t boff = (uint32_t)(k >> 2) * (P * 128) + (uint32_t)(k & 3) * 32;
+            mma_ss(tmem + C::TM_Y, sdesc(sC2 + aoff2, 16, 1024), sdesc(sH + boff, 16, 1024), C::ID_Y3, k > 0);
+          }
+        }
       }
 #pragma unroll
       for (int k = 0; k < kRows / 16; ++k) {
-        mma_ss(tmem + TM_H, sdesc(sXS + k * 2048, kRows * 128, 1024), sdesc(sBT + k * 2048, kRows * 128, 1024),
+        mma_ss(tmem + C::TM_H, sdesc(sXS + k * 2048, kRows * 128, 1024), sdesc(sBT + k * 2048, kRows * 128, 1024),
                C::ID_H, k > 0);
       }
-      mma_commit(mbar);
+      mma_commit(mma_bar);
     }
+    // next tile's per-token coefficients: registers -> smem slot, then start loading the one after
+    if (j + 1 < j1) store_coefs(par ^ 1);
+    if (j + 2 < j1) load_coefs(j + 2);
     {
-      const bool ok = mbar_wait(mbar, phase);
-      phase ^= 1;
+      const bool ok = mbar_wait(mma_bar, mma_phase);
+      mma_phase ^= 1;
       if (__syncthreads_or(!ok)) {
         failed = true;
         break;
       }
     }
     tc_fence_after();
+    // B (and, without kInterInS, C) tiles are free: the next tile's loads may land now
+    const bool prefetch_early = !(FULL && C::kInterInS);
+    if (tid == 0 && prefetch_early && j + 1 < j1) issue_loads(j + 1);
 
     // ---- D: mask S in TMEM (warps 0-3) | state update (warps 4-7)
     if (!state_warp) {
-      const int i = 32 * warp + lane;
-      const int t = i / R;
-      const int t_hi = (32 * warp + 31) / R;
-      const float Lt = Lc[t];
+      if constexpr (FULL) {
+        const int i = 32 * warp + lane;
+        const int t = i / R;
+        const int t_hi = (32 * warp + 31) / R;
+        const float Lt2 = mrec[t].x;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t o[16];
-        if ((32 * c) / R > t_hi) {
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[16];
+          if ((32 * c) / R > t_hi) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) o[e] = 0u;
-        } else {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_base + TM_S + 32 * c, v);
-          tmem_wait_ld();
-          float f[32];
+            for (int e = 0; e < 16; ++e) o[e] = 0u;
+          } else {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_base + C::TM_S + 32 * c, v);
+            tmem_wait_ld();
+            float f[32];
 #pragma unroll
-          for (int jj = 0; jj < 32 / R; ++jj) {
-            const int s = (32 * c) / R + jj;
-            float fac = 0.0f;
-            if (s <= t) fac = __expf(Lt - Lc[s]) * (gam[s] + (s < t ? bpv[s + 1] : 0.0f));
+            for (int jj = 0; jj < 32 / R; ++jj) {
+              const int s = (32 * c) / R + jj;
+              const float4 m = mrec[s];
+              const float w = (s < t) ? m.z : ((s == t) ? m.y : 0.0f);
+              const float fac = (s <= t) ? exp2f(Lt2 - m.x) * w : 0.0f;
 #pragma unroll
-            for (int rr = 0; rr < R; ++rr) f[jj * R + rr] = fac * __uint_as_float(v[jj * R + rr]);
+              for (int rr = 0; rr < R; ++rr) f[jj * R + rr] = fac * __uint_as_float(v[jj * R + rr]);
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = pack_bf16(f[2 * e], f[2 * e + 1]);
           }
-#pragma unroll
-          for (int e = 0; e < 16; ++e) o[e] = pack_bf16(f[2 * e], f[2 * e + 1]);
+          tmem_st16(tmem + lane_base + C::TM_S + 16 * c, o);
         }
-        tmem_st16(tmem + lane_base + TM_S + 16 * c, o);
+        tmem_wait_st();
       }
-      tmem_wait_st();
     } else {
       const float Le = scal[0];
 #pragma unroll 1
       for (int c = 0; c < N / 32; ++c) {
         uint32_t hv[32], sv[32];
-        tmem_ld32(tmem + lane_base + TM_H + 32 * c, hv);
-        tmem_ld32(tmem + lane_base + TM_ST + 32 * c, sv);
-        tmem_wait_ld();
-        float f[32];
+        if constexpr (P == 64) {
+          tmem_ld32(tmem + lane_base + C::TM_H + 32 * c, hv);  // lanes 0-15: H, lanes 16-31: state
+          tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          f[e] = fmaf(Le, __uint_as_float(sv[e]), __uint_as_float(hv[e]));
-          sv[e] = __float_as_uint(f[e]);
-        }
-        tmem_st32(tmem + lane_base + TM_ST + 32 * c, sv);
-        if (pvalid) {
+          for (int e = 0; e < 32; ++e) {
+            const float hlow = __shfl_up_sync(kFull, __uint_as_float(hv[e]), 16);
+            if (lane >= 16) hv[e] = __float_as_uint(fmaf(Le, __uint_as_float(hv[e]), hlow));
+          }
+          tmem_st32(tmem + lane_base + C::TM_ST + 32 * c, hv);
+          if constexpr (FULL && !C::kInterInS) {
+            // (not reached: P == 64 always uses kInterInS)
+          }
+        } else {
+          tmem_ld32(tmem + lane_base + C::TM_H + 32 * c, hv);
+          tmem_ld32(tmem + lane_base + C::TM_ST + 32 * c, sv);
+          tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float f8[8];
+          for (int e = 0; e < 32; ++e)
+            sv[e] = __float_as_uint(fmaf(Le, __uint_as_float(sv[e]), __uint_as_float(hv[e])));
+          tmem_st32(tmem + lane_base + C::TM_ST + 32 * c, sv);
+          if constexpr (FULL && !C::kInterInS) {
+            // MMA3 (which read the old bf16 state) has completed: refresh the bf16 copy
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f8[e] = f[8 * q + e];
-            sts128(sH + sw128(prow, 4 * c + q, P * 128), pack8(f8));
+            for (int q = 0; q < 4; ++q) {
+              float f8[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f8[e] = __uint_as_float(sv[8 * q + e]);
+              sts128(sH + sw128(prow, 4 * c + q, P * 128), pack8(f8));
+            }
           }
         }
       }
       tmem_wait_st();
     }
+    if constexpr (FULL) {
+      fence_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+
+      // ---- E: MMA3 (kInterInS: Ct h+ into the free half of S) and MMA2 (Y += S' X)
+      if (tid == 0) {
+        if constexpr (C::kInterInS) {
+#pragma unroll
+          for (int k = 0; k < N / 16; ++k) {
+            const uint32_t aoff2 = (uint32_t)(k >> 2) * (kRows * 128) + (uint32_t)(k & 3) * 32;
+            const uint32_t boff = (uint32_t)(k >> 2) * (P * 128) + (uint32_t)(k & 3) * 32;
+            mma_ss(tmem + C::TM_YI, sdesc(sCT + aoff2, 16, 1024), sdesc(sH + boff, 16, 1024), C::ID_Y3, k > 0);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < kRows / 16; ++k)
+          mma_ts(tmem + C::TM_Y, tmem + C::TM_S + 8 * k, sdesc(sX + k * 2048, kRows * 128, 1024), C::ID_Y2,
+                 C::kInterInS ? (k > 0) : 1);  // without kInterInS, Y already holds e^{Lc} Ct h+
+        mma_commit(mma_bar);
+      }
+      {
+        const bool ok = mbar_wait(mma_bar, mma_phase);
+        mma_phase ^= 1;
+        if (__syncthreads_or(!ok)) {
+          failed = true;
+          break;
+        }
+      }
+      tc_fence_after();
+      if (tid == 0 && !prefetch_early && j + 1 < j1) issue_loads(j + 1);
+
+      // ---- F: epilogue y_t = sum_r W_o[r] * (Y + e^{Lc_t} Yi)_{t,r} + D x_t; refresh bf16 state
+      {
+        const int i = 32 * q4 + lane;
+        const int t = i / R, r = i % R;
+        const int half = warp >> 2;
+        constexpr int PH = P / 2;
+        constexpr int W = 16 / R;
+        const float dect = decA[t];
+        const int64_t yrow = ((tok_base + c0 + t) * H + hi) * P;
+#pragma unroll 1
+        for (int c = 0; c < PH / 16; ++c) {
+          const int col0 = half * PH + 16 * c;
+          uint32_t v[16];
+          tmem_ld16(tmem + lane_base + C::TM_Y + col0, v);
+          float f[16];
+          if constexpr (C::kInterInS) {
+            uint32_t vi[16];
+            tmem_ld16(tmem + lane_base + C::TM_YI + col0, vi);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) f[e] = fmaf(dect, __uint_as_float(vi[e]), __uint_as_float(v[e]));
+          } else {
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(v[e]);
+          }
+          if (wog) {
+#pragma unroll
+            for (int e4 = 0; e4 < 4; ++e4) {
+              const float4 w4 = __ldg(reinterpret_cast<const float4*>(wog + r * P + col0 + 4 * e4));
+              f[4 * e4] *= w4.x;
+              f[4 * e4 + 1] *= w4.y;
+              f[4 * e4 + 2] *= w4.z;
+              f[4 * e4 + 3] *= w4.w;
+            }
+          }
+#pragma unroll
+          for (int m = 1; m < R; m <<= 1) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) f[e] += __shfl_xor_sync(kFull, f[e], m);
+          }
+          if (t < nv) {
+            float outv[W];
+#pragma unroll
+            for (int e = 0; e < W; ++e) {
+              float sel = f[e];
+#pragma unroll
+              for (int rr = 1; rr < R; ++rr)
+                if (rr == r) sel = f[rr * W + e];
+              outv[e] = sel;
+            }
+            const int pc = col0 + r * W;
+            if (p.D) {
+#pragma unroll
+              for (int e = 0; e < W; ++e) outv[e] = fmaf(Dh, __bfloat162float(xg[yrow + pc + e]), outv[e]);
+            }
+#pragma unroll
+            for (int e = 0; e < W; e += 2)
+              *reinterpret_cast<uint32_t*>(yg + yrow + pc + e) = pack_bf16(outv[e], outv[e + 1]);
+          }
+        }
+        if constexpr (C::kInterInS) {
+          // MMA3 has read the old bf16 state: write the new one (kept in TMEM lanes 16-31)
+          if (state_warp) {
+#pragma unroll 1
+            for (int c2 = 0; c2 < N / 32; ++c2) {
+              uint32_t sv[32];
+              tmem_ld32(tmem + lane_base + C::TM_ST + 32 * c2, sv);
+              tmem_wait_ld();
+              if (st_owner) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  float f8[8];
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) f8[e] = __uint_as_float(sv[8 * q + e]);
+                  sts128(sH + sw128(prow, 4 * c2 + q, P * 128), pack8(f8));
+                }
+              }
+            }
+          }
+        }
+      }
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-
-    // ---- E: MMA2 (Y += S' X), S' read from TMEM
-    if (tid == 0) {
-#pragma unroll
-      for (int k = 0; k < kRows / 16; ++k)
-        mma_ts(tmem + TM_Y, tmem + TM_S + 8 * k, sdesc(sX + k * 2048, kRows * 128, 1024), C::ID_Y2, 1);
-      mma_commit(mbar);
-    }
-    {
-      const bool ok = mbar_wait(mbar, phase);
-      phase ^= 1;
-      if (__syncthreads_or(!ok)) {
-        failed = true;
-        break;
-      }
-    }
-    tc_fence_after();
-
-    // ---- F: epilogue y_t = sum_r W_o[r] * Y_{t,r} + D x_t (all 8 warps, two column halves)
-    {
-      const int i = 32 * q4 + lane;
-      const int t = i / R, r = i % R;
-      const int half = warp >> 2;
-      constexpr int PH = P / 2;
-      constexpr int W = 16 / R;
-      const int64_t yrow = (((int64_t)bi * L + c0 + t) * H + hi) * P;
-#pragma unroll 1
-      for (int c = 0; c < PH / 16; ++c) {
-        const int col0 = half * PH + 16 * c;
-        uint32_t v[16];
-        tmem_ld16(tmem + lane_base + TM_Y + col0, v);
-        tmem_wait_ld();
-        float f[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) f[e] = wo[r * P + col0 + e] * __uint_as_float(v[e]);
-#pragma unroll
-        for (int m = 1; m < R; m <<= 1) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) f[e] += __shfl_xor_sync(kFull, f[e], m);
-        }
-        if (t < nv) {
-          float outv[W];
-#pragma unroll
-          for (int e = 0; e < W; ++e) {
-            float sel = f[e];
-#pragma unroll
-            for (int rr = 1; rr < R; ++rr)
-              if (rr == r) sel = f[rr * W + e];
-            outv[e] = sel;
-          }
-          const int pc = col0 + r * W;
-          if (p.D) {
-#pragma unroll
-            for (int e = 0; e < W; ++e) outv[e] = fmaf(Dh, __bfloat162float(xg[yrow + pc + e]), outv[e]);
-          }
-#pragma unroll
-          for (int e = 0; e < W; e += 2)
-            *reinterpret_cast<uint32_t*>(yg + yrow + pc + e) = pack_bf16(outv[e], outv[e + 1]);
-        }
-      }
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
   }
 
-  // ---- final state: rotate the rotated-frame state back by the total angle; carry
-  if (!failed) {
-    if (state_warp) {
-      float* hout = p.h + (int64_t)bh * N * P;
+  // ---- results
+  if (!failed && j0 < j1) {
+    if constexpr (FULL) {
+      if (last_seg) {
+        // final state: rotate the segment-frame state back by the segment's total angle
+        if (state_warp) {
+          float* hout = p.h + (int64_t)bh * N * P;
 #pragma unroll 1
-      for (int c = 0; c < N / 32; ++c) {
-        uint32_t sv[32];
-        tmem_ld32(tmem + lane_base + TM_ST + 32 * c, sv);
-        tmem_wait_ld();
-        if (pvalid) {
+          for (int c = 0; c < N / 32; ++c) {
+            uint32_t sv[32];
+            tmem_ld32(tmem + lane_base + C::TM_ST + 32 * c, sv);
+            tmem_wait_ld();
+            if (st_owner) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int k = 16 * c + e;
-            float sn, cn;
-            sincosf((float)base[k], &sn, &cn);
-            const float a0 = __uint_as_float(sv[2 * e]), a1 = __uint_as_float(sv[2 * e + 1]);
-            hout[(int64_t)(2 * k) * P + prow] = cn * a0 - sn * a1;
-            hout[(int64_t)(2 * k + 1) * P + prow] = sn * a0 + cn * a1;
+              for (int e = 0; e < 16; ++e) {
+                const int k = 16 * c + e;
+                float sn, cn;
+                sincosf((float)base[k], &sn, &cn);
+                const float a0 = __uint_as_float(sv[2 * e]), a1 = __uint_as_float(sv[2 * e + 1]);
+                hout[(int64_t)(2 * k) * P + prow] = cn * a0 - sn * a1;
+                hout[(int64_t)(2 * k + 1) * P + prow] = sn * a0 + cn * a1;
+              }
+            }
           }
+        } else {
+          const int64_t tokl = tok_base + (L - 1);
+          const int64_t bc = ((tokl * G + g) * R) * (int64_t)N;
+          for (int i = tid; i < R * N; i += 128) p.carry_B[(int64_t)bh * R * N + i] = __bfloat162float(Bg[bc + i]);
+          const int64_t xr = (tokl * H + hi) * (int64_t)P;
+          for (int i = tid; i < P; i += 128) p.carry_x[(int64_t)bh * P + i] = __bfloat162float(xg[xr + i]);
         }
       }
     } else {
-      const int64_t tokl = (int64_t)bi * L + (L - 1);
-      const int64_t bc = ((tokl * G + g) * R) * (int64_t)N;
-      for (int i = tid; i < R * N; i += 128) p.carry_B[(int64_t)bh * R * N + i] = __bfloat162float(Bg[bc + i]);
-      const int64_t xr = (tokl * H + hi) * (int64_t)P;
-      for (int i = tid; i < P; i += 128) p.carry_x[(int64_t)bh * P + i] = __bfloat162float(xg[xr + i]);
+      // segment summary: end state (segment frame, zero start), total log decay, total angle
+      const int64_t sidx = (int64_t)bh * (sg.nseg - 1) + seg;
+      if (state_warp) {
+        float* wh = sg.ws_h + sidx * N * P;
+#pragma unroll 1
+        for (int c = 0; c < N / 32; ++c) {
+          uint32_t sv[32];
+          tmem_ld32(tmem + lane_base + C::TM_ST + 32 * c, sv);
+          tmem_wait_ld();
+          if (st_owner) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) wh[(int64_t)(32 * c + e) * P + prow] = __uint_as_float(sv[e]);
+          }
+        }
+      }
+      if (tid == 0) sg.ws_l[sidx] = seg_logdec;
+      for (int k = tid; k < K2; k += kThreads) sg.ws_phi[sidx * K2 + k] = base[k];
     }
-  } else if (tid == 0) {
-    set_status(p.status, M3_ERR_TIMEOUT);
   }
+  if (failed && tid == 0) set_status(p.status, M3_ERR_TIMEOUT);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const cuuint64_t* dims,
+              const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return fn(m, dt, (cuuint32_t)rank, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct Maps {
+  CUtensorMap B, C, X, T;
+};
+
+bool make_maps(const Params& p, int Q, Maps* m) {
+  const cuuint64_t toks = (cuuint64_t)(p.b * p.L);
+  const cuuint64_t K2 = (cuuint64_t)(p.N / 2);
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)p.N, (cuuint64_t)p.R, (cuuint64_t)p.G, toks};
+    const cuuint64_t str[3] = {(cuuint64_t)p.N * 2, (cuuint64_t)p.R * p.N * 2, (cuuint64_t)p.G * p.R * p.N * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)p.R, 1, (cuuint32_t)Q};
+    if (!make_map(&m->B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, p.B, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return false;
+    if (!make_map(&m->C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, p.C, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return false;
+  }
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)p.P, (cuuint64_t)p.H, toks};
+    const cuuint64_t str[2] = {(cuuint64_t)p.P * 2, (cuuint64_t)p.H * p.P * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)p.P, 1, (cuuint32_t)Q};
+    if (!make_map(&m->X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.x, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return false;
+  }
+  {
+    const cuuint64_t dims[3] = {K2, (cuuint64_t)p.G, toks};
+    const cuuint64_t str[2] = {K2 * 4, (cuuint64_t)p.G * K2 * 4};
+    const cuuint32_t box[3] = {(cuuint32_t)K2, 1, (cuuint32_t)Q};
+    if (!make_map(&m->T, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p.theta, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return false;
+  }
+  return true;
+}
+
 template <int R, int N, int P>
-cudaError_t launch_cfg(const Params& p, cudaStream_t stream) {
-  using Cf = Cfg<R, N, P>;
-  auto k = scan_tc_kernel<R, N, P>;
+constexpr int ctas_per_sm() {
+  return (P == 64 && N == 64) ? 2 : 1;
+}
+
+template <int R, int N, int P, int MODE>
+cudaError_t launch_mode(const Maps& m, const Params& p, const SegInfo& sg, unsigned grid, cudaStream_t stream) {
+  using Cf = Cfg<R, N, P, MODE>;
+  auto k = scan_tc_kernel<R, N, P, MODE>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
   if (e != cudaSuccess) return e;
-  k<<<(unsigned)(p.b * p.H), kThreads, Cf::SMEM, stream>>>(p);
+  k<<<grid, kThreads, Cf::SMEM, stream>>>(m.B, m.C, m.X, m.T, p, sg);
   return cudaGetLastError();
 }
 
-template <int R>
-cudaError_t launch_r(const Params& p, cudaStream_t stream) {
-  if (p.N == 64 && p.P == 64) return launch_cfg<R, 64, 64>(p, stream);
-  if (p.N == 64 && p.P == 128) return launch_cfg<R, 64, 128>(p, stream);
-  if (p.N == 128 && p.P == 64) return launch_cfg<R, 128, 64>(p, stream);
-  return launch_cfg<R, 128, 128>(p, stream);
+// Number of segments per sequence: enough CTAs to fill the SMs, at least 2 tiles each.
+int plan_segments(int64_t nseq, int64_t ntiles, int per_sm) {
+  int dev = 0, nsm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t slots = (int64_t)nsm * per_sm;
+  int64_t nseg = nseq >= slots ? 1 : slots / nseq;
+  const int64_t maxseg = ntiles / 2;
+  if (nseg > maxseg) nseg = maxseg;
+  if (nseg < 1) nseg = 1;
+  if (nseg > 64) nseg = 64;
+  return (int)nseg;
+}
+
+template <int R, int N, int P>
+size_t ws_bytes_for(const Params& p, int* nseg_out, int* seg_tiles_out) {
+  constexpr int Q = kRows / R;
+  const int64_t ntiles = (p.L + Q - 1) / Q;
+  const int64_t nseq = p.b * p.H;
+  const int nseg = plan_segments(nseq, ntiles, ctas_per_sm<R, N, P>());
+  const int seg_tiles = (int)((ntiles + nseg - 1) / nseg);
+  const int nseg_eff = (int)((ntiles + seg_tiles - 1) / seg_tiles);
+  if (nseg_out) *nseg_out = nseg_eff;
+  if (seg_tiles_out) *seg_tiles_out = seg_tiles;
+  if (nseg_eff <= 1) return 0;
+  const size_t np = (size_t)N * P;
+  const size_t s1 = (size_t)(nseg_eff - 1);
+  size_t bytes = 0;
+  bytes += 4 * (size_t)nseq * np;                       // ws_init
+  bytes += 4 * (size_t)nseq * s1 * np;                  // ws_h
+  bytes = (bytes + 4 * (size_t)nseq * s1 + 255) & ~(size_t)255;   // ws_l, then align
+  bytes += 8 * (size_t)nseq * s1 * (N / 2);             // ws_phi
+  return bytes;
+}
+
+template <int R, int N, int P>
+cudaError_t launch_cfg(const Params& p, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  constexpr int Q = kRows / R;
+  int nseg = 1, seg_tiles = 1;
+  const size_t need = ws_bytes_for<R, N, P>(p, &nseg, &seg_tiles);
+  if (need > ws_bytes || (need > 0 && ws == nullptr)) return cudaErrorInvalidValue;
+  Maps m;
+  if (!make_maps(p, Q, &m)) return cudaErrorInvalidValue;
+  SegInfo sg;
+  sg.nseg = nseg;
+  sg.seg_tiles = seg_tiles;
+  sg.ws_init = sg.ws_h = sg.ws_l = nullptr;
+  sg.ws_phi = nullptr;
+  const int64_t nseq = p.b * p.H;
+  if (nseg > 1) {
+    const size_t np = (size_t)N * P;
+    const size_t s1 = (size_t)(nseg - 1);
+    char* w = static_cast<char*>(ws);
+    sg.ws_init = reinterpret_cast<float*>(w);
+    sg.ws_h = sg.ws_init + (size_t)nseq * np;
+    sg.ws_l = sg.ws_h + (size_t)nseq * s1 * np;
+    size_t off = (4 * ((size_t)nseq * np + (size_t)nseq * s1 * np + (size_t)nseq * s1) + 255) & ~(size_t)255;
+    sg.ws_phi = reinterpret_cast<double*>(w + off);
+    cudaError_t e = launch_mode<R, N, P, MODE_STATE>(m, p, sg, (unsigned)(nseq * (nseg - 1)), stream);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_mode<R, N, P, MODE_FULL>(m, p, sg, (unsigned)(nseq * nseg), stream);
 }
 
 template <int R, int N, int P>
 constexpr bool fits() {
-  return Cfg<R, N, P>::SMEM <= 227 * 1024;
+  return Cfg<R, N, P, MODE_FULL>::SMEM <= 227 * 1024;
+}
+
+template <int R>
+cudaError_t launch_r(const Params& p, void* ws, size_t wsb, cudaStream_t s) {
+  if (p.N == 64 && p.P == 64) return launch_cfg<R, 64, 64>(p, ws, wsb, s);
+  if (p.N == 64 && p.P == 128) return launch_cfg<R, 64, 128>(p, ws, wsb, s);
+  if (p.N == 128 && p.P == 64) return launch_cfg<R, 128, 64>(p, ws, wsb, s);
+  return launch_cfg<R, 128, 128>(p, ws, wsb, s);
+}
+
+template <int R>
+size_t ws_r(const Params& p) {
+  if (p.N == 64 && p.P == 64) return ws_bytes_for<R, 64, 64>(p, nullptr, nullptr);
+  if (p.N == 64 && p.P == 128) return ws_bytes_for<R, 64, 128>(p, nullptr, nullptr);
+  if (p.N == 128 && p.P == 64) return ws_bytes_for<R, 128, 64>(p, nullptr, nullptr);
+  return ws_bytes_for<R, 128, 128>(p, nullptr, nullptr);
+}
+
+template <int R>
+bool fits_r(const Params& p) {
+  if (p.N == 64 && p.P == 64) return fits<R, 64, 64>();
+  if (p.N == 64 && p.P == 128) return fits<R, 64, 128>();
+  if (p.N == 128 && p.P == 64) return fits<R, 128, 64>();
+  return fits<R, 128, 128>();
 }
 
 }  // namespace
@@ -734,30 +1148,31 @@ constexpr bool fits() {
 bool tc_scan_supported(const Params& p) {
   if (p.dtype != M3_BF16) return false;
   if (!((p.N == 64 || p.N == 128) && (p.P == 64 || p.P == 128))) return false;
+  if (p.b * p.L > 0x7fffffffLL) return false;  // TMA token coordinate is 32-bit
   switch (p.R) {
-    case 1:
-      return p.N == 64 ? (p.P == 64 ? fits<1, 64, 64>() : fits<1, 64, 128>())
-                       : (p.P == 64 ? fits<1, 128, 64>() : fits<1, 128, 128>());
-    case 2:
-      return p.N == 64 ? (p.P == 64 ? fits<2, 64, 64>() : fits<2, 64, 128>())
-                       : (p.P == 64 ? fits<2, 128, 64>() : fits<2, 128, 128>());
-    case 4:
-      return p.N == 64 ? (p.P == 64 ? fits<4, 64, 64>() : fits<4, 64, 128>())
-                       : (p.P == 64 ? fits<4, 128, 64>() : fits<4, 128, 128>());
-    case 8:
-      return p.N == 64 ? (p.P == 64 ? fits<8, 64, 64>() : fits<8, 64, 128>())
-                       : (p.P == 64 ? fits<8, 128, 64>() : fits<8, 128, 128>());
-    default:
-      return false;
+    case 1: return fits_r<1>(p);
+    case 2: return fits_r<2>(p);
+    case 4: return fits_r<4>(p);
+    case 8: return fits_r<8>(p);
+    default: return false;
   }
 }
 
-cudaError_t launch_scan_tc(const Params& p, cudaStream_t stream) {
+size_t tc_scan_workspace_bytes(const Params& p) {
   switch (p.R) {
-    case 1: return launch_r<1>(p, stream);
-    case 2: return launch_r<2>(p, stream);
-    case 4: return launch_r<4>(p, stream);
-    default: return launch_r<8>(p, stream);
+    case 1: return ws_r<1>(p);
+    case 2: return ws_r<2>(p);
+    case 4: return ws_r<4>(p);
+    default: return ws_r<8>(p);
+  }
+}
+
+cudaError_t launch_scan_tc(const Params& p, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  switch (p.R) {
+    case 1: return launch_r<1>(p, ws, ws_bytes, stream);
+    case 2: return launch_r<2>(p, ws, ws_bytes, stream);
+    case 4: return launch_r<4>(p, ws, ws_bytes, stream);
+    default: return launch_r<8>(p, ws, ws_bytes, stream);
   }
 }
 

@@ -123,3 +123,19 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(m3, "_lib", None)
     with pytest.raises(m3.M3Error):
         m3.lib()
+
+
+def test_workspace_size_and_missing_workspace(L):
+    # a long sequence with few (batch, head) pairs is split into segments that need scratch
+    d = m3.make_dims(1, 4096, 2, 64, 64, 2, 1, "bf16")
+    n = ctypes.c_size_t()
+    assert L.m3_scan_workspace_size(ctypes.byref(d), ctypes.byref(n)) == 0
+    assert n.value > 0
+    st = _fake_state(L, d)
+    ok = ctypes.c_void_p(1 << 24)
+    assert L.m3_scan_fwd(ctypes.byref(d), *([ok] * 7 + [None] * 5), st, ok, None, 0, None) == -5
+    assert L.m3_scan_fwd(ctypes.byref(d), *([ok] * 7 + [None] * 5), st, ok, ok, n.value - 1, None) == -5
+    # the sequential kernel needs none
+    d.flags = 1
+    assert L.m3_scan_workspace_size(ctypes.byref(d), ctypes.byref(n)) == 0 and n.value == 0
+    assert L.m3_state_free(st) == 0

@@ -195,6 +195,8 @@ TC_SHAPES = [
     dict(b=1, L=260, H=2, P=64, N=64, R=1, G=1),
     dict(b=1, L=1, H=2, P=128, N=128, R=4, G=1),     # single token
     dict(b=1, L=33, H=2, P=128, N=128, R=4, G=1),    # one full tile + 1
+    dict(b=1, L=2000, H=2, P=64, N=64, R=2, G=1),    # few sequences: many segments
+    dict(b=2, L=999, H=2, P=128, N=128, R=4, G=2),   # segments + ragged tail + groups
 ]
 
 
@@ -204,6 +206,18 @@ def test_tc_scan_shapes(shape, with_state):
     inp = make_inputs(dtype="bf16", seed=201, extras=True, **shape)
     st = make_state(shape["b"], shape["H"], shape["P"], shape["N"], shape["R"], seed=202) if with_state else None
     check_scan(inp, state=st)
+
+
+def test_workspace_is_required_when_segmented():
+    inp = make_inputs(dtype="bf16", seed=205, b=1, L=1500, H=2, P=64, N=64, R=2, G=1)
+    dims = m3.dims_of(inp)
+    assert m3.m3_scan_workspace_size(dims) > 0
+    dev = m3.to_device(inp)
+    st, _ = m3.state_tensors(dims)
+    y = torch.empty_like(dev["x"])
+    with pytest.raises(m3.M3Error) as e:
+        m3.m3_scan_fwd(dims, *[dev[k] for k in m3._OPERANDS], st, y, workspace=None)
+    assert e.value.code == -5
 
 
 def test_tc_matches_sequential_kernel():
