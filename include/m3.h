@@ -131,6 +131,25 @@ m3_status m3_scan_fwd(const m3_dims* dims, const void* x, const float* dt, const
                       const float* W_o, const float* D, m3_state* state, void* y,
                       void* workspace, size_t workspace_bytes, void* stream);
 
+/* Same as m3_scan_fwd, for callers that cannot provide a workspace: a serving process
+ * whose device memory is all reserved up front by an allocator it does not own, or a
+ * plain C program with no device allocator of its own (a cudaMalloc mid-request may also
+ * synchronise the device).  The paper has no counterpart; this is a property of the
+ * library only.  The scratch m3_scan_fwd would take from `workspace` comes instead from
+ * one fixed 16 MiB device array inside libm3, which every device that loads the library
+ * holds until the process exits.  This call allocates nothing.  Dimensions whose scratch
+ * (m3_scan_workspace_size) exceeds 16 MiB are rejected with M3_ERR_WORKSPACE.  All calls
+ * share the array: calls whose kernels overlap on the GPU (several streams or host
+ * threads) race and give wrong results; calls ordered on one stream are safe.  Nothing
+ * needs clearing between calls (every scratch byte is written before it is read).  The
+ * first call on a device, made with that device current, looks up the array's device
+ * address (cudaGetSymbolAddress); make that first call before any stream capture. */
+m3_status m3_scan_fwd_noalloc(const m3_dims* dims, const void* x, const float* dt, const float* A,
+                              const float* lam, const void* B, const void* C, const float* theta,
+                              const float* bias_B, const float* bias_C, const float* W_x,
+                              const float* W_o, const float* D, m3_state* state, void* y,
+                              void* stream);
+
 /* ---- decode (one token) ------------------------------------------------ */
 
 /* Advance every sequence by one token.  Token inputs have L = 1 in the layouts

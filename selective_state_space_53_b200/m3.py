@@ -51,6 +51,7 @@ SIGNATURES = {
     "m3_state_copy_from_host": (_I, [_VP, _VP, _SZ, _VP]),
     "m3_scan_workspace_size": (_I, [_DP, ctypes.POINTER(_SZ)]),
     "m3_scan_fwd": (_I, [_DP] + [_VP] * 14 + [_VP, _SZ, _VP]),
+    "m3_scan_fwd_noalloc": (_I, [_DP] + [_VP] * 14 + [_VP]),
     "m3_decode_step": (_I, [_DP] + [_VP] * 15),
     "m3_check": (_I, [_VP]),
     "m3_status_str": (ctypes.c_char_p, [_I]),
@@ -168,6 +169,15 @@ def m3_scan_fwd(dims: Dims, x, dt, A, lam, B, C, theta, bias_B, bias_C, W_x, W_o
                              _ptr(theta), _ptr(bias_B), _ptr(bias_C), _ptr(W_x), _ptr(W_o), _ptr(D),
                              state.handle, _ptr(y), _ptr(workspace), ws_bytes, _stream(stream)),
            "m3_scan_fwd")
+
+
+def m3_scan_fwd_noalloc(dims: Dims, x, dt, A, lam, B, C, theta, bias_B, bias_C, W_x, W_o, D, state: State, y,
+                        stream=None):
+    """m3_scan_fwd without a workspace: the library's fixed 16 MiB device scratch is used
+    (for callers that cannot allocate; calls overlapping on the GPU race on it)."""
+    _check(lib().m3_scan_fwd_noalloc(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(lam), _ptr(B), _ptr(C),
+                                     _ptr(theta), _ptr(bias_B), _ptr(bias_C), _ptr(W_x), _ptr(W_o), _ptr(D),
+                                     state.handle, _ptr(y), _stream(stream)), "m3_scan_fwd_noalloc")
 
 
 def m3_decode_step(dims: Dims, x_t, dt_t, A_t, lam_t, B_t, C_t, theta_t, bias_B, bias_C, W_x, W_o, D,
