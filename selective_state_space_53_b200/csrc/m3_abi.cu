@@ -281,7 +281,9 @@ m3_status m3_decode_step(const m3_dims* dims, const void* x_t, const float* dt_t
                              W_x, W_o, D, state, y_t);
   p.status = status_word();
   if (!p.status) return M3_ERR_CUDA;
-  return m3::launch_scan_sequential(p, (cudaStream_t)stream) == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+  const cudaError_t e = m3::decode_supported(p) ? m3::launch_decode(p, (cudaStream_t)stream)
+                                                : m3::launch_scan_sequential(p, (cudaStream_t)stream);
+  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
 }
 
 m3_status m3_check(void* stream) {

@@ -56,6 +56,8 @@ __device__ __forceinline__ void store_out(void* base, int64_t i, float v) {
 
 // Launchers (defined in the kernel files); return cudaGetLastError() of the launch.
 cudaError_t launch_scan_sequential(const Params& p, cudaStream_t stream);
+bool decode_supported(const Params& p);                       // one-token kernel fits on chip
+cudaError_t launch_decode(const Params& p, cudaStream_t stream);
 bool tc_scan_supported(const Params& p);
 size_t tc_scan_workspace_bytes(const Params& p);  // scratch the chunked scan needs (0: none)
 cudaError_t launch_scan_tc(const Params& p, void* workspace, size_t workspace_bytes, cudaStream_t stream);

@@ -216,6 +216,12 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 __device__ __forceinline__ uint32_t sw128(int row, int ch, uint32_t block_bytes) {
   return (uint32_t)(ch >> 3) * block_bytes + (uint32_t)row * 128u + ((uint32_t)((ch & 7) ^ (row & 7)) << 4);
 }
+// 2^x by the hardware approximation (ex2.approx, relative error about 2^-22).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 // sin and cos of an angle of moderate size: Cody-Waite reduction to [-pi, pi] with a two-term
 // split of 2 pi (Cody & Waite, "Software Manual for the Elementary Functions", 1980), then the
 // hardware approximations, which are accurate on that interval.
@@ -252,21 +258,21 @@ struct Cfg {
   static constexpr int OFF_CT = OFF_BT + TILE_N;
   static constexpr int OFF_C2 = OFF_CT + (FULL ? TILE_N : 0);
   static constexpr int OFF_X = OFF_C2 + ((FULL && !kInterInS) ? TILE_N : 0);
-  static constexpr int OFF_XS = OFF_X + (FULL ? TILE_P : 0);
-  static constexpr int OFF_H = OFF_XS + TILE_P;
+  static constexpr int OFF_H = OFF_X + TILE_P;
   static constexpr int OFF_CS = OFF_H + (FULL ? TILE_H : 0);       // float2 [Q][K2]
   static constexpr int OFF_TH = OFF_CS + Q * K2 * 4;                // theta staging: 2nd half of CS
   static constexpr int OFF_XSTG = OFF_CS + Q * K2 * 8;              // x staging [Q][P] bf16
   static constexpr int OFF_WX = OFF_XSTG + Q * P * 2;              // W_x [R][P]
-  static constexpr int OFF_BASE = OFF_WX + R * P * 4;               // double [K2]
+  static constexpr int OFF_WO = OFF_WX + R * P * 4;                 // W_o [R][P]
+  static constexpr int OFF_BASE = OFF_WO + R * P * 4;               // double [K2]
   static constexpr int SEGS = kThreads / K2;                        // angle prefix segments
   static constexpr int SEGLEN = (Q + SEGS - 1) / SEGS;
   static constexpr int OFF_SEGSUM = OFF_BASE + K2 * 8;              // float [SEGS][K2]
   static constexpr int TOKF = Q + 4;
   static constexpr int OFF_TOK = OFF_SEGSUM + SEGS * K2 * 4;        // per-token float arrays
-  static constexpr int NTOKARR = 10;
-  static constexpr int OFF_MREC = OFF_TOK + NTOKARR * TOKF * 4;     // float4 [Q] mask records
-  static constexpr int OFF_MISC = OFF_MREC + Q * 16;
+  static constexpr int NTOKARR = 8;
+  static constexpr int OFF_MREC = OFF_TOK + NTOKARR * TOKF * 4;     // float4 [Q] x 2 per-token records
+  static constexpr int OFF_MISC = OFF_MREC + 2 * Q * 16;
   static constexpr int BYTES = OFF_MISC + 64;
   static constexpr int SMEM = BYTES + 1024;  // slack for 1024-byte alignment
   // tensor memory columns
@@ -286,8 +292,21 @@ struct Cfg {
   static constexpr int TX_T = Q * K2 * 4;
 };
 
-// per-token array slots (each TOKF floats)
-enum { A_DT0 = 0, A_A0, A_LM0, A_DT1, A_A1, A_LM1, A_GAM, A_CW, A_DEC, A_SCAL };
+// per-token array slots (each TOKF floats): raw dt/A/lam of the current and next tile
+enum { A_DT0 = 0, A_A0, A_LM0, A_DT1, A_A1, A_LM1, A_SCAL };
+// scalars in A_SCAL: [0] e^{Le}, [1] Le, [2..3] next-token beta' by parity, [4] state-update
+// scale of H, [5] 1 when the tile uses the pivot factorisation
+//
+// The decay inside a tile, e^{Lc_t - Lc_s}, is split around a pivot m (the middle of the
+// tile's log-decay range) as a_t * b_s with a_t = e^{Lc_t - m}, b_s = e^{m - Lc_s}.  b_s and
+// the trapezoid weight w_s = gamma_s + beta'_{s+1} go into X' = b_s w_s X, a_t is applied to
+// the output rows, so the masked score matrix needs no exponentials: S' = S below the
+// diagonal, S * gamma_s / w_s on it, 0 above.  The state update becomes H = X'^T Bt times the
+// uniform factor e^{Le - m}.  When the range of Lc within a tile exceeds 160 the split could
+// overflow fp32; such tiles take the exact path (a_t = 1, b_s = 1, e^{Lc_t - Lc_s} per element,
+// Bt rows scaled by e^{Le - Lc_t} before the state update).
+// record A[t] = {Lc_t * log2 e, gamma_t / w_t, a_t, b_t w_t};  record B[t] = {C2 row scale,
+// e^{Lc_t}, e^{Le - Lc_t}, 0}
 
 template <int R, int N, int P, int MODE>
 __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
@@ -317,19 +336,18 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
   const int64_t tok_base = (int64_t)bi * L;  // first token of this sequence (flattened b*L index)
 
   const uint32_t sBT = smem_u32(sm + C::OFF_BT), sCT = smem_u32(sm + C::OFF_CT), sC2 = smem_u32(sm + C::OFF_C2);
-  const uint32_t sX = smem_u32(sm + C::OFF_X), sXS = smem_u32(sm + C::OFF_XS), sH = smem_u32(sm + C::OFF_H);
+  const uint32_t sX = smem_u32(sm + C::OFF_X), sH = smem_u32(sm + C::OFF_H);
   const uint32_t sXSTG = smem_u32(sm + C::OFF_XSTG), sTH = smem_u32(sm + C::OFF_TH);
   float2* cs = reinterpret_cast<float2*>(sm + C::OFF_CS);
   const float* th_stg = reinterpret_cast<const float*>(sm + C::OFF_TH);
   float* wx = reinterpret_cast<float*>(sm + C::OFF_WX);
+  float* wo = reinterpret_cast<float*>(sm + C::OFF_WO);
   double* base = reinterpret_cast<double*>(sm + C::OFF_BASE);
   float* segsum = reinterpret_cast<float*>(sm + C::OFF_SEGSUM);
   float* tokf = reinterpret_cast<float*>(sm + C::OFF_TOK);
-  float4* mrec = reinterpret_cast<float4*>(sm + C::OFF_MREC);
-  float* gamA = tokf + A_GAM * C::TOKF;
-  float* cwA = tokf + A_CW * C::TOKF;
-  float* decA = tokf + A_DEC * C::TOKF;
-  float* scal = tokf + A_SCAL * C::TOKF;  // [0] e^{Lc_e}, [1] tile log decay, [2..3] next-token beta' by parity
+  float4* recA = reinterpret_cast<float4*>(sm + C::OFF_MREC);
+  float4* recB = recA + Q;
+  float* scal = tokf + A_SCAL * C::TOKF;
   uint64_t* mma_bar = reinterpret_cast<uint64_t*>(sm + C::OFF_MISC);
   uint64_t* load_bar = reinterpret_cast<uint64_t*>(sm + C::OFF_MISC + 8);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC + 16);
@@ -400,10 +418,12 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
     prefetch_tmap(&tmX);
     prefetch_tmap(&tmT);
   }
-  for (int i = tid; i < R * P; i += kThreads) wx[i] = p.W_x ? p.W_x[(int64_t)hi * R * P + i] : 1.0f;
+  for (int i = tid; i < R * P; i += kThreads) {
+    wx[i] = p.W_x ? p.W_x[(int64_t)hi * R * P + i] : 1.0f;
+    wo[i] = p.W_o ? p.W_o[(int64_t)hi * R * P + i] : 1.0f;
+  }
   const float* biasBg = p.bias_B ? p.bias_B + (int64_t)hi * R * N : nullptr;
   const float* biasCg = p.bias_C ? p.bias_C + (int64_t)hi * R * N : nullptr;
-  const float* wog = p.W_o ? p.W_o + (int64_t)hi * R * P : nullptr;
   for (int k = tid; k < K2; k += kThreads) base[k] = 0.0;
   load_coefs(j0);
   store_coefs(0);
@@ -421,6 +441,18 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
   const bool state_warp = warp >= 4;
   const int prow = (P == 128) ? (32 * q4 + lane) : (16 * q4 + (lane & 15));
   const bool st_owner = (P == 128) || (lane >= 16);  // holds the fp32 state of row prow
+
+  // transform thread mapping: fixed 16-byte column chunk and MIMO branch per thread
+  constexpr int CHN = N / 8;
+  constexpr int ROWS_PER_IT = kThreads / CHN;
+  const int tch = tid % CHN;
+  const int tr = (tid / CHN) % R;  // fixed: ROWS_PER_IT is a multiple of R
+  float bB[8], bC[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    bB[e] = biasBg ? __ldg(biasBg + tr * N + tch * 8 + e) : 0.0f;
+    bC[e] = biasCg ? __ldg(biasCg + tr * N + tch * 8 + e) : 0.0f;
+  }
 
   // ---- incoming rotated-frame state h+ of this segment
   //   nseg == 1 (full pass): h_{-1} + beta'_0 u_{-1} from the state / carry;
@@ -448,7 +480,8 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
           const int n = 32 * c + e;
           float u = 0.0f;
 #pragma unroll
-          for (int r = 0; r < R; ++r) u = fmaf(cB[r * N + n] + (biasBg ? __ldg(biasBg + r * N + n) : 0.0f), xprev[r], u);
+          for (int r = 0; r < R; ++r)
+            u = fmaf(cB[r * N + n] + (biasBg ? __ldg(biasBg + r * N + n) : 0.0f), xprev[r], u);
           v[e] = fmaf(bp0, u, h0[(int64_t)n * P + prow]);
         }
         if (!FULL && sg.nseg > 1 && st_owner) {
@@ -500,6 +533,65 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
   __syncthreads();
   tc_fence_after();
 
+  // state update ST <- e^{Le} ST + hs * H for this thread's TMEM row (state warps)
+  auto state_update = [&](float Le_exp, float hs, bool write_bf16) {
+#pragma unroll 1
+    for (int c = 0; c < N / 32; ++c) {
+      uint32_t hv[32];
+      float f[32];
+      if constexpr (P == 64) {
+        tmem_ld32(tmem + lane_base + C::TM_H + 32 * c, hv);  // lanes 0-15: H, lanes 16-31: state
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float hlow = __shfl_up_sync(kFull, __uint_as_float(hv[e]), 16);
+          f[e] = (lane >= 16) ? fmaf(Le_exp, __uint_as_float(hv[e]), hs * hlow) : __uint_as_float(hv[e]);
+          hv[e] = __float_as_uint(f[e]);
+        }
+        tmem_st32(tmem + lane_base + C::TM_ST + 32 * c, hv);
+      } else {
+        uint32_t sv[32];
+        tmem_ld32(tmem + lane_base + C::TM_H + 32 * c, hv);
+        tmem_ld32(tmem + lane_base + C::TM_ST + 32 * c, sv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          f[e] = fmaf(Le_exp, __uint_as_float(sv[e]), hs * __uint_as_float(hv[e]));
+          sv[e] = __float_as_uint(f[e]);
+        }
+        tmem_st32(tmem + lane_base + C::TM_ST + 32 * c, sv);
+      }
+      if (write_bf16 && st_owner) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float f8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f8[e] = f[8 * q + e];
+          sts128(sH + sw128(prow, 4 * c + q, P * 128), pack8(f8));
+        }
+      }
+    }
+    tmem_wait_st();
+  };
+  // refresh the bf16 copy of the state from TMEM (state warps)
+  auto write_state_bf16 = [&]() {
+#pragma unroll 1
+    for (int c = 0; c < N / 32; ++c) {
+      uint32_t sv[32];
+      tmem_ld32(tmem + lane_base + C::TM_ST + 32 * c, sv);
+      tmem_wait_ld();
+      if (st_owner) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float f8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f8[e] = __uint_as_float(sv[8 * q + e]);
+          sts128(sH + sw128(prow, 4 * c + q, P * 128), pack8(f8));
+        }
+      }
+    }
+  };
+
   uint32_t mma_phase = 0, load_phase = 0;
   bool failed = false;
   float seg_logdec = 0.0f;
@@ -529,7 +621,7 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
 #pragma unroll
       for (int e = 0; e < PER; ++e) {
         const int t = lane * PER + e;
-        run += (t < Q) ? dtA[t] * aA[t] : 0.0f;
+        run += (t < nv) ? dtA[t] * aA[t] : 0.0f;
         loc[e] = run;
       }
       float incl = run;
@@ -540,23 +632,43 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
       }
       const float Le = __shfl_sync(kFull, incl, 31);
       const float excl = incl - run;
+      float lmin = 0.0f, lmax = 0.0f;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) {
+        loc[e] += excl;
+        lmin = fminf(lmin, loc[e]);
+        lmax = fmaxf(lmax, loc[e]);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        lmin = fminf(lmin, __shfl_xor_sync(kFull, lmin, off));
+        lmax = fmaxf(lmax, __shfl_xor_sync(kFull, lmax, off));
+      }
+      const bool fast = (lmax - lmin) <= 160.0f;
+      const float m = fast ? 0.5f * (lmax + lmin) : 0.0f;
 #pragma unroll
       for (int e = 0; e < PER; ++e) {
         const int t = lane * PER + e;
         if (t < Q) {
-          const float Lct = excl + loc[e];
-          const float gm = lmA[t] * dtA[t];
-          const float bpn = (t + 1 < Q) ? (1.0f - lmA[t + 1]) * dtA[t + 1] : scal[2 + par];
-          // mask record: log2 cumulative decay, gamma, gamma + beta'_{t+1}
-          mrec[t] = make_float4(Lct * 1.4426950408889634f, gm, gm + bpn, 0.0f);
-          gamA[t] = gm;
-          cwA[t] = __expf(Le - Lct) * (gm + bpn);
-          decA[t] = __expf(Lct);
+          const float Lct = loc[e];
+          const bool valid = t < nv;
+          const float gm = valid ? lmA[t] * dtA[t] : 0.0f;
+          const float bpn = (t + 1 < Q) ? ((t + 1 < nv) ? (1.0f - lmA[t + 1]) * dtA[t + 1] : 0.0f)
+                                        : (valid ? scal[2 + par] : 0.0f);
+          const float w = gm + bpn;
+          const float dg = (w > 0.0f) ? gm / w : 0.0f;
+          const float at = fast ? __expf(Lct - m) : 1.0f;
+          const float xs = fast ? __expf(m - Lct) * w : w;
+          const float dect = __expf(Lct);
+          recA[t] = make_float4(Lct * 1.4426950408889634f, dg, at, xs);
+          recB[t] = make_float4(fast ? __expf(m) : dect, dect, __expf(Le - Lct), 0.0f);
         }
       }
       if (lane == 0) {
         scal[0] = __expf(Le);
         scal[1] = Le;
+        scal[4] = fast ? __expf(Le - m) : 1.0f;
+        scal[5] = fast ? 1.0f : 0.0f;
       }
     }
     const int ak = tid % K2, aseg = tid / K2;
@@ -573,6 +685,7 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
       segsum[aseg * K2 + ak] = run;
     }
     __syncthreads();
+    const bool fast = scal[5] != 0.0f;
     {
       double total = 0.0;
       float aoff = 0.0f;
@@ -603,77 +716,76 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
       base[ak] = nb;
     }
 
-    // ---- B: rotate B (and C) in place; build X, Xs (and e^{Lc} C~)
+    // ---- B: rotate B (and C) in place; build X' = b_t w_t W_x x (and the scaled C copy)
     {
-      constexpr int CHN = N / 8;
-      constexpr int ROWS_PER_IT = kThreads / CHN;
-      const int ch = tid % CHN;
-      const int r = (tid / CHN) % R;  // fixed: ROWS_PER_IT is a multiple of R
-      float bB[8], bC[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        bB[e] = biasBg ? __ldg(biasBg + r * N + ch * 8 + e) : 0.0f;
-        bC[e] = biasCg ? __ldg(biasCg + r * N + ch * 8 + e) : 0.0f;
-      }
+      const int i0 = tid / CHN;
+      const uint32_t off0 = (uint32_t)(tch >> 3) * (kRows * 128) + (uint32_t)i0 * 128u +
+                            ((uint32_t)((tch & 7) ^ (i0 & 7)) << 4);  // row i0 + k*ROWS_PER_IT keeps i & 7
 #pragma unroll 2
-      for (int i = tid / CHN; i < kRows; i += ROWS_PER_IT) {
+      for (int it = 0; it < kRows / ROWS_PER_IT; ++it) {
+        const int i = i0 + it * ROWS_PER_IT;
         const int t = i / R;
-        const uint32_t off = sw128(i, ch, kRows * 128);
-        const float4 w01 = *reinterpret_cast<const float4*>(&cs[t * K2 + ch * 4]);
-        const float4 w23 = *reinterpret_cast<const float4*>(&cs[t * K2 + ch * 4 + 2]);
+        const uint32_t off = off0 + (uint32_t)(it * ROWS_PER_IT) * 128u;
+        const float4 w01 = *reinterpret_cast<const float4*>(&cs[t * K2 + tch * 4]);
+        const float4 w23 = *reinterpret_cast<const float4*>(&cs[t * K2 + tch * 4 + 2]);
         const float wc[4] = {w01.x, w01.z, w23.x, w23.z};
         const float ws[4] = {w01.y, w01.w, w23.y, w23.w};
-        const bool valid = t < nv;
-        {
-          float f[8];
-          unpack8(lds128(sBT + off), f);
+        if (t < nv) {
+          float bsc = 1.0f;
+          if constexpr (!FULL) bsc = fast ? 1.0f : recB[t].z;  // exact tiles: Bt rows * e^{Le - Lc_t}
+          {
+            float f[8];
+            unpack8(lds128(sBT + off), f);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float b0 = f[2 * q] + bB[2 * q], b1 = f[2 * q + 1] + bB[2 * q + 1];
-            f[2 * q] = valid ? (wc[q] * b0 + ws[q] * b1) : 0.0f;  // Rot(-Phi)
-            f[2 * q + 1] = valid ? (wc[q] * b1 - ws[q] * b0) : 0.0f;
+            for (int q = 0; q < 4; ++q) {
+              const float b0 = f[2 * q] + bB[2 * q], b1 = f[2 * q + 1] + bB[2 * q + 1];
+              f[2 * q] = bsc * (wc[q] * b0 + ws[q] * b1);  // Rot(-Phi)
+              f[2 * q + 1] = bsc * (wc[q] * b1 - ws[q] * b0);
+            }
+            sts128(sBT + off, pack8(f));
           }
-          sts128(sBT + off, pack8(f));
-        }
-        if constexpr (FULL) {
-          float f[8];
-          unpack8(lds128(sCT + off), f);
+          if constexpr (FULL) {
+            float f[8];
+            unpack8(lds128(sCT + off), f);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float d0 = f[2 * q] + bC[2 * q], d1 = f[2 * q + 1] + bC[2 * q + 1];
-            f[2 * q] = valid ? (wc[q] * d0 + ws[q] * d1) : 0.0f;
-            f[2 * q + 1] = valid ? (wc[q] * d1 - ws[q] * d0) : 0.0f;
+            for (int q = 0; q < 4; ++q) {
+              const float d0 = f[2 * q] + bC[2 * q], d1 = f[2 * q + 1] + bC[2 * q + 1];
+              f[2 * q] = wc[q] * d0 + ws[q] * d1;
+              f[2 * q + 1] = wc[q] * d1 - ws[q] * d0;
+            }
+            sts128(sCT + off, pack8(f));
+            if constexpr (!C::kInterInS) {
+              const float dd = recB[t].x;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f[e] *= dd;
+              sts128(sC2 + off, pack8(f));
+            }
           }
-          sts128(sCT + off, pack8(f));
-          if constexpr (!C::kInterInS) {
-            const float dd = decA[t];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] *= dd;
-            sts128(sC2 + off, pack8(f));
+        } else {
+          const uint4 z = make_uint4(0, 0, 0, 0);
+          sts128(sBT + off, z);
+          if constexpr (FULL) {
+            sts128(sCT + off, z);
+            if constexpr (!C::kInterInS) sts128(sC2 + off, z);
           }
         }
       }
       constexpr int CHP = P / 8;
-      for (int idx = tid; idx < Q * CHP; idx += kThreads) {
-        const int t = idx / CHP, chp = idx % CHP;
+      const int xch = tid % CHP;  // fixed column chunk
+      for (int t = tid / CHP; t < Q; t += kThreads / CHP) {
         float fx[8];
-        unpack8(lds128(sXSTG + (uint32_t)(t * P + chp * 8) * 2), fx);
-        const bool valid = t < nv;
-        const float cwt = cwA[t];
+        unpack8(lds128(sXSTG + (uint32_t)(t * P + xch * 8) * 2), fx);
+        const float xs = (t < nv) ? recA[t].w : 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) fx[e] *= xs;
 #pragma unroll
         for (int rr = 0; rr < R; ++rr) {
           const int i = t * R + rr;
-          const float4 w0 = *reinterpret_cast<const float4*>(&wx[rr * P + chp * 8]);
-          const float4 w1 = *reinterpret_cast<const float4*>(&wx[rr * P + chp * 8 + 4]);
-          const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-          float xr[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) xr[e] = valid ? fx[e] * wv[e] : 0.0f;
-          const uint32_t off = sw128(i, chp, kRows * 128);
-          if constexpr (FULL) sts128(sX + off, pack8(xr));
-#pragma unroll
-          for (int e = 0; e < 8; ++e) xr[e] *= cwt;
-          sts128(sXS + off, pack8(xr));
+          const float4 w0 = *reinterpret_cast<const float4*>(&wx[rr * P + xch * 8]);
+          const float4 w1 = *reinterpret_cast<const float4*>(&wx[rr * P + xch * 8 + 4]);
+          const float xr[8] = {fx[0] * w0.x, fx[1] * w0.y, fx[2] * w0.z, fx[3] * w0.w,
+                               fx[4] * w1.x, fx[5] * w1.y, fx[6] * w1.z, fx[7] * w1.w};
+          sts128(sX + sw128(i, xch, kRows * 128), pack8(xr));
         }
       }
     }
@@ -682,10 +794,9 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
     __syncthreads();
     tc_fence_after();
 
-    // ---- C: MMAs that need only this tile's staged operands
+    // ---- C: MMA1 (S), [MMA3 without kInterInS], MMA4 (H = X'^T Bt) unless the tile is exact
+    const bool mma4_early = !FULL || fast;
     if (tid == 0) {
-      // x and theta staging are consumed: prefetch the next tile's ...
-      // (B and C follow once the MMAs that read them have completed)
       if constexpr (FULL) {
 #pragma unroll
         for (int k = 0; k < N / 16; ++k) {
@@ -701,10 +812,11 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
           }
         }
       }
+      if (mma4_early) {
 #pragma unroll
-      for (int k = 0; k < kRows / 16; ++k) {
-        mma_ss(tmem + C::TM_H, sdesc(sXS + k * 2048, kRows * 128, 1024), sdesc(sBT + k * 2048, kRows * 128, 1024),
-               C::ID_H, k > 0);
+        for (int k = 0; k < kRows / 16; ++k)
+          mma_ss(tmem + C::TM_H, sdesc(sX + k * 2048, kRows * 128, 1024), sdesc(sBT + k * 2048, kRows * 128, 1024),
+                 C::ID_H, k > 0);
       }
       mma_commit(mma_bar);
     }
@@ -720,8 +832,8 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
       }
     }
     tc_fence_after();
-    // B (and, without kInterInS, C) tiles are free: the next tile's loads may land now
-    const bool prefetch_early = !(FULL && C::kInterInS);
+    // operand buffers no later MMA of this tile reads: the next tile's loads may land now
+    const bool prefetch_early = !FULL || (!C::kInterInS && fast);
     if (tid == 0 && prefetch_early && j + 1 < j1) issue_loads(j + 1);
 
     // ---- D: mask S in TMEM (warps 0-3) | state update (warps 4-7)
@@ -729,73 +841,57 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
       if constexpr (FULL) {
         const int i = 32 * warp + lane;
         const int t = i / R;
-        const int t_hi = (32 * warp + 31) / R;
-        const float Lt2 = mrec[t].x;
+        const int t_lo = (32 * warp) / R, t_hi = (32 * warp + 31) / R;
+        const float4 ra = recA[t];
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
+          const int s_lo = (32 * c) / R, s_hi = (32 * c + 31) / R;
           uint32_t o[16];
-          if ((32 * c) / R > t_hi) {
+          if (s_lo > t_hi) {  // entirely above the diagonal
 #pragma unroll
             for (int e = 0; e < 16; ++e) o[e] = 0u;
           } else {
             uint32_t v[32];
             tmem_ld32(tmem + lane_base + C::TM_S + 32 * c, v);
             tmem_wait_ld();
-            float f[32];
+            if (fast && s_hi < t_lo) {  // entirely below the diagonal: S' = S
 #pragma unroll
-            for (int jj = 0; jj < 32 / R; ++jj) {
-              const int s = (32 * c) / R + jj;
-              const float4 m = mrec[s];
-              const float w = (s < t) ? m.z : ((s == t) ? m.y : 0.0f);
-              const float fac = (s <= t) ? exp2f(Lt2 - m.x) * w : 0.0f;
+              for (int e = 0; e < 16; ++e) o[e] = pack_bf16(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+            } else {
+              float f[32];
 #pragma unroll
-              for (int rr = 0; rr < R; ++rr) f[jj * R + rr] = fac * __uint_as_float(v[jj * R + rr]);
+              for (int jj = 0; jj < 32 / R; ++jj) {
+                const int s = s_lo + jj;
+                const float4 rs = recA[s];
+                float fac = (s < t) ? 1.0f : ((s == t) ? rs.y : 0.0f);
+                if (!fast && s <= t) fac *= ex2_approx(ra.x - rs.x);
+#pragma unroll
+                for (int rr = 0; rr < R; ++rr) f[jj * R + rr] = fac * __uint_as_float(v[jj * R + rr]);
+              }
+#pragma unroll
+              for (int e = 0; e < 16; ++e) o[e] = pack_bf16(f[2 * e], f[2 * e + 1]);
             }
-#pragma unroll
-            for (int e = 0; e < 16; ++e) o[e] = pack_bf16(f[2 * e], f[2 * e + 1]);
           }
           tmem_st16(tmem + lane_base + C::TM_S + 16 * c, o);
         }
         tmem_wait_st();
       }
+    } else if (mma4_early) {
+      state_update(scal[0], scal[4], FULL && !C::kInterInS);
     } else {
-      const float Le = scal[0];
+      // exact tile: scale Bt rows by e^{Le - Lc_t} in place (MMA1 has read Bt) for MMA4
+      const int lt = tid - 128;
 #pragma unroll 1
-      for (int c = 0; c < N / 32; ++c) {
-        uint32_t hv[32], sv[32];
-        if constexpr (P == 64) {
-          tmem_ld32(tmem + lane_base + C::TM_H + 32 * c, hv);  // lanes 0-15: H, lanes 16-31: state
-          tmem_wait_ld();
+      for (int idx = lt; idx < kRows * CHN; idx += 128) {
+        const int i = idx / CHN, ch = idx % CHN;
+        const uint32_t off = sw128(i, ch, kRows * 128);
+        const float sc = recB[i / R].z;
+        float f[8];
+        unpack8(lds128(sBT + off), f);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float hlow = __shfl_up_sync(kFull, __uint_as_float(hv[e]), 16);
-            if (lane >= 16) hv[e] = __float_as_uint(fmaf(Le, __uint_as_float(hv[e]), hlow));
-          }
-          tmem_st32(tmem + lane_base + C::TM_ST + 32 * c, hv);
-          if constexpr (FULL && !C::kInterInS) {
-            // (not reached: P == 64 always uses kInterInS)
-          }
-        } else {
-          tmem_ld32(tmem + lane_base + C::TM_H + 32 * c, hv);
-          tmem_ld32(tmem + lane_base + C::TM_ST + 32 * c, sv);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            sv[e] = __float_as_uint(fmaf(Le, __uint_as_float(sv[e]), __uint_as_float(hv[e])));
-          tmem_st32(tmem + lane_base + C::TM_ST + 32 * c, sv);
-          if constexpr (FULL && !C::kInterInS) {
-            // MMA3 (which read the old bf16 state) has completed: refresh the bf16 copy
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              float f8[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) f8[e] = __uint_as_float(sv[8 * q + e]);
-              sts128(sH + sw128(prow, 4 * c + q, P * 128), pack8(f8));
-            }
-          }
-        }
+        for (int e = 0; e < 8; ++e) f[e] *= sc;
+        sts128(sBT + off, pack8(f));
       }
-      tmem_wait_st();
     }
     if constexpr (FULL) {
       fence_async_smem();
@@ -803,7 +899,7 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
       __syncthreads();
       tc_fence_after();
 
-      // ---- E: MMA3 (kInterInS: Ct h+ into the free half of S) and MMA2 (Y += S' X)
+      // ---- E: [MMA3 with kInterInS], MMA2 (Y += S' X'), [MMA4 for exact tiles]
       if (tid == 0) {
         if constexpr (C::kInterInS) {
 #pragma unroll
@@ -816,7 +912,13 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
 #pragma unroll
         for (int k = 0; k < kRows / 16; ++k)
           mma_ts(tmem + C::TM_Y, tmem + C::TM_S + 8 * k, sdesc(sX + k * 2048, kRows * 128, 1024), C::ID_Y2,
-                 C::kInterInS ? (k > 0) : 1);  // without kInterInS, Y already holds e^{Lc} Ct h+
+                 C::kInterInS ? (k > 0) : 1);  // without kInterInS, Y already holds the Ct h+ term
+        if (!mma4_early) {
+#pragma unroll
+          for (int k = 0; k < kRows / 16; ++k)
+            mma_ss(tmem + C::TM_H, sdesc(sX + k * 2048, kRows * 128, 1024),
+                   sdesc(sBT + k * 2048, kRows * 128, 1024), C::ID_H, k > 0);
+        }
         mma_commit(mma_bar);
       }
       {
@@ -830,14 +932,15 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
       tc_fence_after();
       if (tid == 0 && !prefetch_early && j + 1 < j1) issue_loads(j + 1);
 
-      // ---- F: epilogue y_t = sum_r W_o[r] * (Y + e^{Lc_t} Yi)_{t,r} + D x_t; refresh bf16 state
+      // ---- F: epilogue y_t = sum_r W_o[r] * (a_t Y [+ e^{Lc_t} Yi])_{t,r} + D x_t
       {
         const int i = 32 * q4 + lane;
         const int t = i / R, r = i % R;
         const int half = warp >> 2;
         constexpr int PH = P / 2;
         constexpr int W = 16 / R;
-        const float dect = decA[t];
+        const float at = recA[t].z;
+        const float dect = recB[t].y;
         const int64_t yrow = ((tok_base + c0 + t) * H + hi) * P;
 #pragma unroll 1
         for (int c = 0; c < PH / 16; ++c) {
@@ -850,26 +953,34 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
             tmem_ld16(tmem + lane_base + C::TM_YI + col0, vi);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) f[e] = fmaf(dect, __uint_as_float(vi[e]), __uint_as_float(v[e]));
+            for (int e = 0; e < 16; ++e) f[e] = fmaf(dect, __uint_as_float(vi[e]), at * __uint_as_float(v[e]));
           } else {
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) f[e] = __uint_as_float(v[e]);
+            for (int e = 0; e < 16; ++e) f[e] = at * __uint_as_float(v[e]);
           }
-          if (wog) {
 #pragma unroll
-            for (int e4 = 0; e4 < 4; ++e4) {
-              const float4 w4 = __ldg(reinterpret_cast<const float4*>(wog + r * P + col0 + 4 * e4));
-              f[4 * e4] *= w4.x;
-              f[4 * e4 + 1] *= w4.y;
-              f[4 * e4 + 2] *= w4.z;
-              f[4 * e4 + 3] *= w4.w;
+          for (int e4 = 0; e4 < 4; ++e4) {
+            const float4 w4 = *reinterpret_cast<const float4*>(&wo[r * P + col0 + 4 * e4]);
+            f[4 * e4] *= w4.x;
+            f[4 * e4 + 1] *= w4.y;
+            f[4 * e4 + 2] *= w4.z;
+            f[4 * e4 + 3] *= w4.w;
+          }
+          // reduce over the R branches (adjacent lanes); lane r keeps columns [r*W, r*W + W)
+#pragma unroll
+          for (int m = R / 2; m >= 1; m >>= 1) {
+            const bool upper = (r & m) != 0;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              // pair columns that differ in the bit of value m*W within the remaining span
+              if ((e / W) % (2 * m) < m) {
+                const float mine = upper ? f[e + m * W] : f[e];
+                const float other = upper ? f[e] : f[e + m * W];
+                const float got = __shfl_xor_sync(kFull, other, m);
+                if (upper) f[e + m * W] = mine + got; else f[e] = mine + got;
+              }
             }
-          }
-#pragma unroll
-          for (int m = 1; m < R; m <<= 1) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) f[e] += __shfl_xor_sync(kFull, f[e], m);
           }
           if (t < nv) {
             float outv[W];
@@ -891,25 +1002,9 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
               *reinterpret_cast<uint32_t*>(yg + yrow + pc + e) = pack_bf16(outv[e], outv[e + 1]);
           }
         }
-        if constexpr (C::kInterInS) {
-          // MMA3 has read the old bf16 state: write the new one (kept in TMEM lanes 16-31)
-          if (state_warp) {
-#pragma unroll 1
-            for (int c2 = 0; c2 < N / 32; ++c2) {
-              uint32_t sv[32];
-              tmem_ld32(tmem + lane_base + C::TM_ST + 32 * c2, sv);
-              tmem_wait_ld();
-              if (st_owner) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  float f8[8];
-#pragma unroll
-                  for (int e = 0; e < 8; ++e) f8[e] = __uint_as_float(sv[8 * q + e]);
-                  sts128(sH + sw128(prow, 4 * c2 + q, P * 128), pack8(f8));
-                }
-              }
-            }
-          }
+        if (state_warp) {
+          if (!mma4_early) state_update(scal[0], 1.0f, true);
+          else if constexpr (C::kInterInS) write_state_bf16();
         }
       }
     }

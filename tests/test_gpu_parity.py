@@ -252,3 +252,22 @@ def test_unsupported_tile_shape_uses_sequential_kernel():
     # the dispatcher runs the sequential kernel instead (same results)
     inp = make_inputs(dtype="bf16", seed=204, extras=True, b=1, L=40, H=2, P=128, N=128, R=1, G=1)
     check_scan(inp)
+
+
+@pytest.mark.parametrize("shape", [
+    dict(b=1, L=300, H=2, P=64, N=64, R=2, G=1),
+    dict(b=1, L=200, H=2, P=128, N=128, R=4, G=1),
+    dict(b=1, L=3000, H=2, P=64, N=64, R=2, G=1),     # segmented
+], ids=["P64", "P128", "P64seg"])
+def test_tc_strong_decay_tiles(shape):
+    # Tokens with dt*A far below -1 make the log decay inside a tile span more than fp32
+    # exponent range allows the pivot split; those tiles run the exact per-element path.
+    inp = make_inputs(dtype="bf16", seed=206, extras=True, **shape)
+    L = shape["L"]
+    burst = np.zeros(L, dtype=bool)
+    burst[L // 5: L // 5 + 40] = True
+    burst[L // 2: L // 2 + 7] = True
+    inp.dt[:, burst, :] = 4.0
+    inp.A[:, burst, :] = -12.0
+    st = make_state(shape["b"], shape["H"], shape["P"], shape["N"], shape["R"], seed=207)
+    check_scan(inp, state=st)
