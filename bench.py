@@ -185,14 +185,25 @@ def barrier(world):
     torch.cuda.synchronize()
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
+    """Max of a per-rank scalar (a timed region) over all ranks of the process group."""
     import torch
     if world == 1:
         return float(x)
     import torch.distributed as dist
-    t = torch.tensor([float(x)], device="cuda", dtype=torch.float64)
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(base_seed, rank):
+    """Every rank draws its own batch (weak scaling: independent sequences per rank)."""
+    return base_seed + 7919 * rank
+
+
+def job_throughput(tokens_per_rank_step, steps, world, max_ms):
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's timed region."""
+    return world * tokens_per_rank_step * steps / (max_ms / 1e3)
 
 
 def make_ring(inp, n_sets, device):
@@ -225,14 +236,14 @@ def run_ours(args):
     device = f"cuda:{local}"
     peaks = measured_peaks()
     cfg = dict(CONFIGS[WORKLOAD])
-    inp = config_inputs(WORKLOAD, seed=SEEDS[WORKLOAD] + rank)
+    inp = config_inputs(WORKLOAD, seed=rank_seed(SEEDS[WORKLOAD], rank))
     dims = m3.dims_of(inp)
     dims1 = m3.dims_of(inp, L=1)
     per_set = prefill_bytes(cfg)
     n_sets = max(2, -(-3 * L2_BYTES // per_set))
     ring = make_ring(inp, n_sets, device)
     # the decode token of each set: a fresh draw's first token
-    tok_inp = config_inputs(WORKLOAD, seed=SEEDS[WORKLOAD] + 100 + rank, L=1)
+    tok_inp = config_inputs(WORKLOAD, seed=rank_seed(SEEDS[WORKLOAD] + 100, rank), L=1)
     tok_dev = token_slice(m3.to_device(tok_inp, device), 0)
     for s in ring:
         s["state1"] = m3.State.wrap(dims1, *s["keep"])
@@ -270,7 +281,7 @@ def run_ours(args):
     ms = max_over_ranks(ms_local, world)
     prefill_ms = [a.elapsed_time(b) for a, b in evs]
     tokens_step = cfg["b"] * (cfg["L"] + 1)
-    value = world * tokens_step * args.steps / (ms / 1e3)
+    value = job_throughput(tokens_step, args.steps, world, ms)
     gpu_launches = (3 if ws_bytes > 0 else 2) * args.steps  # [state pass] + full pass + decode
 
     pf_ms = statistics.mean(prefill_ms)

@@ -249,19 +249,15 @@ struct Cfg {
   static constexpr bool FULL = (MODE == MODE_FULL);
   static constexpr int Q = kRows / R;   // tokens per tile
   static constexpr int K2 = N / 2;      // rotation pairs
-  // P = 64: the inter-chunk readout goes to the free half of the S columns after masking.
-  static constexpr bool kInterInS = (P == 64);
   static constexpr int TILE_N = kRows * N * 2;
   static constexpr int TILE_P = kRows * P * 2;
   static constexpr int TILE_H = P * N * 2;
   static constexpr int OFF_BT = 0;
   static constexpr int OFF_CT = OFF_BT + TILE_N;
-  static constexpr int OFF_C2 = OFF_CT + (FULL ? TILE_N : 0);
-  static constexpr int OFF_X = OFF_C2 + ((FULL && !kInterInS) ? TILE_N : 0);
+  static constexpr int OFF_X = OFF_CT + (FULL ? TILE_N : 0);
   static constexpr int OFF_H = OFF_X + TILE_P;
-  static constexpr int OFF_CS = OFF_H + (FULL ? TILE_H : 0);       // float2 [Q][K2]
-  static constexpr int OFF_TH = OFF_CS + Q * K2 * 4;                // theta staging: 2nd half of CS
-  static constexpr int OFF_XSTG = OFF_CS + Q * K2 * 8;              // x staging [Q][P] bf16
+  static constexpr int OFF_CS = OFF_H + (FULL ? TILE_H : 0);       // float2 [2][Q][K2]
+  static constexpr int OFF_XSTG = OFF_CS + 2 * Q * K2 * 8;          // x staging [Q][P] bf16
   static constexpr int OFF_WX = OFF_XSTG + Q * P * 2;              // W_x [R][P]
   static constexpr int OFF_WO = OFF_WX + R * P * 4;                 // W_o [R][P]
   static constexpr int OFF_BASE = OFF_WO + R * P * 4;               // double [K2]
@@ -269,15 +265,14 @@ struct Cfg {
   static constexpr int SEGLEN = (Q + SEGS - 1) / SEGS;
   static constexpr int OFF_SEGSUM = OFF_BASE + K2 * 8;              // float [SEGS][K2]
   static constexpr int TOKF = Q + 4;
-  static constexpr int OFF_TOK = OFF_SEGSUM + SEGS * K2 * 4;        // per-token float arrays
-  static constexpr int NTOKARR = 8;
-  static constexpr int OFF_MREC = OFF_TOK + NTOKARR * TOKF * 4;     // float4 [Q] x 2 per-token records
-  static constexpr int OFF_MISC = OFF_MREC + 2 * Q * 16;
+  static constexpr int OFF_RAW = OFF_SEGSUM + SEGS * K2 * 4;        // float [2][4][TOKF]: dt, A, lam, (misc)
+  static constexpr int OFF_REC = OFF_RAW + 2 * 4 * TOKF * 4;        // float4 [2][2][Q]
+  static constexpr int OFF_SCAL = OFF_REC + 2 * 2 * Q * 16;         // float [2][8]
+  static constexpr int OFF_MISC = OFF_SCAL + 2 * 8 * 4;
   static constexpr int BYTES = OFF_MISC + 64;
   static constexpr int SMEM = BYTES + 1024;  // slack for 1024-byte alignment
   // tensor memory columns
   static constexpr uint32_t TM_S = 0;
-  static constexpr uint32_t TM_YI = 64;            // kInterInS: Ct h+ in S columns 64..64+P
   static constexpr uint32_t TM_Y = 128;
   static constexpr uint32_t TM_H = 128 + P;
   static constexpr uint32_t TM_ST = (P == 64) ? TM_H : TM_H + N;  // P = 64: lanes 16-31 of H's columns
@@ -289,34 +284,31 @@ struct Cfg {
   static constexpr uint32_t ID_Y2 = idesc_bf16(128, P, false, true);
   static constexpr int TX_B = kRows * N * 2;
   static constexpr int TX_X = Q * P * 2;
-  static constexpr int TX_T = Q * K2 * 4;
+  static constexpr int NT = FULL ? 128 : 256;  // threads that stage operand tiles
 };
 
-// per-token array slots (each TOKF floats): raw dt/A/lam of the current and next tile
-enum { A_DT0 = 0, A_A0, A_LM0, A_DT1, A_A1, A_LM1, A_SCAL };
-// scalars in A_SCAL: [0] e^{Le}, [1] Le, [2..3] next-token beta' by parity, [4] state-update
-// scale of H, [5] 1 when the tile uses the pivot factorisation
-//
 // The decay inside a tile, e^{Lc_t - Lc_s}, is split around a pivot m (the middle of the
 // tile's log-decay range) as a_t * b_s with a_t = e^{Lc_t - m}, b_s = e^{m - Lc_s}.  b_s and
 // the trapezoid weight w_s = gamma_s + beta'_{s+1} go into X' = b_s w_s X, a_t is applied to
 // the output rows, so the masked score matrix needs no exponentials: S' = S below the
-// diagonal, S * gamma_s / w_s on it, 0 above.  The state update becomes H = X'^T Bt times the
+// diagonal, S * gamma_s / w_s on it, 0 above.  The inter-chunk term e^{Lc_t} Ct h+ equals
+// a_t Ct (e^m h+): the bf16 copy of the state is written pre-scaled by e^m, so that product
+// accumulates into the same Y as S' X'.  The state update becomes H = X'^T Bt times the
 // uniform factor e^{Le - m}.  When the range of Lc within a tile exceeds 160 the split could
-// overflow fp32; such tiles take the exact path (a_t = 1, b_s = 1, e^{Lc_t - Lc_s} per element,
-// Bt rows scaled by e^{Le - Lc_t} before the state update).
-// record A[t] = {Lc_t * log2 e, gamma_t / w_t, a_t, b_t w_t};  record B[t] = {C2 row scale,
-// e^{Lc_t}, e^{Le - Lc_t}, 0}
+// overflow fp32; such tiles take the exact path (m = 0, a_t = 1, b_s = 1, e^{Lc_t - Lc_s} per
+// element, Ct rows scaled by e^{Lc_t} and Bt rows by e^{Le - Lc_t} in place).
+// record A[t] = {Lc_t * log2 e, gamma_t / w_t, a_t, b_t w_t};  record B[t] = {e^{Lc_t},
+// e^{Le - Lc_t}, 0, 0};  scalars {e^{Le}, Le, e^{Le - m} or 1, fast, e^m or 1, 0, 0, 0}
 
 template <int R, int N, int P, int MODE>
 __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
     scan_tc_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
-                   const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmT,
-                   const Params p, const SegInfo sg) {
+                   const __grid_constant__ CUtensorMap tmX, const Params p, const SegInfo sg) {
   using C = Cfg<R, N, P, MODE>;
   constexpr bool FULL = C::FULL;
   constexpr int Q = C::Q;
   constexpr int K2 = C::K2;
+  constexpr int NT = C::NT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -335,44 +327,51 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
   const bool last_seg = (seg == sg.nseg - 1);
   const int64_t tok_base = (int64_t)bi * L;  // first token of this sequence (flattened b*L index)
 
-  const uint32_t sBT = smem_u32(sm + C::OFF_BT), sCT = smem_u32(sm + C::OFF_CT), sC2 = smem_u32(sm + C::OFF_C2);
+  const uint32_t sBT = smem_u32(sm + C::OFF_BT), sCT = smem_u32(sm + C::OFF_CT);
   const uint32_t sX = smem_u32(sm + C::OFF_X), sH = smem_u32(sm + C::OFF_H);
-  const uint32_t sXSTG = smem_u32(sm + C::OFF_XSTG), sTH = smem_u32(sm + C::OFF_TH);
-  float2* cs = reinterpret_cast<float2*>(sm + C::OFF_CS);
-  const float* th_stg = reinterpret_cast<const float*>(sm + C::OFF_TH);
+  const uint32_t sXSTG = smem_u32(sm + C::OFF_XSTG);
+  float2* csb = reinterpret_cast<float2*>(sm + C::OFF_CS);
   float* wx = reinterpret_cast<float*>(sm + C::OFF_WX);
   float* wo = reinterpret_cast<float*>(sm + C::OFF_WO);
   double* base = reinterpret_cast<double*>(sm + C::OFF_BASE);
   float* segsum = reinterpret_cast<float*>(sm + C::OFF_SEGSUM);
-  float* tokf = reinterpret_cast<float*>(sm + C::OFF_TOK);
-  float4* recA = reinterpret_cast<float4*>(sm + C::OFF_MREC);
-  float4* recB = recA + Q;
-  float* scal = tokf + A_SCAL * C::TOKF;
+  float* raw = reinterpret_cast<float*>(sm + C::OFF_RAW);
+  float4* recb = reinterpret_cast<float4*>(sm + C::OFF_REC);
+  float* scalb = reinterpret_cast<float*>(sm + C::OFF_SCAL);
   uint64_t* mma_bar = reinterpret_cast<uint64_t*>(sm + C::OFF_MISC);
   uint64_t* load_bar = reinterpret_cast<uint64_t*>(sm + C::OFF_MISC + 8);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC + 16);
+  auto rawA = [&](int slot, int k) { return raw + (slot * 4 + k) * C::TOKF; };
+  auto recA = [&](int slot) { return recb + (slot * 2) * Q; };
+  auto recB = [&](int slot) { return recb + (slot * 2 + 1) * Q; };
+  auto scal = [&](int slot) { return scalb + slot * 8; };
+  auto cs = [&](int slot) { return csb + slot * Q * K2; };
 
   const __nv_bfloat16* xg = static_cast<const __nv_bfloat16*>(p.x);
   const __nv_bfloat16* Bg = static_cast<const __nv_bfloat16*>(p.B);
   __nv_bfloat16* yg = static_cast<__nv_bfloat16*>(p.y);
   const float Dh = (FULL && p.D) ? p.D[hi] : 0.0f;
 
-  // ---- issue the TMA loads of tile j (thread 0); B/C boxes: 64 columns x R x 1 x Q tokens
-  auto issue_loads = [&](int64_t j) {
+  // ---- TMA loads of tile j (thread 0): x first (with the byte count of all), then B, C
+  auto issue_x = [&](int64_t j) {
     const int tok = (int)(tok_base + j * Q);
-    constexpr uint32_t tx = C::TX_B * (FULL ? 2 : 1) + (C::TX_X) + C::TX_T;
+    constexpr uint32_t tx = C::TX_B * (FULL ? 2 : 1) + C::TX_X;
     mbar_expect_tx(load_bar, tx);
+    tma_load_3d(sXSTG, &tmX, 0, hi, tok, load_bar);
+  };
+  auto issue_bc = [&](int64_t j) {
+    const int tok = (int)(tok_base + j * Q);
 #pragma unroll
     for (int blk = 0; blk < N / 64; ++blk) {
       tma_load_4d(sBT + blk * (kRows * 128), &tmB, 64 * blk, 0, g, tok, load_bar);
       if constexpr (FULL) tma_load_4d(sCT + blk * (kRows * 128), &tmC, 64 * blk, 0, g, tok, load_bar);
     }
-    tma_load_3d(sXSTG, &tmX, 0, hi, tok, load_bar);
-    tma_load_3d(sTH, &tmT, 0, g, tok, load_bar);
   };
-  // per-token coefficient loads (registers), tile j: threads t < Q; thread Q loads the
-  // first token after tile j (its beta' is the carry weight of the tile's last token)
+
+  // ---- per-token coefficients and rotation angles, one tile ahead, through registers
+  const int ak = tid % K2, aseg = tid / K2;
   float r_dt = 0.f, r_a = 0.f, r_lm = 0.f;
+  float r_th[C::SEGLEN];
   auto load_coefs = [&](int64_t j) {
     const int64_t c0 = j * Q;
     if (tid < Q) {
@@ -385,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
         r_lm = p.lam[ti];
       }
     } else if (tid == Q) {
-      const int64_t t = c0 + Q;
+      const int64_t t = c0 + Q;  // first token after the tile: its beta' weights the tile's last token
       r_dt = r_lm = 0.0f;
       if (t < L) {
         const int64_t ti = (tok_base + t) * H + hi;
@@ -393,14 +392,126 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
         r_lm = p.lam[ti];
       }
     }
+#pragma unroll
+    for (int e = 0; e < C::SEGLEN; ++e) {
+      const int t = aseg * C::SEGLEN + e;
+      r_th[e] = (t < Q && c0 + t < L) ? p.theta[((tok_base + c0 + t) * G + g) * K2 + ak] : 0.0f;
+    }
   };
-  auto store_coefs = [&](int par) {
+  auto store_coefs = [&](int slot) {
     if (tid < Q) {
-      tokf[(A_DT0 + 3 * par) * C::TOKF + tid] = r_dt;
-      tokf[(A_A0 + 3 * par) * C::TOKF + tid] = r_a;
-      tokf[(A_LM0 + 3 * par) * C::TOKF + tid] = r_lm;
+      rawA(slot, 0)[tid] = r_dt;
+      rawA(slot, 1)[tid] = r_a;
+      rawA(slot, 2)[tid] = r_lm;
     } else if (tid == Q) {
-      scal[2 + par] = (1.0f - r_lm) * r_dt;
+      rawA(slot, 3)[0] = (1.0f - r_lm) * r_dt;
+    }
+  };
+  // coefficients, records and the rotation table of tile j into slot `slot` (all threads;
+  // the raw values of the tile must be in raw slot `slot` and r_th)
+  auto tile_prep = [&](int64_t j, int slot) {
+    const int nv = (int)((L - j * Q) < Q ? (L - j * Q) : Q);
+    const float* dtA = rawA(slot, 0);
+    const float* aA = rawA(slot, 1);
+    const float* lmA = rawA(slot, 2);
+    if (warp == 0) {
+      constexpr int PER = (Q + 31) / 32;
+      float loc[PER];
+      float run = 0.0f;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) {
+        const int t = lane * PER + e;
+        run += (t < nv) ? dtA[t] * aA[t] : 0.0f;
+        loc[e] = run;
+      }
+      float incl = run;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float nbv = __shfl_up_sync(kFull, incl, off);
+        if (lane >= off) incl += nbv;
+      }
+      const float Le = __shfl_sync(kFull, incl, 31);
+      const float excl = incl - run;
+      float lmin = 0.0f, lmax = 0.0f;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) {
+        loc[e] += excl;
+        lmin = fminf(lmin, loc[e]);
+        lmax = fmaxf(lmax, loc[e]);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        lmin = fminf(lmin, __shfl_xor_sync(kFull, lmin, off));
+        lmax = fmaxf(lmax, __shfl_xor_sync(kFull, lmax, off));
+      }
+      const bool fast = (lmax - lmin) <= 160.0f;
+      const float m = fast ? 0.5f * (lmax + lmin) : 0.0f;
+      const float bp_after = rawA(slot, 3)[0];
+      float4* ra = recA(slot);
+      float4* rb = recB(slot);
+#pragma unroll
+      for (int e = 0; e < PER; ++e) {
+        const int t = lane * PER + e;
+        if (t < Q) {
+          const float Lct = loc[e];
+          const bool valid = t < nv;
+          const float gm = valid ? lmA[t] * dtA[t] : 0.0f;
+          const float bpn = (t + 1 < Q) ? ((t + 1 < nv) ? (1.0f - lmA[t + 1]) * dtA[t + 1] : 0.0f)
+                                        : (valid ? bp_after : 0.0f);
+          const float w = gm + bpn;
+          const float dg = (w > 0.0f) ? gm / w : 0.0f;
+          const float at = fast ? __expf(Lct - m) : 1.0f;
+          const float xs = fast ? __expf(m - Lct) * w : w;
+          ra[t] = make_float4(Lct * 1.4426950408889634f, dg, at, xs);
+          rb[t] = make_float4(__expf(Lct), __expf(Le - Lct), 0.0f, 0.0f);
+        }
+      }
+      if (lane == 0) {
+        float* sc = scal(slot);
+        sc[0] = __expf(Le);
+        sc[1] = Le;
+        sc[2] = fast ? __expf(Le - m) : 1.0f;
+        sc[3] = fast ? 1.0f : 0.0f;
+        sc[4] = fast ? __expf(m) : 1.0f;
+      }
+    }
+    float aloc[C::SEGLEN];
+    {
+      float run = 0.0f;
+#pragma unroll
+      for (int e = 0; e < C::SEGLEN; ++e) {
+        const int t = aseg * C::SEGLEN + e;
+        if (t < Q) run += (t < nv) ? dtA[t] * r_th[e] : 0.0f;
+        aloc[e] = run;
+      }
+      segsum[aseg * K2 + ak] = run;
+    }
+    __syncthreads();
+    double total = 0.0;
+    {
+      float aoff = 0.0f;
+      for (int s = 0; s < C::SEGS; ++s) {
+        const float v = segsum[s * K2 + ak];
+        if (s < aseg) aoff += v;
+        total += (double)v;
+      }
+      aoff += (float)base[ak];
+      float2* c2 = cs(slot);
+#pragma unroll
+      for (int e = 0; e < C::SEGLEN; ++e) {
+        const int t = aseg * C::SEGLEN + e;
+        if (t < Q) {
+          float sn, cn;
+          sincos_reduced(aoff + aloc[e], &sn, &cn);
+          c2[t * K2 + ak] = make_float2(cn, sn);
+        }
+      }
+    }
+    __syncthreads();  // every thread has read base[] and segsum[]
+    if (aseg == 0) {
+      double nb = base[ak] + total;
+      nb -= 6.283185307179586 * rint(nb * 0.15915494309189535);
+      base[ak] = nb;
     }
   };
 
@@ -416,7 +527,6 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
     prefetch_tmap(&tmB);
     if constexpr (FULL) prefetch_tmap(&tmC);
     prefetch_tmap(&tmX);
-    prefetch_tmap(&tmT);
   }
   for (int i = tid; i < R * P; i += kThreads) {
     wx[i] = p.W_x ? p.W_x[(int64_t)hi * R * P + i] : 1.0f;
@@ -427,12 +537,16 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
   for (int k = tid; k < K2; k += kThreads) base[k] = 0.0;
   load_coefs(j0);
   store_coefs(0);
-  if (j0 + 1 < j1) load_coefs(j0 + 1);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (tid == 0 && j0 < j1) issue_loads(j0);
+  if (tid == 0 && j0 < j1) {
+    issue_x(j0);
+    issue_bc(j0);
+  }
+  if (j0 < j1) tile_prep(j0, 0);
+  if (j0 + 1 < j1) load_coefs(j0 + 1);
 
   // state warps: TMEM lane of accumulator row p (M = 128: lane = p; M = 64: rows in lanes
   // 0-15 of each quarter, and the state is kept in lanes 16-31 of the same columns)
@@ -442,24 +556,27 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
   const int prow = (P == 128) ? (32 * q4 + lane) : (16 * q4 + (lane & 15));
   const bool st_owner = (P == 128) || (lane >= 16);  // holds the fp32 state of row prow
 
-  // transform thread mapping: fixed 16-byte column chunk and MIMO branch per thread
+  // operand staging threads (FULL: warps 4-7, while warps 0-3 run the previous epilogue)
+  const bool xf_thread = FULL ? (tid >= 128) : true;
+  const int xt = FULL ? tid - 128 : tid;
   constexpr int CHN = N / 8;
-  constexpr int ROWS_PER_IT = kThreads / CHN;
-  const int tch = tid % CHN;
-  const int tr = (tid / CHN) % R;  // fixed: ROWS_PER_IT is a multiple of R
+  constexpr int RPI = NT / CHN;  // rows per pass; a multiple of 8 and of R
+  const int tch = xt % CHN;
+  const int tr = (xt / CHN) % R;
   float bB[8], bC[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
-    bB[e] = biasBg ? __ldg(biasBg + tr * N + tch * 8 + e) : 0.0f;
-    bC[e] = biasCg ? __ldg(biasCg + tr * N + tch * 8 + e) : 0.0f;
+    bB[e] = (xf_thread && biasBg) ? __ldg(biasBg + tr * N + tch * 8 + e) : 0.0f;
+    bC[e] = (xf_thread && biasCg) ? __ldg(biasCg + tr * N + tch * 8 + e) : 0.0f;
   }
 
   // ---- incoming rotated-frame state h+ of this segment
   //   nseg == 1 (full pass): h_{-1} + beta'_0 u_{-1} from the state / carry;
   //   state pass, segment 0: same, written to ws_init; other state-pass segments: zero;
   //   full pass, segment k > 0: ws_init folded through the summaries of segments 0..k-1.
-  if (state_warp) {
+  if (state_warp && j0 < j1) {
     const bool from_state = (sg.nseg == 1) || (!FULL && seg == 0);
+    const float hscale = scal(0)[4];  // e^m of the first tile: the bf16 copy is pre-scaled
     float xprev[R];
     float bp0 = 0.0f;
     if (from_state) {
@@ -520,7 +637,7 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
           for (int q = 0; q < 4; ++q) {
             float f[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = v[8 * q + e];
+            for (int e = 0; e < 8; ++e) f[e] = hscale * v[8 * q + e];
             sts128(sH + sw128(prow, 4 * c + q, P * 128), pack8(f));
           }
         }
@@ -533,8 +650,8 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
   __syncthreads();
   tc_fence_after();
 
-  // state update ST <- e^{Le} ST + hs * H for this thread's TMEM row (state warps)
-  auto state_update = [&](float Le_exp, float hs, bool write_bf16) {
+  // state update ST <- e^{Le} ST + hs * H; with hnext > 0 also the bf16 copy hnext * ST
+  auto state_update = [&](float Le_exp, float hs, float hnext) {
 #pragma unroll 1
     for (int c = 0; c < N / 32; ++c) {
       uint32_t hv[32];
@@ -561,33 +678,75 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
         }
         tmem_st32(tmem + lane_base + C::TM_ST + 32 * c, sv);
       }
-      if (write_bf16 && st_owner) {
+      if (FULL && hnext > 0.0f && st_owner) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           float f8[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f8[e] = f[8 * q + e];
+          for (int e = 0; e < 8; ++e) f8[e] = hnext * f[8 * q + e];
           sts128(sH + sw128(prow, 4 * c + q, P * 128), pack8(f8));
         }
       }
     }
     tmem_wait_st();
   };
-  // refresh the bf16 copy of the state from TMEM (state warps)
-  auto write_state_bf16 = [&]() {
+
+  // epilogue of tile j (warps 0-3): y_t = sum_r W_o[r] * a_t Y_{t,r} + D x_t
+  auto epilogue = [&](int64_t j, int slot) {
+    const int64_t c0 = j * Q;
+    const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
+    const int i = 32 * q4 + lane;
+    const int t = i / R, r = i % R;
+    constexpr int W = 16 / R;
+    const float at = recA(slot)[t].z;
+    const int64_t yrow = ((tok_base + c0 + t) * H + hi) * P;
 #pragma unroll 1
-    for (int c = 0; c < N / 32; ++c) {
-      uint32_t sv[32];
-      tmem_ld32(tmem + lane_base + C::TM_ST + 32 * c, sv);
+    for (int c = 0; c < P / 16; ++c) {
+      const int col0 = 16 * c;
+      uint32_t v[16];
+      tmem_ld16(tmem + lane_base + C::TM_Y + col0, v);
       tmem_wait_ld();
-      if (st_owner) {
+      float f[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float f8[8];
+      for (int e4 = 0; e4 < 4; ++e4) {
+        const float4 w4 = *reinterpret_cast<const float4*>(&wo[r * P + col0 + 4 * e4]);
+        f[4 * e4] = at * w4.x * __uint_as_float(v[4 * e4]);
+        f[4 * e4 + 1] = at * w4.y * __uint_as_float(v[4 * e4 + 1]);
+        f[4 * e4 + 2] = at * w4.z * __uint_as_float(v[4 * e4 + 2]);
+        f[4 * e4 + 3] = at * w4.w * __uint_as_float(v[4 * e4 + 3]);
+      }
+      // reduce over the R branches (adjacent lanes); lane r keeps columns [r*W, r*W + W)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f8[e] = __uint_as_float(sv[8 * q + e]);
-          sts128(sH + sw128(prow, 4 * c + q, P * 128), pack8(f8));
+      for (int m = R / 2; m >= 1; m >>= 1) {
+        const bool upper = (r & m) != 0;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          if ((e / W) % (2 * m) < m) {
+            const float mine = upper ? f[e + m * W] : f[e];
+            const float other = upper ? f[e] : f[e + m * W];
+            const float got = __shfl_xor_sync(kFull, other, m);
+            if (upper) f[e + m * W] = mine + got; else f[e] = mine + got;
+          }
         }
+      }
+      if (t < nv) {
+        float outv[W];
+#pragma unroll
+        for (int e = 0; e < W; ++e) {
+          float sel = f[e];
+#pragma unroll
+          for (int rr = 1; rr < R; ++rr)
+            if (rr == r) sel = f[rr * W + e];
+          outv[e] = sel;
+        }
+        const int pc = col0 + r * W;
+        if (p.D) {
+#pragma unroll
+          for (int e = 0; e < W; ++e) outv[e] = fmaf(Dh, __bfloat162float(xg[yrow + pc + e]), outv[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < W; e += 2)
+          *reinterpret_cast<uint32_t*>(yg + yrow + pc + e) = pack_bf16(outv[e], outv[e + 1]);
       }
     }
   };
@@ -599,203 +758,93 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
     const int64_t c0 = j * Q;
     const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
     const int par = (int)((j - j0) & 1);
-    const float* dtA = tokf + (A_DT0 + 3 * par) * C::TOKF;
-    const float* aA = tokf + (A_A0 + 3 * par) * C::TOKF;
-    const float* lmA = tokf + (A_LM0 + 3 * par) * C::TOKF;
+    const bool has_next = j + 1 < j1;
 
-    // ---- wait for this tile's TMA loads
-    {
-      const bool ok = mbar_wait(load_bar, load_phase);
-      load_phase ^= 1;
-      if (__syncthreads_or(!ok)) {
-        failed = true;
-        break;
-      }
-    }
-
-    // ---- A: coefficients (warp 0), angle prefixes (all threads)
-    if (warp == 0) {
-      constexpr int PER = (Q + 31) / 32;
-      float loc[PER];
-      float run = 0.0f;
-#pragma unroll
-      for (int e = 0; e < PER; ++e) {
-        const int t = lane * PER + e;
-        run += (t < nv) ? dtA[t] * aA[t] : 0.0f;
-        loc[e] = run;
-      }
-      float incl = run;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const float nbv = __shfl_up_sync(kFull, incl, off);
-        if (lane >= off) incl += nbv;
-      }
-      const float Le = __shfl_sync(kFull, incl, 31);
-      const float excl = incl - run;
-      float lmin = 0.0f, lmax = 0.0f;
-#pragma unroll
-      for (int e = 0; e < PER; ++e) {
-        loc[e] += excl;
-        lmin = fminf(lmin, loc[e]);
-        lmax = fmaxf(lmax, loc[e]);
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        lmin = fminf(lmin, __shfl_xor_sync(kFull, lmin, off));
-        lmax = fmaxf(lmax, __shfl_xor_sync(kFull, lmax, off));
-      }
-      const bool fast = (lmax - lmin) <= 160.0f;
-      const float m = fast ? 0.5f * (lmax + lmin) : 0.0f;
-#pragma unroll
-      for (int e = 0; e < PER; ++e) {
-        const int t = lane * PER + e;
-        if (t < Q) {
-          const float Lct = loc[e];
-          const bool valid = t < nv;
-          const float gm = valid ? lmA[t] * dtA[t] : 0.0f;
-          const float bpn = (t + 1 < Q) ? ((t + 1 < nv) ? (1.0f - lmA[t + 1]) * dtA[t + 1] : 0.0f)
-                                        : (valid ? scal[2 + par] : 0.0f);
-          const float w = gm + bpn;
-          const float dg = (w > 0.0f) ? gm / w : 0.0f;
-          const float at = fast ? __expf(Lct - m) : 1.0f;
-          const float xs = fast ? __expf(m - Lct) * w : w;
-          const float dect = __expf(Lct);
-          recA[t] = make_float4(Lct * 1.4426950408889634f, dg, at, xs);
-          recB[t] = make_float4(fast ? __expf(m) : dect, dect, __expf(Le - Lct), 0.0f);
-        }
-      }
-      if (lane == 0) {
-        scal[0] = __expf(Le);
-        scal[1] = Le;
-        scal[4] = fast ? __expf(Le - m) : 1.0f;
-        scal[5] = fast ? 1.0f : 0.0f;
-      }
-    }
-    const int ak = tid % K2, aseg = tid / K2;
-    float aloc[C::SEGLEN];
-    double ang_total = 0.0;
-    {
-      float run = 0.0f;
-#pragma unroll
-      for (int e = 0; e < C::SEGLEN; ++e) {
-        const int t = aseg * C::SEGLEN + e;
-        if (t < Q) run += (t < nv) ? dtA[t] * th_stg[t * K2 + ak] : 0.0f;
-        aloc[e] = run;
-      }
-      segsum[aseg * K2 + ak] = run;
-    }
-    __syncthreads();
-    const bool fast = scal[5] != 0.0f;
-    {
-      double total = 0.0;
-      float aoff = 0.0f;
-      for (int s = 0; s < C::SEGS; ++s) {
-        const float v = segsum[s * K2 + ak];
-        if (s < aseg) aoff += v;
-        total += (double)v;
-      }
-      aoff += (float)base[ak];
-      // theta staging (2nd half of cs) is consumed: every thread read its values above
-#pragma unroll
-      for (int e = 0; e < C::SEGLEN; ++e) {
-        const int t = aseg * C::SEGLEN + e;
-        if (t < Q) {
-          float sn, cn;
-          sincos_reduced(aoff + aloc[e], &sn, &cn);
-          cs[t * K2 + ak] = make_float2(cn, sn);
-        }
-      }
-      ang_total = total;
-    }
-    if (tid == 0) seg_logdec += scal[1];
-    __syncthreads();
-    // every thread has read base[]: advance it by this tile's total angle
-    if (aseg == 0) {
-      double nb = base[ak] + ang_total;
-      nb -= 6.283185307179586 * rint(nb * 0.15915494309189535);
-      base[ak] = nb;
-    }
-
-    // ---- B: rotate B (and C) in place; build X' = b_t w_t W_x x (and the scaled C copy)
-    {
-      const int i0 = tid / CHN;
-      const uint32_t off0 = (uint32_t)(tch >> 3) * (kRows * 128) + (uint32_t)i0 * 128u +
-                            ((uint32_t)((tch & 7) ^ (i0 & 7)) << 4);  // row i0 + k*ROWS_PER_IT keeps i & 7
+    // ---- X: stage tile j (staging threads) | epilogue of tile j-1 (warps 0-3)
+    bool bad = false;
+    if (xf_thread) {
+      bad = !mbar_wait(load_bar, load_phase);
+      if (!bad) {
+        const bool fast = scal(par)[3] != 0.0f;
+        const float2* csj = cs(par);
+        const float4* raj = recA(par);
+        const float4* rbj = recB(par);
+        const int i0 = xt / CHN;
+        const uint32_t off0 = (uint32_t)(tch >> 3) * (kRows * 128) + (uint32_t)i0 * 128u +
+                              ((uint32_t)((tch & 7) ^ (i0 & 7)) << 4);  // i0 + k*RPI keeps i & 7
 #pragma unroll 2
-      for (int it = 0; it < kRows / ROWS_PER_IT; ++it) {
-        const int i = i0 + it * ROWS_PER_IT;
-        const int t = i / R;
-        const uint32_t off = off0 + (uint32_t)(it * ROWS_PER_IT) * 128u;
-        const float4 w01 = *reinterpret_cast<const float4*>(&cs[t * K2 + tch * 4]);
-        const float4 w23 = *reinterpret_cast<const float4*>(&cs[t * K2 + tch * 4 + 2]);
-        const float wc[4] = {w01.x, w01.z, w23.x, w23.z};
-        const float ws[4] = {w01.y, w01.w, w23.y, w23.w};
-        if (t < nv) {
-          float bsc = 1.0f;
-          if constexpr (!FULL) bsc = fast ? 1.0f : recB[t].z;  // exact tiles: Bt rows * e^{Le - Lc_t}
-          {
-            float f[8];
-            unpack8(lds128(sBT + off), f);
+        for (int it = 0; it < kRows / RPI; ++it) {
+          const int i = i0 + it * RPI;
+          const int t = i / R;
+          const uint32_t off = off0 + (uint32_t)(it * RPI) * 128u;
+          if (t < nv) {
+            const float4 w01 = *reinterpret_cast<const float4*>(&csj[t * K2 + tch * 4]);
+            const float4 w23 = *reinterpret_cast<const float4*>(&csj[t * K2 + tch * 4 + 2]);
+            const float wc[4] = {w01.x, w01.z, w23.x, w23.z};
+            const float ws[4] = {w01.y, w01.w, w23.y, w23.w};
+            const float bsc = (!FULL && !fast) ? rbj[t].y : 1.0f;  // state pass, exact tile
+            {
+              float f[8];
+              unpack8(lds128(sBT + off), f);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const float b0 = f[2 * q] + bB[2 * q], b1 = f[2 * q + 1] + bB[2 * q + 1];
-              f[2 * q] = bsc * (wc[q] * b0 + ws[q] * b1);  // Rot(-Phi)
-              f[2 * q + 1] = bsc * (wc[q] * b1 - ws[q] * b0);
+              for (int q = 0; q < 4; ++q) {
+                const float b0 = f[2 * q] + bB[2 * q], b1 = f[2 * q + 1] + bB[2 * q + 1];
+                f[2 * q] = bsc * (wc[q] * b0 + ws[q] * b1);  // Rot(-Phi)
+                f[2 * q + 1] = bsc * (wc[q] * b1 - ws[q] * b0);
+              }
+              sts128(sBT + off, pack8(f));
             }
-            sts128(sBT + off, pack8(f));
+            if constexpr (FULL) {
+              float f[8];
+              unpack8(lds128(sCT + off), f);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const float d0 = f[2 * q] + bC[2 * q], d1 = f[2 * q + 1] + bC[2 * q + 1];
+                f[2 * q] = wc[q] * d0 + ws[q] * d1;
+                f[2 * q + 1] = wc[q] * d1 - ws[q] * d0;
+              }
+              sts128(sCT + off, pack8(f));
+            }
+          } else {
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            sts128(sBT + off, z);
+            if constexpr (FULL) sts128(sCT + off, z);
           }
-          if constexpr (FULL) {
-            float f[8];
-            unpack8(lds128(sCT + off), f);
+        }
+        constexpr int CHP = P / 8;
+        const int xch = xt % CHP;  // fixed column chunk
+        for (int t = xt / CHP; t < Q; t += NT / CHP) {
+          float fx[8];
+          unpack8(lds128(sXSTG + (uint32_t)(t * P + xch * 8) * 2), fx);
+          const float xs = (t < nv) ? raj[t].w : 0.0f;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const float d0 = f[2 * q] + bC[2 * q], d1 = f[2 * q + 1] + bC[2 * q + 1];
-              f[2 * q] = wc[q] * d0 + ws[q] * d1;
-              f[2 * q + 1] = wc[q] * d1 - ws[q] * d0;
-            }
-            sts128(sCT + off, pack8(f));
-            if constexpr (!C::kInterInS) {
-              const float dd = recB[t].x;
+          for (int e = 0; e < 8; ++e) fx[e] *= xs;
 #pragma unroll
-              for (int e = 0; e < 8; ++e) f[e] *= dd;
-              sts128(sC2 + off, pack8(f));
-            }
-          }
-        } else {
-          const uint4 z = make_uint4(0, 0, 0, 0);
-          sts128(sBT + off, z);
-          if constexpr (FULL) {
-            sts128(sCT + off, z);
-            if constexpr (!C::kInterInS) sts128(sC2 + off, z);
+          for (int rr = 0; rr < R; ++rr) {
+            const int i = t * R + rr;
+            const float4 w0 = *reinterpret_cast<const float4*>(&wx[rr * P + xch * 8]);
+            const float4 w1 = *reinterpret_cast<const float4*>(&wx[rr * P + xch * 8 + 4]);
+            const float xr[8] = {fx[0] * w0.x, fx[1] * w0.y, fx[2] * w0.z, fx[3] * w0.w,
+                                 fx[4] * w1.x, fx[5] * w1.y, fx[6] * w1.z, fx[7] * w1.w};
+            sts128(sX + sw128(i, xch, kRows * 128), pack8(xr));
           }
         }
       }
-      constexpr int CHP = P / 8;
-      const int xch = tid % CHP;  // fixed column chunk
-      for (int t = tid / CHP; t < Q; t += kThreads / CHP) {
-        float fx[8];
-        unpack8(lds128(sXSTG + (uint32_t)(t * P + xch * 8) * 2), fx);
-        const float xs = (t < nv) ? recA[t].w : 0.0f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) fx[e] *= xs;
-#pragma unroll
-        for (int rr = 0; rr < R; ++rr) {
-          const int i = t * R + rr;
-          const float4 w0 = *reinterpret_cast<const float4*>(&wx[rr * P + xch * 8]);
-          const float4 w1 = *reinterpret_cast<const float4*>(&wx[rr * P + xch * 8 + 4]);
-          const float xr[8] = {fx[0] * w0.x, fx[1] * w0.y, fx[2] * w0.z, fx[3] * w0.w,
-                               fx[4] * w1.x, fx[5] * w1.y, fx[6] * w1.z, fx[7] * w1.w};
-          sts128(sX + sw128(i, xch, kRows * 128), pack8(xr));
-        }
-      }
+    } else if (FULL && j > j0) {
+      epilogue(j - 1, par ^ 1);
     }
+    load_phase ^= 1;
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
+    if (__syncthreads_or(bad)) {
+      failed = true;
+      break;
+    }
     tc_fence_after();
+    const bool fast = scal(par)[3] != 0.0f;
+    if (tid == 0 && has_next) issue_x(j + 1);  // x staging is consumed
 
-    // ---- C: MMA1 (S), [MMA3 without kInterInS], MMA4 (H = X'^T Bt) unless the tile is exact
-    const bool mma4_early = !FULL || fast;
+    // ---- MMA_A: S = Ct Bt^T; fast tiles also Y = Ct (e^m h+) and H = X'^T Bt
     if (tid == 0) {
       if constexpr (FULL) {
 #pragma unroll
@@ -803,16 +852,16 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
           const uint32_t koff = (uint32_t)(k >> 2) * (kRows * 128) + (uint32_t)(k & 3) * 32;
           mma_ss(tmem + C::TM_S, sdesc(sCT + koff, 16, 1024), sdesc(sBT + koff, 16, 1024), C::ID_S, k > 0);
         }
-        if constexpr (!C::kInterInS) {
+        if (fast) {
 #pragma unroll
           for (int k = 0; k < N / 16; ++k) {
             const uint32_t aoff2 = (uint32_t)(k >> 2) * (kRows * 128) + (uint32_t)(k & 3) * 32;
             const uint32_t boff = (uint32_t)(k >> 2) * (P * 128) + (uint32_t)(k & 3) * 32;
-            mma_ss(tmem + C::TM_Y, sdesc(sC2 + aoff2, 16, 1024), sdesc(sH + boff, 16, 1024), C::ID_Y3, k > 0);
+            mma_ss(tmem + C::TM_Y, sdesc(sCT + aoff2, 16, 1024), sdesc(sH + boff, 16, 1024), C::ID_Y3, k > 0);
           }
         }
       }
-      if (mma4_early) {
+      if (!FULL || fast) {
 #pragma unroll
         for (int k = 0; k < kRows / 16; ++k)
           mma_ss(tmem + C::TM_H, sdesc(sX + k * 2048, kRows * 128, 1024), sdesc(sBT + k * 2048, kRows * 128, 1024),
@@ -820,11 +869,17 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
       }
       mma_commit(mma_bar);
     }
-    // next tile's per-token coefficients: registers -> smem slot, then start loading the one after
-    if (j + 1 < j1) store_coefs(par ^ 1);
-    if (j + 2 < j1) load_coefs(j + 2);
+    // while the tensor cores run: next tile's coefficients and rotation table
+    if (has_next) {
+      store_coefs(par ^ 1);
+      __syncthreads();
+      tile_prep(j + 1, par ^ 1);
+      if (j + 2 < j1) load_coefs(j + 2);
+    }
+    if (tid == 0 && !FULL) seg_logdec += scal(par)[1];
     {
-      const bool ok = mbar_wait(mma_bar, mma_phase);
+      bool ok = true;
+      if (tid == 0) ok = mbar_wait(mma_bar, mma_phase);
       mma_phase ^= 1;
       if (__syncthreads_or(!ok)) {
         failed = true;
@@ -832,17 +887,17 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
       }
     }
     tc_fence_after();
-    // operand buffers no later MMA of this tile reads: the next tile's loads may land now
-    const bool prefetch_early = !FULL || (!C::kInterInS && fast);
-    if (tid == 0 && prefetch_early && j + 1 < j1) issue_loads(j + 1);
+    const float hnext = has_next ? scal(par ^ 1)[4] : 0.0f;  // bf16 state copy scale of tile j+1
+    if (tid == 0 && has_next && (!FULL || fast)) issue_bc(j + 1);  // B (and C) are consumed
 
-    // ---- D: mask S in TMEM (warps 0-3) | state update (warps 4-7)
-    if (!state_warp) {
-      if constexpr (FULL) {
+    // ---- D: mask S (warps 0-3) | state update or exact-tile rescaling (warps 4-7)
+    if constexpr (FULL) {
+      if (!state_warp) {
         const int i = 32 * warp + lane;
         const int t = i / R;
         const int t_lo = (32 * warp) / R, t_hi = (32 * warp + 31) / R;
-        const float4 ra = recA[t];
+        const float4* raj = recA(par);
+        const float Lt2 = raj[t].x;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           const int s_lo = (32 * c) / R, s_hi = (32 * c + 31) / R;
@@ -862,9 +917,9 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
 #pragma unroll
               for (int jj = 0; jj < 32 / R; ++jj) {
                 const int s = s_lo + jj;
-                const float4 rs = recA[s];
+                const float4 rs = raj[s];
                 float fac = (s < t) ? 1.0f : ((s == t) ? rs.y : 0.0f);
-                if (!fast && s <= t) fac *= ex2_approx(ra.x - rs.x);
+                if (!fast && s <= t) fac *= ex2_approx(Lt2 - rs.x);
 #pragma unroll
                 for (int rr = 0; rr < R; ++rr) f[jj * R + rr] = fac * __uint_as_float(v[jj * R + rr]);
               }
@@ -875,143 +930,80 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
           tmem_st16(tmem + lane_base + C::TM_S + 16 * c, o);
         }
         tmem_wait_st();
-      }
-    } else if (mma4_early) {
-      state_update(scal[0], scal[4], FULL && !C::kInterInS);
-    } else {
-      // exact tile: scale Bt rows by e^{Le - Lc_t} in place (MMA1 has read Bt) for MMA4
-      const int lt = tid - 128;
+      } else if (fast) {
+        state_update(scal(par)[0], scal(par)[2], hnext);
+      } else {
+        // exact tile: Ct rows * e^{Lc_t} and Bt rows * e^{Le - Lc_t}, in place (MMA1 has read them)
+        const float4* rbj = recB(par);
+        const int lt = tid - 128;
 #pragma unroll 1
-      for (int idx = lt; idx < kRows * CHN; idx += 128) {
-        const int i = idx / CHN, ch = idx % CHN;
-        const uint32_t off = sw128(i, ch, kRows * 128);
-        const float sc = recB[i / R].z;
-        float f[8];
-        unpack8(lds128(sBT + off), f);
+        for (int idx = lt; idx < kRows * CHN; idx += 128) {
+          const int i = idx / CHN, ch = idx % CHN;
+          const uint32_t off = sw128(i, ch, kRows * 128);
+          const float4 rb = rbj[i / R];
+          float f[8];
+          unpack8(lds128(sBT + off), f);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] *= sc;
-        sts128(sBT + off, pack8(f));
+          for (int e = 0; e < 8; ++e) f[e] *= rb.y;
+          sts128(sBT + off, pack8(f));
+          unpack8(lds128(sCT + off), f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] *= rb.x;
+          sts128(sCT + off, pack8(f));
+        }
       }
+    } else {
+      if (state_warp) state_update(scal(par)[0], scal(par)[2], 0.0f);
     }
-    if constexpr (FULL) {
-      fence_async_smem();
-      tc_fence_before();
-      __syncthreads();
-      tc_fence_after();
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
 
-      // ---- E: [MMA3 with kInterInS], MMA2 (Y += S' X'), [MMA4 for exact tiles]
+    if constexpr (FULL) {
+      // ---- MMA_B: [exact: Y = Ct' h+], Y += S' X', [exact: H = X'^T Bt']
+      bool ok = true;
       if (tid == 0) {
-        if constexpr (C::kInterInS) {
+        if (!fast) {
 #pragma unroll
           for (int k = 0; k < N / 16; ++k) {
             const uint32_t aoff2 = (uint32_t)(k >> 2) * (kRows * 128) + (uint32_t)(k & 3) * 32;
             const uint32_t boff = (uint32_t)(k >> 2) * (P * 128) + (uint32_t)(k & 3) * 32;
-            mma_ss(tmem + C::TM_YI, sdesc(sCT + aoff2, 16, 1024), sdesc(sH + boff, 16, 1024), C::ID_Y3, k > 0);
+            mma_ss(tmem + C::TM_Y, sdesc(sCT + aoff2, 16, 1024), sdesc(sH + boff, 16, 1024), C::ID_Y3, k > 0);
           }
         }
 #pragma unroll
         for (int k = 0; k < kRows / 16; ++k)
-          mma_ts(tmem + C::TM_Y, tmem + C::TM_S + 8 * k, sdesc(sX + k * 2048, kRows * 128, 1024), C::ID_Y2,
-                 C::kInterInS ? (k > 0) : 1);  // without kInterInS, Y already holds the Ct h+ term
-        if (!mma4_early) {
+          mma_ts(tmem + C::TM_Y, tmem + C::TM_S + 8 * k, sdesc(sX + k * 2048, kRows * 128, 1024), C::ID_Y2, 1);
+        if (!fast) {
 #pragma unroll
           for (int k = 0; k < kRows / 16; ++k)
             mma_ss(tmem + C::TM_H, sdesc(sX + k * 2048, kRows * 128, 1024),
                    sdesc(sBT + k * 2048, kRows * 128, 1024), C::ID_H, k > 0);
         }
         mma_commit(mma_bar);
+        ok = mbar_wait(mma_bar, mma_phase);
       }
-      {
-        const bool ok = mbar_wait(mma_bar, mma_phase);
-        mma_phase ^= 1;
-        if (__syncthreads_or(!ok)) {
-          failed = true;
-          break;
-        }
+      mma_phase ^= 1;
+      if (__syncthreads_or(!ok)) {
+        failed = true;
+        break;
       }
       tc_fence_after();
-      if (tid == 0 && !prefetch_early && j + 1 < j1) issue_loads(j + 1);
-
-      // ---- F: epilogue y_t = sum_r W_o[r] * (a_t Y [+ e^{Lc_t} Yi])_{t,r} + D x_t
-      {
-        const int i = 32 * q4 + lane;
-        const int t = i / R, r = i % R;
-        const int half = warp >> 2;
-        constexpr int PH = P / 2;
-        constexpr int W = 16 / R;
-        const float at = recA[t].z;
-        const float dect = recB[t].y;
-        const int64_t yrow = ((tok_base + c0 + t) * H + hi) * P;
-#pragma unroll 1
-        for (int c = 0; c < PH / 16; ++c) {
-          const int col0 = half * PH + 16 * c;
-          uint32_t v[16];
-          tmem_ld16(tmem + lane_base + C::TM_Y + col0, v);
-          float f[16];
-          if constexpr (C::kInterInS) {
-            uint32_t vi[16];
-            tmem_ld16(tmem + lane_base + C::TM_YI + col0, vi);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) f[e] = fmaf(dect, __uint_as_float(vi[e]), at * __uint_as_float(v[e]));
-          } else {
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) f[e] = at * __uint_as_float(v[e]);
-          }
-#pragma unroll
-          for (int e4 = 0; e4 < 4; ++e4) {
-            const float4 w4 = *reinterpret_cast<const float4*>(&wo[r * P + col0 + 4 * e4]);
-            f[4 * e4] *= w4.x;
-            f[4 * e4 + 1] *= w4.y;
-            f[4 * e4 + 2] *= w4.z;
-            f[4 * e4 + 3] *= w4.w;
-          }
-          // reduce over the R branches (adjacent lanes); lane r keeps columns [r*W, r*W + W)
-#pragma unroll
-          for (int m = R / 2; m >= 1; m >>= 1) {
-            const bool upper = (r & m) != 0;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              // pair columns that differ in the bit of value m*W within the remaining span
-              if ((e / W) % (2 * m) < m) {
-                const float mine = upper ? f[e + m * W] : f[e];
-                const float other = upper ? f[e] : f[e + m * W];
-                const float got = __shfl_xor_sync(kFull, other, m);
-                if (upper) f[e + m * W] = mine + got; else f[e] = mine + got;
-              }
-            }
-          }
-          if (t < nv) {
-            float outv[W];
-#pragma unroll
-            for (int e = 0; e < W; ++e) {
-              float sel = f[e];
-#pragma unroll
-              for (int rr = 1; rr < R; ++rr)
-                if (rr == r) sel = f[rr * W + e];
-              outv[e] = sel;
-            }
-            const int pc = col0 + r * W;
-            if (p.D) {
-#pragma unroll
-              for (int e = 0; e < W; ++e) outv[e] = fmaf(Dh, __bfloat162float(xg[yrow + pc + e]), outv[e]);
-            }
-#pragma unroll
-            for (int e = 0; e < W; e += 2)
-              *reinterpret_cast<uint32_t*>(yg + yrow + pc + e) = pack_bf16(outv[e], outv[e + 1]);
-          }
-        }
-        if (state_warp) {
-          if (!mma4_early) state_update(scal[0], 1.0f, true);
-          else if constexpr (C::kInterInS) write_state_bf16();
-        }
+      if (!fast) {
+        if (tid == 0 && has_next) issue_bc(j + 1);
+        if (state_warp) state_update(scal(par)[0], 1.0f, hnext);
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
       }
     }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
+  }
+  if constexpr (FULL) {
+    if (!failed && j0 < j1) {
+      if (!state_warp) epilogue(j1 - 1, (int)((j1 - 1 - j0) & 1));
+    }
   }
 
   // ---- results
@@ -1099,12 +1091,11 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base
 }
 
 struct Maps {
-  CUtensorMap B, C, X, T;
+  CUtensorMap B, C, X;
 };
 
 bool make_maps(const Params& p, int Q, Maps* m) {
   const cuuint64_t toks = (cuuint64_t)(p.b * p.L);
-  const cuuint64_t K2 = (cuuint64_t)(p.N / 2);
   {
     const cuuint64_t dims[4] = {(cuuint64_t)p.N, (cuuint64_t)p.R, (cuuint64_t)p.G, toks};
     const cuuint64_t str[3] = {(cuuint64_t)p.N * 2, (cuuint64_t)p.R * p.N * 2, (cuuint64_t)p.G * p.R * p.N * 2};
@@ -1121,13 +1112,6 @@ bool make_maps(const Params& p, int Q, Maps* m) {
     if (!make_map(&m->X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.x, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
       return false;
   }
-  {
-    const cuuint64_t dims[3] = {K2, (cuuint64_t)p.G, toks};
-    const cuuint64_t str[2] = {K2 * 4, (cuuint64_t)p.G * K2 * 4};
-    const cuuint32_t box[3] = {(cuuint32_t)K2, 1, (cuuint32_t)Q};
-    if (!make_map(&m->T, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p.theta, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
-      return false;
-  }
   return true;
 }
 
@@ -1142,7 +1126,7 @@ cudaError_t launch_mode(const Maps& m, const Params& p, const SegInfo& sg, unsig
   auto k = scan_tc_kernel<R, N, P, MODE>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::SMEM);
   if (e != cudaSuccess) return e;
-  k<<<grid, kThreads, Cf::SMEM, stream>>>(m.B, m.C, m.X, m.T, p, sg);
+  k<<<grid, kThreads, Cf::SMEM, stream>>>(m.B, m.C, m.X, p, sg);
   return cudaGetLastError();
 }
 
