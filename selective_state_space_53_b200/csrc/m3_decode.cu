@@ -3,9 +3,10 @@
 // Decode reads and rewrites the whole fixed-size state every token (Mamba-3 paper note,
 // docsaid.org, section その3: the step is memory-bound; MIMO rank R adds arithmetic per
 // state byte).  One CTA per (batch, head):
-//   * the fp32 state tile (N x P) is brought into shared memory by one bulk copy on the
-//     TMA engine (cp.async.bulk, completion counted in bytes on an mbarrier), so no
-//     registers hold loads in flight and two CTAs fit per SM;
+//   * the fp32 state tile (N x P) is brought into shared memory by two bulk copies on the
+//     TMA engine (cp.async.bulk, completion counted in bytes on an mbarrier per half), so no
+//     registers hold loads in flight, work on the first half starts while the second lands,
+//     and three CTAs fit per SM (the readout partials reuse the tile's space);
 //   * meanwhile the threads stage the token operands: biased B and C rows, the MIMO
 //     branches X_r = W_x[r] * x_t and X'_r = W_x[r] * x_{t-1}, the rotation table;
 //   * each thread then updates a 4-column quad of rotation pairs (2k, 2k+1),
@@ -34,16 +35,17 @@ __device__ __forceinline__ uint64_t globaltimer() {
 struct DecShape {
   int PQ, KG, K;
 };
-__host__ __device__ inline DecShape dec_shape(int P, int N) {
+__host__ __device__ inline DecShape dec_shape(int P, int N, int threads = kThreads) {
   DecShape s;
   s.PQ = P / 4;
   s.K = N / 2;
-  const int kg = kThreads / s.PQ;
+  const int kg = threads / s.PQ;
   s.KG = kg < s.K ? kg : s.K;
   return s;
 }
 
-// shared-memory plan in floats; the state tile comes first (16-byte aligned for the copy)
+// shared-memory plan in floats; the state tile comes first (16-byte aligned for the copy).
+// The readout partials (KG x R x P) reuse the state tile once every thread has read it.
 struct DecSmem {
   int st, bb0, bb1, cb, x0, x1, cs, coef, red, mbar, total;
 };
@@ -59,15 +61,16 @@ __host__ __device__ inline DecSmem dec_smem(int P, int N, int R, int KG) {
   m.cs = o;  o += N;       // (cos, sin) per pair
   m.coef = o; o += 4;
   o = (o + 3) & ~3;
-  m.red = o; o += KG * R * P;
+  m.red = (KG * R * P <= N * P) ? m.st : o;  // reuses the state tile after the update
+  if (KG * R * P > N * P) o += KG * R * P;
   o = (o + 3) & ~3;
-  m.mbar = o; o += 4;
+  m.mbar = o; o += 4;  // two mbarriers
   m.total = o;
   return m;
 }
 
 template <int RT, bool BF16>
-__global__ void __launch_bounds__(kThreads, 2) decode_kernel(Params p) {
+__global__ void __launch_bounds__(kThreads, 3) decode_kernel(Params p) {
   extern __shared__ __align__(16) float sm[];
   const int tid = threadIdx.x;
   const int H = p.H, P = p.P, N = p.N, R = p.R, G = p.G;
@@ -95,19 +98,25 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(Params p) {
   const float* Wx = p.W_x ? p.W_x + (int64_t)hi * R * P : nullptr;
   const float* Wo = p.W_o ? p.W_o + (int64_t)hi * R * P : nullptr;
 
-  // ---- state tile: one bulk copy HBM -> shared memory
+  // ---- state tile: two bulk copies HBM -> shared memory (rows [0, N/2) and [N/2, N))
   if (tid == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bar)));
+    const uint32_t half = (uint32_t)(N / 2 * P * 4);
+#pragma unroll
+    for (int hb = 0; hb < 2; ++hb) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bar + hb)));
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    const uint32_t bytes = (uint32_t)(N * P * 4);
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-                 : "memory");
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(st)),
-        "l"(hg), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
+#pragma unroll
+    for (int hb = 0; hb < 2; ++hb) {
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar + hb)), "r"(half)
+                   : "memory");
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+              smem_u32(st) + hb * half),
+          "l"(hg + (size_t)hb * (N / 2) * P), "r"(half), "r"(smem_u32(bar + hb))
+          : "memory");
+    }
   }
 
   // ---- token operands
@@ -141,27 +150,28 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(Params p) {
     }
   }
   __syncthreads();
-  // ---- wait for the state tile (bounded)
-  {
+  // bounded wait for half `hb` of the state tile
+  auto wait_half = [&](int hb) -> bool {
     uint32_t done = 0;
     const uint64_t t0 = globaltimer();
     while (true) {
       asm volatile(
           "{\n .reg .pred q;\n mbarrier.try_wait.parity.shared::cta.b64 q, [%1], 0;\n selp.u32 %0, 1, 0, q;\n}\n"
           : "=r"(done)
-          : "r"(smem_u32(bar))
+          : "r"(smem_u32(bar + hb))
           : "memory");
       if (done || globaltimer() - t0 > kWaitNs) break;
     }
-    if (__syncthreads_or(!done)) {
-      if (tid == 0) set_status(p.status, M3_ERR_TIMEOUT);
-      return;
-    }
-  }
+    return done != 0;
+  };
+  bool ok = true;
 
   const int pq = tid % sh.PQ;
   const int kg = tid / sh.PQ;
   const int p0 = 4 * pq;
+  float Yacc[RT][4];
+#pragma unroll
+  for (int r = 0; r < RT; ++r) Yacc[r][0] = Yacc[r][1] = Yacc[r][2] = Yacc[r][3] = 0.0f;
   if (kg < sh.KG) {
     const float alpha = coef[0], bp = coef[1], gm = coef[2];
     float4 Xc[RT], Xp[RT];
@@ -174,11 +184,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(Params p) {
         Xc[r] = Xp[r] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
-    float Y[RT][4];
-#pragma unroll
-    for (int r = 0; r < RT; ++r) Y[r][0] = Y[r][1] = Y[r][2] = Y[r][3] = 0.0f;
-#pragma unroll 2
+    float (&Y)[RT][4] = Yacc;
+#pragma unroll 1
     for (int k = kg; k < sh.K; k += sh.KG) {
+      if (k == kg) ok = wait_half(0) && ok;
+      if (2 * k >= N / 2 && 2 * (k - sh.KG) < N / 2) ok = wait_half(1) && ok;  // first pair in rows >= N/2
+      if (!ok) break;
       const float4 s0 = *reinterpret_cast<const float4*>(st + (2 * k) * P + p0);
       const float4 s1 = *reinterpret_cast<const float4*>(st + (2 * k + 1) * P + p0);
       float u0[4] = {0, 0, 0, 0}, u1[4] = {0, 0, 0, 0}, q0[4] = {0, 0, 0, 0}, q1[4] = {0, 0, 0, 0};
@@ -221,12 +232,21 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(Params p) {
         }
       }
     }
+  }
+  if (tid == 0) ok = wait_half(0) && wait_half(1) && ok;  // both copies done before the tile is reused
+  // every thread has read its part of the state tile: the partial readouts may overwrite it
+  if (__syncthreads_or(!ok)) {
+    if (tid == 0) set_status(p.status, M3_ERR_TIMEOUT);
+    return;
+  }
+  if (kg < sh.KG) {
 #pragma unroll
     for (int r = 0; r < RT; ++r)
       if (r < R)
-        *reinterpret_cast<float4*>(red + (kg * R + r) * P + p0) = make_float4(Y[r][0], Y[r][1], Y[r][2], Y[r][3]);
+        *reinterpret_cast<float4*>(red + (kg * R + r) * P + p0) = make_float4(Yacc[r][0], Yacc[r][1], Yacc[r][2], Yacc[r][3]);
   }
   __syncthreads();
+
   // ---- y = sum_r W_o[r] * (sum over pair groups) + D x; new carry = this token's raw B, x
   {
     const int64_t xoff = ((int64_t)bi * H + hi) * P;
@@ -244,6 +264,382 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(Params p) {
     }
     const int64_t bcoff = (((int64_t)bi * G + g) * R) * (int64_t)N;
     for (int i = tid; i < R * N; i += kThreads) cBg[i] = load_in<BF16>(p.B, bcoff + i);
+  }
+}
+
+// ------------------------------------------------------------------ ring form
+// Persistent form: one CTA per SM walks a contiguous range of (batch, head) units, ordered
+// head-major so that the per-head weights change at most a few times per CTA, and keeps
+// `stages` units in flight: while it updates unit i, the TMA engine brings the state tiles and
+// raw token operands of units i+1 .. i+stages-1 into a ring of shared-memory stages.  The
+// updated state goes straight from registers to HBM, so the copy engine only ever reads.
+
+constexpr int kMaxStages = 6;
+constexpr int kRingThreads = 256;
+constexpr int kRingQuads = 1;  // 4-column quads per thread
+constexpr uint32_t kCopyChunk = 0;  // bytes per bulk copy of the state tile (0: one copy)
+
+struct RingPlan {
+  int stages;
+  uint32_t stage_bytes;
+  // byte offsets inside a stage: state tile, raw B_t, raw C_t, carry_B, raw x_t, carry_x,
+  // theta_t, and the three per-unit scalars dt, A, lam
+  uint32_t o_st, o_b, o_c, o_cb, o_x, o_cx, o_th, o_sc;
+  // byte offsets of the single-buffered arrays after the ring: this unit's biased B, C and
+  // MIMO branches, the rotation table and coefficients, the weights of the current head
+  // (bias_B, bias_C, W_x, W_o) and the per-pair-group partial readouts
+  uint32_t o_bbc, o_bbp, o_cbb, o_xc, o_xp, o_xr, o_cs, o_coef, o_wb, o_wc, o_wx, o_wo, o_red, o_bar;
+  uint32_t total;
+};
+
+// thread (pq, kg) of the ring kernel: column quads pq + c * P / (4 * CQ), pairs kg, kg + KG, ...
+__host__ __device__ inline int ring_pq(int P) { return P / (4 * kRingQuads); }
+__host__ __device__ inline int ring_kg(int P, int N) {
+  const int kg = kRingThreads / ring_pq(P);
+  return kg < N / 2 ? kg : N / 2;
+}
+
+__host__ __device__ inline uint32_t pad16(uint32_t x) { return (x + 15u) & ~15u; }
+
+inline RingPlan ring_plan(int P, int N, int R, bool bf16, int max_bytes) {
+  const uint32_t esz = bf16 ? 2u : 4u;
+  RingPlan rp{};
+  uint32_t o = 0;
+  rp.o_st = o; o += pad16((uint32_t)N * P * 4);
+  rp.o_b = o;  o += pad16((uint32_t)R * N * esz);
+  rp.o_c = o;  o += pad16((uint32_t)R * N * esz);
+  rp.o_cb = o; o += pad16((uint32_t)R * N * 4);
+  rp.o_x = o;  o += pad16((uint32_t)P * esz);
+  rp.o_cx = o; o += pad16((uint32_t)P * 4);
+  rp.o_th = o; o += pad16((uint32_t)N / 2 * 4);
+  rp.o_sc = o; o += 16;
+  rp.stage_bytes = (o + 127u) & ~127u;
+  uint32_t f = 0;
+  rp.o_bbc = f; f += pad16((uint32_t)R * N * 4);
+  rp.o_bbp = f; f += pad16((uint32_t)R * N * 4);
+  rp.o_cbb = f; f += pad16((uint32_t)R * N * 4);
+  rp.o_xc = f;  f += pad16((uint32_t)R * P * 4);
+  rp.o_xp = f;  f += pad16((uint32_t)R * P * 4);
+  rp.o_xr = f;  f += pad16((uint32_t)P * 4);
+  rp.o_cs = f;  f += pad16((uint32_t)N / 2 * 8);
+  rp.o_coef = f; f += 16;
+  rp.o_wb = f; f += pad16((uint32_t)R * N * 4);
+  rp.o_wc = f; f += pad16((uint32_t)R * N * 4);
+  rp.o_wx = f; f += pad16((uint32_t)R * P * 4);
+  rp.o_wo = f; f += pad16((uint32_t)R * P * 4);
+  rp.o_red = f; f += pad16((uint32_t)ring_kg(P, N) * P * 4);
+  rp.o_bar = f; f += 8 * kMaxStages;
+  const int room = max_bytes - (int)f;
+  int st = room > 0 ? room / (int)rp.stage_bytes : 0;
+  rp.stages = st < kMaxStages ? st : kMaxStages;
+  const uint32_t ring = (uint32_t)rp.stages * rp.stage_bytes;
+  rp.o_bbc += ring; rp.o_bbp += ring; rp.o_cbb += ring; rp.o_xc += ring; rp.o_xp += ring;
+  rp.o_xr += ring; rp.o_cs += ring; rp.o_coef += ring; rp.o_wb += ring; rp.o_wc += ring;
+  rp.o_wx += ring; rp.o_wo += ring; rp.o_red += ring; rp.o_bar += ring;
+  rp.total = ring + f;
+  return rp;
+}
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+template <bool BF16>
+__device__ __forceinline__ float stage_in(const unsigned char* base, int i) {
+  if constexpr (BF16) {
+    return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(base)[i]);
+  } else {
+    return reinterpret_cast<const float*>(base)[i];
+  }
+}
+
+template <int RT, bool BF16>
+__global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, RingPlan rp) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int tid = threadIdx.x;
+  const int H = p.H, P = p.P, N = p.N, R = p.R, G = p.G;
+  const int64_t nb = p.b;
+  const int64_t U = nb * H;
+  const int64_t u0 = (int64_t)blockIdx.x * U / gridDim.x;
+  const int64_t u1 = (int64_t)(blockIdx.x + 1) * U / gridDim.x;
+  const int S = rp.stages;
+  constexpr uint32_t esz = BF16 ? 2u : 4u;
+  const uint32_t sbase = smem_u32(smem);
+  float* bbc = reinterpret_cast<float*>(smem + rp.o_bbc);
+  float* bbp = reinterpret_cast<float*>(smem + rp.o_bbp);
+  float* cbb = reinterpret_cast<float*>(smem + rp.o_cbb);
+  float* xc = reinterpret_cast<float*>(smem + rp.o_xc);
+  float* xp = reinterpret_cast<float*>(smem + rp.o_xp);
+  float* xr = reinterpret_cast<float*>(smem + rp.o_xr);
+  float2* cs = reinterpret_cast<float2*>(smem + rp.o_cs);
+  float* coef = reinterpret_cast<float*>(smem + rp.o_coef);
+  float* wb = reinterpret_cast<float*>(smem + rp.o_wb);
+  float* wc = reinterpret_cast<float*>(smem + rp.o_wc);
+  float* wx = reinterpret_cast<float*>(smem + rp.o_wx);
+  float* wo = reinterpret_cast<float*>(smem + rp.o_wo);
+  float* red = reinterpret_cast<float*>(smem + rp.o_red);
+  const uint32_t bar0 = sbase + rp.o_bar;
+
+  // unit u = head-major index: head u / b, sequence u % b
+  auto issue = [&](int64_t u, int s) {
+    const int64_t bi = u % nb;
+    const int hi = (int)(u / nb);
+    const int g = hi / (H / G);
+    const int64_t bh = bi * H + hi;
+    const uint32_t st = sbase + (uint32_t)s * rp.stage_bytes;
+    const uint32_t bar = bar0 + 8u * s;
+    const uint32_t n_st = (uint32_t)N * P * 4, n_b = (uint32_t)R * N * esz, n_cb = (uint32_t)R * N * 4;
+    const uint32_t n_x = (uint32_t)P * esz, n_cx = (uint32_t)P * 4, n_th = (uint32_t)N / 2 * 4;
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+                 "r"(n_st + 2 * n_b + n_cb + n_x + n_cx + n_th)
+                 : "memory");
+    const int64_t bc = ((bi * G + g) * R) * (int64_t)N;
+    const uint32_t chunk = kCopyChunk ? kCopyChunk : n_st;
+    for (uint32_t c = 0; c < n_st; c += chunk)
+      bulk_g2s(st + rp.o_st + c, reinterpret_cast<const unsigned char*>(p.h + bh * N * P) + c,
+               n_st - c < chunk ? n_st - c : chunk, bar);
+    bulk_g2s(st + rp.o_b, static_cast<const unsigned char*>(p.B) + bc * esz, n_b, bar);
+    bulk_g2s(st + rp.o_c, static_cast<const unsigned char*>(p.C) + bc * esz, n_b, bar);
+    bulk_g2s(st + rp.o_cb, p.carry_B + bh * R * N, n_cb, bar);
+    bulk_g2s(st + rp.o_x, static_cast<const unsigned char*>(p.x) + bh * P * esz, n_x, bar);
+    bulk_g2s(st + rp.o_cx, p.carry_x + bh * P, n_cx, bar);
+    bulk_g2s(st + rp.o_th, p.theta + (bi * G + g) * (N / 2), n_th, bar);
+    // the three scalars: 4-byte asynchronous copies whose completion is the barrier's second arrival
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(st + rp.o_sc), "l"(p.dt + bh) : "memory");
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(st + rp.o_sc + 4), "l"(p.A + bh) : "memory");
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(st + rp.o_sc + 8), "l"(p.lam + bh) : "memory");
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+  };
+  auto try_wait = [&](int s, uint32_t par) -> bool {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred q;\n mbarrier.try_wait.parity.shared::cta.b64 q, [%1], %2;\n selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(done)
+        : "r"(bar0 + 8u * s), "r"(par)
+        : "memory");
+    return done != 0;
+  };
+  auto wait = [&](int s, uint32_t par) -> bool {
+    if (try_wait(s, par)) return true;
+    const uint64_t t0 = globaltimer();
+    while (!try_wait(s, par)) {
+      if (globaltimer() - t0 > kWaitNs) return false;
+    }
+    return true;
+  };
+
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 2;" ::"r"(bar0 + 8u * s));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int s = 0; s < S && u0 + s < u1; ++s) issue(u0 + s, s);
+  }
+  __syncthreads();
+
+  // thread (pq, kg): column quads pq + c * P / (4 * CQ) for c < CQ, rotation pairs kg, kg + KG, ...
+  constexpr int CQ = kRingQuads;
+  const int PQ = ring_pq(P);
+  const int KG = ring_kg(P, N);
+  const int pq = tid % PQ;
+  const int kg = tid / PQ;
+  int cur_h = -1;
+  float Dh = 0.0f;
+  uint32_t phases = 0;  // bit s: parity of the next completion of stage s
+  int s = 0;
+  bool ok = true;
+  int64_t u = u0;
+  for (; u < u1; ++u) {
+    const uint32_t par = (phases >> s) & 1u;
+    phases ^= 1u << s;
+    const int64_t bi = u % nb;
+    const int hi = (int)(u / nb);
+    const int64_t bh = bi * H + hi;
+    const unsigned char* stg = smem + (size_t)s * rp.stage_bytes;
+    if (hi != cur_h) {  // weights of a new head (uniform: every thread sees the same unit)
+      cur_h = hi;
+      __syncthreads();  // the previous unit's output step has read W_o
+      const float* biasB = p.bias_B ? p.bias_B + (int64_t)hi * R * N : nullptr;
+      const float* biasC = p.bias_C ? p.bias_C + (int64_t)hi * R * N : nullptr;
+      const float* Wx = p.W_x ? p.W_x + (int64_t)hi * R * P : nullptr;
+      const float* Wo = p.W_o ? p.W_o + (int64_t)hi * R * P : nullptr;
+      for (int i = tid; i < R * N; i += kRingThreads) {
+        wb[i] = biasB ? biasB[i] : 0.0f;
+        wc[i] = biasC ? biasC[i] : 0.0f;
+      }
+      for (int i = tid; i < R * P; i += kRingThreads) {
+        wx[i] = Wx ? Wx[i] : 1.0f;
+        wo[i] = Wo ? Wo[i] : 1.0f;
+      }
+      Dh = p.D ? p.D[hi] : 0.0f;
+      __syncthreads();
+    }
+    ok = wait(s, par);
+    if (ok) {
+      // ---- operands of this unit
+      const float* sc = reinterpret_cast<const float*>(stg + rp.o_sc);
+      const float* cBs = reinterpret_cast<const float*>(stg + rp.o_cb);
+      const float* cxs = reinterpret_cast<const float*>(stg + rp.o_cx);
+      const float* ths = reinterpret_cast<const float*>(stg + rp.o_th);
+      float* cBg = p.carry_B + bh * R * N;
+      float* cxg = p.carry_x + bh * P;
+      for (int i = tid; i < R * N; i += kRingThreads) {
+        const float bb = wb[i];
+        const float braw = stage_in<BF16>(stg + rp.o_b, i);
+        bbc[i] = braw + bb;
+        bbp[i] = cBs[i] + bb;
+        cbb[i] = stage_in<BF16>(stg + rp.o_c, i) + wc[i];
+        cBg[i] = braw;  // new carry: this token's raw B
+      }
+      for (int i = tid; i < R * P; i += kRingThreads) {
+        const float w = wx[i];
+        xc[i] = stage_in<BF16>(stg + rp.o_x, i % P) * w;
+        xp[i] = cxs[i % P] * w;
+      }
+      for (int pp = tid; pp < P; pp += kRingThreads) {
+        const float xv = stage_in<BF16>(stg + rp.o_x, pp);
+        xr[pp] = xv;
+        cxg[pp] = xv;  // new carry: this token's raw x
+      }
+      const float delta = sc[0];
+      for (int k = tid; k < N / 2; k += kRingThreads) {
+        float sn, cn;
+        sincosf(delta * ths[k], &sn, &cn);
+        cs[k] = make_float2(cn, sn);
+      }
+      if (tid == 0) {
+        const float lm = sc[2];
+        coef[0] = expf(delta * sc[1]);
+        coef[1] = (1.0f - lm) * delta;
+        coef[2] = lm * delta;
+      }
+    }
+    if (__syncthreads_or(!ok)) {
+      ok = false;
+      phases ^= 1u << s;  // unit u's copies count as outstanding again
+      break;
+    }
+    // ---- state update of the thread's column quads over its rotation pairs
+    if (kg < KG) {
+      const float alpha = coef[0], bp = coef[1], gm = coef[2];
+      const float* stt = reinterpret_cast<const float*>(stg + rp.o_st);
+      float* hg = p.h + bh * N * P;
+      int pc[CQ];
+#pragma unroll
+      for (int c = 0; c < CQ; ++c) pc[c] = 4 * pq + c * (P / CQ);
+      float4 Xc[RT][CQ], Xp[RT][CQ];
+      float Y[RT][CQ][4];
+#pragma unroll
+      for (int r = 0; r < RT; ++r)
+#pragma unroll
+        for (int c = 0; c < CQ; ++c) {
+          Y[r][c][0] = Y[r][c][1] = Y[r][c][2] = Y[r][c][3] = 0.0f;
+          if (r < R) {
+            Xc[r][c] = *reinterpret_cast<const float4*>(xc + r * P + pc[c]);
+            Xp[r][c] = *reinterpret_cast<const float4*>(xp + r * P + pc[c]);
+          } else {
+            Xc[r][c] = Xp[r][c] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+#pragma unroll 2
+      for (int k = kg; k < N / 2; k += KG) {
+        float4 s0[CQ], s1[CQ];
+#pragma unroll
+        for (int c = 0; c < CQ; ++c) {
+          s0[c] = *reinterpret_cast<const float4*>(stt + (2 * k) * P + pc[c]);
+          s1[c] = *reinterpret_cast<const float4*>(stt + (2 * k + 1) * P + pc[c]);
+        }
+        float u0v[CQ][4] = {}, u1v[CQ][4] = {}, q0[CQ][4] = {}, q1[CQ][4] = {};
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          if (r < R) {
+            const float2 bcv = *reinterpret_cast<const float2*>(bbc + r * N + 2 * k);
+            const float2 bqv = *reinterpret_cast<const float2*>(bbp + r * N + 2 * k);
+#pragma unroll
+            for (int c = 0; c < CQ; ++c) {
+              const float xc4[4] = {Xc[r][c].x, Xc[r][c].y, Xc[r][c].z, Xc[r][c].w};
+              const float xp4[4] = {Xp[r][c].x, Xp[r][c].y, Xp[r][c].z, Xp[r][c].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                u0v[c][e] = fmaf(bcv.x, xc4[e], u0v[c][e]);
+                u1v[c][e] = fmaf(bcv.y, xc4[e], u1v[c][e]);
+                q0[c][e] = fmaf(bqv.x, xp4[e], q0[c][e]);
+                q1[c][e] = fmaf(bqv.y, xp4[e], q1[c][e]);
+              }
+            }
+          }
+        }
+        const float2 rc = cs[k];
+        const float ac = alpha * rc.x, as = alpha * rc.y;
+        float n0[CQ][4], n1[CQ][4];
+#pragma unroll
+        for (int c = 0; c < CQ; ++c) {
+          const float a0[4] = {s0[c].x, s0[c].y, s0[c].z, s0[c].w};
+          const float a1[4] = {s1[c].x, s1[c].y, s1[c].z, s1[c].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float v0 = fmaf(bp, q0[c][e], a0[e]);
+            const float v1 = fmaf(bp, q1[c][e], a1[e]);
+            n0[c][e] = fmaf(ac, v0, fmaf(-as, v1, gm * u0v[c][e]));
+            n1[c][e] = fmaf(as, v0, fmaf(ac, v1, gm * u1v[c][e]));
+          }
+          *reinterpret_cast<float4*>(hg + (int64_t)(2 * k) * P + pc[c]) =
+              make_float4(n0[c][0], n0[c][1], n0[c][2], n0[c][3]);
+          *reinterpret_cast<float4*>(hg + (int64_t)(2 * k + 1) * P + pc[c]) =
+              make_float4(n1[c][0], n1[c][1], n1[c][2], n1[c][3]);
+        }
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          if (r < R) {
+            const float2 cc = *reinterpret_cast<const float2*>(cbb + r * N + 2 * k);
+#pragma unroll
+            for (int c = 0; c < CQ; ++c)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) Y[r][c][e] = fmaf(cc.x, n0[c][e], fmaf(cc.y, n1[c][e], Y[r][c][e]));
+          }
+        }
+      }
+      // this pair group's part of sum_r W_o[r] * readout_r; summed over the groups after the barrier
+#pragma unroll
+      for (int c = 0; c < CQ; ++c) {
+        float o[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int r = 0; r < RT; ++r)
+          if (r < R) {
+            const float4 w4 = *reinterpret_cast<const float4*>(wo + r * P + pc[c]);
+            o[0] = fmaf(w4.x, Y[r][c][0], o[0]);
+            o[1] = fmaf(w4.y, Y[r][c][1], o[1]);
+            o[2] = fmaf(w4.z, Y[r][c][2], o[2]);
+            o[3] = fmaf(w4.w, Y[r][c][3], o[3]);
+          }
+        *reinterpret_cast<float4*>(red + kg * P + pc[c]) = make_float4(o[0], o[1], o[2], o[3]);
+      }
+    }
+    __syncthreads();  // stage s is read; the readouts are summed
+    if (tid == 0 && u + S < u1) issue(u + S, s);
+    // ---- y = sum_r W_o[r] * readout_r + D x
+    for (int pp = tid; pp < P; pp += kRingThreads) {
+      float acc0 = 0.0f, acc1 = 0.0f;
+      int q = 0;
+      for (; q + 1 < KG; q += 2) {
+        acc0 += red[q * P + pp];
+        acc1 += red[(q + 1) * P + pp];
+      }
+      if (q < KG) acc0 += red[q * P + pp];
+      store_out<BF16>(p.y, bh * P + pp, fmaf(Dh, xr[pp], acc0 + acc1));
+    }
+    s = (s + 1 == S) ? 0 : s + 1;
+  }
+  if (!ok) {
+    // give up: wait (bounded) for the copies still in flight, then report
+    if (tid == 0) {
+      for (int64_t v = u; v < u1 && v < u + S; ++v) {
+        const int sv = (int)((v - u0) % S);
+        wait(sv, (phases >> sv) & 1u);
+      }
+      set_status(p.status, M3_ERR_TIMEOUT);
+    }
   }
 }
 
@@ -269,14 +665,69 @@ size_t decode_smem_bytes(int P, int N, int R) {
   return sizeof(float) * (size_t)dec_smem(P, N, R, sh.KG).total;
 }
 
+struct DeviceLimits {
+  int sms = 0, smem_optin = 0;
+};
+// SM count and opt-in shared memory per block of the current device (cached per device).
+DeviceLimits device_limits() {
+  static DeviceLimits cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DeviceLimits{};
+  DeviceLimits& d = cache[dev];
+  if (d.sms == 0) {
+    int sms = 0, optin = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      return DeviceLimits{};
+    d.smem_optin = optin;
+    d.sms = sms;
+  }
+  return d;
+}
+
+template <int RT>
+cudaError_t launch_ring_rt(const Params& p, const RingPlan& rp, unsigned grid, cudaStream_t stream) {
+  if (p.dtype == M3_BF16) {
+    auto k = decode_ring_kernel<RT, true>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rp.total);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kRingThreads, rp.total, stream>>>(p, rp);
+  } else {
+    auto k = decode_ring_kernel<RT, false>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rp.total);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kRingThreads, rp.total, stream>>>(p, rp);
+  }
+  return cudaGetLastError();
+}
+
+// The ring form needs two stages on chip at least.
+bool ring_plan_for(const Params& p, RingPlan* out) {
+  const DeviceLimits d = device_limits();
+  if (d.sms == 0) return false;
+  *out = ring_plan(p.P, p.N, p.R, p.dtype == M3_BF16, d.smem_optin);
+  return out->stages >= 2;
+}
+
 }  // namespace
 
 bool decode_supported(const Params& p) {
-  return decode_smem_bytes(p.P, p.N, p.R) <= 200 * 1024;
+  RingPlan rp;
+  return ring_plan_for(p, &rp) || decode_smem_bytes(p.P, p.N, p.R) <= 200 * 1024;
 }
 
 cudaError_t launch_decode(const Params& p, cudaStream_t stream) {
   if (p.b * p.H == 0) return cudaSuccess;
+  RingPlan rp;
+  if (ring_plan_for(p, &rp)) {
+    const int64_t units = p.b * p.H;
+    const int sms = device_limits().sms;
+    const unsigned grid = (unsigned)(units < sms ? units : sms);
+    if (p.R <= 1) return launch_ring_rt<1>(p, rp, grid, stream);
+    if (p.R <= 2) return launch_ring_rt<2>(p, rp, grid, stream);
+    if (p.R <= 4) return launch_ring_rt<4>(p, rp, grid, stream);
+    return launch_ring_rt<8>(p, rp, grid, stream);
+  }
   const size_t smem = decode_smem_bytes(p.P, p.N, p.R);
   if (p.R <= 1) return launch_rt<1>(p, smem, stream);
   if (p.R <= 2) return launch_rt<2>(p, smem, stream);

@@ -76,6 +76,12 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
@@ -136,6 +142,26 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a, uint64_t b, uint3
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
       "r"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+// Warp-collective forms of the two above and of mma_commit: every lane of a converged warp
+// executes them with warp-uniform operands, and the lane that elect.sync picks issues.
+__device__ __forceinline__ void mma_ss_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p, e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void mma_ts_w(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p, e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
+      "r"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+__device__ __forceinline__ void mma_commit_w(uint64_t* bar) {
+  asm volatile(
+      "{\n .reg .pred e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}\n" ::"r"(smem_u32(bar))
+      : "memory");
 }
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -284,7 +310,7 @@ struct Cfg {
   static constexpr uint32_t ID_Y2 = idesc_bf16(128, P, false, true);
   static constexpr int TX_B = kRows * N * 2;
   static constexpr int TX_X = Q * P * 2;
-  static constexpr int NT = FULL ? 128 : 256;  // threads that stage operand tiles
+  static constexpr int NT = 256;  // threads that stage the B, C rows
 };
 
 // The decay inside a tile, e^{Lc_t - Lc_s}, is split around a pivot m (the middle of the
@@ -407,14 +433,14 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
       rawA(slot, 3)[0] = (1.0f - r_lm) * r_dt;
     }
   };
-  // coefficients, records and the rotation table of tile j into slot `slot` (all threads;
-  // the raw values of the tile must be in raw slot `slot` and r_th)
-  auto tile_prep = [&](int64_t j, int slot) {
+  // decay coefficients and per-token records of tile j into slot `slot` (warp 0; the raw
+  // values of the tile must be in raw slot `slot`)
+  auto coef_prep = [&](int64_t j, int slot) {
     const int nv = (int)((L - j * Q) < Q ? (L - j * Q) : Q);
     const float* dtA = rawA(slot, 0);
     const float* aA = rawA(slot, 1);
     const float* lmA = rawA(slot, 2);
-    if (warp == 0) {
+    {
       constexpr int PER = (Q + 31) / 32;
       float loc[PER];
       float run = 0.0f;
@@ -475,6 +501,12 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
         sc[4] = fast ? __expf(m) : 1.0f;
       }
     }
+  };
+  // rotation table of tile j into slot `slot` (all threads; the raw dt of the tile must be in
+  // raw slot `slot` and its theta in r_th)
+  auto angle_prep = [&](int64_t j, int slot) {
+    const int nv = (int)((L - j * Q) < Q ? (L - j * Q) : Q);
+    const float* dtA = rawA(slot, 0);
     float aloc[C::SEGLEN];
     {
       float run = 0.0f;
@@ -490,11 +522,9 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
     double total = 0.0;
     {
       float aoff = 0.0f;
-      for (int s = 0; s < C::SEGS; ++s) {
-        const float v = segsum[s * K2 + ak];
-        if (s < aseg) aoff += v;
-        total += (double)v;
-      }
+      for (int s = 0; s < aseg; ++s) aoff += segsum[s * K2 + ak];
+      if (aseg == 0)
+        for (int s = 0; s < C::SEGS; ++s) total += (double)segsum[s * K2 + ak];
       aoff += (float)base[ak];
       float2* c2 = cs(slot);
 #pragma unroll
@@ -540,12 +570,15 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = __shfl_sync(kFull, *tmem_slot, 0);
   if (tid == 0 && j0 < j1) {
     issue_x(j0);
     issue_bc(j0);
   }
-  if (j0 < j1) tile_prep(j0, 0);
+  if (j0 < j1) {
+    if (warp == 0) coef_prep(j0, 0);
+    angle_prep(j0, 0);
+  }
   if (j0 + 1 < j1) load_coefs(j0 + 1);
 
   // state warps: TMEM lane of accumulator row p (M = 128: lane = p; M = 64: rows in lanes
@@ -556,9 +589,9 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
   const int prow = (P == 128) ? (32 * q4 + lane) : (16 * q4 + (lane & 15));
   const bool st_owner = (P == 128) || (lane >= 16);  // holds the fp32 state of row prow
 
-  // operand staging threads (FULL: warps 4-7, while warps 0-3 run the previous epilogue)
-  const bool xf_thread = FULL ? (tid >= 128) : true;
-  const int xt = FULL ? tid - 128 : tid;
+  // operand staging: B, C rows on all threads; x rows on warps 1-7 (warp 0 prepares the next
+  // tile's coefficients meanwhile)
+  const int xt = tid;
   constexpr int CHN = N / 8;
   constexpr int RPI = NT / CHN;  // rows per pass; a multiple of 8 and of R
   const int tch = xt % CHN;
@@ -566,8 +599,8 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
   float bB[8], bC[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
-    bB[e] = (xf_thread && biasBg) ? __ldg(biasBg + tr * N + tch * 8 + e) : 0.0f;
-    bC[e] = (xf_thread && biasCg) ? __ldg(biasCg + tr * N + tch * 8 + e) : 0.0f;
+    bB[e] = biasBg ? __ldg(biasBg + tr * N + tch * 8 + e) : 0.0f;
+    bC[e] = biasCg ? __ldg(biasCg + tr * N + tch * 8 + e) : 0.0f;
   }
 
   // ---- incoming rotated-frame state h+ of this segment
@@ -700,58 +733,64 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
     constexpr int W = 16 / R;
     const float at = recA(slot)[t].z;
     const int64_t yrow = ((tok_base + c0 + t) * H + hi) * P;
+    const int c2_0 = (warp >> 2) * (P / 64);  // warps 0-3: columns [0, P/2); warps 4-7: [P/2, P)
 #pragma unroll 1
-    for (int c = 0; c < P / 16; ++c) {
-      const int col0 = 16 * c;
-      uint32_t v[16];
-      tmem_ld16(tmem + lane_base + C::TM_Y + col0, v);
+    for (int c2 = c2_0; c2 < c2_0 + P / 64; ++c2) {
+      uint32_t v2[32];  // two 16-column chunks per TMEM wait
+      tmem_ld32(tmem + lane_base + C::TM_Y + 32 * c2, v2);
       tmem_wait_ld();
-      float f[16];
 #pragma unroll
-      for (int e4 = 0; e4 < 4; ++e4) {
-        const float4 w4 = *reinterpret_cast<const float4*>(&wo[r * P + col0 + 4 * e4]);
-        f[4 * e4] = at * w4.x * __uint_as_float(v[4 * e4]);
-        f[4 * e4 + 1] = at * w4.y * __uint_as_float(v[4 * e4 + 1]);
-        f[4 * e4 + 2] = at * w4.z * __uint_as_float(v[4 * e4 + 2]);
-        f[4 * e4 + 3] = at * w4.w * __uint_as_float(v[4 * e4 + 3]);
-      }
-      // reduce over the R branches (adjacent lanes); lane r keeps columns [r*W, r*W + W)
+      for (int half = 0; half < 2; ++half) {
+        const int col0 = 32 * c2 + 16 * half;
+        float f[16];
 #pragma unroll
-      for (int m = R / 2; m >= 1; m >>= 1) {
-        const bool upper = (r & m) != 0;
+        for (int e4 = 0; e4 < 4; ++e4) {
+          const float4 w4 = *reinterpret_cast<const float4*>(&wo[r * P + col0 + 4 * e4]);
+          f[4 * e4] = (at * w4.x) * __uint_as_float(v2[16 * half + 4 * e4]);
+          f[4 * e4 + 1] = (at * w4.y) * __uint_as_float(v2[16 * half + 4 * e4 + 1]);
+          f[4 * e4 + 2] = (at * w4.z) * __uint_as_float(v2[16 * half + 4 * e4 + 2]);
+          f[4 * e4 + 3] = (at * w4.w) * __uint_as_float(v2[16 * half + 4 * e4 + 3]);
+        }
+        // reduce over the R branches held by adjacent lanes: at each step a lane keeps the half of
+        // its columns selected by one bit of r, moved to the front; lane r ends with columns
+        // [r*W, r*W + W) of the sum in f[0..W)
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          if ((e / W) % (2 * m) < m) {
-            const float mine = upper ? f[e + m * W] : f[e];
-            const float other = upper ? f[e] : f[e + m * W];
-            const float got = __shfl_xor_sync(kFull, other, m);
-            if (upper) f[e + m * W] = mine + got; else f[e] = mine + got;
+        for (int m = R / 2, span = 8; m >= 1; m >>= 1, span >>= 1) {
+          const bool upper = (r & m) != 0;
+#pragma unroll
+          for (int e = 0; e < span; ++e) {
+            const float keep = upper ? f[e + span] : f[e];
+            const float give = upper ? f[e] : f[e + span];
+            f[e] = keep + __shfl_xor_sync(kFull, give, m);
           }
         }
-      }
-      if (t < nv) {
-        float outv[W];
+        if (t < nv) {
+          const int pc = col0 + r * W;
+          if (p.D) {
 #pragma unroll
-        for (int e = 0; e < W; ++e) {
-          float sel = f[e];
-#pragma unroll
-          for (int rr = 1; rr < R; ++rr)
-            if (rr == r) sel = f[rr * W + e];
-          outv[e] = sel;
+            for (int e = 0; e < W; ++e) f[e] = fmaf(Dh, __bfloat162float(xg[yrow + pc + e]), f[e]);
+          }
+          if constexpr (W == 16) {
+            uint4 o0 = make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
+            uint4 o1 = make_uint4(pack_bf16(f[8], f[9]), pack_bf16(f[10], f[11]), pack_bf16(f[12], f[13]), pack_bf16(f[14], f[15]));
+            *reinterpret_cast<uint4*>(yg + yrow + pc) = o0;
+            *reinterpret_cast<uint4*>(yg + yrow + pc + 8) = o1;
+          } else if constexpr (W == 8) {
+            *reinterpret_cast<uint4*>(yg + yrow + pc) =
+                make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
+          } else if constexpr (W == 4) {
+            *reinterpret_cast<uint2*>(yg + yrow + pc) = make_uint2(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]));
+          } else {
+            *reinterpret_cast<uint32_t*>(yg + yrow + pc) = pack_bf16(f[0], f[1]);
+          }
         }
-        const int pc = col0 + r * W;
-        if (p.D) {
-#pragma unroll
-          for (int e = 0; e < W; ++e) outv[e] = fmaf(Dh, __bfloat162float(xg[yrow + pc + e]), outv[e]);
-        }
-#pragma unroll
-        for (int e = 0; e < W; e += 2)
-          *reinterpret_cast<uint32_t*>(yg + yrow + pc + e) = pack_bf16(outv[e], outv[e + 1]);
       }
     }
   };
 
   uint32_t mma_phase = 0, load_phase = 0;
+  uint32_t y_phase = 0;    // barrier phase of the last MMA_B
+  bool y_pending = false;  // a fast tile's MMA_B may still run: warps 0-3 wait before TM_Y / sX
   bool failed = false;
   float seg_logdec = 0.0f;
   for (int64_t j = j0; j < j1; ++j) {
@@ -760,78 +799,134 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
     const int par = (int)((j - j0) & 1);
     const bool has_next = j + 1 < j1;
 
-    // ---- X: stage tile j (staging threads) | epilogue of tile j-1 (warps 0-3)
+    // ---- X (all warps): B, C rows of tile j; then, once MMA_B of tile j-1 is done, its
+    //      epilogue (each warp: its TMEM lane quarter, half the columns); then the x rows of
+    //      tile j (warps 1-7) and the coefficients of tile j+1 (warp 0)
     bool bad = false;
-    if (xf_thread) {
-      bad = !mbar_wait(load_bar, load_phase);
-      if (!bad) {
+    if (has_next) store_coefs(par ^ 1);  // raw values of tile j+1 (loaded one window ago)
+    bad = !mbar_wait(load_bar, load_phase);
+    if (!bad) {
+      {
         const bool fast = scal(par)[3] != 0.0f;
         const float2* csj = cs(par);
-        const float4* raj = recA(par);
         const float4* rbj = recB(par);
         const int i0 = xt / CHN;
         const uint32_t off0 = (uint32_t)(tch >> 3) * (kRows * 128) + (uint32_t)i0 * 128u +
                               ((uint32_t)((tch & 7) ^ (i0 & 7)) << 4);  // i0 + k*RPI keeps i & 7
-#pragma unroll 2
-        for (int it = 0; it < kRows / RPI; ++it) {
-          const int i = i0 + it * RPI;
-          const int t = i / R;
-          const uint32_t off = off0 + (uint32_t)(it * RPI) * 128u;
-          if (t < nv) {
-            const float4 w01 = *reinterpret_cast<const float4*>(&csj[t * K2 + tch * 4]);
-            const float4 w23 = *reinterpret_cast<const float4*>(&csj[t * K2 + tch * 4 + 2]);
-            const float wc[4] = {w01.x, w01.z, w23.x, w23.z};
-            const float ws[4] = {w01.y, w01.w, w23.y, w23.w};
-            const float bsc = (!FULL && !fast) ? rbj[t].y : 1.0f;  // state pass, exact tile
+        // rows in groups of UG: all shared-memory loads of a group are issued before any store
+        constexpr int NIT = kRows / RPI;
+        constexpr int UG = NIT >= 2 ? 2 : 1;
+#pragma unroll 1
+        for (int it0 = 0; it0 < NIT; it0 += UG) {
+          uint4 rb[UG], rc[UG];
+          float4 w01[UG], w23[UG];
+          int tt[UG];
+          uint32_t offs[UG];
+#pragma unroll
+          for (int u = 0; u < UG; ++u) {
+            const int i = i0 + (it0 + u) * RPI;
+            tt[u] = i / R;
+            offs[u] = off0 + (uint32_t)((it0 + u) * RPI) * 128u;
+            const int tc = tt[u] < Q ? tt[u] : Q - 1;
+            w01[u] = *reinterpret_cast<const float4*>(&csj[tc * K2 + tch * 4]);
+            w23[u] = *reinterpret_cast<const float4*>(&csj[tc * K2 + tch * 4 + 2]);
+            rb[u] = lds128(sBT + offs[u]);
+            if constexpr (FULL) rc[u] = lds128(sCT + offs[u]);
+          }
+#pragma unroll
+          for (int u = 0; u < UG; ++u) {
+            const int t = tt[u];
+            const bool valid = t < nv;
+            const float wc[4] = {w01[u].x, w01[u].z, w23[u].x, w23[u].z};
+            const float ws[4] = {w01[u].y, w01[u].w, w23[u].y, w23[u].w};
+            if (!valid) {  // past the end of the sequence: zero rows
+              sts128(sBT + offs[u], make_uint4(0, 0, 0, 0));
+              if constexpr (FULL) sts128(sCT + offs[u], make_uint4(0, 0, 0, 0));
+              continue;
+            }
             {
               float f[8];
-              unpack8(lds128(sBT + off), f);
+              unpack8(rb[u], f);
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 const float b0 = f[2 * q] + bB[2 * q], b1 = f[2 * q + 1] + bB[2 * q + 1];
-                f[2 * q] = bsc * (wc[q] * b0 + ws[q] * b1);  // Rot(-Phi)
-                f[2 * q + 1] = bsc * (wc[q] * b1 - ws[q] * b0);
+                f[2 * q] = wc[q] * b0 + ws[q] * b1;  // Rot(-Phi)
+                f[2 * q + 1] = wc[q] * b1 - ws[q] * b0;
               }
-              sts128(sBT + off, pack8(f));
+              if (!FULL && !fast) {  // state pass, exact tile: Bt rows * e^{Le - Lc_t}
+                const float bsc = rbj[t].y;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] *= bsc;
+              }
+              sts128(sBT + offs[u], pack8(f));
             }
             if constexpr (FULL) {
               float f[8];
-              unpack8(lds128(sCT + off), f);
+              unpack8(rc[u], f);
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
                 const float d0 = f[2 * q] + bC[2 * q], d1 = f[2 * q + 1] + bC[2 * q + 1];
                 f[2 * q] = wc[q] * d0 + ws[q] * d1;
                 f[2 * q + 1] = wc[q] * d1 - ws[q] * d0;
               }
-              sts128(sCT + off, pack8(f));
+              sts128(sCT + offs[u], pack8(f));
             }
-          } else {
-            const uint4 z = make_uint4(0, 0, 0, 0);
-            sts128(sBT + off, z);
-            if constexpr (FULL) sts128(sCT + off, z);
-          }
-        }
-        constexpr int CHP = P / 8;
-        const int xch = xt % CHP;  // fixed column chunk
-        for (int t = xt / CHP; t < Q; t += NT / CHP) {
-          float fx[8];
-          unpack8(lds128(sXSTG + (uint32_t)(t * P + xch * 8) * 2), fx);
-          const float xs = (t < nv) ? raj[t].w : 0.0f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) fx[e] *= xs;
-#pragma unroll
-          for (int rr = 0; rr < R; ++rr) {
-            const int i = t * R + rr;
-            const float4 w0 = *reinterpret_cast<const float4*>(&wx[rr * P + xch * 8]);
-            const float4 w1 = *reinterpret_cast<const float4*>(&wx[rr * P + xch * 8 + 4]);
-            const float xr[8] = {fx[0] * w0.x, fx[1] * w0.y, fx[2] * w0.z, fx[3] * w0.w,
-                                 fx[4] * w1.x, fx[5] * w1.y, fx[6] * w1.z, fx[7] * w1.w};
-            sts128(sX + sw128(i, xch, kRows * 128), pack8(xr));
           }
         }
       }
-    } else if (FULL && j > j0) {
-      epilogue(j - 1, par ^ 1);
+    }
+    if (FULL && y_pending && !bad) {
+      bad = !mbar_wait(mma_bar, y_phase);
+      tc_fence_after();
+    }
+    if (FULL && j > j0 && !bad) epilogue(j - 1, par ^ 1);
+    // barrier 1: every thread has stored its raw values of tile j+1 and read the records of
+    // tile j-1 (epilogue), whose slot coef_prep(j+1) overwrites; only warp 0 waits on it
+    if (warp == 0) {
+      named_bar_sync(1, kThreads);
+      if (has_next) coef_prep(j + 1, par ^ 1);
+    } else {
+      named_bar_arrive(1, kThreads);
+      if (!bad) {  // x rows on warps 1-7
+        const float4* raj = recA(par);
+        constexpr int CHP = P / 8;
+        constexpr int NX = kThreads - 32;
+        const int xi = tid - 32;
+        const int xch = xi % CHP;  // fixed column chunk
+        constexpr int TSTEP = NX / CHP;
+        constexpr int XU = (Q / TSTEP) >= 2 ? 2 : 1;
+#pragma unroll 1
+        for (int t0 = xi / CHP; t0 < Q; t0 += XU * TSTEP) {
+          uint4 xv[XU];
+          float xsv[XU];
+#pragma unroll
+          for (int u = 0; u < XU; ++u) {
+            const int t = t0 + u * TSTEP;
+            const int tc = t < Q ? t : Q - 1;
+            xv[u] = lds128(sXSTG + (uint32_t)(tc * P + xch * 8) * 2);
+            xsv[u] = (t < nv) ? raj[tc].w : 0.0f;
+          }
+#pragma unroll
+          for (int u = 0; u < XU; ++u) {
+            const int t = t0 + u * TSTEP;
+            if (t < Q) {
+              float fx[8];
+              unpack8(xv[u], fx);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) fx[e] *= xsv[u];
+#pragma unroll
+              for (int rr = 0; rr < R; ++rr) {
+                const int i = t * R + rr;
+                const float4 w0 = *reinterpret_cast<const float4*>(&wx[rr * P + xch * 8]);
+                const float4 w1 = *reinterpret_cast<const float4*>(&wx[rr * P + xch * 8 + 4]);
+                const float xr[8] = {fx[0] * w0.x, fx[1] * w0.y, fx[2] * w0.z, fx[3] * w0.w,
+                                     fx[4] * w1.x, fx[5] * w1.y, fx[6] * w1.z, fx[7] * w1.w};
+                sts128(sX + sw128(i, xch, kRows * 128), pack8(xr));
+              }
+            }
+          }
+        }
+      }
     }
     load_phase ^= 1;
     fence_async_smem();
@@ -845,35 +940,33 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
     if (tid == 0 && has_next) issue_x(j + 1);  // x staging is consumed
 
     // ---- MMA_A: S = Ct Bt^T; fast tiles also Y = Ct (e^m h+) and H = X'^T Bt
-    if (tid == 0) {
+    if (warp == 0) {
       if constexpr (FULL) {
 #pragma unroll
         for (int k = 0; k < N / 16; ++k) {
           const uint32_t koff = (uint32_t)(k >> 2) * (kRows * 128) + (uint32_t)(k & 3) * 32;
-          mma_ss(tmem + C::TM_S, sdesc(sCT + koff, 16, 1024), sdesc(sBT + koff, 16, 1024), C::ID_S, k > 0);
+          mma_ss_w(tmem + C::TM_S, sdesc(sCT + koff, 16, 1024), sdesc(sBT + koff, 16, 1024), C::ID_S, k > 0);
         }
         if (fast) {
 #pragma unroll
           for (int k = 0; k < N / 16; ++k) {
             const uint32_t aoff2 = (uint32_t)(k >> 2) * (kRows * 128) + (uint32_t)(k & 3) * 32;
             const uint32_t boff = (uint32_t)(k >> 2) * (P * 128) + (uint32_t)(k & 3) * 32;
-            mma_ss(tmem + C::TM_Y, sdesc(sCT + aoff2, 16, 1024), sdesc(sH + boff, 16, 1024), C::ID_Y3, k > 0);
+            mma_ss_w(tmem + C::TM_Y, sdesc(sCT + aoff2, 16, 1024), sdesc(sH + boff, 16, 1024), C::ID_Y3, k > 0);
           }
         }
       }
       if (!FULL || fast) {
 #pragma unroll
         for (int k = 0; k < kRows / 16; ++k)
-          mma_ss(tmem + C::TM_H, sdesc(sX + k * 2048, kRows * 128, 1024), sdesc(sBT + k * 2048, kRows * 128, 1024),
+          mma_ss_w(tmem + C::TM_H, sdesc(sX + k * 2048, kRows * 128, 1024), sdesc(sBT + k * 2048, kRows * 128, 1024),
                  C::ID_H, k > 0);
       }
-      mma_commit(mma_bar);
+      mma_commit_w(mma_bar);
     }
     // while the tensor cores run: next tile's coefficients and rotation table
     if (has_next) {
-      store_coefs(par ^ 1);
-      __syncthreads();
-      tile_prep(j + 1, par ^ 1);
+      angle_prep(j + 1, par ^ 1);
       if (j + 2 < j1) load_coefs(j + 2);
     }
     if (tid == 0 && !FULL) seg_logdec += scal(par)[1];
@@ -963,34 +1056,38 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
     if constexpr (FULL) {
       // ---- MMA_B: [exact: Y = Ct' h+], Y += S' X', [exact: H = X'^T Bt']
       bool ok = true;
-      if (tid == 0) {
+      if (warp == 0) {
         if (!fast) {
 #pragma unroll
           for (int k = 0; k < N / 16; ++k) {
             const uint32_t aoff2 = (uint32_t)(k >> 2) * (kRows * 128) + (uint32_t)(k & 3) * 32;
             const uint32_t boff = (uint32_t)(k >> 2) * (P * 128) + (uint32_t)(k & 3) * 32;
-            mma_ss(tmem + C::TM_Y, sdesc(sCT + aoff2, 16, 1024), sdesc(sH + boff, 16, 1024), C::ID_Y3, k > 0);
+            mma_ss_w(tmem + C::TM_Y, sdesc(sCT + aoff2, 16, 1024), sdesc(sH + boff, 16, 1024), C::ID_Y3, k > 0);
           }
         }
 #pragma unroll
         for (int k = 0; k < kRows / 16; ++k)
-          mma_ts(tmem + C::TM_Y, tmem + C::TM_S + 8 * k, sdesc(sX + k * 2048, kRows * 128, 1024), C::ID_Y2, 1);
+          mma_ts_w(tmem + C::TM_Y, tmem + C::TM_S + 8 * k, sdesc(sX + k * 2048, kRows * 128, 1024), C::ID_Y2, 1);
         if (!fast) {
 #pragma unroll
           for (int k = 0; k < kRows / 16; ++k)
-            mma_ss(tmem + C::TM_H, sdesc(sX + k * 2048, kRows * 128, 1024),
+            mma_ss_w(tmem + C::TM_H, sdesc(sX + k * 2048, kRows * 128, 1024),
                    sdesc(sBT + k * 2048, kRows * 128, 1024), C::ID_H, k > 0);
         }
-        mma_commit(mma_bar);
-        ok = mbar_wait(mma_bar, mma_phase);
+        mma_commit_w(mma_bar);
+        if (!fast && lane == 0) ok = mbar_wait(mma_bar, mma_phase);
       }
+      y_phase = mma_phase;
       mma_phase ^= 1;
-      if (__syncthreads_or(!ok)) {
-        failed = true;
-        break;
-      }
-      tc_fence_after();
+      // fast tile: MMA_B reads only TMEM S and sX, so warps 4-7 go on to the next tile's B, C
+      // rows at once and warps 0-3 wait for it at the top of the next X phase
+      y_pending = fast;
       if (!fast) {
+        if (__syncthreads_or(!ok)) {
+          failed = true;
+          break;
+        }
+        tc_fence_after();
         if (tid == 0 && has_next) issue_bc(j + 1);
         if (state_warp) state_update(scal(par)[0], 1.0f, hnext);
         fence_async_smem();
@@ -1002,7 +1099,15 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
   }
   if constexpr (FULL) {
     if (!failed && j0 < j1) {
-      if (!state_warp) epilogue(j1 - 1, (int)((j1 - 1 - j0) & 1));
+      bool ok = true;
+      if (y_pending) {
+        ok = mbar_wait(mma_bar, y_phase);
+        tc_fence_after();
+      }
+      if (ok)
+        epilogue(j1 - 1, (int)((j1 - 1 - j0) & 1));
+      else
+        set_status(p.status, M3_ERR_TIMEOUT);
     }
   }
 

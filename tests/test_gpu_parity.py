@@ -152,6 +152,23 @@ def test_decode_layer_shape_b16():
     check_decode(inp, 6, st)
 
 
+def test_decode_ring_wraps():
+    # 1024 (batch, head) units: every CTA walks about seven units through its ring of stages,
+    # so each stage is refilled at least once; R = 3 runs the rank-4 kernel with a short rank
+    shape = dict(b=64, L=3, H=16, P=16, N=16, R=3, G=4)
+    inp = make_inputs(dtype="bf16", seed=120, extras=True, **shape)
+    st = make_state(64, 16, 16, 16, 3, seed=121)
+    check_decode(inp, 3, st)
+
+
+def test_decode_large_state_single_stage():
+    # a 128 KiB state tile leaves room for one stage only: the one-unit-per-CTA decode kernel
+    shape = dict(b=2, L=3, H=3, P=256, N=128, R=2, G=1)
+    inp = make_inputs(dtype="bf16", seed=122, extras=True, **shape)
+    st = make_state(2, 3, 256, 128, 2, seed=123)
+    check_decode(inp, 3, st)
+
+
 def test_prefill_then_decode_continues():
     shape = dict(b=2, L=40, H=4, P=64, N=64, R=2, G=1)
     inp = make_inputs(dtype="bf16", seed=107, extras=True, **shape)
