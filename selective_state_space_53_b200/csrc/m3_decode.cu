@@ -268,44 +268,49 @@ __global__ void __launch_bounds__(kThreads, 3) decode_kernel(Params p) {
 }
 
 // ------------------------------------------------------------------ ring form
-// Persistent form: one CTA per SM walks a contiguous range of (batch, head) units, ordered
-// head-major so that the per-head weights change at most a few times per CTA, and keeps
-// `stages` units in flight: while it updates unit i, the TMA engine brings the state tiles and
-// raw token operands of units i+1 .. i+stages-1 into a ring of shared-memory stages.  The
-// updated state goes straight from registers to HBM, so the copy engine only ever reads.
+// Persistent form: each CTA walks a contiguous range of (batch, head) units, ordered head-major
+// so that the per-head weights change at most a few times per CTA.  A unit's state tile is
+// taken in `split` blocks of N / split rows (the readouts are summed over the blocks in shared
+// memory), and the CTA keeps `stages` blocks in flight: while it updates one, the TMA engine
+// brings the next blocks (state rows and raw token operands) into a ring of shared-memory
+// stages.  Blocks are sized so that two CTAs fit per SM where possible, one CTA's
+// operand staging and barriers overlapping the other's arithmetic.  The updated state goes
+// straight from registers to HBM, so the copy engine only ever reads.
 
 constexpr int kMaxStages = 6;
-constexpr int kRingThreads = 256;
-constexpr int kRingQuads = 1;  // 4-column quads per thread
-constexpr uint32_t kCopyChunk = 0;  // bytes per bulk copy of the state tile (0: one copy)
+constexpr int kRingThreads = 512;
+constexpr int kRingCtas = kRingThreads <= 256 ? 2 : 1;  // CTAs per SM the registers allow
+constexpr int kRingMinStages = 2;  // stages a plan must fit before a larger split is tried
 
 struct RingPlan {
-  int stages;
+  int stages, split, ctas_per_sm;
   uint32_t stage_bytes;
-  // byte offsets inside a stage: state tile, raw B_t, raw C_t, carry_B, raw x_t, carry_x,
-  // theta_t, and the three per-unit scalars dt, A, lam
+  // byte offsets inside a stage: state rows of the block, raw B_t, raw C_t, carry_B, raw x_t,
+  // carry_x, theta_t, and the three per-unit scalars dt, A, lam
   uint32_t o_st, o_b, o_c, o_cb, o_x, o_cx, o_th, o_sc;
-  // byte offsets of the single-buffered arrays after the ring: this unit's biased B, C and
+  // byte offsets of the single-buffered arrays after the ring: the block's biased B, C and the
   // MIMO branches, the rotation table and coefficients, the weights of the current head
-  // (bias_B, bias_C, W_x, W_o) and the per-pair-group partial readouts
+  // (bias_B, bias_C, W_x, W_o) and the per-pair-group partial readouts of every block
   uint32_t o_bbc, o_bbp, o_cbb, o_xc, o_xp, o_xr, o_cs, o_coef, o_wb, o_wc, o_wx, o_wo, o_red, o_bar;
   uint32_t total;
 };
 
-// thread (pq, kg) of the ring kernel: column quads pq + c * P / (4 * CQ), pairs kg, kg + KG, ...
-__host__ __device__ inline int ring_pq(int P) { return P / (4 * kRingQuads); }
-__host__ __device__ inline int ring_kg(int P, int N) {
+// thread (pq, kg): columns 4 pq .. 4 pq + 3, rotation pairs kg, kg + KG, ... of the block
+__host__ __device__ inline int ring_pq(int P) { return P / 4; }
+__host__ __device__ inline int ring_kg(int P, int NB) {
   const int kg = kRingThreads / ring_pq(P);
-  return kg < N / 2 ? kg : N / 2;
+  return kg < NB / 2 ? kg : NB / 2;
 }
 
 __host__ __device__ inline uint32_t pad16(uint32_t x) { return (x + 15u) & ~15u; }
 
-inline RingPlan ring_plan(int P, int N, int R, bool bf16, int max_bytes) {
+inline RingPlan ring_plan(int P, int N, int R, bool bf16, int split, int max_bytes) {
   const uint32_t esz = bf16 ? 2u : 4u;
+  const int NB = N / split;
   RingPlan rp{};
+  rp.split = split;
   uint32_t o = 0;
-  rp.o_st = o; o += pad16((uint32_t)N * P * 4);
+  rp.o_st = o; o += pad16((uint32_t)NB * P * 4);
   rp.o_b = o;  o += pad16((uint32_t)R * N * esz);
   rp.o_c = o;  o += pad16((uint32_t)R * N * esz);
   rp.o_cb = o; o += pad16((uint32_t)R * N * 4);
@@ -315,19 +320,19 @@ inline RingPlan ring_plan(int P, int N, int R, bool bf16, int max_bytes) {
   rp.o_sc = o; o += 16;
   rp.stage_bytes = (o + 127u) & ~127u;
   uint32_t f = 0;
-  rp.o_bbc = f; f += pad16((uint32_t)R * N * 4);
-  rp.o_bbp = f; f += pad16((uint32_t)R * N * 4);
-  rp.o_cbb = f; f += pad16((uint32_t)R * N * 4);
+  rp.o_bbc = f; f += pad16((uint32_t)R * NB * 4);
+  rp.o_bbp = f; f += pad16((uint32_t)R * NB * 4);
+  rp.o_cbb = f; f += pad16((uint32_t)R * NB * 4);
   rp.o_xc = f;  f += pad16((uint32_t)R * P * 4);
   rp.o_xp = f;  f += pad16((uint32_t)R * P * 4);
   rp.o_xr = f;  f += pad16((uint32_t)P * 4);
-  rp.o_cs = f;  f += pad16((uint32_t)N / 2 * 8);
+  rp.o_cs = f;  f += pad16((uint32_t)NB / 2 * 8);
   rp.o_coef = f; f += 16;
   rp.o_wb = f; f += pad16((uint32_t)R * N * 4);
   rp.o_wc = f; f += pad16((uint32_t)R * N * 4);
   rp.o_wx = f; f += pad16((uint32_t)R * P * 4);
   rp.o_wo = f; f += pad16((uint32_t)R * P * 4);
-  rp.o_red = f; f += pad16((uint32_t)ring_kg(P, N) * P * 4);
+  rp.o_red = f; f += pad16((uint32_t)split * ring_kg(P, NB) * P * 4);
   rp.o_bar = f; f += 8 * kMaxStages;
   const int room = max_bytes - (int)f;
   int st = room > 0 ? room / (int)rp.stage_bytes : 0;
@@ -356,14 +361,17 @@ __device__ __forceinline__ float stage_in(const unsigned char* base, int i) {
 }
 
 template <int RT, bool BF16>
-__global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, RingPlan rp) {
+__global__ void __launch_bounds__(kRingThreads, kRingCtas) decode_ring_kernel(Params p, RingPlan rp) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int tid = threadIdx.x;
   const int H = p.H, P = p.P, N = p.N, R = p.R, G = p.G;
+  const int SPL = rp.split;
+  const int NB = N / SPL;  // state rows per block
   const int64_t nb = p.b;
   const int64_t U = nb * H;
-  const int64_t u0 = (int64_t)blockIdx.x * U / gridDim.x;
-  const int64_t u1 = (int64_t)(blockIdx.x + 1) * U / gridDim.x;
+  // blocks v = unit * SPL + block index; this CTA takes the blocks of units [u0, u1)
+  const int64_t v0 = (int64_t)blockIdx.x * U / gridDim.x * SPL;
+  const int64_t v1 = (int64_t)(blockIdx.x + 1) * U / gridDim.x * SPL;
   const int S = rp.stages;
   constexpr uint32_t esz = BF16 ? 2u : 4u;
   const uint32_t sbase = smem_u32(smem);
@@ -383,23 +391,22 @@ __global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, 
   const uint32_t bar0 = sbase + rp.o_bar;
 
   // unit u = head-major index: head u / b, sequence u % b
-  auto issue = [&](int64_t u, int s) {
+  auto issue = [&](int64_t v, int s) {
+    const int64_t u = v / SPL;
+    const int blk = (int)(v % SPL);
     const int64_t bi = u % nb;
     const int hi = (int)(u / nb);
     const int g = hi / (H / G);
     const int64_t bh = bi * H + hi;
     const uint32_t st = sbase + (uint32_t)s * rp.stage_bytes;
     const uint32_t bar = bar0 + 8u * s;
-    const uint32_t n_st = (uint32_t)N * P * 4, n_b = (uint32_t)R * N * esz, n_cb = (uint32_t)R * N * 4;
+    const uint32_t n_st = (uint32_t)NB * P * 4, n_b = (uint32_t)R * N * esz, n_cb = (uint32_t)R * N * 4;
     const uint32_t n_x = (uint32_t)P * esz, n_cx = (uint32_t)P * 4, n_th = (uint32_t)N / 2 * 4;
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
                  "r"(n_st + 2 * n_b + n_cb + n_x + n_cx + n_th)
                  : "memory");
     const int64_t bc = ((bi * G + g) * R) * (int64_t)N;
-    const uint32_t chunk = kCopyChunk ? kCopyChunk : n_st;
-    for (uint32_t c = 0; c < n_st; c += chunk)
-      bulk_g2s(st + rp.o_st + c, reinterpret_cast<const unsigned char*>(p.h + bh * N * P) + c,
-               n_st - c < chunk ? n_st - c : chunk, bar);
+    bulk_g2s(st + rp.o_st, p.h + (bh * N + (int64_t)blk * NB) * P, n_st, bar);
     bulk_g2s(st + rp.o_b, static_cast<const unsigned char*>(p.B) + bc * esz, n_b, bar);
     bulk_g2s(st + rp.o_c, static_cast<const unsigned char*>(p.C) + bc * esz, n_b, bar);
     bulk_g2s(st + rp.o_cb, p.carry_B + bh * R * N, n_cb, bar);
@@ -434,32 +441,34 @@ __global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, 
     for (int s = 0; s < S; ++s)
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 2;" ::"r"(bar0 + 8u * s));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    for (int s = 0; s < S && u0 + s < u1; ++s) issue(u0 + s, s);
+    for (int s = 0; s < S && v0 + s < v1; ++s) issue(v0 + s, s);
   }
   __syncthreads();
 
-  // thread (pq, kg): column quads pq + c * P / (4 * CQ) for c < CQ, rotation pairs kg, kg + KG, ...
-  constexpr int CQ = kRingQuads;
   const int PQ = ring_pq(P);
-  const int KG = ring_kg(P, N);
+  const int KG = ring_kg(P, NB);
   const int pq = tid % PQ;
   const int kg = tid / PQ;
+  constexpr int CQ = 1;  // 4-column quads per thread (the compute below takes any count)
   int cur_h = -1;
   float Dh = 0.0f;
   uint32_t phases = 0;  // bit s: parity of the next completion of stage s
   int s = 0;
   bool ok = true;
-  int64_t u = u0;
-  for (; u < u1; ++u) {
+  int64_t v = v0;
+  for (; v < v1; ++v) {
     const uint32_t par = (phases >> s) & 1u;
     phases ^= 1u << s;
+    const int64_t u = v / SPL;
+    const int blk = (int)(v % SPL);
+    const bool last_blk = blk == SPL - 1;
     const int64_t bi = u % nb;
     const int hi = (int)(u / nb);
     const int64_t bh = bi * H + hi;
     const unsigned char* stg = smem + (size_t)s * rp.stage_bytes;
     if (hi != cur_h) {  // weights of a new head (uniform: every thread sees the same unit)
       cur_h = hi;
-      __syncthreads();  // the previous unit's output step has read W_o
+      __syncthreads();  // the previous block's update has read W_o
       const float* biasB = p.bias_B ? p.bias_B + (int64_t)hi * R * N : nullptr;
       const float* biasC = p.bias_C ? p.bias_C + (int64_t)hi * R * N : nullptr;
       const float* Wx = p.W_x ? p.W_x + (int64_t)hi * R * P : nullptr;
@@ -477,35 +486,28 @@ __global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, 
     }
     ok = wait(s, par);
     if (ok) {
-      // ---- operands of this unit
+      // ---- operands of this block
       const float* sc = reinterpret_cast<const float*>(stg + rp.o_sc);
       const float* cBs = reinterpret_cast<const float*>(stg + rp.o_cb);
       const float* cxs = reinterpret_cast<const float*>(stg + rp.o_cx);
       const float* ths = reinterpret_cast<const float*>(stg + rp.o_th);
-      float* cBg = p.carry_B + bh * R * N;
-      float* cxg = p.carry_x + bh * P;
-      for (int i = tid; i < R * N; i += kRingThreads) {
-        const float bb = wb[i];
-        const float braw = stage_in<BF16>(stg + rp.o_b, i);
-        bbc[i] = braw + bb;
-        bbp[i] = cBs[i] + bb;
-        cbb[i] = stage_in<BF16>(stg + rp.o_c, i) + wc[i];
-        cBg[i] = braw;  // new carry: this token's raw B
+      const int n0 = blk * NB;
+      for (int i = tid; i < R * NB; i += kRingThreads) {
+        const int r = i / NB, n = n0 + i % NB;
+        const float bb = wb[r * N + n];
+        bbc[i] = stage_in<BF16>(stg + rp.o_b, r * N + n) + bb;
+        bbp[i] = cBs[r * N + n] + bb;
+        cbb[i] = stage_in<BF16>(stg + rp.o_c, r * N + n) + wc[r * N + n];
       }
       for (int i = tid; i < R * P; i += kRingThreads) {
         const float w = wx[i];
         xc[i] = stage_in<BF16>(stg + rp.o_x, i % P) * w;
         xp[i] = cxs[i % P] * w;
       }
-      for (int pp = tid; pp < P; pp += kRingThreads) {
-        const float xv = stage_in<BF16>(stg + rp.o_x, pp);
-        xr[pp] = xv;
-        cxg[pp] = xv;  // new carry: this token's raw x
-      }
       const float delta = sc[0];
-      for (int k = tid; k < N / 2; k += kRingThreads) {
+      for (int k = tid; k < NB / 2; k += kRingThreads) {
         float sn, cn;
-        sincosf(delta * ths[k], &sn, &cn);
+        sincosf(delta * ths[n0 / 2 + k], &sn, &cn);
         cs[k] = make_float2(cn, sn);
       }
       if (tid == 0) {
@@ -514,17 +516,29 @@ __global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, 
         coef[1] = (1.0f - lm) * delta;
         coef[2] = lm * delta;
       }
+      if (last_blk) {
+        // the unit's last block: every block's copy of the old carry has landed, so the new
+        // carry (this token's raw B and x) may overwrite it
+        float* cBg = p.carry_B + bh * R * N;
+        float* cxg = p.carry_x + bh * P;
+        for (int i = tid; i < R * N; i += kRingThreads) cBg[i] = stage_in<BF16>(stg + rp.o_b, i);
+        for (int pp = tid; pp < P; pp += kRingThreads) {
+          const float xv = stage_in<BF16>(stg + rp.o_x, pp);
+          xr[pp] = xv;
+          cxg[pp] = xv;
+        }
+      }
     }
     if (__syncthreads_or(!ok)) {
       ok = false;
-      phases ^= 1u << s;  // unit u's copies count as outstanding again
+      phases ^= 1u << s;  // block v's copies count as outstanding again
       break;
     }
-    // ---- state update of the thread's column quads over its rotation pairs
+    // ---- state update of the thread's 4 columns over its rotation pairs of the block
     if (kg < KG) {
       const float alpha = coef[0], bp = coef[1], gm = coef[2];
       const float* stt = reinterpret_cast<const float*>(stg + rp.o_st);
-      float* hg = p.h + bh * N * P;
+      float* hg = p.h + (bh * N + (int64_t)blk * NB) * P;
       int pc[CQ];
 #pragma unroll
       for (int c = 0; c < CQ; ++c) pc[c] = 4 * pq + c * (P / CQ);
@@ -543,7 +557,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, 
           }
         }
 #pragma unroll 2
-      for (int k = kg; k < N / 2; k += KG) {
+      for (int k = kg; k < NB / 2; k += KG) {
         float4 s0[CQ], s1[CQ];
 #pragma unroll
         for (int c = 0; c < CQ; ++c) {
@@ -554,8 +568,8 @@ __global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, 
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
           if (r < R) {
-            const float2 bcv = *reinterpret_cast<const float2*>(bbc + r * N + 2 * k);
-            const float2 bqv = *reinterpret_cast<const float2*>(bbp + r * N + 2 * k);
+            const float2 bcv = *reinterpret_cast<const float2*>(bbc + r * NB + 2 * k);
+            const float2 bqv = *reinterpret_cast<const float2*>(bbp + r * NB + 2 * k);
 #pragma unroll
             for (int c = 0; c < CQ; ++c) {
               const float xc4[4] = {Xc[r][c].x, Xc[r][c].y, Xc[r][c].z, Xc[r][c].w};
@@ -592,7 +606,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, 
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
           if (r < R) {
-            const float2 cc = *reinterpret_cast<const float2*>(cbb + r * N + 2 * k);
+            const float2 cc = *reinterpret_cast<const float2*>(cbb + r * NB + 2 * k);
 #pragma unroll
             for (int c = 0; c < CQ; ++c)
 #pragma unroll
@@ -600,7 +614,7 @@ __global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, 
           }
         }
       }
-      // this pair group's part of sum_r W_o[r] * readout_r; summed over the groups after the barrier
+      // this pair group's part of sum_r W_o[r] * readout_r; summed over groups and blocks later
 #pragma unroll
       for (int c = 0; c < CQ; ++c) {
         float o[4] = {0.f, 0.f, 0.f, 0.f};
@@ -613,30 +627,33 @@ __global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, 
             o[2] = fmaf(w4.z, Y[r][c][2], o[2]);
             o[3] = fmaf(w4.w, Y[r][c][3], o[3]);
           }
-        *reinterpret_cast<float4*>(red + kg * P + pc[c]) = make_float4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<float4*>(red + (blk * KG + kg) * P + pc[c]) = make_float4(o[0], o[1], o[2], o[3]);
       }
     }
-    __syncthreads();  // stage s is read; the readouts are summed
-    if (tid == 0 && u + S < u1) issue(u + S, s);
-    // ---- y = sum_r W_o[r] * readout_r + D x
-    for (int pp = tid; pp < P; pp += kRingThreads) {
-      float acc0 = 0.0f, acc1 = 0.0f;
-      int q = 0;
-      for (; q + 1 < KG; q += 2) {
-        acc0 += red[q * P + pp];
-        acc1 += red[(q + 1) * P + pp];
+    __syncthreads();  // stage s is read; the block's readouts are in place
+    if (tid == 0 && v + S < v1) issue(v + S, s);
+    if (last_blk) {
+      // ---- y = sum_r W_o[r] * readout_r + D x, the readouts summed over groups and blocks
+      const int nq = SPL * KG;
+      for (int pp = tid; pp < P; pp += kRingThreads) {
+        float acc0 = 0.0f, acc1 = 0.0f;
+        int q = 0;
+        for (; q + 1 < nq; q += 2) {
+          acc0 += red[q * P + pp];
+          acc1 += red[(q + 1) * P + pp];
+        }
+        if (q < nq) acc0 += red[q * P + pp];
+        store_out<BF16>(p.y, bh * P + pp, fmaf(Dh, xr[pp], acc0 + acc1));
       }
-      if (q < KG) acc0 += red[q * P + pp];
-      store_out<BF16>(p.y, bh * P + pp, fmaf(Dh, xr[pp], acc0 + acc1));
     }
     s = (s + 1 == S) ? 0 : s + 1;
   }
   if (!ok) {
     // give up: wait (bounded) for the copies still in flight, then report
     if (tid == 0) {
-      for (int64_t v = u; v < u1 && v < u + S; ++v) {
-        const int sv = (int)((v - u0) % S);
-        wait(sv, (phases >> sv) & 1u);
+      for (int64_t w = v; w < v1 && w < v + S; ++w) {
+        const int sw = (int)((w - v0) % S);
+        wait(sw, (phases >> sw) & 1u);
       }
       set_status(p.status, M3_ERR_TIMEOUT);
     }
@@ -666,7 +683,7 @@ size_t decode_smem_bytes(int P, int N, int R) {
 }
 
 struct DeviceLimits {
-  int sms = 0, smem_optin = 0;
+  int sms = 0, smem_optin = 0, smem_sm = 0;
 };
 // SM count and opt-in shared memory per block of the current device (cached per device).
 DeviceLimits device_limits() {
@@ -675,11 +692,13 @@ DeviceLimits device_limits() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DeviceLimits{};
   DeviceLimits& d = cache[dev];
   if (d.sms == 0) {
-    int sms = 0, optin = 0;
+    int sms = 0, optin = 0, per_sm = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess)
       return DeviceLimits{};
     d.smem_optin = optin;
+    d.smem_sm = per_sm;
     d.sms = sms;
   }
   return d;
@@ -701,12 +720,27 @@ cudaError_t launch_ring_rt(const Params& p, const RingPlan& rp, unsigned grid, c
   return cudaGetLastError();
 }
 
-// The ring form needs two stages on chip at least.
+// The ring form needs two stages on chip at least.  Preferred: two CTAs per SM with the fewest
+// row blocks per unit; else one CTA per SM with the fewest blocks.
 bool ring_plan_for(const Params& p, RingPlan* out) {
   const DeviceLimits d = device_limits();
   if (d.sms == 0) return false;
-  *out = ring_plan(p.P, p.N, p.R, p.dtype == M3_BF16, d.smem_optin);
-  return out->stages >= 2;
+  const bool bf16 = p.dtype == M3_BF16;
+  for (int min_stages = kRingMinStages; min_stages >= 2; --min_stages)
+    for (int ctas = kRingCtas; ctas >= 1; --ctas) {
+      // 1 KiB of each SM's shared memory is reserved per resident CTA
+      const int room = ctas == 1 ? d.smem_optin : d.smem_sm / ctas - 1024;
+      for (int split = 1; split <= 4; split *= 2) {
+        if (p.N % (2 * split) != 0 || (p.N / split) % 8 != 0) break;
+        RingPlan rp = ring_plan(p.P, p.N, p.R, bf16, split, room < d.smem_optin ? room : d.smem_optin);
+        if (rp.stages >= min_stages) {
+          rp.ctas_per_sm = ctas;
+          *out = rp;
+          return true;
+        }
+      }
+    }
+  return false;
 }
 
 }  // namespace
@@ -721,8 +755,8 @@ cudaError_t launch_decode(const Params& p, cudaStream_t stream) {
   RingPlan rp;
   if (ring_plan_for(p, &rp)) {
     const int64_t units = p.b * p.H;
-    const int sms = device_limits().sms;
-    const unsigned grid = (unsigned)(units < sms ? units : sms);
+    const int64_t slots = (int64_t)device_limits().sms * rp.ctas_per_sm;
+    const unsigned grid = (unsigned)(units < slots ? units : slots);
     if (p.R <= 1) return launch_ring_rt<1>(p, rp, grid, stream);
     if (p.R <= 2) return launch_ring_rt<2>(p, rp, grid, stream);
     if (p.R <= 4) return launch_ring_rt<4>(p, rp, grid, stream);

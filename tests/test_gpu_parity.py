@@ -161,8 +161,9 @@ def test_decode_ring_wraps():
     check_decode(inp, 3, st)
 
 
-def test_decode_large_state_single_stage():
-    # a 128 KiB state tile leaves room for one stage only: the one-unit-per-CTA decode kernel
+def test_decode_large_state_row_blocks():
+    # a 128 KiB state tile is taken in row blocks (four per unit at two CTAs per SM): the
+    # readout sums over the blocks and the carry is rewritten after the unit's last block
     shape = dict(b=2, L=3, H=3, P=256, N=128, R=2, G=1)
     inp = make_inputs(dtype="bf16", seed=122, extras=True, **shape)
     st = make_state(2, 3, 256, 128, 2, seed=123)
