@@ -37,10 +37,10 @@ WORKLOAD = "p1_layer"
 DECODE_WORKLOAD = "decode_b128"
 L2_BYTES = 126 * 1024 * 1024
 
-# dram bytes (read + write) per launch of the prefill kernel from the ncu capture
-# summarised in profiles/scan_tc_p1_layer.md; None until that capture matches the
-# current kernel.
-PREFILL_DRAM_BYTES_PER_LAUNCH = None
+# dram bytes (read + write) of one m3_scan_fwd on p1_layer (state pass + full pass) from the
+# ncu capture summarised in profiles/scan_tc_p1_layer.md; set to None whenever the kernel
+# changes until a new capture is taken.
+PREFILL_DRAM_BYTES_PER_LAUNCH = 61606144
 
 
 def log(*a):
@@ -291,7 +291,7 @@ def run_ours(args):
         "workload": "p1_layer m3_scan_fwd b4 L2048 H24 P64 N64 R2",
         "tokens_per_s": cfg["b"] * cfg["L"] / (pf_ms / 1e3),
         "ms_per_launch": pf_ms,
-        "hbm_gbs": pbytes / (pf_ms / 1e-3) / 1e9 * 1e-6 * 1e6 if False else pbytes / (pf_ms * 1e-3) / 1e9,
+        "hbm_gbs": pbytes / (pf_ms * 1e-3) / 1e9,
         "hbm_frac_of_measured": pbytes / (pf_ms * 1e-3) / 1e9 / peaks["hbm"],
         "tflops": pflops / (pf_ms * 1e-3) / 1e12,
         "tensor_frac_of_measured_burst": pflops / (pf_ms * 1e-3) / 1e12 / peaks["bf16"],
@@ -303,7 +303,7 @@ def run_ours(args):
     ten_frac = prefill["tensor_frac_of_measured_burst"]
     bound = "hbm" if hbm_frac >= ten_frac else "tensor"
     roofline = {
-        "kernel": "scan_tc_kernel (m3_scan_fwd)",
+        "kernel": "m3_scan_fwd (scan_tc_kernel: state pass + full pass)",
         "bound": bound,
         "achieved": prefill["hbm_gbs"] if bound == "hbm" else prefill["tflops"],
         "peak": peaks["hbm"] if bound == "hbm" else peaks["bf16"],
