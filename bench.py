@@ -315,6 +315,7 @@ def run_ours(args):
     }
 
     decode = run_decode(args, device, peaks) if not args.no_decode else None
+    stack = run_stack(args, device, peaks) if not args.no_stack else None
     e2e = run_e2e(args, inp, tok_inp, device, world) if not args.no_e2e else None
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -323,7 +324,7 @@ def run_ours(args):
         "config": {"workload": "p1_layer: m3_scan_fwd over b4 x L2048 (H24 P64 N64 R2, chunk 32) + 1 m3_decode_step",
                    "global_batch": cfg["b"] * world, "seq_len": cfg["L"], "parallelism": f"dp{world}",
                    "l2": f"ring of {n_sets} input sets ({n_sets * per_set / 2**20:.0f} MiB) > L2"},
-        "roofline": roofline, "prefill": prefill, "decode": decode, "e2e": e2e,
+        "roofline": roofline, "prefill": prefill, "decode": decode, "stack": stack, "e2e": e2e,
         "gpu_launches": gpu_launches, "clocks": clk.summary(),
     }
     if rank == 0 and not args.no_cpu:
@@ -376,6 +377,56 @@ def run_decode(args, device, peaks):
             "tokens_per_s": cfg["b"] / (ms * 1e-3), "us_per_step": ms * 1e3,
             "hbm_gbs": by / (ms * 1e-3) / 1e9, "hbm_frac_of_measured": by / (ms * 1e-3) / 1e9 / peaks["hbm"],
             "tflops": fl / (ms * 1e-3) / 1e12, "algorithmic_bytes": by}
+
+
+def run_stack(args, device, peaks):
+    """The 12-layer stack of the page-1 language-model shape (b8 L4096): the whole forward
+    (torch projections around the libm3 core) and its 12 core calls alone."""
+    import torch
+    from selective_state_space_53_b200 import m3
+    from selective_state_space_53_b200.inputs import CONFIGS
+    from selective_state_space_53_b200.stack import Mamba3Stack, StackShape
+    cfg = dict(CONFIGS["p1_stack"])
+    shape = StackShape(layers=cfg["layers"], H=cfg["H"], P=cfg["P"], N=cfg["N"], R=cfg["R"], G=cfg["G"])
+    b, L = cfg["b"], cfg["L"]
+    stack = Mamba3Stack(shape, seed=1002, device=device)
+    gen = torch.Generator(device="cpu").manual_seed(2002)
+    u = torch.randn(b, L, shape.d_model, generator=gen).to(torch.bfloat16).to(device)
+    stream = torch.cuda.current_stream()
+    # core operands of every layer, for timing the core calls alone
+    dims = m3.make_dims(b, L, shape.H, shape.P, shape.N, shape.R, shape.G, "bf16")
+    ws = torch.empty(max(m3.m3_scan_workspace_size(dims), 16), dtype=torch.uint8, device=device)
+    ops = [stack.core_inputs(u, layer)[0] for layer in stack.layers]
+    st, keep = m3.state_tensors(dims, device=device)
+    y = torch.empty_like(ops[0]["x"])
+    for _ in range(2):
+        stack.forward(u)
+        for dev in ops:
+            m3.scan(dims, dev, st, y=y, workspace=ws)
+    torch.cuda.synchronize()
+    iters = 3
+    a, c = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(iters):
+        stack.forward(u)
+    c.record(stream)
+    torch.cuda.synchronize()
+    fwd_ms = a.elapsed_time(c) / iters
+    a.record(stream)
+    for _ in range(iters):
+        for dev in ops:
+            m3.scan(dims, dev, st, y=y, workspace=ws)
+    c.record(stream)
+    torch.cuda.synchronize()
+    assert m3.m3_check() == 0
+    core_ms = a.elapsed_time(c) / iters
+    layer_cfg = dict(cfg, dtype="bf16")
+    by = shape.layers * prefill_bytes(layer_cfg)
+    return {"workload": "p1_stack: 12 layers x (b8 L4096, H24 P64 N64 R2), forward prefill; torch projections "
+                        "around the libm3 core",
+            "tokens_per_s": b * L / (fwd_ms * 1e-3), "ms_per_forward": fwd_ms,
+            "core_tokens_per_s": b * L / (core_ms * 1e-3), "core_ms_per_forward": core_ms,
+            "core_hbm_frac_of_measured": by / (core_ms * 1e-3) / 1e9 / peaks["hbm"]}
 
 
 def run_e2e(args, inp, tok_inp, device, world):
@@ -525,6 +576,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle timing")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-stack", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
