@@ -17,9 +17,6 @@ namespace {
 
 constexpr unsigned long long kWaitNs = 2000000000ull;
 
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -87,7 +84,7 @@ inline RingPlan ring_plan(int P, int N, int R, bool bf16, int split, int max_byt
   rp.o_cbb = f; f += pad16((uint32_t)R * NB * 4);
   rp.o_xc = f;  f += pad16((uint32_t)R * P * 4);
   rp.o_xp = f;  f += pad16((uint32_t)R * P * 4);
-  rp.o_xr = f;  f += pad16((uint32_t)2 * P * 4 + 8);  // raw x and D of the last two units
+  rp.o_xr = f;  f += pad16((uint32_t)P * 4);
   rp.o_cs = f;  f += pad16((uint32_t)NB / 2 * 8);
   rp.o_coef = f; f += 16;
   rp.o_wb = f; f += pad16((uint32_t)R * N * 4);
@@ -213,101 +210,89 @@ __global__ void __launch_bounds__(kRingThreads, kRingCtas) decode_ring_kernel(Pa
   const int kg = tid / PQ;
   constexpr int CQ = 1;  // 4-column quads per thread (the compute below takes any count)
   int cur_h = -1;
-  // Threads [0, NY) write y (NY = P rounded up to whole warps, thread 0 also issues the copies);
-  // threads [NY, kRingThreads) stage the next block's operands meanwhile.
-  const int NY = (P + 31) & ~31;
-  // prepare(v): the weights of v's head if they changed, wait for v's stage, then the biased B, C
-  // rows, MIMO branches, rotation table and coefficients of block v, and after a unit's last block
-  // the new carry (every block's copy of the old one has landed by then), its raw x and D.
-  auto prepare = [&](int64_t v, int sv, uint32_t par, int ptid, int nproc, bool all) -> bool {
-    const int64_t u = v / SPL;
-    const int blk = (int)(v % SPL);
-    const int64_t bi = u % nb;
-    const int hi = (int)(u / nb);
-    const int64_t bh = bi * H + hi;
-    const unsigned char* stg = smem + (size_t)sv * rp.stage_bytes;
-    if (hi != cur_h) {  // uniform over the threads that prepare
-      cur_h = hi;
-      const float* biasB = p.bias_B ? p.bias_B + (int64_t)hi * R * N : nullptr;
-      const float* biasC = p.bias_C ? p.bias_C + (int64_t)hi * R * N : nullptr;
-      const float* Wx = p.W_x ? p.W_x + (int64_t)hi * R * P : nullptr;
-      const float* Wo = p.W_o ? p.W_o + (int64_t)hi * R * P : nullptr;
-      for (int i = ptid; i < R * N; i += nproc) {
-        wb[i] = biasB ? biasB[i] : 0.0f;
-        wc[i] = biasC ? biasC[i] : 0.0f;
-      }
-      for (int i = ptid; i < R * P; i += nproc) {
-        wx[i] = Wx ? Wx[i] : 1.0f;
-        wo[i] = Wo ? Wo[i] : 1.0f;
-      }
-      if (all)
-        __syncthreads();
-      else
-        named_bar_sync(1, nproc);
-    }
-    if (!wait(sv, par)) return false;
-    const float* sc = reinterpret_cast<const float*>(stg + rp.o_sc);
-    const float* cBs = reinterpret_cast<const float*>(stg + rp.o_cb);
-    const float* cxs = reinterpret_cast<const float*>(stg + rp.o_cx);
-    const float* ths = reinterpret_cast<const float*>(stg + rp.o_th);
-    const int n0 = blk * NB;
-    for (int i = ptid; i < R * NB; i += nproc) {
-      const int r = i / NB, n = n0 + i % NB;
-      const float bb = wb[r * N + n];
-      bbc[i] = stage_in<BF16>(stg + rp.o_b, r * N + n) + bb;
-      bbp[i] = cBs[r * N + n] + bb;
-      cbb[i] = stage_in<BF16>(stg + rp.o_c, r * N + n) + wc[r * N + n];
-    }
-    for (int i = ptid; i < R * P; i += nproc) {
-      const float w = wx[i];
-      xc[i] = stage_in<BF16>(stg + rp.o_x, i % P) * w;
-      xp[i] = cxs[i % P] * w;
-    }
-    const float delta = sc[0];
-    for (int k = ptid; k < NB / 2; k += nproc) {
-      float sn, cn;
-      sincosf(delta * ths[n0 / 2 + k], &sn, &cn);
-      cs[k] = make_float2(cn, sn);
-    }
-    if (ptid == 0) {
-      const float lm = sc[2];
-      coef[0] = expf(delta * sc[1]);
-      coef[1] = (1.0f - lm) * delta;
-      coef[2] = lm * delta;
-    }
-    if (blk == SPL - 1) {
-      float* cBg = p.carry_B + bh * R * N;
-      float* cxg = p.carry_x + bh * P;
-      float* xru = xr + (u & 1) * (P + 2);
-      for (int i = ptid; i < R * N; i += nproc) cBg[i] = stage_in<BF16>(stg + rp.o_b, i);
-      for (int pp = ptid; pp < P; pp += nproc) {
-        const float xv = stage_in<BF16>(stg + rp.o_x, pp);
-        xru[pp] = xv;
-        cxg[pp] = xv;
-      }
-      if (ptid == 0) xru[P] = p.D ? p.D[hi] : 0.0f;
-    }
-    return true;
-  };
-
+  float Dh = 0.0f;
   uint32_t phases = 0;  // bit s: parity of the next completion of stage s
   int s = 0;
   bool ok = true;
   int64_t v = v0;
-  if (v0 < v1) {
-    phases ^= 1u;
-    ok = prepare(v0, 0, 0u, tid, kRingThreads, true);
-  }
-  if (__syncthreads_or(!ok)) {
-    ok = false;
-    phases ^= 1u;  // block v0's copies count as outstanding again
-  }
-  for (; ok && v < v1; ++v) {
+  for (; v < v1; ++v) {
+    const uint32_t par = (phases >> s) & 1u;
+    phases ^= 1u << s;
     const int64_t u = v / SPL;
     const int blk = (int)(v % SPL);
     const bool last_blk = blk == SPL - 1;
-    const int64_t bh = (u % nb) * H + (int)(u / nb);
+    const int64_t bi = u % nb;
+    const int hi = (int)(u / nb);
+    const int64_t bh = bi * H + hi;
     const unsigned char* stg = smem + (size_t)s * rp.stage_bytes;
+    if (hi != cur_h) {  // weights of a new head (uniform: every thread sees the same unit)
+      cur_h = hi;
+      __syncthreads();  // the previous block's update has read W_o
+      const float* biasB = p.bias_B ? p.bias_B + (int64_t)hi * R * N : nullptr;
+      const float* biasC = p.bias_C ? p.bias_C + (int64_t)hi * R * N : nullptr;
+      const float* Wx = p.W_x ? p.W_x + (int64_t)hi * R * P : nullptr;
+      const float* Wo = p.W_o ? p.W_o + (int64_t)hi * R * P : nullptr;
+      for (int i = tid; i < R * N; i += kRingThreads) {
+        wb[i] = biasB ? biasB[i] : 0.0f;
+        wc[i] = biasC ? biasC[i] : 0.0f;
+      }
+      for (int i = tid; i < R * P; i += kRingThreads) {
+        wx[i] = Wx ? Wx[i] : 1.0f;
+        wo[i] = Wo ? Wo[i] : 1.0f;
+      }
+      Dh = p.D ? p.D[hi] : 0.0f;
+      __syncthreads();
+    }
+    ok = wait(s, par);
+    if (ok) {
+      // ---- operands of this block
+      const float* sc = reinterpret_cast<const float*>(stg + rp.o_sc);
+      const float* cBs = reinterpret_cast<const float*>(stg + rp.o_cb);
+      const float* cxs = reinterpret_cast<const float*>(stg + rp.o_cx);
+      const float* ths = reinterpret_cast<const float*>(stg + rp.o_th);
+      const int n0 = blk * NB;
+      for (int i = tid; i < R * NB; i += kRingThreads) {
+        const int r = i / NB, n = n0 + i % NB;
+        const float bb = wb[r * N + n];
+        bbc[i] = stage_in<BF16>(stg + rp.o_b, r * N + n) + bb;
+        bbp[i] = cBs[r * N + n] + bb;
+        cbb[i] = stage_in<BF16>(stg + rp.o_c, r * N + n) + wc[r * N + n];
+      }
+      for (int i = tid; i < R * P; i += kRingThreads) {
+        const float w = wx[i];
+        xc[i] = stage_in<BF16>(stg + rp.o_x, i % P) * w;
+        xp[i] = cxs[i % P] * w;
+      }
+      const float delta = sc[0];
+      for (int k = tid; k < NB / 2; k += kRingThreads) {
+        float sn, cn;
+        sincosf(delta * ths[n0 / 2 + k], &sn, &cn);
+        cs[k] = make_float2(cn, sn);
+      }
+      if (tid == 0) {
+        const float lm = sc[2];
+        coef[0] = expf(delta * sc[1]);
+        coef[1] = (1.0f - lm) * delta;
+        coef[2] = lm * delta;
+      }
+      if (last_blk) {
+        // the unit's last block: every block's copy of the old carry has landed, so the new
+        // carry (this token's raw B and x) may overwrite it
+        float* cBg = p.carry_B + bh * R * N;
+        float* cxg = p.carry_x + bh * P;
+        for (int i = tid; i < R * N; i += kRingThreads) cBg[i] = stage_in<BF16>(stg + rp.o_b, i);
+        for (int pp = tid; pp < P; pp += kRingThreads) {
+          const float xv = stage_in<BF16>(stg + rp.o_x, pp);
+          xr[pp] = xv;
+          cxg[pp] = xv;
+        }
+      }
+    }
+    if (__syncthreads_or(!ok)) {
+      ok = false;
+      phases ^= 1u << s;  // block v's copies count as outstanding again
+      break;
+    }
     // ---- state update of the thread's 4 columns over its rotation pairs of the block
     if (kg < KG) {
       const float alpha = coef[0], bp = coef[1], gm = coef[2];
@@ -406,33 +391,21 @@ __global__ void __launch_bounds__(kRingThreads, kRingCtas) decode_ring_kernel(Pa
     }
     __syncthreads();  // stage s is read; the block's readouts are in place
     if (tid == 0 && v + S < v1) issue(v + S, s);
-    const int sn = (s + 1 == S) ? 0 : s + 1;
-    bool okp = true;
-    if (v + 1 < v1) {
-      const uint32_t parn = (phases >> sn) & 1u;
-      phases ^= 1u << sn;
-      if (tid >= NY) okp = prepare(v + 1, sn, parn, tid - NY, kRingThreads - NY, false);
-    }
-    if (last_blk && tid < P) {
+    if (last_blk) {
       // ---- y = sum_r W_o[r] * readout_r + D x, the readouts summed over groups and blocks
       const int nq = SPL * KG;
-      const float* xru = xr + (u & 1) * (P + 2);
-      float acc0 = 0.0f, acc1 = 0.0f;
-      int q = 0;
-      for (; q + 1 < nq; q += 2) {
-        acc0 += red[q * P + tid];
-        acc1 += red[(q + 1) * P + tid];
+      for (int pp = tid; pp < P; pp += kRingThreads) {
+        float acc0 = 0.0f, acc1 = 0.0f;
+        int q = 0;
+        for (; q + 1 < nq; q += 2) {
+          acc0 += red[q * P + pp];
+          acc1 += red[(q + 1) * P + pp];
+        }
+        if (q < nq) acc0 += red[q * P + pp];
+        store_out<BF16>(p.y, bh * P + pp, fmaf(Dh, xr[pp], acc0 + acc1));
       }
-      if (q < nq) acc0 += red[q * P + tid];
-      store_out<BF16>(p.y, bh * P + tid, fmaf(xru[P], xru[tid], acc0 + acc1));
     }
-    if (__syncthreads_or(!okp)) {
-      ok = false;
-      phases ^= 1u << sn;  // block v+1's copies count as outstanding again
-      ++v;
-      break;
-    }
-    s = sn;
+    s = (s + 1 == S) ? 0 : s + 1;
   }
   if (!ok) {
     // give up: wait (bounded) for the copies still in flight, then report
