@@ -554,27 +554,50 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
     mbar_init(mma_bar, 1);
     mbar_init(load_bar, 1);
     fence_mbar_init();
-    prefetch_tmap(&tmB);
-    if constexpr (FULL) prefetch_tmap(&tmC);
-    prefetch_tmap(&tmX);
+    if (j0 < j1) {  // the first tile's operands are in flight from the start
+      issue_x(j0);
+      issue_bc(j0);
+    }
   }
-  for (int i = tid; i < R * P; i += kThreads) {
-    wx[i] = p.W_x ? p.W_x[(int64_t)hi * R * P + i] : 1.0f;
-    wo[i] = p.W_o ? p.W_o[(int64_t)hi * R * P + i] : 1.0f;
+  // every global load of the setup is issued before any of them is consumed
+  constexpr int RPW = (R * P + kThreads - 1) / kThreads;
+  float wxv[RPW], wov[RPW];
+#pragma unroll
+  for (int q = 0; q < RPW; ++q) {
+    const int i = tid + q * kThreads;
+    wxv[q] = (i < R * P && p.W_x) ? p.W_x[(int64_t)hi * R * P + i] : 1.0f;
+    wov[q] = (i < R * P && p.W_o) ? p.W_o[(int64_t)hi * R * P + i] : 1.0f;
   }
+  load_coefs(j0);
   const float* biasBg = p.bias_B ? p.bias_B + (int64_t)hi * R * N : nullptr;
   const float* biasCg = p.bias_C ? p.bias_C + (int64_t)hi * R * N : nullptr;
+  // operand staging: B, C rows on all threads; x rows on warps 1-7 (warp 0 prepares the next
+  // tile's coefficients meanwhile)
+  const int xt = tid;
+  constexpr int CHN = N / 8;
+  constexpr int RPI = NT / CHN;  // rows per pass; a multiple of 8 and of R
+  const int tch = xt % CHN;
+  const int tr = (xt / CHN) % R;
+  float bB[8], bC[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    bB[e] = biasBg ? __ldg(biasBg + tr * N + tch * 8 + e) : 0.0f;
+    bC[e] = biasCg ? __ldg(biasCg + tr * N + tch * 8 + e) : 0.0f;
+  }
+#pragma unroll
+  for (int q = 0; q < RPW; ++q) {
+    const int i = tid + q * kThreads;
+    if (i < R * P) {
+      wx[i] = wxv[q];
+      wo[i] = wov[q];
+    }
+  }
   for (int k = tid; k < K2; k += kThreads) base[k] = 0.0;
-  load_coefs(j0);
   store_coefs(0);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = __shfl_sync(kFull, *tmem_slot, 0);
-  if (tid == 0 && j0 < j1) {
-    issue_x(j0);
-    issue_bc(j0);
-  }
   if (j0 < j1) {
     if (warp == 0) coef_prep(j0, 0);
     angle_prep(j0, 0);
@@ -589,25 +612,27 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
   const int prow = (P == 128) ? (32 * q4 + lane) : (16 * q4 + (lane & 15));
   const bool st_owner = (P == 128) || (lane >= 16);  // holds the fp32 state of row prow
 
-  // operand staging: B, C rows on all threads; x rows on warps 1-7 (warp 0 prepares the next
-  // tile's coefficients meanwhile)
-  const int xt = tid;
-  constexpr int CHN = N / 8;
-  constexpr int RPI = NT / CHN;  // rows per pass; a multiple of 8 and of R
-  const int tch = xt % CHN;
-  const int tr = (xt / CHN) % R;
-  float bB[8], bC[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    bB[e] = biasBg ? __ldg(biasBg + tr * N + tch * 8 + e) : 0.0f;
-    bC[e] = biasCg ? __ldg(biasCg + tr * N + tch * 8 + e) : 0.0f;
-  }
-
   // ---- incoming rotated-frame state h+ of this segment
   //   nseg == 1 (full pass): h_{-1} + beta'_0 u_{-1} from the state / carry;
   //   state pass, segment 0: same, written to ws_init; other state-pass segments: zero;
   //   full pass, segment k > 0: ws_init folded through the summaries of segments 0..k-1.
-  if (state_warp && j0 < j1) {
+  // In the full pass every warp takes part (warp w: the TMEM lanes of quarter w & 3, half the
+  // state columns), and the rotations of the folded segments come from a table that all
+  // threads fill first (in the second rotation-table slot, unused until the first window).
+  const bool fold_tab = FULL && sg.nseg > 1 && seg > 0 && seg <= Q;
+  float2* ftab = cs(1);
+  if (fold_tab && j0 < j1) {
+    for (int i = tid; i < seg * K2; i += kThreads) {
+      const int64_t sidx = (int64_t)bh * (sg.nseg - 1) + i / K2;
+      float sn, cn;
+      sincosf((float)sg.ws_phi[sidx * K2 + i % K2], &sn, &cn);
+      ftab[i] = make_float2(cn, sn);
+    }
+  }
+  __syncthreads();
+  const int c_lo = FULL ? (warp >> 2) * (N / 64) : 0;
+  const int c_hi = FULL ? c_lo + N / 64 : N / 32;
+  if ((FULL || state_warp) && j0 < j1) {
     const bool from_state = (sg.nseg == 1) || (!FULL && seg == 0);
     const float hscale = scal(0)[4];  // e^m of the first tile: the bf16 copy is pre-scaled
     float xprev[R];
@@ -620,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
     const float* h0 = p.h + (int64_t)bh * N * P;
     const float* cB = p.carry_B + (int64_t)bh * R * N;
 #pragma unroll 1
-    for (int c = 0; c < N / 32; ++c) {
+    for (int c = c_lo; c < c_hi; ++c) {
       float v[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) v[e] = 0.0f;
@@ -652,7 +677,13 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
           for (int e = 0; e < 16; ++e) {
             const int n0 = 32 * c + 2 * e;
             float sn, cn;
-            sincosf((float)ph[n0 / 2], &sn, &cn);
+            if (fold_tab) {
+              const float2 t = ftab[k * K2 + n0 / 2];
+              cn = t.x;
+              sn = t.y;
+            } else {
+              sincosf((float)ph[n0 / 2], &sn, &cn);
+            }
             const float a0 = fmaf(dec, v[2 * e], wh[(int64_t)n0 * P + prow]);
             const float a1 = fmaf(dec, v[2 * e + 1], wh[(int64_t)(n0 + 1) * P + prow]);
             v[2 * e] = cn * a0 - sn * a1;
