@@ -242,6 +242,13 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 __device__ __forceinline__ uint32_t sw128(int row, int ch, uint32_t block_bytes) {
   return (uint32_t)(ch >> 3) * block_bytes + (uint32_t)row * 128u + ((uint32_t)((ch & 7) ^ (row & 7)) << 4);
 }
+// Signed-integer key of a float with the same order (negative floats: magnitude bits reversed),
+// and its inverse; lets redux.sync take a warp's float min / max.
+__device__ __forceinline__ int float_key(float f) {
+  const int i = __float_as_int(f);
+  return i >= 0 ? i : (i ^ 0x7fffffff);
+}
+__device__ __forceinline__ float key_float(int k) { return __int_as_float(k >= 0 ? k : (k ^ 0x7fffffff)); }
 // 2^x by the hardware approximation (ex2.approx, relative error about 2^-22).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -465,11 +472,9 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
         lmin = fminf(lmin, loc[e]);
         lmax = fmaxf(lmax, loc[e]);
       }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        lmin = fminf(lmin, __shfl_xor_sync(kFull, lmin, off));
-        lmax = fmaxf(lmax, __shfl_xor_sync(kFull, lmax, off));
-      }
+      // warp min / max in one redux each, on integer keys that order like the floats
+      lmin = key_float(__reduce_min_sync(kFull, float_key(lmin)));
+      lmax = key_float(__reduce_max_sync(kFull, float_key(lmax)));
       const bool fast = (lmax - lmin) <= 160.0f;
       const float m = fast ? 0.5f * (lmax + lmin) : 0.0f;
       const float bp_after = rawA(slot, 3)[0];
@@ -485,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
           const float bpn = (t + 1 < Q) ? ((t + 1 < nv) ? (1.0f - lmA[t + 1]) * dtA[t + 1] : 0.0f)
                                         : (valid ? bp_after : 0.0f);
           const float w = gm + bpn;
-          const float dg = (w > 0.0f) ? gm / w : 0.0f;
+          const float dg = (w > 0.0f) ? __fdividef(gm, w) : 0.0f;
           const float at = fast ? __expf(Lct - m) : 1.0f;
           const float xs = fast ? __expf(m - Lct) * w : w;
           ra[t] = make_float4(Lct * 1.4426950408889634f, dg, at, xs);
@@ -522,9 +527,13 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
     double total = 0.0;
     {
       float aoff = 0.0f;
-      for (int s = 0; s < aseg; ++s) aoff += segsum[s * K2 + ak];
-      if (aseg == 0)
+#pragma unroll
+      for (int s = 0; s < C::SEGS; ++s)  // all loads issued together
+        if (s < aseg) aoff += segsum[s * K2 + ak];
+      if (aseg == 0) {
+#pragma unroll
         for (int s = 0; s < C::SEGS; ++s) total += (double)segsum[s * K2 + ak];
+      }
       aoff += (float)base[ak];
       float2* c2 = cs(slot);
 #pragma unroll
