@@ -269,12 +269,14 @@ __device__ __forceinline__ void sincos_reduced(float x, float* s, float* c) {
 // ------------------------------------------------------------------ configuration
 
 struct SegInfo {
-  int nseg;        // segments per sequence
-  int seg_tiles;   // tiles per segment
+  int nseg;        // full-pass segments per sequence
+  int seg_tiles;   // tiles per full-pass segment
+  int nsub;        // state-pass sub-segments per sequence: they tile segments 0..nseg-2
+  int sub_tiles;   // tiles per sub-segment (divides seg_tiles)
   float* ws_init;  // (b*H, N, P): rotated-frame state entering segment 0 (nseg > 1)
-  float* ws_h;     // (b*H, nseg-1, N, P): end state of segments 0..nseg-2 from a zero start
-  float* ws_l;     // (b*H, nseg-1): total log decay of those segments
-  double* ws_phi;  // (b*H, nseg-1, N/2): total angle of those segments, reduced mod 2 pi
+  float* ws_h;     // (b*H, nsub, N, P): end state of each sub-segment from a zero start
+  float* ws_l;     // (b*H, nsub): total log decay of each sub-segment
+  double* ws_phi;  // (b*H, nsub, N/2): total angle of each sub-segment, reduced mod 2 pi
 };
 
 template <int R, int N, int P, int MODE>
@@ -349,14 +351,15 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
   const int H = p.H, G = p.G;
   const int64_t L = p.L;
   // segment decomposition
-  const int nseg_grid = FULL ? sg.nseg : (sg.nseg - 1);
+  const int nseg_grid = FULL ? sg.nseg : sg.nsub;
   const int bh = blockIdx.x / nseg_grid;
-  const int seg = blockIdx.x % nseg_grid;
+  const int seg = blockIdx.x % nseg_grid;  // state pass: the sub-segment
   const int bi = bh / H, hi = bh % H;
   const int g = hi / (H / G);
   const int64_t ntiles_seq = (L + Q - 1) / Q;
-  const int64_t j0 = (int64_t)seg * sg.seg_tiles;
-  const int64_t j1 = (j0 + sg.seg_tiles < ntiles_seq) ? (j0 + sg.seg_tiles) : ntiles_seq;
+  const int seg_len = FULL ? sg.seg_tiles : sg.sub_tiles;
+  const int64_t j0 = (int64_t)seg * seg_len;
+  const int64_t j1 = (j0 + seg_len < ntiles_seq) ? (j0 + seg_len) : ntiles_seq;
   const bool last_seg = (seg == sg.nseg - 1);
   const int64_t tok_base = (int64_t)bi * L;  // first token of this sequence (flattened b*L index)
 
@@ -628,11 +631,13 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
   // In the full pass every warp takes part (warp w: the TMEM lanes of quarter w & 3, half the
   // state columns), and the rotations of the folded segments come from a table that all
   // threads fill first (in the second rotation-table slot, unused until the first window).
-  const bool fold_tab = FULL && sg.nseg > 1 && seg > 0 && seg <= Q;
+  // segment seg of the full pass starts after sub-segments 0..nfold-1 of the state pass
+  const int nfold = FULL ? seg * (sg.nseg > 1 ? sg.seg_tiles / sg.sub_tiles : 0) : 0;
+  const bool fold_tab = FULL && sg.nseg > 1 && seg > 0 && nfold <= Q;
   float2* ftab = cs(1);
   if (fold_tab && j0 < j1) {
-    for (int i = tid; i < seg * K2; i += kThreads) {
-      const int64_t sidx = (int64_t)bh * (sg.nseg - 1) + i / K2;
+    for (int i = tid; i < nfold * K2; i += kThreads) {
+      const int64_t sidx = (int64_t)bh * sg.nsub + i / K2;
       float sn, cn;
       sincosf((float)sg.ws_phi[sidx * K2 + i % K2], &sn, &cn);
       ftab[i] = make_float2(cn, sn);
@@ -677,8 +682,8 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
         const float* wi = sg.ws_init + (int64_t)bh * N * P;
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = wi[(int64_t)(32 * c + e) * P + prow];
-        for (int k = 0; k < seg; ++k) {
-          const int64_t sidx = (int64_t)bh * (sg.nseg - 1) + k;
+        for (int k = 0; k < nfold; ++k) {
+          const int64_t sidx = (int64_t)bh * sg.nsub + k;
           const float dec = __expf(sg.ws_l[sidx]);
           const float* wh = sg.ws_h + sidx * N * P;
           const double* ph = sg.ws_phi + sidx * K2;
@@ -1185,7 +1190,7 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
       }
     } else {
       // segment summary: end state (segment frame, zero start), total log decay, total angle
-      const int64_t sidx = (int64_t)bh * (sg.nseg - 1) + seg;
+      const int64_t sidx = (int64_t)bh * sg.nsub + seg;
       if (state_warp) {
         float* wh = sg.ws_h + sidx * N * P;
 #pragma unroll 1
@@ -1288,19 +1293,37 @@ int plan_segments(int64_t nseq, int64_t ntiles, int per_sm) {
   return (int)nseg;
 }
 
+// Sub-segments of the state pass: segments 0..nseg-2 are cut into m equal parts (m divides
+// seg_tiles), as many as the free CTA slots allow, so that the state pass, which only has to
+// produce each part's summary, runs in parallel too.
+int plan_subsegments(int64_t nseq, int nseg, int seg_tiles, int per_sm) {
+  int dev = 0, nsm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (nseg <= 1) return 1;
+  const int64_t slots = (int64_t)nsm * per_sm;
+  int64_t m = slots / (nseq * (nseg - 1));
+  if (m > seg_tiles) m = seg_tiles;
+  while (m > 1 && seg_tiles % m != 0) --m;
+  return m < 1 ? 1 : (int)m;
+}
+
+struct SegPlan {
+  int nseg, seg_tiles, nsub, sub_tiles;
+};
+
 template <int R, int N, int P>
-size_t ws_bytes_for(const Params& p, int* nseg_out, int* seg_tiles_out) {
+size_t ws_bytes_for(const Params& p, SegPlan* out) {
   constexpr int Q = kRows / R;
   const int64_t ntiles = (p.L + Q - 1) / Q;
   const int64_t nseq = p.b * p.H;
   const int nseg = plan_segments(nseq, ntiles, ctas_per_sm<R, N, P>());
   const int seg_tiles = (int)((ntiles + nseg - 1) / nseg);
   const int nseg_eff = (int)((ntiles + seg_tiles - 1) / seg_tiles);
-  if (nseg_out) *nseg_out = nseg_eff;
-  if (seg_tiles_out) *seg_tiles_out = seg_tiles;
+  const int m = plan_subsegments(nseq, nseg_eff, seg_tiles, ctas_per_sm<R, N, P>());
+  if (out) *out = SegPlan{nseg_eff, seg_tiles, (nseg_eff - 1) * m, seg_tiles / m};
   if (nseg_eff <= 1) return 0;
   const size_t np = (size_t)N * P;
-  const size_t s1 = (size_t)(nseg_eff - 1);
+  const size_t s1 = (size_t)(nseg_eff - 1) * m;
   size_t bytes = 0;
   bytes += 4 * (size_t)nseq * np;                       // ws_init
   bytes += 4 * (size_t)nseq * s1 * np;                  // ws_h
@@ -1312,27 +1335,30 @@ size_t ws_bytes_for(const Params& p, int* nseg_out, int* seg_tiles_out) {
 template <int R, int N, int P>
 cudaError_t launch_cfg(const Params& p, void* ws, size_t ws_bytes, cudaStream_t stream) {
   constexpr int Q = kRows / R;
-  int nseg = 1, seg_tiles = 1;
-  const size_t need = ws_bytes_for<R, N, P>(p, &nseg, &seg_tiles);
+  SegPlan plan;
+  const size_t need = ws_bytes_for<R, N, P>(p, &plan);
   if (need > ws_bytes || (need > 0 && ws == nullptr)) return cudaErrorInvalidValue;
   Maps m;
   if (!make_maps(p, Q, &m)) return cudaErrorInvalidValue;
   SegInfo sg;
-  sg.nseg = nseg;
-  sg.seg_tiles = seg_tiles;
+  sg.nseg = plan.nseg;
+  sg.seg_tiles = plan.seg_tiles;
+  sg.nsub = plan.nsub;
+  sg.sub_tiles = plan.sub_tiles;
   sg.ws_init = sg.ws_h = sg.ws_l = nullptr;
   sg.ws_phi = nullptr;
   const int64_t nseq = p.b * p.H;
+  const int nseg = plan.nseg;
   if (nseg > 1) {
     const size_t np = (size_t)N * P;
-    const size_t s1 = (size_t)(nseg - 1);
+    const size_t s1 = (size_t)plan.nsub;
     char* w = static_cast<char*>(ws);
     sg.ws_init = reinterpret_cast<float*>(w);
     sg.ws_h = sg.ws_init + (size_t)nseq * np;
     sg.ws_l = sg.ws_h + (size_t)nseq * s1 * np;
     size_t off = (4 * ((size_t)nseq * np + (size_t)nseq * s1 * np + (size_t)nseq * s1) + 255) & ~(size_t)255;
     sg.ws_phi = reinterpret_cast<double*>(w + off);
-    cudaError_t e = launch_mode<R, N, P, MODE_STATE>(m, p, sg, (unsigned)(nseq * (nseg - 1)), stream);
+    cudaError_t e = launch_mode<R, N, P, MODE_STATE>(m, p, sg, (unsigned)(nseq * plan.nsub), stream);
     if (e != cudaSuccess) return e;
   }
   return launch_mode<R, N, P, MODE_FULL>(m, p, sg, (unsigned)(nseq * nseg), stream);
@@ -1353,10 +1379,10 @@ cudaError_t launch_r(const Params& p, void* ws, size_t wsb, cudaStream_t s) {
 
 template <int R>
 size_t ws_r(const Params& p) {
-  if (p.N == 64 && p.P == 64) return ws_bytes_for<R, 64, 64>(p, nullptr, nullptr);
-  if (p.N == 64 && p.P == 128) return ws_bytes_for<R, 64, 128>(p, nullptr, nullptr);
-  if (p.N == 128 && p.P == 64) return ws_bytes_for<R, 128, 64>(p, nullptr, nullptr);
-  return ws_bytes_for<R, 128, 128>(p, nullptr, nullptr);
+  if (p.N == 64 && p.P == 64) return ws_bytes_for<R, 64, 64>(p, nullptr);
+  if (p.N == 64 && p.P == 128) return ws_bytes_for<R, 64, 128>(p, nullptr);
+  if (p.N == 128 && p.P == 64) return ws_bytes_for<R, 128, 64>(p, nullptr);
+  return ws_bytes_for<R, 128, 128>(p, nullptr);
 }
 
 template <int R>
