@@ -15,8 +15,8 @@
  *   X_{t,r} = W_x[h,r,:] * x[b,t,h,:],        u_t = sum_r Bb_{t,r} X_{t,r}^T   (N x P)
  *   h_t = e^{dt_t A_t} Rot(dt_t theta_t) (h_{t-1} + (1-lam_t) dt_t u_{t-1}) + lam_t dt_t u_t
  *   y[b,t,h,:] = sum_r W_o[h,r,:] * (Cb_{t,r}^T h_t) + D[h] x[b,t,h,:]
- * Rot rotates rows (2k, 2k+1) of the state by angle dt_t theta[b,t,g,k] with the
- * matrix [[cos, -sin], [sin, cos]].
+ * Rot rotates rows (2k, 2k+1) of the state by angle dt_t theta[b,t,g,k] (theta[b,t,g,k]
+ * itself with M3_FLAG_ANGLE_DIRECT) with the matrix [[cos, -sin], [sin, cos]].
  *
  * Conventions for every entry point:
  *   - Tensor pointers are caller-owned DEVICE memory, contiguous row-major in the
@@ -51,7 +51,8 @@ extern "C" {
 
 typedef enum {
   M3_OK = 0,
-  M3_ERR_DIMS = -1,        /* bad sizes: N odd, G does not divide H, R/P/N out of range */
+  M3_ERR_DIMS = -1,        /* bad sizes: N odd, G does not divide H, R/P/N out of range;
+                              unknown flag bits */
   M3_ERR_DTYPE = -2,       /* dtype not M3_BF16 / M3_F32 */
   M3_ERR_ALIGN = -3,       /* a tensor pointer is not 16-byte aligned */
   M3_ERR_NULL = -4,        /* a required pointer is NULL */
@@ -66,8 +67,11 @@ enum { M3_F32 = 0, M3_BF16 = 1 };
 
 /* flags */
 enum {
-  M3_FLAG_SEQUENTIAL = 1u  /* run the token-sequential SIMT scan even where the chunked
-                              tensor-core scan applies (diagnostic / cross-check) */
+  M3_FLAG_SEQUENTIAL = 1u,   /* run the token-sequential SIMT scan even where the chunked
+                                tensor-core scan applies (diagnostic / cross-check) */
+  M3_FLAG_ANGLE_DIRECT = 2u  /* variant: theta is the rotation angle of the step itself,
+                                phi_t = theta_t instead of dt_t * theta_t (the rotation
+                                then no longer depends on the head's step size) */
 };
 
 typedef struct {
@@ -82,7 +86,7 @@ typedef struct {
                      exact, so this does not change the result; the kernel packs
                      128/R tokens per tensor-core tile whatever this value is. */
   int32_t dtype;  /* M3_BF16 or M3_F32: storage type of x, B, C, y */
-  uint32_t flags; /* M3_FLAG_* */
+  uint32_t flags; /* M3_FLAG_*; other bits: M3_ERR_DIMS */
 } m3_dims;
 
 typedef struct m3_state m3_state; /* opaque */

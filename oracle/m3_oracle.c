@@ -12,7 +12,8 @@
  *   X_{t,r}  = W_x[h,r,:] * x[b,t,h,:]              (MIMO input branches)
  *   u_t      = sum_r Bb_{t,r} X_{t,r}^T             (N x P, rank <= R update)
  *   alpha_t  = exp(dt_t A_t), beta'_t = (1 - lam_t) dt_t, gamma_t = lam_t dt_t
- *   phi_{t,k}= dt_t theta[b,t,g,k]                  (rotation of complex pair k)
+ *   phi_{t,k}= dt_t theta[b,t,g,k]                  (rotation of complex pair k; theta[b,t,g,k]
+ *                                                    itself in the direct-angle variant)
  *   h_t      = alpha_t Rot(phi_t) (h_{t-1} + beta'_t u_{t-1}) + gamma_t u_t
  *   Y_{t,r}  = Cb_{t,r}^T h_t ;  y[b,t,h,:] = sum_r W_o[h,r,:] * Y_{t,r} + D_h x[b,t,h,:]
  *
@@ -60,6 +61,7 @@
 typedef struct {
   int64_t b, L;
   int32_t H, P, N, R, G;
+  int32_t angle_direct; /* variant: phi_{t,k} = theta[b,t,g,k] (no dt factor) */
 } m3o_dims;
 
 /* One (batch, head) recurrence over all L tokens.  Returns 0, or -1 on OOM. */
@@ -132,7 +134,7 @@ static int scan_one(const m3o_dims* d, int64_t bi, int32_t hi,
     }
     /* h_t = alpha Rot(phi) (h_{t-1} + beta' u_{t-1}) + gamma u_t, pair by pair */
     for (int32_t k = 0; k < K; ++k) {
-      const double phi = delta * th[k];
+      const double phi = d->angle_direct ? th[k] : delta * th[k];
       const double c = cos(phi), s = sin(phi);
       double* h0 = hs + (int64_t)(2 * k) * P;
       double* h1 = hs + (int64_t)(2 * k + 1) * P;

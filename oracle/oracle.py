@@ -26,7 +26,7 @@ _lib = None
 class _Dims(ctypes.Structure):
     _fields_ = [("b", ctypes.c_int64), ("L", ctypes.c_int64), ("H", ctypes.c_int32),
                 ("P", ctypes.c_int32), ("N", ctypes.c_int32), ("R", ctypes.c_int32),
-                ("G", ctypes.c_int32)]
+                ("G", ctypes.c_int32), ("angle_direct", ctypes.c_int32)]
 
 
 def build(force: bool = False) -> str:
@@ -69,7 +69,7 @@ def _ptr(a):
 
 
 def scan(dims, x, dt, A, lam, B, C, theta, bias_B=None, bias_C=None, W_x=None, W_o=None,
-         D=None, h0=None, carry_B0=None, carry_x0=None, sel=None, threads=0):
+         D=None, h0=None, carry_B0=None, carry_x0=None, sel=None, threads=0, angle_direct=False):
     """Sequential fp64 recurrence.
 
     dims: mapping with b, L, H, P, N, R, G.  Arrays in the layouts of m3_oracle.c
@@ -80,7 +80,7 @@ def scan(dims, x, dt, A, lam, B, C, theta, bias_B=None, bias_C=None, W_x=None, W
     """
     lib = _load()
     b, L, H, P, N, R, G = (int(dims[k]) for k in ("b", "L", "H", "P", "N", "R", "G"))
-    d = _Dims(b, L, H, P, N, R, G)
+    d = _Dims(b, L, H, P, N, R, G, 1 if angle_direct else 0)
     h = np.zeros((b, H, N, P)) if h0 is None else np.array(h0, dtype=np.float64, copy=True)
     cB = np.zeros((b, H, R, N)) if carry_B0 is None else np.array(carry_B0, dtype=np.float64, copy=True)
     cx = np.zeros((b, H, P)) if carry_x0 is None else np.array(carry_x0, dtype=np.float64, copy=True)
@@ -103,8 +103,8 @@ def scan(dims, x, dt, A, lam, B, C, theta, bias_B=None, bias_C=None, W_x=None, W
     return y, h, cB, cx
 
 
-def scan_inputs(inp, sel=None, threads=0, h0=None, carry_B0=None, carry_x0=None):
+def scan_inputs(inp, sel=None, threads=0, h0=None, carry_B0=None, carry_x0=None, angle_direct=False):
     """``scan`` on an ``Inputs`` draw from the shared seeded generator."""
     return scan(inp.dims, inp.x, inp.dt, inp.A, inp.lam, inp.B, inp.C, inp.theta, inp.bias_B,
                 inp.bias_C, inp.W_x, inp.W_o, inp.D, h0=h0, carry_B0=carry_B0,
-                carry_x0=carry_x0, sel=sel, threads=threads)
+                carry_x0=carry_x0, sel=sel, threads=threads, angle_direct=angle_direct)

@@ -46,6 +46,7 @@ m3_status check_dims(const m3_dims* d) {
   if (d->N < 8 || d->N > 256 || (d->N % 8) != 0) return M3_ERR_DIMS;
   if ((d->H % d->G) != 0) return M3_ERR_DIMS;
   if (d->chunk < 0) return M3_ERR_DIMS;
+  if (d->flags & ~(uint32_t)(M3_FLAG_SEQUENTIAL | M3_FLAG_ANGLE_DIRECT)) return M3_ERR_DIMS;
   if (d->dtype != M3_F32 && d->dtype != M3_BF16) return M3_ERR_DTYPE;
   if (d->b * (int64_t)d->H > (int64_t)0x7fffffff) return M3_ERR_DIMS;
   if (!m3::seq_scan_supported(d->P, d->N, d->R)) return M3_ERR_UNSUPPORTED;
@@ -95,6 +96,7 @@ m3::Params make_params(const m3_dims* d, int64_t L, const void* x, const float* 
   p.R = d->R;
   p.G = d->G;
   p.dtype = d->dtype;
+  p.angle_direct = (d->flags & M3_FLAG_ANGLE_DIRECT) ? 1 : 0;
   p.x = x;
   p.dt = dt;
   p.A = A;

@@ -14,6 +14,7 @@ struct Params {
   int64_t b, L;
   int H, P, N, R, G;
   int dtype;  // M3_BF16 / M3_F32 for x, B, C, y
+  int angle_direct;  // 1: the step's rotation angle is theta itself (M3_FLAG_ANGLE_DIRECT)
   const void* x;
   const float* dt;
   const float* A;

@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(kRingThreads, kRingCtas) decode_ring_kernel(Pa
       const float delta = sc[0];
       for (int k = tid; k < NB / 2; k += kRingThreads) {
         float sn, cn;
-        sincosf(delta * ths[n0 / 2 + k], &sn, &cn);
+        sincosf(p.angle_direct ? ths[n0 / 2 + k] : delta * ths[n0 / 2 + k], &sn, &cn);
         cs[k] = make_float2(cn, sn);
       }
       if (tid == 0) {

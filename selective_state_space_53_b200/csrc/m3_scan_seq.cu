@@ -128,7 +128,7 @@ scan_seq_kernel(Params p) {
       const float* th = p.theta + (tok * G + g) * (int64_t)(N / 2);
       for (int k = tid; k < N / 2; k += kThreads) {
         float s, c;
-        sincosf(delta * th[k], &s, &c);
+        sincosf(p.angle_direct ? th[k] : delta * th[k], &s, &c);
         cs[k] = make_float2(c, s);
       }
       if (tid == 0) {

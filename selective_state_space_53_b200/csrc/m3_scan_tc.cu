@@ -521,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
 #pragma unroll
       for (int e = 0; e < C::SEGLEN; ++e) {
         const int t = aseg * C::SEGLEN + e;
-        if (t < Q) run += (t < nv) ? dtA[t] * r_th[e] : 0.0f;
+        if (t < Q) run += (t < nv) ? (p.angle_direct ? r_th[e] : dtA[t] * r_th[e]) : 0.0f;
         aloc[e] = run;
       }
       segsum[aseg * K2 + ak] = run;

@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(_HERE, "libm3.so")
 
 M3_F32, M3_BF16 = 0, 1
 M3_FLAG_SEQUENTIAL = 1
+M3_FLAG_ANGLE_DIRECT = 2
 
 _STATUS = {0: "M3_OK", -1: "M3_ERR_DIMS", -2: "M3_ERR_DTYPE", -3: "M3_ERR_ALIGN",
            -4: "M3_ERR_NULL", -5: "M3_ERR_WORKSPACE", -6: "M3_ERR_CUDA", -7: "M3_ERR_TIMEOUT",

@@ -289,3 +289,44 @@ def test_tc_strong_decay_tiles(shape):
     inp.A[:, burst, :] = -12.0
     st = make_state(shape["b"], shape["H"], shape["P"], shape["N"], shape["R"], seed=207)
     check_scan(inp, state=st)
+
+
+# ------------------------------------------------------------------ direct-angle variant
+
+def check_direct(inp, flags=0, tol=None):
+    tol = TOL[inp.dims["dtype"]] if tol is None else tol
+    dims = m3.dims_of(inp, flags=flags | m3.M3_FLAG_ANGLE_DIRECT)
+    dev = m3.to_device(inp)
+    st, (th, tb, tx) = m3.state_tensors(dims)
+    y = m3.scan(dims, dev, st)
+    torch.cuda.synchronize()
+    yr, hr, _, _ = orc.scan_inputs(inp, angle_direct=True)
+    ey, eh = rel_err(y.float().cpu().numpy(), yr), rel_err(th.cpu().numpy(), hr)
+    assert ey < tol and eh < tol, (ey, eh)
+
+
+@pytest.mark.parametrize("shape", [
+    dict(b=1, L=300, H=2, P=64, N=64, R=2, G=1),
+    dict(b=1, L=2000, H=2, P=64, N=64, R=2, G=1),    # segmented
+    dict(b=1, L=200, H=2, P=128, N=128, R=4, G=1),
+], ids=["P64", "P64seg", "P128"])
+def test_direct_angle_tc(shape):
+    check_direct(make_inputs(dtype="bf16", seed=401, extras=True, **shape))
+
+
+def test_direct_angle_sequential_f32():
+    check_direct(make_inputs(dtype="f32", seed=402, extras=True, b=2, L=37, H=4, P=16, N=16, R=2, G=2),
+                 flags=m3.M3_FLAG_SEQUENTIAL)
+
+
+def test_direct_angle_decode():
+    shape = dict(b=3, L=8, H=4, P=32, N=16, R=2, G=2)
+    inp = make_inputs(dtype="bf16", seed=403, extras=True, **shape)
+    dims = m3.dims_of(inp, L=1, flags=m3.M3_FLAG_ANGLE_DIRECT)
+    dev = m3.to_device(inp)
+    st, (th, tb, tx) = m3.state_tensors(dims)
+    ys = [m3.decode(dims, _token(dev, t), st).float() for t in range(shape["L"])]
+    torch.cuda.synchronize()
+    y = torch.stack(ys, dim=1).cpu().numpy()
+    yr, hr, _, _ = orc.scan_inputs(inp, angle_direct=True)
+    assert rel_err(y, yr) < TOL["bf16"] and rel_err(th.cpu().numpy(), hr) < TOL["bf16"]

@@ -351,3 +351,20 @@ def test_bad_dims_rejected():
     with pytest.raises(RuntimeError):
         orc.scan(dict(inp.dims, G=3), inp.x, inp.dt, inp.A, inp.lam,
                  np.zeros((1, 3, 3, 1, 4)), np.zeros((1, 3, 3, 1, 4)), np.zeros((1, 3, 3, 2)))
+
+
+# ------------------------------------------------------------------ direct-angle variant
+
+def test_direct_angle_equals_prescaled_theta():
+    # With one head per group, the direct-angle variant fed theta' = dt * theta is the
+    # default recurrence fed theta: the rotation of each step is the same angle.
+    inp = make_inputs(b=2, L=40, H=3, P=8, N=8, R=2, G=3, dtype="f32", seed=77, extras=True)
+    y0, h0, _, _ = orc.scan_inputs(inp)
+    direct = make_inputs(b=2, L=40, H=3, P=8, N=8, R=2, G=3, dtype="f32", seed=77, extras=True)
+    direct.theta = inp.dt.astype(np.float64)[..., None] * inp.theta.astype(np.float64)
+    y1, h1, _, _ = orc.scan_inputs(direct, angle_direct=True)
+    np.testing.assert_array_equal(y1, y0)
+    np.testing.assert_array_equal(h1, h0)
+    # and the flag matters: the same theta as a direct angle gives another result
+    y2, _, _, _ = orc.scan_inputs(inp, angle_direct=True)
+    assert np.abs(y2 - y0).max() > 1e-3 * np.abs(y0).max()
