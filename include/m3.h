@@ -173,6 +173,14 @@ m3_status m3_decode_step(const m3_dims* dims, const void* x_t, const float* dt_t
  * M3_OK, M3_ERR_TIMEOUT, or M3_ERR_CUDA if the stream reports an error. */
 m3_status m3_check(void* stream);
 
+/* Diagnostic of the error path (no counterpart in the pages): launches one CTA that waits on
+ * an mbarrier nothing arrives at, bounded by limit_ns (at most 10 s, else M3_ERR_DIMS) of
+ * %globaltimer -- the same kind of bounded wait as every wait in the scan and decode kernels.
+ * When the limit passes the kernel records M3_ERR_TIMEOUT in the device status word and
+ * returns; the next m3_check() on `stream` returns M3_ERR_TIMEOUT and clears the word, and the
+ * context stays usable.  Asynchronous on `stream`. */
+m3_status m3_selftest_wait(uint64_t limit_ns, void* stream);
+
 /* Static description of a status code. */
 const char* m3_status_str(m3_status status);
 

@@ -288,6 +288,14 @@ m3_status m3_decode_step(const m3_dims* dims, const void* x_t, const float* dt_t
   return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
 }
 
+m3_status m3_selftest_wait(uint64_t limit_ns, void* stream) {
+  if (limit_ns > 10000000000ull) return M3_ERR_DIMS;
+  int* st = status_word();
+  if (!st) return M3_ERR_CUDA;
+  return m3::launch_selftest_wait(st, (unsigned long long)limit_ns, (cudaStream_t)stream) == cudaSuccess ? M3_OK
+                                                                                                   : M3_ERR_CUDA;
+}
+
 m3_status m3_check(void* stream) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return M3_ERR_CUDA;
   int v = 0;

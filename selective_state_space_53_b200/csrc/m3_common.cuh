@@ -62,5 +62,6 @@ cudaError_t launch_decode(const Params& p, cudaStream_t stream);
 bool tc_scan_supported(const Params& p);
 size_t tc_scan_workspace_bytes(const Params& p);  // scratch the chunked scan needs (0: none)
 cudaError_t launch_scan_tc(const Params& p, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+cudaError_t launch_selftest_wait(int* status, unsigned long long limit_ns, cudaStream_t stream);
 
 }  // namespace m3

@@ -55,6 +55,7 @@ SIGNATURES = {
     "m3_scan_fwd_noalloc": (_I, [_DP] + [_VP] * 14 + [_VP]),
     "m3_decode_step": (_I, [_DP] + [_VP] * 15),
     "m3_check": (_I, [_VP]),
+    "m3_selftest_wait": (_I, [ctypes.c_uint64, _VP]),
     "m3_status_str": (ctypes.c_char_p, [_I]),
     "m3_version": (ctypes.c_char_p, []),
 }
@@ -190,6 +191,10 @@ def m3_decode_step(dims: Dims, x_t, dt_t, A_t, lam_t, B_t, C_t, theta_t, bias_B,
 
 def m3_check(stream=None) -> int:
     return int(lib().m3_check(_stream(stream)))
+
+
+def m3_selftest_wait(limit_ns: int, stream=None):
+    _check(lib().m3_selftest_wait(int(limit_ns), _stream(stream)), "m3_selftest_wait")
 
 
 def m3_status_str(code: int) -> str:

@@ -330,3 +330,16 @@ def test_direct_angle_decode():
     y = torch.stack(ys, dim=1).cpu().numpy()
     yr, hr, _, _ = orc.scan_inputs(inp, angle_direct=True)
     assert rel_err(y, yr) < TOL["bf16"] and rel_err(th.cpu().numpy(), hr) < TOL["bf16"]
+
+
+# ------------------------------------------------------------------ error path
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    # a wait on an mbarrier nothing arrives at gives up after 1 ms, records M3_ERR_TIMEOUT,
+    # and the next m3_check reports (and clears) it; the library keeps working afterwards
+    assert m3.m3_check() == 0
+    m3.m3_selftest_wait(1_000_000)
+    assert m3.m3_check() == -7
+    assert m3.m3_check() == 0
+    inp = make_inputs(dtype="bf16", seed=501, extras=True, b=1, L=70, H=2, P=64, N=64, R=2, G=1)
+    check_scan(inp)
