@@ -24,20 +24,24 @@
 // once, at the end of the sequence.
 //
 // Sequence splitting.  With few (batch, head) sequences the grid is b * H * nseg CTAs: a
-// state-only pass (MODE_STATE: Bt, Xs, MMA4, state update) first runs segments 0..nseg-2 from
-// a zero state and writes each segment's end state, total log decay and total angle to the
-// workspace; the full pass (MODE_FULL) then starts segment k from the combination of those
-// summaries.  Both passes are the same chunk algebra; only the starting state differs.
+// state-only pass (MODE_STATE: Bt, Xs, MMA4, state update) first runs segments 0..nseg-2, cut
+// into m sub-segments each where free CTA slots allow, from a zero state and writes each
+// sub-segment's end state, total log decay and total angle to the workspace; the full pass
+// (MODE_FULL) then starts segment k from the combination of the summaries before it.  Both
+// passes are the same chunk algebra; only the starting state differs.
 //
 // On chip: B and C tiles arrive by TMA (cp.async.bulk.tensor, 128-byte swizzle) directly in
-// the canonical K-major UMMA layout and are rotated in place; x and theta arrive by TMA into
-// staging buffers.  The next tile's loads are issued as soon as the buffers they overwrite
-// are consumed, so they land while the current tile computes.  Accumulators S, Y, H and the
+// the canonical K-major UMMA layout and are rotated in place; x arrives by TMA into a staging
+// buffer; Delta, A, lambda and theta are loaded into registers one tile ahead.  The next tile's
+// loads are issued as soon as the buffers they overwrite are consumed, so they land while the
+// current tile computes.  Accumulators S, Y, H and the
 // fp32 state live in tensor memory; the masked S is written back into TMEM as bf16 pairs and
 // consumed as the A operand of MMA2.
 //
-// Warp roles: all 8 warps stage tiles; thread 0 issues TMA and MMAs and commits the MMAs to
-// an mbarrier; warps 0-3 mask S while warps 4-7 update the state; all warps run the epilogue.
+// Warp roles: all 8 warps stage tiles and run the epilogue (each its TMEM lane quarter, half
+// the columns); thread 0 issues the TMA loads; warp 0 issues the MMAs (one elected lane) and
+// commits them to an mbarrier, and builds the next tile's coefficients; warps 0-3 mask S
+// while warps 4-7 update the state; all warps build the rotation tables.
 // Every mbarrier wait is bounded by %globaltimer; a timeout sets M3_ERR_TIMEOUT in the device
 // status word and the CTA frees its TMEM and returns.
 #include <cuda.h>
