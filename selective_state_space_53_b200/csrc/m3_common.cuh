@@ -59,6 +59,8 @@ __device__ __forceinline__ void store_out(void* base, int64_t i, float v) {
 cudaError_t launch_scan_sequential(const Params& p, cudaStream_t stream);
 bool decode_supported(const Params& p);                       // one-token kernel fits on chip
 cudaError_t launch_decode(const Params& p, cudaStream_t stream);
+bool decode_tc_supported(const Params& p);                    // tensor-core form (d_state = headdim = 128, bf16)
+cudaError_t launch_decode_tc(const Params& p, cudaStream_t stream);
 bool tc_scan_supported(const Params& p);
 size_t tc_scan_workspace_bytes(const Params& p);  // scratch the chunked scan needs (0: none)
 cudaError_t launch_scan_tc(const Params& p, void* workspace, size_t workspace_bytes, cudaStream_t stream);

@@ -483,12 +483,14 @@ bool ring_plan_for(const Params& p, RingPlan* out) {
 }  // namespace
 
 bool decode_supported(const Params& p) {
+  if (decode_tc_supported(p)) return true;
   RingPlan rp;
   return ring_plan_for(p, &rp);
 }
 
 cudaError_t launch_decode(const Params& p, cudaStream_t stream) {
   if (p.b * p.H == 0) return cudaSuccess;
+  if (decode_tc_supported(p)) return launch_decode_tc(p, stream);
   RingPlan rp;
   if (ring_plan_for(p, &rp)) {
     const int64_t units = p.b * p.H;

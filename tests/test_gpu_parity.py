@@ -170,6 +170,43 @@ def test_decode_large_state_row_blocks():
     check_decode(inp, 3, st)
 
 
+# d_state = headdim = 128 with bf16 operands takes the tensor-core decode: the rank-2R update
+# and the readouts are MMAs with bf16 operands, fp32 accumulation and an fp32 state
+
+@pytest.mark.parametrize("R,G", [(1, 1), (3, 2), (8, 2)])
+def test_decode_tc_ranks(R, G):
+    shape = dict(b=3, L=5, H=4, P=128, N=128, R=R, G=G)
+    inp = make_inputs(dtype="bf16", seed=130 + R, extras=True, **shape)
+    st = make_state(3, 4, 128, 128, R, seed=140 + R)
+    check_decode(inp, 5, st)
+
+
+def test_decode_tc_stage_refills():
+    # 320 (batch, head) units over at most 148 CTAs: each CTA refills its two stages
+    shape = dict(b=40, L=3, H=8, P=128, N=128, R=4, G=1)
+    inp = make_inputs(dtype="bf16", seed=150, extras=True, **shape)
+    st = make_state(40, 8, 128, 128, 4, seed=151)
+    check_decode(inp, 3, st)
+
+
+def test_decode_tc_long_run():
+    # 256 tokens: the bf16 rounding of each step's operands must not accumulate in the fp32 state
+    shape = dict(b=2, L=256, H=2, P=128, N=128, R=4, G=1)
+    inp = make_inputs(dtype="bf16", seed=152, extras=True, **shape)
+    st = make_state(2, 2, 128, 128, 4, seed=153)
+    check_decode(inp, 256, st)
+
+
+def test_decode_b512_sampled_heads():
+    # the largest decode batch of the 1.5B-scale layer (16384 units, a 1 GiB state), four tokens;
+    # the oracle follows sampled (batch, head) pairs
+    cfg = dict(CONFIGS["decode_b512"])
+    cfg["L"] = 4
+    inp = make_inputs(seed=SEEDS["decode_b512"], **cfg)
+    st = make_state(cfg["b"], cfg["H"], cfg["P"], cfg["N"], cfg["R"], seed=154)
+    check_decode(inp, 4, st, sel=[(0, 0), (7, 31), (255, 16), (511, 1), (511, 31)])
+
+
 def test_prefill_then_decode_continues():
     shape = dict(b=2, L=40, H=4, P=64, N=64, R=2, G=1)
     inp = make_inputs(dtype="bf16", seed=107, extras=True, **shape)
@@ -322,6 +359,19 @@ def test_direct_angle_sequential_f32():
 def test_direct_angle_decode():
     shape = dict(b=3, L=8, H=4, P=32, N=16, R=2, G=2)
     inp = make_inputs(dtype="bf16", seed=403, extras=True, **shape)
+    dims = m3.dims_of(inp, L=1, flags=m3.M3_FLAG_ANGLE_DIRECT)
+    dev = m3.to_device(inp)
+    st, (th, tb, tx) = m3.state_tensors(dims)
+    ys = [m3.decode(dims, _token(dev, t), st).float() for t in range(shape["L"])]
+    torch.cuda.synchronize()
+    y = torch.stack(ys, dim=1).cpu().numpy()
+    yr, hr, _, _ = orc.scan_inputs(inp, angle_direct=True)
+    assert rel_err(y, yr) < TOL["bf16"] and rel_err(th.cpu().numpy(), hr) < TOL["bf16"]
+
+
+def test_direct_angle_decode_tc():
+    shape = dict(b=2, L=6, H=4, P=128, N=128, R=4, G=2)
+    inp = make_inputs(dtype="bf16", seed=404, extras=True, **shape)
     dims = m3.dims_of(inp, L=1, flags=m3.M3_FLAG_ANGLE_DIRECT)
     dev = m3.to_device(inp)
     st, (th, tb, tx) = m3.state_tensors(dims)
