@@ -315,6 +315,13 @@ def run_ours(args):
     }
 
     decode = run_decode(args, device, peaks) if not args.no_decode else None
+    if decode is not None and not args.no_decode_sweep:
+        # the rest of the decode batch sweep of the 1.5B-scale layer, one line each
+        decode["sweep"] = {}
+        for nm in ("decode_b1", "decode_b16", "decode_b512"):
+            r = run_decode(args, device, peaks, nm)
+            decode["sweep"][nm] = {k: r[k] for k in ("us_per_step", "tokens_per_s", "hbm_gbs", "hbm_frac_of_measured")}
+            torch.cuda.empty_cache()
     stack = run_stack(args, device, peaks) if not args.no_stack else None
     e2e = run_e2e(args, inp, tok_inp, device, world) if not args.no_e2e else None
     line = {
@@ -337,15 +344,15 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
-def run_decode(args, device, peaks):
-    """m3_decode_step on the 1.5B-scale layer, batch 128 (state 256 MiB > L2)."""
+def run_decode(args, device, peaks, name=DECODE_WORKLOAD):
+    """m3_decode_step on the 1.5B-scale layer (batch 128 by default: state 256 MiB > L2)."""
     import torch
     from selective_state_space_53_b200 import m3
     from selective_state_space_53_b200.inputs import CONFIGS, SEEDS, make_inputs, make_state
-    cfg = dict(CONFIGS[DECODE_WORKLOAD])
+    cfg = dict(CONFIGS[name])
     steps = args.decode_steps
     cfg_draw = dict(cfg, L=min(steps, 16))
-    inp = make_inputs(seed=SEEDS[DECODE_WORKLOAD], **cfg_draw)
+    inp = make_inputs(seed=SEEDS[name], **cfg_draw)
     dims1 = m3.dims_of(inp, L=1)
     h, cB, cx = make_state(cfg["b"], cfg["H"], cfg["P"], cfg["N"], cfg["R"], seed=7, scale=0.1)
     st, keep = m3.state_tensors(dims1, device=device, h=h, carry_B=cB, carry_x=cx)
@@ -373,7 +380,7 @@ def run_decode(args, device, peaks):
     by = decode_bytes(cfg)
     fl = decode_flops(cfg)
     del g
-    return {"workload": "decode_b128: m3_decode_step, b128 H32 P128 N128 R4, CUDA graph of %d steps" % steps,
+    return {"workload": "%s: m3_decode_step, b%d H32 P128 N128 R4, CUDA graph of %d steps" % (name, cfg["b"], steps),
             "tokens_per_s": cfg["b"] / (ms * 1e-3), "us_per_step": ms * 1e3,
             "hbm_gbs": by / (ms * 1e-3) / 1e9, "hbm_frac_of_measured": by / (ms * 1e-3) / 1e9 / peaks["hbm"],
             "tflops": fl / (ms * 1e-3) / 1e12, "algorithmic_bytes": by}
@@ -576,6 +583,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle timing")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-decode-sweep", action="store_true", help="decode at batch 128 only")
     ap.add_argument("--no-stack", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
