@@ -11,7 +11,8 @@ every rank runs its own batch; no data-path collective).  Inputs are seeded and
 synthetic; a ring of input sets larger than L2 rotates between steps.
 
 Extra keys: "prefill" / "decode" give each kernel measured on its own (decode on the
-1.5B-scale layer, batch 128, state 256 MiB > L2); "roofline" is the dominant kernel
+1.5B-scale layer, batch 128, state 256 MiB > L2; "decode.sweep" the batches 1, 16 and 512,
+"prefill.sweep_l15b" the 1.5B-scale layer's prefill at 2K, 8K and 32K tokens); "roofline" is the dominant kernel
 (the tensor-core prefill) against MEASURED_PEAKS.json; "cpu_baseline" times the fp64
 oracle (test infrastructure) on a bounded sample; "e2e" times the same step through
 the C ABI with pinned host buffers and the host<->device copies inside the timed region.
@@ -323,6 +324,8 @@ def run_ours(args):
             decode["sweep"][nm] = {k: r[k] for k in ("us_per_step", "tokens_per_s", "hbm_gbs", "hbm_frac_of_measured")}
             torch.cuda.empty_cache()
     stack = run_stack(args, device, peaks) if not args.no_stack else None
+    if not args.no_prefill_sweep:
+        prefill["sweep_l15b"] = run_prefill_sweep(args, device, peaks)
     e2e = run_e2e(args, inp, tok_inp, device, world) if not args.no_e2e else None
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -344,6 +347,48 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
+def run_prefill_sweep(args, device, peaks):
+    """m3_scan_fwd on the 1.5B-scale layer (b2, H32 P128 N128 R4) at seqlen 2K, 8K and 32K: mean of
+    5 calls after 2 warm-up calls, each on its own copy of the inputs when one copy fits in L2."""
+    import torch
+    from selective_state_space_53_b200 import m3
+    from selective_state_space_53_b200.inputs import CONFIGS, config_inputs
+    out = {}
+    stream = torch.cuda.current_stream()
+    for name in ("l15b_2k", "l15b_8k", "l15b_32k"):
+        cfg = dict(CONFIGS[name])
+        inp = config_inputs(name)
+        dims = m3.dims_of(inp)
+        per_set = prefill_bytes(cfg)
+        n_sets = max(1, -(-2 * L2_BYTES // per_set))
+        ring = make_ring(inp, n_sets, device)
+        ws_bytes = m3.m3_scan_workspace_size(dims)
+        ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
+        for i in range(2):
+            s = ring[i % n_sets]
+            m3.scan(dims, s["dev"], s["state"], y=s["y"], workspace=ws)
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
+        for i, (a, b) in enumerate(evs):
+            s = ring[i % n_sets]
+            a.record(stream)
+            m3.scan(dims, s["dev"], s["state"], y=s["y"], workspace=ws)
+            b.record(stream)
+        torch.cuda.synchronize()
+        assert m3.m3_check() == 0
+        ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+        by = prefill_bytes(cfg)
+        fl, fl_intra = prefill_flops(cfg)
+        out[name] = {"ms_per_call": ms, "tokens_per_s": cfg["b"] * cfg["L"] / (ms * 1e-3),
+                     "intra_chunk_tflops": fl_intra / (ms * 1e-3) / 1e12,
+                     "intra_chunk_frac_of_measured_burst": fl_intra / (ms * 1e-3) / 1e12 / peaks["bf16"],
+                     "tflops": fl / (ms * 1e-3) / 1e12, "tensor_frac_of_measured_burst": fl / (ms * 1e-3) / 1e12 / peaks["bf16"],
+                     "hbm_frac_of_measured": by / (ms * 1e-3) / 1e9 / peaks["hbm"], "input_sets": n_sets}
+        del ring, ws
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_decode(args, device, peaks, name=DECODE_WORKLOAD):
     """m3_decode_step on the 1.5B-scale layer (batch 128 by default: state 256 MiB > L2)."""
     import torch
@@ -355,19 +400,26 @@ def run_decode(args, device, peaks, name=DECODE_WORKLOAD):
     inp = make_inputs(seed=SEEDS[name], **cfg_draw)
     dims1 = m3.dims_of(inp, L=1)
     h, cB, cx = make_state(cfg["b"], cfg["H"], cfg["P"], cfg["N"], cfg["R"], seed=7, scale=0.1)
-    st, keep = m3.state_tensors(dims1, device=device, h=h, carry_B=cB, carry_x=cx)
+    # a ring of independent states when one state fits twice in L2 (batch 1 and 16), so that
+    # every step reads and writes its state in HBM
+    state_bytes = 2 * cfg["b"] * cfg["H"] * (cfg["N"] * cfg["P"] + cfg["R"] * cfg["N"] + cfg["P"]) * 4
+    n_states = max(1, -(-2 * L2_BYTES // state_bytes))
+    states = []
+    for _ in range(n_states):
+        st, keep = m3.state_tensors(dims1, device=device, h=h, carry_B=cB, carry_x=cx)
+        states.append((st, keep))
     dev = m3.to_device(inp, device)
     toks = [token_slice(dev, t) for t in range(cfg_draw["L"])]
     y = torch.empty_like(toks[0]["x"])
     stream = torch.cuda.current_stream()
     for i in range(3):
-        m3.decode(dims1, toks[i % len(toks)], st, y=y)
+        m3.decode(dims1, toks[i % len(toks)], states[i % n_states][0], y=y)
     torch.cuda.synchronize()
     # capture the steps in a CUDA graph: launch overhead out of the per-token time
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         for i in range(steps):
-            m3.decode(dims1, toks[i % len(toks)], st, y=y)
+            m3.decode(dims1, toks[i % len(toks)], states[i % n_states][0], y=y)
     g.replay()
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -380,7 +432,8 @@ def run_decode(args, device, peaks, name=DECODE_WORKLOAD):
     by = decode_bytes(cfg)
     fl = decode_flops(cfg)
     del g
-    return {"workload": "%s: m3_decode_step, b%d H32 P128 N128 R4, CUDA graph of %d steps" % (name, cfg["b"], steps),
+    return {"workload": "%s: m3_decode_step, b%d H32 P128 N128 R4, CUDA graph of %d steps over %d state(s) "
+                        "(%.0f MiB)" % (name, cfg["b"], steps, n_states, n_states * state_bytes / 2 / 2**20),
             "tokens_per_s": cfg["b"] / (ms * 1e-3), "us_per_step": ms * 1e3,
             "hbm_gbs": by / (ms * 1e-3) / 1e9, "hbm_frac_of_measured": by / (ms * 1e-3) / 1e9 / peaks["hbm"],
             "tflops": fl / (ms * 1e-3) / 1e12, "algorithmic_bytes": by}
@@ -579,11 +632,12 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--decode-steps", type=int, default=256)
+    ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle timing")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-decode-sweep", action="store_true", help="decode at batch 128 only")
+    ap.add_argument("--no-prefill-sweep", action="store_true", help="skip the 1.5B-scale layer prefill sweep")
     ap.add_argument("--no-stack", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()

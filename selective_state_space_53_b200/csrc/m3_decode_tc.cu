@@ -529,6 +529,358 @@ cudaError_t launch_tc_rt(const Params& p, const TcPlan& tp, unsigned grid, cudaS
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ split form (few units)
+// Few (batch, head) units leave most SMs idle in the persistent form.  Here a cluster of four CTAs
+// takes one unit, each CTA 32 state rows: the rank-2R increment of its rows (D^T = Xcat
+// Bcat_slice^T, M = 128, N = 32), their update, and their part of the readouts (Y^T =
+// h_slice^T Cb_slice, K = 32).  The four partial outputs sum_r W_o[r] Y^T meet in CTA 0 through
+// distributed shared memory; the new state goes straight from registers to HBM.
+constexpr int kSplit = 4;                  // CTAs per unit (cluster size)
+constexpr int kRows = kN / kSplit;         // state rows per CTA
+constexpr int kST = 128;                   // threads per CTA: thread = column p
+constexpr uint32_t kSplitTmemCols = 64;    // D^T 0-31, bf16 pairs of h_new^T 32-47, Y^T 48-63
+constexpr uint32_t kSColHB = 32, kSColY = 48;
+// The split form takes a decode call whose CTAs fit in one wave (kSplit x units <= SMs: batch 1 at
+// 32 heads, 5.5 vs 6.8 us per step on B200); beyond that the persistent form is faster (batch 16:
+// 15.3 vs 25.5 us).
+
+struct SplitPlan {
+  uint32_t o_x;     // Xcat: 128 rows, SW128 K-major (chunks 0-1 used)
+  uint32_t o_b;     // Bcat of the slice: 32 rows, SW128 K-major
+  uint32_t o_cb;    // Cb of the slice: 16 rows, SW128 K-major (the first 32 of 64 K-elements used)
+  uint32_t o_st;    // state rows of the slice, fp32 [32][128]
+  uint32_t o_braw, o_craw, o_cbold, o_xraw, o_cx, o_th;  // token operands of the unit
+  uint32_t o_cs, o_yp, o_tm, o_bar;
+  uint32_t total;
+};
+
+inline SplitPlan split_plan(int R) {
+  SplitPlan t{};
+  uint32_t f = 0;
+  t.o_x = f;     f += 128 * 128;
+  t.o_b = f;     f += kRows * 128;
+  t.o_cb = f;    f += 16 * 128;
+  t.o_st = f;    f += kRows * kP * 4;
+  t.o_braw = f;  f += pad16((uint32_t)R * kN * 2);
+  t.o_craw = f;  f += pad16((uint32_t)R * kN * 2);
+  t.o_cbold = f; f += pad16((uint32_t)R * kN * 4);
+  t.o_xraw = f;  f += pad16((uint32_t)kP * 2);
+  t.o_cx = f;    f += pad16((uint32_t)kP * 4);
+  t.o_th = f;    f += pad16((uint32_t)kN / 2 * 4);
+  t.o_cs = f;    f += kRows / 2 * 8;
+  t.o_yp = f;    f += kP * 4;
+  t.o_tm = f;    f += 16;
+  t.o_bar = f;   f += 16;
+  t.total = f + 1024;  // slack for aligning the base to 1024 bytes
+  return t;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// a float of CTA `rank`'s shared memory at this CTA's shared address `addr`
+__device__ __forceinline__ float ld_dsmem(uint32_t addr, uint32_t rank) {
+  uint32_t ra;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(addr), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+  return v;
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+}
+
+template <int RT>
+__global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kST, 1)
+    decode_tc_split_kernel(Params p, SplitPlan sp) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int H = p.H, R = p.R, G = p.G;
+  const uint32_t crank = cluster_rank();
+  const int64_t nb = p.b;
+  const int64_t u = blockIdx.x / kSplit;
+  const int64_t bi = u % nb;
+  const int hi = (int)(u / nb);
+  const int g = hi / (H / G);
+  const int64_t bh = bi * H + hi;
+  const int n0 = kRows * (int)crank;  // first state row of this CTA
+  const uint32_t sbase = smem_u32(sm);
+  const uint32_t sX = sbase + sp.o_x, sB = sbase + sp.o_b, sC = sbase + sp.o_cb;
+  const uint32_t full = sbase + sp.o_bar, mbar = full + 8;
+  const float* hst = reinterpret_cast<const float*>(sm + sp.o_st);
+  const __nv_bfloat16* Braw = reinterpret_cast<const __nv_bfloat16*>(sm + sp.o_braw);
+  const __nv_bfloat16* Craw = reinterpret_cast<const __nv_bfloat16*>(sm + sp.o_craw);
+  const float* cBs = reinterpret_cast<const float*>(sm + sp.o_cbold);
+  const __nv_bfloat16* xraw = reinterpret_cast<const __nv_bfloat16*>(sm + sp.o_xraw);
+  const float* cxs = reinterpret_cast<const float*>(sm + sp.o_cx);
+  const float* ths = reinterpret_cast<const float*>(sm + sp.o_th);
+  float2* cs = reinterpret_cast<float2*>(sm + sp.o_cs);
+  float* yp = reinterpret_cast<float*>(sm + sp.o_yp);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + sp.o_tm);
+
+  auto try_wait = [&](uint32_t bar, uint32_t par) -> bool {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred q;\n mbarrier.try_wait.parity.shared::cta.b64 q, [%1], %2;\n selp.u32 %0, 1, 0, q;\n}\n"
+        : "=r"(done)
+        : "r"(bar), "r"(par)
+        : "memory");
+    return done != 0;
+  };
+  auto wait = [&](uint32_t bar, uint32_t par) -> bool {
+    if (try_wait(bar, par)) return true;
+    const uint64_t t0 = globaltimer();
+    while (!try_wait(bar, par)) {
+      if (globaltimer() - t0 > kWaitNs) return false;
+    }
+    return true;
+  };
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kSplitTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
+  }
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(full));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(mbar));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    const uint32_t n_st = kRows * kP * 4, n_b = (uint32_t)R * kN * 2, n_cb = (uint32_t)R * kN * 4;
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full),
+                 "r"(n_st + 2 * n_b + n_cb + kP * 2 + kP * 4 + kN / 2 * 4)
+                 : "memory");
+    const int64_t bc = ((bi * G + g) * R) * (int64_t)kN;
+    bulk_g2s(sbase + sp.o_st, p.h + (bh * kN + n0) * kP, n_st, full);
+    bulk_g2s(sbase + sp.o_braw, static_cast<const __nv_bfloat16*>(p.B) + bc, n_b, full);
+    bulk_g2s(sbase + sp.o_craw, static_cast<const __nv_bfloat16*>(p.C) + bc, n_b, full);
+    bulk_g2s(sbase + sp.o_cbold, p.carry_B + bh * R * kN, n_cb, full);
+    bulk_g2s(sbase + sp.o_xraw, static_cast<const __nv_bfloat16*>(p.x) + bh * kP, kP * 2, full);
+    bulk_g2s(sbase + sp.o_cx, p.carry_x + bh * kP, kP * 4, full);
+    bulk_g2s(sbase + sp.o_th, p.theta + (bi * G + g) * (kN / 2), kN / 2 * 4, full);
+  }
+  // per-unit scalars and this thread's weights while the copies land
+  const float delta = __ldg(p.dt + bh), lm = __ldg(p.lam + bh);
+  const float alpha = expf(delta * __ldg(p.A + bh));
+  float wxr[RT], wor[RT];
+#pragma unroll
+  for (int k = 0; k < RT; ++k) {
+    wxr[k] = p.W_x ? __ldg(p.W_x + ((int64_t)hi * R + k) * kP + tid) : 1.0f;
+    wor[k] = p.W_o ? __ldg(p.W_o + ((int64_t)hi * R + k) * kP + tid) : 1.0f;
+  }
+  const float Dh = p.D ? __ldg(p.D + hi) : 0.0f;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+
+  bool ok = wait(full, 0);
+  ok = !__syncthreads_or(!ok);
+  float hv[kRows];
+  if (ok) {
+    // Xcat row p = tid: W_x[k] x_t for k < R, W_x[k-R] x_{t-1} for R <= k < 2R
+    {
+      const float xv = __bfloat162float(xraw[tid]), cxv = cxs[tid];
+      float fx[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) fx[k] = 0.0f;
+#pragma unroll
+      for (int k = 0; k < RT; ++k) {
+        fx[k] = wxr[k] * xv;
+        fx[RT + k] = wxr[k] * cxv;
+      }
+      sts128(sX + sw128(tid, 0, 128 * 128),
+             make_uint4(pack_bf16(fx[0], fx[1]), pack_bf16(fx[2], fx[3]), pack_bf16(fx[4], fx[5]), pack_bf16(fx[6], fx[7])));
+      sts128(sX + sw128(tid, 1, 128 * 128),
+             make_uint4(pack_bf16(fx[8], fx[9]), pack_bf16(fx[10], fx[11]), pack_bf16(fx[12], fx[13]),
+                        pack_bf16(fx[14], fx[15])));
+    }
+    if (warp == 0) {
+      // Bcat row n = n0 + lane: gamma Bb_k for k < R, alpha beta' Rot(Bb'_{k-R}) for R <= k < 2R
+      const int n = n0 + lane, m = n & ~1;
+      float sn, cn;
+      sincos_reduced(p.angle_direct ? ths[n >> 1] : delta * ths[n >> 1], &sn, &cn);
+      if ((lane & 1) == 0) cs[lane >> 1] = make_float2(alpha * cn, alpha * sn);
+      const float gm = lm * delta, ab = alpha * (1.0f - lm) * delta;
+      const float* bB = p.bias_B ? p.bias_B + (int64_t)hi * R * kN : nullptr;
+      float fb[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) fb[k] = 0.0f;
+#pragma unroll
+      for (int k = 0; k < RT; ++k) {
+        const float b0 = bB ? __ldg(bB + k * kN + m) : 0.0f, b1 = bB ? __ldg(bB + k * kN + m + 1) : 0.0f;
+        const float bn = (n & 1) ? b1 : b0;
+        fb[k] = gm * (__bfloat162float(Braw[k * kN + n]) + bn);
+        const float v0 = cBs[k * kN + m] + b0, v1 = cBs[k * kN + m + 1] + b1;
+        fb[RT + k] = ab * ((n & 1) ? fmaf(sn, v0, cn * v1) : fmaf(cn, v0, -sn * v1));
+      }
+      sts128(sB + sw128(lane, 0, kRows * 128),
+             make_uint4(pack_bf16(fb[0], fb[1]), pack_bf16(fb[2], fb[3]), pack_bf16(fb[4], fb[5]), pack_bf16(fb[6], fb[7])));
+      sts128(sB + sw128(lane, 1, kRows * 128),
+             make_uint4(pack_bf16(fb[8], fb[9]), pack_bf16(fb[10], fb[11]), pack_bf16(fb[12], fb[13]),
+                        pack_bf16(fb[14], fb[15])));
+    } else if (warp == 1) {
+      // Cb of the slice: rows r < 16 (zero for r >= R), chunks of 8 elements of n
+      const float* bC = p.bias_C ? p.bias_C + (int64_t)hi * R * kN : nullptr;
+      for (int it = lane; it < 16 * (kRows / 8); it += 32) {
+        const int r = it / (kRows / 8), nc = it % (kRows / 8);
+        float fc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int n = n0 + 8 * nc + e;
+          fc[e] = r < R ? __bfloat162float(Craw[r * kN + n]) + (bC ? __ldg(bC + r * kN + n) : 0.0f) : 0.0f;
+        }
+        sts128(sC + sw128(r, nc, 16 * 128),
+               make_uint4(pack_bf16(fc[0], fc[1]), pack_bf16(fc[2], fc[3]), pack_bf16(fc[4], fc[5]),
+                          pack_bf16(fc[6], fc[7])));
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kRows; ++j) hv[j] = hst[j * kP + tid];
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // ---- MMA 1: D^T = Xcat Bcat_slice^T (M = 128, N = 32, K = 16)
+  if (ok && warp == 0) {
+    mma_ss_w(tmem, sdesc(sX, 16, 1024), sdesc(sB, 16, 1024), idesc_bf16(kP, kRows, false, false), 0);
+    mma_commit_w(mbar);
+  }
+  bool okm = ok ? wait(mbar, 0) : false;
+  tc_fence_after();
+  if (okm) {
+    uint32_t dv[32];
+    tmem_ld32(tmem + lane_base, dv);
+    tmem_wait_ld();
+    float* hg = p.h + (bh * kN + n0) * kP + tid;
+    const float4* cs4 = reinterpret_cast<const float4*>(cs);
+    uint32_t hb[16];
+#pragma unroll
+    for (int jj = 0; jj < 16; jj += 2) {
+      const float4 rc = cs4[jj / 2];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int i = jj + hh;
+        const float ac = hh ? rc.z : rc.x, as = hh ? rc.w : rc.y;
+        const float e0 = fmaf(ac, hv[2 * i], fmaf(-as, hv[2 * i + 1], __uint_as_float(dv[2 * i])));
+        const float e1 = fmaf(as, hv[2 * i], fmaf(ac, hv[2 * i + 1], __uint_as_float(dv[2 * i + 1])));
+        hg[(2 * i) * kP] = e0;
+        hg[(2 * i + 1) * kP] = e1;
+        hb[i] = pack_bf16(e0, e1);
+      }
+    }
+    tmem_st16(tmem + lane_base + kSColHB, hb);
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  okm = !__syncthreads_or(!okm);
+  tc_fence_after();
+  // ---- MMA 2: partial Y^T = h_slice^T Cb_slice (K = 32, h from tensor memory)
+  if (okm && warp == 0) {
+#pragma unroll
+    for (int k = 0; k < kRows / 16; ++k)
+      mma_ts_w(tmem + kSColY, tmem + kSColHB + 8 * k, sdesc(sC + 32 * k, 16, 1024), idesc_bf16(kP, 16, false, false),
+               k > 0);
+    mma_commit_w(mbar);
+  }
+  const bool okm2 = okm ? wait(mbar, 1) : false;
+  tc_fence_after();
+  if (okm2) {
+    uint32_t yv[16];
+    tmem_ld16(tmem + lane_base + kSColY, yv);
+    tmem_wait_ld();
+    float acc = 0.0f;
+#pragma unroll
+    for (int r = 0; r < RT; ++r) acc = fmaf(wor[r], __uint_as_float(yv[r]), acc);
+    yp[tid] = acc;
+  }
+  const bool good = !__syncthreads_or(!okm2);
+  // every CTA of the cluster has its copies landed and its partial output in place
+  cluster_sync();
+  if (good && crank == 0) {
+    float acc = yp[tid] + Dh * __bfloat162float(xraw[tid]);
+#pragma unroll
+    for (uint32_t c = 1; c < kSplit; ++c) acc += ld_dsmem(smem_u32(yp + tid), c);
+    reinterpret_cast<__nv_bfloat16*>(p.y)[bh * kP + tid] = __float2bfloat16_rn(acc);
+  }
+  if (good) {
+    // the new carry, each CTA its slice (every CTA's copy of the old carry has landed)
+    for (int i = tid; i < R * kRows; i += kST) {
+      const int r = i / kRows, n = n0 + i % kRows;
+      p.carry_B[bh * R * kN + r * kN + n] = __bfloat162float(Braw[r * kN + n]);
+    }
+    if (tid / kRows == (int)crank) p.carry_x[bh * kP + tid] = __bfloat162float(xraw[tid]);
+  }
+  if (!good && tid == 0) {
+    wait(full, 0);  // copies still in flight land before the CTA leaves (bounded)
+    set_status(p.status, M3_ERR_TIMEOUT);
+  }
+  // CTA 0 has read the other CTAs' partial outputs
+  cluster_sync();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kSplitTmemCols));
+  }
+}
+
+template <int RT>
+cudaError_t launch_split_rt(const Params& p, const SplitPlan& sp, cudaStream_t stream) {
+  auto k = decode_tc_split_kernel<RT>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
+  if (e != cudaSuccess) return e;
+  k<<<(unsigned)(p.b * p.H * kSplit), kST, sp.total, stream>>>(p, sp);
+  return cudaGetLastError();
+}
+
+// Resident split CTAs per SM stay within the SM's tensor memory (512 columns), so that no
+// allocation ever waits on a CTA that itself waits at a cluster barrier.
+template <int RT>
+bool split_fits(const SplitPlan& sp) {
+  static signed char cache[64] = {0};  // per device: 0 unknown, 1 fits, -1 does not
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (cache[dev] == 0) {
+    int per_sm = 0;
+    auto k = decode_tc_split_kernel<RT>;
+    const bool fits =
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total) == cudaSuccess &&
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kST, sp.total) == cudaSuccess && per_sm >= 1 &&
+        (uint32_t)per_sm * kSplitTmemCols <= 512;
+    cache[dev] = fits ? 1 : -1;
+  }
+  return cache[dev] > 0;
+}
+
+cudaError_t launch_split(const Params& p, cudaStream_t stream, bool* used) {
+  const SplitPlan sp = split_plan(p.R);
+  *used = true;
+  switch (p.R) {
+#define M3_SPLIT_CASE(r) \
+  case r:                \
+    if (!split_fits<r>(sp)) break; \
+    return launch_split_rt<r>(p, sp, stream);
+    M3_SPLIT_CASE(1) M3_SPLIT_CASE(2) M3_SPLIT_CASE(3) M3_SPLIT_CASE(4)
+    M3_SPLIT_CASE(5) M3_SPLIT_CASE(6) M3_SPLIT_CASE(7) M3_SPLIT_CASE(8)
+#undef M3_SPLIT_CASE
+    default: break;
+  }
+  *used = false;
+  return cudaSuccess;
+}
+
 }  // namespace
 
 bool decode_tc_supported(const Params& p) {
@@ -545,6 +897,11 @@ cudaError_t launch_decode_tc(const Params& p, cudaStream_t stream) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t units = p.b * p.H;
+  if (units * kSplit <= (int64_t)sms) {
+    bool used = false;
+    const cudaError_t e = launch_split(p, stream, &used);
+    if (used) return e;
+  }
   const unsigned grid = (unsigned)(units < sms ? units : sms);
   const TcPlan tp = tc_plan(p.R);
   switch (p.R) {

@@ -181,11 +181,22 @@ def test_decode_tc_ranks(R, G):
     check_decode(inp, 5, st)
 
 
+# up to four units per SM take the split form (a cluster of four CTAs per unit, 32 state rows
+# each); more units take the persistent form (one CTA per SM walking its units through two stages)
+
+@pytest.mark.parametrize("R,G", [(1, 1), (3, 2), (8, 2)])
+def test_decode_tc_persistent_ranks(R, G):
+    shape = dict(b=10, L=3, H=64, P=128, N=128, R=R, G=G)  # 640 units
+    inp = make_inputs(dtype="bf16", seed=160 + R, extras=True, **shape)
+    st = make_state(10, 64, 128, 128, R, seed=170 + R)
+    check_decode(inp, 3, st)
+
+
 def test_decode_tc_stage_refills():
-    # 320 (batch, head) units over at most 148 CTAs: each CTA refills its two stages
-    shape = dict(b=40, L=3, H=8, P=128, N=128, R=4, G=1)
+    # 640 (batch, head) units over at most 148 persistent CTAs: each CTA refills its two stages
+    shape = dict(b=40, L=3, H=16, P=128, N=128, R=4, G=1)
     inp = make_inputs(dtype="bf16", seed=150, extras=True, **shape)
-    st = make_state(40, 8, 128, 128, 4, seed=151)
+    st = make_state(40, 16, 128, 128, 4, seed=151)
     check_decode(inp, 3, st)
 
 
