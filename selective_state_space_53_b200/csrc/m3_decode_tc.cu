@@ -151,7 +151,7 @@ struct TcPlan {
   uint32_t o_st, o_b, o_c, o_cb, o_x, o_cx, o_th, o_sc;  // inside a stage
   uint32_t o_bx;    // Bcat (k-chunks 0-1) and Xcat (k-chunks 2-3) of a 128-row SW128 K-major tile
   uint32_t o_cbt;   // bf16 Cb, K-major SW128 (16 rows r, 64-element blocks of n), one per stage
-  uint32_t o_cs;    // rotation table (cos, sin) of the unit
+  uint32_t o_cs;    // rotation table of the unit, (alpha cos, alpha sin) per pair
   uint32_t o_xr;    // x_t of the unit, one copy per stage (read by the output after the stage is reused)
   uint32_t o_w;     // bias_B, bias_C, W_x, W_o of the current head, fp32
   uint32_t o_tm, o_bar, o_stage0;

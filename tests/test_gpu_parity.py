@@ -208,6 +208,24 @@ def test_decode_tc_long_run():
     check_decode(inp, 256, st)
 
 
+# per-head B and C (G = H, the "per-head B/C" variant): each head reads its own B_t, C_t and theta_t
+
+@pytest.mark.parametrize("shape", [
+    dict(b=2, L=150, H=4, P=64, N=64, R=2, G=4),
+    dict(b=1, L=100, H=4, P=128, N=128, R=4, G=4),
+], ids=["P64", "P128"])
+def test_per_head_bc_prefill(shape):
+    check_scan(make_inputs(dtype="bf16", seed=180, extras=True, **shape))
+
+
+@pytest.mark.parametrize("b,H", [(2, 4), (10, 64)], ids=["split", "persistent"])
+def test_per_head_bc_decode_tc(b, H):
+    shape = dict(b=b, L=3, H=H, P=128, N=128, R=4, G=H)
+    inp = make_inputs(dtype="bf16", seed=181, extras=True, **shape)
+    st = make_state(b, H, 128, 128, 4, seed=182)
+    check_decode(inp, 3, st)
+
+
 def test_decode_b512_sampled_heads():
     # the largest decode batch of the 1.5B-scale layer (16384 units, a 1 GiB state), four tokens;
     # the oracle follows sampled (batch, head) pairs
