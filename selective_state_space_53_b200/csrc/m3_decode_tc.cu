@@ -520,10 +520,44 @@ __global__ void __launch_bounds__(kT, 1) decode_tc_kernel(Params p, TcPlan tp) {
   }
 }
 
+// SM count and opt-in shared memory per block of the current device, queried once per device
+struct TcDevice {
+  int sms = 0, optin = 0;
+};
+TcDevice tc_device() {
+  static TcDevice cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TcDevice{};
+  TcDevice& d = cache[dev];
+  if (d.sms == 0) {
+    int sms = 0, optin = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      return TcDevice{};
+    d.optin = optin;
+    d.sms = sms;
+  }
+  return d;
+}
+
+// Dynamic shared memory above 48 KiB needs the kernel attribute: set once per device (`cache`
+// holds the size set so far for each device, per kernel)
+template <typename Kernel>
+cudaError_t ensure_smem(Kernel kernel, int bytes, int* cache) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && cache[dev] >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) cache[dev] = bytes;
+  return e;
+}
+
 template <int RT>
 cudaError_t launch_tc_rt(const Params& p, const TcPlan& tp, unsigned grid, cudaStream_t stream) {
+  static int smem_set[64] = {0};
   auto k = decode_tc_kernel<RT>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tp.total);
+  cudaError_t e = ensure_smem(k, (int)tp.total, smem_set);
   if (e != cudaSuccess) return e;
   k<<<grid, kT, tp.total, stream>>>(p, tp);
   return cudaGetLastError();
@@ -838,8 +872,9 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kST, 1)
 
 template <int RT>
 cudaError_t launch_split_rt(const Params& p, const SplitPlan& sp, cudaStream_t stream) {
+  static int smem_set[64] = {0};
   auto k = decode_tc_split_kernel<RT>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
+  cudaError_t e = ensure_smem(k, (int)sp.total, smem_set);
   if (e != cudaSuccess) return e;
   k<<<(unsigned)(p.b * p.H * kSplit), kST, sp.total, stream>>>(p, sp);
   return cudaGetLastError();
@@ -884,18 +919,14 @@ cudaError_t launch_split(const Params& p, cudaStream_t stream, bool* used) {
 }  // namespace
 
 bool decode_tc_supported(const Params& p) {
-  int dev = 0, optin = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
-    return false;
-  return p.dtype == M3_BF16 && p.N == kN && p.P == kP && p.R >= 1 && p.R <= kMaxR &&
-         (int)tc_plan(p.R).total <= optin;
+  if (!(p.dtype == M3_BF16 && p.N == kN && p.P == kP && p.R >= 1 && p.R <= kMaxR)) return false;
+  const TcDevice d = tc_device();
+  return d.sms > 0 && (int)tc_plan(p.R).total <= d.optin;
 }
 
 cudaError_t launch_decode_tc(const Params& p, cudaStream_t stream) {
   if (p.b * p.H == 0) return cudaSuccess;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = tc_device().sms > 0 ? tc_device().sms : 148;
   const int64_t units = p.b * p.H;
   if (units * kSplit <= (int64_t)sms) {
     bool used = false;
