@@ -181,8 +181,9 @@ def test_decode_tc_ranks(R, G):
     check_decode(inp, 5, st)
 
 
-# up to four units per SM take the split form (a cluster of four CTAs per unit, 32 state rows
-# each); more units take the persistent form (one CTA per SM walking its units through two stages)
+# a call whose split CTAs fit in one wave (4 x units <= SMs) takes the split form (a cluster of four
+# CTAs per unit, 32 state rows each); larger calls take the persistent form (one CTA per SM walking
+# its units through two stages).  The small shapes above run the split form, these the persistent one
 
 @pytest.mark.parametrize("R,G", [(1, 1), (3, 2), (8, 2)])
 def test_decode_tc_persistent_ranks(R, G):
