@@ -193,6 +193,17 @@ def test_decode_tc_persistent_ranks(R, G):
     check_decode(inp, 3, st)
 
 
+@pytest.mark.parametrize("R", [2, 5, 6, 7])
+@pytest.mark.parametrize("b,H,G", [(2, 4, 2), (10, 64, 4)], ids=["split", "persistent"])
+def test_decode_tc_other_ranks(R, b, H, G):
+    # every rank the tensor-core decode is instantiated for; 2R > 8 fills both k-chunks of the
+    # operand tiles (R = 5, 6, 7), 2R <= 8 leaves the second one zero (R = 2)
+    shape = dict(b=b, L=3, H=H, P=128, N=128, R=R, G=G)
+    inp = make_inputs(dtype="bf16", seed=190 + R, extras=True, **shape)
+    st = make_state(b, H, 128, 128, R, seed=200 + R)
+    check_decode(inp, 3, st)
+
+
 def test_decode_tc_stage_refills():
     # 640 (batch, head) units over at most 148 persistent CTAs: each CTA refills its two stages
     shape = dict(b=40, L=3, H=16, P=128, N=128, R=4, G=1)
