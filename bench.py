@@ -38,9 +38,9 @@ WORKLOAD = "p1_layer"
 DECODE_WORKLOAD = "decode_b128"
 L2_BYTES = 126 * 1024 * 1024
 
-# dram bytes (read + write) of one m3_scan_fwd on p1_layer (state pass + full pass) from the
-# ncu capture summarised in profiles/scan_tc_p1_layer.md; set to None whenever the kernel
-# changes until a new capture is taken.
+# dram bytes (read + write) of one m3_scan_fwd on p1_layer (state pass + full pass), from the
+# committed ncu summary of that kernel; set to None whenever the kernel changes until a new
+# capture is taken.
 PREFILL_DRAM_BYTES_PER_LAUNCH = 61815040
 
 

@@ -15,15 +15,17 @@ bool seq_scan_supported(int P, int N, int R);
 namespace {
 // Device address of the status word, looked up once per device.
 int* status_word() {
-  static int* cache[64] = {nullptr};
+  static m3::PerDevice<int*> cache;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!cache[dev]) {
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  int* out = nullptr;
+  const bool ok = cache.get(dev, &out, [](int** v) {
     void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, m3::g_status) != cudaSuccess) return nullptr;
-    cache[dev] = static_cast<int*>(ptr);
-  }
-  return cache[dev];
+    if (cudaGetSymbolAddress(&ptr, m3::g_status) != cudaSuccess) return false;
+    *v = static_cast<int*>(ptr);
+    return true;
+  });
+  return ok ? out : nullptr;
 }
 }  // namespace
 

@@ -5,6 +5,9 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "../../include/m3.h"
 
 namespace m3 {
@@ -54,6 +57,64 @@ __device__ __forceinline__ void store_out(void* base, int64_t i, float v) {
     reinterpret_cast<float*>(base)[i] = v;
   }
 }
+
+// A value per CUDA device, filled once and then read without locking, safe for callers on
+// several host threads: the first caller for a device runs `fill` under a mutex and publishes
+// the value with a release store of `ready`; later callers see `ready` with an acquire load,
+// so they never read a half-written value.  A fill that fails leaves the slot empty (it is
+// retried by the next call).  Devices beyond kMaxDevices are reported as failures.
+template <typename T>
+class PerDevice {
+ public:
+  static constexpr int kMaxDevices = 64;
+  template <typename F>
+  bool get(int dev, T* out, F&& fill) {
+    if (dev < 0 || dev >= kMaxDevices) return false;
+    Slot& s = slots_[dev];
+    if (!s.ready.load(std::memory_order_acquire)) {
+      std::lock_guard<std::mutex> lock(mu_);
+      if (!s.ready.load(std::memory_order_relaxed)) {
+        T v{};
+        if (!fill(&v)) return false;
+        s.value = v;
+        s.ready.store(true, std::memory_order_release);
+      }
+    }
+    *out = s.value;
+    return true;
+  }
+
+ private:
+  struct Slot {
+    std::atomic<bool> ready{false};
+    T value{};
+  };
+  Slot slots_[kMaxDevices];
+  std::mutex mu_;
+};
+
+// Largest dynamic shared memory size set so far on each device for one kernel: the attribute
+// call runs under a mutex, and a size already set is seen through an acquire load.
+class SmemAttr {
+ public:
+  template <typename Kernel>
+  cudaError_t ensure(Kernel kernel, int bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= PerDevice<int>::kMaxDevices) return cudaErrorInvalidDevice;
+    if (set_[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(mu_);
+    if (set_[dev].load(std::memory_order_relaxed) >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) set_[dev].store(bytes, std::memory_order_release);
+    return e;
+  }
+
+ private:
+  std::atomic<int> set_[PerDevice<int>::kMaxDevices] = {};
+  std::mutex mu_;
+};
 
 // Launchers (defined in the kernel files); return cudaGetLastError() of the launch.
 cudaError_t launch_scan_sequential(const Params& p, cudaStream_t stream);

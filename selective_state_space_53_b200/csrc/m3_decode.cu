@@ -424,21 +424,22 @@ struct DeviceLimits {
 };
 // SM count and opt-in shared memory per block of the current device (cached per device).
 DeviceLimits device_limits() {
-  static DeviceLimits cache[64];
+  static PerDevice<DeviceLimits> cache;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DeviceLimits{};
-  DeviceLimits& d = cache[dev];
-  if (d.sms == 0) {
+  if (cudaGetDevice(&dev) != cudaSuccess) return DeviceLimits{};
+  DeviceLimits out{};
+  cache.get(dev, &out, [dev](DeviceLimits* d) {
     int sms = 0, optin = 0, per_sm = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess)
-      return DeviceLimits{};
-    d.smem_optin = optin;
-    d.smem_sm = per_sm;
-    d.sms = sms;
-  }
-  return d;
+      return false;
+    d->sms = sms;
+    d->smem_optin = optin;
+    d->smem_sm = per_sm;
+    return true;
+  });
+  return out;
 }
 
 template <int RT>

@@ -525,39 +525,27 @@ struct TcDevice {
   int sms = 0, optin = 0;
 };
 TcDevice tc_device() {
-  static TcDevice cache[64];
+  static PerDevice<TcDevice> cache;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TcDevice{};
-  TcDevice& d = cache[dev];
-  if (d.sms == 0) {
+  if (cudaGetDevice(&dev) != cudaSuccess) return TcDevice{};
+  TcDevice out{};
+  cache.get(dev, &out, [dev](TcDevice* d) {
     int sms = 0, optin = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
-      return TcDevice{};
-    d.optin = optin;
-    d.sms = sms;
-  }
-  return d;
-}
-
-// Dynamic shared memory above 48 KiB needs the kernel attribute: set once per device (`cache`
-// holds the size set so far for each device, per kernel)
-template <typename Kernel>
-cudaError_t ensure_smem(Kernel kernel, int bytes, int* cache) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && cache[dev] >= bytes) return cudaSuccess;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && dev >= 0 && dev < 64) cache[dev] = bytes;
-  return e;
+      return false;
+    d->sms = sms;
+    d->optin = optin;
+    return true;
+  });
+  return out;
 }
 
 template <int RT>
 cudaError_t launch_tc_rt(const Params& p, const TcPlan& tp, unsigned grid, cudaStream_t stream) {
-  static int smem_set[64] = {0};
+  static SmemAttr smem_set;
   auto k = decode_tc_kernel<RT>;
-  cudaError_t e = ensure_smem(k, (int)tp.total, smem_set);
+  cudaError_t e = smem_set.ensure(k, (int)tp.total);
   if (e != cudaSuccess) return e;
   k<<<grid, kT, tp.total, stream>>>(p, tp);
   return cudaGetLastError();
@@ -872,9 +860,9 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kST, 1)
 
 template <int RT>
 cudaError_t launch_split_rt(const Params& p, const SplitPlan& sp, cudaStream_t stream) {
-  static int smem_set[64] = {0};
+  static SmemAttr smem_set;
   auto k = decode_tc_split_kernel<RT>;
-  cudaError_t e = ensure_smem(k, (int)sp.total, smem_set);
+  cudaError_t e = smem_set.ensure(k, (int)sp.total);
   if (e != cudaSuccess) return e;
   k<<<(unsigned)(p.b * p.H * kSplit), kST, sp.total, stream>>>(p, sp);
   return cudaGetLastError();
@@ -884,19 +872,19 @@ cudaError_t launch_split_rt(const Params& p, const SplitPlan& sp, cudaStream_t s
 // allocation ever waits on a CTA that itself waits at a cluster barrier.
 template <int RT>
 bool split_fits(const SplitPlan& sp) {
-  static signed char cache[64] = {0};  // per device: 0 unknown, 1 fits, -1 does not
+  static PerDevice<bool> cache;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-  if (cache[dev] == 0) {
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  bool fits = false;
+  cache.get(dev, &fits, [&sp](bool* v) {
     int per_sm = 0;
     auto k = decode_tc_split_kernel<RT>;
-    const bool fits =
-        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total) == cudaSuccess &&
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kST, sp.total) == cudaSuccess && per_sm >= 1 &&
-        (uint32_t)per_sm * kSplitTmemCols <= 512;
-    cache[dev] = fits ? 1 : -1;
-  }
-  return cache[dev] > 0;
+    *v = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total) == cudaSuccess &&
+         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kST, sp.total) == cudaSuccess && per_sm >= 1 &&
+         (uint32_t)per_sm * kSplitTmemCols <= 512;
+    return true;
+  });
+  return fits;
 }
 
 cudaError_t launch_split(const Params& p, cudaStream_t stream, bool* used) {

@@ -13,7 +13,10 @@
 // and nothing is cleared.
 #include "m3_common.cuh"
 
-// 16 MiB: the most the segment planner asks for on a 148-SM B200 is about 10 MiB.
+// 16 MiB, sized for a 148-SM B200: there the segment planner asks for at most about 14 MiB
+// (13.95 MiB, at 74 (batch, head) sequences with d_state = headdim = 128).  The planner fills
+// the SMs, so on a part with more SMs the need grows with the SM count (about 16 MiB at 170
+// SMs); dimensions that would need more than the array get M3_ERR_WORKSPACE.
 static constexpr size_t kScratchBytes = size_t(16) << 20;
 static __device__ __align__(256) unsigned char g_scan_scratch[kScratchBytes];
 
@@ -23,15 +26,17 @@ namespace {
 // Device address of g_scan_scratch for the current device, looked up on the first call
 // made with that device current (host code cannot use the symbol itself as an address).
 unsigned char* scratch_address() {
-  static unsigned char* cache[64] = {nullptr};
+  static PerDevice<unsigned char*> cache;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!cache[dev]) {
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  unsigned char* out = nullptr;
+  const bool ok = cache.get(dev, &out, [](unsigned char** v) {
     void* ptr = nullptr;
-    if (cudaGetSymbolAddress((void**)&ptr, g_scan_scratch) != cudaSuccess) return nullptr;
-    cache[dev] = static_cast<unsigned char*>(ptr);
-  }
-  return cache[dev];
+    if (cudaGetSymbolAddress((void**)&ptr, g_scan_scratch) != cudaSuccess) return false;
+    *v = static_cast<unsigned char*>(ptr);
+    return true;
+  });
+  return ok ? out : nullptr;
 }
 
 }  // namespace

@@ -1197,14 +1197,17 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
 // ------------------------------------------------------------------ host side
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  // the driver entry point is the same for every device; it is looked up once, under the
+  // once-flag, so concurrent first calls neither race nor repeat the query
+  static std::once_flag once;
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  std::call_once(once, [] {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
+  });
   return fn;
 }
 
