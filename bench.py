@@ -3,19 +3,20 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-A step is one pass of the whole hot path over one batch of the page-1-shaped layer
-(batch 4, seqlen 2048, 24 heads x 64, d_state 64, MIMO rank 2, bf16 x/B/C, fp32 state):
-m3_scan_fwd over the 4 x 2048 prompt tokens, then m3_decode_step for one more token
-per sequence from the final state.  value = tokens/s over all ranks (weak scaling:
-every rank runs its own batch; no data-path collective).  Inputs are seeded and
-synthetic; a ring of input sets larger than L2 rotates between steps.
+A step is one pass of the whole hot path over one batch of the 1.5B-scale layer (batch 2,
+seqlen 32768, 32 heads x 128, d_state 128, MIMO rank 4, bf16 x/B/C, fp32 state): m3_scan_fwd
+over the 2 x 32768 prompt tokens, then m3_decode_step for one more token per sequence from the
+final state.  value = tokens/s over all ranks (weak scaling: every rank runs its own batch; no
+data-path collective).  Inputs are seeded and synthetic; one input set (1.25 GB) is larger
+than L2, and two sets alternate between steps.
 
-Extra keys: "prefill" / "decode" give each kernel measured on its own (decode on the
-1.5B-scale layer, batch 128, state 256 MiB > L2; "decode.sweep" the batches 1, 16 and 512,
-"prefill.sweep_l15b" the 1.5B-scale layer's prefill at 2K, 8K and 32K tokens); "roofline" is the dominant kernel
-(the tensor-core prefill) against MEASURED_PEAKS.json; "cpu_baseline" times the fp64
-oracle (test infrastructure) on a bounded sample; "e2e" times the same step through
-the C ABI with pinned host buffers and the host<->device copies inside the timed region.
+Extra keys: "prefill" / "decode" give each kernel measured on its own ("prefill.p1_layer" the
+page-1-shaped layer, "prefill.sweep_l15b" the 1.5B-scale layer at 2K and 8K tokens; decode on
+the 1.5B-scale layer at batch 128, "decode.sweep" batches 1, 16 and 512); "roofline" is the
+dominant kernel (the tensor-core prefill) against MEASURED_PEAKS.json; "cpu_baseline" times the
+fp64 oracle (test infrastructure) on a bounded sample and compares its outputs with the GPU's;
+"e2e" times the same step through the C ABI with pinned host buffers and the host<->device
+copies inside the timed region.
 
 --impl reference times the fp64 CPU oracle alone (the reference arm of this build).
 """
@@ -34,14 +35,15 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "Mamba-3 SSM tokens/s (prefill, decode) and % of tensor-core / HBM roofline"
-WORKLOAD = "p1_layer"
+WORKLOAD = "l15b_32k"
+EXTRA_PREFILL = "p1_layer"
 DECODE_WORKLOAD = "decode_b128"
 L2_BYTES = 126 * 1024 * 1024
 
-# dram bytes (read + write) of one m3_scan_fwd on p1_layer (state pass + full pass), from the
-# committed ncu summary of that kernel; set to None whenever the kernel changes until a new
-# capture is taken.
-PREFILL_DRAM_BYTES_PER_LAUNCH = 61815040
+# dram bytes read and written by one m3_scan_fwd on the headline workload (state pass + full
+# pass), from the committed ncu summary of that kernel; None whenever the kernel has changed
+# since the counters were taken.
+PREFILL_DRAM = None  # {"read": bytes, "write": bytes, "note": "..."}
 
 
 def log(*a):
@@ -53,12 +55,20 @@ def log(*a):
 def prefill_bytes(d):
     """Algorithmic HBM bytes of one m3_scan_fwd: every input read once, y written once,
     state (h, carry) read and written once."""
+    r, w = prefill_bytes_rw(d)
+    return r + w
+
+
+def prefill_bytes_rw(d):
+    """(read, written) algorithmic bytes of one m3_scan_fwd: x, B, C, theta, dt, A, lam and
+    the state read once; y and the state written once."""
     b, L, H, P, N, R, G = (d[k] for k in ("b", "L", "H", "P", "N", "R", "G"))
     e = 2 if d["dtype"] == "bf16" else 4
     tok = b * L
-    io = tok * (H * P * e * 2 + 2 * G * R * N * e + G * (N // 2) * 4 + 3 * H * 4)
-    state = 2 * b * H * (N * P + R * N + P) * 4
-    return io + state
+    state = b * H * (N * P + R * N + P) * 4
+    read = tok * (H * P * e + 2 * G * R * N * e + G * (N // 2) * 4 + 3 * H * 4) + state
+    written = tok * H * P * e + state
+    return read, written
 
 
 def prefill_flops(d, chunk=32):
@@ -227,6 +237,26 @@ def token_slice(dev, t):
     return {k: (v[:, t].contiguous() if (v is not None and k in seq) else v) for k, v in dev.items()}
 
 
+def _prefill_record(name, cfg, ms, peaks):
+    """Throughput and roofline fractions of one m3_scan_fwd of `cfg` that took `ms`."""
+    by = prefill_bytes(cfg)
+    fl, fl_intra = prefill_flops(cfg)
+    sec = ms * 1e-3
+    return {
+        "workload": "%s m3_scan_fwd b%d L%d H%d P%d N%d R%d" % (name, cfg["b"], cfg["L"], cfg["H"], cfg["P"],
+                                                              cfg["N"], cfg["R"]),
+        "tokens_per_s": cfg["b"] * cfg["L"] / sec, "ms_per_launch": ms,
+        "tflops": fl / sec / 1e12,
+        "tensor_frac_of_measured_burst": fl / sec / 1e12 / peaks["bf16"],
+        "tensor_frac_of_measured_sustained": fl / sec / 1e12 / peaks["bf16_sus"],
+        "intra_chunk_tflops": fl_intra / sec / 1e12,
+        "intra_chunk_frac_of_measured_burst": fl_intra / sec / 1e12 / peaks["bf16"],
+        "intra_chunk_frac_of_measured_sustained": fl_intra / sec / 1e12 / peaks["bf16_sus"],
+        "hbm_gbs": by / sec / 1e9, "hbm_frac_of_measured": by / sec / 1e9 / peaks["hbm"],
+        "algorithmic_bytes": by, "algorithmic_flops": fl,
+    }
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -237,6 +267,7 @@ def run_ours(args):
     device = f"cuda:{local}"
     peaks = measured_peaks()
     cfg = dict(CONFIGS[WORKLOAD])
+    log(f"drawing the {WORKLOAD} inputs")
     inp = config_inputs(WORKLOAD, seed=rank_seed(SEEDS[WORKLOAD], rank))
     dims = m3.dims_of(inp)
     dims1 = m3.dims_of(inp, L=1)
@@ -286,34 +317,32 @@ def run_ours(args):
     gpu_launches = (3 if ws_bytes > 0 else 2) * args.steps  # [state pass] + full pass + decode
 
     pf_ms = statistics.mean(prefill_ms)
-    pbytes = prefill_bytes(cfg)
-    pflops, pflops_intra = prefill_flops(cfg)
-    prefill = {
-        "workload": "p1_layer m3_scan_fwd b4 L2048 H24 P64 N64 R2",
-        "tokens_per_s": cfg["b"] * cfg["L"] / (pf_ms / 1e3),
-        "ms_per_launch": pf_ms,
-        "hbm_gbs": pbytes / (pf_ms * 1e-3) / 1e9,
-        "hbm_frac_of_measured": pbytes / (pf_ms * 1e-3) / 1e9 / peaks["hbm"],
-        "tflops": pflops / (pf_ms * 1e-3) / 1e12,
-        "tensor_frac_of_measured_burst": pflops / (pf_ms * 1e-3) / 1e12 / peaks["bf16"],
-        "intra_chunk_tflops": pflops_intra / (pf_ms * 1e-3) / 1e12,
-        "intra_chunk_frac_of_measured_burst": pflops_intra / (pf_ms * 1e-3) / 1e12 / peaks["bf16"],
-        "algorithmic_bytes": pbytes, "algorithmic_flops": pflops,
-    }
-    hbm_frac = prefill["hbm_frac_of_measured"]
-    ten_frac = prefill["tensor_frac_of_measured_burst"]
-    bound = "hbm" if hbm_frac >= ten_frac else "tensor"
+    prefill = _prefill_record(WORKLOAD, cfg, pf_ms, peaks)
+    prefill["ms_per_launch_min_max"] = [min(prefill_ms), max(prefill_ms)]
+    alg_r, alg_w = prefill_bytes_rw(cfg)
+    traffic = None
+    if PREFILL_DRAM is not None:
+        traffic = PREFILL_DRAM["read"] + PREFILL_DRAM["write"]
     roofline = {
-        "kernel": "m3_scan_fwd (scan_tc_kernel: state pass + full pass)",
-        "bound": bound,
-        "achieved": prefill["hbm_gbs"] if bound == "hbm" else prefill["tflops"],
-        "peak": peaks["hbm"] if bound == "hbm" else peaks["bf16"],
-        "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
-        "frac": hbm_frac if bound == "hbm" else ten_frac,
-        "traffic": PREFILL_DRAM_BYTES_PER_LAUNCH,
-        "peak_source": f"{peaks['src']} (MEASURED_PEAKS.json burst)" if peaks["src"] == "measured" else "fallback",
-        "other_bound_frac": ten_frac if bound == "hbm" else hbm_frac,
+        "kernel": "m3_scan_fwd (scan_ws_kernel: state pass + full pass)",
+        "bound": "tensor",
+        "achieved": prefill["tflops"],
+        "peak": peaks["bf16"],
+        "unit": "TFLOP/s",
+        "frac": prefill["tensor_frac_of_measured_burst"],
+        "traffic": traffic,
+        "traffic_read": None if PREFILL_DRAM is None else PREFILL_DRAM["read"],
+        "traffic_write": None if PREFILL_DRAM is None else PREFILL_DRAM["write"],
+        "traffic_note": None if PREFILL_DRAM is None else PREFILL_DRAM["note"],
+        "algorithmic_read": alg_r, "algorithmic_write": alg_w,
+        "peak_source": "measured (MEASURED_PEAKS.json, bf16 burst)" if peaks["src"] == "measured" else "fallback",
+        "frac_of_sustained": prefill["tensor_frac_of_measured_sustained"],
+        "intra_chunk_frac": prefill["intra_chunk_frac_of_measured_burst"],
+        "intra_chunk_frac_of_sustained": prefill["intra_chunk_frac_of_measured_sustained"],
+        "other_bound_frac": prefill["hbm_frac_of_measured"],
     }
+    # a y of the ring for the oracle comparison (every set holds the same inputs)
+    y_sample = ring[0]["y"]
 
     decode = run_decode(args, device, peaks) if not args.no_decode else None
     if decode is not None and not args.no_decode_sweep:
@@ -323,22 +352,24 @@ def run_ours(args):
             r = run_decode(args, device, peaks, nm)
             decode["sweep"][nm] = {k: r[k] for k in ("us_per_step", "tokens_per_s", "hbm_gbs", "hbm_frac_of_measured")}
             torch.cuda.empty_cache()
-    stack = run_stack(args, device, peaks) if not args.no_stack else None
     if not args.no_prefill_sweep:
+        prefill[EXTRA_PREFILL] = run_prefill_one(args, device, peaks, EXTRA_PREFILL)
         prefill["sweep_l15b"] = run_prefill_sweep(args, device, peaks)
+    stack = run_stack(args, device, peaks) if not args.no_stack else None
     e2e = run_e2e(args, inp, tok_inp, device, world) if not args.no_e2e else None
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; shapes of the page-1 layer)",
-        "config": {"workload": "p1_layer: m3_scan_fwd over b4 x L2048 (H24 P64 N64 R2, chunk 32) + 1 m3_decode_step",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; shapes of the 1.5B-scale layer)",
+        "config": {"workload": f"{WORKLOAD}: m3_scan_fwd over b{cfg['b']} x L{cfg['L']} (H{cfg['H']} P{cfg['P']} "
+                               f"N{cfg['N']} R{cfg['R']}, chunk 32) + 1 m3_decode_step",
                    "global_batch": cfg["b"] * world, "seq_len": cfg["L"], "parallelism": f"dp{world}",
-                   "l2": f"ring of {n_sets} input sets ({n_sets * per_set / 2**20:.0f} MiB) > L2"},
+                   "l2": f"{n_sets} input sets of {per_set / 2**20:.0f} MiB each (> L2), alternating"},
         "roofline": roofline, "prefill": prefill, "decode": decode, "stack": stack, "e2e": e2e,
         "gpu_launches": gpu_launches, "clocks": clk.summary(),
     }
     if rank == 0 and not args.no_cpu:
-        line["cpu_baseline"] = cpu_baseline(cfg, inp, tokens_step, seconds=args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline(cfg, inp, y_sample, seconds=args.cpu_seconds)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
@@ -347,46 +378,45 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
 
 
-def run_prefill_sweep(args, device, peaks):
-    """m3_scan_fwd on the 1.5B-scale layer (b2, H32 P128 N128 R4) at seqlen 2K, 8K and 32K: mean of
-    5 calls after 2 warm-up calls, each on its own copy of the inputs when one copy fits in L2."""
+def run_prefill_one(args, device, peaks, name, calls=5):
+    """m3_scan_fwd alone on workload `name`: mean of `calls` calls after 2 warm-up calls, each on
+    its own copy of the inputs when one copy fits in L2."""
     import torch
     from selective_state_space_53_b200 import m3
     from selective_state_space_53_b200.inputs import CONFIGS, config_inputs
-    out = {}
+    cfg = dict(CONFIGS[name])
+    inp = config_inputs(name)
+    dims = m3.dims_of(inp)
+    per_set = prefill_bytes(cfg)
+    n_sets = max(1, -(-2 * L2_BYTES // per_set))
+    ring = make_ring(inp, n_sets, device)
+    ws_bytes = m3.m3_scan_workspace_size(dims)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
-    for name in ("l15b_2k", "l15b_8k", "l15b_32k"):
-        cfg = dict(CONFIGS[name])
-        inp = config_inputs(name)
-        dims = m3.dims_of(inp)
-        per_set = prefill_bytes(cfg)
-        n_sets = max(1, -(-2 * L2_BYTES // per_set))
-        ring = make_ring(inp, n_sets, device)
-        ws_bytes = m3.m3_scan_workspace_size(dims)
-        ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
-        for i in range(2):
-            s = ring[i % n_sets]
-            m3.scan(dims, s["dev"], s["state"], y=s["y"], workspace=ws)
-        torch.cuda.synchronize()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
-        for i, (a, b) in enumerate(evs):
-            s = ring[i % n_sets]
-            a.record(stream)
-            m3.scan(dims, s["dev"], s["state"], y=s["y"], workspace=ws)
-            b.record(stream)
-        torch.cuda.synchronize()
-        assert m3.m3_check() == 0
-        ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-        by = prefill_bytes(cfg)
-        fl, fl_intra = prefill_flops(cfg)
-        out[name] = {"ms_per_call": ms, "tokens_per_s": cfg["b"] * cfg["L"] / (ms * 1e-3),
-                     "intra_chunk_tflops": fl_intra / (ms * 1e-3) / 1e12,
-                     "intra_chunk_frac_of_measured_burst": fl_intra / (ms * 1e-3) / 1e12 / peaks["bf16"],
-                     "tflops": fl / (ms * 1e-3) / 1e12, "tensor_frac_of_measured_burst": fl / (ms * 1e-3) / 1e12 / peaks["bf16"],
-                     "hbm_frac_of_measured": by / (ms * 1e-3) / 1e9 / peaks["hbm"], "input_sets": n_sets}
-        del ring, ws
-        torch.cuda.empty_cache()
+    for i in range(2):
+        s = ring[i % n_sets]
+        m3.scan(dims, s["dev"], s["state"], y=s["y"], workspace=ws)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(calls)]
+    for i, (a, b) in enumerate(evs):
+        s = ring[i % n_sets]
+        a.record(stream)
+        m3.scan(dims, s["dev"], s["state"], y=s["y"], workspace=ws)
+        b.record(stream)
+    torch.cuda.synchronize()
+    assert m3.m3_check() == 0
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    out = _prefill_record(name, cfg, ms, peaks)
+    out["input_sets"] = n_sets
+    del ring, ws
+    torch.cuda.empty_cache()
     return out
+
+
+def run_prefill_sweep(args, device, peaks):
+    """m3_scan_fwd on the 1.5B-scale layer (b2, H32 P128 N128 R4) at seqlen 2K and 8K (32K is the
+    headline workload)."""
+    return {name: run_prefill_one(args, device, peaks, name) for name in ("l15b_2k", "l15b_8k")}
 
 
 def run_decode(args, device, peaks, name=DECODE_WORKLOAD):
@@ -584,35 +614,59 @@ def run_e2e(args, inp, tok_inp, device, world):
 
 # ------------------------------------------------------------------ fp64 oracle (CPU)
 
-def _oracle_rate(cfg, inp, pairs, threads=0):
-    """Seconds for the oracle to run `pairs` (batch, head) sequences of the layer."""
+def _prefix(inp, Lp):
+    """The first Lp tokens of every sequence of a draw (the recurrence is causal, so the
+    oracle's outputs on them are the full run's first Lp outputs)."""
+    import copy
+    sub = copy.copy(inp)
+    for k in ("x", "dt", "A", "lam", "B", "C", "theta"):
+        setattr(sub, k, getattr(inp, k)[:, :Lp])
+    sub.dims = dict(inp.dims, L=Lp)
+    return sub
+
+
+def _oracle_time(inp, pairs, threads=0):
+    """(seconds, y) of the oracle on the (batch, head) pairs of a draw."""
     from oracle import oracle as orc
     t = time.perf_counter()
-    orc.scan_inputs(inp, sel=pairs, threads=threads)
-    return time.perf_counter() - t
+    y, _, _, _ = orc.scan_inputs(inp, sel=pairs, threads=threads)
+    return time.perf_counter() - t, y
 
 
-def cpu_baseline(cfg, inp, tokens_step, seconds=12.0):
-    """The fp64 oracle as it stands, OpenMP over (batch, head) on all host cores, on a
-    bounded sample: as many whole (batch, head) sequences of the layer as fit in about
-    `seconds`.  Scaled to layer tokens/s: a layer token needs all H heads."""
+def _sample_len(inp, pairs, seconds, probe_len=64):
+    """Prefix length whose oracle run over `pairs` takes about `seconds`."""
+    t, _ = _oracle_time(_prefix(inp, probe_len), pairs)
+    per_tok = t / probe_len
+    Lp = int(seconds / max(per_tok, 1e-9))
+    return max(probe_len, min(inp.dims["L"], (Lp // 64) * 64))
+
+
+def cpu_baseline(cfg, inp, y_gpu, seconds=12.0):
+    """The fp64 oracle as it stands, OpenMP over (batch, head) on all host cores, on a bounded
+    sample: every (batch, head) sequence of the layer over a prefix of the tokens, sized to take
+    about `seconds`.  tokens/s counts layer tokens (a layer token needs all H heads).  The same
+    sample checks the GPU: its y on those tokens against the oracle's (max relative error and
+    elementwise error, the bf16 tolerance 2e-2)."""
+    import numpy as np
     from oracle import oracle as orc
     H, b = cfg["H"], cfg["b"]
     allp = [(bi, hi) for bi in range(b) for hi in range(H)]
     cores = orc.max_threads()
-    probe = allp[:cores]
-    t1 = _oracle_rate(cfg, inp, probe)
-    per_pair = t1 / len(probe)  # seconds per pair at full parallelism
-    n = int(max(len(probe), min(len(allp), seconds / max(per_pair, 1e-9))))
-    n = max(cores, (n // cores) * cores)
-    n = min(n, len(allp))
-    sample = allp[:n]
-    t = _oracle_rate(cfg, inp, sample)
-    layer_tokens = len(sample) * cfg["L"] / H
-    return {"value": layer_tokens / t, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"{len(sample)} of {len(allp)} (batch, head) sequences x {cfg['L']} tokens of p1_layer "
-                      f"({t:.1f} s); tokens/s counts layer tokens (all {H} heads)",
-            "seconds": t}
+    Lp = _sample_len(inp, allp, seconds)
+    sub = _prefix(inp, Lp)
+    t, yr = _oracle_time(sub, allp)
+    yg = y_gpu[:, :Lp].float().cpu().numpy().astype(np.float64)
+    err = float(np.abs(yg - yr).max() / max(np.abs(yr).max(), 1e-300))
+    floor = 1e-3 * np.abs(yr).max()
+    elem = float((np.abs(yg - yr) / np.maximum(np.abs(yr), floor)).max())
+    return {"value": len(allp) * Lp / H / t, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"all {len(allp)} (batch, head) sequences of {WORKLOAD} over their first {Lp} of "
+                      f"{cfg['L']} tokens ({t:.1f} s); tokens/s counts layer tokens (all {H} heads)",
+            "seconds": t,
+            "parity": {"y_max_rel_err": err, "y_elementwise_rel_err": elem, "tolerance": 2e-2,
+                       "tokens": Lp, "sequences": len(allp),
+                       "metric": "max|gpu - oracle| / max|oracle| over the sample; elementwise: "
+                                 "|gpu - oracle| / max(|oracle|, 1e-3 max|oracle|)"}}
 
 
 def run_reference(args):
@@ -621,30 +675,37 @@ def run_reference(args):
     if rank != 0:
         return
     from oracle import oracle as orc
-    from selective_state_space_53_b200.inputs import CONFIGS, SEEDS, config_inputs
+    from selective_state_space_53_b200.inputs import CONFIGS, SEEDS, make_inputs
     cfg = dict(CONFIGS[WORKLOAD])
-    inp = config_inputs(WORKLOAD)
     H, b = cfg["H"], cfg["b"]
     cores = orc.max_threads()
     allp = [(bi, hi) for bi in range(b) for hi in range(H)]
-    # each step: one sample of `cores` whole (batch, head) sequences (about a second)
-    sample = allp[:min(len(allp), cores)]
+    # each step: every (batch, head) sequence over a prefix of the tokens, sized so that the
+    # whole run takes about three minutes; the draw has the workload's shapes and seed
+    Lmax = 4096
+    draw = dict(cfg, L=Lmax)
+    draw.pop("layers", None)
+    inp = make_inputs(seed=SEEDS[WORKLOAD], **draw)
+    per_step = 180.0 / max(1, args.steps + args.warmup)
+    Lp = _sample_len(inp, allp, per_step)
+    sub = _prefix(inp, Lp)
     for i in range(args.warmup):
-        _oracle_rate(cfg, inp, sample)
+        _oracle_time(sub, allp)
     t = 0.0
     for i in range(args.steps):
-        t += _oracle_rate(cfg, inp, sample)
-    layer_tokens_per_step = len(sample) * cfg["L"] / H
+        t += _oracle_time(sub, allp)[0]
+    layer_tokens_per_step = len(allp) * Lp / H
     value = layer_tokens_per_step * args.steps / t
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded; shapes of the page-1 layer)",
-        "config": {"workload": "p1_layer: m3_scan_fwd over b4 x L2048 (H24 P64 N64 R2, chunk 32) + 1 m3_decode_step",
+        "data": "synthetic (seeded; shapes of the 1.5B-scale layer)",
+        "config": {"workload": f"{WORKLOAD}: m3_scan_fwd over b{cfg['b']} x L{cfg['L']} (H{cfg['H']} P{cfg['P']} "
+                               f"N{cfg['N']} R{cfg['R']}, chunk 32) + 1 m3_decode_step",
                    "global_batch": b, "seq_len": cfg["L"], "parallelism": "host cores"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"each step: {len(sample)} of {len(allp)} (batch, head) sequences x {cfg['L']} "
+                         "sample": f"each step: all {len(allp)} (batch, head) sequences over their first {Lp} "
                                    f"tokens; tokens/s counts layer tokens (all {H} heads)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,

@@ -154,6 +154,50 @@ m3_status m3_scan_fwd_noalloc(const m3_dims* dims, const void* x, const float* d
                               const float* W_o, const float* D, m3_state* state, void* y,
                               void* stream);
 
+/* ---- ranges of a sequence (sequence sharding) ---------------------------- */
+
+/* A sequence split into consecutive token ranges (for instance one per device) runs as: every
+ * range is summarised (m3_scan_summary), the summaries are exchanged, the state entering range k
+ * is the sequence's initial state folded through the summaries of ranges 0..k-1
+ * (m3_state_fold), and range k then runs m3_scan_fwd from that state.  The results equal one
+ * m3_scan_fwd over the whole sequence.  The algebra: the scan combines associatively over
+ * ranges (IBM page "Mamba モデルとは", hardware-aware scan); for the recurrence above a range
+ * of tokens t0..t1 maps the state entering it to
+ *   h_{t1} = e^{logdec} Rot(angle) (h_{t0-1} + bp_first u_{t0-1}) + Z,
+ * logdec = sum_t dt_t A_t, angle_k = sum_t phi_{t,k}, bp_first = (1 - lam_{t0}) dt_{t0}, Z the
+ * range's end state from a fresh start, u_{t0-1} = sum_r (carry_B_r + bias_B_r)(W_x_r * carry_x)^T
+ * the previous-token term built from the carry of the token before the range (Mamba-3 paper
+ * note, sections その1-その3). */
+
+/* Scratch bytes m3_scan_summary needs (dims->L = the range's length, >= 1).  Ranges are
+ * summarised by the chunked tensor-core state pass: bf16 with d_state and headdim in {64, 128}
+ * and R in {1, 2, 4, 8} (R = 1 with d_state = headdim = 128 excepted); other dims give
+ * M3_ERR_UNSUPPORTED. */
+m3_status m3_scan_summary_workspace_size(const m3_dims* dims, size_t* out_bytes);
+
+/* Summary of one range of every sequence of the batch (x, dt, A, lam, B, theta of the range in
+ * the layouts above; bias_B, W_x may be NULL).  Outputs, caller-owned device memory:
+ *   Z (b, H, N, P) fp32        the range's end state from a fresh start
+ *   logdec (b, H) fp32         sum over the range of dt A
+ *   angle (b, H, N/2) fp64     sum over the range of the rotation angles, reduced to [-pi, pi]
+ *   bp_first (b, H) fp32       (1 - lam) dt of the range's first token
+ *   carry_B (b, H, R, N) fp32, carry_x (b, H, P) fp32   the range's last token's raw B and x
+ * workspace: at least m3_scan_summary_workspace_size bytes.  Asynchronous on `stream`. */
+m3_status m3_scan_summary(const m3_dims* dims, const void* x, const float* dt, const float* A,
+                          const float* lam, const void* B, const float* theta, const float* bias_B,
+                          const float* W_x, float* Z, float* logdec, double* angle, float* bp_first,
+                          float* carry_B, float* carry_x, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/* Fold `nranges` range summaries (each array above with a leading nranges axis, ranges in
+ * sequence order) onto `state`: in, the state entering range 0; out, the state entering range
+ * nranges (h and the carry).  nranges = 0 leaves the state unchanged.  bias_B, W_x as for
+ * m3_scan_fwd.  Asynchronous on `stream`. */
+m3_status m3_state_fold(const m3_dims* dims, int32_t nranges, const float* Z, const float* logdec,
+                        const double* angle, const float* bp_first, const float* carry_B,
+                        const float* carry_x, const float* bias_B, const float* W_x,
+                        m3_state* state, void* stream);
+
 /* ---- decode (one token) ------------------------------------------------ */
 
 /* Advance every sequence by one token.  Token inputs have L = 1 in the layouts

@@ -290,6 +290,68 @@ m3_status m3_decode_step(const m3_dims* dims, const void* x_t, const float* dt_t
   return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
 }
 
+m3_status m3_scan_summary_workspace_size(const m3_dims* dims, size_t* out_bytes) {
+  m3_status st = check_dims(dims);
+  if (st != M3_OK) return st;
+  if (!out_bytes) return M3_ERR_NULL;
+  if (dims->L < 1) return M3_ERR_DIMS;
+  m3::Params p = make_params(dims, dims->L, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                             nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+  if (!m3::tc_scan_supported(p)) return M3_ERR_UNSUPPORTED;
+  *out_bytes = m3::scan_summary_workspace_bytes(p);
+  return M3_OK;
+}
+
+m3_status m3_scan_summary(const m3_dims* dims, const void* x, const float* dt, const float* A, const float* lam,
+                          const void* B, const float* theta, const float* bias_B, const float* W_x, float* Z,
+                          float* logdec, double* angle, float* bp_first, float* carry_B, float* carry_x,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  size_t need = 0;
+  m3_status st = m3_scan_summary_workspace_size(dims, &need);
+  if (st != M3_OK) return st;
+  const void* req[] = {x, dt, A, lam, B, theta, Z, logdec, angle, bp_first, carry_B, carry_x, workspace};
+  for (const void* q : req)
+    if (!q) return M3_ERR_NULL;
+  const void* all[] = {x, dt, A, lam, B, theta, bias_B, W_x, Z, logdec, angle, bp_first, carry_B, carry_x, workspace};
+  for (const void* q : all)
+    if (q && !aligned16(q)) return M3_ERR_ALIGN;
+  if (workspace_bytes < need) return M3_ERR_WORKSPACE;
+  if (dims->b * dims->H == 0) return M3_OK;
+  // the state pass reads neither C nor a state: B stands in for C's tensor map
+  m3::Params p = make_params(dims, dims->L, x, dt, A, lam, B, B, theta, bias_B, nullptr, W_x, nullptr, nullptr,
+                             nullptr, nullptr);
+  p.status = status_word();
+  if (!p.status) return M3_ERR_CUDA;
+  const cudaError_t e = m3::launch_range_summary(p, workspace, workspace_bytes, Z, logdec, angle, bp_first, carry_B,
+                                                 carry_x, (cudaStream_t)stream);
+  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
+m3_status m3_state_fold(const m3_dims* dims, int32_t nranges, const float* Z, const float* logdec,
+                        const double* angle, const float* bp_first, const float* carry_B, const float* carry_x,
+                        const float* bias_B, const float* W_x, m3_state* state, void* stream) {
+  m3_status st = check_dims(dims);
+  if (st != M3_OK) return st;
+  if (nranges < 0) return M3_ERR_DIMS;
+  if (!state) return M3_ERR_NULL;
+  if (!same_state_dims(dims, &state->dims)) return M3_ERR_STATE;
+  if (nranges > 0) {
+    const void* req[] = {Z, logdec, angle, bp_first, carry_B, carry_x};
+    for (const void* q : req)
+      if (!q) return M3_ERR_NULL;
+  }
+  const void* all[] = {Z, logdec, angle, bp_first, carry_B, carry_x, bias_B, W_x, state->h, state->carry_B,
+                       state->carry_x};
+  for (const void* q : all)
+    if (q && !aligned16(q)) return M3_ERR_ALIGN;
+  if (dims->b * dims->H == 0 || nranges == 0) return M3_OK;
+  m3::Params p = make_params(dims, 1, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, bias_B, nullptr,
+                             W_x, nullptr, nullptr, state, nullptr);
+  const cudaError_t e = m3::launch_state_fold(p, nranges, Z, logdec, angle, bp_first, carry_B, carry_x,
+                                              (cudaStream_t)stream);
+  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
 m3_status m3_selftest_wait(uint64_t limit_ns, void* stream) {
   if (limit_ns > 10000000000ull) return M3_ERR_DIMS;
   int* st = status_word();

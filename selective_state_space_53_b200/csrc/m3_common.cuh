@@ -125,6 +125,13 @@ cudaError_t launch_decode_tc(const Params& p, cudaStream_t stream);
 bool tc_scan_supported(const Params& p);
 size_t tc_scan_workspace_bytes(const Params& p);  // scratch the chunked scan needs (0: none)
 cudaError_t launch_scan_tc(const Params& p, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+struct SegInfo;
+size_t scan_summary_workspace_bytes(const Params& p);  // scratch of the range summary's state pass
+cudaError_t launch_scan_summary_pass(const Params& p, void* ws, size_t ws_bytes, SegInfo* sg, cudaStream_t stream);
+cudaError_t launch_range_summary(const Params& p, void* ws, size_t ws_bytes, float* Z, float* logdec, double* angle,
+                                 float* bp_first, float* carry_B, float* carry_x, cudaStream_t stream);
+cudaError_t launch_state_fold(const Params& p, int nranges, const float* Z, const float* logdec, const double* angle,
+                              const float* bp_first, const float* carry_B, const float* carry_x, cudaStream_t stream);
 cudaError_t launch_selftest_wait(int* status, unsigned long long limit_ns, cudaStream_t stream);
 
 }  // namespace m3

@@ -48,62 +48,24 @@
 #include <cudaTypedefs.h>
 
 #include "m3_common.cuh"
+#include "m3_ptx.cuh"
+#include "m3_scan_plan.cuh"
 
 namespace m3 {
 namespace {
 
 constexpr int kThreads = 256;
 constexpr int kRows = 128;
-constexpr unsigned kFull = 0xffffffffu;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s bound on any mbarrier wait
 constexpr int MODE_FULL = 0, MODE_STATE = 1;
+// Largest log-decay range of a tile that takes the pivot split.  The split scales X' rows by
+// b_s = e^{m - Lc_s} <= e^{range / 2} and applies a_t only after S' X' has been summed in fp32,
+// so the sum can reach Q R max|S| max|w x| e^{range / 2}; at 64 that is below 1e21 max|w x|,
+// far from the fp32 limit (3.4e38) for any sane input.  Wider tiles take the exact path.
+constexpr float kFastRange = 64.0f;
 
-// ------------------------------------------------------------------ PTX helpers
+// ------------------------------------------------------------------ waits
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
-               "r"(ncols));
-}
-__device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(done)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return done != 0;
-}
 // Bounded wait: false after kWaitNs without the phase completing.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -113,148 +75,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
   return true;
 }
-// TMA tile loads into this CTA alone, completion counted in bytes on `bar`.
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
-      "[%5];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
-      "%5}], [%6];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
-      : "memory");
-}
-// D[tmem] (+)= A[smem or tmem] * B[smem], and the commit of the issued MMAs to an mbarrier:
-// warp-collective -- every lane of a converged warp executes them with warp-uniform operands,
-// and the lane that elect.sync picks issues.
-__device__ __forceinline__ void mma_ss_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n .reg .pred p, e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
-      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc));
-}
-__device__ __forceinline__ void mma_ts_w(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n .reg .pred p, e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
-      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
-      "r"(a), "l"(b), "r"(idesc), "r"(acc));
-}
-__device__ __forceinline__ void mma_commit_w(uint64_t* bar) {
-  asm volatile(
-      "{\n .reg .pred e;\n .reg .b32 r;\n elect.sync r|e, 0xffffffff;\n"
-      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}\n" ::"r"(smem_u32(bar))
-      : "memory");
-}
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
-        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]),
-        "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),
-        "=r"(v[30]), "=r"(v[31])
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
-      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
-      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31]));
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::
-          "r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]));
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 descriptor version 1).
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-// Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, dense.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
-         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-__device__ __forceinline__ void unpack8(const uint4& w, float (&f)[8]) {
-  f[0] = bf_lo(w.x); f[1] = bf_hi(w.x); f[2] = bf_lo(w.y); f[3] = bf_hi(w.y);
-  f[4] = bf_lo(w.z); f[5] = bf_hi(w.z); f[6] = bf_lo(w.w); f[7] = bf_hi(w.w);
-}
-__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
-  return make_uint4(pack_bf16(f[0], f[1]), pack_bf16(f[2], f[3]), pack_bf16(f[4], f[5]), pack_bf16(f[6], f[7]));
-}
-__device__ __forceinline__ void sts128(uint32_t addr, const uint4& v) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-               : "memory");
-}
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
-}
-// Byte offset of 16-byte chunk `ch` of row `row` in a 128B-swizzled tile with 128-byte rows
-// per 64-element block, blocks `block_bytes` apart (the TMA SWIZZLE_128B / UMMA SW128 layout).
-__device__ __forceinline__ uint32_t sw128(int row, int ch, uint32_t block_bytes) {
-  return (uint32_t)(ch >> 3) * block_bytes + (uint32_t)row * 128u + ((uint32_t)((ch & 7) ^ (row & 7)) << 4);
-}
-// Signed-integer key of a float with the same order (negative floats: magnitude bits reversed),
-// and its inverse; lets redux.sync take a warp's float min / max.
-__device__ __forceinline__ int float_key(float f) {
-  const int i = __float_as_int(f);
-  return i >= 0 ? i : (i ^ 0x7fffffff);
-}
-__device__ __forceinline__ float key_float(int k) { return __int_as_float(k >= 0 ? k : (k ^ 0x7fffffff)); }
-// 2^x by the hardware approximation (ex2.approx, relative error about 2^-22).
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-// sin and cos of an angle of moderate size: Cody-Waite reduction to [-pi, pi] with a two-term
-// split of 2 pi (Cody & Waite, "Software Manual for the Elementary Functions", 1980), then the
-// hardware approximations, which are accurate on that interval.
-__device__ __forceinline__ void sincos_reduced(float x, float* s, float* c) {
-  const float n = rintf(x * 0.15915494309189535f);
-  float r = fmaf(-n, 6.28318548202514648f, x);
-  r = fmaf(-n, -1.7484555314695172e-7f, r);
-  *s = __sinf(r);
-  *c = __cosf(r);
-}
-
 // ------------------------------------------------------------------ configuration
 
-struct SegInfo {
-  int nseg;        // full-pass segments per sequence
-  int seg_tiles;   // tiles per full-pass segment
-  int nsub;        // state-pass sub-segments per sequence: they tile segments 0..nseg-2
-  int sub_tiles;   // tiles per sub-segment (divides seg_tiles)
-  float* ws_init;  // (b*H, N, P): rotated-frame state entering segment 0 (nseg > 1)
-  float* ws_h;     // (b*H, nsub, N, P): end state of each sub-segment from a zero start
-  float* ws_l;     // (b*H, nsub): total log decay of each sub-segment
-  double* ws_phi;  // (b*H, nsub, N/2): total angle of each sub-segment, reduced mod 2 pi
-};
 
 template <int R, int N, int P, int MODE>
 struct Cfg {
@@ -306,8 +128,8 @@ struct Cfg {
 // diagonal, S * gamma_s / w_s on it, 0 above.  The inter-chunk term e^{Lc_t} Ct h+ equals
 // a_t Ct (e^m h+): the bf16 copy of the state is written pre-scaled by e^m, so that product
 // accumulates into the same Y as S' X'.  The state update becomes H = X'^T Bt times the
-// uniform factor e^{Le - m}.  When the range of Lc within a tile exceeds 160 the split could
-// overflow fp32; such tiles take the exact path (m = 0, a_t = 1, b_s = 1, e^{Lc_t - Lc_s} per
+// uniform factor e^{Le - m}.  When the range of Lc within a tile exceeds kFastRange the split
+// could overflow fp32; such tiles take the exact path (m = 0, a_t = 1, b_s = 1, e^{Lc_t - Lc_s} per
 // element, Ct rows scaled by e^{Lc_t} and Bt rows by e^{Le - Lc_t} in place).
 // record A[t] = {Lc_t * log2 e, gamma_t / w_t, a_t, b_t w_t};  record B[t] = {e^{Lc_t},
 // e^{Le - Lc_t}, 0, 0};  scalars {e^{Le}, Le, e^{Le - m} or 1, fast, e^m or 1, 0, 0, 0}
@@ -455,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
       // warp min / max in one redux each, on integer keys that order like the floats
       lmin = key_float(__reduce_min_sync(kFull, float_key(lmin)));
       lmax = key_float(__reduce_max_sync(kFull, float_key(lmax)));
-      const bool fast = (lmax - lmin) <= 160.0f;
+      const bool fast = (lmax - lmin) <= kFastRange;
       const float m = fast ? 0.5f * (lmax + lmin) : 0.0f;
       const float bp_after = rawA(slot, 3)[0];
       float4* ra = recA(slot);
@@ -603,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
 
   // ---- incoming rotated-frame state h+ of this segment
   //   nseg == 1 (full pass): h_{-1} + beta'_0 u_{-1} from the state / carry;
-  //   state pass, segment 0: same, written to ws_init; other state-pass segments: zero;
+  //   state pass: zero (sub-segment 0 also writes the state's h+ to ws_init);
   //   full pass, segment k > 0: ws_init folded through the summaries of segments 0..k-1.
   // In the full pass every warp takes part (warp w: the TMEM lanes of quarter w & 3, half the
   // state columns), and the rotations of the folded segments come from a table that all
@@ -624,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
   const int c_lo = FULL ? (warp >> 2) * (N / 64) : 0;
   const int c_hi = FULL ? c_lo + N / 64 : N / 32;
   if ((FULL || state_warp) && j0 < j1) {
-    const bool from_state = (sg.nseg == 1) || (!FULL && seg == 0);
+    const bool from_state = (sg.nseg == 1) || (!FULL && seg == 0 && sg.write_init);
     const float hscale = scal(0)[4];  // e^m of the first tile: the bf16 copy is pre-scaled
     float xprev[R];
     float bp0 = 0.0f;
@@ -654,6 +476,12 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
           float* wi = sg.ws_init + (int64_t)bh * N * P;
 #pragma unroll
           for (int e = 0; e < 32; ++e) wi[(int64_t)(32 * c + e) * P + prow] = v[e];
+        }
+        if constexpr (!FULL) {
+          // the state pass summarises every sub-segment from a zero start; the incoming state
+          // reaches later segments through the fold of ws_init in the full pass
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0.0f;
         }
       } else if (FULL) {
         const float* wi = sg.ws_init + (int64_t)bh * N * P;
@@ -1312,6 +1140,65 @@ size_t ws_bytes_for(const Params& p, SegPlan* out) {
   return bytes;
 }
 
+}  // namespace
+bool ws_scan_supported(const Params& p);
+cudaError_t launch_scan_ws(const CUtensorMap& tmB, const CUtensorMap& tmC, const Params& p, const SegInfo& sg,
+                           cudaStream_t stream);
+cudaError_t launch_scan_ws_state(const CUtensorMap& tmB, const CUtensorMap& tmC, const Params& p,
+                                 const SegInfo& sg, cudaStream_t stream);
+namespace {
+
+// Summary of a whole range (sequence sharding): the state pass over every tile of the range,
+// cut into sub-segments that fill the SMs, each summarised from a zero start.
+template <int R, int N, int P>
+SegInfo summary_plan(const Params& p) {
+  constexpr int Q = kRows / R;
+  int dev = 0, nsm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t nseq = p.b * p.H;
+  const int64_t ntiles = (p.L + Q - 1) / Q;
+  const int64_t slots = (int64_t)nsm * ctas_per_sm<R, N, P>();
+  int64_t m = slots / (nseq > 0 ? nseq : 1);
+  if (m > ntiles / 2) m = ntiles / 2;  // at least two tiles per sub-segment
+  if (m > 256) m = 256;
+  if (m < 1) m = 1;
+  SegInfo sg{};
+  sg.sub_tiles = (int)((ntiles + m - 1) / m);
+  sg.nsub = (int)((ntiles + sg.sub_tiles - 1) / sg.sub_tiles);
+  sg.nseg = 2;  // the state pass reads only the sub-segment fields
+  sg.seg_tiles = sg.nsub * sg.sub_tiles;
+  sg.write_init = 0;
+  return sg;
+}
+
+template <int R, int N, int P>
+size_t summary_ws_for(const Params& p, SegInfo* sg) {
+  *sg = summary_plan<R, N, P>(p);
+  const size_t nseq = (size_t)(p.b * p.H), ns = (size_t)sg->nsub;
+  size_t bytes = 4 * nseq * ns * (size_t)N * P;
+  bytes = (bytes + 4 * nseq * ns + 255) & ~(size_t)255;
+  return bytes + 8 * nseq * ns * (N / 2);
+}
+
+template <int R, int N, int P>
+cudaError_t launch_summary_cfg(const Params& p, void* ws, size_t ws_bytes, SegInfo* sg_out, cudaStream_t stream) {
+  constexpr int Q = kRows / R;
+  SegInfo sg;
+  const size_t need = summary_ws_for<R, N, P>(p, &sg);
+  if (ws == nullptr || ws_bytes < need) return cudaErrorInvalidValue;
+  const size_t nseq = (size_t)(p.b * p.H), ns = (size_t)sg.nsub;
+  char* w = static_cast<char*>(ws);
+  sg.ws_init = nullptr;
+  sg.ws_h = reinterpret_cast<float*>(w);
+  sg.ws_l = sg.ws_h + nseq * ns * N * P;
+  sg.ws_phi = reinterpret_cast<double*>(w + ((4 * nseq * ns * (size_t)N * P + 4 * nseq * ns + 255) & ~(size_t)255));
+  *sg_out = sg;
+  Maps m;
+  if (!make_maps(p, Q, &m)) return cudaErrorInvalidValue;
+  if (ws_scan_supported(p)) return launch_scan_ws_state(m.B, m.C, p, sg, stream);
+  return launch_mode<R, N, P, MODE_STATE>(m, p, sg, (unsigned)(nseq * ns), stream);
+}
+
 template <int R, int N, int P>
 cudaError_t launch_cfg(const Params& p, void* ws, size_t ws_bytes, cudaStream_t stream) {
   constexpr int Q = kRows / R;
@@ -1327,6 +1214,7 @@ cudaError_t launch_cfg(const Params& p, void* ws, size_t ws_bytes, cudaStream_t 
   sg.sub_tiles = plan.sub_tiles;
   sg.ws_init = sg.ws_h = sg.ws_l = nullptr;
   sg.ws_phi = nullptr;
+  sg.write_init = 1;
   const int64_t nseq = p.b * p.H;
   const int nseg = plan.nseg;
   if (nseg > 1) {
@@ -1338,6 +1226,10 @@ cudaError_t launch_cfg(const Params& p, void* ws, size_t ws_bytes, cudaStream_t 
     sg.ws_l = sg.ws_h + (size_t)nseq * s1 * np;
     size_t off = (4 * ((size_t)nseq * np + (size_t)nseq * s1 * np + (size_t)nseq * s1) + 255) & ~(size_t)255;
     sg.ws_phi = reinterpret_cast<double*>(w + off);
+  }
+  // headdim 128 with a rank the warp-specialised kernel covers: that kernel, same plan
+  if (ws_scan_supported(p)) return launch_scan_ws(m.B, m.C, p, sg, stream);
+  if (nseg > 1) {
     cudaError_t e = launch_mode<R, N, P, MODE_STATE>(m, p, sg, (unsigned)(nseq * plan.nsub), stream);
     if (e != cudaSuccess) return e;
   }
@@ -1373,7 +1265,42 @@ bool fits_r(const Params& p) {
   return fits<R, 128, 128>();
 }
 
+template <int R>
+size_t summary_ws_r(const Params& p) {
+  SegInfo sg;
+  if (p.N == 64 && p.P == 64) return summary_ws_for<R, 64, 64>(p, &sg);
+  if (p.N == 64 && p.P == 128) return summary_ws_for<R, 64, 128>(p, &sg);
+  if (p.N == 128 && p.P == 64) return summary_ws_for<R, 128, 64>(p, &sg);
+  return summary_ws_for<R, 128, 128>(p, &sg);
+}
+
+template <int R>
+cudaError_t launch_summary_r(const Params& p, void* ws, size_t wsb, SegInfo* sg, cudaStream_t s) {
+  if (p.N == 64 && p.P == 64) return launch_summary_cfg<R, 64, 64>(p, ws, wsb, sg, s);
+  if (p.N == 64 && p.P == 128) return launch_summary_cfg<R, 64, 128>(p, ws, wsb, sg, s);
+  if (p.N == 128 && p.P == 64) return launch_summary_cfg<R, 128, 64>(p, ws, wsb, sg, s);
+  return launch_summary_cfg<R, 128, 128>(p, ws, wsb, sg, s);
+}
+
 }  // namespace
+
+size_t scan_summary_workspace_bytes(const Params& p) {
+  switch (p.R) {
+    case 1: return summary_ws_r<1>(p);
+    case 2: return summary_ws_r<2>(p);
+    case 4: return summary_ws_r<4>(p);
+    default: return summary_ws_r<8>(p);
+  }
+}
+
+cudaError_t launch_scan_summary_pass(const Params& p, void* ws, size_t ws_bytes, SegInfo* sg, cudaStream_t stream) {
+  switch (p.R) {
+    case 1: return launch_summary_r<1>(p, ws, ws_bytes, sg, stream);
+    case 2: return launch_summary_r<2>(p, ws, ws_bytes, sg, stream);
+    case 4: return launch_summary_r<4>(p, ws, ws_bytes, sg, stream);
+    default: return launch_summary_r<8>(p, ws, ws_bytes, sg, stream);
+  }
+}
 
 bool tc_scan_supported(const Params& p) {
   if (p.dtype != M3_BF16) return false;

@@ -1,0 +1,1010 @@
+// m3_scan_ws.cu -- warp-specialised chunked Mamba-3 prefill on the sm_100a tensor cores, for
+// headdim P = 128 (the 1.5B-scale layer: d_state 128, MIMO rank 4).
+//
+// The chunk algebra is that of the other tensor-core scan (m3_scan_tc.cu): tiles of
+// Q = 128 / R tokens, rows i = t R + r (token t, MIMO branch r), the rotation absorbed into B
+// and C in a rotated frame (Mamba-3 paper note, docsaid.org, section その2, statement 2), the
+// trapezoid weights gamma_s = lam_s dt_s and beta'_{s+1} = (1 - lam_{s+1}) dt_{s+1} (section
+// その1) and the per-branch scales of the MIMO inputs and readouts (section その3).  The
+// chunked form is exact (IBM Mamba page, SSD section), so the tile length does not change the
+// result.  What differs is the layout of the products and the schedule.
+//
+// Transposed products.  With Lc_t the tile-local cumulative log decay and m a pivot in the
+// middle of its range, a_t = e^{Lc_t - m}, b_s = e^{m - Lc_s}, w_s = gamma_s + beta'_{s+1}:
+//   Ct'_i = a_t Rot(-Phi_t)(C_{t,r} + bias_C),   Bt'_i = b_t w_t Rot(-Phi_t)(B_{t,r} + bias_B)
+//   S   = Ct' Bt'^T                      (M = 128 rows i, N = 128 columns j, K = d_state)
+//   S'  = S below the diagonal, S gamma/w on it, 0 above (masking only: the decay
+//         e^{Lc_t - Lc_s} w_s is already a_t b_s w_s)
+//   Y^T = hb^T Ct'^T + X'^T S'^T         (M = P rows p, N = 128 columns i)
+//   ST <- ST + X'^T Bt'                  (M = P, N = d_state, K = 128), ST pre-scaled by e^m
+// with X'_i = W_x[r] * x_t and hb = bf16(e^m h+) the state entering the tile.  The output
+// then has the head dimension p on the tensor-memory lanes, so y_t[p] = sum_r W_o[r,p] Y^T[p,
+// tR + r] (+ D x_t[p]) is a sum inside one thread; the state update needs no exponentials on
+// the operands either (the uniform factor e^{Le - m} is applied once per tile to the state).
+// Tiles whose log-decay range exceeds 64 take an exact form instead: no pivot, the mask applies
+// e^{Lc_t - Lc_s} per element, and after S has read them the rows of Ct' and Bt' are rescaled
+// in place by e^{Lc_t} and e^{Le - Lc_t} for the inter-chunk and state products.  With the
+// range at most 64 every factor a_t, b_s, e^{m}, e^{Le - m} lies within e^{+-32}.
+//
+// Warp roles (23 warps; every wait is an mbarrier wait bounded by %globaltimer):
+//   0      producer: TMA loads of the B and C tiles into two shared-memory stages
+//   1      MMA issue (one elected lane): S, H, Y_inter, Y_intra; tensor-memory allocation
+//   2      coefficients: decay cumsum, pivot, per-token scales, state scale factors
+//   3-10   rotation: cumulative angles and their sin/cos table; Bt', Ct' rotated in place
+//   11-14  mask: S from tensor memory -> S' (bf16, shared memory)
+//   15-18  epilogue: Y^T from tensor memory -> y
+//   19-22  state and inputs: the state rescale and its bf16 copy hb; X'^T into tensor memory
+// The tile pipeline per tile j (MMA order): H(j), Y_inter(j), Y_intra(j), S(j+1).  Each SIMT
+// task has two MMAs' time between the commit that releases it and the MMA that needs it:
+// state rescale SP(j+1) after Y_inter(j), before H(j+1); epilogue E(j) after Y_intra(j), before
+// Y_inter(j+1); mask M(j+1) after S(j+1), before Y_intra(j+1); X'^T is double-buffered.
+//
+// Sequence splitting follows the shared segment plan (m3_scan_plan.cuh): a state pass
+// (MODE 1: rotation of B only, X', H and the state rescale) summarises segments 0..nseg-2 from a
+// zero start; the full pass starts each segment from the folded summaries.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "m3_common.cuh"
+#include "m3_ptx.cuh"
+#include "m3_scan_plan.cuh"
+
+namespace m3 {
+namespace {
+
+constexpr int WP = 128;  // head dim of this kernel
+constexpr int W_PROD = 0, W_MMA = 1, W_COEF = 2, W_ROT = 3, N_ROT = 8, W_MASK = 11, W_EPI = 15, W_SPX = 19;
+constexpr int WS_WARPS = 23;
+constexpr int WS_THREADS = WS_WARPS * 32;
+constexpr int WS_CS = 4;                          // coefficient record slots
+constexpr float WS_FAST_RANGE = 64.0f;            // largest log-decay range of a pivot-split tile
+constexpr unsigned long long WS_WAIT_NS = 2000000000ull;  // 2 s bound on any wait
+constexpr int WS_FULL = 0, WS_STATE = 1;
+constexpr uint32_t BAR_ROT = 1;                   // named barrier of the rotation warps
+
+// barrier indices
+enum {
+  B_BCF = 0,    // [2] B/C tile of a stage landed (TMA bytes)
+  B_BCE = 2,    // [2] stage free (MMA commit)
+  B_CF = 4,     // [CS] coefficient records written
+  B_CE = 8,     // [CS] coefficient records consumed
+  B_ROT = 12,   // [2] Bt', Ct' of a stage rotated
+  B_RESC = 14,  // exact tile: Bt', Ct' rescaled after S
+  B_SF = 15,    // S in tensor memory (MMA commit)
+  B_SPF = 16,   // S' in shared memory (mask warps)
+  B_HF = 17,    // hb and the rescaled state ready (state warps)
+  B_SPGO = 18,  // H and Y_inter done: state and hb may be rewritten (MMA commit)
+  B_XPF = 19,   // [2] X'^T buffer written (state warps)
+  B_XBF = 21,   // [2] X'^T buffer free (MMA commit)
+  B_YF = 23,    // Y^T complete (MMA commit)
+  B_YE = 24,    // Y^T read (epilogue warps)
+  B_DRAIN = 25, // all MMAs complete (end of kernel)
+  B_FIN = 26,   // final angles published (rotation warps)
+  NBAR = 27
+};
+
+template <int R, int N>
+struct WsCfg {
+  static constexpr int Q = 128 / R;
+  static constexpr int K2 = N / 2;
+  static constexpr int NKC = N / 8;                    // 16-byte chunks of a row
+  static constexpr int KCW = NKC / N_ROT;              // chunks per rotation warp
+  static constexpr int TILE_N = 128 * N * 2;           // a B or C tile, bytes
+  static constexpr int BLK = 128 * 128;                // one 64-column block of a 128-row SW128 tile
+  static constexpr int STAGE = 2 * TILE_N;             // B then C
+  static constexpr int OFF_STAGE = 0;
+  static constexpr int OFF_SP = OFF_STAGE + 2 * STAGE;           // S', 128 x 128 bf16
+  static constexpr int OFF_HB = OFF_SP + 128 * 128 * 2;          // hb, 128 (p) x N bf16
+  static constexpr int TAB_ROW = K2 * 8 + 16;                    // (cos, sin) of one token, padded
+  static constexpr int OFF_TAB = OFF_HB + WP * N * 2;
+  static constexpr int BIAS_ROW = N * 4 + 16;
+  static constexpr int OFF_BIAS = OFF_TAB + Q * TAB_ROW;         // bias_B rows r, then bias_C rows r
+  static constexpr int SEGS = 256 / K2;                          // angle prefix segments
+  static constexpr int SEGLEN = Q / SEGS;
+  static constexpr int OFF_SEGSUM = OFF_BIAS + 2 * R * BIAS_ROW;  // float [SEGS][K2]
+  static constexpr int OFF_BASE = OFF_SEGSUM + SEGS * K2 * 4;    // double [K2]
+  static constexpr int REC_SLOT = Q * 16 + Q * 4 + 64;           // float4 rec[Q], float mult[Q], float scal[16]
+  static constexpr int OFF_REC = OFF_BASE + K2 * 8;
+  static constexpr int OFF_BAR = OFF_REC + WS_CS * REC_SLOT;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int SMEM = BYTES + 1024;
+  static constexpr uint32_t TM_S = 0, TM_Y = 128, TM_ST = 256, TM_XP = 256 + N;  // X'^T: two 64-column buffers
+  static constexpr uint32_t TM_COLS = 512;
+  static constexpr uint32_t ID_S = idesc_bf16(128, 128, false, false);
+  static constexpr uint32_t ID_Y = idesc_bf16(WP, 128, false, false);
+  static constexpr uint32_t ID_H = idesc_bf16(WP, N, false, true);
+  static_assert(Q % SEGS == 0 && SEGLEN >= 1, "angle segments");
+  static_assert(NKC % N_ROT == 0, "rotation chunks");
+  static_assert(TM_XP + 128 <= TM_COLS, "tensor memory");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+__device__ __forceinline__ bool ws_try(uint64_t* bar, uint32_t parity) { return mbar_try_wait(bar, parity); }
+
+// Wait for the phase of `parity` to complete; false (and the abort flag set) after WS_WAIT_NS,
+// or false at once when another role has already aborted.
+__device__ __forceinline__ bool ws_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (ws_try(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (!ws_try(bar, parity)) {
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > WS_WAIT_NS) {
+      *abort_flag = 1;
+      return false;
+    }
+  }
+  return true;
+}
+// Wait bounded by time only (used to drain copies and MMAs in flight before the CTA exits).
+__device__ __forceinline__ bool ws_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!ws_try(bar, parity)) {
+    if (globaltimer() - t0 > WS_WAIT_NS) return false;
+  }
+  return true;
+}
+// Phase bits of a set of barriers in one register: bit k is the parity the next wait on
+// barrier k expects.
+struct Phases {
+  uint32_t bits = 0;
+  __device__ __forceinline__ uint32_t operator[](int k) const { return (bits >> k) & 1u; }
+  __device__ __forceinline__ void flip(int k) { bits ^= 1u << k; }
+};
+
+// Named barrier that also ORs a predicate over the participating threads: every thread gets
+// the same answer, so a group decides together whether to stop.
+__device__ __forceinline__ bool bar_any(uint32_t id, uint32_t nthreads, bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(out)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return out != 0;
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Rotate the 8 values of one 16-byte chunk (4 pairs) by the pairs' (cos, sin), after adding the
+// bias, and scale: out = sc * Rot(-Phi)(v + bias).
+__device__ __forceinline__ uint4 rotate_chunk(uint4 raw, const float4& b0, const float4& b1, const float4& cs01,
+                                              const float4& cs23, float sc) {
+  float f[8];
+  unpack8(raw, f);
+  f[0] += b0.x; f[1] += b0.y; f[2] += b0.z; f[3] += b0.w;
+  f[4] += b1.x; f[5] += b1.y; f[6] += b1.z; f[7] += b1.w;
+  const float c[4] = {cs01.x * sc, cs01.z * sc, cs23.x * sc, cs23.z * sc};
+  const float s[4] = {cs01.y * sc, cs01.w * sc, cs23.y * sc, cs23.w * sc};
+  float o[8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    o[2 * q] = fmaf(c[q], f[2 * q], s[q] * f[2 * q + 1]);
+    o[2 * q + 1] = fmaf(c[q], f[2 * q + 1], -s[q] * f[2 * q]);
+  }
+  return pack8(o);
+}
+__device__ __forceinline__ uint4 scale_chunk(uint4 raw, float sc) {
+  float f[8];
+  unpack8(raw, f);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) f[e] *= sc;
+  return pack8(f);
+}
+
+// Row p of the bf16 state copy hb (K-major, 128-byte swizzle): the 32 values of column chunk c,
+// scaled by fh.
+__device__ __forceinline__ void hb_store_row(uint32_t sHB, int pc, int c, const float (&v)[32], float fh) {
+#pragma unroll
+  for (int qq = 0; qq < 4; ++qq) {
+    const int ch = 4 * c + qq;
+    float f8[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f8[e] = fh * v[8 * qq + e];
+    const uint32_t off = (uint32_t)(ch >> 3) * (128 * 128) + (uint32_t)pc * 128u + ((uint32_t)((ch & 7) ^ (pc & 7)) << 4);
+    sts128(sHB + off, pack8(f8));
+  }
+}
+
+template <int R, int N, int MODE>
+__global__ void __maxnreg__(88)
+    scan_ws_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC, const Params p,
+                   const SegInfo sg) {
+  using C = WsCfg<R, N>;
+  constexpr bool FULL = (MODE == WS_FULL);
+  constexpr int Q = C::Q, K2 = C::K2, BLK = C::BLK;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int H = p.H, G = p.G;
+  const int64_t L = p.L;
+  const int nseg_grid = FULL ? sg.nseg : sg.nsub;
+  const int bh = blockIdx.x / nseg_grid;
+  const int seg = blockIdx.x % nseg_grid;
+  const int bi = bh / H, hi = bh % H;
+  const int g = hi / (H / G);
+  const int64_t ntiles_seq = (L + Q - 1) / Q;
+  const int seg_len = FULL ? sg.seg_tiles : sg.sub_tiles;
+  const int64_t j0 = (int64_t)seg * seg_len;
+  const int64_t j1 = (j0 + seg_len < ntiles_seq) ? (j0 + seg_len) : ntiles_seq;
+  const int ntl = j1 > j0 ? (int)(j1 - j0) : 0;
+  const int64_t tok_base = (int64_t)bi * L;
+  const bool last_seg = FULL && (seg == sg.nseg - 1);
+
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + C::OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::OFF_MISC + 4);
+  const uint32_t sStage = smem_u32(sm + C::OFF_STAGE);
+  const uint32_t sSP = smem_u32(sm + C::OFF_SP), sHB = smem_u32(sm + C::OFF_HB);
+  auto sB = [&](int s) { return sStage + (uint32_t)(s * C::STAGE); };
+  auto sC = [&](int s) { return sStage + (uint32_t)(s * C::STAGE + C::TILE_N); };
+  auto recA = [&](int cs) { return reinterpret_cast<float4*>(sm + C::OFF_REC + cs * C::REC_SLOT); };
+  auto mult = [&](int cs) { return reinterpret_cast<float*>(sm + C::OFF_REC + cs * C::REC_SLOT + Q * 16); };
+  auto scal = [&](int cs) { return reinterpret_cast<float*>(sm + C::OFF_REC + cs * C::REC_SLOT + Q * 20); };
+  double* base = reinterpret_cast<double*>(sm + C::OFF_BASE);
+  float* segsum = reinterpret_cast<float*>(sm + C::OFF_SEGSUM);
+  const __nv_bfloat16* xg = static_cast<const __nv_bfloat16*>(p.x);
+
+  // ---- setup
+  if (warp == W_MMA) {
+    tmem_alloc(tmem_slot, C::TM_COLS);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    const int ce = FULL ? (N_ROT + 4 + 4 + 1) : (N_ROT + 4 + 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[B_BCF + s], 1);
+      mbar_init(&bar[B_BCE + s], 1);
+      mbar_init(&bar[B_ROT + s], N_ROT);
+      mbar_init(&bar[B_XPF + s], 4);
+      mbar_init(&bar[B_XBF + s], 1);
+    }
+    for (int c = 0; c < WS_CS; ++c) {
+      mbar_init(&bar[B_CF + c], 1);
+      mbar_init(&bar[B_CE + c], ce);
+    }
+    mbar_init(&bar[B_RESC], N_ROT);
+    mbar_init(&bar[B_SF], 1);
+    mbar_init(&bar[B_SPF], 4);
+    mbar_init(&bar[B_HF], 4);
+    mbar_init(&bar[B_SPGO], 1);
+    mbar_init(&bar[B_YF], 1);
+    mbar_init(&bar[B_YE], 4);
+    mbar_init(&bar[B_DRAIN], 1);
+    mbar_init(&bar[B_FIN], N_ROT);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  {
+    float* bias = reinterpret_cast<float*>(sm + C::OFF_BIAS);
+    for (int i = tid; i < 2 * R * N; i += WS_THREADS) {
+      const int which = i / (R * N), rn = i % (R * N);
+      const float* src = which == 0 ? p.bias_B : p.bias_C;
+      bias[(which * R + rn / N) * (C::BIAS_ROW / 4) + rn % N] = src ? src[(int64_t)hi * R * N + rn] : 0.0f;
+    }
+    for (int k = tid; k < K2; k += WS_THREADS) base[k] = 0.0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (ntl > 0) {
+    if (warp == W_PROD) {
+      // =============================================================== producer
+      if (lane == 0) {
+        Phases ph_e;
+        int issued0 = 0, issued1 = 0;
+        for (int i = 0; i < ntl; ++i) {
+          const int s = i & 1;
+          if (i >= 2) {
+            if (!ws_wait(&bar[B_BCE + s], ph_e[s], abort_flag)) break;
+            ph_e.flip(s);
+          }
+          const int tok = (int)(tok_base + (j0 + i) * Q);
+          mbar_expect_tx(&bar[B_BCF + s], FULL ? C::STAGE : C::TILE_N);
+#pragma unroll
+          for (int blk = 0; blk < N / 64; ++blk) {
+            tma_load_4d(sB(s) + blk * BLK, &tmB, 64 * blk, 0, g, tok, &bar[B_BCF + s]);
+            if constexpr (FULL) tma_load_4d(sC(s) + blk * BLK, &tmC, 64 * blk, 0, g, tok, &bar[B_BCF + s]);
+          }
+          if (s) ++issued1; else ++issued0;
+        }
+        // every copy issued has landed before the CTA may exit
+        if (issued0 > 0) ws_wait_drain(&bar[B_BCF + 0], (uint32_t)((issued0 - 1) & 1));
+        if (issued1 > 0) ws_wait_drain(&bar[B_BCF + 1], (uint32_t)((issued1 - 1) & 1));
+      }
+    } else if (warp == W_COEF) {
+      // =============================================================== coefficients
+      constexpr int TPL = Q >= 32 ? Q / 32 : 1;  // tokens per lane
+      float lrho_prev = 0.0f, seg_logdec = 0.0f;
+      Phases ph_ce;
+      for (int i = 0; i < ntl; ++i) {
+        const int cs = i % WS_CS;
+        const int64_t c0 = (j0 + i) * Q;
+        const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
+        if (i >= WS_CS) {
+          if (!ws_wait(&bar[B_CE + cs], ph_ce[cs], abort_flag)) break;
+          ph_ce.flip(cs);
+        }
+        float dtv[TPL], av[TPL], lmv[TPL], loc[TPL];
+        float run = 0.0f;
+#pragma unroll
+        for (int e = 0; e < TPL; ++e) {
+          const int t = lane * TPL + e;
+          const bool valid = t < nv && t < Q;
+          const int64_t ti = (tok_base + c0 + t) * H + hi;
+          dtv[e] = valid ? p.dt[ti] : 0.0f;
+          av[e] = valid ? p.A[ti] : 0.0f;
+          lmv[e] = valid ? p.lam[ti] : 0.0f;
+          run += dtv[e] * av[e];
+          loc[e] = run;
+        }
+        float incl = run;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const float o = __shfl_up_sync(kFull, incl, off);
+          if (lane >= off) incl += o;
+        }
+        const float Le = __shfl_sync(kFull, incl, 31);
+        const float excl = incl - run;
+        float lmin = 0.0f, lmax = 0.0f;
+#pragma unroll
+        for (int e = 0; e < TPL; ++e) {
+          loc[e] += excl;
+          if (lane * TPL + e < Q) {
+            lmin = fminf(lmin, loc[e]);
+            lmax = fmaxf(lmax, loc[e]);
+          }
+        }
+        lmin = key_float(__reduce_min_sync(kFull, float_key(lmin)));
+        lmax = key_float(__reduce_max_sync(kFull, float_key(lmax)));
+        const bool fast = (lmax - lmin) <= WS_FAST_RANGE;
+        const float m = fast ? 0.5f * (lmax + lmin) : 0.0f;
+        // beta' of the token after each token: the next lane's first token, or the token after the tile
+        float bp_after = 0.0f;
+        if (c0 + Q < L) {
+          const int64_t ti = (tok_base + c0 + Q) * H + hi;
+          bp_after = (1.0f - p.lam[ti]) * p.dt[ti];
+        }
+        const float nxt_dt = __shfl_down_sync(kFull, dtv[0], 1);
+        const float nxt_lm = __shfl_down_sync(kFull, lmv[0], 1);
+        float4* ra = recA(cs);
+        float* mu = mult(cs);
+#pragma unroll
+        for (int e = 0; e < TPL; ++e) {
+          const int t = lane * TPL + e;
+          if (t < Q) {
+            const bool valid = t < nv;
+            const float gm = lmv[e] * dtv[e];
+            float bpn;
+            if (t + 1 >= Q) bpn = valid ? bp_after : 0.0f;
+            else if (e + 1 < TPL) bpn = (1.0f - lmv[e + 1]) * dtv[e + 1];
+            else bpn = (1.0f - nxt_lm) * nxt_dt;  // invalid next tokens carry dt = 0
+            const float w = gm + bpn;
+            const float dg = (w > 0.0f) ? __fdividef(gm, w) : 0.0f;
+            float cb, cc;
+            if (fast) {
+              cb = __expf(m - loc[e]) * w;
+              cc = __expf(loc[e] - m);
+            } else if (FULL) {
+              cb = w;  // rescaled by e^{Le - Lc_t} after S
+              cc = 1.0f;
+            } else {
+              cb = __expf(Le - loc[e]) * w;  // state pass: no S, the final factor at once
+              cc = 1.0f;
+            }
+            ra[t] = make_float4(loc[e], dg, cb, cc);
+            mu[t] = valid ? (p.angle_direct ? 1.0f : dtv[e]) : 0.0f;
+          }
+        }
+        // state scale factors: ST enters tile i as sigma ST_i (sigma = e^m, or e^{Le} on an exact
+        // tile) and leaves it as rho ST_{i+1} (rho = e^{m - Le}, or 1 on an exact tile, whose H
+        // operand already carries e^{Le - Lc_s})
+        const float lsig = fast ? m : Le;
+        const float lrho = fast ? (m - Le) : 0.0f;
+        if (lane == 0) {
+          float* sc = scal(cs);
+          sc[0] = fast ? 1.0f : 0.0f;
+          sc[1] = Le;
+          sc[2] = m;
+          sc[3] = __expf(m - lrho_prev);     // hb = bf16(f_h * tensor-memory state)
+          sc[4] = __expf(lsig - lrho_prev);  // state before H = f_s * tensor-memory state
+          sc[5] = __expf(-lrho);             // true state after the tile = this * tensor-memory state
+          sc[6] = (float)nv;
+        }
+        lrho_prev = lrho;
+        seg_logdec += Le;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[B_CF + cs]);
+      }
+      if constexpr (!FULL) {
+        if (lane == 0 && !*abort_flag) sg.ws_l[(int64_t)bh * sg.nsub + seg] = seg_logdec;
+      }
+    } else if (warp >= W_ROT && warp < W_ROT + N_ROT) {
+      // =============================================================== rotation
+      const int rt = tid - 32 * W_ROT;
+      const int wr = warp - W_ROT;
+      const int ak = rt % K2, aseg = rt / K2;
+      float thr[C::SEGLEN];
+      auto load_theta = [&](int64_t j) {
+        const int64_t c0 = j * Q;
+#pragma unroll
+        for (int e = 0; e < C::SEGLEN; ++e) {
+          const int t = aseg * C::SEGLEN + e;
+          thr[e] = (c0 + t < L) ? p.theta[((tok_base + c0 + t) * G + g) * K2 + ak] : 0.0f;
+        }
+      };
+      load_theta(j0);
+      Phases ph_cf, ph_bcf;
+      const float* biasT = reinterpret_cast<const float*>(sm + C::OFF_BIAS);
+      uint8_t* tab = sm + C::OFF_TAB;
+      for (int i = 0; i < ntl; ++i) {
+        const int cs = i % WS_CS, s = i & 1;
+        const int64_t j = j0 + i;
+        const int64_t c0 = j * Q;
+        const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
+        bool okw = ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag);
+        ph_cf.flip(cs);
+        okw = okw && ws_wait(&bar[B_BCF + s], ph_bcf[s], abort_flag);
+        ph_bcf.flip(s);
+        if (bar_any(BAR_ROT, 32 * N_ROT, !okw || *abort_flag)) break;  // the group stops together
+        const float* mu = mult(cs);
+        const float4* ra = recA(cs);
+        const float* sc = scal(cs);
+        // ---- cumulative angles of the tile and their sin / cos
+        float aloc[C::SEGLEN];
+        {
+          float r2 = 0.0f;
+#pragma unroll
+          for (int e = 0; e < C::SEGLEN; ++e) {
+            r2 = fmaf(mu[aseg * C::SEGLEN + e], thr[e], r2);
+            aloc[e] = r2;
+          }
+          segsum[aseg * K2 + ak] = r2;
+        }
+        named_bar_sync(BAR_ROT, 32 * N_ROT);
+        double tot = 0.0;
+        {
+          float aoff = (float)base[ak];
+#pragma unroll
+          for (int s2 = 0; s2 < C::SEGS; ++s2) {
+            const float v = segsum[s2 * K2 + ak];
+            if (s2 < aseg) aoff += v;
+            if (aseg == 0) tot += (double)v;
+          }
+#pragma unroll
+          for (int e = 0; e < C::SEGLEN; ++e) {
+            const int t = aseg * C::SEGLEN + e;
+            float sn, cn;
+            sincos_reduced(aoff + aloc[e], &sn, &cn);
+            *reinterpret_cast<float2*>(tab + t * C::TAB_ROW + ak * 8) = make_float2(cn, sn);
+          }
+        }
+        if (i + 1 < ntl) load_theta(j + 1);
+        named_bar_sync(BAR_ROT, 32 * N_ROT);  // table complete; base and segsum read
+        if (aseg == 0) {
+          double nb = base[ak] + tot;
+          nb -= 6.283185307179586 * rint(nb * 0.15915494309189535);
+          base[ak] = nb;
+        }
+        // ---- rotate Bt' (and Ct') of the tile in place: lanes take 32 consecutive rows
+#pragma unroll 1
+        for (int q = 0; q < C::KCW; ++q) {
+          const int kc = wr + N_ROT * q;
+          const int r = lane % R;
+          const float4 bb0 = *reinterpret_cast<const float4*>(biasT + r * (C::BIAS_ROW / 4) + 8 * kc);
+          const float4 bb1 = *reinterpret_cast<const float4*>(biasT + r * (C::BIAS_ROW / 4) + 8 * kc + 4);
+          float4 bc0 = make_float4(0.f, 0.f, 0.f, 0.f), bc1 = bc0;
+          if constexpr (FULL) {
+            bc0 = *reinterpret_cast<const float4*>(biasT + (R + r) * (C::BIAS_ROW / 4) + 8 * kc);
+            bc1 = *reinterpret_cast<const float4*>(biasT + (R + r) * (C::BIAS_ROW / 4) + 8 * kc + 4);
+          }
+#pragma unroll 2
+          for (int step = 0; step < 4; ++step) {
+            const int row = 32 * step + lane;
+            const int t = row / R;
+            const uint32_t off = (uint32_t)(kc >> 3) * BLK + (uint32_t)row * 128u +
+                                 ((uint32_t)((kc & 7) ^ (row & 7)) << 4);
+            if (t < nv) {
+              const float4 rec = ra[t];
+              const float4 cs01 = *reinterpret_cast<const float4*>(tab + t * C::TAB_ROW + kc * 32);
+              const float4 cs23 = *reinterpret_cast<const float4*>(tab + t * C::TAB_ROW + kc * 32 + 16);
+              const uint4 rb = lds128(sB(s) + off);
+              uint4 rc;
+              if constexpr (FULL) rc = lds128(sC(s) + off);
+              sts128(sB(s) + off, rotate_chunk(rb, bb0, bb1, cs01, cs23, rec.z));
+              if constexpr (FULL) sts128(sC(s) + off, rotate_chunk(rc, bc0, bc1, cs01, cs23, rec.w));
+            } else {
+              sts128(sB(s) + off, make_uint4(0, 0, 0, 0));
+              if constexpr (FULL) sts128(sC(s) + off, make_uint4(0, 0, 0, 0));
+            }
+          }
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[B_ROT + s]);
+        if (FULL && sc[0] == 0.0f) {
+          // exact tile: after S has read them, Ct' rows * e^{Lc_t} (inter-chunk product) and
+          // Bt' rows * e^{Le - Lc_t} (state product)
+          const bool oks = ws_wait(&bar[B_SF], (uint32_t)(i & 1), abort_flag);
+          if (bar_any(BAR_ROT, 32 * N_ROT, !oks || *abort_flag)) break;
+          const float Le = sc[1];
+#pragma unroll 1
+          for (int q = 0; q < C::KCW; ++q) {
+            const int kc = wr + N_ROT * q;
+            for (int step = 0; step < 4; ++step) {
+              const int row = 32 * step + lane;
+              const int t = row / R;
+              if (t >= nv) continue;
+              const uint32_t off = (uint32_t)(kc >> 3) * BLK + (uint32_t)row * 128u +
+                                   ((uint32_t)((kc & 7) ^ (row & 7)) << 4);
+              const float Lct = ra[t].x;
+              sts128(sC(s) + off, scale_chunk(lds128(sC(s) + off), __expf(Lct)));
+              sts128(sB(s) + off, scale_chunk(lds128(sB(s) + off), __expf(Le - Lct)));
+            }
+          }
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[B_RESC]);
+        }
+        if (lane == 0) mbar_arrive(&bar[B_CE + cs]);
+      }
+      // final angles of the segment: the full pass rotates the state back by them, the state
+      // pass stores them in its summary
+      named_bar_sync(BAR_ROT, 32 * N_ROT);
+      if (!*abort_flag) {
+        if constexpr (!FULL) {
+          if (aseg == 0) sg.ws_phi[((int64_t)bh * sg.nsub + seg) * K2 + ak] = base[ak];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[B_FIN]);
+      }
+    } else if (warp == W_MMA) {
+      // =============================================================== MMA issue
+      Phases ph_cf, ph_rot, ph_xpf;
+      uint32_t ph_hf = 0, ph_resc = 0, ph_ye = 0, ph_spf = 0;
+      bool issued = false, ok = true;
+      auto kdesc = [&](uint32_t base_addr, int k) {  // K-major SW128 operand, K-step k of 16
+        return sdesc(base_addr + (uint32_t)(k >> 2) * BLK + (uint32_t)(k & 3) * 32, 16, 1024);
+      };
+      if (FULL) {
+        ok = ws_wait(&bar[B_ROT + 0], ph_rot[0], abort_flag);
+        ph_rot.flip(0);
+        if (ok) {
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < N / 16; ++k)
+            mma_ss_w(tmem + C::TM_S, kdesc(sC(0), k), kdesc(sB(0), k), C::ID_S, k > 0);
+          mma_commit_w(&bar[B_SF]);
+          issued = true;
+        }
+      }
+      for (int i = 0; ok && i < ntl; ++i) {
+        const int cs = i % WS_CS, s = i & 1, xb = i & 1;
+        if (!ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag)) break;
+        ph_cf.flip(cs);
+        const bool fast = scal(cs)[0] != 0.0f;
+        if (!ws_wait(&bar[B_HF], ph_hf, abort_flag)) break;
+        ph_hf ^= 1;
+        if (FULL && !fast) {
+          if (!ws_wait(&bar[B_RESC], ph_resc, abort_flag)) break;
+          ph_resc ^= 1;
+        }
+        if (!ws_wait(&bar[B_XPF + xb], ph_xpf[xb], abort_flag)) break;
+        ph_xpf.flip(xb);
+        if constexpr (!FULL) {  // the full pass waited for the rotation before S of this tile
+          if (!ws_wait(&bar[B_ROT + s], ph_rot[s], abort_flag)) break;
+          ph_rot.flip(s);
+        }
+        tc_fence_after();
+        // H: ST += X'^T Bt'  (A = X'^T in tensor memory, B = Bt' MN-major)
+#pragma unroll
+        for (int k = 0; k < 128 / 16; ++k)
+          mma_ts_w(tmem + C::TM_ST, tmem + C::TM_XP + 64 * xb + 8 * k,
+                   sdesc(sB(s) + (uint32_t)k * 2048, BLK, 1024), C::ID_H, 1);
+        issued = true;
+        if constexpr (!FULL) {
+          mma_commit_w(&bar[B_SPGO]);
+          mma_commit_w(&bar[B_XBF + xb]);
+          mma_commit_w(&bar[B_BCE + s]);
+        } else {
+          if (i > 0) {
+            if (!ws_wait(&bar[B_YE], ph_ye, abort_flag)) break;
+            ph_ye ^= 1;
+            tc_fence_after();
+          }
+          // Y_inter: Y^T = hb Ct'^T  (A = hb K-major, B = Ct' K-major)
+#pragma unroll
+          for (int k = 0; k < N / 16; ++k)
+            mma_ss_w(tmem + C::TM_Y, kdesc(sHB, k), kdesc(sC(s), k), C::ID_Y, k > 0);
+          mma_commit_w(&bar[B_SPGO]);
+          mma_commit_w(&bar[B_BCE + s]);
+          if (!ws_wait(&bar[B_SPF], ph_spf, abort_flag)) break;
+          ph_spf ^= 1;
+          tc_fence_after();
+          // Y_intra: Y^T += X'^T S'^T  (A = X'^T in tensor memory, B = S' K-major)
+#pragma unroll
+          for (int k = 0; k < 128 / 16; ++k)
+            mma_ts_w(tmem + C::TM_Y, tmem + C::TM_XP + 64 * xb + 8 * k, kdesc(sSP, k), C::ID_Y, 1);
+          mma_commit_w(&bar[B_YF]);
+          mma_commit_w(&bar[B_XBF + xb]);
+          if (i + 1 < ntl) {
+            if (!ws_wait(&bar[B_ROT + (s ^ 1)], ph_rot[s ^ 1], abort_flag)) break;
+            ph_rot.flip(s ^ 1);
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < N / 16; ++k)
+              mma_ss_w(tmem + C::TM_S, kdesc(sC(s ^ 1), k), kdesc(sB(s ^ 1), k), C::ID_S, k > 0);
+            mma_commit_w(&bar[B_SF]);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[B_CE + cs]);
+      }
+      if (issued) {  // every MMA issued has completed before tensor memory is released
+        mma_commit_w(&bar[B_DRAIN]);
+        ws_wait_drain(&bar[B_DRAIN], 0);
+      }
+    } else if (FULL && warp >= W_MASK && warp < W_MASK + 4) {
+      // =============================================================== mask
+      const int q4 = warp & 3;
+      const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+      const int row = 32 * q4 + lane;
+      const int t = row / R;
+      Phases ph_cf;
+      for (int i = 0; i < ntl; ++i) {
+        const int cs = i % WS_CS;
+        if (!ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag)) break;
+        ph_cf.flip(cs);
+        if (!ws_wait(&bar[B_SF], (uint32_t)(i & 1), abort_flag)) break;
+        tc_fence_after();
+        const float4* ra = recA(cs);
+        const bool fast = scal(cs)[0] != 0.0f;
+        const float4 rt4 = ra[t];
+        const float Lt2 = rt4.x * 1.4426950408889634f;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[16];
+          if (c > q4) {  // every column token is after every row token of this warp
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = 0u;
+          } else {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_base + C::TM_S + 32 * c, v);
+            tmem_wait_ld();
+            float f[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
+            if (!fast) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const int st = (32 * c + e) / R;
+                f[e] = (st <= t) ? f[e] * ex2_approx(Lt2 - ra[st].x * 1.4426950408889634f) : 0.0f;
+              }
+            }
+            if (c == q4) {  // the diagonal block: columns of the same token range as the rows
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const int st = (32 * c + e) / R;
+                f[e] = (st < t) ? f[e] : ((st == t) ? f[e] * rt4.y : 0.0f);
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) o[e] = pack_bf16(f[2 * e], f[2 * e + 1]);
+          }
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {
+            const int ch = 4 * c + qq;
+            const uint32_t off = (uint32_t)(ch >> 3) * BLK + (uint32_t)row * 128u +
+                                 ((uint32_t)((ch & 7) ^ (row & 7)) << 4);
+            sts128(sSP + off, make_uint4(o[4 * qq], o[4 * qq + 1], o[4 * qq + 2], o[4 * qq + 3]));
+          }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bar[B_SPF]);
+          mbar_arrive(&bar[B_CE + cs]);
+        }
+      }
+    } else if (FULL && warp >= W_EPI && warp < W_EPI + 4) {
+      // =============================================================== epilogue
+      const int q4 = warp & 3;
+      const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+      const int pc = 32 * q4 + lane;  // head-dim column of this thread
+      float wo[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) wo[r] = p.W_o ? p.W_o[((int64_t)hi * R + r) * WP + pc] : 1.0f;
+      const float Dh = p.D ? p.D[hi] : 0.0f;
+      __nv_bfloat16* yg = static_cast<__nv_bfloat16*>(p.y);
+      constexpr int TPC = 32 / R;  // tokens per 32-column chunk
+      for (int i = 0; i < ntl; ++i) {
+        const int64_t c0 = (j0 + i) * Q;
+        const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
+        if (!ws_wait(&bar[B_YF], (uint32_t)(i & 1), abort_flag)) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          float xv[TPC];
+#pragma unroll
+          for (int u = 0; u < TPC; ++u) {
+            const int t = TPC * c + u;
+            xv[u] = (p.D && t < nv) ? __bfloat162float(xg[((tok_base + c0 + t) * H + hi) * (int64_t)WP + pc]) : 0.0f;
+          }
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_base + C::TM_Y + 32 * c, v);
+          tmem_wait_ld();
+          if (c == 3) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[B_YE]);
+          }
+#pragma unroll
+          for (int u = 0; u < TPC; ++u) {
+            const int t = TPC * c + u;
+            float acc = Dh * xv[u];
+#pragma unroll
+            for (int r = 0; r < R; ++r) acc = fmaf(wo[r], __uint_as_float(v[u * R + r]), acc);
+            if (t < nv) yg[((tok_base + c0 + t) * H + hi) * (int64_t)WP + pc] = __float2bfloat16_rn(acc);
+          }
+        }
+      }
+    } else if (warp >= W_SPX && warp < W_SPX + 4) {
+      // =============================================================== state and inputs
+      const int q4 = warp & 3;
+      const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+      const int pc = 32 * q4 + lane;
+      float wx[R];
+#pragma unroll
+      for (int r = 0; r < R; ++r) wx[r] = p.W_x ? p.W_x[((int64_t)hi * R + r) * WP + pc] : 1.0f;
+      Phases ph_cf, ph_xbf;
+      constexpr int TPC = 32 / R;
+      // X'^T of tile i: X'^T[p, tR + r] = W_x[r, p] x_t[p], bf16 pairs along the columns
+      auto build_xp = [&](int i) -> bool {
+        const int xb = i & 1;
+        if (i >= 2) {
+          if (!ws_wait(&bar[B_XBF + xb], ph_xbf[xb], abort_flag)) return false;
+          ph_xbf.flip(xb);
+        }
+        const int64_t c0 = (j0 + i) * Q;
+        const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
+        tc_fence_after();
+#pragma unroll 1
+        for (int gq = 0; gq < 4; ++gq) {
+          float xv[TPC];
+#pragma unroll
+          for (int u = 0; u < TPC; ++u) {
+            const int t = TPC * gq + u;
+            xv[u] = (t < nv) ? __bfloat162float(xg[((tok_base + c0 + t) * H + hi) * (int64_t)WP + pc]) : 0.0f;
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c2 = 2 * e;  // column pair (c2, c2 + 1) of this 32-column group
+            w[e] = pack_bf16(wx[c2 % R] * xv[c2 / R], wx[(c2 + 1) % R] * xv[(c2 + 1) / R]);
+          }
+          tmem_st16(tmem + lane_base + C::TM_XP + 64 * xb + 16 * gq, w);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar[B_XPF + xb]);
+        return true;
+      };
+      bool ok = build_xp(0);
+      for (int i = 0; ok && i < ntl; ++i) {
+        const int cs = i % WS_CS;
+        if (!ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag)) break;
+        ph_cf.flip(cs);
+        const float fh = scal(cs)[3], fs = scal(cs)[4];
+        if (i == 0) {
+          // the rotated-frame state entering the segment (h+: it includes the previous token's
+          // trapezoid term beta'_0 u_{-1})
+          const bool from_state = FULL ? (seg == 0) : false;
+          const bool make_init = !FULL && seg == 0 && sg.write_init;
+          const bool fold = FULL && seg > 0;
+          const int nfold = fold ? seg * (sg.seg_tiles / sg.sub_tiles) : 0;
+          float bp0 = 0.0f, xprev[R];
+          if (from_state || make_init) {
+            bp0 = (1.0f - p.lam[tok_base * H + hi]) * p.dt[tok_base * H + hi];
+#pragma unroll
+            for (int r = 0; r < R; ++r) xprev[r] = wx[r] * p.carry_x[(int64_t)bh * WP + pc];
+          }
+          const float* h0 = p.h + (int64_t)bh * N * WP;
+          const float* cB = p.carry_B + (int64_t)bh * R * N;
+          const float* bB = p.bias_B ? p.bias_B + (int64_t)hi * R * N : nullptr;
+#pragma unroll 1
+          for (int c = 0; c < N / 32; ++c) {
+            float v[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = 0.0f;
+            if (from_state || make_init) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const int n = 32 * c + e;
+                float u = 0.0f;
+#pragma unroll
+                for (int r = 0; r < R; ++r) u = fmaf(cB[r * N + n] + (bB ? bB[r * N + n] : 0.0f), xprev[r], u);
+                v[e] = fmaf(bp0, u, h0[(int64_t)n * WP + pc]);
+              }
+              if (make_init) {
+                float* wi = sg.ws_init + (int64_t)bh * N * WP;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) wi[(int64_t)(32 * c + e) * WP + pc] = v[e];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = 0.0f;  // the state pass starts from zero
+              }
+            } else if (fold) {
+              const float* wi = sg.ws_init + (int64_t)bh * N * WP;
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] = wi[(int64_t)(32 * c + e) * WP + pc];
+              for (int k = 0; k < nfold; ++k) {
+                const int64_t sidx = (int64_t)bh * sg.nsub + k;
+                const float dec = __expf(sg.ws_l[sidx]);
+                const float* wh = sg.ws_h + sidx * N * WP;
+                const double* ph = sg.ws_phi + sidx * K2;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                  const int n0 = 32 * c + 2 * e;
+                  float sn, cn;
+                  sincosf((float)ph[n0 / 2], &sn, &cn);
+                  const float a0 = fmaf(dec, v[2 * e], wh[(int64_t)n0 * WP + pc]);
+                  const float a1 = fmaf(dec, v[2 * e + 1], wh[(int64_t)(n0 + 1) * WP + pc]);
+                  v[2 * e] = cn * a0 - sn * a1;
+                  v[2 * e + 1] = sn * a0 + cn * a1;
+                }
+              }
+            }
+            uint32_t u32[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) u32[e] = __float_as_uint(fs * v[e]);
+            tmem_st32(tmem + lane_base + C::TM_ST + 32 * c, u32);
+            if constexpr (FULL) hb_store_row(sHB, pc, c, v, fh);
+          }
+        } else {
+          if (!ws_wait(&bar[B_SPGO], (uint32_t)((i - 1) & 1), abort_flag)) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < N / 32; ++c) {
+            uint32_t u32[32];
+            tmem_ld32(tmem + lane_base + C::TM_ST + 32 * c, u32);
+            tmem_wait_ld();
+            float v[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              v[e] = __uint_as_float(u32[e]);
+              u32[e] = __float_as_uint(fs * v[e]);
+            }
+            tmem_st32(tmem + lane_base + C::TM_ST + 32 * c, u32);
+            if constexpr (FULL) hb_store_row(sHB, pc, c, v, fh);
+          }
+        }
+        tmem_wait_st();
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&bar[B_HF]);
+          mbar_arrive(&bar[B_CE + cs]);
+        }
+        if (i + 1 < ntl) ok = build_xp(i + 1);
+      }
+      // ---- results: the state after the last tile
+      const bool results = ok && !*abort_flag && (!FULL || last_seg);
+      if (results && ws_wait(&bar[B_SPGO], (uint32_t)((ntl - 1) & 1), abort_flag)) {
+        tc_fence_after();
+        const float inv_rho = scal((ntl - 1) % WS_CS)[5];
+        if constexpr (FULL) {
+          // rotate back from the segment frame by the segment's total angle
+          if (ws_wait(&bar[B_FIN], 0, abort_flag)) {
+            float* hout = p.h + (int64_t)bh * N * WP;
+#pragma unroll 1
+            for (int c = 0; c < N / 32; ++c) {
+              uint32_t sv[32];
+              tmem_ld32(tmem + lane_base + C::TM_ST + 32 * c, sv);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const int k = 16 * c + e;
+                float sn, cn;
+                sincosf((float)base[k], &sn, &cn);
+                const float a0 = inv_rho * __uint_as_float(sv[2 * e]);
+                const float a1 = inv_rho * __uint_as_float(sv[2 * e + 1]);
+                hout[(int64_t)(2 * k) * WP + pc] = cn * a0 - sn * a1;
+                hout[(int64_t)(2 * k + 1) * WP + pc] = sn * a0 + cn * a1;
+              }
+            }
+            // the carry: the last token's raw B and x
+            const int64_t tokl = tok_base + (L - 1);
+            const __nv_bfloat16* Bg = static_cast<const __nv_bfloat16*>(p.B);
+            const int64_t bc = ((tokl * G + g) * R) * (int64_t)N;
+            for (int k = pc; k < R * N; k += WP) p.carry_B[(int64_t)bh * R * N + k] = __bfloat162float(Bg[bc + k]);
+            p.carry_x[(int64_t)bh * WP + pc] = __bfloat162float(xg[(tokl * H + hi) * (int64_t)WP + pc]);
+          }
+        } else {
+          float* wh = sg.ws_h + ((int64_t)bh * sg.nsub + seg) * N * WP;
+#pragma unroll 1
+          for (int c = 0; c < N / 32; ++c) {
+            uint32_t sv[32];
+            tmem_ld32(tmem + lane_base + C::TM_ST + 32 * c, sv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) wh[(int64_t)(32 * c + e) * WP + pc] = inv_rho * __uint_as_float(sv[e]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && *abort_flag) set_status(p.status, M3_ERR_TIMEOUT);
+  if (warp == W_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TM_COLS);
+  }
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ host side
+
+bool ws_scan_supported(const Params& p) {
+  if (p.dtype != M3_BF16 || p.P != WP) return false;
+  if (p.N == 128) return p.R == 4 || p.R == 8;
+  if (p.N == 64) return p.R == 2 || p.R == 4 || p.R == 8;
+  return false;
+}
+
+namespace {
+template <int R, int N, int MODE>
+cudaError_t launch_ws_mode(const CUtensorMap& tmB, const CUtensorMap& tmC, const Params& p, const SegInfo& sg,
+                           unsigned grid, cudaStream_t stream) {
+  using Cf = WsCfg<R, N>;
+  static SmemAttr attr;
+  auto k = scan_ws_kernel<R, N, MODE>;
+  cudaError_t e = attr.ensure(k, Cf::SMEM);
+  if (e != cudaSuccess) return e;
+  k<<<grid, WS_THREADS, Cf::SMEM, stream>>>(tmB, tmC, p, sg);
+  return cudaGetLastError();
+}
+
+template <int R, int N>
+cudaError_t launch_ws_rn(const CUtensorMap& tmB, const CUtensorMap& tmC, const Params& p, const SegInfo& sg,
+                         cudaStream_t stream) {
+  const int64_t nseq = p.b * p.H;
+  if (sg.nseg > 1) {
+    cudaError_t e = launch_ws_mode<R, N, WS_STATE>(tmB, tmC, p, sg, (unsigned)(nseq * sg.nsub), stream);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_ws_mode<R, N, WS_FULL>(tmB, tmC, p, sg, (unsigned)(nseq * sg.nseg), stream);
+}
+}  // namespace
+
+cudaError_t launch_scan_ws_state(const CUtensorMap& tmB, const CUtensorMap& tmC, const Params& p,
+                                 const SegInfo& sg, cudaStream_t stream) {
+  const unsigned grid = (unsigned)(p.b * p.H * sg.nsub);
+  if (p.N == 128) return p.R == 4 ? launch_ws_mode<4, 128, WS_STATE>(tmB, tmC, p, sg, grid, stream)
+                                  : launch_ws_mode<8, 128, WS_STATE>(tmB, tmC, p, sg, grid, stream);
+  switch (p.R) {
+    case 2: return launch_ws_mode<2, 64, WS_STATE>(tmB, tmC, p, sg, grid, stream);
+    case 4: return launch_ws_mode<4, 64, WS_STATE>(tmB, tmC, p, sg, grid, stream);
+    default: return launch_ws_mode<8, 64, WS_STATE>(tmB, tmC, p, sg, grid, stream);
+  }
+}
+
+cudaError_t launch_scan_ws(const CUtensorMap& tmB, const CUtensorMap& tmC, const Params& p, const SegInfo& sg,
+                           cudaStream_t stream) {
+  if (p.N == 128) return p.R == 4 ? launch_ws_rn<4, 128>(tmB, tmC, p, sg, stream)
+                                  : launch_ws_rn<8, 128>(tmB, tmC, p, sg, stream);
+  switch (p.R) {
+    case 2: return launch_ws_rn<2, 64>(tmB, tmC, p, sg, stream);
+    case 4: return launch_ws_rn<4, 64>(tmB, tmC, p, sg, stream);
+    default: return launch_ws_rn<8, 64>(tmB, tmC, p, sg, stream);
+  }
+}
+
+}  // namespace m3

@@ -54,6 +54,9 @@ SIGNATURES = {
     "m3_scan_fwd": (_I, [_DP] + [_VP] * 14 + [_VP, _SZ, _VP]),
     "m3_scan_fwd_noalloc": (_I, [_DP] + [_VP] * 14 + [_VP]),
     "m3_decode_step": (_I, [_DP] + [_VP] * 15),
+    "m3_scan_summary_workspace_size": (_I, [_DP, ctypes.POINTER(_SZ)]),
+    "m3_scan_summary": (_I, [_DP] + [_VP] * 14 + [_VP, _SZ, _VP]),
+    "m3_state_fold": (_I, [_DP, ctypes.c_int32] + [_VP] * 8 + [_VP, _VP]),
     "m3_check": (_I, [_VP]),
     "m3_selftest_wait": (_I, [ctypes.c_uint64, _VP]),
     "m3_status_str": (ctypes.c_char_p, [_I]),
@@ -187,6 +190,29 @@ def m3_decode_step(dims: Dims, x_t, dt_t, A_t, lam_t, B_t, C_t, theta_t, bias_B,
     _check(lib().m3_decode_step(ctypes.byref(dims), _ptr(x_t), _ptr(dt_t), _ptr(A_t), _ptr(lam_t), _ptr(B_t),
                                 _ptr(C_t), _ptr(theta_t), _ptr(bias_B), _ptr(bias_C), _ptr(W_x), _ptr(W_o),
                                 _ptr(D), state.handle, _ptr(y_t), _stream(stream)), "m3_decode_step")
+
+
+def m3_scan_summary_workspace_size(dims: Dims) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().m3_scan_summary_workspace_size(ctypes.byref(dims), ctypes.byref(n)),
+           "m3_scan_summary_workspace_size")
+    return n.value
+
+
+def m3_scan_summary(dims: Dims, x, dt, A, lam, B, theta, bias_B, W_x, Z, logdec, angle, bp_first, carry_B,
+                    carry_x, workspace, stream=None):
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().m3_scan_summary(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(lam), _ptr(B), _ptr(theta),
+                                 _ptr(bias_B), _ptr(W_x), _ptr(Z), _ptr(logdec), _ptr(angle), _ptr(bp_first),
+                                 _ptr(carry_B), _ptr(carry_x), _ptr(workspace), ws_bytes, _stream(stream)),
+           "m3_scan_summary")
+
+
+def m3_state_fold(dims: Dims, nranges: int, Z, logdec, angle, bp_first, carry_B, carry_x, bias_B, W_x,
+                  state: State, stream=None):
+    _check(lib().m3_state_fold(ctypes.byref(dims), int(nranges), _ptr(Z), _ptr(logdec), _ptr(angle),
+                               _ptr(bp_first), _ptr(carry_B), _ptr(carry_x), _ptr(bias_B), _ptr(W_x),
+                               state.handle, _stream(stream)), "m3_state_fold")
 
 
 def m3_check(stream=None) -> int:

@@ -379,6 +379,21 @@ def test_tc_scan_shapes(shape, with_state):
     check_scan(inp, state=st)
 
 
+@pytest.mark.parametrize("shape", [
+    dict(b=1, L=3000, H=2, P=64, N=64, R=2, G=1),
+    dict(b=1, L=4000, H=2, P=128, N=128, R=4, G=1),
+], ids=["P64", "P128"])
+def test_segmented_slow_decay_carries_initial_state(shape):
+    # With dt*A near zero the initial state survives the whole sequence, so every segment's
+    # incoming state must carry it exactly once (segments are summarised from a zero start
+    # and folded onto the initial state)
+    inp = make_inputs(dtype="bf16", seed=208, extras=True, **shape)
+    inp.A[:] = -1e-3
+    st = make_state(shape["b"], shape["H"], shape["P"], shape["N"], shape["R"], seed=209, scale=2.0)
+    assert m3.m3_scan_workspace_size(m3.dims_of(inp)) > 0  # the launch is segmented
+    check_scan(inp, state=st)
+
+
 def test_workspace_is_required_when_segmented():
     inp = make_inputs(dtype="bf16", seed=205, b=1, L=1500, H=2, P=64, N=64, R=2, G=1)
     dims = m3.dims_of(inp)
@@ -442,6 +457,56 @@ def test_tc_strong_decay_tiles(shape):
     inp.A[:, burst, :] = -12.0
     st = make_state(shape["b"], shape["H"], shape["P"], shape["N"], shape["R"], seed=207)
     check_scan(inp, state=st)
+
+
+@pytest.mark.parametrize("P,R,rng", [
+    (128, 4, 60.0), (128, 4, 63.5), (128, 4, 64.5), (128, 4, 100.0),   # headdim 128: limit 64
+    (64, 2, 60.0), (64, 2, 63.5), (64, 2, 64.5), (64, 2, 159.0),       # headdim 64: limit 64
+], ids=lambda v: str(v))
+def test_tc_decay_range_near_pivot_limit(P, R, rng):
+    # Every tile's cumulative log decay spans `rng` (dt = 1, A = -rng / Q per token), B = C is
+    # one fixed unit-RMS vector for every token and branch (so |Ct . Bt| ~ d_state), theta = 0
+    # (no rotation to spread them) and x is large: the pivot-split factors e^{+-rng/2} meet the
+    # largest scores.  Ranges just below each kernel's limit take the pivot split, just above
+    # the exact per-element path; both must stay within tolerance.
+    Q = 128 // R
+    shape = dict(b=1, L=4 * Q + 5, H=2, P=P, N=64, R=R, G=1)
+    inp = make_inputs(dtype="bf16", seed=210, extras=True, **shape)
+    inp.dt[:] = 1.0
+    inp.A[:] = -rng / Q
+    inp.theta[:] = 0.0
+    v = np.random.default_rng(211).standard_normal(shape["N"])
+    v = v / np.sqrt(np.mean(v * v))
+    from selective_state_space_53_b200.inputs import round_to_bf16
+    vb = round_to_bf16(v.astype(np.float32))
+    inp.B[:] = vb
+    inp.C[:] = vb
+    inp.x = round_to_bf16(4.0 * inp.x)
+    check_scan(inp)
+
+
+# headdim 128 runs the warp-specialised kernel for N = 128 with R = 4, 8 and N = 64 with R = 2, 4, 8
+WS_SHAPES = [
+    dict(b=1, L=64, H=2, P=128, N=64, R=2, G=1),
+    dict(b=2, L=333, H=3, P=128, N=64, R=4, G=3),
+    dict(b=1, L=257, H=2, P=128, N=64, R=8, G=2),
+    dict(b=1, L=130, H=2, P=128, N=128, R=8, G=1),
+    dict(b=3, L=97, H=4, P=128, N=128, R=4, G=2),
+    dict(b=1, L=5000, H=1, P=128, N=128, R=4, G=1),  # one sequence: many segments and sub-segments
+]
+
+
+@pytest.mark.parametrize("shape", WS_SHAPES, ids=lambda s: "L{L}N{N}R{R}G{G}".format(**s))
+def test_ws_scan_shapes(shape):
+    inp = make_inputs(dtype="bf16", seed=212, extras=True, **shape)
+    st = make_state(shape["b"], shape["H"], shape["P"], shape["N"], shape["R"], seed=213, scale=0.5)
+    check_scan(inp, state=st)
+
+
+def test_ws_scan_null_weights_and_bias():
+    inp = make_inputs(2, 150, 2, 128, 128, 4, 1, "bf16", seed=214, with_weights=False)
+    inp.bias_B = inp.bias_C = None
+    check_scan(inp)
 
 
 # ------------------------------------------------------------------ direct-angle variant
