@@ -154,6 +154,47 @@ m3_status m3_scan_fwd_noalloc(const m3_dims* dims, const void* x, const float* d
                               const float* W_o, const float* D, m3_state* state, void* y,
                               void* stream);
 
+/* ---- backward pass ----------------------------------------------------------- */
+
+/* Gradients of the layer core: every pointer is caller-owned device memory in the layout of
+ * the operand it belongs to.  dx, dB, dC in dims->dtype; everything else fp32. */
+typedef struct {
+  void* dx;          /* (b, L, H, P)                                  required */
+  float* ddt;        /* (b, L, H)                                     required */
+  float* dA;         /* (b, L, H)                                     required */
+  float* dlam;       /* (b, L, H)                                     required */
+  void* dB;          /* (b, L, G, R, N), summed over a group's heads  required */
+  void* dC;          /* (b, L, G, R, N), summed over a group's heads  required */
+  float* dtheta;     /* (b, L, G, N/2), summed over a group's heads   required */
+  float* dbias_B;    /* (H, R, N), summed over batch and tokens       may be NULL (not computed) */
+  float* dbias_C;    /* (H, R, N)                                     may be NULL */
+  float* dW_x;       /* (H, R, P)                                     may be NULL */
+  float* dW_o;       /* (H, R, P)                                     may be NULL */
+  float* dD;         /* (H)                                           may be NULL */
+  float* dh0;        /* (b, H, N, P): the initial state h             required */
+  float* dcarry_B;   /* (b, H, R, N): the initial carry               required */
+  float* dcarry_x;   /* (b, H, P)                                     required */
+} m3_grads;
+
+/* Scratch bytes m3_scan_bwd needs: the forward states it recomputes (one every ~sqrt(L)
+ * tokens, plus one block of ~sqrt(L) states, per (batch, head)) and fp32 accumulators of dB
+ * and dC. */
+m3_status m3_scan_bwd_workspace_size(const m3_dims* dims, size_t* out_bytes);
+
+/* Backward pass of m3_scan_fwd: the gradients of sum(dy * y) + sum(dh_final * h_L) with
+ * respect to every operand and the initial state.  The operands are those the forward call
+ * took; state0 is the state it started from (not modified).  dy: (b, L, H, P) in dims->dtype;
+ * dh_final: (b, H, N, P) fp32 or NULL (zero).  Gradients whose operand was NULL (no bias, unit
+ * weights, no skip term) are still the gradients at that value.  The chain rule is taken
+ * through the recurrence of the Mamba-3 paper note (sections その1-その3) exactly as written
+ * at the top of this header; the forward states are recomputed in fp32 from checkpoints.
+ * L must be at least 1 (M3_ERR_DIMS otherwise).  Asynchronous on `stream`; allocates nothing. */
+m3_status m3_scan_bwd(const m3_dims* dims, const void* x, const float* dt, const float* A,
+                      const float* lam, const void* B, const void* C, const float* theta,
+                      const float* bias_B, const float* bias_C, const float* W_x, const float* W_o,
+                      const float* D, const m3_state* state0, const void* dy, const float* dh_final,
+                      const m3_grads* grads, void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---- ranges of a sequence (sequence sharding) ---------------------------- */
 
 /* A sequence split into consecutive token ranges (for instance one per device) runs as: every

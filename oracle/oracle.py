@@ -29,6 +29,14 @@ class _Dims(ctypes.Structure):
                 ("G", ctypes.c_int32), ("angle_direct", ctypes.c_int32)]
 
 
+GRAD_KEYS = ("dx", "ddt", "dA", "dlam", "dB", "dC", "dtheta", "dbias_B", "dbias_C", "dW_x", "dW_o", "dD",
+             "dh0", "dcarry_B", "dcarry_x")
+
+
+class _Grads(ctypes.Structure):
+    _fields_ = [(k, ctypes.POINTER(ctypes.c_double)) for k in GRAD_KEYS]
+
+
 def build(force: bool = False) -> str:
     """Compile m3_oracle.c with gcc (-O2, OpenMP) into libm3oracle.so."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
@@ -48,6 +56,8 @@ def _load():
         lib.m3o_scan.argtypes = [ctypes.POINTER(_Dims)] + [dp] * 16 + [
             ctypes.POINTER(ctypes.c_int64), ctypes.c_int64, ctypes.c_int]
         lib.m3o_max_threads.restype = ctypes.c_int
+        lib.m3o_scan_bwd.restype = ctypes.c_int
+        lib.m3o_scan_bwd.argtypes = [ctypes.POINTER(_Dims)] + [dp] * 17 + [ctypes.POINTER(_Grads)]
         _lib = lib
     return _lib
 
@@ -108,3 +118,31 @@ def scan_inputs(inp, sel=None, threads=0, h0=None, carry_B0=None, carry_x0=None,
     return scan(inp.dims, inp.x, inp.dt, inp.A, inp.lam, inp.B, inp.C, inp.theta, inp.bias_B,
                 inp.bias_C, inp.W_x, inp.W_o, inp.D, h0=h0, carry_B0=carry_B0,
                 carry_x0=carry_x0, sel=sel, threads=threads, angle_direct=angle_direct)
+
+
+def scan_bwd(dims, x, dt, A, lam, B, C, theta, bias_B=None, bias_C=None, W_x=None, W_o=None, D=None,
+             h0=None, carry_B0=None, carry_x0=None, dy=None, dh_final=None, angle_direct=False):
+    """Reverse-mode gradient of ``scan`` (m3o_scan_bwd in m3_oracle.c): the gradients of
+    sum(dy * y) + sum(dh_final * h_final) with respect to every operand and the initial state.
+    Returns a dict keyed by GRAD_KEYS (float64; None for an operand passed as None)."""
+    lib = _load()
+    b, L, H, P, N, R, G = (int(dims[k]) for k in ("b", "L", "H", "P", "N", "R", "G"))
+    d = _Dims(b, L, H, P, N, R, G, 1 if angle_direct else 0)
+    h = np.zeros((b, H, N, P)) if h0 is None else _f64(h0)
+    cB = np.zeros((b, H, R, N)) if carry_B0 is None else _f64(carry_B0)
+    cx = np.zeros((b, H, P)) if carry_x0 is None else _f64(carry_x0)
+    arrs = [_f64(a) for a in (x, dt, A, lam, B, C, theta, bias_B, bias_C, W_x, W_o, D)]
+    shapes = {"dx": (b, L, H, P), "ddt": (b, L, H), "dA": (b, L, H), "dlam": (b, L, H), "dB": (b, L, G, R, N),
+              "dC": (b, L, G, R, N), "dtheta": (b, L, G, N // 2), "dbias_B": (H, R, N), "dbias_C": (H, R, N),
+              "dW_x": (H, R, P), "dW_o": (H, R, P), "dD": (H,), "dh0": (b, H, N, P), "dcarry_B": (b, H, R, N),
+              "dcarry_x": (b, H, P)}
+    out = {k: np.zeros(v) for k, v in shapes.items()}
+    gr = _Grads(*[_ptr(out[k]) for k in GRAD_KEYS])
+    rc = lib.m3o_scan_bwd(ctypes.byref(d), *[_ptr(a) for a in arrs], _ptr(h), _ptr(cB), _ptr(cx),
+                          _ptr(_f64(dy)), _ptr(_f64(dh_final)), ctypes.byref(gr))
+    if rc != 0:
+        raise RuntimeError(f"m3o_scan_bwd failed with code {rc}")
+    for k, a in (("dbias_B", bias_B), ("dbias_C", bias_C), ("dW_x", W_x), ("dW_o", W_o), ("dD", D)):
+        if a is None:
+            out[k] = None
+    return out

@@ -290,6 +290,51 @@ m3_status m3_decode_step(const m3_dims* dims, const void* x_t, const float* dt_t
   return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
 }
 
+m3_status m3_scan_bwd_workspace_size(const m3_dims* dims, size_t* out_bytes) {
+  m3_status st = check_dims(dims);
+  if (st != M3_OK) return st;
+  if (!out_bytes) return M3_ERR_NULL;
+  m3::Params p = make_params(dims, dims->L, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                             nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+  if (!m3::bwd_supported(p)) return M3_ERR_UNSUPPORTED;
+  *out_bytes = m3::scan_bwd_workspace_bytes(p);
+  return M3_OK;
+}
+
+m3_status m3_scan_bwd(const m3_dims* dims, const void* x, const float* dt, const float* A, const float* lam,
+                      const void* B, const void* C, const float* theta, const float* bias_B, const float* bias_C,
+                      const float* W_x, const float* W_o, const float* D, const m3_state* state0, const void* dy,
+                      const float* dh_final, const m3_grads* gr, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  size_t need = 0;
+  m3_status st = m3_scan_bwd_workspace_size(dims, &need);
+  if (st != M3_OK) return st;
+  if (!gr) return M3_ERR_NULL;
+  if (dims->L < 1) return M3_ERR_DIMS;  // the backward pass of an empty scan is not defined here
+  const bool tokens = dims->b * dims->L > 0;
+  st = check_operands(dims, x, dt, A, lam, B, C, theta, bias_B, bias_C, W_x, W_o, D, state0, dy, tokens);
+  if (st != M3_OK) return st;
+  const void* req[] = {gr->dx, gr->ddt, gr->dA, gr->dlam, gr->dB, gr->dC, gr->dtheta, gr->dh0, gr->dcarry_B,
+                       gr->dcarry_x};
+  for (const void* q : req)
+    if (!q) return M3_ERR_NULL;
+  const void* all[] = {gr->dx, gr->ddt, gr->dA, gr->dlam, gr->dB, gr->dC, gr->dtheta, gr->dbias_B, gr->dbias_C,
+                       gr->dW_x, gr->dW_o, gr->dD, gr->dh0, gr->dcarry_B, gr->dcarry_x, dh_final, workspace};
+  for (const void* q : all)
+    if (q && !aligned16(q)) return M3_ERR_ALIGN;
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return M3_ERR_WORKSPACE;
+  if (dims->b * dims->H == 0) return M3_OK;
+  m3::Params p = make_params(dims, dims->L, x, dt, A, lam, B, C, theta, bias_B, bias_C, W_x, W_o, D,
+                             const_cast<m3_state*>(state0), nullptr);
+  p.status = status_word();
+  if (!p.status) return M3_ERR_CUDA;
+  const cudaError_t e = m3::launch_scan_bwd(p, dy, dh_final, gr->dx, gr->ddt, gr->dA, gr->dlam, gr->dB, gr->dC,
+                                            gr->dtheta, gr->dbias_B, gr->dbias_C, gr->dW_x, gr->dW_o, gr->dD,
+                                            gr->dh0, gr->dcarry_B, gr->dcarry_x, workspace, workspace_bytes,
+                                            (cudaStream_t)stream);
+  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
 m3_status m3_scan_summary_workspace_size(const m3_dims* dims, size_t* out_bytes) {
   m3_status st = check_dims(dims);
   if (st != M3_OK) return st;

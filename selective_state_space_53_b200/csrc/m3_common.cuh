@@ -132,6 +132,12 @@ cudaError_t launch_range_summary(const Params& p, void* ws, size_t ws_bytes, flo
                                  float* bp_first, float* carry_B, float* carry_x, cudaStream_t stream);
 cudaError_t launch_state_fold(const Params& p, int nranges, const float* Z, const float* logdec, const double* angle,
                               const float* bp_first, const float* carry_B, const float* carry_x, cudaStream_t stream);
+bool bwd_supported(const Params& p);
+size_t scan_bwd_workspace_bytes(const Params& p);
+cudaError_t launch_scan_bwd(const Params& p, const void* dy, const float* dh_final, void* dx, float* ddt, float* dA,
+                            float* dlam, void* dB, void* dC, float* dtheta, float* dbias_B, float* dbias_C,
+                            float* dW_x, float* dW_o, float* dD, float* dh0, float* dcarry_B, float* dcarry_x,
+                            void* ws, size_t ws_bytes, cudaStream_t stream);
 cudaError_t launch_selftest_wait(int* status, unsigned long long limit_ns, cudaStream_t stream);
 
 }  // namespace m3

@@ -54,6 +54,8 @@ SIGNATURES = {
     "m3_scan_fwd": (_I, [_DP] + [_VP] * 14 + [_VP, _SZ, _VP]),
     "m3_scan_fwd_noalloc": (_I, [_DP] + [_VP] * 14 + [_VP]),
     "m3_decode_step": (_I, [_DP] + [_VP] * 15),
+    "m3_scan_bwd_workspace_size": (_I, [_DP, ctypes.POINTER(_SZ)]),
+    "m3_scan_bwd": (_I, [_DP] + [_VP] * 12 + [_VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "m3_scan_summary_workspace_size": (_I, [_DP, ctypes.POINTER(_SZ)]),
     "m3_scan_summary": (_I, [_DP] + [_VP] * 14 + [_VP, _SZ, _VP]),
     "m3_state_fold": (_I, [_DP, ctypes.c_int32] + [_VP] * 8 + [_VP, _VP]),
@@ -213,6 +215,51 @@ def m3_state_fold(dims: Dims, nranges: int, Z, logdec, angle, bp_first, carry_B,
     _check(lib().m3_state_fold(ctypes.byref(dims), int(nranges), _ptr(Z), _ptr(logdec), _ptr(angle),
                                _ptr(bp_first), _ptr(carry_B), _ptr(carry_x), _ptr(bias_B), _ptr(W_x),
                                state.handle, _stream(stream)), "m3_state_fold")
+
+
+GRAD_KEYS = ("dx", "ddt", "dA", "dlam", "dB", "dC", "dtheta", "dbias_B", "dbias_C", "dW_x", "dW_o", "dD",
+             "dh0", "dcarry_B", "dcarry_x")
+
+
+class Grads(ctypes.Structure):
+    """m3_grads: device pointers of the gradients (None where not wanted)."""
+    _fields_ = [(k, ctypes.c_void_p) for k in GRAD_KEYS]
+
+
+def m3_scan_bwd_workspace_size(dims: Dims) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().m3_scan_bwd_workspace_size(ctypes.byref(dims), ctypes.byref(n)), "m3_scan_bwd_workspace_size")
+    return n.value
+
+
+def m3_scan_bwd(dims: Dims, x, dt, A, lam, B, C, theta, bias_B, bias_C, W_x, W_o, D, state0: State, dy,
+                dh_final, grads: dict, workspace=None, stream=None):
+    g = Grads(*[(None if grads.get(k) is None else grads[k].data_ptr()) for k in GRAD_KEYS])
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().m3_scan_bwd(ctypes.byref(dims), _ptr(x), _ptr(dt), _ptr(A), _ptr(lam), _ptr(B), _ptr(C),
+                             _ptr(theta), _ptr(bias_B), _ptr(bias_C), _ptr(W_x), _ptr(W_o), _ptr(D), state0.handle,
+                             _ptr(dy), _ptr(dh_final), ctypes.byref(g), _ptr(workspace), ws_bytes, _stream(stream)),
+           "m3_scan_bwd")
+
+
+def scan_backward(dims: Dims, dev: dict, state0: State, dy, dh_final=None, stream=None):
+    """m3_scan_bwd on a dict from ``to_device``: allocates the gradients (every one of them) and
+    the workspace; returns the gradients keyed by GRAD_KEYS."""
+    import torch
+    d = dev["x"].device
+    b, L, H, P, N, R, G = dims.b, dims.L, dims.H, dims.P, dims.N, dims.R, dims.G
+    f32 = dict(dtype=torch.float32, device=d)
+    out = {"dx": torch.empty_like(dev["x"]), "ddt": torch.empty((b, L, H), **f32), "dA": torch.empty((b, L, H), **f32),
+           "dlam": torch.empty((b, L, H), **f32), "dB": torch.empty_like(dev["B"]), "dC": torch.empty_like(dev["C"]),
+           "dtheta": torch.empty((b, L, G, N // 2), **f32), "dbias_B": torch.empty((H, R, N), **f32),
+           "dbias_C": torch.empty((H, R, N), **f32), "dW_x": torch.empty((H, R, P), **f32),
+           "dW_o": torch.empty((H, R, P), **f32), "dD": torch.empty((H,), **f32),
+           "dh0": torch.empty((b, H, N, P), **f32), "dcarry_B": torch.empty((b, H, R, N), **f32),
+           "dcarry_x": torch.empty((b, H, P), **f32)}
+    n = m3_scan_bwd_workspace_size(dims)
+    ws = torch.empty(max(n, 16), dtype=torch.uint8, device=d)
+    m3_scan_bwd(dims, *[dev[k] for k in _OPERANDS], state0, dy, dh_final, out, workspace=ws, stream=stream)
+    return out
 
 
 def m3_check(stream=None) -> int:

@@ -3,9 +3,10 @@
 A pin is only worth something if a plausible mistake in the oracle makes it fail.  Each
 case below plants one such mistake in a copy of oracle/m3_oracle.c (a wrong sign, a
 dropped term, a swapped coefficient, a wrong index), builds the copy in a temporary
-directory, and runs the whole pin suite (tests/test_oracle_pins.py) against it in a child
-process; the suite must fail.  The unmodified copy must pass, so that a failure means
-the planted mistake was caught and not that the harness is broken.
+directory, and runs the pin suites (tests/test_oracle_pins.py and the finite-difference pins of
+the backward pass, tests/test_oracle_grad.py) against it in a child process; they must fail.
+The unmodified copy must pass, so that a failure means the planted mistake was caught and not
+that the harness is broken.
 
 The mistakes follow the recurrence the oracle states (Mamba-3 paper note, docsaid.org:
 section その1 for the trapezoid coefficients and the previous-token term, その2 for the
@@ -21,9 +22,10 @@ import sys
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
+PINS = [os.path.join(ROOT, "tests", "test_oracle_pins.py"), os.path.join(ROOT, "tests", "test_oracle_grad.py")]
+BWD = "static int bwd_one("  # the backward pass follows the forward recurrence in the file
 
-# (name, text in m3_oracle.c, replacement); each text occurs exactly once
+# (name, text in m3_oracle.c, replacement); the first occurrence of the text is replaced
 MUTANTS = [
     ("rotation_sign", "h0[p] = alpha * (c * v0 - s * v1)", "h0[p] = alpha * (c * v0 + s * v1)"),
     ("beta_without_rotation",
@@ -51,6 +53,11 @@ MUTANTS = [
     ("angle_without_dt", "d->angle_direct ? th[k] : delta * th[k]", "d->angle_direct ? th[k] : th[k]"),
     ("decay_without_dt", "const double alpha = exp(delta * a);", "const double alpha = exp(a);"),
     ("skip_term_dropped", "yt[p] = s + dh * xt[p];", "yt[p] = s;"),
+    # the backward pass (pinned by the finite-difference tests)
+    ("bwd_rotation_transpose", "dz[i0] = c * dm0 + s * dm1;", "dz[i0] = c * dm0 - s * dm1;"),
+    ("bwd_previous_input_dropped", "duN[i] = bprime * dz[i];", "duN[i] = 0.0 * dz[i];"),
+    ("bwd_lambda_beta_term_dropped", "gr->dlam[tok * H + hi] += (dgamma - dbp) * delta;",
+     "gr->dlam[tok * H + hi] += dgamma * delta;"),
 ]
 
 
@@ -64,7 +71,7 @@ def _run_pins(tmp_path, name, src_text):
     env = dict(os.environ)
     # the copy comes first on the path; the repository root provides everything else
     env["PYTHONPATH"] = os.pathsep.join([str(work), ROOT])
-    cmd = [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider", PINS]
+    cmd = [sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider", *PINS]
     return subprocess.run(cmd, cwd=str(work), env=env, capture_output=True, text=True, timeout=600)
 
 
@@ -81,6 +88,10 @@ def test_unmodified_copy_passes_the_pins(tmp_path, source):
 
 @pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
 def test_planted_mistake_fails_a_pin(tmp_path, source, name, old, new):
-    assert source.count(old) == 1, f"mutation site of {name} not found exactly once"
-    r = _run_pins(tmp_path, name, source.replace(old, new))
+    # a forward mistake is planted in the forward recurrence (the first occurrence, before the
+    # backward pass, which restates some of its lines); a backward one in the backward pass
+    at = source.find(old)
+    assert at >= 0, f"mutation site of {name} not found"
+    assert (at > source.find(BWD)) == name.startswith("bwd_"), f"mutation site of {name} in the wrong pass"
+    r = _run_pins(tmp_path, name, source[:at] + new + source[at + len(old):])
     assert r.returncode == 1, f"{name}: the pins did not catch it\n" + r.stdout[-2000:]
