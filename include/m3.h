@@ -69,9 +69,12 @@ enum { M3_F32 = 0, M3_BF16 = 1 };
 enum {
   M3_FLAG_SEQUENTIAL = 1u,   /* run the token-sequential SIMT scan even where the chunked
                                 tensor-core scan applies (diagnostic / cross-check) */
-  M3_FLAG_ANGLE_DIRECT = 2u  /* variant: theta is the rotation angle of the step itself,
+  M3_FLAG_ANGLE_DIRECT = 2u, /* variant: theta is the rotation angle of the step itself,
                                 phi_t = theta_t instead of dt_t * theta_t (the rotation
                                 then no longer depends on the head's step size) */
+  M3_FLAG_RAW_INPUTS = 4u    /* m3_scan_fwd: B, C, dt, A, lam are the block's raw projections;
+                                the core applies the front-end of m3_frontend to them itself
+                                (the workspace then also holds the transformed operands) */
 };
 
 typedef struct {
@@ -256,6 +259,30 @@ m3_status m3_decode_step(const m3_dims* dims, const void* x_t, const float* dt_t
                          const void* C_t, const float* theta_t, const float* bias_B,
                          const float* bias_C, const float* W_x, const float* W_o,
                          const float* D, m3_state* state, void* y_t, void* stream);
+
+/* ---- the block's front-end -------------------------------------------------------- */
+
+/* The block's front-end on raw projections: B and C RMS-normalised over N per (token, group,
+ * branch) row, B = B_raw / sqrt(mean_N B_raw^2 + 1e-6) (no weight; the biases are added later
+ * by the core), dt = softplus(dt_raw), A = -exp(A_raw), lam = sigmoid(lam_raw) -- the B/C norm
+ * of the Cartesia blog "Mamba-3" and the docsaid note (section アーキテクチャ) and the
+ * parameterisation of the discretisation of section その1.  Raw and transformed tensors in the
+ * layouts of m3_scan_fwd (B, C in dims->dtype; the others fp32); outputs may be the inputs.
+ * m3_decode_step takes transformed operands: run this on the token first.  Asynchronous. */
+m3_status m3_frontend(const m3_dims* dims, const void* B_raw, const void* C_raw, const float* dt_raw,
+                      const float* A_raw, const float* lam_raw, void* B, void* C, float* dt, float* A,
+                      float* lam, void* stream);
+
+/* ---- the hybrid model's output norm ---------------------------------------------- */
+
+/* The norm before the output projection that the Mamba-3 paper note (section アーキテクチャ)
+ * removes in the pure Mamba-3 model and keeps in the hybrid one, with the block's gate z
+ * applied first when given.  Per (batch, token, head) row of P values:
+ *   v = y * silu(z)  (v = y when z is NULL),   out = weight[h] * v / sqrt(mean_p v^2 + eps).
+ * y, z, out: (b, L, H, P) in dims->dtype (out may be y); weight: (H, P) fp32 or NULL (ones);
+ * eps >= 0 (M3_ERR_DIMS otherwise).  Asynchronous on `stream`. */
+m3_status m3_output_norm(const m3_dims* dims, const void* y, const void* z, const float* weight,
+                         float eps, void* out, void* stream);
 
 /* ---- status -------------------------------------------------------------- */
 

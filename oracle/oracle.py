@@ -146,3 +146,44 @@ def scan_bwd(dims, x, dt, A, lam, B, C, theta, bias_B=None, bias_C=None, W_x=Non
         if a is None:
             out[k] = None
     return out
+
+
+def output_norm(y, z=None, weight=None, eps=1e-6):
+    """The hybrid model's output norm (test infrastructure), in float64: per (batch, token,
+    head) row of P values, v = y * silu(z) (v = y without a gate), then
+    out = weight[h] * v / sqrt(mean_p v^2 + eps).  y, z: (b, L, H, P); weight: (H, P) or None
+    (ones).  Mamba-3 paper note (docsaid.org), section アーキテクチャ: the norm before the output
+    projection is removed in the pure Mamba-3 model and kept in the hybrid one."""
+    v = np.asarray(y, dtype=np.float64)
+    if z is not None:
+        zz = np.asarray(z, dtype=np.float64)
+        v = v * (zz / (1.0 + np.exp(-zz)))
+    rms = np.sqrt(np.mean(v * v, axis=-1, keepdims=True) + eps)
+    out = v / rms
+    if weight is not None:
+        out = out * np.asarray(weight, dtype=np.float64)[None, None]
+    return out
+
+
+BCNORM_EPS = 1e-6
+
+
+def frontend(inp):
+    """The block's front-end on a raw draw (test infrastructure), in float64: a copy of the
+    draw whose B, C are RMS-normalised over N per (token, group, branch) row (B / sqrt(mean_N
+    B^2 + 1e-6), no weight: the QK-norm-like BCNorm of the Cartesia blog and the docsaid note,
+    section アーキテクチャ), dt = softplus(dt_raw), A = -exp(A_raw) and lam = sigmoid(lam_raw)
+    (the parameterisation of the step, decay and trapezoid weight in section その1's
+    discretisation).  The biases are added by the core after the norm."""
+    import copy
+    out = copy.copy(inp)
+    B = np.asarray(inp.B, dtype=np.float64)
+    C = np.asarray(inp.C, dtype=np.float64)
+    out.B = B / np.sqrt(np.mean(B * B, axis=-1, keepdims=True) + BCNORM_EPS)
+    out.C = C / np.sqrt(np.mean(C * C, axis=-1, keepdims=True) + BCNORM_EPS)
+    d = np.asarray(inp.dt, dtype=np.float64)
+    out.dt = np.logaddexp(0.0, d)
+    out.A = -np.exp(np.asarray(inp.A, dtype=np.float64))
+    out.lam = 1.0 / (1.0 + np.exp(-np.asarray(inp.lam, dtype=np.float64)))
+    out.extra = dict(inp.extra, raw=False)
+    return out

@@ -48,7 +48,7 @@ m3_status check_dims(const m3_dims* d) {
   if (d->N < 8 || d->N > 256 || (d->N % 8) != 0) return M3_ERR_DIMS;
   if ((d->H % d->G) != 0) return M3_ERR_DIMS;
   if (d->chunk < 0) return M3_ERR_DIMS;
-  if (d->flags & ~(uint32_t)(M3_FLAG_SEQUENTIAL | M3_FLAG_ANGLE_DIRECT)) return M3_ERR_DIMS;
+  if (d->flags & ~(uint32_t)(M3_FLAG_SEQUENTIAL | M3_FLAG_ANGLE_DIRECT | M3_FLAG_RAW_INPUTS)) return M3_ERR_DIMS;
   if (d->dtype != M3_F32 && d->dtype != M3_BF16) return M3_ERR_DTYPE;
   if (d->b * (int64_t)d->H > (int64_t)0x7fffffff) return M3_ERR_DIMS;
   if (!m3::seq_scan_supported(d->P, d->N, d->R)) return M3_ERR_UNSUPPORTED;
@@ -117,6 +117,28 @@ m3::Params make_params(const m3_dims* d, int64_t L, const void* x, const float* 
   p.y = y;
   p.status = nullptr;
   return p;
+}
+
+// Bytes of the scan's own scratch and, with M3_FLAG_RAW_INPUTS, where the transformed operands
+// start in the workspace (after the scan's scratch, 256-byte aligned) and how many bytes they take.
+struct WsLayout {
+  size_t scan, fe_off, fe_bytes;
+};
+
+WsLayout ws_layout(const m3_dims* dims) {
+  WsLayout w{0, 0, 0};
+  if (dims->b * dims->L == 0) return w;
+  m3::Params p = make_params(dims, dims->L, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                             nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+  if (!(dims->flags & M3_FLAG_SEQUENTIAL) && m3::tc_scan_supported(p)) w.scan = m3::tc_scan_workspace_bytes(p);
+  if (dims->flags & M3_FLAG_RAW_INPUTS) {
+    const size_t e = dims->dtype == M3_BF16 ? 2 : 4;
+    const size_t nbc = (size_t)(dims->b * dims->L) * dims->G * dims->R * dims->N;
+    const size_t nsc = (size_t)(dims->b * dims->L) * dims->H;
+    w.fe_off = (w.scan + 255) & ~(size_t)255;
+    w.fe_bytes = 2 * ((nbc * e + 255) & ~(size_t)255) + 3 * ((nsc * 4 + 255) & ~(size_t)255);
+  }
+  return w;
 }
 
 }  // namespace
@@ -230,15 +252,13 @@ m3_status m3_state_copy_from_host(m3_state* state, const void* src, size_t nbyte
   return M3_OK;
 }
 
+
 m3_status m3_scan_workspace_size(const m3_dims* dims, size_t* out_bytes) {
   m3_status st = check_dims(dims);
   if (st != M3_OK) return st;
   if (!out_bytes) return M3_ERR_NULL;
-  *out_bytes = 0;
-  if (dims->b * dims->L == 0) return M3_OK;
-  m3::Params p = make_params(dims, dims->L, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
-                             nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
-  if (!(dims->flags & M3_FLAG_SEQUENTIAL) && m3::tc_scan_supported(p)) *out_bytes = m3::tc_scan_workspace_bytes(p);
+  const WsLayout w = ws_layout(dims);
+  *out_bytes = w.fe_bytes ? w.fe_off + w.fe_bytes : w.scan;
   return M3_OK;
 }
 
@@ -257,15 +277,32 @@ m3_status m3_scan_fwd(const m3_dims* dims, const void* x, const float* dt, const
   m3::Params p = make_params(dims, dims->L, x, dt, A, lam, B, C, theta, bias_B, bias_C, W_x, W_o,
                              D, state, y);
   const bool tc = !(dims->flags & M3_FLAG_SEQUENTIAL) && m3::tc_scan_supported(p);
-  if (tc) {
-    const size_t need = m3::tc_scan_workspace_bytes(p);
-    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return M3_ERR_WORKSPACE;
-    if (need > 0 && !aligned16(workspace)) return M3_ERR_ALIGN;
-  }
+  const WsLayout w = ws_layout(dims);
+  const size_t need = w.fe_bytes ? w.fe_off + w.fe_bytes : w.scan;
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return M3_ERR_WORKSPACE;
+  if (need > 0 && !aligned16(workspace)) return M3_ERR_ALIGN;
   p.status = status_word();
   if (!p.status) return M3_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;
-  const cudaError_t e = tc ? m3::launch_scan_tc(p, workspace, workspace_bytes, s) : m3::launch_scan_sequential(p, s);
+  if (dims->flags & M3_FLAG_RAW_INPUTS) {
+    // the front-end writes the transformed operands into the workspace after the scan's scratch
+    char* fe = static_cast<char*>(workspace) + w.fe_off;
+    const size_t e = dims->dtype == M3_BF16 ? 2 : 4;
+    const size_t bc = ((size_t)(dims->b * dims->L) * dims->G * dims->R * dims->N * e + 255) & ~(size_t)255;
+    const size_t sc = ((size_t)(dims->b * dims->L) * dims->H * 4 + 255) & ~(size_t)255;
+    void* tB = fe;
+    void* tC = fe + bc;
+    float* tdt = reinterpret_cast<float*>(fe + 2 * bc);
+    float* tA = reinterpret_cast<float*>(fe + 2 * bc + sc);
+    float* tlam = reinterpret_cast<float*>(fe + 2 * bc + 2 * sc);
+    if (m3::launch_frontend(p, B, C, dt, A, lam, tB, tC, tdt, tA, tlam, s) != cudaSuccess) return M3_ERR_CUDA;
+    p.B = tB;
+    p.C = tC;
+    p.dt = tdt;
+    p.A = tA;
+    p.lam = tlam;
+  }
+  const cudaError_t e = tc ? m3::launch_scan_tc(p, workspace, w.scan, s) : m3::launch_scan_sequential(p, s);
   return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
 }
 
@@ -276,6 +313,7 @@ m3_status m3_decode_step(const m3_dims* dims, const void* x_t, const float* dt_t
                          const float* D, m3_state* state, void* y_t, void* stream) {
   m3_status st = check_dims(dims);
   if (st != M3_OK) return st;
+  if (dims->flags & M3_FLAG_RAW_INPUTS) return M3_ERR_UNSUPPORTED;  // m3_frontend on the token first
   const bool tokens = dims->b > 0;
   st = check_operands(dims, x_t, dt_t, A_t, lam_t, B_t, C_t, theta_t, bias_B, bias_C, W_x, W_o, D,
                       state, y_t, tokens);
@@ -310,7 +348,8 @@ m3_status m3_scan_bwd(const m3_dims* dims, const void* x, const float* dt, const
   m3_status st = m3_scan_bwd_workspace_size(dims, &need);
   if (st != M3_OK) return st;
   if (!gr) return M3_ERR_NULL;
-  if (dims->L < 1) return M3_ERR_DIMS;  // the backward pass of an empty scan is not defined here
+  if (dims->L < 1) return M3_ERR_DIMS;
+  if (dims->flags & M3_FLAG_RAW_INPUTS) return M3_ERR_UNSUPPORTED;  // the backward pass of an empty scan is not defined here
   const bool tokens = dims->b * dims->L > 0;
   st = check_operands(dims, x, dt, A, lam, B, C, theta, bias_B, bias_C, W_x, W_o, D, state0, dy, tokens);
   if (st != M3_OK) return st;
@@ -340,6 +379,7 @@ m3_status m3_scan_summary_workspace_size(const m3_dims* dims, size_t* out_bytes)
   if (st != M3_OK) return st;
   if (!out_bytes) return M3_ERR_NULL;
   if (dims->L < 1) return M3_ERR_DIMS;
+  if (dims->flags & M3_FLAG_RAW_INPUTS) return M3_ERR_UNSUPPORTED;
   m3::Params p = make_params(dims, dims->L, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                              nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
   if (!m3::tc_scan_supported(p)) return M3_ERR_UNSUPPORTED;
@@ -394,6 +434,41 @@ m3_status m3_state_fold(const m3_dims* dims, int32_t nranges, const float* Z, co
                              W_x, nullptr, nullptr, state, nullptr);
   const cudaError_t e = m3::launch_state_fold(p, nranges, Z, logdec, angle, bp_first, carry_B, carry_x,
                                               (cudaStream_t)stream);
+  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
+m3_status m3_frontend(const m3_dims* dims, const void* B_raw, const void* C_raw, const float* dt_raw,
+                      const float* A_raw, const float* lam_raw, void* B, void* C, float* dt, float* A, float* lam,
+                      void* stream) {
+  m3_status st = check_dims(dims);
+  if (st != M3_OK) return st;
+  if (dims->b * dims->L == 0) return M3_OK;
+  const void* req[] = {B_raw, C_raw, dt_raw, A_raw, lam_raw, B, C, dt, A, lam};
+  for (const void* q : req) {
+    if (!q) return M3_ERR_NULL;
+    if (!aligned16(q)) return M3_ERR_ALIGN;
+  }
+  m3::Params p = make_params(dims, dims->L, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                             nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+  const cudaError_t e = m3::launch_frontend(p, B_raw, C_raw, dt_raw, A_raw, lam_raw, B, C, dt, A, lam,
+                                            (cudaStream_t)stream);
+  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+}
+
+m3_status m3_output_norm(const m3_dims* dims, const void* y, const void* z, const float* weight, float eps,
+                         void* out, void* stream) {
+  m3_status st = check_dims(dims);
+  if (st != M3_OK) return st;
+  if (!(eps >= 0.0f)) return M3_ERR_DIMS;
+  const bool rows = dims->b * dims->L * dims->H > 0;
+  if (rows && (!y || !out)) return M3_ERR_NULL;
+  const void* all[] = {y, z, weight, out};
+  for (const void* q : all)
+    if (q && !aligned16(q)) return M3_ERR_ALIGN;
+  if (!rows) return M3_OK;
+  m3::Params p = make_params(dims, dims->L, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                             nullptr, nullptr, nullptr, nullptr, nullptr, const_cast<void*>(y));
+  const cudaError_t e = m3::launch_output_norm(p, z, weight, eps, out, (cudaStream_t)stream);
   return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
 }
 

@@ -138,6 +138,11 @@ cudaError_t launch_scan_bwd(const Params& p, const void* dy, const float* dh_fin
                             float* dlam, void* dB, void* dC, float* dtheta, float* dbias_B, float* dbias_C,
                             float* dW_x, float* dW_o, float* dD, float* dh0, float* dcarry_B, float* dcarry_x,
                             void* ws, size_t ws_bytes, cudaStream_t stream);
+cudaError_t launch_output_norm(const Params& p, const void* z, const float* weight, float eps, void* out,
+                               cudaStream_t stream);
+cudaError_t launch_frontend(const Params& p, const void* Braw, const void* Craw, const float* dt_raw,
+                            const float* A_raw, const float* lam_raw, void* B, void* C, float* dt, float* A,
+                            float* lam, cudaStream_t stream);
 cudaError_t launch_selftest_wait(int* status, unsigned long long limit_ns, cudaStream_t stream);
 
 }  // namespace m3

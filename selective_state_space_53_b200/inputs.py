@@ -155,6 +155,39 @@ def make_inputs(b, L, H, P, N, R, G=1, dtype="bf16", seed=0, *, extras=False,
     return Inputs(dims, x, dt, A, lam, theta, B, C, bias_B, bias_C, W_x, W_o, D, seed=seed)
 
 
+def make_raw_inputs(b, L, H, P, N, R, G=1, dtype="bf16", seed=0, *, extras=False, bias=0.02) -> Inputs:
+    """Draw the layer's raw projections (for M3_FLAG_RAW_INPUTS, where the core applies the
+    front-end itself): dt_raw ~ N(-2, 0.5), A_raw ~ U(0, 1), lam_raw ~ N(0, 1) (the arguments of
+    softplus, -exp and sigmoid in the recipe above), and B_raw, C_raw ~ N(0, 1) scaled per
+    (token, group, branch) row by U(0.25, 4) so that the row norms vary, cast to the storage
+    dtype.  x, theta, biases and weights as in make_inputs.  The returned draw holds the raw
+    values in dt, A, lam, B, C and extra["raw"] = True."""
+    if N % 2:
+        raise ValueError("d_state N must be even (complex pairs)")
+    rng = np.random.default_rng(seed)
+    x = _normal(rng, (b, L, H, P), dtype)
+    dt = (-2.0 + 0.5 * rng.standard_normal((b, L, H))).astype(np.float32)
+    A = rng.uniform(0.0, 1.0, (b, L, H)).astype(np.float32)
+    lam = rng.standard_normal((b, L, H)).astype(np.float32)
+    theta = rng.uniform(-math.pi, math.pi, (b, L, G, N // 2)).astype(np.float32)
+    Bs = rng.uniform(0.25, 4.0, (b, L, G, R, 1))
+    B = _cast(Bs * rng.standard_normal((b, L, G, R, N)), dtype)
+    Cs = rng.uniform(0.25, 4.0, (b, L, G, R, 1))
+    C = _cast(Cs * rng.standard_normal((b, L, G, R, N)), dtype)
+    W_x = (1.0 + 0.1 * rng.standard_normal((H, R, P))).astype(np.float32)
+    W_o = ((1.0 + 0.1 * rng.standard_normal((H, R, P))) / R).astype(np.float32)
+    if extras:
+        bias_B = (bias + 0.1 * rng.standard_normal((H, R, N))).astype(np.float32)
+        bias_C = (bias + 0.1 * rng.standard_normal((H, R, N))).astype(np.float32)
+        D = rng.standard_normal(H).astype(np.float32)
+    else:
+        bias_B = np.full((H, R, N), bias, dtype=np.float32)
+        bias_C = np.full((H, R, N), bias, dtype=np.float32)
+        D = None
+    dims = dict(b=b, L=L, H=H, P=P, N=N, R=R, G=G, dtype=dtype)
+    return Inputs(dims, x, dt, A, lam, theta, B, C, bias_B, bias_C, W_x, W_o, D, seed=seed, extra={"raw": True})
+
+
 def make_state(b, H, P, N, R, seed, scale=1.0):
     """A seeded non-zero initial state (h, carry_B, carry_x) for continuation tests."""
     rng = np.random.default_rng(seed)

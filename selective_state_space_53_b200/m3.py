@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libm3.so")
 M3_F32, M3_BF16 = 0, 1
 M3_FLAG_SEQUENTIAL = 1
 M3_FLAG_ANGLE_DIRECT = 2
+M3_FLAG_RAW_INPUTS = 4
 
 _STATUS = {0: "M3_OK", -1: "M3_ERR_DIMS", -2: "M3_ERR_DTYPE", -3: "M3_ERR_ALIGN",
            -4: "M3_ERR_NULL", -5: "M3_ERR_WORKSPACE", -6: "M3_ERR_CUDA", -7: "M3_ERR_TIMEOUT",
@@ -54,6 +55,8 @@ SIGNATURES = {
     "m3_scan_fwd": (_I, [_DP] + [_VP] * 14 + [_VP, _SZ, _VP]),
     "m3_scan_fwd_noalloc": (_I, [_DP] + [_VP] * 14 + [_VP]),
     "m3_decode_step": (_I, [_DP] + [_VP] * 15),
+    "m3_output_norm": (_I, [_DP, _VP, _VP, _VP, ctypes.c_float, _VP, _VP]),
+    "m3_frontend": (_I, [_DP] + [_VP] * 10 + [_VP]),
     "m3_scan_bwd_workspace_size": (_I, [_DP, ctypes.POINTER(_SZ)]),
     "m3_scan_bwd": (_I, [_DP] + [_VP] * 12 + [_VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "m3_scan_summary_workspace_size": (_I, [_DP, ctypes.POINTER(_SZ)]),
@@ -215,6 +218,16 @@ def m3_state_fold(dims: Dims, nranges: int, Z, logdec, angle, bp_first, carry_B,
     _check(lib().m3_state_fold(ctypes.byref(dims), int(nranges), _ptr(Z), _ptr(logdec), _ptr(angle),
                                _ptr(bp_first), _ptr(carry_B), _ptr(carry_x), _ptr(bias_B), _ptr(W_x),
                                state.handle, _stream(stream)), "m3_state_fold")
+
+
+def m3_frontend(dims: Dims, B_raw, C_raw, dt_raw, A_raw, lam_raw, B, C, dt, A, lam, stream=None):
+    _check(lib().m3_frontend(ctypes.byref(dims), _ptr(B_raw), _ptr(C_raw), _ptr(dt_raw), _ptr(A_raw), _ptr(lam_raw),
+                             _ptr(B), _ptr(C), _ptr(dt), _ptr(A), _ptr(lam), _stream(stream)), "m3_frontend")
+
+
+def m3_output_norm(dims: Dims, y, z, weight, eps, out, stream=None):
+    _check(lib().m3_output_norm(ctypes.byref(dims), _ptr(y), _ptr(z), _ptr(weight), float(eps), _ptr(out),
+                                _stream(stream)), "m3_output_norm")
 
 
 GRAD_KEYS = ("dx", "ddt", "dA", "dlam", "dB", "dC", "dtheta", "dbias_B", "dbias_C", "dW_x", "dW_o", "dD",

@@ -47,7 +47,7 @@ def _dims(**kw):
 
 @pytest.mark.parametrize("kw,code", [
     (dict(N=15), -1), (dict(N=12), -1), (dict(P=12), -1), (dict(G=3), -1), (dict(R=0), -1),
-    (dict(R=9), -1), (dict(P=512), -1), (dict(b=-1), -1), (dict(dtype=7), -2), (dict(flags=4), -1)])
+    (dict(R=9), -1), (dict(P=512), -1), (dict(b=-1), -1), (dict(dtype=7), -2), (dict(flags=8), -1)])
 def test_bad_dims_rejected_on_host(L, kw, code):
     d = _dims(**kw)
     n = ctypes.c_size_t()
