@@ -301,6 +301,10 @@ m3_status m3_selftest_wait(uint64_t limit_ns, void* stream);
 /* Static description of a status code. */
 const char* m3_status_str(m3_status status);
 
+/* Text of the last CUDA runtime error behind an M3_ERR_CUDA returned to this host thread
+ * ("no CUDA error" if there was none).  The string is static. */
+const char* m3_last_error(void);
+
 /* Library version string. */
 const char* m3_version(void);
 

@@ -41,6 +41,15 @@ namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The last CUDA error a call of this host thread met (m3_last_error reports it).
+thread_local cudaError_t g_last_cuda = cudaSuccess;
+
+m3_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return M3_OK;
+  g_last_cuda = e;
+  return M3_ERR_CUDA;
+}
+
 m3_status check_dims(const m3_dims* d) {
   if (!d) return M3_ERR_NULL;
   if (d->b < 0 || d->L < 0 || d->H < 1 || d->G < 1 || d->R < 1 || d->R > 8) return M3_ERR_DIMS;
@@ -99,6 +108,7 @@ m3::Params make_params(const m3_dims* d, int64_t L, const void* x, const float* 
   p.G = d->G;
   p.dtype = d->dtype;
   p.angle_direct = (d->flags & M3_FLAG_ANGLE_DIRECT) ? 1 : 0;
+  p.raw_inputs = (d->flags & M3_FLAG_RAW_INPUTS) ? 1 : 0;
   p.x = x;
   p.dt = dt;
   p.A = A;
@@ -119,6 +129,15 @@ m3::Params make_params(const m3_dims* d, int64_t L, const void* x, const float* 
   return p;
 }
 
+// Raw inputs go through the warp-specialised scan's load stage directly (the front-end fused);
+// every other kernel gets them transformed by m3_frontend into the workspace first.
+bool fused_frontend(const m3_dims* dims) {
+  if (!(dims->flags & M3_FLAG_RAW_INPUTS) || (dims->flags & M3_FLAG_SEQUENTIAL)) return false;
+  m3::Params p = make_params(dims, dims->L, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                             nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+  return m3::tc_scan_supported(p) && m3::ws_scan_supported(p);
+}
+
 // Bytes of the scan's own scratch and, with M3_FLAG_RAW_INPUTS, where the transformed operands
 // start in the workspace (after the scan's scratch, 256-byte aligned) and how many bytes they take.
 struct WsLayout {
@@ -131,7 +150,7 @@ WsLayout ws_layout(const m3_dims* dims) {
   m3::Params p = make_params(dims, dims->L, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                              nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
   if (!(dims->flags & M3_FLAG_SEQUENTIAL) && m3::tc_scan_supported(p)) w.scan = m3::tc_scan_workspace_bytes(p);
-  if (dims->flags & M3_FLAG_RAW_INPUTS) {
+  if ((dims->flags & M3_FLAG_RAW_INPUTS) && !fused_frontend(dims)) {
     const size_t e = dims->dtype == M3_BF16 ? 2 : 4;
     const size_t nbc = (size_t)(dims->b * dims->L) * dims->G * dims->R * dims->N;
     const size_t nsc = (size_t)(dims->b * dims->L) * dims->H;
@@ -284,7 +303,7 @@ m3_status m3_scan_fwd(const m3_dims* dims, const void* x, const float* dt, const
   p.status = status_word();
   if (!p.status) return M3_ERR_CUDA;
   cudaStream_t s = (cudaStream_t)stream;
-  if (dims->flags & M3_FLAG_RAW_INPUTS) {
+  if (w.fe_bytes) {
     // the front-end writes the transformed operands into the workspace after the scan's scratch
     char* fe = static_cast<char*>(workspace) + w.fe_off;
     const size_t e = dims->dtype == M3_BF16 ? 2 : 4;
@@ -301,9 +320,10 @@ m3_status m3_scan_fwd(const m3_dims* dims, const void* x, const float* dt, const
     p.dt = tdt;
     p.A = tA;
     p.lam = tlam;
+    p.raw_inputs = 0;
   }
   const cudaError_t e = tc ? m3::launch_scan_tc(p, workspace, w.scan, s) : m3::launch_scan_sequential(p, s);
-  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+  return cuda_status(e);
 }
 
 m3_status m3_decode_step(const m3_dims* dims, const void* x_t, const float* dt_t,
@@ -325,7 +345,7 @@ m3_status m3_decode_step(const m3_dims* dims, const void* x_t, const float* dt_t
   if (!p.status) return M3_ERR_CUDA;
   const cudaError_t e = m3::decode_supported(p) ? m3::launch_decode(p, (cudaStream_t)stream)
                                                 : m3::launch_scan_sequential(p, (cudaStream_t)stream);
-  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+  return cuda_status(e);
 }
 
 m3_status m3_scan_bwd_workspace_size(const m3_dims* dims, size_t* out_bytes) {
@@ -371,7 +391,7 @@ m3_status m3_scan_bwd(const m3_dims* dims, const void* x, const float* dt, const
                                             gr->dtheta, gr->dbias_B, gr->dbias_C, gr->dW_x, gr->dW_o, gr->dD,
                                             gr->dh0, gr->dcarry_B, gr->dcarry_x, workspace, workspace_bytes,
                                             (cudaStream_t)stream);
-  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+  return cuda_status(e);
 }
 
 m3_status m3_scan_summary_workspace_size(const m3_dims* dims, size_t* out_bytes) {
@@ -409,7 +429,7 @@ m3_status m3_scan_summary(const m3_dims* dims, const void* x, const float* dt, c
   if (!p.status) return M3_ERR_CUDA;
   const cudaError_t e = m3::launch_range_summary(p, workspace, workspace_bytes, Z, logdec, angle, bp_first, carry_B,
                                                  carry_x, (cudaStream_t)stream);
-  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+  return cuda_status(e);
 }
 
 m3_status m3_state_fold(const m3_dims* dims, int32_t nranges, const float* Z, const float* logdec,
@@ -434,7 +454,7 @@ m3_status m3_state_fold(const m3_dims* dims, int32_t nranges, const float* Z, co
                              W_x, nullptr, nullptr, state, nullptr);
   const cudaError_t e = m3::launch_state_fold(p, nranges, Z, logdec, angle, bp_first, carry_B, carry_x,
                                               (cudaStream_t)stream);
-  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+  return cuda_status(e);
 }
 
 m3_status m3_frontend(const m3_dims* dims, const void* B_raw, const void* C_raw, const float* dt_raw,
@@ -452,7 +472,7 @@ m3_status m3_frontend(const m3_dims* dims, const void* B_raw, const void* C_raw,
                              nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
   const cudaError_t e = m3::launch_frontend(p, B_raw, C_raw, dt_raw, A_raw, lam_raw, B, C, dt, A, lam,
                                             (cudaStream_t)stream);
-  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+  return cuda_status(e);
 }
 
 m3_status m3_output_norm(const m3_dims* dims, const void* y, const void* z, const float* weight, float eps,
@@ -469,15 +489,14 @@ m3_status m3_output_norm(const m3_dims* dims, const void* y, const void* z, cons
   m3::Params p = make_params(dims, dims->L, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                              nullptr, nullptr, nullptr, nullptr, nullptr, const_cast<void*>(y));
   const cudaError_t e = m3::launch_output_norm(p, z, weight, eps, out, (cudaStream_t)stream);
-  return e == cudaSuccess ? M3_OK : M3_ERR_CUDA;
+  return cuda_status(e);
 }
 
 m3_status m3_selftest_wait(uint64_t limit_ns, void* stream) {
   if (limit_ns > 10000000000ull) return M3_ERR_DIMS;
   int* st = status_word();
   if (!st) return M3_ERR_CUDA;
-  return m3::launch_selftest_wait(st, (unsigned long long)limit_ns, (cudaStream_t)stream) == cudaSuccess ? M3_OK
-                                                                                                   : M3_ERR_CUDA;
+  return cuda_status(m3::launch_selftest_wait(st, (unsigned long long)limit_ns, (cudaStream_t)stream));
 }
 
 m3_status m3_check(void* stream) {
@@ -506,6 +525,8 @@ const char* m3_status_str(m3_status status) {
   }
   return "unknown status";
 }
+
+const char* m3_last_error(void) { return g_last_cuda == cudaSuccess ? "no CUDA error" : cudaGetErrorString(g_last_cuda); }
 
 const char* m3_version(void) { return "m3 0.1 (sm_100a)"; }
 

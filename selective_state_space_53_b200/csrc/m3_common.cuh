@@ -18,6 +18,7 @@ struct Params {
   int H, P, N, R, G;
   int dtype;  // M3_BF16 / M3_F32 for x, B, C, y
   int angle_direct;  // 1: the step's rotation angle is theta itself (M3_FLAG_ANGLE_DIRECT)
+  int raw_inputs;    // 1: B, C, dt, A, lam are raw projections, transformed in the load stage
   const void* x;
   const float* dt;
   const float* A;
@@ -36,6 +37,13 @@ struct Params {
   void* y;
   int* status;          // device status word (M3_OK / M3_ERR_TIMEOUT)
 };
+
+// The block's front-end on raw projections (m3_frontend): the activations of the step, the
+// decay and the trapezoid weight, and the eps of the B/C RMS norm.
+constexpr float kBcNormEps = 1e-6f;
+__device__ __forceinline__ float fe_softplus(float v) { return v > 20.0f ? v : log1pf(__expf(v)); }
+__device__ __forceinline__ float fe_negexp(float v) { return -__expf(v); }
+__device__ __forceinline__ float fe_sigmoid(float v) { return 1.0f / (1.0f + __expf(-v)); }
 
 // Record a failure in the device status word (first failure wins).
 __device__ __forceinline__ void set_status(int* word, int s) { atomicCAS(word, 0, s); }
@@ -123,6 +131,7 @@ cudaError_t launch_decode(const Params& p, cudaStream_t stream);
 bool decode_tc_supported(const Params& p);                    // tensor-core form (d_state = headdim = 128, bf16)
 cudaError_t launch_decode_tc(const Params& p, cudaStream_t stream);
 bool tc_scan_supported(const Params& p);
+bool ws_scan_supported(const Params& p);  // the warp-specialised kernel (headdim 128) takes these dims
 size_t tc_scan_workspace_bytes(const Params& p);  // scratch the chunked scan needs (0: none)
 cudaError_t launch_scan_tc(const Params& p, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 struct SegInfo;

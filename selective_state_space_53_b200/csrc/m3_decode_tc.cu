@@ -26,6 +26,26 @@
 namespace m3 {
 namespace {
 
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Launch with programmatic stream serialisation (the kernels call griddepcontrol.wait before any
+// global access).
+template <typename Kernel, typename... Args>
+cudaError_t launch_pdl(Kernel k, unsigned grid, unsigned block, size_t smem, cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, args...);
+}
+
 constexpr int kCT = 512;         // compute threads (16 warps)
 constexpr int kT = kCT + 32;     // + one producer warp
 constexpr int kN = 128;          // d_state
@@ -229,6 +249,10 @@ __global__ void __launch_bounds__(kT, 1) decode_tc_kernel(Params p, TcPlan tp) {
     return true;
   };
 
+  // Programmatic dependent launch: the next decode step may start its set-up (tensor memory,
+  // barriers) while this one runs; every global access of a step comes after its griddepcontrol.wait,
+  // which returns once the previous kernel of the stream has finished and its writes are visible.
+  griddep_launch_dependents();
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(kTmemCols));
@@ -246,6 +270,7 @@ __global__ void __launch_bounds__(kT, 1) decode_tc_kernel(Params p, TcPlan tp) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();
 
   if (warp == kCT / 32) {
     // ---- producer: the state and token operands of unit j into stage j % 2, once the compute
@@ -547,7 +572,8 @@ cudaError_t launch_tc_rt(const Params& p, const TcPlan& tp, unsigned grid, cudaS
   auto k = decode_tc_kernel<RT>;
   cudaError_t e = smem_set.ensure(k, (int)tp.total);
   if (e != cudaSuccess) return e;
-  k<<<grid, kT, tp.total, stream>>>(p, tp);
+  e = launch_pdl(k, grid, kT, tp.total, stream, p, tp);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -668,6 +694,9 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kST, 1)
     return true;
   };
 
+  // programmatic dependent launch, as in the persistent form: set-up before the wait, every global
+  // access after it
+  griddep_launch_dependents();
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(kSplitTmemCols));
@@ -677,6 +706,9 @@ __global__ void __cluster_dims__(kSplit, 1, 1) __launch_bounds__(kST, 1)
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(full));
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(mbar));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  griddep_wait();
+  if (tid == 0) {
     const uint32_t n_st = kRows * kP * 4, n_b = (uint32_t)R * kN * 2, n_cb = (uint32_t)R * kN * 4;
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full),
                  "r"(n_st + 2 * n_b + n_cb + kP * 2 + kP * 4 + kN / 2 * 4)
@@ -864,7 +896,8 @@ cudaError_t launch_split_rt(const Params& p, const SplitPlan& sp, cudaStream_t s
   auto k = decode_tc_split_kernel<RT>;
   cudaError_t e = smem_set.ensure(k, (int)sp.total);
   if (e != cudaSuccess) return e;
-  k<<<(unsigned)(p.b * p.H * kSplit), kST, sp.total, stream>>>(p, sp);
+  e = launch_pdl(k, (unsigned)(p.b * p.H * kSplit), kST, sp.total, stream, p, sp);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -15,7 +15,6 @@ namespace m3 {
 namespace {
 
 constexpr int kFeWarps = 8;
-constexpr float kBcNormEps = 1e-6f;
 
 template <bool BF16>
 __global__ void __launch_bounds__(32 * kFeWarps)
@@ -48,10 +47,9 @@ __global__ void __launch_bounds__(32 * kFeWarps)
   }
   const int64_t tstride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nscal; i += tstride) {
-    const float d = dt_raw[i];
-    dt[i] = d > 20.0f ? d : log1pf(__expf(d));
-    A[i] = -__expf(A_raw[i]);
-    lam[i] = 1.0f / (1.0f + __expf(-lam_raw[i]));
+    dt[i] = fe_softplus(dt_raw[i]);
+    A[i] = fe_negexp(A_raw[i]);
+    lam[i] = fe_sigmoid(lam_raw[i]);
   }
 }
 

@@ -481,8 +481,7 @@ cudaError_t launch_bwd_t(const Params& p, const BwdArgs& q, cudaStream_t stream)
   if (nk <= 2) return launch_bwd_nk<T, 2>(p, q, stream);
   if (nk <= 4) return launch_bwd_nk<T, 4>(p, q, stream);
   if (nk <= 8) return launch_bwd_nk<T, 8>(p, q, stream);
-  if (nk <= 16) return launch_bwd_nk<T, 16>(p, q, stream);
-  return launch_bwd_nk<T, 32>(p, q, stream);
+  return launch_bwd_nk<T, 16>(p, q, stream);
 }
 
 }  // namespace
@@ -505,7 +504,9 @@ size_t scan_bwd_workspace_bytes(const Params& p) {
 }
 
 bool bwd_supported(const Params& p) {
-  return p.P <= kBwdThreads && p.R <= 8 && bwd_smem(p.P, p.N, p.R).total * 4 <= 200 * 1024;
+  // at most 16 rotation pairs per thread (registers); headdim 256 with d_state >= 128 exceeds that
+  return p.P <= kBwdThreads && p.R <= 8 && bwd_shape(p.P, p.N).NK <= 16 &&
+         bwd_smem(p.P, p.N, p.R).total * 4 <= 200 * 1024;
 }
 
 cudaError_t launch_scan_bwd(const Params& p, const void* dy, const float* dh_final, void* dx, float* ddt, float* dA,

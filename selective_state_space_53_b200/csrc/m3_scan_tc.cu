@@ -1142,10 +1142,10 @@ size_t ws_bytes_for(const Params& p, SegPlan* out) {
 
 }  // namespace
 bool ws_scan_supported(const Params& p);
-cudaError_t launch_scan_ws(const CUtensorMap& tmB, const CUtensorMap& tmC, const Params& p, const SegInfo& sg,
-                           cudaStream_t stream);
-cudaError_t launch_scan_ws_state(const CUtensorMap& tmB, const CUtensorMap& tmC, const Params& p,
-                                 const SegInfo& sg, cudaStream_t stream);
+cudaError_t launch_scan_ws(const CUtensorMap& tmB, const CUtensorMap& tmC, const CUtensorMap& tmX, const Params& p,
+                           const SegInfo& sg, cudaStream_t stream);
+cudaError_t launch_scan_ws_state(const CUtensorMap& tmB, const CUtensorMap& tmC, const CUtensorMap& tmX,
+                                 const Params& p, const SegInfo& sg, cudaStream_t stream);
 namespace {
 
 // Summary of a whole range (sequence sharding): the state pass over every tile of the range,
@@ -1195,7 +1195,7 @@ cudaError_t launch_summary_cfg(const Params& p, void* ws, size_t ws_bytes, SegIn
   *sg_out = sg;
   Maps m;
   if (!make_maps(p, Q, &m)) return cudaErrorInvalidValue;
-  if (ws_scan_supported(p)) return launch_scan_ws_state(m.B, m.C, p, sg, stream);
+  if (ws_scan_supported(p)) return launch_scan_ws_state(m.B, m.C, m.X, p, sg, stream);
   return launch_mode<R, N, P, MODE_STATE>(m, p, sg, (unsigned)(nseq * ns), stream);
 }
 
@@ -1228,7 +1228,7 @@ cudaError_t launch_cfg(const Params& p, void* ws, size_t ws_bytes, cudaStream_t 
     sg.ws_phi = reinterpret_cast<double*>(w + off);
   }
   // headdim 128 with a rank the warp-specialised kernel covers: that kernel, same plan
-  if (ws_scan_supported(p)) return launch_scan_ws(m.B, m.C, p, sg, stream);
+  if (ws_scan_supported(p)) return launch_scan_ws(m.B, m.C, m.X, p, sg, stream);
   if (nseg > 1) {
     cudaError_t e = launch_mode<R, N, P, MODE_STATE>(m, p, sg, (unsigned)(nseq * plan.nsub), stream);
     if (e != cudaSuccess) return e;

@@ -45,6 +45,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cuda_fp16.h>
+
 #include "m3_common.cuh"
 #include "m3_ptx.cuh"
 #include "m3_scan_plan.cuh"
@@ -61,6 +63,7 @@ constexpr float WS_FAST_RANGE = 64.0f;            // largest log-decay range of 
 constexpr unsigned long long WS_WAIT_NS = 2000000000ull;  // 2 s bound on any wait
 constexpr int WS_FULL = 0, WS_STATE = 1;
 constexpr uint32_t BAR_ROT = 1;                   // named barrier of the rotation warps
+constexpr uint32_t BAR_SPX = 2;                   // named barrier of the state warps
 
 // barrier indices
 enum {
@@ -80,7 +83,9 @@ enum {
   B_YE = 24,    // Y^T read (epilogue warps)
   B_DRAIN = 25, // all MMAs complete (end of kernel)
   B_FIN = 26,   // final angles published (rotation warps)
-  NBAR = 27
+  B_XF = 27,    // [2] x of a slot landed (TMA bytes)
+  B_XE = 29,    // [2] x slot consumed (state warps)
+  NBAR = 31
 };
 
 template <int R, int N>
@@ -95,17 +100,18 @@ struct WsCfg {
   static constexpr int OFF_STAGE = 0;
   static constexpr int OFF_SP = OFF_STAGE + 2 * STAGE;           // S', 128 x 128 bf16
   static constexpr int OFF_HB = OFF_SP + 128 * 128 * 2;          // hb, 128 (p) x N bf16
-  static constexpr int TAB_ROW = K2 * 8 + 16;                    // (cos, sin) of one token, padded
+  static constexpr int TAB_ROW = K2 * 4 + 16;                    // (cos, sin) of one token in fp16, padded
   static constexpr int OFF_TAB = OFF_HB + WP * N * 2;
-  static constexpr int BIAS_ROW = N * 4 + 16;
-  static constexpr int OFF_BIAS = OFF_TAB + Q * TAB_ROW;         // bias_B rows r, then bias_C rows r
+  static constexpr int XSLOT = Q * WP * 2;                       // x of one tile, (token, p) bf16
+  static constexpr int OFF_X = OFF_TAB + Q * TAB_ROW;            // [2] slots, TMA destination
   static constexpr int SEGS = 256 / K2;                          // angle prefix segments
   static constexpr int SEGLEN = Q / SEGS;
-  static constexpr int OFF_SEGSUM = OFF_BIAS + 2 * R * BIAS_ROW;  // float [SEGS][K2]
+  static constexpr int OFF_SEGSUM = OFF_X + 2 * XSLOT;           // float [SEGS][K2]
   static constexpr int OFF_BASE = OFF_SEGSUM + SEGS * K2 * 4;    // double [K2]
   static constexpr int REC_SLOT = Q * 16 + Q * 4 + 64;           // float4 rec[Q], float mult[Q], float scal[16]
   static constexpr int OFF_REC = OFF_BASE + K2 * 8;
-  static constexpr int OFF_BAR = OFF_REC + WS_CS * REC_SLOT;
+  static constexpr int OFF_ROWSS = OFF_REC + WS_CS * REC_SLOT;    // float [2][128]: B, C row sums of squares
+  static constexpr int OFF_BAR = OFF_ROWSS + 2 * 128 * 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM = BYTES + 1024;
@@ -166,16 +172,21 @@ __device__ __forceinline__ bool bar_any(uint32_t id, uint32_t nthreads, bool pre
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-// Rotate the 8 values of one 16-byte chunk (4 pairs) by the pairs' (cos, sin), after adding the
-// bias, and scale: out = sc * Rot(-Phi)(v + bias).
-__device__ __forceinline__ uint4 rotate_chunk(uint4 raw, const float4& b0, const float4& b1, const float4& cs01,
-                                              const float4& cs23, float sc) {
+// Rotate the 8 values of one 16-byte chunk (4 pairs) by the pairs' (cos, sin) (half precision:
+// (c0, s0, c1, s1) and (c2, s2, c3, s3)), after the row's norm factor and the bias, and scale:
+// out = sc * Rot(-Phi)(nrm v + bias).
+__device__ __forceinline__ uint4 rotate_chunk(uint4 raw, const float4& b0, const float4& b1, const uint2& cs01,
+                                              const uint2& cs23, float nrm, float sc) {
   float f[8];
   unpack8(raw, f);
-  f[0] += b0.x; f[1] += b0.y; f[2] += b0.z; f[3] += b0.w;
-  f[4] += b1.x; f[5] += b1.y; f[6] += b1.z; f[7] += b1.w;
-  const float c[4] = {cs01.x * sc, cs01.z * sc, cs23.x * sc, cs23.z * sc};
-  const float s[4] = {cs01.y * sc, cs01.w * sc, cs23.y * sc, cs23.w * sc};
+  f[0] = fmaf(nrm, f[0], b0.x); f[1] = fmaf(nrm, f[1], b0.y); f[2] = fmaf(nrm, f[2], b0.z); f[3] = fmaf(nrm, f[3], b0.w);
+  f[4] = fmaf(nrm, f[4], b1.x); f[5] = fmaf(nrm, f[5], b1.y); f[6] = fmaf(nrm, f[6], b1.z); f[7] = fmaf(nrm, f[7], b1.w);
+  const float2 p0 = __half22float2(*reinterpret_cast<const __half2*>(&cs01.x));
+  const float2 p1 = __half22float2(*reinterpret_cast<const __half2*>(&cs01.y));
+  const float2 p2 = __half22float2(*reinterpret_cast<const __half2*>(&cs23.x));
+  const float2 p3 = __half22float2(*reinterpret_cast<const __half2*>(&cs23.y));
+  const float c[4] = {p0.x * sc, p1.x * sc, p2.x * sc, p3.x * sc};
+  const float s[4] = {p0.y * sc, p1.y * sc, p2.y * sc, p3.y * sc};
   float o[8];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
@@ -207,9 +218,9 @@ __device__ __forceinline__ void hb_store_row(uint32_t sHB, int pc, int c, const 
 }
 
 template <int R, int N, int MODE>
-__global__ void __maxnreg__(88)
-    scan_ws_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC, const Params p,
-                   const SegInfo sg) {
+__global__ void __maxnreg__(80)
+    scan_ws_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
+                   const __grid_constant__ CUtensorMap tmX, const Params p, const SegInfo sg) {
   using C = WsCfg<R, N>;
   constexpr bool FULL = (MODE == WS_FULL);
   constexpr int Q = C::Q, K2 = C::K2, BLK = C::BLK;
@@ -237,12 +248,14 @@ __global__ void __maxnreg__(88)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::OFF_MISC + 4);
   const uint32_t sStage = smem_u32(sm + C::OFF_STAGE);
   const uint32_t sSP = smem_u32(sm + C::OFF_SP), sHB = smem_u32(sm + C::OFF_HB);
+  const uint32_t sXr = smem_u32(sm + C::OFF_X);
   auto sB = [&](int s) { return sStage + (uint32_t)(s * C::STAGE); };
   auto sC = [&](int s) { return sStage + (uint32_t)(s * C::STAGE + C::TILE_N); };
   auto recA = [&](int cs) { return reinterpret_cast<float4*>(sm + C::OFF_REC + cs * C::REC_SLOT); };
   auto mult = [&](int cs) { return reinterpret_cast<float*>(sm + C::OFF_REC + cs * C::REC_SLOT + Q * 16); };
   auto scal = [&](int cs) { return reinterpret_cast<float*>(sm + C::OFF_REC + cs * C::REC_SLOT + Q * 20); };
   double* base = reinterpret_cast<double*>(sm + C::OFF_BASE);
+  float* rowss = reinterpret_cast<float*>(sm + C::OFF_ROWSS);
   float* segsum = reinterpret_cast<float*>(sm + C::OFF_SEGSUM);
   const __nv_bfloat16* xg = static_cast<const __nv_bfloat16*>(p.x);
 
@@ -273,18 +286,14 @@ __global__ void __maxnreg__(88)
     mbar_init(&bar[B_YE], 4);
     mbar_init(&bar[B_DRAIN], 1);
     mbar_init(&bar[B_FIN], N_ROT);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[B_XF + s], 1);
+      mbar_init(&bar[B_XE + s], 4);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  {
-    float* bias = reinterpret_cast<float*>(sm + C::OFF_BIAS);
-    for (int i = tid; i < 2 * R * N; i += WS_THREADS) {
-      const int which = i / (R * N), rn = i % (R * N);
-      const float* src = which == 0 ? p.bias_B : p.bias_C;
-      bias[(which * R + rn / N) * (C::BIAS_ROW / 4) + rn % N] = src ? src[(int64_t)hi * R * N + rn] : 0.0f;
-    }
-    for (int k = tid; k < K2; k += WS_THREADS) base[k] = 0.0;
-  }
+  for (int k = tid; k < K2; k += WS_THREADS) base[k] = 0.0;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -294,15 +303,23 @@ __global__ void __maxnreg__(88)
     if (warp == W_PROD) {
       // =============================================================== producer
       if (lane == 0) {
-        Phases ph_e;
-        int issued0 = 0, issued1 = 0;
+        Phases ph_e, ph_xe;
+        int issued0 = 0, issued1 = 0, xissued0 = 0, xissued1 = 0;
         for (int i = 0; i < ntl; ++i) {
           const int s = i & 1;
+          const int tok = (int)(tok_base + (j0 + i) * Q);
+          // x of the tile (for X'^T) into its slot, once the state warps have read the slot's last tile
+          if (i >= 2) {
+            if (!ws_wait(&bar[B_XE + s], ph_xe[s], abort_flag)) break;
+            ph_xe.flip(s);
+          }
+          mbar_expect_tx(&bar[B_XF + s], C::XSLOT);
+          tma_load_3d(sXr + (uint32_t)(s * C::XSLOT), &tmX, 0, hi, tok, &bar[B_XF + s]);
+          if (s) ++xissued1; else ++xissued0;
           if (i >= 2) {
             if (!ws_wait(&bar[B_BCE + s], ph_e[s], abort_flag)) break;
             ph_e.flip(s);
           }
-          const int tok = (int)(tok_base + (j0 + i) * Q);
           mbar_expect_tx(&bar[B_BCF + s], FULL ? C::STAGE : C::TILE_N);
 #pragma unroll
           for (int blk = 0; blk < N / 64; ++blk) {
@@ -314,6 +331,8 @@ __global__ void __maxnreg__(88)
         // every copy issued has landed before the CTA may exit
         if (issued0 > 0) ws_wait_drain(&bar[B_BCF + 0], (uint32_t)((issued0 - 1) & 1));
         if (issued1 > 0) ws_wait_drain(&bar[B_BCF + 1], (uint32_t)((issued1 - 1) & 1));
+        if (xissued0 > 0) ws_wait_drain(&bar[B_XF + 0], (uint32_t)((xissued0 - 1) & 1));
+        if (xissued1 > 0) ws_wait_drain(&bar[B_XF + 1], (uint32_t)((xissued1 - 1) & 1));
       }
     } else if (warp == W_COEF) {
       // =============================================================== coefficients
@@ -338,6 +357,11 @@ __global__ void __maxnreg__(88)
           dtv[e] = valid ? p.dt[ti] : 0.0f;
           av[e] = valid ? p.A[ti] : 0.0f;
           lmv[e] = valid ? p.lam[ti] : 0.0f;
+          if (p.raw_inputs && valid) {  // the front-end, fused: the operands are raw projections
+            dtv[e] = fe_softplus(dtv[e]);
+            av[e] = fe_negexp(av[e]);
+            lmv[e] = fe_sigmoid(lmv[e]);
+          }
           run += dtv[e] * av[e];
           loc[e] = run;
         }
@@ -366,7 +390,9 @@ __global__ void __maxnreg__(88)
         float bp_after = 0.0f;
         if (c0 + Q < L) {
           const int64_t ti = (tok_base + c0 + Q) * H + hi;
-          bp_after = (1.0f - p.lam[ti]) * p.dt[ti];
+          const float la = p.raw_inputs ? fe_sigmoid(p.lam[ti]) : p.lam[ti];
+          const float da = p.raw_inputs ? fe_softplus(p.dt[ti]) : p.dt[ti];
+          bp_after = (1.0f - la) * da;
         }
         const float nxt_dt = __shfl_down_sync(kFull, dtv[0], 1);
         const float nxt_lm = __shfl_down_sync(kFull, lmv[0], 1);
@@ -438,7 +464,6 @@ __global__ void __maxnreg__(88)
       };
       load_theta(j0);
       Phases ph_cf, ph_bcf;
-      const float* biasT = reinterpret_cast<const float*>(sm + C::OFF_BIAS);
       uint8_t* tab = sm + C::OFF_TAB;
       for (int i = 0; i < ntl; ++i) {
         const int cs = i % WS_CS, s = i & 1;
@@ -450,6 +475,7 @@ __global__ void __maxnreg__(88)
         okw = okw && ws_wait(&bar[B_BCF + s], ph_bcf[s], abort_flag);
         ph_bcf.flip(s);
         if (bar_any(BAR_ROT, 32 * N_ROT, !okw || *abort_flag)) break;  // the group stops together
+        if (p.raw_inputs) rowss[rt] = 0.0f;  // ordered before the row sums by the barriers below
         const float* mu = mult(cs);
         const float4* ra = recA(cs);
         const float* sc = scal(cs);
@@ -479,7 +505,7 @@ __global__ void __maxnreg__(88)
             const int t = aseg * C::SEGLEN + e;
             float sn, cn;
             sincos_reduced(aoff + aloc[e], &sn, &cn);
-            *reinterpret_cast<float2*>(tab + t * C::TAB_ROW + ak * 8) = make_float2(cn, sn);
+            *reinterpret_cast<__half2*>(tab + t * C::TAB_ROW + ak * 4) = __floats2half2_rn(cn, sn);
           }
         }
         if (i + 1 < ntl) load_theta(j + 1);
@@ -489,17 +515,49 @@ __global__ void __maxnreg__(88)
           nb -= 6.283185307179586 * rint(nb * 0.15915494309189535);
           base[ak] = nb;
         }
+        if (p.raw_inputs) {
+          // the fused B/C RMS norm: every row's sum of squares over N, from each warp's chunks
+#pragma unroll 1
+          for (int q = 0; q < C::KCW; ++q) {
+            const int kc = wr + N_ROT * q;
+            for (int step = 0; step < 4; ++step) {
+              const int row = 32 * step + lane;
+              if (row / R >= nv) continue;
+              const uint32_t off = (uint32_t)(kc >> 3) * BLK + (uint32_t)row * 128u +
+                                   ((uint32_t)((kc & 7) ^ (row & 7)) << 4);
+              float f[8];
+              unpack8(lds128(sB(s) + off), f);
+              float ss = 0.0f;
+#pragma unroll
+              for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+              atomicAdd(&rowss[row], ss);
+              if constexpr (FULL) {
+                unpack8(lds128(sC(s) + off), f);
+                ss = 0.0f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+                atomicAdd(&rowss[128 + row], ss);
+              }
+            }
+          }
+          named_bar_sync(BAR_ROT, 32 * N_ROT);
+        }
         // ---- rotate Bt' (and Ct') of the tile in place: lanes take 32 consecutive rows
 #pragma unroll 1
         for (int q = 0; q < C::KCW; ++q) {
           const int kc = wr + N_ROT * q;
           const int r = lane % R;
-          const float4 bb0 = *reinterpret_cast<const float4*>(biasT + r * (C::BIAS_ROW / 4) + 8 * kc);
-          const float4 bb1 = *reinterpret_cast<const float4*>(biasT + r * (C::BIAS_ROW / 4) + 8 * kc + 4);
-          float4 bc0 = make_float4(0.f, 0.f, 0.f, 0.f), bc1 = bc0;
+          const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4* bB4 = p.bias_B ? reinterpret_cast<const float4*>(p.bias_B + ((int64_t)hi * R + r) * N + 8 * kc)
+                                       : nullptr;
+          const float4 bb0 = bB4 ? __ldg(bB4) : z4, bb1 = bB4 ? __ldg(bB4 + 1) : z4;
+          float4 bc0 = z4, bc1 = z4;
           if constexpr (FULL) {
-            bc0 = *reinterpret_cast<const float4*>(biasT + (R + r) * (C::BIAS_ROW / 4) + 8 * kc);
-            bc1 = *reinterpret_cast<const float4*>(biasT + (R + r) * (C::BIAS_ROW / 4) + 8 * kc + 4);
+            if (p.bias_C) {
+              const float4* bC4 = reinterpret_cast<const float4*>(p.bias_C + ((int64_t)hi * R + r) * N + 8 * kc);
+              bc0 = __ldg(bC4);
+              bc1 = __ldg(bC4 + 1);
+            }
           }
 #pragma unroll 2
           for (int step = 0; step < 4; ++step) {
@@ -509,13 +567,18 @@ __global__ void __maxnreg__(88)
                                  ((uint32_t)((kc & 7) ^ (row & 7)) << 4);
             if (t < nv) {
               const float4 rec = ra[t];
-              const float4 cs01 = *reinterpret_cast<const float4*>(tab + t * C::TAB_ROW + kc * 32);
-              const float4 cs23 = *reinterpret_cast<const float4*>(tab + t * C::TAB_ROW + kc * 32 + 16);
+              float nb = 1.0f, nc = 1.0f;
+              if (p.raw_inputs) {  // 1 / rms of the raw rows: the B/C norm, before the bias
+                nb = rsqrtf(rowss[row] * (1.0f / N) + kBcNormEps);
+                if constexpr (FULL) nc = rsqrtf(rowss[128 + row] * (1.0f / N) + kBcNormEps);
+              }
+              const uint2 cs01 = *reinterpret_cast<const uint2*>(tab + t * C::TAB_ROW + kc * 16);
+              const uint2 cs23 = *reinterpret_cast<const uint2*>(tab + t * C::TAB_ROW + kc * 16 + 8);
               const uint4 rb = lds128(sB(s) + off);
               uint4 rc;
               if constexpr (FULL) rc = lds128(sC(s) + off);
-              sts128(sB(s) + off, rotate_chunk(rb, bb0, bb1, cs01, cs23, rec.z));
-              if constexpr (FULL) sts128(sC(s) + off, rotate_chunk(rc, bc0, bc1, cs01, cs23, rec.w));
+              sts128(sB(s) + off, rotate_chunk(rb, bb0, bb1, cs01, cs23, nb, rec.z));
+              if constexpr (FULL) sts128(sC(s) + off, rotate_chunk(rc, bc0, bc1, cs01, cs23, nc, rec.w));
             } else {
               sts128(sB(s) + off, make_uint4(0, 0, 0, 0));
               if constexpr (FULL) sts128(sC(s) + off, make_uint4(0, 0, 0, 0));
@@ -760,7 +823,7 @@ __global__ void __maxnreg__(88)
       float wx[R];
 #pragma unroll
       for (int r = 0; r < R; ++r) wx[r] = p.W_x ? p.W_x[((int64_t)hi * R + r) * WP + pc] : 1.0f;
-      Phases ph_cf, ph_xbf;
+      Phases ph_cf, ph_xbf, ph_xf;
       constexpr int TPC = 32 / R;
       // X'^T of tile i: X'^T[p, tR + r] = W_x[r, p] x_t[p], bf16 pairs along the columns
       auto build_xp = [&](int i) -> bool {
@@ -771,14 +834,17 @@ __global__ void __maxnreg__(88)
         }
         const int64_t c0 = (j0 + i) * Q;
         const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
+        if (!ws_wait(&bar[B_XF + xb], ph_xf[xb], abort_flag)) return false;
+        ph_xf.flip(xb);
         tc_fence_after();
+        const __nv_bfloat16* xs = reinterpret_cast<const __nv_bfloat16*>(sm + C::OFF_X + xb * C::XSLOT);
 #pragma unroll 1
         for (int gq = 0; gq < 4; ++gq) {
           float xv[TPC];
 #pragma unroll
           for (int u = 0; u < TPC; ++u) {
             const int t = TPC * gq + u;
-            xv[u] = (t < nv) ? __bfloat162float(xg[((tok_base + c0 + t) * H + hi) * (int64_t)WP + pc]) : 0.0f;
+            xv[u] = (t < nv) ? __bfloat162float(xs[t * WP + pc]) : 0.0f;
           }
           uint32_t w[16];
 #pragma unroll
@@ -791,7 +857,10 @@ __global__ void __maxnreg__(88)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[B_XPF + xb]);
+        if (lane == 0) {
+          mbar_arrive(&bar[B_XPF + xb]);
+          mbar_arrive(&bar[B_XE + xb]);  // the x slot is read
+        }
         return true;
       };
       bool ok = build_xp(0);
@@ -809,7 +878,9 @@ __global__ void __maxnreg__(88)
           const int nfold = fold ? seg * (sg.seg_tiles / sg.sub_tiles) : 0;
           float bp0 = 0.0f, xprev[R];
           if (from_state || make_init) {
-            bp0 = (1.0f - p.lam[tok_base * H + hi]) * p.dt[tok_base * H + hi];
+            const float l0 = p.raw_inputs ? fe_sigmoid(p.lam[tok_base * H + hi]) : p.lam[tok_base * H + hi];
+            const float d0 = p.raw_inputs ? fe_softplus(p.dt[tok_base * H + hi]) : p.dt[tok_base * H + hi];
+            bp0 = (1.0f - l0) * d0;
 #pragma unroll
             for (int r = 0; r < R; ++r) xprev[r] = wx[r] * p.carry_x[(int64_t)bh * WP + pc];
           }
@@ -893,13 +964,17 @@ __global__ void __maxnreg__(88)
         if (i + 1 < ntl) ok = build_xp(i + 1);
       }
       // ---- results: the state after the last tile
-      const bool results = ok && !*abort_flag && (!FULL || last_seg);
-      if (results && ws_wait(&bar[B_SPGO], (uint32_t)((ntl - 1) & 1), abort_flag)) {
+      bool go = ok && !*abort_flag && (!FULL || last_seg);
+      if (go) go = ws_wait(&bar[B_SPGO], (uint32_t)((ntl - 1) & 1), abort_flag);
+      if (FULL && go) go = ws_wait(&bar[B_FIN], 0, abort_flag);
+      // the raw-input carry below synchronises the four state warps: they decide together
+      if (FULL && last_seg && p.raw_inputs && bar_any(BAR_SPX, 128, !go)) go = false;
+      if (go) {
         tc_fence_after();
         const float inv_rho = scal((ntl - 1) % WS_CS)[5];
         if constexpr (FULL) {
           // rotate back from the segment frame by the segment's total angle
-          if (ws_wait(&bar[B_FIN], 0, abort_flag)) {
+          {
             float* hout = p.h + (int64_t)bh * N * WP;
 #pragma unroll 1
             for (int c = 0; c < N / 32; ++c) {
@@ -917,11 +992,25 @@ __global__ void __maxnreg__(88)
                 hout[(int64_t)(2 * k + 1) * WP + pc] = sn * a0 + cn * a1;
               }
             }
-            // the carry: the last token's raw B and x
+            // the carry: the last token's B (as the core used it: normalised when the operands are
+            // raw) and raw x
             const int64_t tokl = tok_base + (L - 1);
             const __nv_bfloat16* Bg = static_cast<const __nv_bfloat16*>(p.B);
             const int64_t bc = ((tokl * G + g) * R) * (int64_t)N;
-            for (int k = pc; k < R * N; k += WP) p.carry_B[(int64_t)bh * R * N + k] = __bfloat162float(Bg[bc + k]);
+            if (p.raw_inputs) {  // the rotation warps are done with rowss (B_FIN)
+              if (pc < R) rowss[pc] = 0.0f;
+              named_bar_sync(BAR_SPX, 128);
+              for (int k = pc; k < R * N; k += WP) {
+                const float v = __bfloat162float(Bg[bc + k]);
+                atomicAdd(&rowss[k / N], v * v);
+              }
+              named_bar_sync(BAR_SPX, 128);
+            }
+            for (int k = pc; k < R * N; k += WP) {
+              float v = __bfloat162float(Bg[bc + k]);
+              if (p.raw_inputs) v *= rsqrtf(rowss[k / N] * (1.0f / N) + kBcNormEps);
+              p.carry_B[(int64_t)bh * R * N + k] = v;
+            }
             p.carry_x[(int64_t)bh * WP + pc] = __bfloat162float(xg[(tokl * H + hi) * (int64_t)WP + pc]);
           }
         } else {
@@ -961,49 +1050,53 @@ bool ws_scan_supported(const Params& p) {
 
 namespace {
 template <int R, int N, int MODE>
-cudaError_t launch_ws_mode(const CUtensorMap& tmB, const CUtensorMap& tmC, const Params& p, const SegInfo& sg,
-                           unsigned grid, cudaStream_t stream) {
+cudaError_t launch_ws_mode(const CUtensorMap& tmB, const CUtensorMap& tmC, const CUtensorMap& tmX, const Params& p,
+                           const SegInfo& sg, unsigned grid, cudaStream_t stream) {
   using Cf = WsCfg<R, N>;
   static SmemAttr attr;
   auto k = scan_ws_kernel<R, N, MODE>;
   cudaError_t e = attr.ensure(k, Cf::SMEM);
   if (e != cudaSuccess) return e;
-  k<<<grid, WS_THREADS, Cf::SMEM, stream>>>(tmB, tmC, p, sg);
+  int per_sm = 0;  // one CTA must fit an SM (registers of the warps, rounded up, and shared memory)
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, WS_THREADS, Cf::SMEM);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorLaunchOutOfResources;
+  k<<<grid, WS_THREADS, Cf::SMEM, stream>>>(tmB, tmC, tmX, p, sg);
   return cudaGetLastError();
 }
 
 template <int R, int N>
-cudaError_t launch_ws_rn(const CUtensorMap& tmB, const CUtensorMap& tmC, const Params& p, const SegInfo& sg,
-                         cudaStream_t stream) {
+cudaError_t launch_ws_rn(const CUtensorMap& tmB, const CUtensorMap& tmC, const CUtensorMap& tmX, const Params& p,
+                         const SegInfo& sg, cudaStream_t stream) {
   const int64_t nseq = p.b * p.H;
   if (sg.nseg > 1) {
-    cudaError_t e = launch_ws_mode<R, N, WS_STATE>(tmB, tmC, p, sg, (unsigned)(nseq * sg.nsub), stream);
+    cudaError_t e = launch_ws_mode<R, N, WS_STATE>(tmB, tmC, tmX, p, sg, (unsigned)(nseq * sg.nsub), stream);
     if (e != cudaSuccess) return e;
   }
-  return launch_ws_mode<R, N, WS_FULL>(tmB, tmC, p, sg, (unsigned)(nseq * sg.nseg), stream);
+  return launch_ws_mode<R, N, WS_FULL>(tmB, tmC, tmX, p, sg, (unsigned)(nseq * sg.nseg), stream);
 }
 }  // namespace
 
-cudaError_t launch_scan_ws_state(const CUtensorMap& tmB, const CUtensorMap& tmC, const Params& p,
-                                 const SegInfo& sg, cudaStream_t stream) {
+cudaError_t launch_scan_ws_state(const CUtensorMap& tmB, const CUtensorMap& tmC, const CUtensorMap& tmX,
+                                 const Params& p, const SegInfo& sg, cudaStream_t stream) {
   const unsigned grid = (unsigned)(p.b * p.H * sg.nsub);
-  if (p.N == 128) return p.R == 4 ? launch_ws_mode<4, 128, WS_STATE>(tmB, tmC, p, sg, grid, stream)
-                                  : launch_ws_mode<8, 128, WS_STATE>(tmB, tmC, p, sg, grid, stream);
+  if (p.N == 128) return p.R == 4 ? launch_ws_mode<4, 128, WS_STATE>(tmB, tmC, tmX, p, sg, grid, stream)
+                                  : launch_ws_mode<8, 128, WS_STATE>(tmB, tmC, tmX, p, sg, grid, stream);
   switch (p.R) {
-    case 2: return launch_ws_mode<2, 64, WS_STATE>(tmB, tmC, p, sg, grid, stream);
-    case 4: return launch_ws_mode<4, 64, WS_STATE>(tmB, tmC, p, sg, grid, stream);
-    default: return launch_ws_mode<8, 64, WS_STATE>(tmB, tmC, p, sg, grid, stream);
+    case 2: return launch_ws_mode<2, 64, WS_STATE>(tmB, tmC, tmX, p, sg, grid, stream);
+    case 4: return launch_ws_mode<4, 64, WS_STATE>(tmB, tmC, tmX, p, sg, grid, stream);
+    default: return launch_ws_mode<8, 64, WS_STATE>(tmB, tmC, tmX, p, sg, grid, stream);
   }
 }
 
-cudaError_t launch_scan_ws(const CUtensorMap& tmB, const CUtensorMap& tmC, const Params& p, const SegInfo& sg,
-                           cudaStream_t stream) {
-  if (p.N == 128) return p.R == 4 ? launch_ws_rn<4, 128>(tmB, tmC, p, sg, stream)
-                                  : launch_ws_rn<8, 128>(tmB, tmC, p, sg, stream);
+cudaError_t launch_scan_ws(const CUtensorMap& tmB, const CUtensorMap& tmC, const CUtensorMap& tmX, const Params& p,
+                           const SegInfo& sg, cudaStream_t stream) {
+  if (p.N == 128) return p.R == 4 ? launch_ws_rn<4, 128>(tmB, tmC, tmX, p, sg, stream)
+                                  : launch_ws_rn<8, 128>(tmB, tmC, tmX, p, sg, stream);
   switch (p.R) {
-    case 2: return launch_ws_rn<2, 64>(tmB, tmC, p, sg, stream);
-    case 4: return launch_ws_rn<4, 64>(tmB, tmC, p, sg, stream);
-    default: return launch_ws_rn<8, 64>(tmB, tmC, p, sg, stream);
+    case 2: return launch_ws_rn<2, 64>(tmB, tmC, tmX, p, sg, stream);
+    case 4: return launch_ws_rn<4, 64>(tmB, tmC, tmX, p, sg, stream);
+    default: return launch_ws_rn<8, 64>(tmB, tmC, tmX, p, sg, stream);
   }
 }
 

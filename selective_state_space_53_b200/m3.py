@@ -66,6 +66,7 @@ SIGNATURES = {
     "m3_selftest_wait": (_I, [ctypes.c_uint64, _VP]),
     "m3_status_str": (ctypes.c_char_p, [_I]),
     "m3_version": (ctypes.c_char_p, []),
+    "m3_last_error": (ctypes.c_char_p, []),
 }
 
 
@@ -86,6 +87,8 @@ def lib():
 
 def _check(code, what):
     if code != 0:
+        if code == -6:
+            what = f"{what} ({lib().m3_last_error().decode()})"
         raise M3Error(code, what)
 
 

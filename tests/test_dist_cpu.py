@@ -44,7 +44,7 @@ def _worker(rank, world, port, out):
 
 def test_two_ranks_max_time_and_independent_batches():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     ms0, seed0, xs0 = out[0]

@@ -2,8 +2,9 @@
 gradient (m3o_scan_bwd, itself pinned by central finite differences of the forward recurrence).
 
 Metric: max|got - ref| / max|ref| per gradient tensor; bounds 2e-2 for bf16 x/B/C/dy (the
-gradients of dx, dB, dC are stored in bf16) and 1e-3 for fp32 operands (the recomputed
-forward states and the sums over tokens run in fp32, in an order set by atomics).
+gradients dx, dB, dC are stored in bf16) and 1e-4 for fp32 operands, the bounds of the forward
+pass (the recomputed forward states and the sums over tokens run in fp32, in an order set by
+atomics).
 """
 
 import numpy as np
@@ -16,7 +17,7 @@ from selective_state_space_53_b200.inputs import make_inputs, make_state, round_
 
 pytestmark = pytest.mark.gpu
 
-TOL = {"bf16": 2e-2, "f32": 1e-3}
+TOL = {"bf16": 2e-2, "f32": 1e-4}
 
 
 def rel_err(got, ref):

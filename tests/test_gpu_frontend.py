@@ -1,5 +1,6 @@
 """The block's front-end on the GPU: m3_frontend alone, and m3_scan_fwd with
-M3_FLAG_RAW_INPUTS (raw B, C, dt, A, lam), against the oracle's front-end composed with the
+M3_FLAG_RAW_INPUTS (raw B, C, dt, A, lam) -- fused into the load stage of the headdim-128 kernel,
+run as m3_frontend before the other kernels -- against the oracle's front-end composed with the
 oracle's scan."""
 
 import numpy as np
@@ -35,10 +36,11 @@ def test_frontend_kernel_matches_oracle(dtype):
 
 
 @pytest.mark.parametrize("shape", [
-    dict(b=2, L=300, H=4, P=128, N=128, R=4, G=1),   # warp-specialised kernel
-    dict(b=1, L=200, H=2, P=64, N=64, R=2, G=1),     # headdim-64 tensor-core kernel
-    dict(b=1, L=40, H=2, P=32, N=16, R=2, G=2),      # sequential kernel
-], ids=["P128", "P64", "seq"])
+    dict(b=2, L=300, H=4, P=128, N=128, R=4, G=1),   # warp-specialised kernel: front-end fused
+    dict(b=1, L=3000, H=2, P=128, N=64, R=2, G=1),   # fused, segmented (state pass too)
+    dict(b=1, L=200, H=2, P=64, N=64, R=2, G=1),     # headdim-64 tensor-core kernel: m3_frontend first
+    dict(b=1, L=40, H=2, P=32, N=16, R=2, G=2),      # sequential kernel: m3_frontend first
+], ids=["P128", "P128seg", "P64", "seq"])
 def test_scan_with_raw_inputs_matches_oracle(shape):
     inp = make_raw_inputs(dtype="bf16", seed=961, extras=True, **shape)
     st = make_state(shape["b"], shape["H"], shape["P"], shape["N"], shape["R"], seed=962, scale=0.5)

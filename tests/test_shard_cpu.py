@@ -50,7 +50,7 @@ def _worker(rank, world, port, out):
 
 def test_two_rank_sequence_sharding_equals_one_scan():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     inp, st = _draw()
