@@ -11,29 +11,35 @@
 //
 // Transposed products.  With Lc_t the tile-local cumulative log decay and m a pivot in the
 // middle of its range, a_t = e^{Lc_t - m}, b_s = e^{m - Lc_s}, w_s = gamma_s + beta'_{s+1}:
-//   Ct'_i = a_t Rot(-Phi_t)(C_{t,r} + bias_C),   Bt'_i = b_t w_t Rot(-Phi_t)(B_{t,r} + bias_B)
-//   S   = Ct' Bt'^T                      (M = 128 rows i, N = 128 columns j, K = d_state)
-//   S'  = S below the diagonal, S gamma/w on it, 0 above (masking only: the decay
-//         e^{Lc_t - Lc_s} w_s is already a_t b_s w_s)
-//   Y^T = hb^T Ct'^T + X'^T S'^T         (M = P rows p, N = 128 columns i)
-//   ST <- ST + X'^T Bt'                  (M = P, N = d_state, K = 128), ST pre-scaled by e^m
-// with X'_i = W_x[r] * x_t and hb = bf16(e^m h+) the state entering the tile.  The output
-// then has the head dimension p on the tensor-memory lanes, so y_t[p] = sum_r W_o[r,p] Y^T[p,
-// tR + r] (+ D x_t[p]) is a sum inside one thread; the state update needs no exponentials on
-// the operands either (the uniform factor e^{Le - m} is applied once per tile to the state).
-// Tiles whose log-decay range exceeds 64 take an exact form instead: no pivot, the mask applies
-// e^{Lc_t - Lc_s} per element, and after S has read them the rows of Ct' and Bt' are rescaled
-// in place by e^{Lc_t} and e^{Le - Lc_t} for the inter-chunk and state products.  With the
-// range at most 64 every factor a_t, b_s, e^{m}, e^{Le - m} lies within e^{+-32}.
+//   Ct_i = Rot(-Phi_t)(C_{t,r} + bias_C),   Bt_i = Rot(-Phi_t)(B_{t,r} + bias_B)
+//   S   = Ct Bt^T                        (M = 128 rows i, N = 128 columns j, K = d_state)
+//   S'  = S below the diagonal, S gamma/w on it, 0 above (masking only)
+//   X'_s = b_s w_s W_x[r] x_t            (the column factor of the decay, per input row)
+//   Y^T = hb^T Ct^T + X'^T S'^T          (M = P rows p, N = 128 columns i)
+//   y_t[p] = a_t sum_r W_o[r,p] Y^T[p, tR + r] (+ D x_t[p])   (the row factor, in the epilogue)
+//   ST <- ST + X'^T Bt                   (M = P, N = d_state, K = 128), ST pre-scaled by e^m
+// with hb = bf16(e^m h+) the state entering the tile: the decay e^{Lc_t - Lc_s} w_s of the
+// intra-chunk term is a_t b_s w_s, split between the input rows and the output columns, so the
+// rotated operands carry no per-row factor.  The output has the head dimension p on the
+// tensor-memory lanes, so the combine over r is a sum inside one thread; the uniform factor
+// e^{Le - m} is applied once per tile to the state.  Tiles whose log-decay range exceeds 64 take
+// an exact form instead: no pivot (X'_s = w_s W_x x_t, a_t = 1), the mask applies
+// e^{Lc_t - Lc_s} per element, and after S has read them the rows of Ct and Bt are rescaled in
+// place by e^{Lc_t} and e^{Le - Lc_t} for the inter-chunk and state products.  With the range at
+// most 64 every factor a_t, b_s, e^{m}, e^{Le - m} lies within e^{+-32}.
 //
-// Warp roles (23 warps; every wait is an mbarrier wait bounded by %globaltimer):
-//   0      producer: TMA loads of the B and C tiles into two shared-memory stages
+// Warp roles, one warpgroup each (24 warps; every wait is an mbarrier wait that sleeps in the
+// instruction, bounded by %globaltimer):
+//   0      producer: TMA loads of the B and C tiles into two shared-memory stages, and of x
 //   1      MMA issue (one elected lane): S, H, Y_inter, Y_intra; tensor-memory allocation
 //   2      coefficients: decay cumsum, pivot, per-token scales, state scale factors
-//   3-10   rotation: cumulative angles and their sin/cos table; Bt', Ct' rotated in place
-//   11-14  mask: S from tensor memory -> S' (bf16, shared memory)
-//   15-18  epilogue: Y^T from tensor memory -> y
-//   19-22  state and inputs: the state rescale and its bf16 copy hb; X'^T into tensor memory
+//   3      idle
+//   4-11   rotation: cumulative angles and their sin/cos table; Bt, Ct rotated in place
+//   12-15  mask: S from tensor memory -> S' (bf16, shared memory)
+//   16-19  epilogue: Y^T from tensor memory -> y
+//   20-23  state and inputs: the state rescale and its bf16 copy hb; X'^T into tensor memory
+// The block is launched with 80 registers a thread; the control warpgroup gives some back and
+// the rotation warpgroups take them (setmaxnreg), since the rotation holds the most live values.
 // The tile pipeline per tile j (MMA order): H(j), Y_inter(j), Y_intra(j), S(j+1).  Each SIMT
 // task has two MMAs' time between the commit that releases it and the MMA that needs it:
 // state rescale SP(j+1) after Y_inter(j), before H(j+1); epilogue E(j) after Y_intra(j), before
@@ -55,9 +61,14 @@ namespace m3 {
 namespace {
 
 constexpr int WP = 128;  // head dim of this kernel
-constexpr int W_PROD = 0, W_MMA = 1, W_COEF = 2, W_ROT = 3, N_ROT = 8, W_MASK = 11, W_EPI = 15, W_SPX = 19;
-constexpr int WS_WARPS = 23;
+constexpr int W_PROD = 0, W_MMA = 1, W_COEF = 2, W_ROT = 4, N_ROT = 8, W_MASK = 12, W_EPI = 16, W_SPX = 20;
+constexpr int WS_WARPS = 24;
 constexpr int WS_THREADS = WS_WARPS * 32;
+// registers a thread: at launch, and per warpgroup after the reallocation
+constexpr int WS_REG_LAUNCH = 80, WS_REG_CTRL = 48, WS_REG_ROT = 96;
+static_assert(128 * (WS_REG_CTRL + 2 * WS_REG_ROT + 3 * WS_REG_LAUNCH) <= WS_THREADS * WS_REG_LAUNCH,
+              "the warpgroups' registers after setmaxnreg must fit the launch's total");
+constexpr uint32_t WS_SLEEP_NS = 1000000;          // suspend-time hint of a wait (1 ms)
 constexpr int WS_CS = 4;                          // coefficient record slots
 constexpr float WS_FAST_RANGE = 64.0f;            // largest log-decay range of a pivot-split tile
 constexpr unsigned long long WS_WAIT_NS = 2000000000ull;  // 2 s bound on any wait
@@ -83,9 +94,9 @@ enum {
   B_YE = 24,    // Y^T read (epilogue warps)
   B_DRAIN = 25, // all MMAs complete (end of kernel)
   B_FIN = 26,   // final angles published (rotation warps)
-  B_XF = 27,    // [2] x of a slot landed (TMA bytes)
-  B_XE = 29,    // [2] x slot consumed (state warps)
-  NBAR = 31
+  B_XF = 27,    // x of a tile landed (TMA bytes)
+  B_XE = 28,    // the x slot consumed (state warps)
+  NBAR = 29
 };
 
 template <int R, int N>
@@ -93,25 +104,27 @@ struct WsCfg {
   static constexpr int Q = 128 / R;
   static constexpr int K2 = N / 2;
   static constexpr int NKC = N / 8;                    // 16-byte chunks of a row
-  static constexpr int KCW = NKC / N_ROT;              // chunks per rotation warp
+  static constexpr int CPT = NKC / 2;                  // chunks of a row per rotation thread (two per row)
   static constexpr int TILE_N = 128 * N * 2;           // a B or C tile, bytes
   static constexpr int BLK = 128 * 128;                // one 64-column block of a 128-row SW128 tile
   static constexpr int STAGE = 2 * TILE_N;             // B then C
   static constexpr int OFF_STAGE = 0;
   static constexpr int OFF_SP = OFF_STAGE + 2 * STAGE;           // S', 128 x 128 bf16
   static constexpr int OFF_HB = OFF_SP + 128 * 128 * 2;          // hb, 128 (p) x N bf16
-  static constexpr int TAB_ROW = K2 * 4 + 16;                    // (cos, sin) of one token in fp16, padded
+  static constexpr int TAB_ROW = K2 * 4 + 16;                    // (cos, sin) of one token in bf16, padded
   static constexpr int OFF_TAB = OFF_HB + WP * N * 2;
   static constexpr int XSLOT = Q * WP * 2;                       // x of one tile, (token, p) bf16
-  static constexpr int OFF_X = OFF_TAB + Q * TAB_ROW;            // [2] slots, TMA destination
+  static constexpr int OFF_X = OFF_TAB + Q * TAB_ROW;            // one slot, TMA destination
+  static constexpr int BIAS_ROW = NKC * 8 + 4;                   // floats of one (operand, branch) bias row, padded
+  static constexpr int OFF_BIAS = OFF_X + XSLOT;                 // float [2][R][BIAS_ROW], staged pair layout
   static constexpr int SEGS = 256 / K2;                          // angle prefix segments
   static constexpr int SEGLEN = Q / SEGS;
-  static constexpr int OFF_SEGSUM = OFF_X + 2 * XSLOT;           // float [SEGS][K2]
+  static constexpr int OFF_SEGSUM = OFF_BIAS + 2 * R * BIAS_ROW * 4;  // float [SEGS][K2]
   static constexpr int OFF_BASE = OFF_SEGSUM + SEGS * K2 * 4;    // double [K2]
-  static constexpr int REC_SLOT = Q * 16 + Q * 4 + 64;           // float4 rec[Q], float mult[Q], float scal[16]
+  static constexpr int REC_SLOT = Q * 24 + 64;  // float4 rec[Q], float mult[Q], float ycol[Q], float scal[16]
   static constexpr int OFF_REC = OFF_BASE + K2 * 8;
-  static constexpr int OFF_ROWSS = OFF_REC + WS_CS * REC_SLOT;    // float [2][128]: B, C row sums of squares
-  static constexpr int OFF_BAR = OFF_ROWSS + 2 * 128 * 4;
+  static constexpr int OFF_ROWSS = OFF_REC + WS_CS * REC_SLOT;    // float [2][2][128]: half-row sums of squares
+  static constexpr int OFF_BAR = OFF_ROWSS + 4 * 128 * 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM = BYTES + 1024;
@@ -121,12 +134,14 @@ struct WsCfg {
   static constexpr uint32_t ID_Y = idesc_bf16(WP, 128, false, false);
   static constexpr uint32_t ID_H = idesc_bf16(WP, N, false, true);
   static_assert(Q % SEGS == 0 && SEGLEN >= 1, "angle segments");
-  static_assert(NKC % N_ROT == 0, "rotation chunks");
+  static_assert(2 * 128 == 32 * N_ROT && (CPT == 8 || CPT == 4), "rotation threads: a row half each");
   static_assert(TM_XP + 128 <= TM_COLS, "tensor memory");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
-__device__ __forceinline__ bool ws_try(uint64_t* bar, uint32_t parity) { return mbar_try_wait(bar, parity); }
+__device__ __forceinline__ bool ws_try(uint64_t* bar, uint32_t parity) {
+  return mbar_try_wait_sleep(bar, parity, WS_SLEEP_NS);
+}
 
 // Wait for the phase of `parity` to complete; false (and the abort flag set) after WS_WAIT_NS,
 // or false at once when another role has already aborted.
@@ -172,29 +187,43 @@ __device__ __forceinline__ bool bar_any(uint32_t id, uint32_t nthreads, bool pre
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-// Rotate the 8 values of one 16-byte chunk (4 pairs) by the pairs' (cos, sin) (half precision:
-// (c0, s0, c1, s1) and (c2, s2, c3, s3)), after the row's norm factor and the bias, and scale:
-// out = sc * Rot(-Phi)(nrm v + bias).
-__device__ __forceinline__ uint4 rotate_chunk(uint4 raw, const float4& b0, const float4& b1, const uint2& cs01,
-                                              const uint2& cs23, float nrm, float sc) {
-  float f[8];
-  unpack8(raw, f);
-  f[0] = fmaf(nrm, f[0], b0.x); f[1] = fmaf(nrm, f[1], b0.y); f[2] = fmaf(nrm, f[2], b0.z); f[3] = fmaf(nrm, f[3], b0.w);
-  f[4] = fmaf(nrm, f[4], b1.x); f[5] = fmaf(nrm, f[5], b1.y); f[6] = fmaf(nrm, f[6], b1.z); f[7] = fmaf(nrm, f[7], b1.w);
-  const float2 p0 = __half22float2(*reinterpret_cast<const __half2*>(&cs01.x));
-  const float2 p1 = __half22float2(*reinterpret_cast<const __half2*>(&cs01.y));
-  const float2 p2 = __half22float2(*reinterpret_cast<const __half2*>(&cs23.x));
-  const float2 p3 = __half22float2(*reinterpret_cast<const __half2*>(&cs23.y));
-  const float c[4] = {p0.x * sc, p1.x * sc, p2.x * sc, p3.x * sc};
-  const float s[4] = {p0.y * sc, p1.y * sc, p2.y * sc, p3.y * sc};
-  float o[8];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    o[2 * q] = fmaf(c[q], f[2 * q], s[q] * f[2 * q + 1]);
-    o[2 * q + 1] = fmaf(c[q], f[2 * q + 1], -s[q] * f[2 * q]);
-  }
-  return pack8(o);
+// cos, sin and -sin of the four rotation pairs k0..k0+3 of a 16-byte chunk, as f32x2 pairs
+// (k0, k0+1) and (k0+2, k0+3), from the table's half-precision words (c_k0, c_k0+1),
+// (s_k0, s_k0+1), (c_k0+2, c_k0+3), (s_k0+2, s_k0+3).
+struct RotCS {
+  uint64_t c01, s01, n01, c23, s23, n23;
+};
+__device__ __forceinline__ RotCS rot_cs(const uint4& w) {
+  const float2 c01 = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
+  const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
+  const float2 c23 = __half22float2(*reinterpret_cast<const __half2*>(&w.z));
+  const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&w.w));
+  return {f2(c01.x, c01.y), f2(s01.x, s01.y), f2(-s01.x, -s01.y),
+          f2(c23.x, c23.y), f2(s23.x, s23.y), f2(-s23.x, -s23.y)};
 }
+// Rot(-Phi)(n v + bias) on the 8 values of one 16-byte chunk (pair q in word q: first element in
+// the low half), in fp32.  The first elements of two pairs share an f32x2 lane pair and the second
+// elements another, so the rotation is four packed products per two pairs.  The bias comes in the
+// same layout: be01 = (b0, b2), bo01 = (b1, b3), be23 = (b4, b6), bo23 = (b5, b7).
+__device__ __forceinline__ uint4 rotate16(const uint4& raw, const RotCS& r, uint64_t n2, uint64_t be01,
+                                          uint64_t bo01, uint64_t be23, uint64_t bo23) {
+  const uint64_t v0a = f2_fma(n2, f2(bf_lo(raw.x), bf_lo(raw.y)), be01);
+  const uint64_t v1a = f2_fma(n2, f2(bf_hi(raw.x), bf_hi(raw.y)), bo01);
+  const uint64_t v0b = f2_fma(n2, f2(bf_lo(raw.z), bf_lo(raw.w)), be23);
+  const uint64_t v1b = f2_fma(n2, f2(bf_hi(raw.z), bf_hi(raw.w)), bo23);
+  const uint64_t o0a = f2_fma(r.c01, v0a, f2_mul(r.s01, v1a));  // c v0 + s v1
+  const uint64_t o1a = f2_fma(r.c01, v1a, f2_mul(r.n01, v0a));  // c v1 - s v0
+  const uint64_t o0b = f2_fma(r.c23, v0b, f2_mul(r.s23, v1b));
+  const uint64_t o1b = f2_fma(r.c23, v1b, f2_mul(r.n23, v0b));
+  float a0, a1, b0, b1, c0, c1, d0, d1;
+  f2_split(o0a, a0, a1);
+  f2_split(o1a, b0, b1);
+  f2_split(o0b, c0, c1);
+  f2_split(o1b, d0, d1);
+  return make_uint4(pack_bf16(a0, b0), pack_bf16(a1, b1), pack_bf16(c0, d0), pack_bf16(c1, d1));
+}
+// Position of value j of a chunk in the staged bias layout (b0, b2, b1, b3, b4, b6, b5, b7).
+__host__ __device__ constexpr int bias_pos(int j) { return (j & 4) | ((j & 1) << 1) | ((j >> 1) & 1); }
 __device__ __forceinline__ uint4 scale_chunk(uint4 raw, float sc) {
   float f[8];
   unpack8(raw, f);
@@ -205,20 +234,25 @@ __device__ __forceinline__ uint4 scale_chunk(uint4 raw, float sc) {
 
 // Row p of the bf16 state copy hb (K-major, 128-byte swizzle): the 32 values of column chunk c,
 // scaled by fh.
-__device__ __forceinline__ void hb_store_row(uint32_t sHB, int pc, int c, const float (&v)[32], float fh) {
+__device__ __forceinline__ void hb_store_row(uint32_t sHB, int pc, int c, const uint32_t (&v)[32], float fh) {
+  const uint64_t fh2 = f2(fh, fh);
 #pragma unroll
   for (int qq = 0; qq < 4; ++qq) {
     const int ch = 4 * c + qq;
-    float f8[8];
+    uint32_t w[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) f8[e] = fh * v[8 * qq + e];
+    for (int e = 0; e < 4; ++e) {
+      float a, b;
+      f2_split(f2_mul(fh2, f2(__uint_as_float(v[8 * qq + 2 * e]), __uint_as_float(v[8 * qq + 2 * e + 1]))), a, b);
+      w[e] = pack_bf16(a, b);
+    }
     const uint32_t off = (uint32_t)(ch >> 3) * (128 * 128) + (uint32_t)pc * 128u + ((uint32_t)((ch & 7) ^ (pc & 7)) << 4);
-    sts128(sHB + off, pack8(f8));
+    sts128(sHB + off, make_uint4(w[0], w[1], w[2], w[3]));
   }
 }
 
 template <int R, int N, int MODE>
-__global__ void __maxnreg__(80)
+__global__ void __maxnreg__(WS_REG_LAUNCH)
     scan_ws_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
                    const __grid_constant__ CUtensorMap tmX, const Params p, const SegInfo sg) {
   using C = WsCfg<R, N>;
@@ -253,7 +287,8 @@ __global__ void __maxnreg__(80)
   auto sC = [&](int s) { return sStage + (uint32_t)(s * C::STAGE + C::TILE_N); };
   auto recA = [&](int cs) { return reinterpret_cast<float4*>(sm + C::OFF_REC + cs * C::REC_SLOT); };
   auto mult = [&](int cs) { return reinterpret_cast<float*>(sm + C::OFF_REC + cs * C::REC_SLOT + Q * 16); };
-  auto scal = [&](int cs) { return reinterpret_cast<float*>(sm + C::OFF_REC + cs * C::REC_SLOT + Q * 20); };
+  auto ycol = [&](int cs) { return reinterpret_cast<float*>(sm + C::OFF_REC + cs * C::REC_SLOT + Q * 20); };
+  auto scal = [&](int cs) { return reinterpret_cast<float*>(sm + C::OFF_REC + cs * C::REC_SLOT + Q * 24); };
   double* base = reinterpret_cast<double*>(sm + C::OFF_BASE);
   float* rowss = reinterpret_cast<float*>(sm + C::OFF_ROWSS);
   float* segsum = reinterpret_cast<float*>(sm + C::OFF_SEGSUM);
@@ -265,7 +300,7 @@ __global__ void __maxnreg__(80)
     tmem_relinquish();
   }
   if (tid == 0) {
-    const int ce = FULL ? (N_ROT + 4 + 4 + 1) : (N_ROT + 4 + 1);
+    const int ce = FULL ? (N_ROT + 4 + 4 + 4 + 1) : (N_ROT + 4 + 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[B_BCF + s], 1);
       mbar_init(&bar[B_BCE + s], 1);
@@ -286,10 +321,8 @@ __global__ void __maxnreg__(80)
     mbar_init(&bar[B_YE], 4);
     mbar_init(&bar[B_DRAIN], 1);
     mbar_init(&bar[B_FIN], N_ROT);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar[B_XF + s], 1);
-      mbar_init(&bar[B_XE + s], 4);
-    }
+    mbar_init(&bar[B_XF], 1);
+    mbar_init(&bar[B_XE], 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -298,733 +331,773 @@ __global__ void __maxnreg__(80)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  if (ntl > 0) {
-    if (warp == W_PROD) {
-      // =============================================================== producer
-      if (lane == 0) {
-        Phases ph_e, ph_xe;
-        int issued0 = 0, issued1 = 0, xissued0 = 0, xissued1 = 0;
-        for (int i = 0; i < ntl; ++i) {
-          const int s = i & 1;
-          const int tok = (int)(tok_base + (j0 + i) * Q);
-          // x of the tile (for X'^T) into its slot, once the state warps have read the slot's last tile
-          if (i >= 2) {
-            if (!ws_wait(&bar[B_XE + s], ph_xe[s], abort_flag)) break;
-            ph_xe.flip(s);
-          }
-          mbar_expect_tx(&bar[B_XF + s], C::XSLOT);
-          tma_load_3d(sXr + (uint32_t)(s * C::XSLOT), &tmX, 0, hi, tok, &bar[B_XF + s]);
-          if (s) ++xissued1; else ++xissued0;
-          if (i >= 2) {
-            if (!ws_wait(&bar[B_BCE + s], ph_e[s], abort_flag)) break;
-            ph_e.flip(s);
-          }
-          mbar_expect_tx(&bar[B_BCF + s], FULL ? C::STAGE : C::TILE_N);
-#pragma unroll
-          for (int blk = 0; blk < N / 64; ++blk) {
-            tma_load_4d(sB(s) + blk * BLK, &tmB, 64 * blk, 0, g, tok, &bar[B_BCF + s]);
-            if constexpr (FULL) tma_load_4d(sC(s) + blk * BLK, &tmC, 64 * blk, 0, g, tok, &bar[B_BCF + s]);
-          }
-          if (s) ++issued1; else ++issued0;
-        }
-        // every copy issued has landed before the CTA may exit
-        if (issued0 > 0) ws_wait_drain(&bar[B_BCF + 0], (uint32_t)((issued0 - 1) & 1));
-        if (issued1 > 0) ws_wait_drain(&bar[B_BCF + 1], (uint32_t)((issued1 - 1) & 1));
-        if (xissued0 > 0) ws_wait_drain(&bar[B_XF + 0], (uint32_t)((xissued0 - 1) & 1));
-        if (xissued1 > 0) ws_wait_drain(&bar[B_XF + 1], (uint32_t)((xissued1 - 1) & 1));
-      }
-    } else if (warp == W_COEF) {
-      // =============================================================== coefficients
-      constexpr int TPL = Q >= 32 ? Q / 32 : 1;  // tokens per lane
-      float lrho_prev = 0.0f, seg_logdec = 0.0f;
-      Phases ph_ce;
-      for (int i = 0; i < ntl; ++i) {
-        const int cs = i % WS_CS;
-        const int64_t c0 = (j0 + i) * Q;
-        const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
-        if (i >= WS_CS) {
-          if (!ws_wait(&bar[B_CE + cs], ph_ce[cs], abort_flag)) break;
-          ph_ce.flip(cs);
-        }
-        float dtv[TPL], av[TPL], lmv[TPL], loc[TPL];
-        float run = 0.0f;
-#pragma unroll
-        for (int e = 0; e < TPL; ++e) {
-          const int t = lane * TPL + e;
-          const bool valid = t < nv && t < Q;
-          const int64_t ti = (tok_base + c0 + t) * H + hi;
-          dtv[e] = valid ? p.dt[ti] : 0.0f;
-          av[e] = valid ? p.A[ti] : 0.0f;
-          lmv[e] = valid ? p.lam[ti] : 0.0f;
-          if (p.raw_inputs && valid) {  // the front-end, fused: the operands are raw projections
-            dtv[e] = fe_softplus(dtv[e]);
-            av[e] = fe_negexp(av[e]);
-            lmv[e] = fe_sigmoid(lmv[e]);
-          }
-          run += dtv[e] * av[e];
-          loc[e] = run;
-        }
-        float incl = run;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const float o = __shfl_up_sync(kFull, incl, off);
-          if (lane >= off) incl += o;
-        }
-        const float Le = __shfl_sync(kFull, incl, 31);
-        const float excl = incl - run;
-        float lmin = 0.0f, lmax = 0.0f;
-#pragma unroll
-        for (int e = 0; e < TPL; ++e) {
-          loc[e] += excl;
-          if (lane * TPL + e < Q) {
-            lmin = fminf(lmin, loc[e]);
-            lmax = fmaxf(lmax, loc[e]);
-          }
-        }
-        lmin = key_float(__reduce_min_sync(kFull, float_key(lmin)));
-        lmax = key_float(__reduce_max_sync(kFull, float_key(lmax)));
-        const bool fast = (lmax - lmin) <= WS_FAST_RANGE;
-        const float m = fast ? 0.5f * (lmax + lmin) : 0.0f;
-        // beta' of the token after each token: the next lane's first token, or the token after the tile
-        float bp_after = 0.0f;
-        if (c0 + Q < L) {
-          const int64_t ti = (tok_base + c0 + Q) * H + hi;
-          const float la = p.raw_inputs ? fe_sigmoid(p.lam[ti]) : p.lam[ti];
-          const float da = p.raw_inputs ? fe_softplus(p.dt[ti]) : p.dt[ti];
-          bp_after = (1.0f - la) * da;
-        }
-        const float nxt_dt = __shfl_down_sync(kFull, dtv[0], 1);
-        const float nxt_lm = __shfl_down_sync(kFull, lmv[0], 1);
-        float4* ra = recA(cs);
-        float* mu = mult(cs);
-#pragma unroll
-        for (int e = 0; e < TPL; ++e) {
-          const int t = lane * TPL + e;
-          if (t < Q) {
-            const bool valid = t < nv;
-            const float gm = lmv[e] * dtv[e];
-            float bpn;
-            if (t + 1 >= Q) bpn = valid ? bp_after : 0.0f;
-            else if (e + 1 < TPL) bpn = (1.0f - lmv[e + 1]) * dtv[e + 1];
-            else bpn = (1.0f - nxt_lm) * nxt_dt;  // invalid next tokens carry dt = 0
-            const float w = gm + bpn;
-            const float dg = (w > 0.0f) ? __fdividef(gm, w) : 0.0f;
-            float cb, cc;
-            if (fast) {
-              cb = __expf(m - loc[e]) * w;
-              cc = __expf(loc[e] - m);
-            } else if (FULL) {
-              cb = w;  // rescaled by e^{Le - Lc_t} after S
-              cc = 1.0f;
-            } else {
-              cb = __expf(Le - loc[e]) * w;  // state pass: no S, the final factor at once
-              cc = 1.0f;
-            }
-            ra[t] = make_float4(loc[e], dg, cb, cc);
-            mu[t] = valid ? (p.angle_direct ? 1.0f : dtv[e]) : 0.0f;
-          }
-        }
-        // state scale factors: ST enters tile i as sigma ST_i (sigma = e^m, or e^{Le} on an exact
-        // tile) and leaves it as rho ST_{i+1} (rho = e^{m - Le}, or 1 on an exact tile, whose H
-        // operand already carries e^{Le - Lc_s})
-        const float lsig = fast ? m : Le;
-        const float lrho = fast ? (m - Le) : 0.0f;
+  const int wg = warp >> 2;
+  if (wg == 0) {
+    regs_dec<WS_REG_CTRL>();
+    if (ntl > 0) {
+      if (warp == W_PROD) {
+        // =============================================================== producer
         if (lane == 0) {
-          float* sc = scal(cs);
-          sc[0] = fast ? 1.0f : 0.0f;
-          sc[1] = Le;
-          sc[2] = m;
-          sc[3] = __expf(m - lrho_prev);     // hb = bf16(f_h * tensor-memory state)
-          sc[4] = __expf(lsig - lrho_prev);  // state before H = f_s * tensor-memory state
-          sc[5] = __expf(-lrho);             // true state after the tile = this * tensor-memory state
-          sc[6] = (float)nv;
-        }
-        lrho_prev = lrho;
-        seg_logdec += Le;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[B_CF + cs]);
-      }
-      if constexpr (!FULL) {
-        if (lane == 0 && !*abort_flag) sg.ws_l[(int64_t)bh * sg.nsub + seg] = seg_logdec;
-      }
-    } else if (warp >= W_ROT && warp < W_ROT + N_ROT) {
-      // =============================================================== rotation
-      const int rt = tid - 32 * W_ROT;
-      const int wr = warp - W_ROT;
-      const int ak = rt % K2, aseg = rt / K2;
-      float thr[C::SEGLEN];
-      auto load_theta = [&](int64_t j) {
-        const int64_t c0 = j * Q;
+          Phases ph_e, ph_xe;
+          int issued0 = 0, issued1 = 0, xissued = 0;
+          for (int i = 0; i < ntl; ++i) {
+            const int s = i & 1;
+            const int tok = (int)(tok_base + (j0 + i) * Q);
+            if (i >= 2) {
+              if (!ws_wait(&bar[B_BCE + s], ph_e[s], abort_flag)) break;
+              ph_e.flip(s);
+            }
+            mbar_expect_tx(&bar[B_BCF + s], FULL ? C::STAGE : C::TILE_N);
 #pragma unroll
-        for (int e = 0; e < C::SEGLEN; ++e) {
-          const int t = aseg * C::SEGLEN + e;
-          thr[e] = (c0 + t < L) ? p.theta[((tok_base + c0 + t) * G + g) * K2 + ak] : 0.0f;
-        }
-      };
-      load_theta(j0);
-      Phases ph_cf, ph_bcf;
-      uint8_t* tab = sm + C::OFF_TAB;
-      for (int i = 0; i < ntl; ++i) {
-        const int cs = i % WS_CS, s = i & 1;
-        const int64_t j = j0 + i;
-        const int64_t c0 = j * Q;
-        const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
-        bool okw = ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag);
-        ph_cf.flip(cs);
-        okw = okw && ws_wait(&bar[B_BCF + s], ph_bcf[s], abort_flag);
-        ph_bcf.flip(s);
-        if (bar_any(BAR_ROT, 32 * N_ROT, !okw || *abort_flag)) break;  // the group stops together
-        if (p.raw_inputs) rowss[rt] = 0.0f;  // ordered before the row sums by the barriers below
-        const float* mu = mult(cs);
-        const float4* ra = recA(cs);
-        const float* sc = scal(cs);
-        // ---- cumulative angles of the tile and their sin / cos
-        float aloc[C::SEGLEN];
-        {
-          float r2 = 0.0f;
-#pragma unroll
-          for (int e = 0; e < C::SEGLEN; ++e) {
-            r2 = fmaf(mu[aseg * C::SEGLEN + e], thr[e], r2);
-            aloc[e] = r2;
+            for (int blk = 0; blk < N / 64; ++blk) {
+              tma_load_4d(sB(s) + blk * BLK, &tmB, 64 * blk, 0, g, tok, &bar[B_BCF + s]);
+              if constexpr (FULL) tma_load_4d(sC(s) + blk * BLK, &tmC, 64 * blk, 0, g, tok, &bar[B_BCF + s]);
+            }
+            if (s) ++issued1; else ++issued0;
+            // x of the tile (for X'^T) into the slot, once the state warps have read the last one
+            if (i >= 1) {
+              if (!ws_wait(&bar[B_XE], ph_xe[0], abort_flag)) break;
+              ph_xe.flip(0);
+            }
+            mbar_expect_tx(&bar[B_XF], C::XSLOT);
+            tma_load_3d(sXr, &tmX, 0, hi, tok, &bar[B_XF]);
+            ++xissued;
           }
-          segsum[aseg * K2 + ak] = r2;
+          // every copy issued has landed before the CTA may exit
+          if (issued0 > 0) ws_wait_drain(&bar[B_BCF + 0], (uint32_t)((issued0 - 1) & 1));
+          if (issued1 > 0) ws_wait_drain(&bar[B_BCF + 1], (uint32_t)((issued1 - 1) & 1));
+          if (xissued > 0) ws_wait_drain(&bar[B_XF], (uint32_t)((xissued - 1) & 1));
         }
-        named_bar_sync(BAR_ROT, 32 * N_ROT);
-        double tot = 0.0;
-        {
-          float aoff = (float)base[ak];
-#pragma unroll
-          for (int s2 = 0; s2 < C::SEGS; ++s2) {
-            const float v = segsum[s2 * K2 + ak];
-            if (s2 < aseg) aoff += v;
-            if (aseg == 0) tot += (double)v;
+      } else if (warp == W_COEF) {
+        // =============================================================== coefficients
+        constexpr int TPL = Q >= 32 ? Q / 32 : 1;  // tokens per lane
+        float lrho_prev = 0.0f, seg_logdec = 0.0f;
+        Phases ph_ce;
+        for (int i = 0; i < ntl; ++i) {
+          const int cs = i % WS_CS;
+          const int64_t c0 = (j0 + i) * Q;
+          const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
+          if (i >= WS_CS) {
+            if (!ws_wait(&bar[B_CE + cs], ph_ce[cs], abort_flag)) break;
+            ph_ce.flip(cs);
           }
+          float dtv[TPL], av[TPL], lmv[TPL], loc[TPL];
+          float run = 0.0f;
+#pragma unroll
+          for (int e = 0; e < TPL; ++e) {
+            const int t = lane * TPL + e;
+            const bool valid = t < nv && t < Q;
+            const int64_t ti = (tok_base + c0 + t) * H + hi;
+            dtv[e] = valid ? p.dt[ti] : 0.0f;
+            av[e] = valid ? p.A[ti] : 0.0f;
+            lmv[e] = valid ? p.lam[ti] : 0.0f;
+            if (p.raw_inputs && valid) {  // the front-end, fused: the operands are raw projections
+              dtv[e] = fe_softplus(dtv[e]);
+              av[e] = fe_negexp(av[e]);
+              lmv[e] = fe_sigmoid(lmv[e]);
+            }
+            run += dtv[e] * av[e];
+            loc[e] = run;
+          }
+          float incl = run;
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const float o = __shfl_up_sync(kFull, incl, off);
+            if (lane >= off) incl += o;
+          }
+          const float Le = __shfl_sync(kFull, incl, 31);
+          const float excl = incl - run;
+          float lmin = 0.0f, lmax = 0.0f;
+#pragma unroll
+          for (int e = 0; e < TPL; ++e) {
+            loc[e] += excl;
+            if (lane * TPL + e < Q) {
+              lmin = fminf(lmin, loc[e]);
+              lmax = fmaxf(lmax, loc[e]);
+            }
+          }
+          lmin = key_float(__reduce_min_sync(kFull, float_key(lmin)));
+          lmax = key_float(__reduce_max_sync(kFull, float_key(lmax)));
+          const bool fast = (lmax - lmin) <= WS_FAST_RANGE;
+          const float m = fast ? 0.5f * (lmax + lmin) : 0.0f;
+          // beta' of the token after each token: the next lane's first token, or the token after the tile
+          float bp_after = 0.0f;
+          if (c0 + Q < L) {
+            const int64_t ti = (tok_base + c0 + Q) * H + hi;
+            const float la = p.raw_inputs ? fe_sigmoid(p.lam[ti]) : p.lam[ti];
+            const float da = p.raw_inputs ? fe_softplus(p.dt[ti]) : p.dt[ti];
+            bp_after = (1.0f - la) * da;
+          }
+          const float nxt_dt = __shfl_down_sync(kFull, dtv[0], 1);
+          const float nxt_lm = __shfl_down_sync(kFull, lmv[0], 1);
+          float4* ra = recA(cs);
+          float* mu = mult(cs);
+#pragma unroll
+          for (int e = 0; e < TPL; ++e) {
+            const int t = lane * TPL + e;
+            if (t < Q) {
+              const bool valid = t < nv;
+              const float gm = lmv[e] * dtv[e];
+              float bpn;
+              if (t + 1 >= Q) bpn = valid ? bp_after : 0.0f;
+              else if (e + 1 < TPL) bpn = (1.0f - lmv[e + 1]) * dtv[e + 1];
+              else bpn = (1.0f - nxt_lm) * nxt_dt;  // invalid next tokens carry dt = 0
+              const float w = gm + bpn;
+              const float dg = (w > 0.0f) ? __fdividef(gm, w) : 0.0f;
+              float xs, ys;  // factors of X' (input rows) and of the output columns
+              if (fast) {
+                xs = __expf(m - loc[e]) * w;
+                ys = __expf(loc[e] - m);
+              } else if (FULL) {
+                xs = w;  // Bt rescaled by e^{Le - Lc_t} after S
+                ys = 1.0f;
+              } else {
+                xs = __expf(Le - loc[e]) * w;  // state pass: no S, the final factor at once
+                ys = 1.0f;
+              }
+              ra[t] = make_float4(loc[e], dg, xs, ys);
+              mu[t] = valid ? (p.angle_direct ? 1.0f : dtv[e]) : 0.0f;
+              ycol(cs)[t] = ys;
+            }
+          }
+          // state scale factors: ST enters tile i as sigma ST_i (sigma = e^m, or e^{Le} on an exact
+          // tile) and leaves it as rho ST_{i+1} (rho = e^{m - Le}, or 1 on an exact tile, whose H
+          // operand already carries e^{Le - Lc_s})
+          const float lsig = fast ? m : Le;
+          const float lrho = fast ? (m - Le) : 0.0f;
+          if (lane == 0) {
+            float* sc = scal(cs);
+            sc[0] = fast ? 1.0f : 0.0f;
+            sc[1] = Le;
+            sc[2] = m;
+            sc[3] = __expf(m - lrho_prev);     // hb = bf16(f_h * tensor-memory state)
+            sc[4] = __expf(lsig - lrho_prev);  // state before H = f_s * tensor-memory state
+            sc[5] = __expf(-lrho);             // true state after the tile = this * tensor-memory state
+            sc[6] = (float)nv;
+          }
+          lrho_prev = lrho;
+          seg_logdec += Le;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[B_CF + cs]);
+        }
+        if constexpr (!FULL) {
+          if (lane == 0 && !*abort_flag) sg.ws_l[(int64_t)bh * sg.nsub + seg] = seg_logdec;
+        }
+      } else if (warp == W_MMA) {
+        // =============================================================== MMA issue
+        Phases ph_cf, ph_rot, ph_xpf;
+        uint32_t ph_hf = 0, ph_resc = 0, ph_ye = 0, ph_spf = 0;
+        bool issued = false, ok = true;
+        auto kdesc = [&](uint32_t base_addr, int k) {  // K-major SW128 operand, K-step k of 16
+          return sdesc(base_addr + (uint32_t)(k >> 2) * BLK + (uint32_t)(k & 3) * 32, 16, 1024);
+        };
+        if (FULL) {
+          ok = ws_wait(&bar[B_ROT + 0], ph_rot[0], abort_flag);
+          ph_rot.flip(0);
+          if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < N / 16; ++k)
+              mma_ss_w(tmem + C::TM_S, kdesc(sC(0), k), kdesc(sB(0), k), C::ID_S, k > 0);
+            mma_commit_w(&bar[B_SF]);
+            issued = true;
+          }
+        }
+        for (int i = 0; ok && i < ntl; ++i) {
+          const int cs = i % WS_CS, s = i & 1, xb = i & 1;
+          if (!ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag)) break;
+          ph_cf.flip(cs);
+          const bool fast = scal(cs)[0] != 0.0f;
+          if (!ws_wait(&bar[B_HF], ph_hf, abort_flag)) break;
+          ph_hf ^= 1;
+          if (FULL && !fast) {
+            if (!ws_wait(&bar[B_RESC], ph_resc, abort_flag)) break;
+            ph_resc ^= 1;
+          }
+          if (!ws_wait(&bar[B_XPF + xb], ph_xpf[xb], abort_flag)) break;
+          ph_xpf.flip(xb);
+          if constexpr (!FULL) {  // the full pass waited for the rotation before S of this tile
+            if (!ws_wait(&bar[B_ROT + s], ph_rot[s], abort_flag)) break;
+            ph_rot.flip(s);
+          }
+          tc_fence_after();
+          // H: ST += X'^T Bt'  (A = X'^T in tensor memory, B = Bt' MN-major)
+#pragma unroll
+          for (int k = 0; k < 128 / 16; ++k)
+            mma_ts_w(tmem + C::TM_ST, tmem + C::TM_XP + 64 * xb + 8 * k,
+                     sdesc(sB(s) + (uint32_t)k * 2048, BLK, 1024), C::ID_H, 1);
+          issued = true;
+          if constexpr (!FULL) {
+            mma_commit_w(&bar[B_SPGO]);
+            mma_commit_w(&bar[B_XBF + xb]);
+            mma_commit_w(&bar[B_BCE + s]);
+          } else {
+            if (i > 0) {
+              if (!ws_wait(&bar[B_YE], ph_ye, abort_flag)) break;
+              ph_ye ^= 1;
+              tc_fence_after();
+            }
+            // Y_inter: Y^T = hb Ct'^T  (A = hb K-major, B = Ct' K-major)
+#pragma unroll
+            for (int k = 0; k < N / 16; ++k)
+              mma_ss_w(tmem + C::TM_Y, kdesc(sHB, k), kdesc(sC(s), k), C::ID_Y, k > 0);
+            mma_commit_w(&bar[B_SPGO]);
+            mma_commit_w(&bar[B_BCE + s]);
+            if (!ws_wait(&bar[B_SPF], ph_spf, abort_flag)) break;
+            ph_spf ^= 1;
+            tc_fence_after();
+            // Y_intra: Y^T += X'^T S'^T  (A = X'^T in tensor memory, B = S' K-major)
+#pragma unroll
+            for (int k = 0; k < 128 / 16; ++k)
+              mma_ts_w(tmem + C::TM_Y, tmem + C::TM_XP + 64 * xb + 8 * k, kdesc(sSP, k), C::ID_Y, 1);
+            mma_commit_w(&bar[B_YF]);
+            mma_commit_w(&bar[B_XBF + xb]);
+            if (i + 1 < ntl) {
+              if (!ws_wait(&bar[B_ROT + (s ^ 1)], ph_rot[s ^ 1], abort_flag)) break;
+              ph_rot.flip(s ^ 1);
+              tc_fence_after();
+#pragma unroll
+              for (int k = 0; k < N / 16; ++k)
+                mma_ss_w(tmem + C::TM_S, kdesc(sC(s ^ 1), k), kdesc(sB(s ^ 1), k), C::ID_S, k > 0);
+              mma_commit_w(&bar[B_SF]);
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[B_CE + cs]);
+        }
+        if (issued) {  // every MMA issued has completed before tensor memory is released
+          mma_commit_w(&bar[B_DRAIN]);
+          ws_wait_drain(&bar[B_DRAIN], 0);
+        }
+      }
+    }
+  } else if (wg <= 2) {
+    regs_inc<WS_REG_ROT>();
+    if (ntl > 0) {
+        // =============================================================== rotation
+        const int rt = tid - 32 * W_ROT;
+        const int wr = warp - W_ROT;
+        const int ak = rt % K2, aseg = rt / K2;  // angles: pair ak over token segment aseg
+        // rotation: row rrow, chunks kc0 .. kc0 + CPT - 1 (lanes take 32 consecutive rows)
+        const int rrow = rt & 127, kc0 = (rt >> 7) * C::CPT, rr = rrow % R;
+        const int rx = (kc0 & 7) ^ (rrow & 7);  // swizzled chunk j of the row is chunk rx ^ j
+        const uint32_t rbase = (uint32_t)(kc0 >> 3) * BLK + (uint32_t)rrow * 128u;
+        // the biases of the head, staged once as fp32 in the pair layout of rotate16
+        float* sbias = reinterpret_cast<float*>(sm + C::OFF_BIAS);
+        for (int e = rt; e < 2 * R * N; e += 32 * N_ROT) {
+          const int op = e / (R * N), rem = e % (R * N), r = rem / N, n = rem % N;
+          const float* src = op ? p.bias_C : p.bias_B;
+          sbias[(op * R + r) * C::BIAS_ROW + (n >> 3) * 8 + bias_pos(n & 7)] =
+              src ? src[((int64_t)hi * R + r) * N + n] : 0.0f;
+        }
+        const float* biasB = sbias + rr * C::BIAS_ROW;
+        const float* biasC = sbias + (R + rr) * C::BIAS_ROW;
+        float thr[C::SEGLEN];
+        auto load_theta = [&](int64_t j) {
+          const int64_t c0 = j * Q;
 #pragma unroll
           for (int e = 0; e < C::SEGLEN; ++e) {
             const int t = aseg * C::SEGLEN + e;
-            float sn, cn;
-            sincos_reduced(aoff + aloc[e], &sn, &cn);
-            *reinterpret_cast<__half2*>(tab + t * C::TAB_ROW + ak * 4) = __floats2half2_rn(cn, sn);
+            thr[e] = (c0 + t < L) ? p.theta[((tok_base + c0 + t) * G + g) * K2 + ak] : 0.0f;
           }
-        }
-        if (i + 1 < ntl) load_theta(j + 1);
-        named_bar_sync(BAR_ROT, 32 * N_ROT);  // table complete; base and segsum read
-        if (aseg == 0) {
-          double nb = base[ak] + tot;
-          nb -= 6.283185307179586 * rint(nb * 0.15915494309189535);
-          base[ak] = nb;
-        }
-        if (p.raw_inputs) {
-          // the fused B/C RMS norm: every row's sum of squares over N, from each warp's chunks
-#pragma unroll 1
-          for (int q = 0; q < C::KCW; ++q) {
-            const int kc = wr + N_ROT * q;
-            for (int step = 0; step < 4; ++step) {
-              const int row = 32 * step + lane;
-              if (row / R >= nv) continue;
-              const uint32_t off = (uint32_t)(kc >> 3) * BLK + (uint32_t)row * 128u +
-                                   ((uint32_t)((kc & 7) ^ (row & 7)) << 4);
-              float f[8];
-              unpack8(lds128(sB(s) + off), f);
-              float ss = 0.0f;
+        };
+        load_theta(j0);
+        Phases ph_cf, ph_bcf;
+        uint8_t* tab = sm + C::OFF_TAB;
+        for (int i = 0; i < ntl; ++i) {
+          const int cs = i % WS_CS, s = i & 1;
+          const int64_t j = j0 + i;
+          const int64_t c0 = j * Q;
+          const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
+          bool okw = ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag);
+          ph_cf.flip(cs);
+          okw = okw && ws_wait(&bar[B_BCF + s], ph_bcf[s], abort_flag);
+          ph_bcf.flip(s);
+          if (bar_any(BAR_ROT, 32 * N_ROT, !okw || *abort_flag)) break;  // the group stops together
+          const float* mu = mult(cs);
+          const float4* ra = recA(cs);
+          const float* sc = scal(cs);
+          // ---- cumulative angles of the tile and their sin / cos
+          float aloc[C::SEGLEN];
+          {
+            float r2 = 0.0f;
 #pragma unroll
-              for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
-              atomicAdd(&rowss[row], ss);
-              if constexpr (FULL) {
-                unpack8(lds128(sC(s) + off), f);
-                ss = 0.0f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
-                atomicAdd(&rowss[128 + row], ss);
-              }
+            for (int e = 0; e < C::SEGLEN; ++e) {
+              r2 = fmaf(mu[aseg * C::SEGLEN + e], thr[e], r2);
+              aloc[e] = r2;
             }
+            segsum[aseg * K2 + ak] = r2;
           }
           named_bar_sync(BAR_ROT, 32 * N_ROT);
-        }
-        // ---- rotate Bt' (and Ct') of the tile in place: lanes take 32 consecutive rows
-#pragma unroll 1
-        for (int q = 0; q < C::KCW; ++q) {
-          const int kc = wr + N_ROT * q;
-          const int r = lane % R;
-          const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
-          const float4* bB4 = p.bias_B ? reinterpret_cast<const float4*>(p.bias_B + ((int64_t)hi * R + r) * N + 8 * kc)
-                                       : nullptr;
-          const float4 bb0 = bB4 ? __ldg(bB4) : z4, bb1 = bB4 ? __ldg(bB4 + 1) : z4;
-          float4 bc0 = z4, bc1 = z4;
-          if constexpr (FULL) {
-            if (p.bias_C) {
-              const float4* bC4 = reinterpret_cast<const float4*>(p.bias_C + ((int64_t)hi * R + r) * N + 8 * kc);
-              bc0 = __ldg(bC4);
-              bc1 = __ldg(bC4 + 1);
+          double tot = 0.0;
+          {
+            float aoff = (float)base[ak];
+#pragma unroll
+            for (int s2 = 0; s2 < C::SEGS; ++s2) {
+              const float v = segsum[s2 * K2 + ak];
+              if (s2 < aseg) aoff += v;
+              if (aseg == 0) tot += (double)v;
+            }
+#pragma unroll
+            for (int e = 0; e < C::SEGLEN; ++e) {
+              const int t = aseg * C::SEGLEN + e;
+              float sn, cn;
+              sincos_reduced(aoff + aloc[e], &sn, &cn);
+              // per two pairs (k, k+1): half2 (c_k, c_k+1) then half2 (s_k, s_k+1); the lanes of
+              // pairs k (even) and k+1 (odd) are neighbours
+              const float other = __shfl_xor_sync(kFull, (ak & 1) ? cn : sn, 1);
+              const __half2 hv = (ak & 1) ? __floats2half2_rn(other, sn) : __floats2half2_rn(cn, other);
+              *reinterpret_cast<__half2*>(tab + t * C::TAB_ROW + (ak >> 1) * 8 + (ak & 1) * 4) = hv;
             }
           }
-#pragma unroll 2
-          for (int step = 0; step < 4; ++step) {
-            const int row = 32 * step + lane;
-            const int t = row / R;
-            const uint32_t off = (uint32_t)(kc >> 3) * BLK + (uint32_t)row * 128u +
-                                 ((uint32_t)((kc & 7) ^ (row & 7)) << 4);
-            if (t < nv) {
-              const float4 rec = ra[t];
-              float nb = 1.0f, nc = 1.0f;
-              if (p.raw_inputs) {  // 1 / rms of the raw rows: the B/C norm, before the bias
-                nb = rsqrtf(rowss[row] * (1.0f / N) + kBcNormEps);
-                if constexpr (FULL) nc = rsqrtf(rowss[128 + row] * (1.0f / N) + kBcNormEps);
+          if (i + 1 < ntl) load_theta(j + 1);
+          named_bar_sync(BAR_ROT, 32 * N_ROT);  // table complete; base and segsum read
+          if (aseg == 0) {
+            double nb = base[ak] + tot;
+            nb -= 6.283185307179586 * rint(nb * 0.15915494309189535);
+            base[ak] = nb;
+          }
+          // ---- rotate Bt (and Ct) of the tile in place: this thread's row, chunks kc0 ..
+          {
+            const int t = rrow / R;
+            const bool valid = t < nv;
+            const uint32_t rB = sB(s) + rbase, rC = sC(s) + rbase;
+            float nb = 1.0f, nc = 1.0f;
+            if (p.raw_inputs) {
+              // the fused B/C RMS norm: each half row's sum of squares, then the row's
+              float ssb = 0.0f, ssc = 0.0f;
+              if (valid) {
+#pragma unroll
+                for (int j = 0; j < C::CPT; ++j) {
+                  const uint32_t off = (uint32_t)(rx ^ j) << 4;
+                  float f[8];
+                  unpack8(lds128(rB + off), f);
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) ssb = fmaf(f[e], f[e], ssb);
+                  if constexpr (FULL) {
+                    unpack8(lds128(rC + off), f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) ssc = fmaf(f[e], f[e], ssc);
+                  }
+                }
               }
-              const uint2 cs01 = *reinterpret_cast<const uint2*>(tab + t * C::TAB_ROW + kc * 16);
-              const uint2 cs23 = *reinterpret_cast<const uint2*>(tab + t * C::TAB_ROW + kc * 16 + 8);
-              const uint4 rb = lds128(sB(s) + off);
-              uint4 rc;
-              if constexpr (FULL) rc = lds128(sC(s) + off);
-              sts128(sB(s) + off, rotate_chunk(rb, bb0, bb1, cs01, cs23, nb, rec.z));
-              if constexpr (FULL) sts128(sC(s) + off, rotate_chunk(rc, bc0, bc1, cs01, cs23, nc, rec.w));
-            } else {
-              sts128(sB(s) + off, make_uint4(0, 0, 0, 0));
-              if constexpr (FULL) sts128(sC(s) + off, make_uint4(0, 0, 0, 0));
+              rowss[(2 * (kc0 != 0) + 0) * 128 + rrow] = ssb;
+              rowss[(2 * (kc0 != 0) + 1) * 128 + rrow] = ssc;
+              named_bar_sync(BAR_ROT, 32 * N_ROT);
+              nb = rsqrtf((rowss[rrow] + rowss[256 + rrow]) * (1.0f / N) + kBcNormEps);
+              nc = rsqrtf((rowss[128 + rrow] + rowss[384 + rrow]) * (1.0f / N) + kBcNormEps);
             }
-          }
-        }
-        fence_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[B_ROT + s]);
-        if (FULL && sc[0] == 0.0f) {
-          // exact tile: after S has read them, Ct' rows * e^{Lc_t} (inter-chunk product) and
-          // Bt' rows * e^{Le - Lc_t} (state product)
-          const bool oks = ws_wait(&bar[B_SF], (uint32_t)(i & 1), abort_flag);
-          if (bar_any(BAR_ROT, 32 * N_ROT, !oks || *abort_flag)) break;
-          const float Le = sc[1];
-#pragma unroll 1
-          for (int q = 0; q < C::KCW; ++q) {
-            const int kc = wr + N_ROT * q;
-            for (int step = 0; step < 4; ++step) {
-              const int row = 32 * step + lane;
-              const int t = row / R;
-              if (t >= nv) continue;
-              const uint32_t off = (uint32_t)(kc >> 3) * BLK + (uint32_t)row * 128u +
-                                   ((uint32_t)((kc & 7) ^ (row & 7)) << 4);
-              const float Lct = ra[t].x;
-              sts128(sC(s) + off, scale_chunk(lds128(sC(s) + off), __expf(Lct)));
-              sts128(sB(s) + off, scale_chunk(lds128(sB(s) + off), __expf(Le - Lct)));
+            const uint8_t* trow = tab + t * C::TAB_ROW;
+            const uint64_t nb2 = f2(nb, nb), nc2 = f2(nc, nc);
+#pragma unroll
+            for (int j = 0; j < C::CPT; ++j) {
+              const int kc = kc0 + j;
+              const uint32_t off = (uint32_t)(rx ^ j) << 4;
+              if (valid) {
+                const RotCS rcs = rot_cs(*reinterpret_cast<const uint4*>(trow + kc * 16));
+                const float4 be = *reinterpret_cast<const float4*>(biasB + kc * 8);
+                const float4 bo = *reinterpret_cast<const float4*>(biasB + kc * 8 + 4);
+                sts128(rB + off, rotate16(lds128(rB + off), rcs, nb2, f2(be.x, be.y), f2(be.z, be.w), f2(bo.x, bo.y),
+                                          f2(bo.z, bo.w)));
+                if constexpr (FULL) {
+                  const float4 ce = *reinterpret_cast<const float4*>(biasC + kc * 8);
+                  const float4 co = *reinterpret_cast<const float4*>(biasC + kc * 8 + 4);
+                  sts128(rC + off, rotate16(lds128(rC + off), rcs, nc2, f2(ce.x, ce.y), f2(ce.z, ce.w),
+                                            f2(co.x, co.y), f2(co.z, co.w)));
+                }
+              } else {
+                sts128(rB + off, make_uint4(0, 0, 0, 0));
+                if constexpr (FULL) sts128(rC + off, make_uint4(0, 0, 0, 0));
+              }
             }
           }
           fence_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bar[B_RESC]);
-        }
-        if (lane == 0) mbar_arrive(&bar[B_CE + cs]);
-      }
-      // final angles of the segment: the full pass rotates the state back by them, the state
-      // pass stores them in its summary
-      named_bar_sync(BAR_ROT, 32 * N_ROT);
-      if (!*abort_flag) {
-        if constexpr (!FULL) {
-          if (aseg == 0) sg.ws_phi[((int64_t)bh * sg.nsub + seg) * K2 + ak] = base[ak];
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[B_FIN]);
-      }
-    } else if (warp == W_MMA) {
-      // =============================================================== MMA issue
-      Phases ph_cf, ph_rot, ph_xpf;
-      uint32_t ph_hf = 0, ph_resc = 0, ph_ye = 0, ph_spf = 0;
-      bool issued = false, ok = true;
-      auto kdesc = [&](uint32_t base_addr, int k) {  // K-major SW128 operand, K-step k of 16
-        return sdesc(base_addr + (uint32_t)(k >> 2) * BLK + (uint32_t)(k & 3) * 32, 16, 1024);
-      };
-      if (FULL) {
-        ok = ws_wait(&bar[B_ROT + 0], ph_rot[0], abort_flag);
-        ph_rot.flip(0);
-        if (ok) {
-          tc_fence_after();
+          if (lane == 0) mbar_arrive(&bar[B_ROT + s]);
+          if (FULL && sc[0] == 0.0f) {
+            // exact tile: after S has read them, Ct rows * e^{Lc_t} (inter-chunk product) and
+            // Bt rows * e^{Le - Lc_t} (state product)
+            const bool oks = ws_wait(&bar[B_SF], (uint32_t)(i & 1), abort_flag);
+            if (bar_any(BAR_ROT, 32 * N_ROT, !oks || *abort_flag)) break;
+            const float Le = sc[1];
+            const int t = rrow / R;
+            if (t < nv) {
+              const float Lct = reinterpret_cast<const float*>(ra)[4 * t];
+              const float fc = __expf(Lct), fb = __expf(Le - Lct);
+              const uint32_t rB = sB(s) + rbase, rC = sC(s) + rbase;
 #pragma unroll
-          for (int k = 0; k < N / 16; ++k)
-            mma_ss_w(tmem + C::TM_S, kdesc(sC(0), k), kdesc(sB(0), k), C::ID_S, k > 0);
-          mma_commit_w(&bar[B_SF]);
-          issued = true;
-        }
-      }
-      for (int i = 0; ok && i < ntl; ++i) {
-        const int cs = i % WS_CS, s = i & 1, xb = i & 1;
-        if (!ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag)) break;
-        ph_cf.flip(cs);
-        const bool fast = scal(cs)[0] != 0.0f;
-        if (!ws_wait(&bar[B_HF], ph_hf, abort_flag)) break;
-        ph_hf ^= 1;
-        if (FULL && !fast) {
-          if (!ws_wait(&bar[B_RESC], ph_resc, abort_flag)) break;
-          ph_resc ^= 1;
-        }
-        if (!ws_wait(&bar[B_XPF + xb], ph_xpf[xb], abort_flag)) break;
-        ph_xpf.flip(xb);
-        if constexpr (!FULL) {  // the full pass waited for the rotation before S of this tile
-          if (!ws_wait(&bar[B_ROT + s], ph_rot[s], abort_flag)) break;
-          ph_rot.flip(s);
-        }
-        tc_fence_after();
-        // H: ST += X'^T Bt'  (A = X'^T in tensor memory, B = Bt' MN-major)
-#pragma unroll
-        for (int k = 0; k < 128 / 16; ++k)
-          mma_ts_w(tmem + C::TM_ST, tmem + C::TM_XP + 64 * xb + 8 * k,
-                   sdesc(sB(s) + (uint32_t)k * 2048, BLK, 1024), C::ID_H, 1);
-        issued = true;
-        if constexpr (!FULL) {
-          mma_commit_w(&bar[B_SPGO]);
-          mma_commit_w(&bar[B_XBF + xb]);
-          mma_commit_w(&bar[B_BCE + s]);
-        } else {
-          if (i > 0) {
-            if (!ws_wait(&bar[B_YE], ph_ye, abort_flag)) break;
-            ph_ye ^= 1;
-            tc_fence_after();
-          }
-          // Y_inter: Y^T = hb Ct'^T  (A = hb K-major, B = Ct' K-major)
-#pragma unroll
-          for (int k = 0; k < N / 16; ++k)
-            mma_ss_w(tmem + C::TM_Y, kdesc(sHB, k), kdesc(sC(s), k), C::ID_Y, k > 0);
-          mma_commit_w(&bar[B_SPGO]);
-          mma_commit_w(&bar[B_BCE + s]);
-          if (!ws_wait(&bar[B_SPF], ph_spf, abort_flag)) break;
-          ph_spf ^= 1;
-          tc_fence_after();
-          // Y_intra: Y^T += X'^T S'^T  (A = X'^T in tensor memory, B = S' K-major)
-#pragma unroll
-          for (int k = 0; k < 128 / 16; ++k)
-            mma_ts_w(tmem + C::TM_Y, tmem + C::TM_XP + 64 * xb + 8 * k, kdesc(sSP, k), C::ID_Y, 1);
-          mma_commit_w(&bar[B_YF]);
-          mma_commit_w(&bar[B_XBF + xb]);
-          if (i + 1 < ntl) {
-            if (!ws_wait(&bar[B_ROT + (s ^ 1)], ph_rot[s ^ 1], abort_flag)) break;
-            ph_rot.flip(s ^ 1);
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < N / 16; ++k)
-              mma_ss_w(tmem + C::TM_S, kdesc(sC(s ^ 1), k), kdesc(sB(s ^ 1), k), C::ID_S, k > 0);
-            mma_commit_w(&bar[B_SF]);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar[B_CE + cs]);
-      }
-      if (issued) {  // every MMA issued has completed before tensor memory is released
-        mma_commit_w(&bar[B_DRAIN]);
-        ws_wait_drain(&bar[B_DRAIN], 0);
-      }
-    } else if (FULL && warp >= W_MASK && warp < W_MASK + 4) {
-      // =============================================================== mask
-      const int q4 = warp & 3;
-      const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
-      const int row = 32 * q4 + lane;
-      const int t = row / R;
-      Phases ph_cf;
-      for (int i = 0; i < ntl; ++i) {
-        const int cs = i % WS_CS;
-        if (!ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag)) break;
-        ph_cf.flip(cs);
-        if (!ws_wait(&bar[B_SF], (uint32_t)(i & 1), abort_flag)) break;
-        tc_fence_after();
-        const float4* ra = recA(cs);
-        const bool fast = scal(cs)[0] != 0.0f;
-        const float4 rt4 = ra[t];
-        const float Lt2 = rt4.x * 1.4426950408889634f;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[16];
-          if (c > q4) {  // every column token is after every row token of this warp
-#pragma unroll
-            for (int e = 0; e < 16; ++e) o[e] = 0u;
-          } else {
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_base + C::TM_S + 32 * c, v);
-            tmem_wait_ld();
-            float f[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
-            if (!fast) {
-#pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                const int st = (32 * c + e) / R;
-                f[e] = (st <= t) ? f[e] * ex2_approx(Lt2 - ra[st].x * 1.4426950408889634f) : 0.0f;
+              for (int j = 0; j < C::CPT; ++j) {
+                const uint32_t off = (uint32_t)(rx ^ j) << 4;
+                sts128(rC + off, scale_chunk(lds128(rC + off), fc));
+                sts128(rB + off, scale_chunk(lds128(rB + off), fb));
               }
             }
-            if (c == q4) {  // the diagonal block: columns of the same token range as the rows
-#pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                const int st = (32 * c + e) / R;
-                f[e] = (st < t) ? f[e] : ((st == t) ? f[e] * rt4.y : 0.0f);
-              }
-            }
-#pragma unroll
-            for (int e = 0; e < 16; ++e) o[e] = pack_bf16(f[2 * e], f[2 * e + 1]);
-          }
-#pragma unroll
-          for (int qq = 0; qq < 4; ++qq) {
-            const int ch = 4 * c + qq;
-            const uint32_t off = (uint32_t)(ch >> 3) * BLK + (uint32_t)row * 128u +
-                                 ((uint32_t)((ch & 7) ^ (row & 7)) << 4);
-            sts128(sSP + off, make_uint4(o[4 * qq], o[4 * qq + 1], o[4 * qq + 2], o[4 * qq + 3]));
-          }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&bar[B_SPF]);
-          mbar_arrive(&bar[B_CE + cs]);
-        }
-      }
-    } else if (FULL && warp >= W_EPI && warp < W_EPI + 4) {
-      // =============================================================== epilogue
-      const int q4 = warp & 3;
-      const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
-      const int pc = 32 * q4 + lane;  // head-dim column of this thread
-      float wo[R];
-#pragma unroll
-      for (int r = 0; r < R; ++r) wo[r] = p.W_o ? p.W_o[((int64_t)hi * R + r) * WP + pc] : 1.0f;
-      const float Dh = p.D ? p.D[hi] : 0.0f;
-      __nv_bfloat16* yg = static_cast<__nv_bfloat16*>(p.y);
-      constexpr int TPC = 32 / R;  // tokens per 32-column chunk
-      for (int i = 0; i < ntl; ++i) {
-        const int64_t c0 = (j0 + i) * Q;
-        const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
-        if (!ws_wait(&bar[B_YF], (uint32_t)(i & 1), abort_flag)) break;
-        tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          float xv[TPC];
-#pragma unroll
-          for (int u = 0; u < TPC; ++u) {
-            const int t = TPC * c + u;
-            xv[u] = (p.D && t < nv) ? __bfloat162float(xg[((tok_base + c0 + t) * H + hi) * (int64_t)WP + pc]) : 0.0f;
-          }
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_base + C::TM_Y + 32 * c, v);
-          tmem_wait_ld();
-          if (c == 3) {
-            tc_fence_before();
+            fence_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[B_YE]);
+            if (lane == 0) mbar_arrive(&bar[B_RESC]);
           }
-#pragma unroll
-          for (int u = 0; u < TPC; ++u) {
-            const int t = TPC * c + u;
-            float acc = Dh * xv[u];
-#pragma unroll
-            for (int r = 0; r < R; ++r) acc = fmaf(wo[r], __uint_as_float(v[u * R + r]), acc);
-            if (t < nv) yg[((tok_base + c0 + t) * H + hi) * (int64_t)WP + pc] = __float2bfloat16_rn(acc);
+          if (lane == 0) mbar_arrive(&bar[B_CE + cs]);
+        }
+        // final angles of the segment: the full pass rotates the state back by them, the state
+        // pass stores them in its summary
+        named_bar_sync(BAR_ROT, 32 * N_ROT);
+        if (!*abort_flag) {
+          if constexpr (!FULL) {
+            if (aseg == 0) sg.ws_phi[((int64_t)bh * sg.nsub + seg) * K2 + ak] = base[ak];
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[B_FIN]);
         }
-      }
-    } else if (warp >= W_SPX && warp < W_SPX + 4) {
-      // =============================================================== state and inputs
-      const int q4 = warp & 3;
-      const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
-      const int pc = 32 * q4 + lane;
-      float wx[R];
-#pragma unroll
-      for (int r = 0; r < R; ++r) wx[r] = p.W_x ? p.W_x[((int64_t)hi * R + r) * WP + pc] : 1.0f;
-      Phases ph_cf, ph_xbf, ph_xf;
-      constexpr int TPC = 32 / R;
-      // X'^T of tile i: X'^T[p, tR + r] = W_x[r, p] x_t[p], bf16 pairs along the columns
-      auto build_xp = [&](int i) -> bool {
-        const int xb = i & 1;
-        if (i >= 2) {
-          if (!ws_wait(&bar[B_XBF + xb], ph_xbf[xb], abort_flag)) return false;
-          ph_xbf.flip(xb);
-        }
-        const int64_t c0 = (j0 + i) * Q;
-        const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
-        if (!ws_wait(&bar[B_XF + xb], ph_xf[xb], abort_flag)) return false;
-        ph_xf.flip(xb);
-        tc_fence_after();
-        const __nv_bfloat16* xs = reinterpret_cast<const __nv_bfloat16*>(sm + C::OFF_X + xb * C::XSLOT);
+    }
+  } else if (wg == 3) {
+    if (FULL && ntl > 0) {
+        // =============================================================== mask
+        const int q4 = warp & 3;
+        const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+        const int row = 32 * q4 + lane;
+        const int t = row / R;
+        Phases ph_cf;
+        for (int i = 0; i < ntl; ++i) {
+          const int cs = i % WS_CS;
+          if (!ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag)) break;
+          ph_cf.flip(cs);
+          if (!ws_wait(&bar[B_SF], (uint32_t)(i & 1), abort_flag)) break;
+          tc_fence_after();
+          const float4* ra = recA(cs);
+          const bool fast = scal(cs)[0] != 0.0f;
+          const float* rf = reinterpret_cast<const float*>(ra);  // scalar reads of the records
+          const float Lt2 = rf[4 * t] * 1.4426950408889634f;
+          const float dgt = rf[4 * t + 1];
 #pragma unroll 1
-        for (int gq = 0; gq < 4; ++gq) {
-          float xv[TPC];
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[16];
+            if (c > q4) {  // every column token is after every row token of this warp
 #pragma unroll
-          for (int u = 0; u < TPC; ++u) {
-            const int t = TPC * gq + u;
-            xv[u] = (t < nv) ? __bfloat162float(xs[t * WP + pc]) : 0.0f;
-          }
-          uint32_t w[16];
+              for (int e = 0; e < 16; ++e) o[e] = 0u;
+            } else {
+              uint32_t v[32];
+              tmem_ld32(tmem + lane_base + C::TM_S + 32 * c, v);
+              tmem_wait_ld();
+              float f[32];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c2 = 2 * e;  // column pair (c2, c2 + 1) of this 32-column group
-            w[e] = pack_bf16(wx[c2 % R] * xv[c2 / R], wx[(c2 + 1) % R] * xv[(c2 + 1) / R]);
+              for (int e = 0; e < 32; ++e) f[e] = __uint_as_float(v[e]);
+              if (!fast) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                  const int st = (32 * c + e) / R;
+                  f[e] = (st <= t) ? f[e] * ex2_approx(Lt2 - rf[4 * st] * 1.4426950408889634f) : 0.0f;
+                }
+              }
+              if (c == q4) {  // the diagonal block: column token e / R against the row's lane / R
+                const int lt = lane / R;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) f[e] = (e / R < lt) ? f[e] : ((e / R == lt) ? f[e] * dgt : 0.0f);
+              }
+#pragma unroll
+              for (int e = 0; e < 16; ++e) o[e] = pack_bf16(f[2 * e], f[2 * e + 1]);
+            }
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              const int ch = 4 * c + qq;
+              const uint32_t off = (uint32_t)(ch >> 3) * BLK + (uint32_t)row * 128u +
+                                   ((uint32_t)((ch & 7) ^ (row & 7)) << 4);
+              sts128(sSP + off, make_uint4(o[4 * qq], o[4 * qq + 1], o[4 * qq + 2], o[4 * qq + 3]));
+            }
           }
-          tmem_st16(tmem + lane_base + C::TM_XP + 64 * xb + 16 * gq, w);
+          fence_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&bar[B_SPF]);
+            mbar_arrive(&bar[B_CE + cs]);
+          }
         }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&bar[B_XPF + xb]);
-          mbar_arrive(&bar[B_XE + xb]);  // the x slot is read
-        }
-        return true;
-      };
-      bool ok = build_xp(0);
-      for (int i = 0; ok && i < ntl; ++i) {
-        const int cs = i % WS_CS;
-        if (!ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag)) break;
-        ph_cf.flip(cs);
-        const float fh = scal(cs)[3], fs = scal(cs)[4];
-        if (i == 0) {
-          // the rotated-frame state entering the segment (h+: it includes the previous token's
-          // trapezoid term beta'_0 u_{-1})
-          const bool from_state = FULL ? (seg == 0) : false;
-          const bool make_init = !FULL && seg == 0 && sg.write_init;
-          const bool fold = FULL && seg > 0;
-          const int nfold = fold ? seg * (sg.seg_tiles / sg.sub_tiles) : 0;
-          float bp0 = 0.0f, xprev[R];
-          if (from_state || make_init) {
-            const float l0 = p.raw_inputs ? fe_sigmoid(p.lam[tok_base * H + hi]) : p.lam[tok_base * H + hi];
-            const float d0 = p.raw_inputs ? fe_softplus(p.dt[tok_base * H + hi]) : p.dt[tok_base * H + hi];
-            bp0 = (1.0f - l0) * d0;
+    }
+  } else if (wg == 4) {
+    if (FULL && ntl > 0) {
+        // =============================================================== epilogue
+        const int q4 = warp & 3;
+        const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+        const int pc = 32 * q4 + lane;  // head-dim column of this thread
+        float wo[R];
 #pragma unroll
-            for (int r = 0; r < R; ++r) xprev[r] = wx[r] * p.carry_x[(int64_t)bh * WP + pc];
-          }
-          const float* h0 = p.h + (int64_t)bh * N * WP;
-          const float* cB = p.carry_B + (int64_t)bh * R * N;
-          const float* bB = p.bias_B ? p.bias_B + (int64_t)hi * R * N : nullptr;
+        for (int r = 0; r < R; ++r) wo[r] = p.W_o ? p.W_o[((int64_t)hi * R + r) * WP + pc] : 1.0f;
+        const float Dh = p.D ? p.D[hi] : 0.0f;
+        __nv_bfloat16* yg = static_cast<__nv_bfloat16*>(p.y);
+        constexpr int TPC = 16 / R;  // tokens per 16-column chunk
+        const int64_t tstride = (int64_t)H * WP;  // elements between consecutive tokens of y and x
+        Phases ph_cf;
+        for (int i = 0; i < ntl; ++i) {
+          const int cs = i % WS_CS;
+          const int64_t c0 = (j0 + i) * Q;
+          const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
+          if (!ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag)) break;
+          ph_cf.flip(cs);
+          if (!ws_wait(&bar[B_YF], (uint32_t)(i & 1), abort_flag)) break;
+          tc_fence_after();
+          const float* yc = ycol(cs);
+          const int64_t e0 = ((tok_base + c0) * H + hi) * (int64_t)WP + pc;
+          __nv_bfloat16* yrow = yg + e0;
+          const __nv_bfloat16* xrow = xg + e0;
+          const bool plain = (nv == Q) && (p.D == nullptr);  // a full tile without the skip term
 #pragma unroll 1
-          for (int c = 0; c < N / 32; ++c) {
-            float v[32];
+          for (int c = 0; c < 8; ++c) {
+            uint32_t v[16];
+            tmem_ld16(tmem + lane_base + C::TM_Y + 16 * c, v);
+            float a[TPC];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = 0.0f;
-            if (from_state || make_init) {
+            for (int u = 0; u < TPC; ++u) a[u] = yc[TPC * c + u];  // the column factors a_t
+            tmem_wait_ld();
+            if (c == 7) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bar[B_YE]);
+            }
+            __nv_bfloat16* yp = yrow + (int64_t)(TPC * c) * tstride;
+            if (plain) {
 #pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                const int n = 32 * c + e;
-                float u = 0.0f;
+              for (int u = 0; u < TPC; ++u) {
+                float acc = 0.0f;
 #pragma unroll
-                for (int r = 0; r < R; ++r) u = fmaf(cB[r * N + n] + (bB ? bB[r * N + n] : 0.0f), xprev[r], u);
-                v[e] = fmaf(bp0, u, h0[(int64_t)n * WP + pc]);
+                for (int r = 0; r < R; ++r) acc = fmaf(wo[r], __uint_as_float(v[u * R + r]), acc);
+                *yp = __float2bfloat16_rn(a[u] * acc);
+                yp += tstride;
               }
-              if (make_init) {
-                float* wi = sg.ws_init + (int64_t)bh * N * WP;
+            } else {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) wi[(int64_t)(32 * c + e) * WP + pc] = v[e];
+              for (int u = 0; u < TPC; ++u) {
+                const int t = TPC * c + u;
+                if (t < nv) {
+                  float acc = 0.0f;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = 0.0f;  // the state pass starts from zero
-              }
-            } else if (fold) {
-              const float* wi = sg.ws_init + (int64_t)bh * N * WP;
-#pragma unroll
-              for (int e = 0; e < 32; ++e) v[e] = wi[(int64_t)(32 * c + e) * WP + pc];
-              for (int k = 0; k < nfold; ++k) {
-                const int64_t sidx = (int64_t)bh * sg.nsub + k;
-                const float dec = __expf(sg.ws_l[sidx]);
-                const float* wh = sg.ws_h + sidx * N * WP;
-                const double* ph = sg.ws_phi + sidx * K2;
-#pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                  const int n0 = 32 * c + 2 * e;
-                  float sn, cn;
-                  sincosf((float)ph[n0 / 2], &sn, &cn);
-                  const float a0 = fmaf(dec, v[2 * e], wh[(int64_t)n0 * WP + pc]);
-                  const float a1 = fmaf(dec, v[2 * e + 1], wh[(int64_t)(n0 + 1) * WP + pc]);
-                  v[2 * e] = cn * a0 - sn * a1;
-                  v[2 * e + 1] = sn * a0 + cn * a1;
+                  for (int r = 0; r < R; ++r) acc = fmaf(wo[r], __uint_as_float(v[u * R + r]), acc);
+                  const float dx = p.D ? Dh * __bfloat162float(xrow[t * tstride]) : 0.0f;
+                  yp[u * tstride] = __float2bfloat16_rn(fmaf(a[u], acc, dx));
                 }
               }
             }
-            uint32_t u32[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) u32[e] = __float_as_uint(fs * v[e]);
-            tmem_st32(tmem + lane_base + C::TM_ST + 32 * c, u32);
-            if constexpr (FULL) hb_store_row(sHB, pc, c, v, fh);
           }
-        } else {
-          if (!ws_wait(&bar[B_SPGO], (uint32_t)((i - 1) & 1), abort_flag)) break;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar[B_CE + cs]);
+        }
+    }
+  } else {
+    if (ntl > 0) {
+        // =============================================================== state and inputs
+        const int q4 = warp & 3;
+        const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+        const int pc = 32 * q4 + lane;
+        float wx[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) wx[r] = p.W_x ? p.W_x[((int64_t)hi * R + r) * WP + pc] : 1.0f;
+        Phases ph_cf, ph_xbf, ph_xf;
+        constexpr int TPC = 32 / R;
+        // X'^T of tile i: X'^T[p, tR + r] = W_x[r, p] x_t[p], bf16 pairs along the columns
+        auto build_xp = [&](int i) -> bool {
+          const int xb = i & 1, cs = i % WS_CS;
+          if (i >= 2) {
+            if (!ws_wait(&bar[B_XBF + xb], ph_xbf[xb], abort_flag)) return false;
+            ph_xbf.flip(xb);
+          }
+          const int64_t c0 = (j0 + i) * Q;
+          const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
+          // the tile's X' factors (the main loop waits for the same phase of this slot again)
+          if (!ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag)) return false;
+          if (!ws_wait(&bar[B_XF], ph_xf[0], abort_flag)) return false;
+          ph_xf.flip(0);
           tc_fence_after();
+          const __nv_bfloat16* xs = reinterpret_cast<const __nv_bfloat16*>(sm + C::OFF_X);
+          const float4* ra = recA(cs);
 #pragma unroll 1
-          for (int c = 0; c < N / 32; ++c) {
-            uint32_t u32[32];
-            tmem_ld32(tmem + lane_base + C::TM_ST + 32 * c, u32);
-            tmem_wait_ld();
-            float v[32];
+          for (int gq = 0; gq < 4; ++gq) {
+            float xv[TPC];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              v[e] = __uint_as_float(u32[e]);
-              u32[e] = __float_as_uint(fs * v[e]);
+            for (int u = 0; u < TPC; ++u) {
+              const int t = TPC * gq + u;
+              xv[u] = (t < nv) ? reinterpret_cast<const float*>(ra)[4 * t + 2] * __bfloat162float(xs[t * WP + pc]) : 0.0f;
             }
-            tmem_st32(tmem + lane_base + C::TM_ST + 32 * c, u32);
-            if constexpr (FULL) hb_store_row(sHB, pc, c, v, fh);
+            uint32_t w[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int c2 = 2 * e;  // column pair (c2, c2 + 1) of this 32-column group
+              w[e] = pack_bf16(wx[c2 % R] * xv[c2 / R], wx[(c2 + 1) % R] * xv[(c2 + 1) / R]);
+            }
+            tmem_st16(tmem + lane_base + C::TM_XP + 64 * xb + 16 * gq, w);
           }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&bar[B_XPF + xb]);
+            mbar_arrive(&bar[B_XE]);  // the x slot is read
+          }
+          return true;
+        };
+        bool ok = build_xp(0);
+        for (int i = 0; ok && i < ntl; ++i) {
+          const int cs = i % WS_CS;
+          if (!ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag)) break;
+          ph_cf.flip(cs);
+          const float fh = scal(cs)[3], fs = scal(cs)[4];
+          if (i == 0) {
+            // the rotated-frame state entering the segment (h+: it includes the previous token's
+            // trapezoid term beta'_0 u_{-1})
+            const bool from_state = FULL ? (seg == 0) : false;
+            const bool make_init = !FULL && seg == 0 && sg.write_init;
+            const bool fold = FULL && seg > 0;
+            const int nfold = fold ? seg * (sg.seg_tiles / sg.sub_tiles) : 0;
+            float bp0 = 0.0f, xprev[R];
+            if (from_state || make_init) {
+              const float l0 = p.raw_inputs ? fe_sigmoid(p.lam[tok_base * H + hi]) : p.lam[tok_base * H + hi];
+              const float d0 = p.raw_inputs ? fe_softplus(p.dt[tok_base * H + hi]) : p.dt[tok_base * H + hi];
+              bp0 = (1.0f - l0) * d0;
+#pragma unroll
+              for (int r = 0; r < R; ++r) xprev[r] = wx[r] * p.carry_x[(int64_t)bh * WP + pc];
+            }
+            const float* h0 = p.h + (int64_t)bh * N * WP;
+            const float* cB = p.carry_B + (int64_t)bh * R * N;
+            const float* bB = p.bias_B ? p.bias_B + (int64_t)hi * R * N : nullptr;
+#pragma unroll 1
+            for (int c = 0; c < N / 32; ++c) {
+              float v[32];
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] = 0.0f;
+              if (from_state || make_init) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                  const int n = 32 * c + e;
+                  float u = 0.0f;
+#pragma unroll
+                  for (int r = 0; r < R; ++r) u = fmaf(cB[r * N + n] + (bB ? bB[r * N + n] : 0.0f), xprev[r], u);
+                  v[e] = fmaf(bp0, u, h0[(int64_t)n * WP + pc]);
+                }
+                if (make_init) {
+                  float* wi = sg.ws_init + (int64_t)bh * N * WP;
+#pragma unroll
+                  for (int e = 0; e < 32; ++e) wi[(int64_t)(32 * c + e) * WP + pc] = v[e];
+#pragma unroll
+                  for (int e = 0; e < 32; ++e) v[e] = 0.0f;  // the state pass starts from zero
+                }
+              } else if (fold) {
+                const float* wi = sg.ws_init + (int64_t)bh * N * WP;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = wi[(int64_t)(32 * c + e) * WP + pc];
+                for (int k = 0; k < nfold; ++k) {
+                  const int64_t sidx = (int64_t)bh * sg.nsub + k;
+                  const float dec = __expf(sg.ws_l[sidx]);
+                  const float* wh = sg.ws_h + sidx * N * WP;
+                  const double* ph = sg.ws_phi + sidx * K2;
+#pragma unroll
+                  for (int e = 0; e < 16; ++e) {
+                    const int n0 = 32 * c + 2 * e;
+                    float sn, cn;
+                    sincosf((float)ph[n0 / 2], &sn, &cn);
+                    const float a0 = fmaf(dec, v[2 * e], wh[(int64_t)n0 * WP + pc]);
+                    const float a1 = fmaf(dec, v[2 * e + 1], wh[(int64_t)(n0 + 1) * WP + pc]);
+                    v[2 * e] = cn * a0 - sn * a1;
+                    v[2 * e + 1] = sn * a0 + cn * a1;
+                  }
+                }
+              }
+              uint32_t u32[32];
+#pragma unroll
+              for (int e = 0; e < 32; ++e) u32[e] = __float_as_uint(v[e]);
+              if constexpr (FULL) hb_store_row(sHB, pc, c, u32, fh);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) u32[e] = __float_as_uint(fs * v[e]);
+              tmem_st32(tmem + lane_base + C::TM_ST + 32 * c, u32);
+            }
+          } else {
+            if (!ws_wait(&bar[B_SPGO], (uint32_t)((i - 1) & 1), abort_flag)) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < N / 32; ++c) {
+              uint32_t u32[32];
+              tmem_ld32(tmem + lane_base + C::TM_ST + 32 * c, u32);
+              tmem_wait_ld();
+              if constexpr (FULL) hb_store_row(sHB, pc, c, u32, fh);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {  // the rescale in f32x2 pairs, in place
+                float a, b;
+                f2_split(f2_mul(f2(fs, fs), f2(__uint_as_float(u32[2 * e]), __uint_as_float(u32[2 * e + 1]))), a, b);
+                u32[2 * e] = __float_as_uint(a);
+                u32[2 * e + 1] = __float_as_uint(b);
+              }
+              tmem_st32(tmem + lane_base + C::TM_ST + 32 * c, u32);
+            }
+          }
+          tmem_wait_st();
+          fence_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&bar[B_HF]);
+            mbar_arrive(&bar[B_CE + cs]);
+          }
+          if (i + 1 < ntl) ok = build_xp(i + 1);
         }
-        tmem_wait_st();
-        fence_async_smem();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&bar[B_HF]);
-          mbar_arrive(&bar[B_CE + cs]);
-        }
-        if (i + 1 < ntl) ok = build_xp(i + 1);
-      }
-      // ---- results: the state after the last tile
-      bool go = ok && !*abort_flag && (!FULL || last_seg);
-      if (go) go = ws_wait(&bar[B_SPGO], (uint32_t)((ntl - 1) & 1), abort_flag);
-      if (FULL && go) go = ws_wait(&bar[B_FIN], 0, abort_flag);
-      // the raw-input carry below synchronises the four state warps: they decide together
-      if (FULL && last_seg && p.raw_inputs && bar_any(BAR_SPX, 128, !go)) go = false;
-      if (go) {
-        tc_fence_after();
-        const float inv_rho = scal((ntl - 1) % WS_CS)[5];
-        if constexpr (FULL) {
-          // rotate back from the segment frame by the segment's total angle
-          {
-            float* hout = p.h + (int64_t)bh * N * WP;
+        // ---- results: the state after the last tile
+        bool go = ok && !*abort_flag && (!FULL || last_seg);
+        if (go) go = ws_wait(&bar[B_SPGO], (uint32_t)((ntl - 1) & 1), abort_flag);
+        if (FULL && go) go = ws_wait(&bar[B_FIN], 0, abort_flag);
+        // the raw-input carry below synchronises the four state warps: they decide together
+        if (FULL && last_seg && p.raw_inputs && bar_any(BAR_SPX, 128, !go)) go = false;
+        if (go) {
+          tc_fence_after();
+          const float inv_rho = scal((ntl - 1) % WS_CS)[5];
+          if constexpr (FULL) {
+            // rotate back from the segment frame by the segment's total angle
+            {
+              float* hout = p.h + (int64_t)bh * N * WP;
+#pragma unroll 1
+              for (int c = 0; c < N / 32; ++c) {
+                uint32_t sv[32];
+                tmem_ld32(tmem + lane_base + C::TM_ST + 32 * c, sv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                  const int k = 16 * c + e;
+                  float sn, cn;
+                  sincosf((float)base[k], &sn, &cn);
+                  const float a0 = inv_rho * __uint_as_float(sv[2 * e]);
+                  const float a1 = inv_rho * __uint_as_float(sv[2 * e + 1]);
+                  hout[(int64_t)(2 * k) * WP + pc] = cn * a0 - sn * a1;
+                  hout[(int64_t)(2 * k + 1) * WP + pc] = sn * a0 + cn * a1;
+                }
+              }
+              // the carry: the last token's B (as the core used it: normalised when the operands are
+              // raw) and raw x
+              const int64_t tokl = tok_base + (L - 1);
+              const __nv_bfloat16* Bg = static_cast<const __nv_bfloat16*>(p.B);
+              const int64_t bc = ((tokl * G + g) * R) * (int64_t)N;
+              if (p.raw_inputs) {  // the rotation warps are done with rowss (B_FIN)
+                if (pc < R) rowss[pc] = 0.0f;
+                named_bar_sync(BAR_SPX, 128);
+                for (int k = pc; k < R * N; k += WP) {
+                  const float v = __bfloat162float(Bg[bc + k]);
+                  atomicAdd(&rowss[k / N], v * v);
+                }
+                named_bar_sync(BAR_SPX, 128);
+              }
+              for (int k = pc; k < R * N; k += WP) {
+                float v = __bfloat162float(Bg[bc + k]);
+                if (p.raw_inputs) v *= rsqrtf(rowss[k / N] * (1.0f / N) + kBcNormEps);
+                p.carry_B[(int64_t)bh * R * N + k] = v;
+              }
+              p.carry_x[(int64_t)bh * WP + pc] = __bfloat162float(xg[(tokl * H + hi) * (int64_t)WP + pc]);
+            }
+          } else {
+            float* wh = sg.ws_h + ((int64_t)bh * sg.nsub + seg) * N * WP;
 #pragma unroll 1
             for (int c = 0; c < N / 32; ++c) {
               uint32_t sv[32];
               tmem_ld32(tmem + lane_base + C::TM_ST + 32 * c, sv);
               tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const int k = 16 * c + e;
-                float sn, cn;
-                sincosf((float)base[k], &sn, &cn);
-                const float a0 = inv_rho * __uint_as_float(sv[2 * e]);
-                const float a1 = inv_rho * __uint_as_float(sv[2 * e + 1]);
-                hout[(int64_t)(2 * k) * WP + pc] = cn * a0 - sn * a1;
-                hout[(int64_t)(2 * k + 1) * WP + pc] = sn * a0 + cn * a1;
-              }
+              for (int e = 0; e < 32; ++e) wh[(int64_t)(32 * c + e) * WP + pc] = inv_rho * __uint_as_float(sv[e]);
             }
-            // the carry: the last token's B (as the core used it: normalised when the operands are
-            // raw) and raw x
-            const int64_t tokl = tok_base + (L - 1);
-            const __nv_bfloat16* Bg = static_cast<const __nv_bfloat16*>(p.B);
-            const int64_t bc = ((tokl * G + g) * R) * (int64_t)N;
-            if (p.raw_inputs) {  // the rotation warps are done with rowss (B_FIN)
-              if (pc < R) rowss[pc] = 0.0f;
-              named_bar_sync(BAR_SPX, 128);
-              for (int k = pc; k < R * N; k += WP) {
-                const float v = __bfloat162float(Bg[bc + k]);
-                atomicAdd(&rowss[k / N], v * v);
-              }
-              named_bar_sync(BAR_SPX, 128);
-            }
-            for (int k = pc; k < R * N; k += WP) {
-              float v = __bfloat162float(Bg[bc + k]);
-              if (p.raw_inputs) v *= rsqrtf(rowss[k / N] * (1.0f / N) + kBcNormEps);
-              p.carry_B[(int64_t)bh * R * N + k] = v;
-            }
-            p.carry_x[(int64_t)bh * WP + pc] = __bfloat162float(xg[(tokl * H + hi) * (int64_t)WP + pc]);
-          }
-        } else {
-          float* wh = sg.ws_h + ((int64_t)bh * sg.nsub + seg) * N * WP;
-#pragma unroll 1
-          for (int c = 0; c < N / 32; ++c) {
-            uint32_t sv[32];
-            tmem_ld32(tmem + lane_base + C::TM_ST + 32 * c, sv);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) wh[(int64_t)(32 * c + e) * WP + pc] = inv_rho * __uint_as_float(sv[e]);
           }
         }
-      }
     }
   }
 

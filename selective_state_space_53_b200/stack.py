@@ -3,24 +3,26 @@ page-1 article ("Mamba3をゼロから実装して...": 12 pure Mamba-3 layers, 
 MIMO rank 2, d_state 64, chunk 32).
 
 Only the SSM core is this library's product, and every step of it runs in libm3
-(``m3.scan`` -> m3_scan_fwd).  The block around the core is plain torch with random-init
-weights, so that the core runs, and is timed, on inputs shaped the way the full model makes
-them:
+(``m3.scan`` -> m3_scan_fwd with M3_FLAG_RAW_INPUTS, so the core also applies the block's
+front-end: BCNorm of B and C, softplus, -exp and sigmoid).  The block around the core is
+plain torch with random-init weights, so that the core runs, and is timed, on inputs shaped
+the way the full model makes them:
 
 * pre-norm: RMSNorm of the residual stream (weight 1);
-* input projection (one bf16 GEMM, weights N(0, 0.02)) to x, the gate z, B and C (R ranks of
-  N per group), and per-head pre-activations of Delta, A and lambda, and per-group rotation
-  angles theta;
-* B and C normalised over N (BCNorm; the core adds the 0.02 bias, docsaid note on Mamba-3,
-  section アーキテクチャ), Delta = softplus(. - 2), A = -exp(. + 0.5), lambda = sigmoid(.),
-  theta used as produced (radians);
-* the core, y = Mamba-3 SSM(x, Delta, A, lambda, B, C, theta) with D = 1;
+* input projections (bf16 GEMMs, weights N(0, 0.02)), one per operand so that each lands
+  contiguous in the layout the core reads: x, the gate z, B and C (R ranks of N per group),
+  and one fp32 projection with a bias for the per-head pre-activations of Delta, A and lambda
+  and the per-group rotation angles theta;
+* the core on the raw projections: B and C normalised over N (BCNorm, after which the core
+  adds the 0.02 bias; docsaid note on Mamba-3, section アーキテクチャ), Delta =
+  softplus(dt_raw), A = -exp(A_raw), lambda = sigmoid(lam_raw), theta used as produced
+  (radians), D = 1;
 * gate y * silu(z), output projection (bf16 GEMM, N(0, 0.02)) and the residual add.
 
-The pages fix the shapes and the core; the block's details (pre-norm, the -2 / +0.5 offsets,
-which put Delta and A in the same ranges as the layer workloads' draws) are this harness's
-readings and do not enter any parity claim: parity is checked on the core of every layer, with
-the inputs this harness produced.
+The pages fix the shapes and the core; the block's details (pre-norm, the projection bias of
+-2 on dt_raw and +0.5 on A_raw, which put Delta and A in the same ranges as the layer
+workloads' draws) are this harness's readings and do not enter any parity claim: parity is
+checked on the core of every layer, with the raw inputs this harness produced.
 """
 
 from __future__ import annotations
@@ -66,56 +68,66 @@ class Mamba3Stack:
         g = torch.Generator(device="cpu").manual_seed(seed)
         cols, width = shape.split()
         self.cols, self.width = cols, width
+        H = shape.H
         self.layers = []
         for _ in range(shape.layers):
-            w_in = (0.02 * torch.randn(shape.d_model, width, generator=g)).to(torch.bfloat16)
+            w_in = 0.02 * torch.randn(shape.d_model, width, generator=g)
             w_out = (0.02 * torch.randn(shape.d_inner, shape.d_model, generator=g)).to(torch.bfloat16)
             W_x = 1.0 + 0.1 * torch.randn(shape.H, shape.R, shape.P, generator=g)
             W_o = (1.0 + 0.1 * torch.randn(shape.H, shape.R, shape.P, generator=g)) / shape.R
+
+            def block(*keys, dtype=torch.bfloat16):
+                return torch.cat([w_in[:, cols[k][0]:cols[k][1]] for k in keys], 1).to(dtype).contiguous().to(device)
+
+            # per-head scalars and angles: [dt | A | lam | theta], one fp32 GEMM with the offsets as bias
+            s_bias = torch.zeros(3 * H + shape.G * shape.N // 2)
+            s_bias[:H] = -2.0
+            s_bias[H:2 * H] = 0.5
             self.layers.append(dict(
-                w_in=w_in.to(device), w_out=w_out.to(device),
+                w_x=block("x"), w_z=block("z"), w_B=block("B"), w_C=block("C"),
+                w_s=block("dt", "A", "lam", "theta", dtype=torch.float32), s_bias=s_bias.to(device),
+                w_out=w_out.to(device),
                 bias_B=torch.full((shape.H, shape.R, shape.N), 0.02, device=device),
                 bias_C=torch.full((shape.H, shape.R, shape.N), 0.02, device=device),
                 W_x=W_x.to(device).contiguous(), W_o=W_o.to(device).contiguous(),
                 D=torch.ones(shape.H, device=device)))
         self._ws = {}
 
+    def dims(self, b, L):
+        s = self.s
+        return m3.make_dims(b, L, s.H, s.P, s.N, s.R, s.G, "bf16", flags=m3.M3_FLAG_RAW_INPUTS)
+
     def core_inputs(self, u, layer):
-        """The core's operands for residual stream u (b, L, d_model) bf16 at one layer."""
+        """The core's raw operands for residual stream u (b, L, d_model) bf16 at one layer, and
+        the gate z."""
         import torch
-        import torch.nn.functional as F
-        s, c = self.s, self.cols
+        s = self.s
         b, L, _ = u.shape
+        H = s.H
         uf = u.float()
-        h = (uf * torch.rsqrt(uf.pow(2).mean(-1, keepdim=True) + 1e-6)).to(torch.bfloat16)
-        proj = (h.view(b * L, -1) @ layer["w_in"]).view(b, L, -1)
-
-        def part(k):
-            return proj[..., c[k][0]:c[k][1]]
-
-        def bcnorm(t):
-            t = t.float().view(b, L, s.G, s.R, s.N)
-            return (t * torch.rsqrt(t.pow(2).mean(-1, keepdim=True) + 1e-6)).to(torch.bfloat16).contiguous()
-
+        h = (uf * torch.rsqrt(uf.pow(2).mean(-1, keepdim=True) + 1e-6)).to(torch.bfloat16).view(b * L, -1)
+        sc = torch.addmm(layer["s_bias"], h.float(), layer["w_s"])
         dev = dict(
-            x=part("x").contiguous().view(b, L, s.H, s.P),
-            dt=F.softplus(part("dt").float() - 2.0).contiguous(),
-            A=(-torch.exp(part("A").float() + 0.5)).contiguous(),
-            lam=torch.sigmoid(part("lam").float()).contiguous(),
-            B=bcnorm(part("B")), C=bcnorm(part("C")),
-            theta=part("theta").float().contiguous().view(b, L, s.G, s.N // 2),
+            x=(h @ layer["w_x"]).view(b, L, s.H, s.P),
+            dt=sc[:, :H].contiguous().view(b, L, H),
+            A=sc[:, H:2 * H].contiguous().view(b, L, H),
+            lam=sc[:, 2 * H:3 * H].contiguous().view(b, L, H),
+            B=(h @ layer["w_B"]).view(b, L, s.G, s.R, s.N),
+            C=(h @ layer["w_C"]).view(b, L, s.G, s.R, s.N),
+            theta=sc[:, 3 * H:].contiguous().view(b, L, s.G, s.N // 2),
             bias_B=layer["bias_B"], bias_C=layer["bias_C"], W_x=layer["W_x"], W_o=layer["W_o"],
             D=layer["D"])
-        return dev, part("z")
+        z = (h @ layer["w_z"]).view(b, L, -1)
+        return dev, z
 
     def forward(self, u, check=None):
         """The stack on residual stream u (b, L, d_model) bf16; returns the final stream.
-        check(layer_index, core_operands, y) is called after each layer's core, if given."""
+        check(layer_index, core_operands, y) is called after each layer's core, if given
+        (the operands are the raw projections the core's front-end consumed)."""
         import torch
         import torch.nn.functional as F
-        s = self.s
         b, L, _ = u.shape
-        dims = m3.make_dims(b, L, s.H, s.P, s.N, s.R, s.G, "bf16")
+        dims = self.dims(b, L)
         key = (b, L)
         if key not in self._ws:
             n = m3.m3_scan_workspace_size(dims)

@@ -1,8 +1,10 @@
 """GPU parity of the core inside the 12-layer stack (b8 L4096, the page-1 language-model shape).
 
-Every layer's core (m3_scan_fwd through the C ABI) is compared with the fp64 oracle on sampled
-(batch, head) sequences of that layer, on the operands the stack produced for it: the inputs
-of deeper layers come from the residual stream of the model, not from the seeded generator.
+Every layer's core (m3_scan_fwd with M3_FLAG_RAW_INPUTS through the C ABI: the core applies the
+block's front-end itself) is compared with the fp64 oracle composed with the oracle's front-end
+on sampled (batch, head) sequences of that layer, on the raw operands the stack produced for it:
+the inputs of deeper layers come from the residual stream of the model, not from the seeded
+generator.
 Tolerance as for every bf16 case: max relative error 2e-2 per output tensor.
 """
 
@@ -43,7 +45,8 @@ def pair_inputs(dev, bi, hi, shape, L):
         B=host(dev["B"][bi:bi + 1, :, g:g + 1]),
         C=host(dev["C"][bi:bi + 1, :, g:g + 1]),
         bias_B=host(dev["bias_B"][hi:hi + 1]), bias_C=host(dev["bias_C"][hi:hi + 1]),
-        W_x=host(dev["W_x"][hi:hi + 1]), W_o=host(dev["W_o"][hi:hi + 1]), D=host(dev["D"][hi:hi + 1]))
+        W_x=host(dev["W_x"][hi:hi + 1]), W_o=host(dev["W_o"][hi:hi + 1]), D=host(dev["D"][hi:hi + 1]),
+        extra={"raw": True})
 
 
 def test_twelve_layer_stack_core_parity():
@@ -59,7 +62,7 @@ def test_twelve_layer_stack_core_parity():
     def check(li, dev, y):
         pairs = [(int(rng.integers(b)), int(rng.integers(shape.H))) for _ in range(2)]
         for bi, hi in pairs:
-            inp = pair_inputs(dev, bi, hi, shape, L)
+            inp = orc.frontend(pair_inputs(dev, bi, hi, shape, L))
             yr, _, _, _ = orc.scan_inputs(inp)
             got = y[bi:bi + 1, :, hi:hi + 1].float().cpu().numpy()
             errs.append((li, bi, hi, rel_err(got, yr)))
