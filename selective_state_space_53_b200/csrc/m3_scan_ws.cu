@@ -104,7 +104,7 @@ struct WsCfg {
   static constexpr int Q = 128 / R;
   static constexpr int K2 = N / 2;
   static constexpr int NKC = N / 8;                    // 16-byte chunks of a row
-  static constexpr int CPT = NKC / 2;                  // chunks of a row per rotation thread (two per row)
+  static constexpr int KCW = NKC / N_ROT;              // chunks per rotation warp
   static constexpr int TILE_N = 128 * N * 2;           // a B or C tile, bytes
   static constexpr int BLK = 128 * 128;                // one 64-column block of a 128-row SW128 tile
   static constexpr int STAGE = 2 * TILE_N;             // B then C
@@ -123,8 +123,8 @@ struct WsCfg {
   static constexpr int OFF_BASE = OFF_SEGSUM + SEGS * K2 * 4;    // double [K2]
   static constexpr int REC_SLOT = Q * 24 + 64;  // float4 rec[Q], float mult[Q], float ycol[Q], float scal[16]
   static constexpr int OFF_REC = OFF_BASE + K2 * 8;
-  static constexpr int OFF_ROWSS = OFF_REC + WS_CS * REC_SLOT;    // float [2][2][128]: half-row sums of squares
-  static constexpr int OFF_BAR = OFF_ROWSS + 4 * 128 * 4;
+  static constexpr int OFF_ROWSS = OFF_REC + WS_CS * REC_SLOT;    // float [2][128]: B, C row sums of squares
+  static constexpr int OFF_BAR = OFF_ROWSS + 2 * 128 * 4;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM = BYTES + 1024;
@@ -134,7 +134,7 @@ struct WsCfg {
   static constexpr uint32_t ID_Y = idesc_bf16(WP, 128, false, false);
   static constexpr uint32_t ID_H = idesc_bf16(WP, N, false, true);
   static_assert(Q % SEGS == 0 && SEGLEN >= 1, "angle segments");
-  static_assert(2 * 128 == 32 * N_ROT && (CPT == 8 || CPT == 4), "rotation threads: a row half each");
+  static_assert(NKC % N_ROT == 0, "rotation chunks");
   static_assert(TM_XP + 128 <= TM_COLS, "tensor memory");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
@@ -578,10 +578,8 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
         const int rt = tid - 32 * W_ROT;
         const int wr = warp - W_ROT;
         const int ak = rt % K2, aseg = rt / K2;  // angles: pair ak over token segment aseg
-        // rotation: row rrow, chunks kc0 .. kc0 + CPT - 1 (lanes take 32 consecutive rows)
-        const int rrow = rt & 127, kc0 = (rt >> 7) * C::CPT, rr = rrow % R;
-        const int rx = (kc0 & 7) ^ (rrow & 7);  // swizzled chunk j of the row is chunk rx ^ j
-        const uint32_t rbase = (uint32_t)(kc0 >> 3) * BLK + (uint32_t)rrow * 128u;
+        // rotation: chunks kc = wr + N_ROT q of rows 32 step + lane (the branch r = lane % R is fixed)
+        const int rr = lane % R;
         // the biases of the head, staged once as fp32 in the pair layout of rotate16
         float* sbias = reinterpret_cast<float*>(sm + C::OFF_BIAS);
         for (int e = rt; e < 2 * R * N; e += 32 * N_ROT) {
@@ -594,12 +592,11 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
         const float* biasC = sbias + (R + rr) * C::BIAS_ROW;
         float thr[C::SEGLEN];
         auto load_theta = [&](int64_t j) {
-          const int64_t c0 = j * Q;
+          const int64_t t0 = j * Q + aseg * C::SEGLEN;  // first token of this thread's segment
+          const float* th = p.theta + ((tok_base + t0) * G + g) * K2 + ak;
+          const int nth = (int)(L - t0 < C::SEGLEN ? (L - t0 > 0 ? L - t0 : 0) : C::SEGLEN);
 #pragma unroll
-          for (int e = 0; e < C::SEGLEN; ++e) {
-            const int t = aseg * C::SEGLEN + e;
-            thr[e] = (c0 + t < L) ? p.theta[((tok_base + c0 + t) * G + g) * K2 + ak] : 0.0f;
-          }
+          for (int e = 0; e < C::SEGLEN; ++e) thr[e] = (e < nth) ? __ldg(th + e * G * K2) : 0.0f;
         };
         load_theta(j0);
         Phases ph_cf, ph_bcf;
@@ -611,8 +608,6 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
           const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
           bool okw = ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag);
           ph_cf.flip(cs);
-          okw = okw && ws_wait(&bar[B_BCF + s], ph_bcf[s], abort_flag);
-          ph_bcf.flip(s);
           if (bar_any(BAR_ROT, 32 * N_ROT, !okw || *abort_flag)) break;  // the group stops together
           const float* mu = mult(cs);
           const float4* ra = recA(cs);
@@ -651,63 +646,80 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
             }
           }
           if (i + 1 < ntl) load_theta(j + 1);
-          named_bar_sync(BAR_ROT, 32 * N_ROT);  // table complete; base and segsum read
+          // the angles needed no B or C: their copy lands meanwhile
+          okw = ws_wait(&bar[B_BCF + s], ph_bcf[s], abort_flag);
+          ph_bcf.flip(s);
+          // table complete, base and segsum read, the tile's B and C in place
+          if (bar_any(BAR_ROT, 32 * N_ROT, !okw || *abort_flag)) break;
           if (aseg == 0) {
             double nb = base[ak] + tot;
             nb -= 6.283185307179586 * rint(nb * 0.15915494309189535);
             base[ak] = nb;
           }
-          // ---- rotate Bt (and Ct) of the tile in place: this thread's row, chunks kc0 ..
-          {
-            const int t = rrow / R;
-            const bool valid = t < nv;
-            const uint32_t rB = sB(s) + rbase, rC = sC(s) + rbase;
-            float nb = 1.0f, nc = 1.0f;
-            if (p.raw_inputs) {
-              // the fused B/C RMS norm: each half row's sum of squares, then the row's
-              float ssb = 0.0f, ssc = 0.0f;
-              if (valid) {
+          if (p.raw_inputs) {
+            // the fused B/C RMS norm: every row's sum of squares over N, from each warp's chunks
+            rowss[rt] = 0.0f;
+            named_bar_sync(BAR_ROT, 32 * N_ROT);
+#pragma unroll 1
+            for (int q = 0; q < C::KCW; ++q) {
+              const int kc = wr + N_ROT * q;
+              const uint32_t cb = (uint32_t)(kc >> 3) * BLK + (uint32_t)lane * 128u + ((uint32_t)((kc & 7) ^ (lane & 7)) << 4);
+              for (int step = 0; step < 4; ++step) {
+                const int row = 32 * step + lane;
+                if (row / R >= nv) continue;
+                float f[8], ss = 0.0f;
+                unpack8(lds128(sB(s) + cb + step * 4096), f);
 #pragma unroll
-                for (int j = 0; j < C::CPT; ++j) {
-                  const uint32_t off = (uint32_t)(rx ^ j) << 4;
-                  float f[8];
-                  unpack8(lds128(rB + off), f);
+                for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+                atomicAdd(&rowss[row], ss);
+                if constexpr (FULL) {
+                  unpack8(lds128(sC(s) + cb + step * 4096), f);
+                  ss = 0.0f;
 #pragma unroll
-                  for (int e = 0; e < 8; ++e) ssb = fmaf(f[e], f[e], ssb);
-                  if constexpr (FULL) {
-                    unpack8(lds128(rC + off), f);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) ssc = fmaf(f[e], f[e], ssc);
-                  }
+                  for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+                  atomicAdd(&rowss[128 + row], ss);
                 }
               }
-              rowss[(2 * (kc0 != 0) + 0) * 128 + rrow] = ssb;
-              rowss[(2 * (kc0 != 0) + 1) * 128 + rrow] = ssc;
-              named_bar_sync(BAR_ROT, 32 * N_ROT);
-              nb = rsqrtf((rowss[rrow] + rowss[256 + rrow]) * (1.0f / N) + kBcNormEps);
-              nc = rsqrtf((rowss[128 + rrow] + rowss[384 + rrow]) * (1.0f / N) + kBcNormEps);
             }
-            const uint8_t* trow = tab + t * C::TAB_ROW;
-            const uint64_t nb2 = f2(nb, nb), nc2 = f2(nc, nc);
-#pragma unroll
-            for (int j = 0; j < C::CPT; ++j) {
-              const int kc = kc0 + j;
-              const uint32_t off = (uint32_t)(rx ^ j) << 4;
-              if (valid) {
-                const RotCS rcs = rot_cs(*reinterpret_cast<const uint4*>(trow + kc * 16));
-                const float4 be = *reinterpret_cast<const float4*>(biasB + kc * 8);
-                const float4 bo = *reinterpret_cast<const float4*>(biasB + kc * 8 + 4);
-                sts128(rB + off, rotate16(lds128(rB + off), rcs, nb2, f2(be.x, be.y), f2(be.z, be.w), f2(bo.x, bo.y),
-                                          f2(bo.z, bo.w)));
-                if constexpr (FULL) {
-                  const float4 ce = *reinterpret_cast<const float4*>(biasC + kc * 8);
-                  const float4 co = *reinterpret_cast<const float4*>(biasC + kc * 8 + 4);
-                  sts128(rC + off, rotate16(lds128(rC + off), rcs, nc2, f2(ce.x, ce.y), f2(ce.z, ce.w),
-                                            f2(co.x, co.y), f2(co.z, co.w)));
+            named_bar_sync(BAR_ROT, 32 * N_ROT);
+          }
+          // ---- rotate Bt (and Ct) of the tile in place: lanes take 32 consecutive rows, the branch
+          // r = lane % R and so the chunk's biases are fixed per thread
+#pragma unroll 1
+          for (int q = 0; q < C::KCW; ++q) {
+            const int kc = wr + N_ROT * q;
+            // row 32 step + lane, chunk kc: 128-byte swizzle with (row & 7) = (lane & 7)
+            const uint32_t cb = (uint32_t)(kc >> 3) * BLK + (uint32_t)lane * 128u + ((uint32_t)((kc & 7) ^ (lane & 7)) << 4);
+            const float4 bBe = *reinterpret_cast<const float4*>(biasB + kc * 8);
+            const float4 bBo = *reinterpret_cast<const float4*>(biasB + kc * 8 + 4);
+            const uint64_t bB0 = f2(bBe.x, bBe.y), bB1 = f2(bBe.z, bBe.w), bB2 = f2(bBo.x, bBo.y), bB3 = f2(bBo.z, bBo.w);
+            uint64_t bC0 = 0, bC1 = 0, bC2 = 0, bC3 = 0;
+            if constexpr (FULL) {
+              const float4 bCe = *reinterpret_cast<const float4*>(biasC + kc * 8);
+              const float4 bCo = *reinterpret_cast<const float4*>(biasC + kc * 8 + 4);
+              bC0 = f2(bCe.x, bCe.y), bC1 = f2(bCe.z, bCe.w), bC2 = f2(bCo.x, bCo.y), bC3 = f2(bCo.z, bCo.w);
+            }
+            const uint8_t* tk = tab + kc * 16;
+#pragma unroll 2
+            for (int step = 0; step < 4; ++step) {
+              const int row = 32 * step + lane;
+              const int t = row / R;
+              const uint32_t off = cb + (uint32_t)step * 4096u;
+              if (t < nv) {
+                float nb = 1.0f, nc = 1.0f;
+                if (p.raw_inputs) {  // 1 / rms of the raw rows: the B/C norm, before the bias
+                  nb = rsqrtf(rowss[row] * (1.0f / N) + kBcNormEps);
+                  if constexpr (FULL) nc = rsqrtf(rowss[128 + row] * (1.0f / N) + kBcNormEps);
                 }
+                const RotCS rcs = rot_cs(*reinterpret_cast<const uint4*>(tk + t * C::TAB_ROW));
+                const uint4 rb = lds128(sB(s) + off);
+                uint4 rc;
+                if constexpr (FULL) rc = lds128(sC(s) + off);
+                sts128(sB(s) + off, rotate16(rb, rcs, f2(nb, nb), bB0, bB1, bB2, bB3));
+                if constexpr (FULL) sts128(sC(s) + off, rotate16(rc, rcs, f2(nc, nc), bC0, bC1, bC2, bC3));
               } else {
-                sts128(rB + off, make_uint4(0, 0, 0, 0));
-                if constexpr (FULL) sts128(rC + off, make_uint4(0, 0, 0, 0));
+                sts128(sB(s) + off, make_uint4(0, 0, 0, 0));
+                if constexpr (FULL) sts128(sC(s) + off, make_uint4(0, 0, 0, 0));
               }
             }
           }
@@ -720,16 +732,17 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
             const bool oks = ws_wait(&bar[B_SF], (uint32_t)(i & 1), abort_flag);
             if (bar_any(BAR_ROT, 32 * N_ROT, !oks || *abort_flag)) break;
             const float Le = sc[1];
-            const int t = rrow / R;
-            if (t < nv) {
-              const float Lct = reinterpret_cast<const float*>(ra)[4 * t];
-              const float fc = __expf(Lct), fb = __expf(Le - Lct);
-              const uint32_t rB = sB(s) + rbase, rC = sC(s) + rbase;
-#pragma unroll
-              for (int j = 0; j < C::CPT; ++j) {
-                const uint32_t off = (uint32_t)(rx ^ j) << 4;
-                sts128(rC + off, scale_chunk(lds128(rC + off), fc));
-                sts128(rB + off, scale_chunk(lds128(rB + off), fb));
+#pragma unroll 1
+            for (int q = 0; q < C::KCW; ++q) {
+              const int kc = wr + N_ROT * q;
+              const uint32_t cb = (uint32_t)(kc >> 3) * BLK + (uint32_t)lane * 128u + ((uint32_t)((kc & 7) ^ (lane & 7)) << 4);
+              for (int step = 0; step < 4; ++step) {
+                const int t = (32 * step + lane) / R;
+                if (t >= nv) continue;
+                const uint32_t off = cb + (uint32_t)step * 4096u;
+                const float Lct = reinterpret_cast<const float*>(ra)[4 * t];
+                sts128(sC(s) + off, scale_chunk(lds128(sC(s) + off), __expf(Lct)));
+                sts128(sB(s) + off, scale_chunk(lds128(sB(s) + off), __expf(Le - Lct)));
               }
             }
             fence_async_smem();
