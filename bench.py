@@ -363,6 +363,7 @@ def run_ours(args):
         prefill[EXTRA_PREFILL] = run_prefill_one(args, device, peaks, EXTRA_PREFILL)
         prefill["sweep_l15b"] = run_prefill_sweep(args, device, peaks)
     stack = run_stack(args, device, peaks) if not args.no_stack else None
+    backward = run_backward(args, device) if not args.no_backward else None
     e2e = run_e2e(args, inp, tok_inp, device, world) if not args.no_e2e else None
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -372,7 +373,7 @@ def run_ours(args):
                                f"N{cfg['N']} R{cfg['R']}, chunk 32) + 1 m3_decode_step",
                    "global_batch": cfg["b"] * world, "seq_len": cfg["L"], "parallelism": f"dp{world}",
                    "l2": f"{n_sets} input sets of {per_set / 2**20:.0f} MiB each (> L2), alternating"},
-        "roofline": roofline, "prefill": prefill, "decode": decode, "stack": stack, "e2e": e2e,
+        "roofline": roofline, "prefill": prefill, "decode": decode, "stack": stack, "backward": backward, "e2e": e2e,
         "gpu_launches": gpu_launches, "clocks": clk.summary(),
     }
     if rank == 0 and not args.no_cpu:
@@ -474,6 +475,42 @@ def run_decode(args, device, peaks, name=DECODE_WORKLOAD):
             "tokens_per_s": cfg["b"] / (ms * 1e-3), "us_per_step": ms * 1e3,
             "hbm_gbs": by / (ms * 1e-3) / 1e9, "hbm_frac_of_measured": by / (ms * 1e-3) / 1e9 / peaks["hbm"],
             "tflops": fl / (ms * 1e-3) / 1e12, "algorithmic_bytes": by}
+
+
+def run_backward(args, device, names=("p1_layer", "l15b_2k"), calls=2):
+    """m3_scan_bwd (every gradient) on the page-1 layer and the 1.5B-scale layer at 2K tokens: the
+    mean of `calls` calls after one warm-up call, gradient and workspace buffers allocated once."""
+    import torch
+    from selective_state_space_53_b200 import m3
+    from selective_state_space_53_b200.inputs import CONFIGS, config_inputs
+    out = {}
+    for name in names:
+        cfg = dict(CONFIGS[name])
+        inp = config_inputs(name)
+        dims = m3.dims_of(inp)
+        dev = m3.to_device(inp, device)
+        st, keep = m3.state_tensors(dims, device=device)
+        g = torch.Generator(device="cpu").manual_seed(31)
+        dy = torch.randn(dev["x"].shape, generator=g).to(dev["x"].dtype).to(device)
+        m3.scan_backward(dims, dev, st, dy)
+        torch.cuda.synchronize()
+        stream = torch.cuda.current_stream()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(calls):
+            m3.scan_backward(dims, dev, st, dy)
+        b.record(stream)
+        torch.cuda.synchronize()
+        assert m3.m3_check() == 0
+        ms = a.elapsed_time(b) / calls
+        out[name] = {"workload": "%s: m3_scan_bwd b%d L%d H%d P%d N%d R%d, every gradient" %
+                                 (name, cfg["b"], cfg["L"], cfg["H"], cfg["P"], cfg["N"], cfg["R"]),
+                     "ms_per_call": ms, "tokens_per_s": cfg["b"] * cfg["L"] / (ms * 1e-3),
+                     "note": "token-sequential SIMT kernel with checkpointed recomputation (one block per "
+                             "(batch, head)); includes allocation of the gradient buffers and workspace"}
+        del dev, st, keep, dy
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_stack(args, device, peaks):
@@ -734,6 +771,7 @@ def main():
     ap.add_argument("--no-prefill-sweep", action="store_true", help="skip the 1.5B-scale layer prefill sweep")
     ap.add_argument("--no-stack", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -101,6 +101,42 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Sums each of 16 values over the 32 lanes of a warp in 16 shuffles (a transposed butterfly:
+// every step keeps half of the values and adds the partner lane's copy of them, the last step
+// adds the neighbour's total).  Lane l returns the total of value l / 2.
+__device__ __forceinline__ float warp_sum16(float (&v)[16], int lane) {
+#pragma unroll
+  for (int s = 8, off = 16; s >= 1; s >>= 1, off >>= 1) {
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      const float give = up ? v[i] : v[i + s];
+      const float keep = up ? v[i + s] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, give, off);
+    }
+  }
+  return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+}
+
+// The terms of one rotation pair (2 values per branch r < R: rows n0, n1) summed over the
+// columns p into red[r N + n]: a warp butterfly when every lane of the warp holds this pair
+// (wide), element atomics otherwise.
+__device__ __forceinline__ void pair_reduce(float (&v)[16], bool wide, int lane, int R, int N, int n0, int n1,
+                                            float* red) {
+  if (wide) {
+    const float tot = warp_sum16(v, lane);
+    const int vi = lane >> 1, r = vi >> 1;
+    if ((lane & 1) == 0 && r < R) atomicAdd(&red[r * N + ((vi & 1) ? n1 : n0)], tot);
+  } else {
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      if (r >= R) break;
+      atomicAdd(&red[r * N + n0], v[2 * r]);
+      atomicAdd(&red[r * N + n1], v[2 * r + 1]);
+    }
+  }
+}
+
 // zero the fp32 gradient buffers that several CTAs add into
 __global__ void bwd_zero_kernel(float* a, int64_t na, float* b, int64_t nb, float* c, int64_t nc, float* d,
                                 int64_t nd, float* e, int64_t ne) {
@@ -141,6 +177,7 @@ __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(const Params p, c
   const BwdSmem ms = bwd_smem(P, N, R);
   const int pc = tid % P, grp = tid / P;
   const bool active = grp < sh.KG;
+  const bool wide = P % 32 == 0;  // a warp's lanes are columns of one pair group
   float* const Bb = sm + ms.bb;
   float* const Bbp = sm + ms.bbp;
   float* const Cb = sm + ms.cb;
@@ -312,16 +349,23 @@ __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(const Params p, c
         const int n0 = 2 * k, n1 = 2 * k + 1;
         const float ht0 = ht[(int64_t)n0 * P + pc], ht1 = ht[(int64_t)n1 * P + pc];
         const float hp0 = hp[(int64_t)n0 * P + pc], hp1 = hp[(int64_t)n1 * P + pc];
-        // readout: g += sum_r Cb_r dY_r^T; dCb_r += h_t dY_r; Y_r partial
+        // readout: g += sum_r Cb_r dY_r^T; dCb_r += h_t dY_r (summed over the warp's columns
+        // below); Y_r partial.  sv holds the pair's column terms: dCb (r, n0), (r, n1), then dBb
         float g0 = gr0[j], g1 = gr1[j];
-        for (int r = 0; r < R; ++r) {
-          const float dy_r = dYr[r * P + pc];
-          g0 = fmaf(Cb[r * N + n0], dy_r, g0);
-          g1 = fmaf(Cb[r * N + n1], dy_r, g1);
-          atomicAdd(&red_cb[r * N + n0], ht0 * dy_r);
-          atomicAdd(&red_cb[r * N + n1], ht1 * dy_r);
-          py[r] = fmaf(Cb[r * N + n0], ht0, fmaf(Cb[r * N + n1], ht1, py[r]));
+        float sv[16];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          sv[2 * r] = sv[2 * r + 1] = 0.0f;
+          if (r < R) {
+            const float dy_r = dYr[r * P + pc];
+            g0 = fmaf(Cb[r * N + n0], dy_r, g0);
+            g1 = fmaf(Cb[r * N + n1], dy_r, g1);
+            sv[2 * r] = ht0 * dy_r;
+            sv[2 * r + 1] = ht1 * dy_r;
+            py[r] = fmaf(Cb[r * N + n0], ht0, fmaf(Cb[r * N + n1], ht1, py[r]));
+          }
         }
+        pair_reduce(sv, wide, tid & 31, R, N, n0, n1, red_cb);
         // step
         float u0 = 0.f, u1 = 0.f, q0 = 0.f, q1 = 0.f;
         for (int r = 0; r < R; ++r) {
@@ -338,22 +382,35 @@ __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(const Params p, c
         const float du0 = fmaf(gamma, g0, dn0[j]), du1 = fmaf(gamma, g1, dn1[j]);
         const float dm0 = alpha * g0, dm1 = alpha * g1;
         const float dz0 = cc.x * dm0 + cc.y * dm1, dz1 = -cc.y * dm0 + cc.x * dm1;
-        atomicAdd(&red_phi[k], dm0 * (-cc.y * z0 - cc.x * z1) + dm1 * (cc.x * z0 - cc.y * z1));
+        const float phi_t = dm0 * (-cc.y * z0 - cc.x * z1) + dm1 * (cc.x * z0 - cc.y * z1);
+        if (wide) {
+          const float ps = warp_sum(phi_t);
+          if ((tid & 31) == 0) atomicAdd(&red_phi[k], ps);
+        } else {
+          atomicAdd(&red_phi[k], phi_t);
+        }
         s_bp = fmaf(dz0, q0, fmaf(dz1, q1, s_bp));
         dn0[j] = bprime * dz0;
         dn1[j] = bprime * dz1;
         gr0[j] = dz0;
         gr1[j] = dz1;
         // u_t = sum_r Bb_r X_r^T
-        for (int r = 0; r < R; ++r) {
-          const float xr = X[r * P + pc];
-          atomicAdd(&red_bb[r * N + n0], du0 * xr);
-          atomicAdd(&red_bb[r * N + n1], du1 * xr);
-          px[r] = fmaf(du0, Bb[r * N + n0], fmaf(du1, Bb[r * N + n1], px[r]));
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          sv[2 * r] = sv[2 * r + 1] = 0.0f;
+          if (r < R) {
+            const float xr = X[r * P + pc];
+            sv[2 * r] = du0 * xr;
+            sv[2 * r + 1] = du1 * xr;
+            px[r] = fmaf(du0, Bb[r * N + n0], fmaf(du1, Bb[r * N + n1], px[r]));
+          }
         }
+        pair_reduce(sv, wide, tid & 31, R, N, n0, n1, red_bb);
       }
       if (active) {
-        for (int r = 0; r < R; ++r) {
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          if (r >= R) break;
           atomicAdd(&red_x[r * P + pc], px[r]);
           atomicAdd(&red_y[r * P + pc], py[r]);
         }
@@ -423,15 +480,22 @@ __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(const Params p, c
     for (int j = 0; j < NK; ++j) {
       const int k = grp + j * sh.KG;
       if (!active || k >= K2) continue;
-      for (int r = 0; r < R; ++r) {
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        if (r >= R) break;
         const float xr = Xp[r * P + pc];
         atomicAdd(&red_bb[r * N + 2 * k], dn0[j] * xr);
         atomicAdd(&red_bb[r * N + 2 * k + 1], dn1[j] * xr);
         px[r] = fmaf(dn0[j], Bbp[r * N + 2 * k], fmaf(dn1[j], Bbp[r * N + 2 * k + 1], px[r]));
       }
     }
-    if (active)
-      for (int r = 0; r < R; ++r) atomicAdd(&red_x[r * P + pc], px[r]);
+    if (active) {
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        if (r >= R) break;
+        atomicAdd(&red_x[r * P + pc], px[r]);
+      }
+    }
   }
   __syncthreads();
   for (int i = tid; i < R * N; i += kBwdThreads) {

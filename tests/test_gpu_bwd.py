@@ -78,3 +78,58 @@ def test_bwd_page1_layer_shape_sampled():
     # the page-1 layer's head shape over a full-length sequence (one batch row, 4 heads)
     inp = make_inputs(dtype="bf16", seed=904, extras=True, b=1, L=2048, H=4, P=64, N=64, R=2, G=1)
     check_bwd(inp)
+
+
+def _head_subset(inp, sel):
+    """The draw restricted to heads `sel` (G = 1: B, C and theta are shared by every head)."""
+    import copy
+    sub = copy.copy(inp)
+    sub.dims = dict(inp.dims, H=len(sel))
+    for k in ("x", "dt", "A", "lam"):
+        setattr(sub, k, np.ascontiguousarray(getattr(inp, k)[:, :, sel]))
+    for k in ("bias_B", "bias_C", "W_x", "W_o", "D"):
+        a = getattr(inp, k)
+        setattr(sub, k, None if a is None else np.ascontiguousarray(a[sel]))
+    return sub
+
+
+@pytest.mark.parametrize("cfg", ["p1_layer", "l15b_2k"])
+def test_bwd_full_config_sampled_heads(cfg):
+    """The backward at a layer workload's full size on the GPU, with cotangents on two sampled heads
+    only: their per-head gradients and the shared B, C, theta gradients (the other heads add
+    nothing) against the oracle run on those heads."""
+    from selective_state_space_53_b200.inputs import CONFIGS, SEEDS
+    c = dict(CONFIGS[cfg])
+    inp = make_inputs(seed=SEEDS[cfg] + 7, extras=True, **{k: c[k] for k in ("b", "L", "H", "P", "N", "R", "G", "dtype")})
+    d = inp.dims
+    rng = np.random.default_rng(905)
+    sel = sorted(int(h) for h in rng.choice(d["H"], 2, replace=False))
+    dy = np.zeros((d["b"], d["L"], d["H"], d["P"]), np.float32)
+    dy[:, :, sel] = round_to_bf16(rng.standard_normal((d["b"], d["L"], 2, d["P"])).astype(np.float32))
+    dhf = np.zeros((d["b"], d["H"], d["N"], d["P"]), np.float32)
+    dhf[:, sel] = rng.standard_normal((d["b"], 2, d["N"], d["P"])).astype(np.float32)
+    dims = m3.dims_of(inp)
+    dev = m3.to_device(inp)
+    st, keep = m3.state_tensors(dims)
+    got = m3.scan_backward(dims, dev, st, torch.from_numpy(dy).to(torch.bfloat16).cuda(), torch.from_numpy(dhf).cuda())
+    torch.cuda.synchronize()
+    assert m3.m3_check() == 0
+    sub = _head_subset(inp, sel)
+    ref = orc.scan_bwd(sub.dims, sub.x, sub.dt, sub.A, sub.lam, sub.B, sub.C, sub.theta, sub.bias_B, sub.bias_C,
+                       sub.W_x, sub.W_o, sub.D, dy=dy[:, :, sel], dh_final=dhf[:, sel])
+    per_head_tok = ("dx", "ddt", "dA", "dlam")
+    per_head = ("dbias_B", "dbias_C", "dW_x", "dW_o", "dD")
+    per_seq_head = ("dh0", "dcarry_B", "dcarry_x")
+    errs = {}
+    for k in m3.GRAD_KEYS:
+        g = got[k].float().cpu().numpy()
+        if k in per_head_tok:
+            g = g[:, :, sel]
+        elif k in per_head:
+            g = g[sel]
+        elif k in per_seq_head:
+            g = g[:, sel]
+        errs[k] = rel_err(g, ref[k])
+    print(f"{cfg} bwd (heads {sel}): " + ", ".join(f"{k} {v:.1e}" for k, v in errs.items()))
+    bad = {k: v for k, v in errs.items() if not v < TOL["bf16"]}
+    assert not bad, bad
