@@ -25,4 +25,9 @@ struct SegInfo {
                    // summary, which reads no incoming state)
 };
 
+// The MIMO rank a chunked tensor-core kernel runs a rank R at: the next of 1, 2, 4, 8.  Branches
+// R .. rank-1 are zero padding: their B and C rows are the zero fill of the tile copies and their
+// W_x, W_o and biases are zero, so they add nothing to the state or the output.
+__host__ __device__ inline int tile_rank(int R) { return R <= 1 ? 1 : R <= 2 ? 2 : R <= 4 ? 4 : 8; }
+
 }  // namespace m3

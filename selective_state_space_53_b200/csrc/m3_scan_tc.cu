@@ -376,12 +376,13 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
 #pragma unroll
   for (int q = 0; q < RPW; ++q) {
     const int i = tid + q * kThreads;
-    wxv[q] = (i < R * P && p.W_x) ? p.W_x[(int64_t)hi * R * P + i] : 1.0f;
-    wov[q] = (i < R * P && p.W_o) ? p.W_o[(int64_t)hi * R * P + i] : 1.0f;
+    // branches p.R .. R-1 of the tile are zero padding: zero weights
+    wxv[q] = i < p.R * P ? (p.W_x ? p.W_x[(int64_t)hi * p.R * P + i] : 1.0f) : 0.0f;
+    wov[q] = i < p.R * P ? (p.W_o ? p.W_o[(int64_t)hi * p.R * P + i] : 1.0f) : 0.0f;
   }
   load_coefs(j0);
-  const float* biasBg = p.bias_B ? p.bias_B + (int64_t)hi * R * N : nullptr;
-  const float* biasCg = p.bias_C ? p.bias_C + (int64_t)hi * R * N : nullptr;
+  const float* biasBg = p.bias_B ? p.bias_B + (int64_t)hi * p.R * N : nullptr;
+  const float* biasCg = p.bias_C ? p.bias_C + (int64_t)hi * p.R * N : nullptr;
   // operand staging: B, C rows on all threads; x rows on warps 1-7 (warp 0 prepares the next
   // tile's coefficients meanwhile)
   const int xt = tid;
@@ -392,8 +393,8 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
   float bB[8], bC[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
-    bB[e] = biasBg ? __ldg(biasBg + tr * N + tch * 8 + e) : 0.0f;
-    bC[e] = biasCg ? __ldg(biasCg + tr * N + tch * 8 + e) : 0.0f;
+    bB[e] = (biasBg && tr < p.R) ? __ldg(biasBg + tr * N + tch * 8 + e) : 0.0f;
+    bC[e] = (biasCg && tr < p.R) ? __ldg(biasCg + tr * N + tch * 8 + e) : 0.0f;
   }
 #pragma unroll
   for (int q = 0; q < RPW; ++q) {
@@ -456,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
       for (int r = 0; r < R; ++r) xprev[r] = wx[r * P + prow] * p.carry_x[(int64_t)bh * P + prow];
     }
     const float* h0 = p.h + (int64_t)bh * N * P;
-    const float* cB = p.carry_B + (int64_t)bh * R * N;
+    const float* cB = p.carry_B + (int64_t)bh * p.R * N;
 #pragma unroll 1
     for (int c = c_lo; c < c_hi; ++c) {
       float v[32];
@@ -469,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
           float u = 0.0f;
 #pragma unroll
           for (int r = 0; r < R; ++r)
-            u = fmaf(cB[r * N + n] + (biasBg ? __ldg(biasBg + r * N + n) : 0.0f), xprev[r], u);
+            if (r < p.R) u = fmaf(cB[r * N + n] + (biasBg ? __ldg(biasBg + r * N + n) : 0.0f), xprev[r], u);
           v[e] = fmaf(bp0, u, h0[(int64_t)n * P + prow]);
         }
         if (!FULL && sg.nseg > 1 && st_owner) {
@@ -987,8 +988,8 @@ __global__ void __launch_bounds__(kThreads, (P == 64 && N == 64) ? 2 : 1)
           }
         } else {
           const int64_t tokl = tok_base + (L - 1);
-          const int64_t bc = ((tokl * G + g) * R) * (int64_t)N;
-          for (int i = tid; i < R * N; i += 128) p.carry_B[(int64_t)bh * R * N + i] = __bfloat162float(Bg[bc + i]);
+          const int64_t bc = ((tokl * G + g) * p.R) * (int64_t)N;
+          for (int i = tid; i < p.R * N; i += 128) p.carry_B[(int64_t)bh * p.R * N + i] = __bfloat162float(Bg[bc + i]);
           const int64_t xr = (tokl * H + hi) * (int64_t)P;
           for (int i = tid; i < P; i += 128) p.carry_x[(int64_t)bh * P + i] = __bfloat162float(xg[xr + i]);
         }
@@ -1052,12 +1053,14 @@ struct Maps {
   CUtensorMap B, C, X;
 };
 
-bool make_maps(const Params& p, int Q, Maps* m) {
+// B and C tiles of Q tokens x RT branches: with RT above the operands' rank p.R the branch rows
+// past p.R lie outside the tensor and the copy fills them with zeros.
+bool make_maps(const Params& p, int Q, int RT, Maps* m) {
   const cuuint64_t toks = (cuuint64_t)(p.b * p.L);
   {
     const cuuint64_t dims[4] = {(cuuint64_t)p.N, (cuuint64_t)p.R, (cuuint64_t)p.G, toks};
     const cuuint64_t str[3] = {(cuuint64_t)p.N * 2, (cuuint64_t)p.R * p.N * 2, (cuuint64_t)p.G * p.R * p.N * 2};
-    const cuuint32_t box[4] = {64, (cuuint32_t)p.R, 1, (cuuint32_t)Q};
+    const cuuint32_t box[4] = {64, (cuuint32_t)RT, 1, (cuuint32_t)Q};
     if (!make_map(&m->B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, p.B, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
       return false;
     if (!make_map(&m->C, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, p.C, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -1194,7 +1197,7 @@ cudaError_t launch_summary_cfg(const Params& p, void* ws, size_t ws_bytes, SegIn
   sg.ws_phi = reinterpret_cast<double*>(w + ((4 * nseq * ns * (size_t)N * P + 4 * nseq * ns + 255) & ~(size_t)255));
   *sg_out = sg;
   Maps m;
-  if (!make_maps(p, Q, &m)) return cudaErrorInvalidValue;
+  if (!make_maps(p, Q, R, &m)) return cudaErrorInvalidValue;
   if (ws_scan_supported(p)) return launch_scan_ws_state(m.B, m.C, m.X, p, sg, stream);
   return launch_mode<R, N, P, MODE_STATE>(m, p, sg, (unsigned)(nseq * ns), stream);
 }
@@ -1206,7 +1209,7 @@ cudaError_t launch_cfg(const Params& p, void* ws, size_t ws_bytes, cudaStream_t 
   const size_t need = ws_bytes_for<R, N, P>(p, &plan);
   if (need > ws_bytes || (need > 0 && ws == nullptr)) return cudaErrorInvalidValue;
   Maps m;
-  if (!make_maps(p, Q, &m)) return cudaErrorInvalidValue;
+  if (!make_maps(p, Q, R, &m)) return cudaErrorInvalidValue;
   SegInfo sg;
   sg.nseg = plan.nseg;
   sg.seg_tiles = plan.seg_tiles;
@@ -1285,7 +1288,7 @@ cudaError_t launch_summary_r(const Params& p, void* ws, size_t wsb, SegInfo* sg,
 }  // namespace
 
 size_t scan_summary_workspace_bytes(const Params& p) {
-  switch (p.R) {
+  switch (tile_rank(p.R)) {
     case 1: return summary_ws_r<1>(p);
     case 2: return summary_ws_r<2>(p);
     case 4: return summary_ws_r<4>(p);
@@ -1294,7 +1297,7 @@ size_t scan_summary_workspace_bytes(const Params& p) {
 }
 
 cudaError_t launch_scan_summary_pass(const Params& p, void* ws, size_t ws_bytes, SegInfo* sg, cudaStream_t stream) {
-  switch (p.R) {
+  switch (tile_rank(p.R)) {
     case 1: return launch_summary_r<1>(p, ws, ws_bytes, sg, stream);
     case 2: return launch_summary_r<2>(p, ws, ws_bytes, sg, stream);
     case 4: return launch_summary_r<4>(p, ws, ws_bytes, sg, stream);
@@ -1306,17 +1309,17 @@ bool tc_scan_supported(const Params& p) {
   if (p.dtype != M3_BF16) return false;
   if (!((p.N == 64 || p.N == 128) && (p.P == 64 || p.P == 128))) return false;
   if (p.b * p.L > 0x7fffffffLL) return false;  // TMA token coordinate is 32-bit
-  switch (p.R) {
+  if (p.R < 1 || p.R > 8) return false;
+  switch (tile_rank(p.R)) {  // ranks 3, 5, 6, 7 run padded to the next tile rank
     case 1: return fits_r<1>(p);
     case 2: return fits_r<2>(p);
     case 4: return fits_r<4>(p);
-    case 8: return fits_r<8>(p);
-    default: return false;
+    default: return fits_r<8>(p);
   }
 }
 
 size_t tc_scan_workspace_bytes(const Params& p) {
-  switch (p.R) {
+  switch (tile_rank(p.R)) {
     case 1: return ws_r<1>(p);
     case 2: return ws_r<2>(p);
     case 4: return ws_r<4>(p);
@@ -1325,7 +1328,7 @@ size_t tc_scan_workspace_bytes(const Params& p) {
 }
 
 cudaError_t launch_scan_tc(const Params& p, void* ws, size_t ws_bytes, cudaStream_t stream) {
-  switch (p.R) {
+  switch (tile_rank(p.R)) {
     case 1: return launch_r<1>(p, ws, ws_bytes, stream);
     case 2: return launch_r<2>(p, ws, ws_bytes, stream);
     case 4: return launch_r<4>(p, ws, ws_bytes, stream);

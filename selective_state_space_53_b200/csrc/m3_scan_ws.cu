@@ -263,6 +263,7 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = p.H, G = p.G;
+  const int RR = p.R;  // the operands' MIMO rank; branches RR .. R-1 of the tile are zero padding
   const int64_t L = p.L;
   const int nseg_grid = FULL ? sg.nseg : sg.nsub;
   const int bh = blockIdx.x / nseg_grid;
@@ -586,7 +587,7 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
           const int op = e / (R * N), rem = e % (R * N), r = rem / N, n = rem % N;
           const float* src = op ? p.bias_C : p.bias_B;
           sbias[(op * R + r) * C::BIAS_ROW + (n >> 3) * 8 + bias_pos(n & 7)] =
-              src ? src[((int64_t)hi * R + r) * N + n] : 0.0f;
+              (src && r < RR) ? src[((int64_t)hi * RR + r) * N + n] : 0.0f;
         }
         const float* biasB = sbias + rr * C::BIAS_ROW;
         const float* biasC = sbias + (R + rr) * C::BIAS_ROW;
@@ -834,7 +835,7 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
         const int pc = 32 * q4 + lane;  // head-dim column of this thread
         float wo[R];
 #pragma unroll
-        for (int r = 0; r < R; ++r) wo[r] = p.W_o ? p.W_o[((int64_t)hi * R + r) * WP + pc] : 1.0f;
+        for (int r = 0; r < R; ++r) wo[r] = r < RR ? (p.W_o ? p.W_o[((int64_t)hi * RR + r) * WP + pc] : 1.0f) : 0.0f;
         const float Dh = p.D ? p.D[hi] : 0.0f;
         __nv_bfloat16* yg = static_cast<__nv_bfloat16*>(p.y);
         constexpr int TPC = 16 / R;  // tokens per 16-column chunk
@@ -902,7 +903,7 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
         const int pc = 32 * q4 + lane;
         float wx[R];
 #pragma unroll
-        for (int r = 0; r < R; ++r) wx[r] = p.W_x ? p.W_x[((int64_t)hi * R + r) * WP + pc] : 1.0f;
+        for (int r = 0; r < R; ++r) wx[r] = r < RR ? (p.W_x ? p.W_x[((int64_t)hi * RR + r) * WP + pc] : 1.0f) : 0.0f;
         Phases ph_cf, ph_xbf, ph_xf;
         constexpr int TPC = 32 / R;
         // X'^T of tile i: X'^T[p, tR + r] = W_x[r, p] x_t[p], bf16 pairs along the columns
@@ -968,8 +969,8 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
               for (int r = 0; r < R; ++r) xprev[r] = wx[r] * p.carry_x[(int64_t)bh * WP + pc];
             }
             const float* h0 = p.h + (int64_t)bh * N * WP;
-            const float* cB = p.carry_B + (int64_t)bh * R * N;
-            const float* bB = p.bias_B ? p.bias_B + (int64_t)hi * R * N : nullptr;
+            const float* cB = p.carry_B + (int64_t)bh * RR * N;
+            const float* bB = p.bias_B ? p.bias_B + (int64_t)hi * RR * N : nullptr;
 #pragma unroll 1
             for (int c = 0; c < N / 32; ++c) {
               float v[32];
@@ -981,7 +982,8 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
                   const int n = 32 * c + e;
                   float u = 0.0f;
 #pragma unroll
-                  for (int r = 0; r < R; ++r) u = fmaf(cB[r * N + n] + (bB ? bB[r * N + n] : 0.0f), xprev[r], u);
+                  for (int r = 0; r < R; ++r)
+                    if (r < RR) u = fmaf(cB[r * N + n] + (bB ? bB[r * N + n] : 0.0f), xprev[r], u);
                   v[e] = fmaf(bp0, u, h0[(int64_t)n * WP + pc]);
                 }
                 if (make_init) {
@@ -1082,20 +1084,20 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
               // raw) and raw x
               const int64_t tokl = tok_base + (L - 1);
               const __nv_bfloat16* Bg = static_cast<const __nv_bfloat16*>(p.B);
-              const int64_t bc = ((tokl * G + g) * R) * (int64_t)N;
+              const int64_t bc = ((tokl * G + g) * RR) * (int64_t)N;
               if (p.raw_inputs) {  // the rotation warps are done with rowss (B_FIN)
-                if (pc < R) rowss[pc] = 0.0f;
+                if (pc < RR) rowss[pc] = 0.0f;
                 named_bar_sync(BAR_SPX, 128);
-                for (int k = pc; k < R * N; k += WP) {
+                for (int k = pc; k < RR * N; k += WP) {
                   const float v = __bfloat162float(Bg[bc + k]);
                   atomicAdd(&rowss[k / N], v * v);
                 }
                 named_bar_sync(BAR_SPX, 128);
               }
-              for (int k = pc; k < R * N; k += WP) {
+              for (int k = pc; k < RR * N; k += WP) {
                 float v = __bfloat162float(Bg[bc + k]);
                 if (p.raw_inputs) v *= rsqrtf(rowss[k / N] * (1.0f / N) + kBcNormEps);
-                p.carry_B[(int64_t)bh * R * N + k] = v;
+                p.carry_B[(int64_t)bh * RR * N + k] = v;
               }
               p.carry_x[(int64_t)bh * WP + pc] = __bfloat162float(xg[(tokl * H + hi) * (int64_t)WP + pc]);
             }
@@ -1128,9 +1130,10 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
 // ------------------------------------------------------------------ host side
 
 bool ws_scan_supported(const Params& p) {
-  if (p.dtype != M3_BF16 || p.P != WP) return false;
-  if (p.N == 128) return p.R == 4 || p.R == 8;
-  if (p.N == 64) return p.R == 2 || p.R == 4 || p.R == 8;
+  if (p.dtype != M3_BF16 || p.P != WP || p.R < 1 || p.R > 8) return false;
+  const int rt = tile_rank(p.R);
+  if (p.N == 128) return rt == 4 || rt == 8;
+  if (p.N == 64) return rt == 2 || rt == 4 || rt == 8;
   return false;
 }
 
@@ -1166,9 +1169,9 @@ cudaError_t launch_ws_rn(const CUtensorMap& tmB, const CUtensorMap& tmC, const C
 cudaError_t launch_scan_ws_state(const CUtensorMap& tmB, const CUtensorMap& tmC, const CUtensorMap& tmX,
                                  const Params& p, const SegInfo& sg, cudaStream_t stream) {
   const unsigned grid = (unsigned)(p.b * p.H * sg.nsub);
-  if (p.N == 128) return p.R == 4 ? launch_ws_mode<4, 128, WS_STATE>(tmB, tmC, tmX, p, sg, grid, stream)
-                                  : launch_ws_mode<8, 128, WS_STATE>(tmB, tmC, tmX, p, sg, grid, stream);
-  switch (p.R) {
+  if (p.N == 128) return tile_rank(p.R) == 4 ? launch_ws_mode<4, 128, WS_STATE>(tmB, tmC, tmX, p, sg, grid, stream)
+                                            : launch_ws_mode<8, 128, WS_STATE>(tmB, tmC, tmX, p, sg, grid, stream);
+  switch (tile_rank(p.R)) {
     case 2: return launch_ws_mode<2, 64, WS_STATE>(tmB, tmC, tmX, p, sg, grid, stream);
     case 4: return launch_ws_mode<4, 64, WS_STATE>(tmB, tmC, tmX, p, sg, grid, stream);
     default: return launch_ws_mode<8, 64, WS_STATE>(tmB, tmC, tmX, p, sg, grid, stream);
@@ -1177,9 +1180,9 @@ cudaError_t launch_scan_ws_state(const CUtensorMap& tmB, const CUtensorMap& tmC,
 
 cudaError_t launch_scan_ws(const CUtensorMap& tmB, const CUtensorMap& tmC, const CUtensorMap& tmX, const Params& p,
                            const SegInfo& sg, cudaStream_t stream) {
-  if (p.N == 128) return p.R == 4 ? launch_ws_rn<4, 128>(tmB, tmC, tmX, p, sg, stream)
-                                  : launch_ws_rn<8, 128>(tmB, tmC, tmX, p, sg, stream);
-  switch (p.R) {
+  if (p.N == 128) return tile_rank(p.R) == 4 ? launch_ws_rn<4, 128>(tmB, tmC, tmX, p, sg, stream)
+                                            : launch_ws_rn<8, 128>(tmB, tmC, tmX, p, sg, stream);
+  switch (tile_rank(p.R)) {
     case 2: return launch_ws_rn<2, 64>(tmB, tmC, tmX, p, sg, stream);
     case 4: return launch_ws_rn<4, 64>(tmB, tmC, tmX, p, sg, stream);
     default: return launch_ws_rn<8, 64>(tmB, tmC, tmX, p, sg, stream);

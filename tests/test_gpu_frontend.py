@@ -40,7 +40,8 @@ def test_frontend_kernel_matches_oracle(dtype):
     dict(b=1, L=3000, H=2, P=128, N=64, R=2, G=1),   # fused, segmented (state pass too)
     dict(b=1, L=200, H=2, P=64, N=64, R=2, G=1),     # headdim-64 tensor-core kernel: m3_frontend first
     dict(b=1, L=40, H=2, P=32, N=16, R=2, G=2),      # sequential kernel: m3_frontend first
-], ids=["P128", "P128seg", "P64", "seq"])
+    dict(b=1, L=600, H=2, P=128, N=128, R=3, G=1),   # fused, rank 3 padded to tile rank 4
+], ids=["P128", "P128seg", "P64", "seq", "P128R3"])
 def test_scan_with_raw_inputs_matches_oracle(shape):
     inp = make_raw_inputs(dtype="bf16", seed=961, extras=True, **shape)
     st = make_state(shape["b"], shape["H"], shape["P"], shape["N"], shape["R"], seed=962, scale=0.5)

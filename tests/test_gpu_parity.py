@@ -574,3 +574,21 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     assert m3.m3_check() == 0
     inp = make_inputs(dtype="bf16", seed=501, extras=True, b=1, L=70, H=2, P=64, N=64, R=2, G=1)
     check_scan(inp)
+
+
+@pytest.mark.parametrize("shape", [
+    dict(b=1, L=1000, H=2, P=128, N=128, R=3, G=1),   # warp-specialised kernel, tile rank 4
+    dict(b=1, L=1000, H=2, P=128, N=128, R=5, G=1),   # warp-specialised kernel, tile rank 8
+    dict(b=1, L=700, H=2, P=128, N=64, R=7, G=1),     # warp-specialised kernel at d_state 64, tile rank 8
+    dict(b=1, L=1000, H=2, P=64, N=64, R=3, G=1),     # headdim-64 kernel, tile rank 4
+    dict(b=2, L=500, H=2, P=64, N=128, R=6, G=1),     # headdim-64 kernel at d_state 128, tile rank 8
+], ids=lambda s: "P{P}N{N}R{R}".format(**s))
+@pytest.mark.parametrize("with_state", [False, True])
+def test_padded_rank_tc(shape, with_state):
+    """MIMO ranks 3, 5, 6, 7 run on the chunked tensor-core kernels padded to the next tile rank
+    (zero branches); few sequences over a long L make the plan segmented, which only those kernels
+    do (a workspace is asked for), so the test shows they ran."""
+    inp = make_inputs(dtype="bf16", seed=240 + shape["R"], extras=True, **shape)
+    assert m3.m3_scan_workspace_size(m3.dims_of(inp)) > 0
+    st = make_state(shape["b"], shape["H"], shape["P"], shape["N"], shape["R"], seed=241, scale=0.5) if with_state else None
+    check_scan(inp, state=st)
