@@ -121,14 +121,19 @@ m3_status m3_state_copy_from_host(m3_state* state, const void* src, size_t nbyte
 
 /* ---- prefill (chunked scan) ------------------------------------------- */
 
-/* Scratch bytes m3_scan_fwd needs for these dims (0 when it needs none). */
+/* Scratch bytes m3_scan_fwd needs for these dims (0 when it needs none).  For the chunked
+ * tensor-core scan the workspace is required; for the token-sequential SIMT scan (fp32 inputs,
+ * shapes outside the tensor-core tiles, M3_FLAG_SEQUENTIAL excepted) it lets the sequences be
+ * split into segments scanned in parallel (summaries of the earlier segments folded into each
+ * segment's entering state), and without it they are walked whole. */
 m3_status m3_scan_workspace_size(const m3_dims* dims, size_t* out_bytes);
 
 /* Run the layer core over L tokens of every sequence of the batch.
  * state: in = state before token 0 (fresh or carried), out = state after token
  * L-1 (h_{L-1} and the carry of token L-1).  y: (b, L, H, P) in dims->dtype.
  * workspace: device scratch of at least m3_scan_workspace_size bytes (may be NULL
- * when that size is 0).  L = 0 leaves the state unchanged and writes nothing.
+ * when that size is 0, or on the sequential path, which then does not split the sequences).
+ * L = 0 leaves the state unchanged and writes nothing.
  * Mamba-3 paper note, sections その1-その3 (recurrence above); the chunked form
  * follows the IBM Mamba page's SSD description (matrix form within a chunk,
  * state passed between chunks). */

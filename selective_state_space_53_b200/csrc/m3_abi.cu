@@ -150,6 +150,7 @@ WsLayout ws_layout(const m3_dims* dims) {
   m3::Params p = make_params(dims, dims->L, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                              nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
   if (!(dims->flags & M3_FLAG_SEQUENTIAL) && m3::tc_scan_supported(p)) w.scan = m3::tc_scan_workspace_bytes(p);
+  else if (!(dims->flags & M3_FLAG_SEQUENTIAL)) w.scan = m3::seq_scan_workspace_bytes(p);  // segments in parallel
   if ((dims->flags & M3_FLAG_RAW_INPUTS) && !fused_frontend(dims)) {
     const size_t e = dims->dtype == M3_BF16 ? 2 : 4;
     const size_t nbc = (size_t)(dims->b * dims->L) * dims->G * dims->R * dims->N;
@@ -296,7 +297,16 @@ m3_status m3_scan_fwd(const m3_dims* dims, const void* x, const float* dt, const
   m3::Params p = make_params(dims, dims->L, x, dt, A, lam, B, C, theta, bias_B, bias_C, W_x, W_o,
                              D, state, y);
   const bool tc = !(dims->flags & M3_FLAG_SEQUENTIAL) && m3::tc_scan_supported(p);
-  const WsLayout w = ws_layout(dims);
+  WsLayout w = ws_layout(dims);
+  // the sequential kernel's segments are optional: without the workspace they asked for, the
+  // sequences are walked whole, token by token (the front-end's part, if any, stays required)
+  if (!tc && w.scan > 0 && (workspace == nullptr || workspace_bytes < (w.fe_bytes ? w.fe_off + w.fe_bytes : w.scan))) {
+    const bool fe_fits = w.fe_bytes == 0 || (workspace != nullptr && workspace_bytes >= w.fe_bytes);
+    if (fe_fits) {
+      w.scan = 0;
+      w.fe_off = 0;
+    }
+  }
   const size_t need = w.fe_bytes ? w.fe_off + w.fe_bytes : w.scan;
   if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return M3_ERR_WORKSPACE;
   if (need > 0 && !aligned16(workspace)) return M3_ERR_ALIGN;
@@ -322,7 +332,9 @@ m3_status m3_scan_fwd(const m3_dims* dims, const void* x, const float* dt, const
     p.lam = tlam;
     p.raw_inputs = 0;
   }
-  const cudaError_t e = tc ? m3::launch_scan_tc(p, workspace, w.scan, s) : m3::launch_scan_sequential(p, s);
+  const cudaError_t e = tc                ? m3::launch_scan_tc(p, workspace, w.scan, s)
+                        : w.scan > 0      ? m3::launch_scan_seq_chunked(p, workspace, w.scan, s)
+                                          : m3::launch_scan_sequential(p, s);
   return cuda_status(e);
 }
 

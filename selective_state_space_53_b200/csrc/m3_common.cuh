@@ -126,6 +126,9 @@ class SmemAttr {
 
 // Launchers (defined in the kernel files); return cudaGetLastError() of the launch.
 cudaError_t launch_scan_sequential(const Params& p, cudaStream_t stream);
+// the chunk-parallel form of the sequential scan (segments summarised, folded, then scanned)
+size_t seq_scan_workspace_bytes(const Params& p);
+cudaError_t launch_scan_seq_chunked(const Params& p, void* ws, size_t ws_bytes, cudaStream_t stream);
 bool decode_supported(const Params& p);                       // one-token kernel fits on chip
 cudaError_t launch_decode(const Params& p, cudaStream_t stream);
 bool decode_tc_supported(const Params& p);                    // tensor-core form (d_state = headdim = 128, bf16)

@@ -16,6 +16,14 @@
 //     HBM-bound (8 bytes of state traffic per state element per token);
 //   * m3_scan_fwd for fp32 inputs, shapes the tensor-core scan does not cover,
 //     and M3_FLAG_SEQUENTIAL.
+//
+// With a workspace, m3_scan_fwd splits every sequence into segments walked in parallel (the scan
+// combines associatively over token ranges: IBM page "Mamba モデルとは", hardware-aware scan):
+// a first launch summarises segments 0..S-2 from a zero start (end state Z, total log decay,
+// total angle per pair), seq_fold_kernel folds the summaries into the state entering each
+// segment, h_k = e^{logdec} Rot(angle) (h_{k-1} + beta'_{t0} u_{t0-1}) + Z, and a second launch
+// scans every segment from its entering state, writing y (and, for the last one, the final
+// state and carry).
 #include "m3_common.cuh"
 
 namespace m3 {
@@ -61,14 +69,31 @@ __host__ __device__ inline SeqSmem seq_smem(int P, int N, int R, int KG) {
   return m;
 }
 
+// Segments of the chunk-parallel form (nseg = 1: the whole sequence in one block).
+struct SeqSegs {
+  int nseg;          // segments per sequence
+  int mode;          // 0: scan each segment from its entering state; 1: summaries of segments 0..nseg-2
+  int64_t seg_len;   // tokens per segment (the last may be shorter)
+  float* h_in;       // (b*H, nseg, N, P) state entering each segment (segments 1..nseg-1)
+  float* Z;          // (nseg-1, b*H, N, P) end state of each summarised segment from a zero start
+  float* logdec;     // (nseg-1, b*H) sum of dt A over the segment
+  double* angle;     // (nseg-1, b*H, N/2) sum of the rotation angles, reduced mod 2 pi
+};
+
 template <int RT, int NK, bool BF16>
 __global__ void __launch_bounds__(kThreads)
-scan_seq_kernel(Params p) {
+scan_seq_kernel(Params p, SeqSegs sgs) {
   extern __shared__ __align__(16) float sm[];
   const int tid = threadIdx.x;
   const int H = p.H, P = p.P, N = p.N, R = p.R, G = p.G;
   const int64_t L = p.L;
-  const int bi = blockIdx.x / H, hi = blockIdx.x % H;
+  const bool summary = sgs.mode == 1;
+  const int nsg = summary ? sgs.nseg - 1 : sgs.nseg;  // blocks per sequence
+  const int bh = blockIdx.x / nsg, seg = blockIdx.x % nsg;
+  const int64_t t0 = (int64_t)seg * sgs.seg_len;
+  const int64_t t1 = (t0 + sgs.seg_len < L) ? t0 + sgs.seg_len : L;
+  const bool last = !summary && seg == sgs.nseg - 1;
+  const int bi = bh / H, hi = bh % H;
   const int g = hi / (H / G);
   const SeqShape sh = seq_shape(P, N);
   const SeqSmem ms = seq_smem(P, N, R, sh.KG);
@@ -84,9 +109,11 @@ scan_seq_kernel(Params p) {
   float* const coef = sm + ms.coef;
   float* const red = sm + ms.red;
 
-  float* hbase = p.h + ((int64_t)blockIdx.x * N) * P;
-  float* cBb = p.carry_B + ((int64_t)blockIdx.x * R) * N;
-  float* cxb = p.carry_x + (int64_t)blockIdx.x * P;
+  // the entering state: the sequence's for segment 0, the folded one after it, zero in a summary
+  float* hstate = p.h + ((int64_t)bh * N) * P;
+  const float* hbase = seg == 0 ? hstate : sgs.h_in + ((int64_t)bh * sgs.nseg + seg) * N * P;
+  float* cBb = p.carry_B + ((int64_t)bh * R) * N;
+  float* cxb = p.carry_x + (int64_t)bh * P;
   const float* biasB = p.bias_B ? p.bias_B + (int64_t)hi * R * N : nullptr;
   const float* biasC = p.bias_C ? p.bias_C + (int64_t)hi * R * N : nullptr;
   const float* Wx = p.W_x ? p.W_x + (int64_t)hi * R * P : nullptr;
@@ -98,7 +125,7 @@ scan_seq_kernel(Params p) {
 #pragma unroll
   for (int j = 0; j < NK; ++j) {
     const int k = kg + j * sh.KG;
-    if (active && k < sh.K) {
+    if (active && k < sh.K && !summary) {
       h0[j] = *reinterpret_cast<const float4*>(hbase + (int64_t)(2 * k) * P + p0);
       h1[j] = *reinterpret_cast<const float4*>(hbase + (int64_t)(2 * k + 1) * P + p0);
     } else {
@@ -107,12 +134,26 @@ scan_seq_kernel(Params p) {
     }
   }
 
-  // ---- previous-token slot from the carry
-  for (int i = tid; i < R * N; i += kThreads) bbs[1][i] = cBb[i] + (biasB ? biasB[i] : 0.0f);
-  for (int i = tid; i < R * P; i += kThreads) xs[1][i] = cxb[i % P] * (Wx ? Wx[i] : 1.0f);
+  // ---- previous-token slot: the carry for segment 0, the token before the segment after it, none
+  //      in a summary (a fresh start)
+  if (summary) {
+    for (int i = tid; i < R * N; i += kThreads) bbs[1][i] = 0.0f;
+    for (int i = tid; i < R * P; i += kThreads) xs[1][i] = 0.0f;
+  } else if (seg == 0) {
+    for (int i = tid; i < R * N; i += kThreads) bbs[1][i] = cBb[i] + (biasB ? biasB[i] : 0.0f);
+    for (int i = tid; i < R * P; i += kThreads) xs[1][i] = cxb[i % P] * (Wx ? Wx[i] : 1.0f);
+  } else {
+    const int64_t tp = (int64_t)bi * L + t0 - 1;
+    for (int i = tid; i < R * N; i += kThreads)
+      bbs[1][i] = load_in<BF16>(p.B, ((tp * G + g) * R) * (int64_t)N + i) + (biasB ? biasB[i] : 0.0f);
+    for (int i = tid; i < R * P; i += kThreads)
+      xs[1][i] = load_in<BF16>(p.x, (tp * H + hi) * (int64_t)P + (i % P)) * (Wx ? Wx[i] : 1.0f);
+  }
+  float ldsum = 0.0f;   // summary: sum of dt A (thread 0)
+  double angsum = 0.0;  // summary: sum of the angles of pair tid (tid < N / 2)
 
   int cur = 0;
-  for (int64_t t = 0; t < L; ++t) {
+  for (int64_t t = t0; t < t1; ++t) {
     const int64_t tok = (int64_t)bi * L + t;
     // ---- stage token t
     {
@@ -128,14 +169,17 @@ scan_seq_kernel(Params p) {
       const float* th = p.theta + (tok * G + g) * (int64_t)(N / 2);
       for (int k = tid; k < N / 2; k += kThreads) {
         float s, c;
-        sincosf(p.angle_direct ? th[k] : delta * th[k], &s, &c);
+        const float phi = p.angle_direct ? th[k] : delta * th[k];
+        sincosf(phi, &s, &c);
         cs[k] = make_float2(c, s);
+        if (summary) angsum += (double)phi;
       }
       if (tid == 0) {
         const float lm = p.lam[tok * H + hi];
         coef[0] = expf(delta * p.A[tok * H + hi]);  // alpha
         coef[1] = (1.0f - lm) * delta;             // beta'
         coef[2] = lm * delta;                      // gamma
+        if (summary) ldsum += delta * p.A[tok * H + hi];
       }
     }
     __syncthreads();
@@ -211,7 +255,7 @@ scan_seq_kernel(Params p) {
     __syncthreads();
 
     // ---- combine: y = sum_r W_o[r] * (sum over pair groups) + D x
-    {
+    if (!summary) {
       const int64_t xoff = (tok * H + hi) * (int64_t)P;
       for (int pp = tid; pp < P; pp += kThreads) {
         float acc = 0.0f;
@@ -227,13 +271,29 @@ scan_seq_kernel(Params p) {
     cur ^= 1;
   }
 
-  // ---- state and carry back
+  // ---- a summary: Z, the total log decay and angles; else the last segment: state and carry back
+  if (summary) {
+    const int64_t si = (int64_t)seg * (p.b * H) + bh;
+    float* z = sgs.Z + si * N * P;
+#pragma unroll
+    for (int j = 0; j < NK; ++j) {
+      const int k = kg + j * sh.KG;
+      if (active && k < sh.K) {
+        *reinterpret_cast<float4*>(z + (int64_t)(2 * k) * P + p0) = h0[j];
+        *reinterpret_cast<float4*>(z + (int64_t)(2 * k + 1) * P + p0) = h1[j];
+      }
+    }
+    if (tid == 0) sgs.logdec[si] = ldsum;
+    if (tid < N / 2) sgs.angle[si * (N / 2) + tid] = angsum - 6.283185307179586 * rint(angsum * 0.15915494309189535);
+    return;
+  }
+  if (!last) return;
 #pragma unroll
   for (int j = 0; j < NK; ++j) {
     const int k = kg + j * sh.KG;
     if (active && k < sh.K) {
-      *reinterpret_cast<float4*>(hbase + (int64_t)(2 * k) * P + p0) = h0[j];
-      *reinterpret_cast<float4*>(hbase + (int64_t)(2 * k + 1) * P + p0) = h1[j];
+      *reinterpret_cast<float4*>(hstate + (int64_t)(2 * k) * P + p0) = h0[j];
+      *reinterpret_cast<float4*>(hstate + (int64_t)(2 * k + 1) * P + p0) = h1[j];
     }
   }
   if (L > 0) {
@@ -245,30 +305,130 @@ scan_seq_kernel(Params p) {
   }
 }
 
+// The state entering every segment s = 1..nseg-1: the sequence's state folded through the
+// summaries of segments 0..s-1 (thread = one column of one rotation pair).  The previous-token
+// term of segment s-1's first token t0 comes from the carry (s-1 = 0) or the input token t0 - 1.
+template <bool BF16>
+__global__ void __launch_bounds__(kThreads) seq_fold_kernel(const Params p, const SeqSegs sgs) {
+  const int bh = blockIdx.x;
+  const int H = p.H, P = p.P, N = p.N, R = p.R, G = p.G, K2 = N / 2;
+  const int bi = bh / H, hi = bh % H, g = hi / (H / G);
+  const int64_t L = p.L, nbh = p.b * H;
+  for (int idx = threadIdx.x; idx < K2 * P; idx += blockDim.x) {
+    const int k = idx / P, pc = idx % P;
+    float h0 = p.h[((int64_t)bh * N + 2 * k) * P + pc], h1 = p.h[((int64_t)bh * N + 2 * k + 1) * P + pc];
+    for (int s = 1; s < sgs.nseg; ++s) {
+      const int64_t t0 = (int64_t)(s - 1) * sgs.seg_len;  // first token of the folded segment
+      float u0 = 0.0f, u1 = 0.0f;
+      for (int r = 0; r < R; ++r) {
+        float b0, b1, xv;
+        if (s == 1) {
+          b0 = p.carry_B[((int64_t)bh * R + r) * N + 2 * k];
+          b1 = p.carry_B[((int64_t)bh * R + r) * N + 2 * k + 1];
+          xv = p.carry_x[(int64_t)bh * P + pc];
+        } else {
+          const int64_t tp = (int64_t)bi * L + t0 - 1;
+          b0 = load_in<BF16>(p.B, ((tp * G + g) * R + r) * (int64_t)N + 2 * k);
+          b1 = load_in<BF16>(p.B, ((tp * G + g) * R + r) * (int64_t)N + 2 * k + 1);
+          xv = load_in<BF16>(p.x, (tp * H + hi) * (int64_t)P + pc);
+        }
+        if (p.bias_B) {
+          b0 += p.bias_B[((int64_t)hi * R + r) * N + 2 * k];
+          b1 += p.bias_B[((int64_t)hi * R + r) * N + 2 * k + 1];
+        }
+        const float xr = (p.W_x ? p.W_x[((int64_t)hi * R + r) * P + pc] : 1.0f) * xv;
+        u0 = fmaf(b0, xr, u0);
+        u1 = fmaf(b1, xr, u1);
+      }
+      const int64_t tf = ((int64_t)bi * L + t0) * H + hi;
+      const float bp = (1.0f - p.lam[tf]) * p.dt[tf];
+      const int64_t si = (int64_t)(s - 1) * nbh + bh;
+      const float a0 = fmaf(bp, u0, h0), a1 = fmaf(bp, u1, h1);
+      const float dec = __expf(sgs.logdec[si]);
+      float sn, cn;
+      sincosf((float)sgs.angle[si * K2 + k], &sn, &cn);
+      const float* z = sgs.Z + (si * N + 2 * k) * P + pc;
+      h0 = fmaf(dec, cn * a0 - sn * a1, z[0]);
+      h1 = fmaf(dec, sn * a0 + cn * a1, z[P]);
+      float* hi_ = sgs.h_in + (((int64_t)bh * sgs.nseg + s) * N + 2 * k) * P + pc;
+      hi_[0] = h0;
+      hi_[P] = h1;
+    }
+  }
+}
+
 template <int RT, int NK>
-cudaError_t launch_rt_nk(const Params& p, size_t smem, cudaStream_t stream) {
-  const dim3 grid((unsigned)(p.b * p.H));
+cudaError_t launch_rt_nk(const Params& p, const SeqSegs& sgs, size_t smem, cudaStream_t stream) {
+  const int nsg = sgs.mode == 1 ? sgs.nseg - 1 : sgs.nseg;
+  const dim3 grid((unsigned)(p.b * p.H * nsg));
   if (p.dtype == M3_BF16) {
     auto k = scan_seq_kernel<RT, NK, true>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, kThreads, smem, stream>>>(p);
+    k<<<grid, kThreads, smem, stream>>>(p, sgs);
   } else {
     auto k = scan_seq_kernel<RT, NK, false>;
     if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, kThreads, smem, stream>>>(p);
+    k<<<grid, kThreads, smem, stream>>>(p, sgs);
   }
   return cudaGetLastError();
 }
 
 template <int RT>
-cudaError_t launch_rt(const Params& p, int nk, size_t smem, cudaStream_t stream) {
+cudaError_t launch_rt(const Params& p, const SeqSegs& sgs, int nk, size_t smem, cudaStream_t stream) {
   switch (nk) {
-    case 1: return launch_rt_nk<RT, 1>(p, smem, stream);
-    case 2: return launch_rt_nk<RT, 2>(p, smem, stream);
-    case 4: return launch_rt_nk<RT, 4>(p, smem, stream);
-    case 8: return launch_rt_nk<RT, 8>(p, smem, stream);
-    default: return launch_rt_nk<RT, 16>(p, smem, stream);
+    case 1: return launch_rt_nk<RT, 1>(p, sgs, smem, stream);
+    case 2: return launch_rt_nk<RT, 2>(p, sgs, smem, stream);
+    case 4: return launch_rt_nk<RT, 4>(p, sgs, smem, stream);
+    case 8: return launch_rt_nk<RT, 8>(p, sgs, smem, stream);
+    default: return launch_rt_nk<RT, 16>(p, sgs, smem, stream);
   }
+}
+
+cudaError_t launch_seq(const Params& p, const SeqSegs& sgs, cudaStream_t stream) {
+  const SeqShape sh = seq_shape(p.P, p.N);
+  int nk = (sh.K + sh.KG - 1) / sh.KG;
+  int nk2 = 1;
+  while (nk2 < nk) nk2 *= 2;
+  const size_t smem = sizeof(float) * (size_t)seq_smem(p.P, p.N, p.R, sh.KG).total;
+  if (p.R <= 1) return launch_rt<1>(p, sgs, nk2, smem, stream);
+  if (p.R <= 2) return launch_rt<2>(p, sgs, nk2, smem, stream);
+  if (p.R <= 4) return launch_rt<4>(p, sgs, nk2, smem, stream);
+  return launch_rt<8>(p, sgs, nk2, smem, stream);
+}
+
+// Segments per sequence for the chunk-parallel form: enough blocks for two per SM, at least 32
+// tokens per segment, at most 64 segments, and a workspace (entering states and summaries) of
+// at most 12 MiB; 1 means the plain token-sequential walk.
+constexpr size_t kSeqWsCap = size_t(12) << 20;
+int seq_segments(const Params& p, int64_t* seg_len) {
+  int dev = 0, nsm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t nbh = p.b * p.H;
+  int64_t s = nbh > 0 ? (2 * (int64_t)nsm + nbh - 1) / nbh : 1;
+  if (s > p.L / 32) s = p.L / 32;
+  if (s > 64) s = 64;
+  const size_t per = 2 * (size_t)nbh * p.N * p.P * 4 + (size_t)nbh * (4 + 8 * (p.N / 2));
+  while (s > 1 && per * (size_t)s > kSeqWsCap) --s;
+  if (s < 2) {
+    *seg_len = p.L;
+    return 1;
+  }
+  *seg_len = (p.L + s - 1) / s;
+  return (int)((p.L + *seg_len - 1) / *seg_len);
+}
+
+struct SeqWs {
+  size_t h_in, z, ld, ang, total;
+};
+SeqWs seq_ws(const Params& p, int nseg) {
+  const size_t nbh = (size_t)(p.b * p.H), np = (size_t)p.N * p.P;
+  SeqWs w{};
+  w.h_in = 0;
+  w.z = (4 * nbh * nseg * np + 255) & ~(size_t)255;
+  w.ld = w.z + ((4 * nbh * (nseg - 1) * np + 255) & ~(size_t)255);
+  w.ang = w.ld + ((4 * nbh * (nseg - 1) + 255) & ~(size_t)255);
+  w.total = w.ang + 8 * nbh * (nseg - 1) * (p.N / 2);
+  return w;
 }
 
 }  // namespace
@@ -282,15 +442,43 @@ bool seq_scan_supported(int P, int N, int R) {
 
 cudaError_t launch_scan_sequential(const Params& p, cudaStream_t stream) {
   if (p.b * p.H == 0) return cudaSuccess;
-  const SeqShape sh = seq_shape(p.P, p.N);
-  int nk = (sh.K + sh.KG - 1) / sh.KG;
-  int nk2 = 1;
-  while (nk2 < nk) nk2 *= 2;
-  const size_t smem = sizeof(float) * (size_t)seq_smem(p.P, p.N, p.R, sh.KG).total;
-  if (p.R <= 1) return launch_rt<1>(p, nk2, smem, stream);
-  if (p.R <= 2) return launch_rt<2>(p, nk2, smem, stream);
-  if (p.R <= 4) return launch_rt<4>(p, nk2, smem, stream);
-  return launch_rt<8>(p, nk2, smem, stream);
+  SeqSegs one{};
+  one.nseg = 1;
+  one.mode = 0;
+  one.seg_len = p.L;
+  return launch_seq(p, one, stream);
+}
+
+size_t seq_scan_workspace_bytes(const Params& p) {
+  int64_t len = 0;
+  const int nseg = seq_segments(p, &len);
+  return nseg > 1 ? seq_ws(p, nseg).total : 0;
+}
+
+cudaError_t launch_scan_seq_chunked(const Params& p, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (p.b * p.H == 0) return cudaSuccess;
+  int64_t len = 0;
+  const int nseg = seq_segments(p, &len);
+  if (nseg < 2) return launch_scan_sequential(p, stream);
+  const SeqWs w = seq_ws(p, nseg);
+  if (ws == nullptr || ws_bytes < w.total) return cudaErrorInvalidValue;
+  char* b = static_cast<char*>(ws);
+  SeqSegs sg{};
+  sg.nseg = nseg;
+  sg.seg_len = len;
+  sg.h_in = reinterpret_cast<float*>(b + w.h_in);
+  sg.Z = reinterpret_cast<float*>(b + w.z);
+  sg.logdec = reinterpret_cast<float*>(b + w.ld);
+  sg.angle = reinterpret_cast<double*>(b + w.ang);
+  sg.mode = 1;
+  cudaError_t e = launch_seq(p, sg, stream);
+  if (e != cudaSuccess) return e;
+  if (p.dtype == M3_BF16) seq_fold_kernel<true><<<(unsigned)(p.b * p.H), kThreads, 0, stream>>>(p, sg);
+  else seq_fold_kernel<false><<<(unsigned)(p.b * p.H), kThreads, 0, stream>>>(p, sg);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  sg.mode = 0;
+  return launch_seq(p, sg, stream);
 }
 
 }  // namespace m3
