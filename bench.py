@@ -358,7 +358,7 @@ def run_ours(args):
     if decode is not None and not args.no_decode_sweep:
         # the rest of the decode batch sweep of the 1.5B-scale layer, one line each
         decode["sweep"] = {}
-        for nm in ("decode_b1", "decode_b16", "decode_b512"):
+        for nm in ("decode_b1", "decode_b16", "decode_b512", "decode_p1_b128"):
             r = run_decode(args, device, peaks, nm)
             decode["sweep"][nm] = {k: r[k] for k in ("us_per_step", "tokens_per_s", "hbm_gbs", "hbm_frac_of_measured")}
             torch.cuda.empty_cache()
@@ -473,8 +473,9 @@ def run_decode(args, device, peaks, name=DECODE_WORKLOAD):
     by = decode_bytes(cfg)
     fl = decode_flops(cfg)
     del g
-    return {"workload": "%s: m3_decode_step, b%d H32 P128 N128 R4, CUDA graph of %d steps over %d state(s) "
-                        "(%.0f MiB)" % (name, cfg["b"], steps, n_states, n_states * state_bytes / 2 / 2**20),
+    return {"workload": "%s: m3_decode_step, b%d H%d P%d N%d R%d, CUDA graph of %d steps over %d state(s) "
+                        "(%.0f MiB)" % (name, cfg["b"], cfg["H"], cfg["P"], cfg["N"], cfg["R"], steps, n_states,
+                                        n_states * state_bytes / 2 / 2**20),
             "tokens_per_s": cfg["b"] / (ms * 1e-3), "us_per_step": ms * 1e3,
             "hbm_gbs": by / (ms * 1e-3) / 1e9, "hbm_frac_of_measured": by / (ms * 1e-3) / 1e9 / peaks["hbm"],
             "tflops": fl / (ms * 1e-3) / 1e12, "algorithmic_bytes": by}

@@ -50,12 +50,14 @@ CONFIGS = {
     "decode_b16": dict(b=16, L=1024, H=32, P=128, N=128, R=4, G=1, dtype="bf16"),
     "decode_b128": dict(b=128, L=1024, H=32, P=128, N=128, R=4, G=1, dtype="bf16"),
     "decode_b512": dict(b=512, L=1024, H=32, P=128, N=128, R=4, G=1, dtype="bf16"),
+    # decode on the page-1 layer (N = P = 64, R = 2) at batch 128
+    "decode_p1_b128": dict(b=128, L=1024, H=24, P=64, N=64, R=2, G=1, dtype="bf16"),
 }
 
 # seed = 1000 + index of the workload family in the list above's families
 SEEDS = {"tiny_f32": 1000, "p1_layer": 1001, "p1_stack": 1002,
          "l15b_2k": 1003, "l15b_8k": 1003, "l15b_32k": 1003,
-         "decode_b1": 1004, "decode_b16": 1004, "decode_b128": 1004, "decode_b512": 1004}
+         "decode_b1": 1004, "decode_b16": 1004, "decode_b128": 1004, "decode_b512": 1004, "decode_p1_b128": 1001}
 
 _CHUNK = 1 << 22  # draws are made in blocks of this many values to bound host memory
 

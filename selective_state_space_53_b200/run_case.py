@@ -5,7 +5,7 @@
 
 The inputs are the seeded draw of the workload (``inputs.config_inputs``), uploaded once;
 each call runs through the C ABI on the current stream, and the library's error flag is
-checked at the end.  ``--L`` shortens the sequence (a smaller capture of the same kernel),
+checked at the end.  ``--L`` (and ``--b --H --P --N --R``) override the workload's sizes (a smaller capture of the same kernel),
 ``--raw`` passes the draw as raw projections (M3_FLAG_RAW_INPUTS).  Prints one line with the
 mean time of the calls (CUDA events; not a bench figure under a profiler).
 """
@@ -22,6 +22,8 @@ def main():
     ap.add_argument("--op", choices=["scan", "decode", "bwd"], default="scan")
     ap.add_argument("--calls", type=int, default=3)
     ap.add_argument("--L", type=int, default=0, help="sequence length override")
+    for k in ("b", "H", "P", "N", "R"):
+        ap.add_argument("--" + k, type=int, default=0, help=f"{k} override")
     ap.add_argument("--raw", action="store_true")
     args = ap.parse_args()
 
@@ -31,8 +33,9 @@ def main():
 
     cfg = dict(CONFIGS[args.workload])
     cfg.pop("layers", None)
-    if args.L:
-        cfg["L"] = args.L
+    for k in ("L", "b", "H", "P", "N", "R"):
+        if getattr(args, k):
+            cfg[k] = getattr(args, k)
     seed = SEEDS.get(args.workload, 0)
     if args.raw:
         inp = make_raw_inputs(seed=seed, **cfg)
