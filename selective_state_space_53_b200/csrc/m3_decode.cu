@@ -27,47 +27,51 @@ __device__ __forceinline__ uint64_t globaltimer() {
 }
 
 // ------------------------------------------------------------------ ring form
-// Persistent form: each CTA walks a contiguous range of (batch, head) units, ordered head-major
-// so that the per-head weights change at most a few times per CTA.  A unit's state tile is
-// taken in `split` blocks of N / split rows (the readouts are summed over the blocks in shared
-// memory), and the CTA keeps `stages` blocks in flight: while it updates one, the TMA engine
-// brings the next blocks (state rows and raw token operands) into a ring of shared-memory
-// stages.  Blocks are sized so that two CTAs fit per SM where possible, one CTA's
-// operand staging and barriers overlapping the other's arithmetic.  The updated state goes
-// straight from registers to HBM, so the copy engine only ever reads.
+// Persistent form: each CTA takes a contiguous range of (batch, head) units, ordered head-major
+// so that the per-head weights change at most a few times per CTA.  The CTA's threads form
+// `teams` independent teams (named barriers, no CTA-wide synchronisation after set-up); team t
+// walks units t, t + teams, ... of the range, so that while one team waits on a barrier or on
+// its copies the others update theirs.  A unit's state tile is taken in `split` blocks of
+// N / split rows (the readouts are summed over the blocks in shared memory), and each team
+// keeps `stages` blocks in flight: while it updates one, the TMA engine brings the next blocks
+// (state rows and raw token operands) into the team's ring of shared-memory stages.  The
+// updated state goes straight from registers to HBM, so the copy engine only ever reads.
 
 constexpr int kMaxStages = 6;
 constexpr int kRingThreads = 512;
-constexpr int kRingCtas = kRingThreads <= 256 ? 2 : 1;  // CTAs per SM the registers allow
-constexpr int kRingMinStages = 2;  // stages a plan must fit before a larger split is tried
+constexpr int kMaxTeams = 4;
 
 struct RingPlan {
-  int stages, split, ctas_per_sm;
-  uint32_t stage_bytes;
+  int stages, split, teams, team_threads;
+  uint32_t stage_bytes, team_bytes;
   // byte offsets inside a stage: state rows of the block, raw B_t, raw C_t, carry_B, raw x_t,
   // carry_x, theta_t, and the three per-unit scalars dt, A, lam
   uint32_t o_st, o_b, o_c, o_cb, o_x, o_cx, o_th, o_sc;
-  // byte offsets of the single-buffered arrays after the ring: the block's biased B, C and the
-  // MIMO branches, the rotation table and coefficients, the weights of the current head
-  // (bias_B, bias_C, W_x, W_o) and the per-pair-group partial readouts of every block
+  // byte offsets (inside a team's region, after its stages) of the single-buffered arrays: the
+  // block's biased B, C and the MIMO branches, the rotation table and coefficients, the weights
+  // of the current head (bias_B, bias_C, W_x, W_o) and the per-pair-group partial readouts of
+  // every block of the unit
   uint32_t o_bbc, o_bbp, o_cbb, o_xc, o_xp, o_xr, o_cs, o_coef, o_wb, o_wc, o_wx, o_wo, o_red, o_bar;
   uint32_t total;
 };
 
-// thread (pq, kg): columns 4 pq .. 4 pq + 3, rotation pairs kg, kg + KG, ... of the block
+// thread (pq, kg) of a team: columns 4 pq .. 4 pq + 3, rotation pairs kg, kg + KG, ... of the block
 __host__ __device__ inline int ring_pq(int P) { return P / 4; }
-__host__ __device__ inline int ring_kg(int P, int NB) {
-  const int kg = kRingThreads / ring_pq(P);
+__host__ __device__ inline int ring_kg(int P, int NB, int team_threads) {
+  const int kg = team_threads / ring_pq(P);
   return kg < NB / 2 ? kg : NB / 2;
 }
 
 __host__ __device__ inline uint32_t pad16(uint32_t x) { return (x + 15u) & ~15u; }
 
-inline RingPlan ring_plan(int P, int N, int R, bool bf16, int split, int max_bytes) {
+// Layout of one team's region for `teams` teams sharing max_bytes; stages = 0 if none fits.
+inline RingPlan ring_plan(int P, int N, int R, bool bf16, int split, int teams, int max_bytes) {
   const uint32_t esz = bf16 ? 2u : 4u;
   const int NB = N / split;
   RingPlan rp{};
   rp.split = split;
+  rp.teams = teams;
+  rp.team_threads = kRingThreads / teams;
   uint32_t o = 0;
   rp.o_st = o; o += pad16((uint32_t)NB * P * 4);
   rp.o_b = o;  o += pad16((uint32_t)R * N * esz);
@@ -91,16 +95,18 @@ inline RingPlan ring_plan(int P, int N, int R, bool bf16, int split, int max_byt
   rp.o_wc = f; f += pad16((uint32_t)R * N * 4);
   rp.o_wx = f; f += pad16((uint32_t)R * P * 4);
   rp.o_wo = f; f += pad16((uint32_t)R * P * 4);
-  rp.o_red = f; f += pad16((uint32_t)split * ring_kg(P, NB) * P * 4);
+  rp.o_red = f; f += pad16((uint32_t)split * ring_kg(P, NB, rp.team_threads) * P * 4);
   rp.o_bar = f; f += 8 * kMaxStages;
-  const int room = max_bytes - (int)f;
+  f = (f + 127u) & ~127u;
+  const int room = max_bytes / teams - (int)f;
   int st = room > 0 ? room / (int)rp.stage_bytes : 0;
   rp.stages = st < kMaxStages ? st : kMaxStages;
   const uint32_t ring = (uint32_t)rp.stages * rp.stage_bytes;
   rp.o_bbc += ring; rp.o_bbp += ring; rp.o_cbb += ring; rp.o_xc += ring; rp.o_xp += ring;
   rp.o_xr += ring; rp.o_cs += ring; rp.o_coef += ring; rp.o_wb += ring; rp.o_wc += ring;
   rp.o_wx += ring; rp.o_wo += ring; rp.o_red += ring; rp.o_bar += ring;
-  rp.total = ring + f;
+  rp.team_bytes = ring + f;
+  rp.total = rp.team_bytes * (uint32_t)teams;
   return rp;
 }
 
@@ -108,6 +114,21 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                "l"(src), "r"(bytes), "r"(bar)
                : "memory");
+}
+
+// named barrier of one team (id >= 1; id 0 is __syncthreads)
+__device__ __forceinline__ void team_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// named barrier that also returns whether any thread of the team passed `pred` true
+__device__ __forceinline__ bool team_sync_or(int id, int nthreads, bool pred) {
+  uint32_t any;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(any)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return any != 0;
 }
 
 template <bool BF16>
@@ -119,18 +140,39 @@ __device__ __forceinline__ float stage_in(const unsigned char* base, int i) {
   }
 }
 
+// Position of a team in its walk: unit u (head-major: head hi, sequence bi) and block blk.
+struct RingCursor {
+  int64_t bi;
+  int hi, blk;
+  __device__ __forceinline__ void next(int split, int teams, int64_t nb) {
+    if (++blk < split) return;
+    blk = 0;
+    bi += teams;
+    while (bi >= nb) {
+      bi -= nb;
+      ++hi;
+    }
+  }
+};
+
 template <int RT, bool BF16>
-__global__ void __launch_bounds__(kRingThreads, kRingCtas) decode_ring_kernel(Params p, RingPlan rp) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const int tid = threadIdx.x;
+__global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, RingPlan rp) {
+  extern __shared__ __align__(128) unsigned char smem_cta[];
+  const int TT = rp.team_threads;
+  const int team = threadIdx.x / TT;
+  const int tid = threadIdx.x % TT;
+  const int bar_id = 1 + team;
+  unsigned char* smem = smem_cta + (size_t)team * rp.team_bytes;
   const int H = p.H, P = p.P, N = p.N, R = p.R, G = p.G;
   const int SPL = rp.split;
   const int NB = N / SPL;  // state rows per block
+  const int T = rp.teams;
   const int64_t nb = p.b;
   const int64_t U = nb * H;
-  // blocks v = unit * SPL + block index; this CTA takes the blocks of units [u0, u1)
-  const int64_t v0 = (int64_t)blockIdx.x * U / gridDim.x * SPL;
-  const int64_t v1 = (int64_t)(blockIdx.x + 1) * U / gridDim.x * SPL;
+  // this CTA's units [u0, u1); the team takes u0 + team, u0 + team + T, ..., each in SPL blocks
+  const int64_t u0 = (int64_t)blockIdx.x * U / gridDim.x;
+  const int64_t u1 = (int64_t)(blockIdx.x + 1) * U / gridDim.x;
+  const int64_t nv = (u0 + team < u1 ? (u1 - u0 - team + T - 1) / T : 0) * SPL;
   const int S = rp.stages;
   constexpr uint32_t esz = BF16 ? 2u : 4u;
   const uint32_t sbase = smem_u32(smem);
@@ -148,15 +190,15 @@ __global__ void __launch_bounds__(kRingThreads, kRingCtas) decode_ring_kernel(Pa
   float* wo = reinterpret_cast<float*>(smem + rp.o_wo);
   float* red = reinterpret_cast<float*>(smem + rp.o_red);
   const uint32_t bar0 = sbase + rp.o_bar;
+  RingCursor first{0, 0, 0};
+  if (nv > 0) {
+    first.bi = (u0 + team) % nb;
+    first.hi = (int)((u0 + team) / nb);
+  }
 
-  // unit u = head-major index: head u / b, sequence u % b
-  auto issue = [&](int64_t v, int s) {
-    const int64_t u = v / SPL;
-    const int blk = (int)(v % SPL);
-    const int64_t bi = u % nb;
-    const int hi = (int)(u / nb);
-    const int g = hi / (H / G);
-    const int64_t bh = bi * H + hi;
+  auto issue = [&](const RingCursor& c, int s) {
+    const int g = c.hi / (H / G);
+    const int64_t bh = c.bi * H + c.hi;
     const uint32_t st = sbase + (uint32_t)s * rp.stage_bytes;
     const uint32_t bar = bar0 + 8u * s;
     const uint32_t n_st = (uint32_t)NB * P * 4, n_b = (uint32_t)R * N * esz, n_cb = (uint32_t)R * N * 4;
@@ -164,14 +206,14 @@ __global__ void __launch_bounds__(kRingThreads, kRingCtas) decode_ring_kernel(Pa
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
                  "r"(n_st + 2 * n_b + n_cb + n_x + n_cx + n_th)
                  : "memory");
-    const int64_t bc = ((bi * G + g) * R) * (int64_t)N;
-    bulk_g2s(st + rp.o_st, p.h + (bh * N + (int64_t)blk * NB) * P, n_st, bar);
+    const int64_t bc = ((c.bi * G + g) * R) * (int64_t)N;
+    bulk_g2s(st + rp.o_st, p.h + (bh * N + (int64_t)c.blk * NB) * P, n_st, bar);
     bulk_g2s(st + rp.o_b, static_cast<const unsigned char*>(p.B) + bc * esz, n_b, bar);
     bulk_g2s(st + rp.o_c, static_cast<const unsigned char*>(p.C) + bc * esz, n_b, bar);
     bulk_g2s(st + rp.o_cb, p.carry_B + bh * R * N, n_cb, bar);
     bulk_g2s(st + rp.o_x, static_cast<const unsigned char*>(p.x) + bh * P * esz, n_x, bar);
     bulk_g2s(st + rp.o_cx, p.carry_x + bh * P, n_cx, bar);
-    bulk_g2s(st + rp.o_th, p.theta + (bi * G + g) * (N / 2), n_th, bar);
+    bulk_g2s(st + rp.o_th, p.theta + (c.bi * G + g) * (N / 2), n_th, bar);
     // the three scalars: 4-byte asynchronous copies whose completion is the barrier's second arrival
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(st + rp.o_sc), "l"(p.dt + bh) : "memory");
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(st + rp.o_sc + 4), "l"(p.A + bh) : "memory");
@@ -196,16 +238,20 @@ __global__ void __launch_bounds__(kRingThreads, kRingCtas) decode_ring_kernel(Pa
     return true;
   };
 
+  RingCursor ahead = first;  // the next block to issue (the team leader's)
   if (tid == 0) {
     for (int s = 0; s < S; ++s)
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 2;" ::"r"(bar0 + 8u * s));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    for (int s = 0; s < S && v0 + s < v1; ++s) issue(v0 + s, s);
+    for (int s = 0; s < S && s < nv; ++s) {
+      issue(ahead, s);
+      ahead.next(SPL, T, nb);
+    }
   }
-  __syncthreads();
+  __syncthreads();  // barriers initialised (the only CTA-wide synchronisation)
 
   const int PQ = ring_pq(P);
-  const int KG = ring_kg(P, NB);
+  const int KG = ring_kg(P, NB, TT);
   const int pq = tid % PQ;
   const int kg = tid / PQ;
   constexpr int CQ = 1;  // 4-column quads per thread (the compute below takes any count)
@@ -214,34 +260,33 @@ __global__ void __launch_bounds__(kRingThreads, kRingCtas) decode_ring_kernel(Pa
   uint32_t phases = 0;  // bit s: parity of the next completion of stage s
   int s = 0;
   bool ok = true;
-  int64_t v = v0;
-  for (; v < v1; ++v) {
+  RingCursor cur = first;
+  int64_t j = 0;
+  for (; j < nv; ++j) {
     const uint32_t par = (phases >> s) & 1u;
     phases ^= 1u << s;
-    const int64_t u = v / SPL;
-    const int blk = (int)(v % SPL);
+    const int blk = cur.blk;
     const bool last_blk = blk == SPL - 1;
-    const int64_t bi = u % nb;
-    const int hi = (int)(u / nb);
-    const int64_t bh = bi * H + hi;
+    const int hi = cur.hi;
+    const int64_t bh = cur.bi * H + hi;
     const unsigned char* stg = smem + (size_t)s * rp.stage_bytes;
-    if (hi != cur_h) {  // weights of a new head (uniform: every thread sees the same unit)
+    if (hi != cur_h) {  // weights of a new head (uniform: the whole team sees the same unit)
       cur_h = hi;
-      __syncthreads();  // the previous block's update has read W_o
+      team_sync(bar_id, TT);  // the previous block's update has read W_o
       const float* biasB = p.bias_B ? p.bias_B + (int64_t)hi * R * N : nullptr;
       const float* biasC = p.bias_C ? p.bias_C + (int64_t)hi * R * N : nullptr;
       const float* Wx = p.W_x ? p.W_x + (int64_t)hi * R * P : nullptr;
       const float* Wo = p.W_o ? p.W_o + (int64_t)hi * R * P : nullptr;
-      for (int i = tid; i < R * N; i += kRingThreads) {
+      for (int i = tid; i < R * N; i += TT) {
         wb[i] = biasB ? biasB[i] : 0.0f;
         wc[i] = biasC ? biasC[i] : 0.0f;
       }
-      for (int i = tid; i < R * P; i += kRingThreads) {
+      for (int i = tid; i < R * P; i += TT) {
         wx[i] = Wx ? Wx[i] : 1.0f;
         wo[i] = Wo ? Wo[i] : 1.0f;
       }
       Dh = p.D ? p.D[hi] : 0.0f;
-      __syncthreads();
+      team_sync(bar_id, TT);
     }
     ok = wait(s, par);
     if (ok) {
@@ -251,20 +296,20 @@ __global__ void __launch_bounds__(kRingThreads, kRingCtas) decode_ring_kernel(Pa
       const float* cxs = reinterpret_cast<const float*>(stg + rp.o_cx);
       const float* ths = reinterpret_cast<const float*>(stg + rp.o_th);
       const int n0 = blk * NB;
-      for (int i = tid; i < R * NB; i += kRingThreads) {
+      for (int i = tid; i < R * NB; i += TT) {
         const int r = i / NB, n = n0 + i % NB;
         const float bb = wb[r * N + n];
         bbc[i] = stage_in<BF16>(stg + rp.o_b, r * N + n) + bb;
         bbp[i] = cBs[r * N + n] + bb;
         cbb[i] = stage_in<BF16>(stg + rp.o_c, r * N + n) + wc[r * N + n];
       }
-      for (int i = tid; i < R * P; i += kRingThreads) {
+      for (int i = tid; i < R * P; i += TT) {
         const float w = wx[i];
         xc[i] = stage_in<BF16>(stg + rp.o_x, i % P) * w;
         xp[i] = cxs[i % P] * w;
       }
       const float delta = sc[0];
-      for (int k = tid; k < NB / 2; k += kRingThreads) {
+      for (int k = tid; k < NB / 2; k += TT) {
         float sn, cn;
         sincosf(p.angle_direct ? ths[n0 / 2 + k] : delta * ths[n0 / 2 + k], &sn, &cn);
         cs[k] = make_float2(cn, sn);
@@ -280,17 +325,17 @@ __global__ void __launch_bounds__(kRingThreads, kRingCtas) decode_ring_kernel(Pa
         // carry (this token's raw B and x) may overwrite it
         float* cBg = p.carry_B + bh * R * N;
         float* cxg = p.carry_x + bh * P;
-        for (int i = tid; i < R * N; i += kRingThreads) cBg[i] = stage_in<BF16>(stg + rp.o_b, i);
-        for (int pp = tid; pp < P; pp += kRingThreads) {
+        for (int i = tid; i < R * N; i += TT) cBg[i] = stage_in<BF16>(stg + rp.o_b, i);
+        for (int pp = tid; pp < P; pp += TT) {
           const float xv = stage_in<BF16>(stg + rp.o_x, pp);
           xr[pp] = xv;
           cxg[pp] = xv;
         }
       }
     }
-    if (__syncthreads_or(!ok)) {
+    if (team_sync_or(bar_id, TT, !ok)) {
       ok = false;
-      phases ^= 1u << s;  // block v's copies count as outstanding again
+      phases ^= 1u << s;  // block j's copies count as outstanding again
       break;
     }
     // ---- state update of the thread's 4 columns over its rotation pairs of the block
@@ -389,12 +434,15 @@ __global__ void __launch_bounds__(kRingThreads, kRingCtas) decode_ring_kernel(Pa
         *reinterpret_cast<float4*>(red + (blk * KG + kg) * P + pc[c]) = make_float4(o[0], o[1], o[2], o[3]);
       }
     }
-    __syncthreads();  // stage s is read; the block's readouts are in place
-    if (tid == 0 && v + S < v1) issue(v + S, s);
+    team_sync(bar_id, TT);  // stage s is read; the block's readouts are in place
+    if (tid == 0 && j + S < nv) {
+      issue(ahead, s);
+      ahead.next(SPL, T, nb);
+    }
     if (last_blk) {
       // ---- y = sum_r W_o[r] * readout_r + D x, the readouts summed over groups and blocks
       const int nq = SPL * KG;
-      for (int pp = tid; pp < P; pp += kRingThreads) {
+      for (int pp = tid; pp < P; pp += TT) {
         float acc0 = 0.0f, acc1 = 0.0f;
         int q = 0;
         for (; q + 1 < nq; q += 2) {
@@ -406,12 +454,13 @@ __global__ void __launch_bounds__(kRingThreads, kRingCtas) decode_ring_kernel(Pa
       }
     }
     s = (s + 1 == S) ? 0 : s + 1;
+    cur.next(SPL, T, nb);
   }
   if (!ok) {
-    // give up: wait (bounded) for the copies still in flight, then report
+    // give up: wait (bounded) for the team's copies still in flight, then report
     if (tid == 0) {
-      for (int64_t w = v; w < v1 && w < v + S; ++w) {
-        const int sw = (int)((w - v0) % S);
+      for (int64_t w = j; w < nv && w < j + S; ++w) {
+        const int sw = (int)(w % S);
         wait(sw, (phases >> sw) & 1u);
       }
       set_status(p.status, M3_ERR_TIMEOUT);
@@ -458,26 +507,23 @@ cudaError_t launch_ring_rt(const Params& p, const RingPlan& rp, unsigned grid, c
   return cudaGetLastError();
 }
 
-// The ring form needs two stages on chip at least.  Preferred: two CTAs per SM with the fewest
-// row blocks per unit; else one CTA per SM with the fewest blocks.
+// The ring form needs two stages per team at least.  Preferred: the most teams (units in flight
+// per CTA) whose threads each get a column quad, at the fewest row blocks per unit.
 bool ring_plan_for(const Params& p, RingPlan* out) {
   const DeviceLimits d = device_limits();
   if (d.sms == 0) return false;
   const bool bf16 = p.dtype == M3_BF16;
-  for (int min_stages = kRingMinStages; min_stages >= 2; --min_stages)
-    for (int ctas = kRingCtas; ctas >= 1; --ctas) {
-      // 1 KiB of each SM's shared memory is reserved per resident CTA
-      const int room = ctas == 1 ? d.smem_optin : d.smem_sm / ctas - 1024;
-      for (int split = 1; split <= 4; split *= 2) {
-        if (p.N % (2 * split) != 0 || (p.N / split) % 8 != 0) break;
-        RingPlan rp = ring_plan(p.P, p.N, p.R, bf16, split, room < d.smem_optin ? room : d.smem_optin);
-        if (rp.stages >= min_stages) {
-          rp.ctas_per_sm = ctas;
-          *out = rp;
-          return true;
-        }
+  for (int teams = kMaxTeams; teams >= 1; teams /= 2) {
+    if (kRingThreads / teams < ring_pq(p.P)) continue;
+    for (int split = 1; split <= 4; split *= 2) {
+      if (p.N % (2 * split) != 0 || (p.N / split) % 8 != 0) break;
+      const RingPlan rp = ring_plan(p.P, p.N, p.R, bf16, split, teams, d.smem_optin);
+      if (rp.stages >= 2) {
+        *out = rp;
+        return true;
       }
     }
+  }
   return false;
 }
 
@@ -495,7 +541,7 @@ cudaError_t launch_decode(const Params& p, cudaStream_t stream) {
   RingPlan rp;
   if (ring_plan_for(p, &rp)) {
     const int64_t units = p.b * p.H;
-    const int64_t slots = (int64_t)device_limits().sms * rp.ctas_per_sm;
+    const int64_t slots = device_limits().sms;
     const unsigned grid = (unsigned)(units < slots ? units : slots);
     if (p.R <= 1) return launch_ring_rt<1>(p, rp, grid, stream);
     if (p.R <= 2) return launch_ring_rt<2>(p, rp, grid, stream);

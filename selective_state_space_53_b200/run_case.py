@@ -5,7 +5,8 @@
 
 The inputs are the seeded draw of the workload (``inputs.config_inputs``), uploaded once;
 each call runs through the C ABI on the current stream, and the library's error flag is
-checked at the end.  ``--L`` (and ``--b --H --P --N --R``) override the workload's sizes (a smaller capture of the same kernel),
+checked at the end.  ``--L`` (and ``--b --H --P --N --R``, ``--dtype``) override the workload's sizes and storage type
+(a smaller capture of the same kernel, or another kernel's shape);
 ``--raw`` passes the draw as raw projections (M3_FLAG_RAW_INPUTS).  Prints one line with the
 mean time of the calls (CUDA events; not a bench figure under a profiler).
 """
@@ -24,6 +25,7 @@ def main():
     ap.add_argument("--L", type=int, default=0, help="sequence length override")
     for k in ("b", "H", "P", "N", "R"):
         ap.add_argument("--" + k, type=int, default=0, help=f"{k} override")
+    ap.add_argument("--dtype", choices=["bf16", "f32"], default=None, help="storage dtype override")
     ap.add_argument("--raw", action="store_true")
     args = ap.parse_args()
 
@@ -36,6 +38,8 @@ def main():
     for k in ("L", "b", "H", "P", "N", "R"):
         if getattr(args, k):
             cfg[k] = getattr(args, k)
+    if args.dtype:
+        cfg["dtype"] = args.dtype
     seed = SEEDS.get(args.workload, 0)
     if args.raw:
         inp = make_raw_inputs(seed=seed, **cfg)

@@ -167,20 +167,29 @@ def test_decode_layer_shape_b16():
 
 
 def test_decode_ring_wraps():
-    # 1024 (batch, head) units: every CTA walks about seven units through its ring of stages,
-    # so each stage is refilled at least once; R = 3 runs the rank-4 kernel with a short rank
-    shape = dict(b=64, L=3, H=16, P=16, N=16, R=3, G=4)
+    # 4096 (batch, head) units: each of a CTA's four teams walks about seven units through its
+    # six stages, so every stage is refilled; R = 3 runs the rank-4 kernel with a short rank
+    shape = dict(b=256, L=3, H=16, P=16, N=16, R=3, G=4)
     inp = make_inputs(dtype="bf16", seed=120, extras=True, **shape)
-    st = make_state(64, 16, 16, 16, 3, seed=121)
+    st = make_state(256, 16, 16, 16, 3, seed=121)
     check_decode(inp, 3, st)
 
 
 def test_decode_large_state_row_blocks():
-    # a 128 KiB state tile is taken in row blocks (four per unit at two CTAs per SM): the
+    # a 128 KiB state tile is taken in row blocks (four per unit, two teams per CTA): the
     # readout sums over the blocks and the carry is rewritten after the unit's last block
     shape = dict(b=2, L=3, H=3, P=256, N=128, R=2, G=1)
     inp = make_inputs(dtype="bf16", seed=122, extras=True, **shape)
     st = make_state(2, 3, 256, 128, 2, seed=123)
+    check_decode(inp, 3, st)
+
+
+def test_decode_ring_teams_row_blocks_f32():
+    # fp32 operands at d_state = headdim = 128 take the ring form: four teams per CTA, the 64 KiB
+    # state tile in four row blocks; 320 units leave most CTAs two or three teams at work
+    shape = dict(b=40, L=3, H=8, P=128, N=128, R=2, G=2)
+    inp = make_inputs(dtype="f32", seed=124, extras=True, **shape)
+    st = make_state(40, 8, 128, 128, 2, seed=125)
     check_decode(inp, 3, st)
 
 
