@@ -30,12 +30,15 @@ __device__ __forceinline__ uint64_t globaltimer() {
 // Persistent form: each CTA takes a contiguous range of (batch, head) units, ordered head-major
 // so that the per-head weights change at most a few times per CTA.  The CTA's threads form
 // `teams` independent teams (named barriers, no CTA-wide synchronisation after set-up); team t
-// walks units t, t + teams, ... of the range, so that while one team waits on a barrier or on
-// its copies the others update theirs.  A unit's state tile is taken in `split` blocks of
-// N / split rows (the readouts are summed over the blocks in shared memory), and each team
-// keeps `stages` blocks in flight: while it updates one, the TMA engine brings the next blocks
-// (state rows and raw token operands) into the team's ring of shared-memory stages.  The
-// updated state goes straight from registers to HBM, so the copy engine only ever reads.
+// walks units t, t + teams, ... of the range, so that while one team waits on a barrier the
+// others update their units.  A unit's state tile is taken in `split` blocks of N / split rows,
+// and each team keeps `stages` blocks in flight: while it updates one, the TMA engine brings the
+// next blocks (state rows, the same rows of B, C and carry_B, and the token's x) into the team's
+// ring of shared-memory stages.  One named barrier per block: the operands a block derives
+// (biased B and C, rotation table, coefficients) alternate between two buffers, each thread
+// sums its readout partial over the unit's blocks in registers, and the unit's output sum is
+// written by half of the team during the next block's update.  The updated state goes straight
+// from registers to HBM, so the copy engine only ever reads.
 
 constexpr int kMaxStages = 6;
 constexpr int kRingThreads = 512;
@@ -44,14 +47,17 @@ constexpr int kMaxTeams = 4;
 struct RingPlan {
   int stages, split, teams, team_threads;
   uint32_t stage_bytes, team_bytes;
-  // byte offsets inside a stage: state rows of the block, raw B_t, raw C_t, carry_B, raw x_t,
-  // carry_x, theta_t, and the three per-unit scalars dt, A, lam
+  // byte offsets inside a stage: state rows of the block and the same rows of raw B_t, raw C_t,
+  // carry_B (R x NB each) and theta_t, raw x_t, carry_x, and the three per-unit scalars dt, A, lam
   uint32_t o_st, o_b, o_c, o_cb, o_x, o_cx, o_th, o_sc;
-  // byte offsets (inside a team's region, after its stages) of the single-buffered arrays: the
-  // block's biased B, C and the MIMO branches, the rotation table and coefficients, the weights
-  // of the current head (bias_B, bias_C, W_x, W_o) and the per-pair-group partial readouts of
-  // every block of the unit
-  uint32_t o_bbc, o_bbp, o_cbb, o_xc, o_xp, o_xr, o_cs, o_coef, o_wb, o_wc, o_wx, o_wo, o_red, o_bar;
+  // a block buffer (two per team, blocks alternate): the block's biased B_t, B_{t-1} and C_t,
+  // the rotation table and the step's coefficients
+  uint32_t blk_bytes, o_bbc, o_bbp, o_cbb, o_cs, o_coef;
+  // a unit buffer (two per team, units alternate): the per-pair-group partial outputs of the unit
+  uint32_t unit_bytes, o_red;
+  // byte offsets inside a team's region, after its stages: the block and unit buffers, the
+  // weights of the current head (bias_B, bias_C, W_x, W_o) and the stage barriers
+  uint32_t o_blk, o_unit, o_wb, o_wc, o_wx, o_wo, o_bar;
   uint32_t total;
 };
 
@@ -74,37 +80,39 @@ inline RingPlan ring_plan(int P, int N, int R, bool bf16, int split, int teams, 
   rp.team_threads = kRingThreads / teams;
   uint32_t o = 0;
   rp.o_st = o; o += pad16((uint32_t)NB * P * 4);
-  rp.o_b = o;  o += pad16((uint32_t)R * N * esz);
-  rp.o_c = o;  o += pad16((uint32_t)R * N * esz);
-  rp.o_cb = o; o += pad16((uint32_t)R * N * 4);
+  rp.o_b = o;  o += pad16((uint32_t)R * NB * esz);
+  rp.o_c = o;  o += pad16((uint32_t)R * NB * esz);
+  rp.o_cb = o; o += pad16((uint32_t)R * NB * 4);
   rp.o_x = o;  o += pad16((uint32_t)P * esz);
   rp.o_cx = o; o += pad16((uint32_t)P * 4);
-  rp.o_th = o; o += pad16((uint32_t)N / 2 * 4);
+  rp.o_th = o; o += pad16((uint32_t)NB / 2 * 4);
   rp.o_sc = o; o += 16;
   rp.stage_bytes = (o + 127u) & ~127u;
+  o = 0;
+  rp.o_bbc = o; o += pad16((uint32_t)R * NB * 4);
+  rp.o_bbp = o; o += pad16((uint32_t)R * NB * 4);
+  rp.o_cbb = o; o += pad16((uint32_t)R * NB * 4);
+  rp.o_cs = o;  o += pad16((uint32_t)NB / 2 * 8);
+  rp.o_coef = o; o += 16;
+  rp.blk_bytes = o;
+  o = 0;
+  rp.o_red = o; o += pad16((uint32_t)ring_kg(P, NB, rp.team_threads) * P * 4);
+  rp.unit_bytes = o;
   uint32_t f = 0;
-  rp.o_bbc = f; f += pad16((uint32_t)R * NB * 4);
-  rp.o_bbp = f; f += pad16((uint32_t)R * NB * 4);
-  rp.o_cbb = f; f += pad16((uint32_t)R * NB * 4);
-  rp.o_xc = f;  f += pad16((uint32_t)R * P * 4);
-  rp.o_xp = f;  f += pad16((uint32_t)R * P * 4);
-  rp.o_xr = f;  f += pad16((uint32_t)P * 4);
-  rp.o_cs = f;  f += pad16((uint32_t)NB / 2 * 8);
-  rp.o_coef = f; f += 16;
+  rp.o_blk = f;  f += 2 * rp.blk_bytes;
+  rp.o_unit = f; f += 2 * rp.unit_bytes;
   rp.o_wb = f; f += pad16((uint32_t)R * N * 4);
   rp.o_wc = f; f += pad16((uint32_t)R * N * 4);
   rp.o_wx = f; f += pad16((uint32_t)R * P * 4);
   rp.o_wo = f; f += pad16((uint32_t)R * P * 4);
-  rp.o_red = f; f += pad16((uint32_t)split * ring_kg(P, NB, rp.team_threads) * P * 4);
   rp.o_bar = f; f += 8 * kMaxStages;
   f = (f + 127u) & ~127u;
   const int room = max_bytes / teams - (int)f;
   int st = room > 0 ? room / (int)rp.stage_bytes : 0;
   rp.stages = st < kMaxStages ? st : kMaxStages;
   const uint32_t ring = (uint32_t)rp.stages * rp.stage_bytes;
-  rp.o_bbc += ring; rp.o_bbp += ring; rp.o_cbb += ring; rp.o_xc += ring; rp.o_xp += ring;
-  rp.o_xr += ring; rp.o_cs += ring; rp.o_coef += ring; rp.o_wb += ring; rp.o_wc += ring;
-  rp.o_wx += ring; rp.o_wo += ring; rp.o_red += ring; rp.o_bar += ring;
+  rp.o_blk += ring; rp.o_unit += ring; rp.o_bar += ring;
+  rp.o_wb += ring; rp.o_wc += ring; rp.o_wx += ring; rp.o_wo += ring;
   rp.team_bytes = ring + f;
   rp.total = rp.team_bytes * (uint32_t)teams;
   return rp;
@@ -176,19 +184,6 @@ __global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, 
   const int S = rp.stages;
   constexpr uint32_t esz = BF16 ? 2u : 4u;
   const uint32_t sbase = smem_u32(smem);
-  float* bbc = reinterpret_cast<float*>(smem + rp.o_bbc);
-  float* bbp = reinterpret_cast<float*>(smem + rp.o_bbp);
-  float* cbb = reinterpret_cast<float*>(smem + rp.o_cbb);
-  float* xc = reinterpret_cast<float*>(smem + rp.o_xc);
-  float* xp = reinterpret_cast<float*>(smem + rp.o_xp);
-  float* xr = reinterpret_cast<float*>(smem + rp.o_xr);
-  float2* cs = reinterpret_cast<float2*>(smem + rp.o_cs);
-  float* coef = reinterpret_cast<float*>(smem + rp.o_coef);
-  float* wb = reinterpret_cast<float*>(smem + rp.o_wb);
-  float* wc = reinterpret_cast<float*>(smem + rp.o_wc);
-  float* wx = reinterpret_cast<float*>(smem + rp.o_wx);
-  float* wo = reinterpret_cast<float*>(smem + rp.o_wo);
-  float* red = reinterpret_cast<float*>(smem + rp.o_red);
   const uint32_t bar0 = sbase + rp.o_bar;
   RingCursor first{0, 0, 0};
   if (nv > 0) {
@@ -201,19 +196,22 @@ __global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, 
     const int64_t bh = c.bi * H + c.hi;
     const uint32_t st = sbase + (uint32_t)s * rp.stage_bytes;
     const uint32_t bar = bar0 + 8u * s;
-    const uint32_t n_st = (uint32_t)NB * P * 4, n_b = (uint32_t)R * N * esz, n_cb = (uint32_t)R * N * 4;
-    const uint32_t n_x = (uint32_t)P * esz, n_cx = (uint32_t)P * 4, n_th = (uint32_t)N / 2 * 4;
+    const uint32_t n_st = (uint32_t)NB * P * 4, n_b = (uint32_t)NB * esz, n_cb = (uint32_t)NB * 4;
+    const uint32_t n_x = (uint32_t)P * esz, n_cx = (uint32_t)P * 4, n_th = (uint32_t)NB / 2 * 4;
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
-                 "r"(n_st + 2 * n_b + n_cb + n_x + n_cx + n_th)
+                 "r"(n_st + (uint32_t)R * (2 * n_b + n_cb) + n_x + n_cx + n_th)
                  : "memory");
-    const int64_t bc = ((c.bi * G + g) * R) * (int64_t)N;
-    bulk_g2s(st + rp.o_st, p.h + (bh * N + (int64_t)c.blk * NB) * P, n_st, bar);
-    bulk_g2s(st + rp.o_b, static_cast<const unsigned char*>(p.B) + bc * esz, n_b, bar);
-    bulk_g2s(st + rp.o_c, static_cast<const unsigned char*>(p.C) + bc * esz, n_b, bar);
-    bulk_g2s(st + rp.o_cb, p.carry_B + bh * R * N, n_cb, bar);
+    const int n0 = c.blk * NB;
+    const int64_t bc = ((c.bi * G + g) * R) * (int64_t)N + n0;  // row n0 of branch 0
+    bulk_g2s(st + rp.o_st, p.h + (bh * N + n0) * P, n_st, bar);
+    for (int r = 0; r < R; ++r) {
+      bulk_g2s(st + rp.o_b + r * n_b, static_cast<const unsigned char*>(p.B) + (bc + (int64_t)r * N) * esz, n_b, bar);
+      bulk_g2s(st + rp.o_c + r * n_b, static_cast<const unsigned char*>(p.C) + (bc + (int64_t)r * N) * esz, n_b, bar);
+      bulk_g2s(st + rp.o_cb + r * n_cb, p.carry_B + (bh * R + r) * N + n0, n_cb, bar);
+    }
     bulk_g2s(st + rp.o_x, static_cast<const unsigned char*>(p.x) + bh * P * esz, n_x, bar);
     bulk_g2s(st + rp.o_cx, p.carry_x + bh * P, n_cx, bar);
-    bulk_g2s(st + rp.o_th, p.theta + (c.bi * G + g) * (N / 2), n_th, bar);
+    bulk_g2s(st + rp.o_th, p.theta + (c.bi * G + g) * (N / 2) + n0 / 2, n_th, bar);
     // the three scalars: 4-byte asynchronous copies whose completion is the barrier's second arrival
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(st + rp.o_sc), "l"(p.dt + bh) : "memory");
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(st + rp.o_sc + 4), "l"(p.A + bh) : "memory");
@@ -254,13 +252,39 @@ __global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, 
   const int KG = ring_kg(P, NB, TT);
   const int pq = tid % PQ;
   const int kg = tid / PQ;
-  constexpr int CQ = 1;  // 4-column quads per thread (the compute below takes any count)
+  // y = sum_r W_o[r] * readout_r + D x of a finished unit: the partials of its pair groups
+  // (D x rides in group 0's) summed, by the upper half of the team while the lower half starts
+  // the next block's update
+  auto finish_unit = [&](const unsigned char* ubuf, int64_t ybh, int lane0, int nlanes) {
+    const float* red = reinterpret_cast<const float*>(ubuf + rp.o_red);
+    const int nq = KG;
+    for (int pp = tid - lane0; pp < P; pp += nlanes) {
+      float acc0 = 0.0f, acc1 = 0.0f;
+      int q = 0;
+      for (; q + 1 < nq; q += 2) {
+        acc0 += red[q * P + pp];
+        acc1 += red[(q + 1) * P + pp];
+      }
+      if (q < nq) acc0 += red[q * P + pp];
+      store_out<BF16>(p.y, ybh * P + pp, acc0 + acc1);
+    }
+  };
+  float* wb = reinterpret_cast<float*>(smem + rp.o_wb);
+  float* wc = reinterpret_cast<float*>(smem + rp.o_wc);
+  float* wx = reinterpret_cast<float*>(smem + rp.o_wx);
+  float* wo = reinterpret_cast<float*>(smem + rp.o_wo);
   int cur_h = -1;
   float Dh = 0.0f;
   uint32_t phases = 0;  // bit s: parity of the next completion of stage s
   int s = 0;
   bool ok = true;
   RingCursor cur = first;
+  int ub = 0;            // unit buffer of the unit being updated
+  bool pending = false;  // a finished unit whose y is still to be written
+  int64_t pend_bh = 0;
+  float oacc[4] = {0.f, 0.f, 0.f, 0.f};  // the thread's readout partial, summed over the unit's blocks
+  const int half = TT / 2;
+  const int pc = 4 * pq;  // the thread's first column
   int64_t j = 0;
   for (; j < nv; ++j) {
     const uint32_t par = (phases >> s) & 1u;
@@ -270,9 +294,17 @@ __global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, 
     const int hi = cur.hi;
     const int64_t bh = cur.bi * H + hi;
     const unsigned char* stg = smem + (size_t)s * rp.stage_bytes;
+    unsigned char* bbuf = smem + rp.o_blk + (size_t)(j & 1) * rp.blk_bytes;
+    unsigned char* ubuf = smem + rp.o_unit + (size_t)ub * rp.unit_bytes;
+    float* bbc = reinterpret_cast<float*>(bbuf + rp.o_bbc);
+    float* bbp = reinterpret_cast<float*>(bbuf + rp.o_bbp);
+    float* cbb = reinterpret_cast<float*>(bbuf + rp.o_cbb);
+    float2* cs = reinterpret_cast<float2*>(bbuf + rp.o_cs);
+    float* coef = reinterpret_cast<float*>(bbuf + rp.o_coef);
+    float* red = reinterpret_cast<float*>(ubuf + rp.o_red);
     if (hi != cur_h) {  // weights of a new head (uniform: the whole team sees the same unit)
       cur_h = hi;
-      team_sync(bar_id, TT);  // the previous block's update has read W_o
+      team_sync(bar_id, TT);  // every thread has finished the previous block's update (W_x, W_o)
       const float* biasB = p.bias_B ? p.bias_B + (int64_t)hi * R * N : nullptr;
       const float* biasC = p.bias_C ? p.bias_C + (int64_t)hi * R * N : nullptr;
       const float* Wx = p.W_x ? p.W_x + (int64_t)hi * R * P : nullptr;
@@ -290,47 +322,43 @@ __global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, 
     }
     ok = wait(s, par);
     if (ok) {
-      // ---- operands of this block
+      // ---- operands of this block (into the block buffer the previous block does not use)
       const float* sc = reinterpret_cast<const float*>(stg + rp.o_sc);
       const float* cBs = reinterpret_cast<const float*>(stg + rp.o_cb);
-      const float* cxs = reinterpret_cast<const float*>(stg + rp.o_cx);
       const float* ths = reinterpret_cast<const float*>(stg + rp.o_th);
       const int n0 = blk * NB;
+      // the block's rows of the new carry (this token's raw B): this block's copy of the old
+      // rows has landed, and no other block reads them
+      float* cBg = p.carry_B + bh * R * N + n0;
       for (int i = tid; i < R * NB; i += TT) {
-        const int r = i / NB, n = n0 + i % NB;
-        const float bb = wb[r * N + n];
-        bbc[i] = stage_in<BF16>(stg + rp.o_b, r * N + n) + bb;
-        bbp[i] = cBs[r * N + n] + bb;
-        cbb[i] = stage_in<BF16>(stg + rp.o_c, r * N + n) + wc[r * N + n];
-      }
-      for (int i = tid; i < R * P; i += TT) {
-        const float w = wx[i];
-        xc[i] = stage_in<BF16>(stg + rp.o_x, i % P) * w;
-        xp[i] = cxs[i % P] * w;
+        const int r = i / NB;
+        const int rn = r * N + n0 + (i - r * NB);
+        const float braw = stage_in<BF16>(stg + rp.o_b, i);
+        const float bb = wb[rn];
+        bbc[i] = braw + bb;
+        bbp[i] = cBs[i] + bb;
+        cbb[i] = stage_in<BF16>(stg + rp.o_c, i) + wc[rn];
+        cBg[rn - n0] = braw;
       }
       const float delta = sc[0];
-      for (int k = tid; k < NB / 2; k += TT) {
+      // the rotation table from the team's last threads, the coefficients from its middle one,
+      // so that the first warp (which issues the copies) carries no extra work
+      for (int k = TT - 1 - tid; k < NB / 2; k += TT) {
         float sn, cn;
-        sincosf(p.angle_direct ? ths[n0 / 2 + k] : delta * ths[n0 / 2 + k], &sn, &cn);
+        sincosf(p.angle_direct ? ths[k] : delta * ths[k], &sn, &cn);
         cs[k] = make_float2(cn, sn);
       }
-      if (tid == 0) {
+      if (tid == half) {
         const float lm = sc[2];
         coef[0] = expf(delta * sc[1]);
         coef[1] = (1.0f - lm) * delta;
         coef[2] = lm * delta;
       }
       if (last_blk) {
-        // the unit's last block: every block's copy of the old carry has landed, so the new
-        // carry (this token's raw B and x) may overwrite it
-        float* cBg = p.carry_B + bh * R * N;
+        // the unit's last block: every block's copy of the old carry_x has landed, so the new
+        // one (this token's raw x) may overwrite it
         float* cxg = p.carry_x + bh * P;
-        for (int i = tid; i < R * N; i += TT) cBg[i] = stage_in<BF16>(stg + rp.o_b, i);
-        for (int pp = tid; pp < P; pp += TT) {
-          const float xv = stage_in<BF16>(stg + rp.o_x, pp);
-          xr[pp] = xv;
-          cxg[pp] = xv;
-        }
+        for (int pp = tid; pp < P; pp += TT) cxg[pp] = stage_in<BF16>(stg + rp.o_x, pp);
       }
     }
     if (team_sync_or(bar_id, TT, !ok)) {
@@ -338,133 +366,125 @@ __global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, 
       phases ^= 1u << s;  // block j's copies count as outstanding again
       break;
     }
+    // every thread is past the previous block's update: its stage may be refilled
+    if (tid == 0 && j >= 1 && j - 1 + S < nv) {
+      issue(ahead, s == 0 ? S - 1 : s - 1);
+      ahead.next(SPL, T, nb);
+    }
+    if (pending) {
+      if (tid >= half)
+        finish_unit(smem + rp.o_unit + (size_t)(ub ^ 1) * rp.unit_bytes, pend_bh, half, TT - half);
+      pending = false;
+    }
     // ---- state update of the thread's 4 columns over its rotation pairs of the block
     if (kg < KG) {
       const float alpha = coef[0], bp = coef[1], gm = coef[2];
       const float* stt = reinterpret_cast<const float*>(stg + rp.o_st);
       float* hg = p.h + (bh * N + (int64_t)blk * NB) * P;
-      int pc[CQ];
+      // the MIMO branches of this column quad: X_r = W_x[r] x_t, X'_r = W_x[r] x_{t-1}
+      float xq[4];
+      if constexpr (BF16) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(stg + rp.o_x + 2 * pc);
+        const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+        const float2 hi2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+        xq[0] = lo.x; xq[1] = lo.y; xq[2] = hi2.x; xq[3] = hi2.y;
+      } else {
+        const float4 v = *reinterpret_cast<const float4*>(stg + rp.o_x + 4 * pc);
+        xq[0] = v.x; xq[1] = v.y; xq[2] = v.z; xq[3] = v.w;
+      }
+      const float4 cx4 = *reinterpret_cast<const float4*>(stg + rp.o_cx + 4 * pc);
+      const float cq[4] = {cx4.x, cx4.y, cx4.z, cx4.w};
+      float Xc[RT][4], Xp[RT][4], Y[RT][4];
 #pragma unroll
-      for (int c = 0; c < CQ; ++c) pc[c] = 4 * pq + c * (P / CQ);
-      float4 Xc[RT][CQ], Xp[RT][CQ];
-      float Y[RT][CQ][4];
+      for (int r = 0; r < RT; ++r) {
+        const float4 w4 = r < R ? *reinterpret_cast<const float4*>(wx + r * P + pc) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float wq[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-      for (int r = 0; r < RT; ++r)
-#pragma unroll
-        for (int c = 0; c < CQ; ++c) {
-          Y[r][c][0] = Y[r][c][1] = Y[r][c][2] = Y[r][c][3] = 0.0f;
-          if (r < R) {
-            Xc[r][c] = *reinterpret_cast<const float4*>(xc + r * P + pc[c]);
-            Xp[r][c] = *reinterpret_cast<const float4*>(xp + r * P + pc[c]);
-          } else {
-            Xc[r][c] = Xp[r][c] = make_float4(0.f, 0.f, 0.f, 0.f);
-          }
+        for (int e = 0; e < 4; ++e) {
+          Y[r][e] = 0.0f;
+          Xc[r][e] = r < R ? xq[e] * wq[e] : 0.0f;
+          Xp[r][e] = r < R ? cq[e] * wq[e] : 0.0f;
         }
+      }
 #pragma unroll 2
       for (int k = kg; k < NB / 2; k += KG) {
-        float4 s0[CQ], s1[CQ];
-#pragma unroll
-        for (int c = 0; c < CQ; ++c) {
-          s0[c] = *reinterpret_cast<const float4*>(stt + (2 * k) * P + pc[c]);
-          s1[c] = *reinterpret_cast<const float4*>(stt + (2 * k + 1) * P + pc[c]);
-        }
-        float u0v[CQ][4] = {}, u1v[CQ][4] = {}, q0[CQ][4] = {}, q1[CQ][4] = {};
+        const float4 s0 = *reinterpret_cast<const float4*>(stt + (2 * k) * P + pc);
+        const float4 s1 = *reinterpret_cast<const float4*>(stt + (2 * k + 1) * P + pc);
+        float u0v[4] = {}, u1v[4] = {}, q0[4] = {}, q1[4] = {};
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
           if (r < R) {
             const float2 bcv = *reinterpret_cast<const float2*>(bbc + r * NB + 2 * k);
             const float2 bqv = *reinterpret_cast<const float2*>(bbp + r * NB + 2 * k);
 #pragma unroll
-            for (int c = 0; c < CQ; ++c) {
-              const float xc4[4] = {Xc[r][c].x, Xc[r][c].y, Xc[r][c].z, Xc[r][c].w};
-              const float xp4[4] = {Xp[r][c].x, Xp[r][c].y, Xp[r][c].z, Xp[r][c].w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                u0v[c][e] = fmaf(bcv.x, xc4[e], u0v[c][e]);
-                u1v[c][e] = fmaf(bcv.y, xc4[e], u1v[c][e]);
-                q0[c][e] = fmaf(bqv.x, xp4[e], q0[c][e]);
-                q1[c][e] = fmaf(bqv.y, xp4[e], q1[c][e]);
-              }
+            for (int e = 0; e < 4; ++e) {
+              u0v[e] = fmaf(bcv.x, Xc[r][e], u0v[e]);
+              u1v[e] = fmaf(bcv.y, Xc[r][e], u1v[e]);
+              q0[e] = fmaf(bqv.x, Xp[r][e], q0[e]);
+              q1[e] = fmaf(bqv.y, Xp[r][e], q1[e]);
             }
           }
         }
         const float2 rc = cs[k];
         const float ac = alpha * rc.x, as = alpha * rc.y;
-        float n0[CQ][4], n1[CQ][4];
+        const float a0[4] = {s0.x, s0.y, s0.z, s0.w};
+        const float a1[4] = {s1.x, s1.y, s1.z, s1.w};
+        float n0[4], n1[4];
 #pragma unroll
-        for (int c = 0; c < CQ; ++c) {
-          const float a0[4] = {s0[c].x, s0[c].y, s0[c].z, s0[c].w};
-          const float a1[4] = {s1[c].x, s1[c].y, s1[c].z, s1[c].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float v0 = fmaf(bp, q0[c][e], a0[e]);
-            const float v1 = fmaf(bp, q1[c][e], a1[e]);
-            n0[c][e] = fmaf(ac, v0, fmaf(-as, v1, gm * u0v[c][e]));
-            n1[c][e] = fmaf(as, v0, fmaf(ac, v1, gm * u1v[c][e]));
-          }
-          *reinterpret_cast<float4*>(hg + (int64_t)(2 * k) * P + pc[c]) =
-              make_float4(n0[c][0], n0[c][1], n0[c][2], n0[c][3]);
-          *reinterpret_cast<float4*>(hg + (int64_t)(2 * k + 1) * P + pc[c]) =
-              make_float4(n1[c][0], n1[c][1], n1[c][2], n1[c][3]);
+        for (int e = 0; e < 4; ++e) {
+          const float v0 = fmaf(bp, q0[e], a0[e]);
+          const float v1 = fmaf(bp, q1[e], a1[e]);
+          n0[e] = fmaf(ac, v0, fmaf(-as, v1, gm * u0v[e]));
+          n1[e] = fmaf(as, v0, fmaf(ac, v1, gm * u1v[e]));
         }
+        *reinterpret_cast<float4*>(hg + (int64_t)(2 * k) * P + pc) = make_float4(n0[0], n0[1], n0[2], n0[3]);
+        *reinterpret_cast<float4*>(hg + (int64_t)(2 * k + 1) * P + pc) = make_float4(n1[0], n1[1], n1[2], n1[3]);
 #pragma unroll
         for (int r = 0; r < RT; ++r) {
           if (r < R) {
             const float2 cc = *reinterpret_cast<const float2*>(cbb + r * NB + 2 * k);
 #pragma unroll
-            for (int c = 0; c < CQ; ++c)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) Y[r][c][e] = fmaf(cc.x, n0[c][e], fmaf(cc.y, n1[c][e], Y[r][c][e]));
+            for (int e = 0; e < 4; ++e) Y[r][e] = fmaf(cc.x, n0[e], fmaf(cc.y, n1[e], Y[r][e]));
           }
         }
       }
-      // this pair group's part of sum_r W_o[r] * readout_r; summed over groups and blocks later
+      // this pair group's part of sum_r W_o[r] * readout_r (+ D x in group 0), summed over the
+      // unit's blocks in registers and over the pair groups when the unit's y is written
+      if (blk == 0) {
 #pragma unroll
-      for (int c = 0; c < CQ; ++c) {
-        float o[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int r = 0; r < RT; ++r)
-          if (r < R) {
-            const float4 w4 = *reinterpret_cast<const float4*>(wo + r * P + pc[c]);
-            o[0] = fmaf(w4.x, Y[r][c][0], o[0]);
-            o[1] = fmaf(w4.y, Y[r][c][1], o[1]);
-            o[2] = fmaf(w4.z, Y[r][c][2], o[2]);
-            o[3] = fmaf(w4.w, Y[r][c][3], o[3]);
-          }
-        *reinterpret_cast<float4*>(red + (blk * KG + kg) * P + pc[c]) = make_float4(o[0], o[1], o[2], o[3]);
+        for (int e = 0; e < 4; ++e) oacc[e] = kg == 0 ? Dh * xq[e] : 0.0f;
       }
-    }
-    team_sync(bar_id, TT);  // stage s is read; the block's readouts are in place
-    if (tid == 0 && j + S < nv) {
-      issue(ahead, s);
-      ahead.next(SPL, T, nb);
-    }
-    if (last_blk) {
-      // ---- y = sum_r W_o[r] * readout_r + D x, the readouts summed over groups and blocks
-      const int nq = SPL * KG;
-      for (int pp = tid; pp < P; pp += TT) {
-        float acc0 = 0.0f, acc1 = 0.0f;
-        int q = 0;
-        for (; q + 1 < nq; q += 2) {
-          acc0 += red[q * P + pp];
-          acc1 += red[(q + 1) * P + pp];
+#pragma unroll
+      for (int r = 0; r < RT; ++r)
+        if (r < R) {
+          const float4 w4 = *reinterpret_cast<const float4*>(wo + r * P + pc);
+          oacc[0] = fmaf(w4.x, Y[r][0], oacc[0]);
+          oacc[1] = fmaf(w4.y, Y[r][1], oacc[1]);
+          oacc[2] = fmaf(w4.z, Y[r][2], oacc[2]);
+          oacc[3] = fmaf(w4.w, Y[r][3], oacc[3]);
         }
-        if (q < nq) acc0 += red[q * P + pp];
-        store_out<BF16>(p.y, bh * P + pp, fmaf(Dh, xr[pp], acc0 + acc1));
-      }
+      if (last_blk) *reinterpret_cast<float4*>(red + kg * P + pc) = make_float4(oacc[0], oacc[1], oacc[2], oacc[3]);
+    }
+    if (last_blk) {  // the unit's y is written during the next block's update
+      pending = true;
+      pend_bh = bh;
+      ub ^= 1;
     }
     s = (s + 1 == S) ? 0 : s + 1;
     cur.next(SPL, T, nb);
   }
-  if (!ok) {
-    // give up: wait (bounded) for the team's copies still in flight, then report
-    if (tid == 0) {
-      for (int64_t w = j; w < nv && w < j + S; ++w) {
-        const int sw = (int)(w % S);
-        wait(sw, (phases >> sw) & 1u);
-      }
-      set_status(p.status, M3_ERR_TIMEOUT);
+  if (ok) {
+    team_sync(bar_id, TT);  // the last unit's readouts are in place
+    if (pending) finish_unit(smem + rp.o_unit + (size_t)(ub ^ 1) * rp.unit_bytes, pend_bh, 0, TT);
+  } else if (tid == 0) {
+    // give up: wait (bounded) for the team's copies still in flight (blocks j .. j + S - 2, or
+    // the first S when the first wait failed), then report
+    const int64_t last = j == 0 ? S - 1 : j + S - 2;
+    for (int64_t w = j; w <= last && w < nv; ++w) {
+      const int sw = (int)(w % S);
+      wait(sw, (phases >> sw) & 1u);
     }
+    set_status(p.status, M3_ERR_TIMEOUT);
   }
 }
 
