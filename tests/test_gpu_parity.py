@@ -246,10 +246,10 @@ def test_decode_tc_long_run():
 # decode as the decode workloads state it: 1024 one-token steps from a state that m3_scan_fwd
 # produced on a prefix, on the 1.5B-scale layer (32 heads x 128, d_state 128, rank 4)
 
-def _long_decode(b, prefix, steps, pairs, seed):
+def _long_decode(b, prefix, steps, pairs, seed, workload="decode_b1"):
     """Prefill `prefix` tokens with m3_scan_fwd, then `steps` m3_decode_step calls; compare y of
     every step and the final state with the oracle run over prefix + steps tokens for `pairs`."""
-    cfg = dict(CONFIGS["decode_b1"], b=b, L=prefix)
+    cfg = dict(CONFIGS[workload], b=b, L=prefix)
     pre = make_inputs(seed=seed, **cfg)
     dims = m3.dims_of(pre)
     st, (th, tb, tx) = m3.state_tensors(dims)
@@ -302,6 +302,12 @@ def test_decode_b1_1024_steps_all_heads():
 def test_decode_b128_1024_steps_sampled():
     # batch 128: the persistent form; a 256-token prefix keeps the host draw small
     _long_decode(128, 256, 1024, [(0, 0), (17, 9), (64, 31), (127, 16)], seed=620)
+
+
+def test_decode_headdim64_b128_1024_steps_sampled():
+    # the headdim-64 layer (24 heads x 64, d_state 64, rank 2) at batch 128: the SIMT ring form,
+    # four teams per CTA, 1024 steps from a headdim-64 tensor-core prefill
+    _long_decode(128, 256, 1024, [(0, 0), (31, 7), (77, 23), (127, 12)], seed=630, workload="decode_p1_b128")
 
 
 # per-head B and C (G = H, the "per-head B/C" variant): each head reads its own B_t, C_t and theta_t
