@@ -101,12 +101,15 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Sums each of 16 values over the 32 lanes of a warp in 16 shuffles (a transposed butterfly:
-// every step keeps half of the values and adds the partner lane's copy of them, the last step
-// adds the neighbour's total).  Lane l returns the total of value l / 2.
-__device__ __forceinline__ float warp_sum16(float (&v)[16], int lane) {
+// Sums each of NV values (a power of two, 2..16) over the 32 lanes of a warp in a transposed
+// butterfly: log2 NV steps each keep half of the values and add the partner lane's copy of them
+// (offsets 16, 8, ...), then the lanes that hold the same value add theirs.  Lane l returns the
+// total of value l / (32 / NV).
+template <int NV>
+__device__ __forceinline__ float warp_sum_n(float (&v)[NV], int lane) {
+  int off = 16;
 #pragma unroll
-  for (int s = 8, off = 16; s >= 1; s >>= 1, off >>= 1) {
+  for (int s = NV / 2; s >= 1; s >>= 1, off >>= 1) {
     const bool up = (lane & off) != 0;
 #pragma unroll
     for (int i = 0; i < s; ++i) {
@@ -115,24 +118,30 @@ __device__ __forceinline__ float warp_sum16(float (&v)[16], int lane) {
       v[i] = keep + __shfl_xor_sync(0xffffffffu, give, off);
     }
   }
-  return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 1);
+  float t = v[0];
+#pragma unroll
+  for (; off >= 1; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+  return t;
 }
 
-// The terms of one rotation pair (2 values per branch r < R: rows n0, n1) summed over the
+// The terms of one rotation pair (2 values per branch r < R <= RT: rows n0, n1) summed over the
 // columns p into red[r N + n]: a warp butterfly when every lane of the warp holds this pair
 // (wide), element atomics otherwise.
-__device__ __forceinline__ void pair_reduce(float (&v)[16], bool wide, int lane, int R, int N, int n0, int n1,
+template <int RT>
+__device__ __forceinline__ void pair_reduce(float (&v)[2 * RT], bool wide, int lane, int R, int N, int n0, int n1,
                                             float* red) {
   if (wide) {
-    const float tot = warp_sum16(v, lane);
-    const int vi = lane >> 1, r = vi >> 1;
-    if ((lane & 1) == 0 && r < R) atomicAdd(&red[r * N + ((vi & 1) ? n1 : n0)], tot);
+    constexpr int span = 32 / (2 * RT);  // lanes that end with the same value
+    const float tot = warp_sum_n<2 * RT>(v, lane);
+    const int vi = lane / span, r = vi >> 1;
+    if (lane % span == 0 && r < R) atomicAdd(&red[r * N + ((vi & 1) ? n1 : n0)], tot);
   } else {
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      if (r >= R) break;
-      atomicAdd(&red[r * N + n0], v[2 * r]);
-      atomicAdd(&red[r * N + n1], v[2 * r + 1]);
+    for (int r = 0; r < RT; ++r) {
+      if (r < R) {
+        atomicAdd(&red[r * N + n0], v[2 * r]);
+        atomicAdd(&red[r * N + n1], v[2 * r + 1]);
+      }
     }
   }
 }
@@ -166,7 +175,7 @@ __global__ void bwd_store_kernel(const float* accB, const float* accC, void* dB,
   }
 }
 
-template <typename T, int NK>
+template <typename T, int NK, int RT>
 __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(const Params p, const BwdArgs q) {
   extern __shared__ __align__(16) float sm[];
   const int tid = threadIdx.x;
@@ -250,11 +259,17 @@ __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(const Params p, c
       const int k = grp + j * sh.KG;
       if (!active || k >= K2) continue;
       float u0 = 0.f, u1 = 0.f, q0 = 0.f, q1 = 0.f;
-      for (int r = 0; r < R; ++r) {
-        u0 = fmaf(Bb[r * N + 2 * k], X[r * P + pc], u0);
-        u1 = fmaf(Bb[r * N + 2 * k + 1], X[r * P + pc], u1);
-        q0 = fmaf(Bbp[r * N + 2 * k], Xp[r * P + pc], q0);
-        q1 = fmaf(Bbp[r * N + 2 * k + 1], Xp[r * P + pc], q1);
+#pragma unroll
+      for (int r = 0; r < RT; ++r) {
+        if (r < R) {
+          const float2 b2 = *reinterpret_cast<const float2*>(Bb + r * N + 2 * k);
+          const float2 bp2 = *reinterpret_cast<const float2*>(Bbp + r * N + 2 * k);
+          const float xr = X[r * P + pc], xpr = Xp[r * P + pc];
+          u0 = fmaf(b2.x, xr, u0);
+          u1 = fmaf(b2.y, xr, u1);
+          q0 = fmaf(bp2.x, xpr, q0);
+          q1 = fmaf(bp2.y, xpr, q1);
+        }
       }
       const float z0 = fmaf(co[1], q0, h0[j]), z1 = fmaf(co[1], q1, h1[j]);
       const float2 c = cs[k];
@@ -339,9 +354,9 @@ __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(const Params p, c
       const float* hp = t > t0 ? blk + (t - t0 - 1) * NP : ck + c * NP;
       const float alpha = co[0], bprime = co[1], gamma = co[2];
       float s_alpha = 0.f, s_gamma = 0.f, s_bp = 0.f;
-      float px[8], py[8];  // partial dX and Y of this thread's column, per branch (R <= 8)
+      float px[RT], py[RT];  // partial dX and Y of this thread's column, per branch (R <= RT)
 #pragma unroll
-      for (int r = 0; r < 8; ++r) px[r] = py[r] = 0.0f;
+      for (int r = 0; r < RT; ++r) px[r] = py[r] = 0.0f;
 #pragma unroll
       for (int j = 0; j < NK; ++j) {
         const int k = grp + j * sh.KG;
@@ -352,27 +367,36 @@ __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(const Params p, c
         // readout: g += sum_r Cb_r dY_r^T; dCb_r += h_t dY_r (summed over the warp's columns
         // below); Y_r partial.  sv holds the pair's column terms: dCb (r, n0), (r, n1), then dBb
         float g0 = gr0[j], g1 = gr1[j];
-        float sv[16];
+        float sv[2 * RT];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
+        for (int r = 0; r < RT; ++r) {
           sv[2 * r] = sv[2 * r + 1] = 0.0f;
           if (r < R) {
             const float dy_r = dYr[r * P + pc];
-            g0 = fmaf(Cb[r * N + n0], dy_r, g0);
-            g1 = fmaf(Cb[r * N + n1], dy_r, g1);
+            const float2 c2 = *reinterpret_cast<const float2*>(Cb + r * N + n0);
+            g0 = fmaf(c2.x, dy_r, g0);
+            g1 = fmaf(c2.y, dy_r, g1);
             sv[2 * r] = ht0 * dy_r;
             sv[2 * r + 1] = ht1 * dy_r;
-            py[r] = fmaf(Cb[r * N + n0], ht0, fmaf(Cb[r * N + n1], ht1, py[r]));
+            py[r] = fmaf(c2.x, ht0, fmaf(c2.y, ht1, py[r]));
           }
         }
-        pair_reduce(sv, wide, tid & 31, R, N, n0, n1, red_cb);
+        pair_reduce<RT>(sv, wide, tid & 31, R, N, n0, n1, red_cb);
         // step
         float u0 = 0.f, u1 = 0.f, q0 = 0.f, q1 = 0.f;
-        for (int r = 0; r < R; ++r) {
-          u0 = fmaf(Bb[r * N + n0], X[r * P + pc], u0);
-          u1 = fmaf(Bb[r * N + n1], X[r * P + pc], u1);
-          q0 = fmaf(Bbp[r * N + n0], Xp[r * P + pc], q0);
-          q1 = fmaf(Bbp[r * N + n1], Xp[r * P + pc], q1);
+        float2 bbr[RT];  // Bb rows n0, n1 of each branch (reused by u_t's gradient below)
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+          bbr[r] = make_float2(0.f, 0.f);
+          if (r < R) {
+            bbr[r] = *reinterpret_cast<const float2*>(Bb + r * N + n0);
+            const float2 bp2 = *reinterpret_cast<const float2*>(Bbp + r * N + n0);
+            const float xr = X[r * P + pc], xpr = Xp[r * P + pc];
+            u0 = fmaf(bbr[r].x, xr, u0);
+            u1 = fmaf(bbr[r].y, xr, u1);
+            q0 = fmaf(bp2.x, xpr, q0);
+            q1 = fmaf(bp2.y, xpr, q1);
+          }
         }
         const float z0 = fmaf(bprime, q0, hp0), z1 = fmaf(bprime, q1, hp1);
         const float2 cc = cs[k];
@@ -396,23 +420,24 @@ __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(const Params p, c
         gr1[j] = dz1;
         // u_t = sum_r Bb_r X_r^T
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
+        for (int r = 0; r < RT; ++r) {
           sv[2 * r] = sv[2 * r + 1] = 0.0f;
           if (r < R) {
             const float xr = X[r * P + pc];
             sv[2 * r] = du0 * xr;
             sv[2 * r + 1] = du1 * xr;
-            px[r] = fmaf(du0, Bb[r * N + n0], fmaf(du1, Bb[r * N + n1], px[r]));
+            px[r] = fmaf(du0, bbr[r].x, fmaf(du1, bbr[r].y, px[r]));
           }
         }
-        pair_reduce(sv, wide, tid & 31, R, N, n0, n1, red_bb);
+        pair_reduce<RT>(sv, wide, tid & 31, R, N, n0, n1, red_bb);
       }
       if (active) {
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          if (r >= R) break;
-          atomicAdd(&red_x[r * P + pc], px[r]);
-          atomicAdd(&red_y[r * P + pc], py[r]);
+        for (int r = 0; r < RT; ++r) {
+          if (r < R) {
+            atomicAdd(&red_x[r * P + pc], px[r]);
+            atomicAdd(&red_y[r * P + pc], py[r]);
+          }
         }
       }
       s_alpha = warp_sum(s_alpha);
@@ -473,15 +498,15 @@ __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(const Params p, c
   for (int i = tid; i < R * P; i += kBwdThreads) red_x[i] = 0.0f;
   __syncthreads();
   {
-    float px[8];
+    float px[RT];
 #pragma unroll
-    for (int r = 0; r < 8; ++r) px[r] = 0.0f;
+    for (int r = 0; r < RT; ++r) px[r] = 0.0f;
 #pragma unroll
     for (int j = 0; j < NK; ++j) {
       const int k = grp + j * sh.KG;
       if (!active || k >= K2) continue;
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
+      for (int r = 0; r < RT; ++r) {
         if (r >= R) break;
         const float xr = Xp[r * P + pc];
         atomicAdd(&red_bb[r * N + 2 * k], dn0[j] * xr);
@@ -491,7 +516,7 @@ __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(const Params p, c
     }
     if (active) {
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
+      for (int r = 0; r < RT; ++r) {
         if (r >= R) break;
         atomicAdd(&red_x[r * P + pc], px[r]);
       }
@@ -524,11 +549,11 @@ __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(const Params p, c
   }
 }
 
-template <typename T, int NK>
+template <typename T, int NK, int RT>
 cudaError_t launch_bwd_nk(const Params& p, const BwdArgs& q, cudaStream_t stream) {
   const BwdSmem ms = bwd_smem(p.P, p.N, p.R);
   const size_t smem = sizeof(float) * (size_t)ms.total;
-  auto k = scan_bwd_kernel<T, NK>;
+  auto k = scan_bwd_kernel<T, NK, RT>;
   if (smem > 48 * 1024) {
     static SmemAttr attr;
     cudaError_t e = attr.ensure(k, (int)smem);
@@ -538,14 +563,21 @@ cudaError_t launch_bwd_nk(const Params& p, const BwdArgs& q, cudaStream_t stream
   return cudaGetLastError();
 }
 
+template <typename T, int RT>
+cudaError_t launch_bwd_rt(const Params& p, const BwdArgs& q, cudaStream_t stream) {
+  const int nk = bwd_shape(p.P, p.N).NK;
+  if (nk <= 1) return launch_bwd_nk<T, 1, RT>(p, q, stream);
+  if (nk <= 2) return launch_bwd_nk<T, 2, RT>(p, q, stream);
+  if (nk <= 4) return launch_bwd_nk<T, 4, RT>(p, q, stream);
+  if (nk <= 8) return launch_bwd_nk<T, 8, RT>(p, q, stream);
+  return launch_bwd_nk<T, 16, RT>(p, q, stream);
+}
+
 template <typename T>
 cudaError_t launch_bwd_t(const Params& p, const BwdArgs& q, cudaStream_t stream) {
-  const int nk = bwd_shape(p.P, p.N).NK;
-  if (nk <= 1) return launch_bwd_nk<T, 1>(p, q, stream);
-  if (nk <= 2) return launch_bwd_nk<T, 2>(p, q, stream);
-  if (nk <= 4) return launch_bwd_nk<T, 4>(p, q, stream);
-  if (nk <= 8) return launch_bwd_nk<T, 8>(p, q, stream);
-  return launch_bwd_nk<T, 16>(p, q, stream);
+  if (p.R <= 2) return launch_bwd_rt<T, 2>(p, q, stream);
+  if (p.R <= 4) return launch_bwd_rt<T, 4>(p, q, stream);
+  return launch_bwd_rt<T, 8>(p, q, stream);
 }
 
 }  // namespace
