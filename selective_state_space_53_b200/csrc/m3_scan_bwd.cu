@@ -44,6 +44,7 @@ struct BwdArgs {
   float* ckpt;                     // (b*H, nck + K, N, P) workspace of forward states
   int K;                           // tokens per recomputed block
   int nck;                         // blocks = ceil(L / K)
+  int cs;                          // CTAs per (batch, head), each owning P / cs columns
 };
 
 struct BwdShape {
@@ -181,12 +182,16 @@ __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(const Params p, c
   const int tid = threadIdx.x;
   const int H = p.H, P = p.P, N = p.N, R = p.R, G = p.G, K2 = N / 2;
   const int64_t L = p.L;
-  const int bh = blockIdx.x, bi = bh / H, hi = bh % H, g = hi / (H / G);
-  const BwdShape sh = bwd_shape(P, N);
+  // the columns of a state evolve independently (the rotation mixes rows): cs CTAs share a
+  // (batch, head), CTA c owning columns c0 .. c0 + PL - 1; sums over columns are added up
+  // across them with the global atomics that already sum over heads or the batch
+  const int bh = blockIdx.x / q.cs, bi = bh / H, hi = bh % H, g = hi / (H / G);
+  const int PL = P / q.cs, c0 = (blockIdx.x % q.cs) * PL;
+  const BwdShape sh = bwd_shape(PL, N);
   const BwdSmem ms = bwd_smem(P, N, R);
-  const int pc = tid % P, grp = tid / P;
+  const int pc = c0 + tid % PL, grp = tid / PL;
   const bool active = grp < sh.KG;
-  const bool wide = P % 32 == 0;  // a warp's lanes are columns of one pair group
+  const bool wide = PL % 32 == 0;  // a warp's lanes are columns of one pair group
   float* const Bb = sm + ms.bb;
   float* const Bbp = sm + ms.bbp;
   float* const Cb = sm + ms.cb;
@@ -457,7 +462,7 @@ __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(const Params p, c
         acc_bC[i] += red_cb[i];
         acc_bB[i] += red_bb[i];
       }
-      for (int i = tid; i < P; i += kBwdThreads) {
+      for (int i = c0 + tid; i < c0 + PL; i += kBwdThreads) {
         float dxv = Dh * dyt[i];
         for (int r = 0; r < R; ++r) {
           dxv = fmaf(Wx ? Wx[r * P + i] : 1.0f, red_x[r * P + i], dxv);
@@ -480,13 +485,13 @@ __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(const Params p, c
         if ((tid & 31) == 0 && tid < K2) atomicAdd(&red_s[4], sdt);
       }
       __syncthreads();
-      if (tid == 0) {
+      if (tid == 0) {  // this CTA's columns' share (the scalars' gradients are linear in the sums)
         const float dth = K2 > 32 ? red_s[4] : sdt;
         const float da = red_s[0], dg = red_s[1], db = red_s[2];
         const float al = co[0];
-        q.ddt[tok * H + hi] = da * al * a + dg * lm + db * (1.0f - lm) + dth;
-        q.dA[tok * H + hi] = da * al * delta;
-        q.dlam[tok * H + hi] = (dg - db) * delta;
+        atomicAdd(&q.ddt[tok * H + hi], da * al * a + dg * lm + db * (1.0f - lm) + dth);
+        atomicAdd(&q.dA[tok * H + hi], da * al * delta);
+        atomicAdd(&q.dlam[tok * H + hi], (dg - db) * delta);
       }
     }
   }
@@ -524,10 +529,10 @@ __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(const Params p, c
   }
   __syncthreads();
   for (int i = tid; i < R * N; i += kBwdThreads) {
-    q.dcarry_B[(int64_t)bh * R * N + i] = red_bb[i];
+    atomicAdd(&q.dcarry_B[(int64_t)bh * R * N + i], red_bb[i]);
     acc_bB[i] += red_bb[i];
   }
-  for (int i = tid; i < P; i += kBwdThreads) {
+  for (int i = c0 + tid; i < c0 + PL; i += kBwdThreads) {
     float dcx = 0.0f;
     for (int r = 0; r < R; ++r) {
       dcx = fmaf(Wx ? Wx[r * P + i] : 1.0f, red_x[r * P + i], dcx);
@@ -537,7 +542,7 @@ __global__ void __launch_bounds__(kBwdThreads) scan_bwd_kernel(const Params p, c
   }
   // ---- per-head parameters, summed over the batch
   accD = warp_sum(accD);
-  if ((tid & 31) == 0 && q.dD && tid < P) atomicAdd(q.dD + hi, accD);
+  if ((tid & 31) == 0 && q.dD && tid < PL) atomicAdd(q.dD + hi, accD);
   __syncthreads();
   for (int i = tid; i < R * N; i += kBwdThreads) {
     if (q.dbias_B) atomicAdd(q.dbias_B + (int64_t)hi * R * N + i, acc_bB[i]);
@@ -559,13 +564,13 @@ cudaError_t launch_bwd_nk(const Params& p, const BwdArgs& q, cudaStream_t stream
     cudaError_t e = attr.ensure(k, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  k<<<(unsigned)(p.b * p.H), kBwdThreads, smem, stream>>>(p, q);
+  k<<<(unsigned)(p.b * p.H * q.cs), kBwdThreads, smem, stream>>>(p, q);
   return cudaGetLastError();
 }
 
 template <typename T, int RT>
 cudaError_t launch_bwd_rt(const Params& p, const BwdArgs& q, cudaStream_t stream) {
-  const int nk = bwd_shape(p.P, p.N).NK;
+  const int nk = bwd_shape(p.P / q.cs, p.N).NK;
   if (nk <= 1) return launch_bwd_nk<T, 1, RT>(p, q, stream);
   if (nk <= 2) return launch_bwd_nk<T, 2, RT>(p, q, stream);
   if (nk <= 4) return launch_bwd_nk<T, 4, RT>(p, q, stream);
@@ -581,6 +586,17 @@ cudaError_t launch_bwd_t(const Params& p, const BwdArgs& q, cudaStream_t stream)
 }
 
 }  // namespace
+
+// CTAs per (batch, head): split the columns in two or four while the grid still fits one wave
+// and every CTA keeps whole warps of columns
+int bwd_col_split(const Params& p) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 1;
+  for (int cs = 4; cs >= 2; cs /= 2)
+    if (p.P % (32 * cs) == 0 && p.b * p.H * cs <= sms) return cs;
+  return 1;
+}
 
 // tokens per recomputed block and the workspace the backward pass needs
 int bwd_block(int64_t L) {
@@ -615,6 +631,7 @@ cudaError_t launch_scan_bwd(const Params& p, const void* dy, const float* dh_fin
   q.dh0 = dh0; q.dcarry_B = dcarry_B; q.dcarry_x = dcarry_x;
   q.K = bwd_block(p.L);
   q.nck = (int)((p.L + q.K - 1) / q.K);
+  q.cs = bwd_col_split(p);
   const size_t nbh = (size_t)(p.b * p.H);
   const size_t states = nbh * (size_t)(q.nck + q.K) * p.N * p.P * 4;
   const int64_t nbc = p.b * p.L * p.G * p.R * p.N;
@@ -629,6 +646,9 @@ cudaError_t launch_scan_bwd(const Params& p, const void* dy, const float* dh_fin
   bwd_zero_kernel<<<64, 256, 0, stream>>>(dW_x, dW_x ? (int64_t)p.H * p.R * p.P : 0, dW_o,
                                           dW_o ? (int64_t)p.H * p.R * p.P : 0, dD, dD ? p.H : 0, nullptr, 0,
                                           nullptr, 0);
+  // the per-token scalars' gradients and dcarry_B are sums over columns, added by every CTA
+  bwd_zero_kernel<<<256, 256, 0, stream>>>(ddt, p.b * p.L * p.H, dA, p.b * p.L * p.H, dlam, p.b * p.L * p.H,
+                                           dcarry_B, p.b * p.H * p.R * p.N, nullptr, 0);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = p.dtype == M3_BF16 ? launch_bwd_t<__nv_bfloat16>(p, q, stream) : launch_bwd_t<float>(p, q, stream);
