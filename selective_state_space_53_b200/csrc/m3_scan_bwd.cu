@@ -13,15 +13,18 @@
 // followed by the readout's and u_t's chain rules and the scalar chains of alpha, beta',
 // gamma and phi through dt, A, lam and theta.
 //
-// One CTA per (batch, head) walks the tokens backwards.  The fp32 gradient g and u_t's share
-// from the next token live in registers (a thread owns one column p and the rotation pairs
-// k = grp, grp + KG, ...), the forward states come from a checkpointed recomputation: a first
+// One CTA per (batch, head) walks the tokens backwards (or 2 or 4 CTAs, each owning a slice of
+// the columns p, when that fills more SMs: the columns evolve independently).  The fp32
+// gradient g and u_t's share from the next token live in registers (a thread owns one column p
+// and the rotation pairs k = grp, grp + KG, ...), the forward states come from a checkpointed
+// recomputation: a first
 // sweep stores the state before every K-th token in the workspace, and each block of K tokens
 // is recomputed into the workspace before it is walked backwards (K about sqrt(L)).  Sums over
 // the columns or rows of a token (the readout's and u_t's gradients, the rotation angles' and
 // the scalars') are reduced with shared-memory atomics.  Gradients of operands shared by the
-// heads of a group (B, C, theta) or by the batch (biases, W_x, W_o, D) are added into global
-// memory with atomics, after a first kernel has zeroed them.
+// heads of a group (B, C, theta) or by the batch (biases, W_x, W_o, D), and the sums over
+// columns when several CTAs share a (batch, head), are added into global memory with atomics,
+// after a first kernel has zeroed them.
 #include "m3_common.cuh"
 
 namespace m3 {
