@@ -510,8 +510,9 @@ def run_backward(args, device, names=("p1_layer", "l15b_2k"), calls=2):
         out[name] = {"workload": "%s: m3_scan_bwd b%d L%d H%d P%d N%d R%d, every gradient" %
                                  (name, cfg["b"], cfg["L"], cfg["H"], cfg["P"], cfg["N"], cfg["R"]),
                      "ms_per_call": ms, "tokens_per_s": cfg["b"] * cfg["L"] / (ms * 1e-3),
-                     "note": "token-sequential SIMT kernel with checkpointed recomputation (one block per "
-                             "(batch, head)); includes allocation of the gradient buffers and workspace"}
+                     "note": "token-sequential SIMT kernel with checkpointed recomputation (one to four "
+                             "blocks per (batch, head), each owning a slice of the columns); includes allocation "
+                             "of the gradient buffers and workspace"}
         del dev, st, keep, dy
         torch.cuda.empty_cache()
     return out
