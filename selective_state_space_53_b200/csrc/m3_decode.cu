@@ -124,6 +124,11 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
                : "memory");
 }
 
+// programmatic dependent launch: the next step's grid may start its set-up early; its first
+// global access waits for this grid's completion
+__device__ __forceinline__ void ring_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void ring_griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // named barrier of one team (id >= 1; id 0 is __syncthreads)
 __device__ __forceinline__ void team_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -237,10 +242,14 @@ __global__ void __launch_bounds__(kRingThreads, 1) decode_ring_kernel(Params p, 
   };
 
   RingCursor ahead = first;  // the next block to issue (the team leader's)
+  ring_launch_dependents();
   if (tid == 0) {
     for (int s = 0; s < S; ++s)
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 2;" ::"r"(bar0 + 8u * s));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  ring_griddep_wait();  // the previous step's state, carry and outputs are visible from here on
+  if (tid == 0) {
     for (int s = 0; s < S && s < nv; ++s) {
       issue(ahead, s);
       ahead.next(SPL, T, nb);
@@ -511,20 +520,30 @@ DeviceLimits device_limits() {
   return out;
 }
 
+// launch with programmatic stream serialisation (the kernel waits on the previous grid before
+// its first global access)
+template <typename Kernel>
+cudaError_t launch_ring_pdl(Kernel k, unsigned grid, size_t smem, cudaStream_t stream, const Params& p,
+                            const RingPlan& rp) {
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kRingThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, p, rp);
+}
+
 template <int RT>
 cudaError_t launch_ring_rt(const Params& p, const RingPlan& rp, unsigned grid, cudaStream_t stream) {
-  if (p.dtype == M3_BF16) {
-    auto k = decode_ring_kernel<RT, true>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rp.total);
-    if (e != cudaSuccess) return e;
-    k<<<grid, kRingThreads, rp.total, stream>>>(p, rp);
-  } else {
-    auto k = decode_ring_kernel<RT, false>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rp.total);
-    if (e != cudaSuccess) return e;
-    k<<<grid, kRingThreads, rp.total, stream>>>(p, rp);
-  }
-  return cudaGetLastError();
+  return p.dtype == M3_BF16 ? launch_ring_pdl(decode_ring_kernel<RT, true>, grid, rp.total, stream, p, rp)
+                            : launch_ring_pdl(decode_ring_kernel<RT, false>, grid, rp.total, stream, p, rp);
 }
 
 // The ring form needs two stages per team at least.  Preferred: the most teams (units in flight
