@@ -573,8 +573,7 @@ cudaError_t launch_bwd_nk(const Params& p, const BwdArgs& q, cudaStream_t stream
 
 template <typename T, int RT>
 cudaError_t launch_bwd_rt(const Params& p, const BwdArgs& q, cudaStream_t stream) {
-  const int nk = bwd_shape(p.P / q.cs, p.N).NK;
-  if (nk <= 1) return launch_bwd_nk<T, 1, RT>(p, q, stream);
+  const int nk = bwd_shape(p.P / q.cs, p.N).NK;  // pairs per thread; the loops skip pairs past N/2
   if (nk <= 2) return launch_bwd_nk<T, 2, RT>(p, q, stream);
   if (nk <= 4) return launch_bwd_nk<T, 4, RT>(p, q, stream);
   if (nk <= 8) return launch_bwd_nk<T, 8, RT>(p, q, stream);
