@@ -37,6 +37,7 @@
 //   4-11   rotation: cumulative angles and their sin/cos table; Bt, Ct rotated in place
 //   12-15  mask: S from tensor memory -> S' (bf16, shared memory)
 //   16-19  epilogue: Y^T from tensor memory -> y
+//          (in the state pass, with N = 128 and plain inputs, warps 12-19 rotate half of B's chunks)
 //   20-23  state and inputs: the state rescale and its bf16 copy hb; X'^T into tensor memory
 // The block is launched with 80 registers a thread; the control warpgroup gives some back and
 // the rotation warpgroups take them (setmaxnreg), since the rotation holds the most live values.
@@ -75,6 +76,8 @@ constexpr unsigned long long WS_WAIT_NS = 2000000000ull;  // 2 s bound on any wa
 constexpr int WS_FULL = 0, WS_STATE = 1;
 constexpr uint32_t BAR_ROT = 1;                   // named barrier of the rotation warps
 constexpr uint32_t BAR_SPX = 2;                   // named barrier of the state warps
+constexpr uint32_t BAR_RH = 3;                    // rotation warps and their helpers (state pass)
+constexpr int N_HELP = 8;                         // helper warps: the mask and epilogue groups
 
 // barrier indices
 enum {
@@ -300,12 +303,16 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
     tmem_alloc(tmem_slot, C::TM_COLS);
     tmem_relinquish();
   }
+  // In the state pass the mask and epilogue groups have no work of their own: with N = 128 and
+  // plain inputs they rotate half of each tile's B chunks (the rotation group computes the
+  // angle table and rotates the other half).  Both sides meet on BAR_RH twice per tile.
+  const bool helpers = !FULL && !p.raw_inputs && C::NKC == 2 * N_ROT;
   if (tid == 0) {
     const int ce = FULL ? (N_ROT + 4 + 4 + 4 + 1) : (N_ROT + 4 + 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[B_BCF + s], 1);
       mbar_init(&bar[B_BCE + s], 1);
-      mbar_init(&bar[B_ROT + s], N_ROT);
+      mbar_init(&bar[B_ROT + s], helpers ? N_ROT + N_HELP : N_ROT);
       mbar_init(&bar[B_XPF + s], 4);
       mbar_init(&bar[B_XBF + s], 1);
     }
@@ -332,6 +339,43 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // State pass, N = 128, plain inputs: a helper warp of the mask or epilogue group rotates B chunk
+  // N_ROT + (its index) of every tile, between the rotation group's two barriers of the tile (the
+  // table is complete and B in place after the second; the helpers are done with the table when
+  // they reach the next tile's first).
+  auto rotate_help = [&]() {
+    const int kc = N_ROT + (warp - W_MASK);
+    const float* biasB = reinterpret_cast<const float*>(sm + C::OFF_BIAS) + (lane % R) * C::BIAS_ROW;
+    const uint8_t* tk = sm + C::OFF_TAB + kc * 16;
+    const uint32_t cb = (uint32_t)(kc >> 3) * C::BLK + (uint32_t)lane * 128u + ((uint32_t)((kc & 7) ^ (lane & 7)) << 4);
+    Phases ph_bcf;
+    for (int i = 0; i < ntl; ++i) {
+      const int s = i & 1;
+      const int64_t c0 = (j0 + i) * Q;
+      const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
+      if (bar_any(BAR_RH, 32 * (N_ROT + N_HELP), *abort_flag != 0)) break;
+      const bool okb = ws_wait(&bar[B_BCF + s], ph_bcf[s], abort_flag);
+      ph_bcf.flip(s);
+      if (bar_any(BAR_RH, 32 * (N_ROT + N_HELP), !okb || *abort_flag)) break;
+      const float4 bBe = *reinterpret_cast<const float4*>(biasB + kc * 8);
+      const float4 bBo = *reinterpret_cast<const float4*>(biasB + kc * 8 + 4);
+      const uint64_t bB0 = f2(bBe.x, bBe.y), bB1 = f2(bBe.z, bBe.w), bB2 = f2(bBo.x, bBo.y), bB3 = f2(bBo.z, bBo.w);
+#pragma unroll 2
+      for (int step = 0; step < 4; ++step) {
+        const int t = (32 * step + lane) / R;
+        const uint32_t off = cb + (uint32_t)step * 4096u;
+        if (t < nv) {
+          const RotCS rcs = rot_cs(*reinterpret_cast<const uint4*>(tk + t * C::TAB_ROW));
+          sts128(sB(s) + off, rotate16(lds128(sB(s) + off), rcs, f2(1.0f, 1.0f), bB0, bB1, bB2, bB3));
+        } else {
+          sts128(sB(s) + off, make_uint4(0, 0, 0, 0));
+        }
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar[B_ROT + s]);
+    }
+  };
   const int wg = warp >> 2;
   if (wg == 0) {
     regs_dec<WS_REG_CTRL>();
@@ -609,7 +653,11 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
           const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
           bool okw = ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag);
           ph_cf.flip(cs);
-          if (bar_any(BAR_ROT, 32 * N_ROT, !okw || *abort_flag)) break;  // the group stops together
+          // the group stops together (with its helpers in the state pass: they are then done with
+          // the previous tile's table)
+          if (helpers ? bar_any(BAR_RH, 32 * (N_ROT + N_HELP), !okw || *abort_flag)
+                      : bar_any(BAR_ROT, 32 * N_ROT, !okw || *abort_flag))
+            break;
           const float* mu = mult(cs);
           const float4* ra = recA(cs);
           const float* sc = scal(cs);
@@ -651,7 +699,9 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
           okw = ws_wait(&bar[B_BCF + s], ph_bcf[s], abort_flag);
           ph_bcf.flip(s);
           // table complete, base and segsum read, the tile's B and C in place
-          if (bar_any(BAR_ROT, 32 * N_ROT, !okw || *abort_flag)) break;
+          if (helpers ? bar_any(BAR_RH, 32 * (N_ROT + N_HELP), !okw || *abort_flag)
+                      : bar_any(BAR_ROT, 32 * N_ROT, !okw || *abort_flag))
+            break;
           if (aseg == 0) {
             double nb = base[ak] + tot;
             nb -= 6.283185307179586 * rint(nb * 0.15915494309189535);
@@ -685,9 +735,11 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
             named_bar_sync(BAR_ROT, 32 * N_ROT);
           }
           // ---- rotate Bt (and Ct) of the tile in place: lanes take 32 consecutive rows, the branch
-          // r = lane % R and so the chunk's biases are fixed per thread
+          // r = lane % R and so the chunk's biases are fixed per thread (chunks wr + N_ROT q; with
+          // helpers, chunk wr only)
+          const int kcw = helpers ? 1 : C::KCW;
 #pragma unroll 1
-          for (int q = 0; q < C::KCW; ++q) {
+          for (int q = 0; q < kcw; ++q) {
             const int kc = wr + N_ROT * q;
             // row 32 step + lane, chunk kc: 128-byte swizzle with (row & 7) = (lane & 7)
             const uint32_t cb = (uint32_t)(kc >> 3) * BLK + (uint32_t)lane * 128u + ((uint32_t)((kc & 7) ^ (lane & 7)) << 4);
@@ -764,6 +816,7 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
         }
     }
   } else if (wg == 3) {
+    if (!FULL && helpers && ntl > 0) rotate_help();
     if (FULL && ntl > 0) {
         // =============================================================== mask
         const int q4 = warp & 3;
@@ -828,6 +881,7 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
         }
     }
   } else if (wg == 4) {
+    if (!FULL && helpers && ntl > 0) rotate_help();
     if (FULL && ntl > 0) {
         // =============================================================== epilogue
         const int q4 = warp & 3;
