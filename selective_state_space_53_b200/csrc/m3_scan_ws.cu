@@ -304,15 +304,18 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
     tmem_relinquish();
   }
   // In the state pass the mask and epilogue groups have no work of their own: with N = 128 and
-  // plain inputs they rotate half of each tile's B chunks (the rotation group computes the
-  // angle table and rotates the other half).  Both sides meet on BAR_RH twice per tile.
+  // plain inputs they rotate every tile's B, while the rotation group builds the angle tables one
+  // tile ahead into two buffers (the second in the S' area, which the state pass does not use).
+  // The two sides meet on BAR_RH once per tile ("table i complete and B of tile i in place"); the
+  // buffer the rotation group fills next, for tile i + 1, was last read by the helpers for tile
+  // i - 1, which they finished before reaching that barrier for tile i.
   const bool helpers = !FULL && !p.raw_inputs && C::NKC == 2 * N_ROT;
   if (tid == 0) {
     const int ce = FULL ? (N_ROT + 4 + 4 + 4 + 1) : (N_ROT + 4 + 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bar[B_BCF + s], 1);
       mbar_init(&bar[B_BCE + s], 1);
-      mbar_init(&bar[B_ROT + s], helpers ? N_ROT + N_HELP : N_ROT);
+      mbar_init(&bar[B_ROT + s], helpers ? N_HELP : N_ROT);
       mbar_init(&bar[B_XPF + s], 4);
       mbar_init(&bar[B_XBF + s], 1);
     }
@@ -339,36 +342,38 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // State pass, N = 128, plain inputs: a helper warp of the mask or epilogue group rotates B chunk
-  // N_ROT + (its index) of every tile, between the rotation group's two barriers of the tile (the
-  // table is complete and B in place after the second; the helpers are done with the table when
-  // they reach the next tile's first).
+  // State pass, N = 128, plain inputs: helper warp hw (0..7) of the mask and epilogue groups
+  // rotates B chunks hw and hw + 8 of every tile, after the tile's BAR_RH barrier.
   auto rotate_help = [&]() {
-    const int kc = N_ROT + (warp - W_MASK);
+    const int hw = warp - W_MASK;
     const float* biasB = reinterpret_cast<const float*>(sm + C::OFF_BIAS) + (lane % R) * C::BIAS_ROW;
-    const uint8_t* tk = sm + C::OFF_TAB + kc * 16;
-    const uint32_t cb = (uint32_t)(kc >> 3) * C::BLK + (uint32_t)lane * 128u + ((uint32_t)((kc & 7) ^ (lane & 7)) << 4);
     Phases ph_bcf;
     for (int i = 0; i < ntl; ++i) {
       const int s = i & 1;
       const int64_t c0 = (j0 + i) * Q;
       const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
-      if (bar_any(BAR_RH, 32 * (N_ROT + N_HELP), *abort_flag != 0)) break;
       const bool okb = ws_wait(&bar[B_BCF + s], ph_bcf[s], abort_flag);
       ph_bcf.flip(s);
-      if (bar_any(BAR_RH, 32 * (N_ROT + N_HELP), !okb || *abort_flag)) break;
-      const float4 bBe = *reinterpret_cast<const float4*>(biasB + kc * 8);
-      const float4 bBo = *reinterpret_cast<const float4*>(biasB + kc * 8 + 4);
-      const uint64_t bB0 = f2(bBe.x, bBe.y), bB1 = f2(bBe.z, bBe.w), bB2 = f2(bBo.x, bBo.y), bB3 = f2(bBo.z, bBo.w);
+      if (bar_any(BAR_RH, 32 * (N_ROT + N_HELP), !okb || *abort_flag)) break;  // table i complete
+      const uint8_t* tb = s ? sm + C::OFF_SP : sm + C::OFF_TAB;
+#pragma unroll 1
+      for (int q = 0; q < 2; ++q) {
+        const int kc = hw + N_ROT * q;
+        const uint32_t cb = (uint32_t)(kc >> 3) * C::BLK + (uint32_t)lane * 128u + ((uint32_t)((kc & 7) ^ (lane & 7)) << 4);
+        const float4 bBe = *reinterpret_cast<const float4*>(biasB + kc * 8);
+        const float4 bBo = *reinterpret_cast<const float4*>(biasB + kc * 8 + 4);
+        const uint64_t bB0 = f2(bBe.x, bBe.y), bB1 = f2(bBe.z, bBe.w), bB2 = f2(bBo.x, bBo.y), bB3 = f2(bBo.z, bBo.w);
+        const uint8_t* tk = tb + kc * 16;
 #pragma unroll 2
-      for (int step = 0; step < 4; ++step) {
-        const int t = (32 * step + lane) / R;
-        const uint32_t off = cb + (uint32_t)step * 4096u;
-        if (t < nv) {
-          const RotCS rcs = rot_cs(*reinterpret_cast<const uint4*>(tk + t * C::TAB_ROW));
-          sts128(sB(s) + off, rotate16(lds128(sB(s) + off), rcs, f2(1.0f, 1.0f), bB0, bB1, bB2, bB3));
-        } else {
-          sts128(sB(s) + off, make_uint4(0, 0, 0, 0));
+        for (int step = 0; step < 4; ++step) {
+          const int t = (32 * step + lane) / R;
+          const uint32_t off = cb + (uint32_t)step * 4096u;
+          if (t < nv) {
+            const RotCS rcs = rot_cs(*reinterpret_cast<const uint4*>(tk + t * C::TAB_ROW));
+            sts128(sB(s) + off, rotate16(lds128(sB(s) + off), rcs, f2(1.0f, 1.0f), bB0, bB1, bB2, bB3));
+          } else {
+            sts128(sB(s) + off, make_uint4(0, 0, 0, 0));
+          }
         }
       }
       fence_async_smem();
@@ -646,6 +651,59 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
         load_theta(j0);
         Phases ph_cf, ph_bcf;
         uint8_t* tab = sm + C::OFF_TAB;
+        if (!FULL && helpers) {
+          // ---- state pass with helpers: the angle tables only, one tile ahead of the rotation
+          for (int i = 0; i < ntl; ++i) {
+            const int cs = i % WS_CS, s = i & 1;
+            const int64_t j = j0 + i;
+            uint8_t* tb = s ? sm + C::OFF_SP : sm + C::OFF_TAB;
+            const bool okw = ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag);
+            ph_cf.flip(cs);
+            // the group decides together; a stop is taken on the next BAR_RH barrier, with the helpers
+            const bool bad = bar_any(BAR_ROT, 32 * N_ROT, !okw || *abort_flag);
+            double tot = 0.0;
+            if (!bad) {
+              const float* mu = mult(cs);
+              float aloc[C::SEGLEN];
+              float r2 = 0.0f;
+#pragma unroll
+              for (int e = 0; e < C::SEGLEN; ++e) {
+                r2 = fmaf(mu[aseg * C::SEGLEN + e], thr[e], r2);
+                aloc[e] = r2;
+              }
+              segsum[aseg * K2 + ak] = r2;
+              named_bar_sync(BAR_ROT, 32 * N_ROT);
+              float aoff = (float)base[ak];
+#pragma unroll
+              for (int s2 = 0; s2 < C::SEGS; ++s2) {
+                const float v = segsum[s2 * K2 + ak];
+                if (s2 < aseg) aoff += v;
+                if (aseg == 0) tot += (double)v;
+              }
+#pragma unroll
+              for (int e = 0; e < C::SEGLEN; ++e) {
+                const int t = aseg * C::SEGLEN + e;
+                float sn, cn;
+                sincos_reduced(aoff + aloc[e], &sn, &cn);
+                const float other = __shfl_xor_sync(kFull, (ak & 1) ? cn : sn, 1);
+                const __half2 hv = (ak & 1) ? __floats2half2_rn(other, sn) : __floats2half2_rn(cn, other);
+                *reinterpret_cast<__half2*>(tb + t * C::TAB_ROW + (ak >> 1) * 8 + (ak & 1) * 4) = hv;
+              }
+              if (i + 1 < ntl) load_theta(j + 1);
+            }
+            const bool okb = !bad && ws_wait(&bar[B_BCF + s], ph_bcf[s], abort_flag);
+            ph_bcf.flip(s);
+            // table i complete, B of tile i in place: the helpers rotate it
+            if (bar_any(BAR_RH, 32 * (N_ROT + N_HELP), bad || !okb || *abort_flag)) break;
+            if (aseg == 0) {
+              double nb = base[ak] + tot;
+              nb -= 6.283185307179586 * rint(nb * 0.15915494309189535);
+              base[ak] = nb;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[B_CE + cs]);
+          }
+        } else
         for (int i = 0; i < ntl; ++i) {
           const int cs = i % WS_CS, s = i & 1;
           const int64_t j = j0 + i;
@@ -653,11 +711,8 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
           const int nv = (int)((L - c0) < Q ? (L - c0) : Q);
           bool okw = ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag);
           ph_cf.flip(cs);
-          // the group stops together (with its helpers in the state pass: they are then done with
-          // the previous tile's table)
-          if (helpers ? bar_any(BAR_RH, 32 * (N_ROT + N_HELP), !okw || *abort_flag)
-                      : bar_any(BAR_ROT, 32 * N_ROT, !okw || *abort_flag))
-            break;
+          // the group stops together
+          if (bar_any(BAR_ROT, 32 * N_ROT, !okw || *abort_flag)) break;
           const float* mu = mult(cs);
           const float4* ra = recA(cs);
           const float* sc = scal(cs);
@@ -699,9 +754,7 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
           okw = ws_wait(&bar[B_BCF + s], ph_bcf[s], abort_flag);
           ph_bcf.flip(s);
           // table complete, base and segsum read, the tile's B and C in place
-          if (helpers ? bar_any(BAR_RH, 32 * (N_ROT + N_HELP), !okw || *abort_flag)
-                      : bar_any(BAR_ROT, 32 * N_ROT, !okw || *abort_flag))
-            break;
+          if (bar_any(BAR_ROT, 32 * N_ROT, !okw || *abort_flag)) break;
           if (aseg == 0) {
             double nb = base[ak] + tot;
             nb -= 6.283185307179586 * rint(nb * 0.15915494309189535);
@@ -735,11 +788,9 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
             named_bar_sync(BAR_ROT, 32 * N_ROT);
           }
           // ---- rotate Bt (and Ct) of the tile in place: lanes take 32 consecutive rows, the branch
-          // r = lane % R and so the chunk's biases are fixed per thread (chunks wr + N_ROT q; with
-          // helpers, chunk wr only)
-          const int kcw = helpers ? 1 : C::KCW;
+          // r = lane % R and so the chunk's biases are fixed per thread
 #pragma unroll 1
-          for (int q = 0; q < kcw; ++q) {
+          for (int q = 0; q < C::KCW; ++q) {
             const int kc = wr + N_ROT * q;
             // row 32 step + lane, chunk kc: 128-byte swizzle with (row & 7) = (lane & 7)
             const uint32_t cb = (uint32_t)(kc >> 3) * BLK + (uint32_t)lane * 128u + ((uint32_t)((kc & 7) ^ (lane & 7)) << 4);
