@@ -37,7 +37,8 @@
 //   4-11   rotation: cumulative angles and their sin/cos table; Bt, Ct rotated in place
 //   12-15  mask: S from tensor memory -> S' (bf16, shared memory)
 //   16-19  epilogue: Y^T from tensor memory -> y
-//          (in the state pass, with N = 128 and plain inputs, warps 12-19 rotate half of B's chunks)
+//          (in the state pass, with N = 128 and plain inputs, warps 12-19 rotate B while warps 4-11
+//          build the next tile's angle table)
 //   20-23  state and inputs: the state rescale and its bf16 copy hb; X'^T into tensor memory
 // The block is launched with 80 registers a thread; the control warpgroup gives some back and
 // the rotation warpgroups take them (setmaxnreg), since the rotation holds the most live values.
