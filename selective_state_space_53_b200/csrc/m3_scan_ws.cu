@@ -102,6 +102,7 @@ enum {
   B_XE = 28,    // the x slot consumed (state warps)
   NBAR = 29
 };
+static_assert(B_CE - B_CF == WS_CS && B_ROT - B_CE == WS_CS, "one pair of barriers per coefficient record slot");
 
 template <int R, int N>
 struct WsCfg {
