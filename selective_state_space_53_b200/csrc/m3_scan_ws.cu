@@ -661,10 +661,11 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
             uint8_t* tb = s ? sm + C::OFF_SP : sm + C::OFF_TAB;
             const bool okw = ws_wait(&bar[B_CF + cs], ph_cf[cs], abort_flag);
             ph_cf.flip(cs);
-            // the group decides together; a stop is taken on the next BAR_RH barrier, with the helpers
-            const bool bad = bar_any(BAR_ROT, 32 * N_ROT, !okw || *abort_flag);
+            // a failed wait is carried to this tile's BAR_RH barrier, where everyone stops together
+            // (the table is built regardless, from whatever the record holds); the previous tile's
+            // segment sums were read before that tile's BAR_RH barrier
             double tot = 0.0;
-            if (!bad) {
+            {
               const float* mu = mult(cs);
               float aloc[C::SEGLEN];
               float r2 = 0.0f;
@@ -693,10 +694,10 @@ __global__ void __maxnreg__(WS_REG_LAUNCH)
               }
               if (i + 1 < ntl) load_theta(j + 1);
             }
-            const bool okb = !bad && ws_wait(&bar[B_BCF + s], ph_bcf[s], abort_flag);
+            const bool okb = okw && ws_wait(&bar[B_BCF + s], ph_bcf[s], abort_flag);
             ph_bcf.flip(s);
             // table i complete, B of tile i in place: the helpers rotate it
-            if (bar_any(BAR_RH, 32 * (N_ROT + N_HELP), bad || !okb || *abort_flag)) break;
+            if (bar_any(BAR_RH, 32 * (N_ROT + N_HELP), !okb || *abort_flag)) break;
             if (aseg == 0) {
               double nb = base[ak] + tot;
               nb -= 6.283185307179586 * rint(nb * 0.15915494309189535);
